@@ -1,0 +1,351 @@
+"""Plain, slow fp64 CPU statement of the single-GPU fused mixture-of-experts layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU baseline /
+reference arm may use it.  It shares no code with the CUDA library.
+
+What the layer computes (sources, by page and section):
+
+* "Prime Intellect Fused MoE Kernel: 3.11x MoE Training Speed", section
+  "What a mixture-of-experts layer actually does": a router sends each token to
+  a few experts; the fused call does the dispatch, both expert linear layers,
+  SwiGLU and the combine.
+* "Prime Intellect's Prime Mega MoE Trains Giant AI Models 55% Faster",
+  section "Where MoE training loses time": dispatch tokens to their experts
+  (token sorting), run the expert MLPs, return the outputs to their original
+  positions; the backward pass repeats the exchange for gradients.
+* "Mario/overlap moe kernel integration (prime-rl PR #3651)", Overview and the
+  custom-op commit note: the fused compute consumes undispatched tokens plus
+  the routing (top scores, selected expert indices), runs in bf16 and returns
+  gradients in the inputs' dtypes.
+
+Readings taken where the pages are silent (each one is listed in the design doc):
+
+* routing: softmax over all E router logits, keep the k largest, renormalise
+  over the kept k.  The k largest are chosen on the fp32 logits themselves
+  (softmax is strictly increasing, so the set is the same), ordered by value
+  descending and, on ties, by lower expert index.  Slot j of a token is its
+  j-th choice in that order.
+* dispatch order: experts ascending; inside an expert, tokens ascending
+  (a stable counting sort of the flattened choices t*k + j).
+* expert MLP: W_gate_up[e] is [2I, d] with rows 0..I-1 the gate and rows
+  I..2I-1 the up projection; W_down[e] is [d, I].  h = W_gate_up[e] x,
+  a = silu(h_gate) * h_up, y = W_down[e] a.  No bias, no clamp.
+* combine: out[t] = sum over slots j = 0..k-1, in slot order, of w[t,j] y_(t,j).
+* dscore[t,j] is the gradient with respect to the renormalised weight w[t,j];
+  dlogits is the gradient with respect to the router logits through the
+  renormalised softmax (zero outside the chosen k).
+
+All arithmetic is float64 on the exactly widened inputs.  Matrix products use
+numpy (a library primitive); there is no blocking, fusion or reordering.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "route", "dispatch", "silu", "sigmoid", "expert_forward",
+    "combine_forward", "forward", "backward", "dense_forward",
+    "forward_tokens", "backward_tokens", "backward_experts",
+]
+
+
+# ----------------------------------------------------------------------------
+# elementwise functions (definitions, written out)
+# ----------------------------------------------------------------------------
+def sigmoid(z):
+    """sigma(z) = 1 / (1 + exp(-z)), in float64."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-z))
+
+
+def silu(z):
+    """silu(z) = z * sigma(z) (the gate of SwiGLU)."""
+    z = np.asarray(z, dtype=np.float64)
+    return z * sigmoid(z)
+
+
+def silu_grad(z):
+    """d silu / dz = sigma(z) * (1 + z * (1 - sigma(z)))."""
+    s = sigmoid(z)
+    return s * (1.0 + z * (1.0 - s))
+
+
+# ----------------------------------------------------------------------------
+# routing and dispatch
+# ----------------------------------------------------------------------------
+def route(logits, k):
+    """Top-k routing with renormalised softmax weights.
+
+    logits: float32 [T, E] router logits (finite).  Returns
+      idx  int32  [T, k]  chosen experts, slot j = j-th largest logit
+                          (ties: lower expert index first)
+      w    float64 [T, k] softmax over all E, restricted to the chosen k and
+                          renormalised to sum to 1.
+    """
+    logits = np.asarray(logits)
+    T, E = logits.shape
+    if not (1 <= k <= E):
+        raise ValueError("need 1 <= k <= E")
+    lo = logits.astype(np.float64)  # exact widening of fp32 values
+    expert = np.broadcast_to(np.arange(E), (T, E))
+    # np.lexsort sorts by the last key first: value descending, then index
+    order = np.lexsort((expert, -lo), axis=-1)
+    idx = order[:, :k].astype(np.int32)
+    # softmax over all experts, then renormalise over the kept k
+    m = lo.max(axis=1, keepdims=True)
+    p = np.exp(lo - m)
+    p = p / p.sum(axis=1, keepdims=True)
+    pk = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    w = pk / pk.sum(axis=1, keepdims=True)
+    return idx, w
+
+
+def dispatch(idx, E):
+    """Group the T*k (token, slot) pairs by expert.
+
+    Returns counts [E], offsets [E+1] (exclusive scan of counts), perm [T*k]
+    (sorted position -> flat pair index t*k + j; experts ascending, tokens
+    ascending inside an expert) and inv [T, k] (pair -> sorted position).
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    flat = idx.reshape(-1).astype(np.int64)
+    counts = np.bincount(flat, minlength=E).astype(np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.argsort(flat, kind="stable").astype(np.int32)
+    inv = np.empty(T * k, dtype=np.int32)
+    inv[perm] = np.arange(T * k, dtype=np.int32)
+    return counts, offsets, perm, inv.reshape(T, k)
+
+
+# ----------------------------------------------------------------------------
+# one expert's MLP
+# ----------------------------------------------------------------------------
+def expert_forward(xe, wgu_e, wd_e):
+    """SwiGLU expert on a block of rows.
+
+    xe [n, d]; wgu_e [2I, d]; wd_e [d, I].  Returns (h [n, 2I], a [n, I], y [n, d]).
+    """
+    I = wd_e.shape[1]
+    h = xe @ wgu_e.T
+    g, u = h[:, :I], h[:, I:]
+    a = silu(g) * u
+    y = a @ wd_e.T
+    return h, a, y
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# forward
+# ----------------------------------------------------------------------------
+def combine_forward(x, idx, w, wgu, wd):
+    """Layer output for a given routing (idx, w): out[t] = sum_j w[t,j] y_(t,j)."""
+    x, w, wgu, wd = _f64(x), _f64(w), _f64(wgu), _f64(wd)
+    T, k = idx.shape
+    E = wgu.shape[0]
+    counts, offsets, perm, inv = dispatch(idx, E)
+    d = x.shape[1]
+    y_pair = np.zeros((T * k, d))
+    for e in range(E):
+        pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
+        if pairs.size == 0:
+            continue
+        _, _, y = expert_forward(x[pairs // k], wgu[e], wd[e])
+        y_pair[pairs] = y
+    y_pair = y_pair.reshape(T, k, d)
+    out = np.zeros((T, d))
+    for j in range(k):  # slot order
+        out += w[:, j:j + 1] * y_pair[:, j, :]
+    return out
+
+
+def forward(x, logits, wgu, wd, k):
+    """Full forward.  Returns a dict with out and every intermediate.
+
+    h, a, y are stored per flat pair index (t*k + j) so that they do not depend
+    on any particular sorted layout.
+    """
+    x, wgu, wd = _f64(x), _f64(wgu), _f64(wd)
+    T, d = x.shape
+    E, twoI, _ = wgu.shape
+    I = twoI // 2
+    idx, w = route(logits, k)
+    counts, offsets, perm, inv = dispatch(idx, E)
+    h = np.zeros((T * k, twoI))
+    a = np.zeros((T * k, I))
+    y = np.zeros((T * k, d))
+    for e in range(E):
+        pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
+        if pairs.size == 0:
+            continue
+        he, ae, ye = expert_forward(x[pairs // k], wgu[e], wd[e])
+        h[pairs], a[pairs], y[pairs] = he, ae, ye
+    out = np.zeros((T, d))
+    yk = y.reshape(T, k, d)
+    for j in range(k):
+        out += w[:, j:j + 1] * yk[:, j, :]
+    return dict(out=out, idx=idx, w=w, counts=counts, offsets=offsets,
+                perm=perm, inv=inv, h=h, a=a, y=y)
+
+
+def dense_forward(x, logits, wgu, wd, k):
+    """Brute force: every expert on every token, masked by the routing.
+
+    M[t, e] = w[t, j] if expert e is token t's j-th choice, else 0;
+    out = sum_e M[:, e] * expert_e(x).  Used only to pin the sparse path.
+    """
+    x, wgu, wd = _f64(x), _f64(wgu), _f64(wd)
+    T, d = x.shape
+    E = wgu.shape[0]
+    idx, w = route(logits, k)
+    M = np.zeros((T, E))
+    for t in range(T):
+        for j in range(k):
+            M[t, idx[t, j]] = w[t, j]
+    out = np.zeros((T, d))
+    for e in range(E):
+        _, _, ye = expert_forward(x, wgu[e], wd[e])
+        out += M[:, e:e + 1] * ye
+    return out
+
+
+# ----------------------------------------------------------------------------
+# backward
+# ----------------------------------------------------------------------------
+def _pair_backward(x_rows, gout_rows, w_rows, wgu_e, wd_e):
+    """Backward of one expert's block of pairs.
+
+    Returns (dx_rows [n,d] unscaled contribution to dx[t], dscore [n],
+    dwgu_e [2I,d], dwd_e [d,I], dh [n,2I]).
+    """
+    I = wd_e.shape[1]
+    h = x_rows @ wgu_e.T
+    g, u = h[:, :I], h[:, I:]
+    a = silu(g) * u
+    G = gout_rows @ wd_e                    # W_down[e]^T gout[t]   [n, I]
+    dscore = np.sum(G * a, axis=1)          # <G, a> = <gout[t], y_p>
+    da = w_rows[:, None] * G
+    dg = da * u * silu_grad(g)
+    du = da * silu(g)
+    dh = np.concatenate([dg, du], axis=1)   # [n, 2I]
+    dwd_e = (w_rows[:, None] * gout_rows).T @ a   # sum_p (w gout) (x) a
+    dx_rows = dh @ wgu_e                    # W_gate_up[e]^T dh      [n, d]
+    dwgu_e = dh.T @ x_rows                  # sum_p dh (x) x[t]
+    return dx_rows, dscore, dwgu_e, dwd_e, dh
+
+
+def routing_backward(w, dscore):
+    """dlogits from dscore through the renormalised top-k softmax.
+
+    For chosen experts i: dlogit_i = w_i (dscore_i - sum_j w_j dscore_j);
+    unchosen experts get 0.  Returned in slot layout [T, k].
+    """
+    w, dscore = _f64(w), _f64(dscore)
+    s = np.sum(w * dscore, axis=1, keepdims=True)
+    return w * (dscore - s)
+
+
+def backward(x, logits, wgu, wd, k, gout, fwd=None):
+    """Full backward for loss L with dL/dout = gout.
+
+    Returns dict(dx [T,d], dwgu [E,2I,d], dwd [E,d,I], dscore [T,k],
+    dlogits [T,E], dh [T*k, 2I] per flat pair).
+    """
+    x, wgu, wd, gout = _f64(x), _f64(wgu), _f64(wd), _f64(gout)
+    T, d = x.shape
+    E, twoI, _ = wgu.shape
+    if fwd is None:
+        idx, w = route(logits, k)
+        counts, offsets, perm, inv = dispatch(idx, E)
+    else:
+        idx, w, offsets, perm = fwd["idx"], fwd["w"], fwd["offsets"], fwd["perm"]
+    dx_pair = np.zeros((T * k, d))
+    dscore = np.zeros(T * k)
+    dh = np.zeros((T * k, twoI))
+    dwgu = np.zeros_like(wgu)
+    dwd = np.zeros_like(wd)
+    wf = w.reshape(-1)
+    for e in range(E):
+        pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
+        if pairs.size == 0:
+            continue
+        t = pairs // k
+        dxr, ds, dwgu[e], dwd[e], dhe = _pair_backward(x[t], gout[t], wf[pairs], wgu[e], wd[e])
+        dx_pair[pairs], dscore[pairs], dh[pairs] = dxr, ds, dhe
+    dx = np.zeros((T, d))
+    dxk = dx_pair.reshape(T, k, d)
+    for j in range(k):  # slot order
+        dx += dxk[:, j, :]
+    dscore = dscore.reshape(T, k)
+    dl_slots = routing_backward(w, dscore)
+    dlogits = np.zeros((T, E))
+    np.put_along_axis(dlogits, idx.astype(np.int64), dl_slots, axis=1)
+    return dict(dx=dx, dwgu=dwgu, dwd=dwd, dscore=dscore, dlogits=dlogits, dh=dh)
+
+
+# ----------------------------------------------------------------------------
+# sampled variants, for checking very large layers one output at a time
+# ----------------------------------------------------------------------------
+def forward_tokens(x, logits, wgu, wd, k, tokens):
+    """out rows for the listed tokens only (same arithmetic as forward)."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    idx, w = route(np.asarray(logits)[tokens], k)
+    xt = _f64(np.asarray(x)[tokens])
+    out = np.zeros((tokens.size, xt.shape[1]))
+    for j in range(k):
+        for r in range(tokens.size):
+            e = int(idx[r, j])
+            _, _, y = expert_forward(xt[r:r + 1], _f64(wgu[e]), _f64(wd[e]))
+            out[r] += w[r, j] * y[0]
+    return dict(out=out, idx=idx, w=w)
+
+
+def backward_tokens(x, logits, wgu, wd, k, gout, tokens):
+    """dx, dscore and dlogits rows for the listed tokens only."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    logits = np.asarray(logits)
+    E = logits.shape[1]
+    idx, w = route(logits[tokens], k)
+    xt = _f64(np.asarray(x)[tokens])
+    gt = _f64(np.asarray(gout)[tokens])
+    dx = np.zeros_like(xt)
+    dscore = np.zeros((tokens.size, k))
+    for j in range(k):
+        for r in range(tokens.size):
+            e = int(idx[r, j])
+            dxr, ds, _, _, _ = _pair_backward(xt[r:r + 1], gt[r:r + 1], w[r, j:j + 1],
+                                              _f64(wgu[e]), _f64(wd[e]))
+            dx[r] += dxr[0]
+            dscore[r, j] = ds[0]
+    dl_slots = routing_backward(w, dscore)
+    dlogits = np.zeros((tokens.size, E))
+    np.put_along_axis(dlogits, idx.astype(np.int64), dl_slots, axis=1)
+    return dict(dx=dx, dscore=dscore, dlogits=dlogits, idx=idx, w=w)
+
+
+def backward_experts(x, logits, wgu, wd, k, gout, experts):
+    """dW_gate_up[e] and dW_down[e] for the listed experts only."""
+    logits = np.asarray(logits)
+    E = logits.shape[1]
+    idx, w = route(logits, k)
+    counts, offsets, perm, inv = dispatch(idx, E)
+    wf = w.reshape(-1)
+    res = {}
+    for e in experts:
+        e = int(e)
+        pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
+        wgu_e, wd_e = _f64(wgu[e]), _f64(wd[e])
+        if pairs.size == 0:
+            res[e] = (np.zeros_like(wgu_e), np.zeros_like(wd_e))
+            continue
+        t = pairs // k
+        _, _, dwgu_e, dwd_e, _ = _pair_backward(_f64(np.asarray(x)[t]), _f64(np.asarray(gout)[t]),
+                                                wf[pairs], wgu_e, wd_e)
+        res[e] = (dwgu_e, dwd_e)
+    return res
