@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoE layer (forward + backward) on B200.
+
+One step = one full pass of the layer's hot path: routing (top-k, histogram,
+scan, permutation), the gate/up grouped GEMM with the TMA row-gather dispatch
+and the SwiGLU epilogue, the down grouped GEMM with the ordered combine, and
+the backward (down dgrad + SwiGLU backward, both weight gradients, gate/up
+dgrad with the ordered scatter, routing-score gradients), all through the C
+ABI of libmoe.so on device-resident synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+N > 1 is launched by torchrun; every rank runs an independent replica of the
+layer on its own GPU (the layer has no data-path exchange on one GPU), timing
+is the max over ranks and ``value`` counts the work of all ranks.
+``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused MoE layer fwd+bwd TFLOP/s & % of bf16 tensor peak (Qwen3-30B-A3B shape)"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="qwen3_30b_a3b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0 = auto)")
+    ap.add_argument("--override", default="", help="comma list of size overrides, e.g. T=4096,E=32 "
+                                                     "(smaller profiling cases; not a bench workload)")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def workload_config(name, cfg, extra=None):
+    c = {"workload": name, "T": cfg["T"], "d": cfg["d"], "E": cfg["E"], "top_k": cfg["k"], "I": cfg["I"]}
+    if "zipf_s" in cfg:
+        c["zipf_s"] = cfg["zipf_s"]
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() in ("active", "1"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "samples": len(loaded), "power_w_max": max(r["power"] for r in rows), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(cfg, inp, n_tokens):
+    """Inputs of the first n_tokens tokens as float64 arrays (weights stay whole)."""
+    import numpy as np
+    sl = slice(0, n_tokens)
+    x = inp["x"][sl].float().numpy().astype(np.float64)
+    lg = inp["logits"][sl].numpy()
+    gout = inp["gout"][sl].float().numpy().astype(np.float64)
+    return x, lg, gout
+
+
+def time_oracle_step(cfg, inp, wgu64, wd64, n_tokens):
+    from oracle import moe_oracle as O
+    x, lg, gout = oracle_sample(cfg, inp, n_tokens)
+    t0 = time.perf_counter()
+    f = O.forward(x, lg, wgu64, wd64, cfg["k"])
+    O.backward(x, lg, wgu64, wd64, cfg["k"], gout, f)
+    return time.perf_counter() - t0
+
+
+def oracle_weights(inp):
+    import numpy as np
+    return inp["wgu"].float().numpy().astype(np.float64), inp["wd"].float().numpy().astype(np.float64)
+
+
+def cpu_baseline(cfg, inp, n_tokens=0, budget_s=15.0):
+    from grouped_gemm_route_b200 import inputs as IN
+    wgu64, wd64 = oracle_weights(inp)
+    n = n_tokens or 64
+    dt = time_oracle_step(cfg, inp, wgu64, wd64, n)
+    if not n_tokens:  # grow the sample to about budget_s of work
+        n = int(min(cfg["T"], max(64, n * budget_s / max(dt, 1e-3) * 0.8)))
+        dt = time_oracle_step(cfg, inp, wgu64, wd64, n)
+    flops = IN.flops_fwd(T=n, **{k: cfg[k] for k in ("d", "E", "k", "I")}) + \
+        IN.flops_bwd(T=n, **{k: cfg[k] for k in ("d", "E", "k", "I")})
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, forward+backward of the first {n} of {cfg['T']} tokens "
+                      f"(all experts' weights), {dt:.2f} s"}, n, dt
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return 0
+    from grouped_gemm_route_b200 import inputs as IN
+    cfg, inp = IN.make_workload(args.workload, seed=args.seed, device="cpu")
+    wgu64, wd64 = oracle_weights(inp)
+    # per-step sample sized so that warmup + steps finish in a few minutes
+    probe = 64
+    dt = time_oracle_step(cfg, inp, wgu64, wd64, probe)
+    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    n = args.cpu_tokens or int(min(cfg["T"], max(16, probe * per_step_budget / max(dt, 1e-3) * 0.8)))
+    for _ in range(args.warmup):
+        time_oracle_step(cfg, inp, wgu64, wd64, n)
+    times = [time_oracle_step(cfg, inp, wgu64, wd64, n) for _ in range(args.steps)]
+    total = sum(times)
+    dims = {k: cfg[k] for k in ("d", "E", "k", "I")}
+    flops = (IN.flops_fwd(T=n, **dims) + IN.flops_bwd(T=n, **dims)) * args.steps
+    value = flops / total / 1e12
+    sample = f"fp64 numpy oracle, forward+backward of the first {n} of {cfg['T']} tokens per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args.workload, cfg, {"oracle_tokens_per_step": n}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+
+    from grouped_gemm_route_b200 import inputs as IN
+    from grouped_gemm_route_b200 import moe as M
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    cfg = dict(IN.WORKLOADS[args.workload])
+    for item in filter(None, args.override.split(",")):
+        key, val = item.split("=")
+        cfg[key] = int(val)
+    host = IN.make_inputs(seed=args.seed + rank, device="cpu", **cfg)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    x, lg, wgu, wd, gout = (host[n].to(dev) for n in ("x", "logits", "wgu", "wd", "gout"))
+    layer = M.MoELayer(T, d, E, k, I, device=str(dev))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.forward(x, lg, wgu, wd, stream)
+        layer.backward(gout, x, wgu, wd, True, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if layer.status(stream) != 0:
+        raise SystemExit(f"device status {layer.status(stream)} after warm-up")
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    # ---- device-resident timed region (per-kernel events enabled) ----
+    M.profile_read()
+    M.profile_enable(True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    M.profile_enable(False)
+    per_kernel = M.profile_read()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if layer.status(stream) != 0:
+        raise SystemExit("device status error in the timed region")
+    if pg is not None:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    flops_step = IN.flops_fwd(**cfg) + IN.flops_bwd(**cfg)
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel ----
+    peaks, peak_src = load_peaks()
+    P = T * k
+    gemm_flops = {"gemm_gateup_fwd": 4.0 * P * d * I, "gemm_down_fwd_combine": 2.0 * P * I * d,
+                  "gemm_down_dgrad": 2.0 * P * d * I, "gemm_down_wgrad": 2.0 * P * d * I,
+                  "gemm_gateup_dgrad_scatter": 4.0 * P * d * I, "gemm_gateup_wgrad": 4.0 * P * d * I}
+    total_kernel_ms = sum(v[0] for v in per_kernel.values()) or 1.0
+    dom = max(gemm_flops, key=lambda n: per_kernel.get(n, (0.0, 0))[0])
+    dom_ms, dom_n = per_kernel[dom]
+    dom_avg_ms = dom_ms / max(dom_n, 1)
+    achieved = gemm_flops[dom] / (dom_avg_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            from grouped_gemm_route_b200 import build as B
+            with open(tpath) as f:
+                tr = json.load(f)
+            ent = tr.get(dom, {})
+            if ent.get("source_hash") == B.source_hash() and ent.get("workload") == args.workload:
+                traffic = ent.get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    gemm_ms = sum(per_kernel.get(n, (0.0, 0))[0] for n in gemm_flops) / args.steps
+    route_names = ("route_topk", "route_scan", "route_perm")
+    route_ms = sum(per_kernel.get(n, (0.0, 0))[0] for n in route_names) / args.steps
+    routing = {"bytes_per_step": IN.routing_bytes(T, E, k), "ms_per_step": route_ms,
+               "achieved_gbs": IN.routing_bytes(T, E, k) / (route_ms * 1e-3) / 1e9 if route_ms else None,
+               "peak_gbs": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))}
+    breakdown = {n: {"ms_per_step": v[0] / args.steps, "share": v[0] / total_kernel_ms,
+                     "launches": v[1]} for n, v in per_kernel.items() if v[1]}
+    launches = int(sum(v[1] for v in per_kernel.values()))
+
+    # ---- end-to-end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        hx, hlg, hg = (host[n].pin_memory() for n in ("x", "logits", "gout"))
+        hout = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+        hdx = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+        hds = torch.empty(T, k, dtype=torch.float32).pin_memory()
+        dx_, dlg_, dg_ = torch.empty_like(x), torch.empty_like(lg), torch.empty_like(gout)
+
+        def e2e_step():
+            dx_.copy_(hx, non_blocking=True)
+            dlg_.copy_(hlg, non_blocking=True)
+            dg_.copy_(hg, non_blocking=True)
+            layer.forward(dx_, dlg_, wgu, wd, stream)
+            layer.backward(dg_, dx_, wgu, wd, True, stream)
+            hout.copy_(layer.out, non_blocking=True)
+            hdx.copy_(layer.dx, non_blocking=True)
+            hds.copy_(layer.dscore, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if pg is not None:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        bi = sum(t.numel() * t.element_size() for t in (hx, hlg, hg))
+        bo = sum(t.numel() * t.element_size() for t in (hout, hdx, hds))
+        e2e = {"value": flops_step * world / (e_ms / args.e2e_steps * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": args.e2e_steps}
+
+    # ---- CPU baseline (rank 0, N = 1 only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _, _ = cpu_baseline(cfg, host, args.cpu_tokens)
+
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(args.workload, cfg, {"parallelism": f"replicas{world}",
+                                                       "l2": "inputs larger than L2 (expert weights 1.15 GB at "
+                                                             "the 30B shape), no flush"}),
+        "frac_of_bf16_peak": {"step": value / world / peak, "gemm_only": (flops_step / (gemm_ms * 1e-3) / 1e12) / peak
+                              if gemm_ms else None, "peak": peak, "peak_source": roofline["peak_source"]},
+        "roofline": roofline, "routing": routing, "kernels": breakdown, "gpu_launches": launches,
+        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,498 @@
+// Host side of libmoe.so: argument validation, workspace layout, TMA tensor
+// maps, the launch sequence of the forward and backward passes, the status
+// word and optional per-kernel event timing.  The C ABI is declared in
+// include/moe.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "moe.h"
+#include "moe_internal.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Plan {
+    int64_t T;
+    int d, E, k, I;
+    int64_t P;          // T*k pairs
+    int64_t p_cap;      // sorted-layout row capacity
+    int64_t m_tiles;    // p_cap / 128
+    int n_chunks;       // routing blocks
+    int bn_d;           // N tile of the GEMMs whose N is d
+    int bn_i;           // N tile of the GEMMs whose N is I
+    int cnt_stride;     // d / bn_d
+    int dpart_stride;   // I / bn_i
+    // workspace layout (byte offsets)
+    size_t ws_status, ws_cnt, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
+    size_t ws_dh, ws_dpart, bwd_bytes;
+    size_t saved[MOE_SAVED_FIELDS];
+};
+
+int make_plan(const moe_shape_t *s, Plan *p) {
+    if (!s) return MOE_ERR_ARG;
+    if (s->T < 1 || s->E < 1 || s->k < 1 || s->k > s->E || s->d < 1 || s->I < 1 || s->max_sms < 0)
+        return MOE_ERR_ARG;
+    if (s->E > kMaxExperts || s->k > kMaxTopK) return MOE_ERR_SHAPE;
+    if (s->d % 128 != 0 || s->I % 128 != 0) return MOE_ERR_SHAPE;
+    if (s->dtype != MOE_BF16) return s->dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_ARG;
+    const int64_t P = s->T * s->k;
+    const int64_t widest = s->d > 2 * s->I ? s->d : 2 * static_cast<int64_t>(s->I);
+    const int64_t nonempty = s->E < P ? s->E : P;
+    const int64_t p_cap = (P + 127 * nonempty + 127) / 128 * 128;
+    if (p_cap * widest >= (int64_t(1) << 31) || P * s->d >= (int64_t(1) << 31)) return MOE_ERR_SHAPE;
+    p->T = s->T;
+    p->d = s->d;
+    p->E = s->E;
+    p->k = s->k;
+    p->I = s->I;
+    p->P = P;
+    p->p_cap = p_cap;
+    p->m_tiles = p_cap / 128;
+    p->n_chunks = static_cast<int>((s->T + kRouteChunk - 1) / kRouteChunk);
+    p->bn_d = s->d % 256 == 0 ? 256 : 128;
+    p->bn_i = s->I % 256 == 0 ? 256 : 128;
+    p->cnt_stride = s->d / p->bn_d;
+    p->dpart_stride = s->I / p->bn_i;
+
+    size_t off = 0;
+    p->ws_status = off;
+    off = align_up(off + 16);
+    p->ws_cnt = off;
+    off = align_up(off + static_cast<size_t>(s->T) * p->cnt_stride * 4);
+    p->ws_stage = off;
+    off = align_up(off + static_cast<size_t>(P) * s->d * 2);
+    const size_t common = off;
+    p->ws_chunk_counts = off;
+    off = align_up(off + static_cast<size_t>(p->n_chunks) * s->E * 4);
+    p->ws_chunk_base = off;
+    off = align_up(off + static_cast<size_t>(p->n_chunks) * s->E * 4);
+    p->fwd_bytes = off;
+    off = common;
+    p->ws_dh = off;
+    off = align_up(off + static_cast<size_t>(p_cap) * 2 * s->I * 2);
+    p->ws_dpart = off;
+    off = align_up(off + static_cast<size_t>(p_cap) * p->dpart_stride * 4);
+    p->bwd_bytes = off;
+
+    const size_t Tk = static_cast<size_t>(P);
+    p->saved[0] = Tk * 4;                                   // topk_idx
+    p->saved[1] = Tk * 4;                                   // topk_w
+    p->saved[2] = static_cast<size_t>(s->E) * 4;            // counts
+    p->saved[3] = static_cast<size_t>(s->E + 1) * 4;        // offsets
+    p->saved[4] = static_cast<size_t>(s->E + 1) * 4;        // group_start
+    p->saved[5] = static_cast<size_t>(p->m_tiles) * 4;      // tile_expert
+    p->saved[6] = static_cast<size_t>(p_cap) * 4;           // perm
+    p->saved[7] = Tk * 4;                                   // inv
+    p->saved[8] = static_cast<size_t>(p_cap) * 2 * s->I * 2;  // h
+    p->saved[9] = static_cast<size_t>(p_cap) * s->I * 2;      // aw
+    return MOE_OK;
+}
+
+bool aligned16(const void *ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------
+// per-device properties
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    bool ok = false;
+    int sms = 0;
+    int major = 0, minor = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_info(DeviceInfo *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_dev[dev].ok) {
+        DeviceInfo d;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return MOE_ERR_LAUNCH;
+        d.ok = true;
+        g_dev[dev] = d;
+    }
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return MOE_ERR_LAUNCH;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = g_dev[dev];
+    if (out->major != 10 || out->minor != 0) return MOE_ERR_ARCH;
+    return MOE_OK;
+}
+
+// 2-d bf16 tensor [rows, cols] (row-major), box = box_rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint32_t box_rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// per-kernel timing (host bookkeeping only)
+// ---------------------------------------------------------------------------
+struct Timing {
+    bool on = false;
+    struct Rec {
+        int kind;
+        cudaEvent_t a, b;
+    };
+    std::vector<Rec> recs;
+    std::vector<cudaEvent_t> pool;
+};
+Timing g_tm;
+
+cudaEvent_t take_event() {
+    if (!g_tm.pool.empty()) {
+        cudaEvent_t e = g_tm.pool.back();
+        g_tm.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+struct Launch {
+    int kind;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    Launch(int k, cudaStream_t st) : kind(k), s(st) {
+        if (g_tm.on) {
+            std::lock_guard<std::mutex> lock(g_mu);
+            a = take_event();
+            b = take_event();
+            if (a) cudaEventRecord(a, s);
+        }
+    }
+    int done(cudaError_t e) {
+        if (a && b) {
+            cudaEventRecord(b, s);
+            std::lock_guard<std::mutex> lock(g_mu);
+            g_tm.recs.push_back({kind, a, b});
+        }
+        return e == cudaSuccess ? MOE_OK : MOE_ERR_LAUNCH;
+    }
+};
+
+const char *kKindNames[kNumKernelKinds] = {
+    "route_topk",       "route_scan",       "route_perm",           "gemm_gateup_fwd",      "gemm_down_fwd_combine",
+    "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd"};
+
+struct Saved {
+    int32_t *idx;
+    float *w;
+    int32_t *counts, *offsets, *group_start, *tile_expert, *perm, *inv;
+    __nv_bfloat16 *h, *aw;
+};
+
+int check_saved(const moe_saved_t *s) {
+    if (!s) return MOE_ERR_ARG;
+    const void *ptrs[MOE_SAVED_FIELDS] = {s->topk_idx, s->topk_w, s->counts, s->offsets, s->group_start,
+                                         s->tile_expert, s->perm, s->inv, s->h, s->aw};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+int grid_for(const moe_shape_t *s, const DeviceInfo &dev) {
+    int g = dev.sms;
+    if (s->max_sms > 0 && s->max_sms < g) g = s->max_sms;
+    return g;
+}
+
+int run_route(const moe_shape_t *shape, const Plan &pl, const float *logits, moe_saved_t *saved, uint8_t *ws,
+              cudaStream_t st) {
+    int *status = reinterpret_cast<int *>(ws + pl.ws_status);
+    int32_t *chunk_counts = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_counts);
+    int32_t *chunk_base = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_base);
+    int32_t *cnt = reinterpret_cast<int32_t *>(ws + pl.ws_cnt);
+    (void)shape;
+    int rc;
+    {
+        Launch L(kKindRouteTopk, st);
+        rc = L.done(launch_route_topk(logits, static_cast<int>(pl.T), pl.E, pl.k, saved->topk_idx, saved->topk_w,
+                                      chunk_counts, cnt, pl.cnt_stride, st));
+        if (rc) return rc;
+    }
+    {
+        Launch L(kKindRouteScan, st);
+        rc = L.done(launch_route_scan(static_cast<int>(pl.T), pl.E, pl.n_chunks, chunk_counts, chunk_base,
+                                      saved->counts, saved->offsets, saved->group_start, saved->tile_expert,
+                                      saved->perm, pl.p_cap, status, st));
+        if (rc) return rc;
+    }
+    {
+        Launch L(kKindRoutePerm, st);
+        rc = L.done(launch_route_perm(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_idx, chunk_base, saved->perm,
+                                      saved->inv, pl.p_cap, status, st));
+    }
+    return rc;
+}
+
+GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.T = static_cast<int>(pl.T);
+    a.d = pl.d;
+    a.E = pl.E;
+    a.k = pl.k;
+    a.I = pl.I;
+    a.cnt_stride = pl.cnt_stride;
+    a.dpart_stride = pl.dpart_stride;
+    a.perm = sv->perm;
+    a.group_start = sv->group_start;
+    a.tile_expert = sv->tile_expert;
+    a.topk_w = sv->topk_w;
+    a.h = reinterpret_cast<__nv_bfloat16 *>(sv->h);
+    a.aw = reinterpret_cast<__nv_bfloat16 *>(sv->aw);
+    a.stage = reinterpret_cast<__nv_bfloat16 *>(ws + pl.ws_stage);
+    a.cnt = reinterpret_cast<int *>(ws + pl.ws_cnt);
+    a.status = reinterpret_cast<int *>(ws + pl.ws_status);
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_saved_sizes(const moe_shape_t *shape, size_t sizes[MOE_SAVED_FIELDS], int64_t *p_cap) {
+    Plan pl;
+    const int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (sizes)
+        for (int i = 0; i < MOE_SAVED_FIELDS; ++i) sizes[i] = pl.saved[i];
+    if (p_cap) *p_cap = pl.p_cap;
+    return MOE_OK;
+}
+
+int moe_workspace_size(const moe_shape_t *shape, size_t *fwd_bytes, size_t *bwd_bytes) {
+    Plan pl;
+    const int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (fwd_bytes) *fwd_bytes = pl.fwd_bytes;
+    if (bwd_bytes) *bwd_bytes = pl.bwd_bytes;
+    return MOE_OK;
+}
+
+int moe_route(const moe_shape_t *shape, const float *logits, moe_saved_t *saved, void *ws, size_t ws_bytes,
+              void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(logits) || !aligned16(ws) || (rc = check_saved(saved))) return rc ? rc : MOE_ERR_ARG;
+    if (ws_bytes < pl.fwd_bytes) return MOE_ERR_WS;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    return run_route(shape, pl, logits, saved, w8, st);
+}
+
+int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const void *w_gate_up, const void *w_down,
+            void *out, moe_saved_t *saved, void *ws, size_t ws_bytes, void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(x) || !aligned16(logits) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out) ||
+        !aligned16(ws))
+        return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    if (ws_bytes < pl.fwd_bytes) return MOE_ERR_WS;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+
+    CUtensorMap tm_x, tm_wgu, tm_aw, tm_wd;
+    if (!make_map(&tm_x, x, pl.T, pl.d, 1) ||
+        !make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 128) ||
+        !make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) ||
+        !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
+        return MOE_ERR_LAUNCH;
+
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    if ((rc = run_route(shape, pl, logits, saved, w8, st))) return rc;
+    const int grid = grid_for(shape, dev);
+
+    GemmArgs a = base_args(pl, saved, w8);
+    a.n_tiles = pl.I / 128;
+    a.num_k_blocks = pl.d / kTileK;
+    {
+        Launch L(kKindGemmGateUpFwd, st);
+        if ((rc = L.done(launch_gemm(kGateUpFwd, 256, a, tm_x, tm_wgu, grid, st)))) return rc;
+    }
+    a.n_tiles = pl.d / pl.bn_d;
+    a.num_k_blocks = pl.I / kTileK;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    {
+        Launch L(kKindGemmDownFwd, st);
+        rc = L.done(launch_gemm(kDownFwd, pl.bn_d, a, tm_aw, tm_wd, grid, st));
+    }
+    return rc;
+}
+
+int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const void *w_gate_up, const void *w_down,
+            const moe_saved_t *saved, void *dx, void *dw_gate_up, void *dw_down, float *dscore, float *dlogits,
+            void *ws, size_t ws_bytes, void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(grad_out) || !aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(dx) ||
+        !aligned16(dw_gate_up) || !aligned16(dw_down) || !aligned16(dscore) || !aligned16(ws) ||
+        (dlogits && !aligned16(dlogits)))
+        return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    if (ws_bytes < pl.bwd_bytes) return MOE_ERR_WS;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    __nv_bfloat16 *dh = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_dh);
+    float *dpart = reinterpret_cast<float *>(w8 + pl.ws_dpart);
+
+    CUtensorMap tm_gout_rows, tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn, tm_x_rows;
+    const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I;
+    const int64_t Ed = static_cast<int64_t>(pl.E) * pl.d;
+    if (!make_map(&tm_gout_rows, grad_out, pl.T, pl.d, 1) || !make_map(&tm_wd_mn, w_down, Ed, pl.I, 64) ||
+        !make_map(&tm_dh_rows, dh, pl.p_cap, 2 * pl.I, 128) || !make_map(&tm_wgu_mn, w_gate_up, EI2, pl.d, 64) ||
+        !make_map(&tm_aw_mn, saved->aw, pl.p_cap, pl.I, 64) || !make_map(&tm_dh_mn, dh, pl.p_cap, 2 * pl.I, 64) ||
+        !make_map(&tm_x_rows, x, pl.T, pl.d, 1))
+        return MOE_ERR_LAUNCH;
+
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    const int grid = grid_for(shape, dev);
+    GemmArgs a = base_args(pl, const_cast<moe_saved_t *>(saved), w8);
+    a.dh = dh;
+    a.dpart = dpart;
+
+    // b1: down dgrad, dscore partials, SwiGLU backward -> dh; zeroes the dx counters
+    a.n_tiles = pl.I / pl.bn_i;
+    a.num_k_blocks = pl.d / kTileK;
+    {
+        Launch L(kKindGemmDownDgrad, st);
+        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, a, tm_gout_rows, tm_wd_mn, grid, st)))) return rc;
+    }
+    // b3: down wgrad  dW_down[e] = sum_p gout[t] (x) aw_p
+    a.m_tiles = pl.d / kTileM;
+    a.n_tiles = pl.I / pl.bn_i;
+    a.dw = static_cast<__nv_bfloat16 *>(dw_down);
+    {
+        Launch L(kKindGemmDownWgrad, st);
+        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, a, tm_gout_rows, tm_aw_mn, grid, st)))) return rc;
+    }
+    // b4: gate/up dgrad + ordered scatter-sum into dx
+    a.n_tiles = pl.d / pl.bn_d;
+    a.num_k_blocks = 2 * pl.I / kTileK;
+    a.out = static_cast<__nv_bfloat16 *>(dx);
+    {
+        Launch L(kKindGemmGateUpDgrad, st);
+        if ((rc = L.done(launch_gemm(kGateUpDgrad, pl.bn_d, a, tm_dh_rows, tm_wgu_mn, grid, st)))) return rc;
+    }
+    // b5: gate/up wgrad  dW_gu[e] = sum_p dh_p (x) x[t]
+    a.m_tiles = 2 * pl.I / kTileM;
+    a.n_tiles = pl.d / pl.bn_d;
+    a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
+    {
+        Launch L(kKindGemmGateUpWgrad, st);
+        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, a, tm_dh_mn, tm_x_rows, grid, st)))) return rc;
+    }
+    // b6: dscore (ordered sum of partials) and dlogits
+    {
+        Launch L(kKindRouteBwd, st);
+        rc = L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_w, saved->topk_idx, saved->inv,
+                                     dpart, pl.dpart_stride, dscore, dlogits, st));
+    }
+    return rc;
+}
+
+int moe_get_status(const void *ws, void *stream, int *device_status) {
+    if (!ws || !device_status) return MOE_ERR_ARG;
+    int h = 0;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_LAUNCH;
+    if (cudaMemcpy(&h, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_LAUNCH;
+    *device_status = h == kStatusOk ? MOE_OK : (h == kStatusTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE);
+    return MOE_OK;
+}
+
+const char *moe_error_string(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument (null or misaligned pointer, or k/T/E out of range)";
+        case MOE_ERR_SHAPE: return "unsupported shape (d and I must be multiples of 128; E <= 512; k <= 64)";
+        case MOE_ERR_WS: return "workspace too small";
+        case MOE_ERR_ARCH: return "device is not an sm_100 (B200-class) GPU";
+        case MOE_ERR_LAUNCH: return "CUDA launch or runtime call failed";
+        case MOE_ERR_TIMEOUT: return "a device-side bounded wait expired";
+        case MOE_ERR_DEVICE: return "a device-side index check failed";
+        case MOE_ERR_UNSUPPORTED: return "dtype not implemented";
+        default: return "unknown error code";
+    }
+}
+
+int moe_profile_enable(int on) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_tm.on = on != 0;
+    return MOE_OK;
+}
+
+int moe_profile_read(double *ms, int64_t *launches, int n_kinds) {
+    std::vector<Timing::Rec> recs;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        recs.swap(g_tm.recs);
+    }
+    for (int i = 0; i < n_kinds; ++i) {
+        if (ms) ms[i] = 0.0;
+        if (launches) launches[i] = 0;
+    }
+    int rc = MOE_OK;
+    for (auto &r : recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            rc = MOE_ERR_LAUNCH;
+        if (r.kind < n_kinds) {
+            if (ms) ms[r.kind] += t;
+            if (launches) launches[r.kind] += 1;
+        }
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (auto &r : recs) {
+        g_tm.pool.push_back(r.a);
+        g_tm.pool.push_back(r.b);
+    }
+    return rc;
+}
+
+const char *moe_kernel_name(int kind) {
+    if (kind < 0 || kind >= kNumKernelKinds) return nullptr;
+    return kKindNames[kind];
+}
+
+}  // extern "C"

@@ -1,0 +1,593 @@
+// Persistent grouped GEMMs of the fused MoE layer on the sm_100a tensor cores.
+//
+// One kernel template serves the six expert GEMMs of the layer (two forward,
+// four backward).  Each CTA owns one SM and walks a static list of output
+// tiles.  Inside a CTA the work is split by warp:
+//   warp 0      producer: TMA loads of A and B K-blocks into a 4- or 6-stage
+//               shared-memory ring.  Token rows are fetched with the TMA row
+//               gather (tile::gather4) straight from x or grad_out through the
+//               dispatch permutation, so no permuted copy of the tokens exists.
+//   warp 1      allocates tensor memory and issues tcgen05.mma (one thread),
+//               accumulating a 128 x BN fp32 tile in TMEM; two TMEM buffers
+//               let the epilogue of one tile overlap the mainloop of the next.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               output row per thread) and the fused per-mode epilogue.
+//
+// Modes (see GemmMode): the expert MLP of "Prime Intellect Fused MoE Kernel:
+// 3.11x MoE Training Speed", section "What a mixture-of-experts layer actually
+// does" (both expert linear layers and SwiGLU), the combine back into token
+// order, and for the backward pass (the exchange repeated for gradients,
+// "Prime Intellect's Prime Mega MoE Trains Giant AI Models 55% Faster", section
+// "Where MoE training loses time") the two dgrads, the two wgrads and the
+// scatter of token gradients back to token order.
+//
+// The combine and the scatter are deterministic: each (token, slot) row writes
+// its tile slice to a slot-addressed staging buffer and bumps a per-(token,
+// column tile) counter; the row that brings the counter to k sums the k slots
+// in slot order.  No thread ever waits on another CTA.
+//
+// Every wait on an mbarrier is bounded in time.  On expiry the kernel records
+// a timeout in the status word, stops issuing work, waits (bounded) for its own
+// copies and MMAs in flight, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB: 128 rows x 64 bf16
+constexpr int kChunkBytes = 64 * kTileK * 2;  // 8 KB: one 64-wide MN chunk of an MN-major K-block
+constexpr uint32_t kSbo = 1024;               // 8 rows x 128 B swizzle atom
+constexpr uint32_t kMnLbo = kChunkBytes;      // MN-major: distance between 64-wide chunks
+
+template <int BN>
+struct Cfg {
+    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kBBytes = BN * kTileK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kBarOffset = kStages * kStageBytes;
+    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1 KB alignment slack
+    static constexpr uint32_t kTmemCols = 2 * BN;
+};
+
+template <int MODE>
+struct ModeTraits {
+    static constexpr bool kMTiled = MODE <= kGateUpDgrad;            // M = sorted rows
+    static constexpr bool kAGather = MODE == kGateUpFwd || MODE == kDownDgrad || MODE == kDownWgrad;
+    static constexpr bool kBGather = MODE == kGateUpWgrad;  // only the gate/up wgrad gathers B
+    static constexpr bool kAMn = MODE == kDownWgrad || MODE == kGateUpWgrad;
+    static constexpr bool kBMn = MODE == kDownDgrad || MODE == kGateUpDgrad || MODE == kDownWgrad ||
+                                 MODE == kGateUpWgrad;
+};
+
+struct Tile {
+    int e;      // expert
+    int mt;     // M tile
+    int nt;     // N tile
+    int nkb;    // K blocks
+    int kpos0;  // wgrad: first sorted row of the expert's group
+};
+
+template <int MODE>
+__device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a) {
+    Tile t;
+    if constexpr (ModeTraits<MODE>::kMTiled) {
+        t.mt = tile / a.n_tiles;
+        t.nt = tile - t.mt * a.n_tiles;
+        t.e = __ldg(a.tile_expert + t.mt);
+        t.nkb = a.num_k_blocks;
+        t.kpos0 = 0;
+    } else {
+        const int per = a.m_tiles * a.n_tiles;
+        t.e = tile / per;
+        const int r = tile - t.e * per;
+        t.mt = r / a.n_tiles;
+        t.nt = r - t.mt * a.n_tiles;
+        const int gs = __ldg(a.group_start + t.e), ge = __ldg(a.group_start + t.e + 1);
+        t.nkb = (ge - gs) / kTileK;
+        t.kpos0 = gs;
+    }
+    if (t.e < 0 || t.e >= a.E) {  // corrupted routing state: do no work for this tile
+        t.e = 0;
+        t.nkb = 0;
+    }
+    return t;
+}
+
+template <int MODE>
+__device__ __forceinline__ int total_tiles(const GemmArgs &a) {
+    if constexpr (ModeTraits<MODE>::kMTiled) {
+        return (__ldg(a.group_start + a.E) / kTileM) * a.n_tiles;
+    } else {
+        return a.E * a.m_tiles * a.n_tiles;
+    }
+}
+
+// Token row of a sorted position (padding rows read token 0; their products
+// are masked or multiplied by zero rows of the other operand).
+__device__ __forceinline__ int token_of(const GemmArgs &a, int pos) {
+    const int p = __ldg(a.perm + pos);
+    if (p < 0 || p >= a.T * a.k) return 0;
+    return p / a.k;
+}
+
+__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const uint32_t (&p)[16]) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+}
+
+__device__ __forceinline__ void load_row32(const __nv_bfloat16 *src, uint32_t (&p)[16]) {
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = s4[i];
+        p[4 * i] = v.x;
+        p[4 * i + 1] = v.y;
+        p[4 * i + 2] = v.z;
+        p[4 * i + 3] = v.w;
+    }
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ void raise_abort(volatile int *abort_flag, int *status) {
+    *abort_flag = 1;
+    report_status(status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// producer (warp 0)
+// ---------------------------------------------------------------------------
+template <int MODE, int BN>
+__device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, const GemmArgs &a, uint8_t *smem,
+                              uint64_t *full, uint64_t *empty, volatile int *abort_flag) {
+    using C = Cfg<BN>;
+    using TR = ModeTraits<MODE>;
+    const int lane = threadIdx.x & 31;
+    const int total = total_tiles<MODE>(a);
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const Tile t = decode_tile<MODE>(tile, a);
+        int tok[4] = {0, 0, 0, 0};
+        if constexpr (TR::kMTiled && TR::kAGather) {
+            const int pos = t.mt * kTileM + 4 * lane;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tok[i] = token_of(a, pos + i);
+        }
+        for (int kb = 0; kb < t.nkb; ++kb) {
+            const int s = it % C::kStages;
+            const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
+            if (!warp_wait(&empty[s], ph ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            __syncwarp();
+            uint8_t *As = smem + s * C::kStageBytes;
+            uint8_t *Bs = As + kABytes;
+            const int k0 = kb * kTileK;
+            if constexpr (!TR::kMTiled) {
+                // wgrad: the K block is 64 sorted rows of expert e; 16 groups of 4
+                const int g = lane & 15;
+                const int pos = t.kpos0 + k0 + 4 * g;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tok[i] = TR::kAGather || TR::kBGather ? token_of(a, pos + i) : 0;
+            }
+            if constexpr (MODE == kGateUpFwd) {
+                tma_gather4(As + lane * 512, tmA, &full[s], k0, tok[0], tok[1], tok[2], tok[3]);
+                if (lane == 0) {
+                    const int row = t.e * 2 * a.I + t.nt * (BN / 2);
+                    tma_load_2d(Bs, tmB, &full[s], k0, row);                         // gate rows
+                    tma_load_2d(Bs + (BN / 2) * 128, tmB, &full[s], k0, row + a.I);  // up rows
+                }
+            } else if constexpr (MODE == kDownFwd) {
+                if (lane == 0) {
+                    tma_load_2d(As, tmA, &full[s], k0, t.mt * kTileM);
+                    tma_load_2d(Bs, tmB, &full[s], k0, t.e * a.d + t.nt * BN);
+                }
+            } else if constexpr (MODE == kDownDgrad) {
+                tma_gather4(As + lane * 512, tmA, &full[s], k0, tok[0], tok[1], tok[2], tok[3]);
+                if (lane < BN / 64) tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.e * a.d + k0);
+            } else if constexpr (MODE == kGateUpDgrad) {
+                if (lane == 0) tma_load_2d(As, tmA, &full[s], k0, t.mt * kTileM);
+                if (lane < BN / 64)
+                    tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.e * 2 * a.I + k0);
+            } else if constexpr (MODE == kDownWgrad) {
+                const int c = lane >> 4, g = lane & 15;
+                tma_gather4(As + c * kChunkBytes + g * 512, tmA, &full[s], t.mt * kTileM + 64 * c, tok[0], tok[1],
+                            tok[2], tok[3]);
+                if (lane < BN / 64) tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.kpos0 + k0);
+            } else {  // kGateUpWgrad
+                if (lane < 2) tma_load_2d(As + lane * kChunkBytes, tmA, &full[s], t.mt * kTileM + 64 * lane, t.kpos0 + k0);
+                const int g = lane & 15;
+                for (int c = lane >> 4; c < BN / 64; c += 2)
+                    tma_gather4(Bs + c * kChunkBytes + g * 512, tmB, &full[s], t.nt * BN + 64 * c, tok[0], tok[1],
+                                tok[2], tok[3]);
+            }
+            ++it;
+        }
+    }
+    if (!ok) {
+        raise_abort(abort_flag, a.status);
+        // let the copies already issued land before the CTA can exit
+        if (lane == 0) {
+            for (int i = it > C::kStages ? it - C::kStages : 0; i < it; ++i)
+                mbar_wait(&full[i % C::kStages], static_cast<uint32_t>(i / C::kStages) & 1u, nullptr);
+        }
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (warp 1, one thread)
+// ---------------------------------------------------------------------------
+template <int MODE, int BN>
+__device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty, uint64_t *tfull,
+                         uint64_t *tempty, uint64_t *drain, uint32_t tmem_base, volatile int *abort_flag) {
+    using C = Cfg<BN>;
+    using TR = ModeTraits<MODE>;
+    constexpr uint32_t kIdesc = instr_desc_bf16(kTileM, BN, TR::kAMn, TR::kBMn);
+    const int total = total_tiles<MODE>(a);
+    int it = 0, local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+        const Tile t = decode_tile<MODE>(tile, a);
+        const int acc = local & 1;
+        const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+            const int s = it % C::kStages;
+            const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
+            if (!mbar_wait(&full[s], ph, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
+            const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+                const uint64_t ad = TR::kAMn ? smem_desc_sw128(a_base + kk * 2048, kMnLbo, kSbo)
+                                             : smem_desc_sw128(a_base + kk * 32, 16, kSbo);
+                const uint64_t bd = TR::kBMn ? smem_desc_sw128(b_base + kk * 2048, kMnLbo, kSbo)
+                                             : smem_desc_sw128(b_base + kk * 32, 16, kSbo);
+                mma_bf16(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+    }
+    if (!ok) {
+        raise_abort(abort_flag, a.status);
+        mma_commit(drain);
+        mbar_wait(drain, 0u, nullptr);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// epilogues (warps 2..5; thread = one accumulator row)
+// ---------------------------------------------------------------------------
+template <int BN>
+__device__ __forceinline__ void release_accumulator(uint64_t *tempty_acc) {
+    tc_fence_before_sync();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(tempty_acc);
+}
+
+// gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up
+template <int BN>
+__device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
+                                               uint64_t *tempty_acc) {
+    constexpr int kHalf = BN / 2;
+    const int pos = t.mt * kTileM + r;
+    const int p = __ldg(a.perm + pos);
+    const bool valid = p >= 0 && p < a.T * a.k;
+    const float wv = valid ? __ldg(a.topk_w + p) : 0.f;
+    __nv_bfloat16 *hrow = a.h + static_cast<size_t>(pos) * 2 * a.I + t.nt * kHalf;
+    __nv_bfloat16 *arow = a.aw + static_cast<size_t>(pos) * a.I + t.nt * kHalf;
+#pragma unroll 1
+    for (int c = 0; c < kHalf / 32; ++c) {
+        uint32_t gr[32], ur[32];
+        tmem_load32(taddr + c * 32, gr);
+        tmem_load32(taddr + kHalf + c * 32, ur);
+        tmem_load_wait();
+        tmem_regs_ready(gr);
+        tmem_regs_ready(ur);
+        float g[32], u[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            g[i] = __uint_as_float(gr[i]);
+            u[i] = __uint_as_float(ur[i]);
+        }
+        uint32_t pg[16], pu[16], pa[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (valid) {
+                const float g0 = g[2 * i], g1 = g[2 * i + 1], u0 = u[2 * i], u1 = u[2 * i + 1];
+                const float s0 = __fdividef(1.f, 1.f + __expf(-g0));
+                const float s1 = __fdividef(1.f, 1.f + __expf(-g1));
+                pg[i] = pack_bf16x2(g0, g1);
+                pu[i] = pack_bf16x2(u0, u1);
+                pa[i] = pack_bf16x2(wv * g0 * s0 * u0, wv * g1 * s1 * u1);
+            } else {
+                pg[i] = pu[i] = pa[i] = 0u;
+            }
+        }
+        store_row32(hrow + c * 32, pg);
+        store_row32(hrow + a.I + c * 32, pu);
+        store_row32(arow + c * 32, pa);
+    }
+    release_accumulator<BN>(tempty_acc);
+}
+
+// down forward / gate-up dgrad: stage the slot's row slice, last arriver sums slots in order
+template <int BN>
+__device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
+                                           uint64_t *tempty_acc) {
+    const int pos = t.mt * kTileM + r;
+    const int p = __ldg(a.perm + pos);
+    const bool valid = p >= 0 && p < a.T * a.k;
+    const int col0 = t.nt * BN;
+    __nv_bfloat16 *srow = a.stage + static_cast<size_t>(valid ? p : 0) * a.d + col0;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_load32_sync(taddr + c * 32, v);
+        if (valid) {
+            uint32_t pv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            store_row32(srow + c * 32, pv);
+        }
+    }
+    release_accumulator<BN>(tempty_acc);
+    if (!valid) return;
+    const int tok = p / a.k;
+    __threadfence();
+    int *ctr = a.cnt + static_cast<size_t>(tok) * a.cnt_stride + t.nt;
+    const int arrived = atomicAdd(ctr, 1);
+    if (arrived != a.k - 1) return;
+    __threadfence();
+    const __nv_bfloat16 *slots = a.stage + static_cast<size_t>(tok) * a.k * a.d + col0;
+    __nv_bfloat16 *orow = a.out + static_cast<size_t>(tok) * a.d + col0;
+#pragma unroll 1
+    for (int col = 0; col < BN; col += 8) {
+        float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < a.k; ++j) {  // slot order
+            const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(slots + static_cast<size_t>(j) * a.d + col));
+            acc8[0] += bf16_lo(u.x);
+            acc8[1] += bf16_hi(u.x);
+            acc8[2] += bf16_lo(u.y);
+            acc8[3] += bf16_hi(u.y);
+            acc8[4] += bf16_lo(u.z);
+            acc8[5] += bf16_hi(u.z);
+            acc8[6] += bf16_lo(u.w);
+            acc8[7] += bf16_hi(u.w);
+        }
+        *reinterpret_cast<uint4 *>(orow + col) =
+            make_uint4(pack_bf16x2(acc8[0], acc8[1]), pack_bf16x2(acc8[2], acc8[3]), pack_bf16x2(acc8[4], acc8[5]),
+                       pack_bf16x2(acc8[6], acc8[7]));
+    }
+    *ctr = 0;  // ready for the next call
+}
+
+// down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh
+template <int BN>
+__device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
+                                               uint64_t *tempty_acc) {
+    const int pos = t.mt * kTileM + r;
+    const int p = __ldg(a.perm + pos);
+    const bool valid = p >= 0 && p < a.T * a.k;
+    const float wv = valid ? __ldg(a.topk_w + p) : 0.f;
+    const __nv_bfloat16 *hrow = a.h + static_cast<size_t>(pos) * 2 * a.I + t.nt * BN;
+    __nv_bfloat16 *dhrow = a.dh + static_cast<size_t>(pos) * 2 * a.I + t.nt * BN;
+    float ds = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        float G[32];
+        tmem_load32_sync(taddr + c * 32, G);
+        uint32_t pdg[16], pdu[16];
+        if (valid) {
+            uint32_t hg[16], hu[16];
+            load_row32(hrow + c * 32, hg);
+            load_row32(hrow + a.I + c * 32, hu);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float dgv[2], duv[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const float g = h2 ? bf16_hi(hg[i]) : bf16_lo(hg[i]);
+                    const float u = h2 ? bf16_hi(hu[i]) : bf16_lo(hu[i]);
+                    const float gr = G[2 * i + h2];
+                    const float sg = __fdividef(1.f, 1.f + __expf(-g));
+                    const float sl = g * sg;
+                    ds += gr * (sl * u);
+                    const float da = wv * gr;
+                    dgv[h2] = da * u * sg * (1.f + g * (1.f - sg));
+                    duv[h2] = da * sl;
+                }
+                pdg[i] = pack_bf16x2(dgv[0], dgv[1]);
+                pdu[i] = pack_bf16x2(duv[0], duv[1]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pdg[i] = pdu[i] = 0u;
+        }
+        store_row32(dhrow + c * 32, pdg);
+        store_row32(dhrow + a.I + c * 32, pdu);
+    }
+    release_accumulator<BN>(tempty_acc);
+    a.dpart[static_cast<size_t>(pos) * a.dpart_stride + t.nt] = valid ? ds : 0.f;
+    if (valid && t.nt == 0) {  // counters of the dx scatter that follows
+        const int tok = p / a.k;
+        for (int c = 0; c < a.cnt_stride; ++c) a.cnt[static_cast<size_t>(tok) * a.cnt_stride + c] = 0;
+    }
+}
+
+// weight gradients: store the tile (zeros for an expert without tokens)
+template <int MODE, int BN>
+__device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
+                                          uint64_t *tempty_acc) {
+    const int Mtot = MODE == kDownWgrad ? a.d : 2 * a.I;
+    const int Ntot = MODE == kDownWgrad ? a.I : a.d;
+    __nv_bfloat16 *row =
+        a.dw + (static_cast<size_t>(t.e) * Mtot + t.mt * kTileM + r) * static_cast<size_t>(Ntot) + t.nt * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pv[16];
+        if (t.nkb > 0) {
+            float v[32];
+            tmem_load32_sync(taddr + c * 32, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pv[i] = 0u;
+        }
+        store_row32(row + c * 32, pv);
+    }
+    release_accumulator<BN>(tempty_acc);
+}
+
+template <int MODE, int BN>
+__device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *tempty, uint32_t tmem_base,
+                              volatile int *abort_flag) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quad = warp & 3;  // TMEM lanes this warp may access: 32*quad .. 32*quad+31
+    const int r = quad * 32 + lane;
+    const int total = total_tiles<MODE>(a);
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+        const Tile t = decode_tile<MODE>(tile, a);
+        const int acc = local & 1;
+        const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
+        if (!warp_wait(&tfull[acc], aph, abort_flag)) {
+            raise_abort(abort_flag, a.status);
+            return;
+        }
+        tc_fence_after_sync();
+        const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
+        if constexpr (MODE == kGateUpFwd) {
+            epi_gateup_fwd<BN>(a, t, r, taddr, &tempty[acc]);
+        } else if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
+            epi_combine<BN>(a, t, r, taddr, &tempty[acc]);
+        } else if constexpr (MODE == kDownDgrad) {
+            epi_down_dgrad<BN>(a, t, r, taddr, &tempty[acc]);
+        } else {
+            epi_wgrad<MODE, BN>(a, t, r, taddr, &tempty[acc]);
+        }
+    }
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmArgs args) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
+    uint64_t *empty = full + C::kStages;
+    uint64_t *tfull = empty + C::kStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        producer_loop<MODE, BN>(&tmA, &tmB, args, smem, full, empty, abort_flag);
+    } else if (warp == 1) {
+        if ((threadIdx.x & 31) == 0)
+            mma_loop<MODE, BN>(args, smem, full, empty, tfull, tempty, drain, tmem_base, abort_flag);
+        __syncwarp();
+    } else {
+        epilogue_loop<MODE, BN>(args, tfull, tempty, tmem_base, abort_flag);
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+template <int MODE, int BN>
+cudaError_t launch_one(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
+                       cudaStream_t s) {
+    static bool attr_set = false;  // per instantiation; the attribute is per function and process-wide
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    grouped_gemm_kernel<MODE, BN><<<grid, kThreads, Cfg<BN>::kSmemBytes, s>>>(tmA, tmB, args);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_mode(int bn, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
+                        cudaStream_t s) {
+    if (bn == 256) return launch_one<MODE, 256>(args, tmA, tmB, grid, s);
+    if (bn == 128) return launch_one<MODE, 128>(args, tmA, tmB, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(GemmMode mode, int bn, const GemmArgs &args, const CUtensorMap &tmA,
+                        const CUtensorMap &tmB, int grid, cudaStream_t s) {
+    switch (mode) {
+        case kGateUpFwd: return launch_mode<kGateUpFwd>(bn, args, tmA, tmB, grid, s);
+        case kDownFwd: return launch_mode<kDownFwd>(bn, args, tmA, tmB, grid, s);
+        case kDownDgrad: return launch_mode<kDownDgrad>(bn, args, tmA, tmB, grid, s);
+        case kGateUpDgrad: return launch_mode<kGateUpDgrad>(bn, args, tmA, tmB, grid, s);
+        case kDownWgrad: return launch_mode<kDownWgrad>(bn, args, tmA, tmB, grid, s);
+        case kGateUpWgrad: return launch_mode<kGateUpWgrad>(bn, args, tmA, tmB, grid, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,81 @@
+// Declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Device status codes written to the workspace status word.
+enum : int { kStatusOk = 0, kStatusTimeout = 1, kStatusBadIndex = 2 };
+
+constexpr int kTileM = 128;       // rows of one GEMM tile (and the padding unit of an expert group)
+constexpr int kTileK = 64;        // K elements per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int kRouteChunk = 64;   // tokens per routing block
+constexpr int kMaxExperts = 512;
+constexpr int kMaxTopK = 64;
+
+// Kernel kinds, for per-kernel timing.
+enum KernelKind : int {
+    kKindRouteTopk = 0,
+    kKindRouteScan,
+    kKindRoutePerm,
+    kKindGemmGateUpFwd,
+    kKindGemmDownFwd,
+    kKindGemmDownDgrad,
+    kKindGemmDownWgrad,
+    kKindGemmGateUpDgrad,
+    kKindGemmGateUpWgrad,
+    kKindRouteBwd,
+    kNumKernelKinds
+};
+
+// Which GEMM of the layer a launch computes; selects operand loading and epilogue.
+enum GemmMode : int {
+    kGateUpFwd = 0,    // h = x[perm] W_gu[e]^T ; epilogue SwiGLU -> h, aw
+    kDownFwd = 1,      // y = aw W_down[e]^T   ; epilogue slot-ordered combine -> out
+    kDownDgrad = 2,    // G = gout[perm] W_down[e] ; epilogue dscore partials, SwiGLU bwd -> dh
+    kGateUpDgrad = 3,  // dx_p = dh W_gu[e]     ; epilogue slot-ordered scatter-sum -> dx
+    kDownWgrad = 4,    // dW_down[e] = gout[perm]^T aw
+    kGateUpWgrad = 5,  // dW_gu[e] = dh^T x[perm]
+};
+
+struct GemmArgs {
+    int T, d, E, k, I;
+    int n_tiles;          // tiles along N
+    int m_tiles;          // wgrad: tiles along M of one expert's weight
+    int num_k_blocks;     // M-tiled modes: K / 64
+    int cnt_stride;       // combine counters per token
+    int dpart_stride;     // dscore partials per sorted row
+    const int *perm;
+    const int *group_start;
+    const int *tile_expert;
+    const float *topk_w;
+    __nv_bfloat16 *h;
+    __nv_bfloat16 *aw;
+    __nv_bfloat16 *stage;
+    int *cnt;
+    __nv_bfloat16 *out;   // out (fwd) or dx (bwd)
+    __nv_bfloat16 *dh;
+    float *dpart;
+    __nv_bfloat16 *dw;    // weight gradient (wgrad modes)
+    int *status;
+};
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
+                              int32_t *chunk_counts, int32_t *cnt, int cnt_per_token, cudaStream_t s);
+cudaError_t launch_route_scan(int T, int E, int n_chunks, const int32_t *chunk_counts, int32_t *chunk_base,
+                              int32_t *counts, int32_t *offsets, int32_t *group_start, int32_t *tile_expert,
+                              int32_t *perm, int64_t p_cap, int *status, cudaStream_t s);
+cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int32_t *chunk_base, int32_t *perm,
+                              int32_t *inv, int64_t p_cap, int *status, cudaStream_t s);
+cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t *idx, const int32_t *inv,
+                             const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s);
+
+cudaError_t launch_gemm(GemmMode mode, int bn, const GemmArgs &args, const CUtensorMap &tmA,
+                        const CUtensorMap &tmB, int grid, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,228 @@
+"""Python binding of libmoe.so (the fused MoE layer's C ABI, include/moe.h).
+
+Argument marshalling only: every step of routing, dispatch, the expert GEMMs,
+SwiGLU, the combine and the backward runs inside the CUDA library.  PyTorch is
+used here only to allocate device memory and to name the current stream.  If
+the library is missing or no sm_100 GPU is present the calls raise; there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+MOE_BF16, MOE_MXFP8 = 0, 1
+MOE_OK = 0
+MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_WS, MOE_ERR_ARCH = -1, -2, -3, -4
+MOE_ERR_LAUNCH, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE, MOE_ERR_UNSUPPORTED = -5, -6, -7, -8
+
+SAVED_FIELDS = ("topk_idx", "topk_w", "counts", "offsets", "group_start", "tile_expert", "perm", "inv", "h", "aw")
+EXPORTS = ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
+           "moe_error_string", "moe_profile_enable", "moe_profile_read", "moe_kernel_name")
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("I", ctypes.c_int32), ("dtype", ctypes.c_int32), ("max_sms", ctypes.c_int32)]
+
+
+class MoeSaved(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in SAVED_FIELDS]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {code} ({error_string(code)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so once (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with grouped_gemm_route_b200.build.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    P, S = ctypes.c_void_p, ctypes.POINTER(MoeShape)
+    L.moe_saved_sizes.argtypes = [S, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_int64)]
+    L.moe_workspace_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_route.argtypes = [S, P, ctypes.POINTER(MoeSaved), P, ctypes.c_size_t, P]
+    L.moe_fwd.argtypes = [S, P, P, P, P, P, ctypes.POINTER(MoeSaved), P, ctypes.c_size_t, P]
+    L.moe_bwd.argtypes = [S, P, P, P, P, ctypes.POINTER(MoeSaved), P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
+    L.moe_error_string.argtypes = [ctypes.c_int]
+    L.moe_error_string.restype = ctypes.c_char_p
+    L.moe_profile_enable.argtypes = [ctypes.c_int]
+    L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
+    L.moe_kernel_name.argtypes = [ctypes.c_int]
+    L.moe_kernel_name.restype = ctypes.c_char_p
+    for name in ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
+                 "moe_profile_enable", "moe_profile_read"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def error_string(code: int) -> str:
+    try:
+        return lib().moe_error_string(int(code)).decode()
+    except Exception:  # library not loadable: still give a readable message
+        return "unknown"
+
+
+def _check(rc: int, where: str):
+    if rc != MOE_OK:
+        raise MoeError(rc, where)
+
+
+def make_shape(T, d, E, k, I, dtype=MOE_BF16, max_sms=0) -> MoeShape:
+    return MoeShape(int(T), int(d), int(E), int(k), int(I), int(dtype), int(max_sms))
+
+
+def saved_sizes(shape: MoeShape):
+    sizes = (ctypes.c_size_t * len(SAVED_FIELDS))()
+    p_cap = ctypes.c_int64()
+    _check(lib().moe_saved_sizes(ctypes.byref(shape), sizes, ctypes.byref(p_cap)), "moe_saved_sizes")
+    return [int(s) for s in sizes], int(p_cap.value)
+
+
+def workspace_size(shape: MoeShape):
+    f, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().moe_workspace_size(ctypes.byref(shape), ctypes.byref(f), ctypes.byref(b)), "moe_workspace_size")
+    return int(f.value), int(b.value)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def saved_struct(saved: dict) -> MoeSaved:
+    return MoeSaved(*[saved[n].data_ptr() for n in SAVED_FIELDS])
+
+
+def route(shape, logits, saved: dict, ws, stream=None):
+    st = saved_struct(saved)
+    _check(lib().moe_route(ctypes.byref(shape), _ptr(logits), ctypes.byref(st), _ptr(ws), ws.numel(),
+                           _stream(stream)), "moe_route")
+
+
+def fwd(shape, x, logits, wgu, wd, out, saved: dict, ws, stream=None):
+    st = saved_struct(saved)
+    _check(lib().moe_fwd(ctypes.byref(shape), _ptr(x), _ptr(logits), _ptr(wgu), _ptr(wd), _ptr(out),
+                         ctypes.byref(st), _ptr(ws), ws.numel(), _stream(stream)), "moe_fwd")
+
+
+def bwd(shape, gout, x, wgu, wd, saved: dict, dx, dwgu, dwd, dscore, dlogits, ws, stream=None):
+    st = saved_struct(saved)
+    _check(lib().moe_bwd(ctypes.byref(shape), _ptr(gout), _ptr(x), _ptr(wgu), _ptr(wd), ctypes.byref(st),
+                         _ptr(dx), _ptr(dwgu), _ptr(dwd), _ptr(dscore), _ptr(dlogits), _ptr(ws), ws.numel(),
+                         _stream(stream)), "moe_bwd")
+
+
+def get_status(ws, stream=None) -> int:
+    s = ctypes.c_int()
+    _check(lib().moe_get_status(_ptr(ws), _stream(stream), ctypes.byref(s)), "moe_get_status")
+    return int(s.value)
+
+
+def kernel_names():
+    names, i = [], 0
+    while True:
+        n = lib().moe_kernel_name(i)
+        if n is None:
+            return names
+        names.append(n.decode())
+        i += 1
+
+
+def profile_enable(on: bool):
+    _check(lib().moe_profile_enable(1 if on else 0), "moe_profile_enable")
+
+
+def profile_read():
+    """{kernel name: (summed ms, launches)} since the last read."""
+    names = kernel_names()
+    ms = (ctypes.c_double * len(names))()
+    n = (ctypes.c_int64 * len(names))()
+    _check(lib().moe_profile_read(ms, n, len(names)), "moe_profile_read")
+    return {name: (ms[i], int(n[i])) for i, name in enumerate(names)}
+
+
+# ----------------------------------------------------------------------------
+# buffer allocation for one layer (torch allocates, the library computes)
+# ----------------------------------------------------------------------------
+_SAVED_DTYPES = dict(topk_idx=torch.int32, topk_w=torch.float32, counts=torch.int32, offsets=torch.int32,
+                     group_start=torch.int32, tile_expert=torch.int32, perm=torch.int32, inv=torch.int32,
+                     h=torch.bfloat16, aw=torch.bfloat16)
+
+
+def alloc_saved(shape: MoeShape, device) -> dict:
+    sizes, p_cap = saved_sizes(shape)
+    T, E, k, I = shape.T, shape.E, shape.k, shape.I
+    shapes = dict(topk_idx=(T, k), topk_w=(T, k), counts=(E,), offsets=(E + 1,), group_start=(E + 1,),
+                  tile_expert=(p_cap // 128,), perm=(p_cap,), inv=(T, k), h=(p_cap, 2 * I), aw=(p_cap, I))
+    out = {}
+    for name, nbytes in zip(SAVED_FIELDS, sizes):
+        t = torch.empty(shapes[name], dtype=_SAVED_DTYPES[name], device=device)
+        assert t.numel() * t.element_size() == nbytes, name
+        out[name] = t
+    return out
+
+
+def alloc_workspace(shape: MoeShape, device) -> torch.Tensor:
+    f, b = workspace_size(shape)
+    return torch.empty(max(f, b), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class MoELayer:
+    """One fused MoE layer's buffers on a device; forward/backward call the C ABI."""
+    T: int
+    d: int
+    E: int
+    k: int
+    I: int
+    device: str = "cuda"
+    max_sms: int = 0
+
+    def __post_init__(self):
+        if not torch.cuda.is_available():
+            raise RuntimeError("the fused MoE layer needs a CUDA device (sm_100)")
+        self.shape = make_shape(self.T, self.d, self.E, self.k, self.I, MOE_BF16, self.max_sms)
+        self.saved = alloc_saved(self.shape, self.device)
+        self.ws = alloc_workspace(self.shape, self.device)
+        dev = self.device
+        self.out = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=dev)
+        self.dx = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=dev)
+        self.dwgu = torch.empty(self.E, 2 * self.I, self.d, dtype=torch.bfloat16, device=dev)
+        self.dwd = torch.empty(self.E, self.d, self.I, dtype=torch.bfloat16, device=dev)
+        self.dscore = torch.empty(self.T, self.k, dtype=torch.float32, device=dev)
+        self.dlogits = torch.empty(self.T, self.E, dtype=torch.float32, device=dev)
+
+    def forward(self, x, logits, wgu, wd, stream=None):
+        fwd(self.shape, x, logits, wgu, wd, self.out, self.saved, self.ws, stream)
+        return self.out
+
+    def backward(self, gout, x, wgu, wd, with_dlogits=True, stream=None):
+        bwd(self.shape, gout, x, wgu, wd, self.saved, self.dx, self.dwgu, self.dwd, self.dscore,
+            self.dlogits if with_dlogits else None, self.ws, stream)
+        return dict(dx=self.dx, dwgu=self.dwgu, dwd=self.dwd, dscore=self.dscore,
+                    dlogits=self.dlogits if with_dlogits else None)
+
+    def status(self, stream=None) -> int:
+        return get_status(self.ws, stream)

@@ -1,0 +1,158 @@
+/*
+ * moe.h -- C ABI of libmoe.so, a single-GPU fused mixture-of-experts layer
+ * (forward and backward) for NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes.  "Prime Intellect Fused MoE Kernel: 3.11x MoE
+ * Training Speed", section "What a mixture-of-experts layer actually does":
+ * a router sends each token to a few experts and one fused call performs the
+ * dispatch, both expert linear layers, SwiGLU and the combine.  "Prime
+ * Intellect's Prime Mega MoE Trains Giant AI Models 55% Faster", section
+ * "Where MoE training loses time": tokens are sorted by expert, the expert
+ * MLPs run, the outputs return to their original positions, and the backward
+ * pass repeats the exchange for gradients.  "Mario/overlap moe kernel
+ * integration (prime-rl PR #3651)", Overview and the custom-op commit note:
+ * the fused compute takes undispatched tokens plus their routing, runs in
+ * bf16 and returns gradients in the inputs' dtypes.  Here the expert-parallel
+ * network exchange of those pages becomes an on-GPU gather (dispatch) and an
+ * ordered reduction (combine / scatter).
+ *
+ * Definitions (P = T*k token-slot pairs; pair (t,j) is flat index t*k+j):
+ *   routing   idx[t,:] = the k largest logits[t,:] (ties -> lower expert index),
+ *             slot j = j-th largest; w[t,j] = exp(l_j - l_max) / sum over the
+ *             chosen k of exp(l_i - l_max)  (softmax renormalised over the k)
+ *   dispatch  counts[e] = #pairs routed to e; offsets = exclusive scan(counts);
+ *             pairs sorted by expert, tokens ascending inside an expert
+ *   expert    h = W_gate_up[e] x[t]  (W_gate_up[e] is [2I,d]: gate rows then up rows)
+ *             a = silu(h[0:I]) * h[I:2I];  y = W_down[e] a  (W_down[e] is [d,I])
+ *   combine   out[t] = sum_{j=0..k-1, in slot order} w[t,j] y_(t,j)
+ *   backward  dscore[t,j] = <gout[t], y_(t,j)>,  dx, dW_gate_up, dW_down,
+ *             dlogits[t,i] = w_i (dscore_i - sum_j w_j dscore_j) for chosen i, else 0
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers unless stated otherwise; every tensor is
+ *     row-major and contiguous.  bf16 = IEEE bfloat16 (2 bytes).
+ *   - The caller owns and allocates every buffer (outputs, saved state and the
+ *     workspace).  The library never allocates or frees device memory and keeps
+ *     no state between calls except cached per-device properties.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Calls that share a workspace must not overlap on the GPU.
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Arguments are
+ *     validated on the host before anything is launched; on an argument error
+ *     nothing is launched.  Device-side problems (a bounded wait that expired, an
+ *     out-of-range index) are recorded in a status word inside the workspace
+ *     and reported by moe_get_status.
+ *   - Shape limits: 1 <= k <= min(E, 64), E <= 512, d and I multiples of 128,
+ *     T >= 1, T*k*max(d,2I) < 2^31.  Pointers must be 16-byte aligned.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define MOE_OK 0
+#define MOE_ERR_ARG (-1)         /* null / misaligned pointer, k < 1, k > E, T < 1 ... */
+#define MOE_ERR_SHAPE (-2)       /* d or I not a multiple of 128, E or k above the limits */
+#define MOE_ERR_WS (-3)          /* workspace smaller than moe_workspace_size reports */
+#define MOE_ERR_ARCH (-4)        /* current device is not compute capability 10.0 */
+#define MOE_ERR_LAUNCH (-5)      /* a CUDA launch or runtime call failed */
+#define MOE_ERR_TIMEOUT (-6)     /* a device-side bounded wait expired (moe_get_status) */
+#define MOE_ERR_DEVICE (-7)      /* a device-side index check failed (moe_get_status) */
+#define MOE_ERR_UNSUPPORTED (-8) /* dtype not implemented */
+
+/* Operand precision of the expert GEMMs. */
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_dtype_t;
+
+/* Layer shape.  T tokens, hidden size d, E experts, top-k, expert width I.
+ * max_sms caps the persistent grids (0 = every SM). */
+typedef struct {
+    int64_t T;
+    int32_t d, E, k, I;
+    int32_t dtype;   /* moe_dtype_t */
+    int32_t max_sms;
+} moe_shape_t;
+
+/* State written by moe_fwd (and moe_route) and read by moe_bwd.  Every field
+ * is a caller-allocated device buffer of the size moe_saved_sizes reports, in
+ * this order.  "Sorted layout": pairs grouped by expert; expert e's group starts
+ * at row group_start[e], a multiple of 128, and holds counts[e] pairs followed by
+ * padding rows up to the next multiple of 128.  P_cap (the row capacity of the
+ * sorted layout) is reported by moe_saved_sizes. */
+typedef struct {
+    int32_t *topk_idx;    /* [T,k]   chosen experts, slot order                        */
+    float *topk_w;        /* [T,k]   renormalised routing weights                      */
+    int32_t *counts;      /* [E]     pairs per expert                                  */
+    int32_t *offsets;     /* [E+1]   exclusive scan of counts (unpadded)               */
+    int32_t *group_start; /* [E+1]   padded group starts; group_start[E] = rows used   */
+    int32_t *tile_expert; /* [P_cap/128] expert owning each 128-row tile               */
+    int32_t *perm;        /* [P_cap] sorted row -> pair t*k+j, or -1 for a padding row */
+    int32_t *inv;         /* [T,k]   pair -> sorted row                                */
+    void *h;              /* bf16 [P_cap, 2I] gate/up pre-activations, sorted layout   */
+    void *aw;             /* bf16 [P_cap, I]  w[t,j] * silu(gate) * up, sorted layout  */
+} moe_saved_t;
+
+#define MOE_SAVED_FIELDS 10
+
+/* Bytes of each moe_saved_t field (in declaration order) and the sorted-layout
+ * row capacity.  Pure host function; touches no GPU. */
+int moe_saved_sizes(const moe_shape_t *shape, size_t sizes[MOE_SAVED_FIELDS], int64_t *p_cap);
+
+/* Workspace bytes needed by moe_fwd and by moe_bwd (one buffer of the larger
+ * size serves both).  Pure host function; touches no GPU. */
+int moe_workspace_size(const moe_shape_t *shape, size_t *fwd_bytes, size_t *bwd_bytes);
+
+/* Routing and dispatch only (steps: top-k + weights, histogram + scan,
+ * stable permutation).  logits: fp32 [T,E].  Fills topk_idx, topk_w, counts,
+ * offsets, group_start, tile_expert, perm and inv of `saved`. */
+int moe_route(const moe_shape_t *shape, const float *logits, moe_saved_t *saved,
+              void *ws, size_t ws_bytes, void *stream);
+
+/* Forward.  x: bf16 [T,d]; logits: fp32 [T,E]; w_gate_up: bf16 [E,2I,d];
+ * w_down: bf16 [E,d,I]; out: bf16 [T,d].  Runs moe_route, then the gate/up
+ * grouped GEMM (tokens gathered by TMA from x, SwiGLU in the epilogue; writes
+ * saved->h and saved->aw), then the down grouped GEMM whose epilogue performs
+ * the weighted combine as a deterministic slot-ordered reduction into out. */
+int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits,
+            const void *w_gate_up, const void *w_down, void *out,
+            moe_saved_t *saved, void *ws, size_t ws_bytes, void *stream);
+
+/* Backward for a loss L with dL/dout = grad_out (bf16 [T,d]).  Reads the state
+ * moe_fwd saved.  Writes dx bf16 [T,d], dw_gate_up bf16 [E,2I,d], dw_down bf16
+ * [E,d,I], dscore fp32 [T,k] (gradient w.r.t. topk_w) and, when dlogits is not
+ * NULL, dlogits fp32 [T,E].  Experts that received no token get exact-zero
+ * weight gradients.  All reductions have a fixed order: results are bitwise
+ * reproducible. */
+int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x,
+            const void *w_gate_up, const void *w_down, const moe_saved_t *saved,
+            void *dx, void *dw_gate_up, void *dw_down, float *dscore, float *dlogits,
+            void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then reads the device status word of `ws` written by
+ * the most recent moe_route / moe_fwd / moe_bwd on that workspace:
+ * *device_status = MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE.  Returns MOE_OK
+ * or MOE_ERR_LAUNCH if the copy itself failed. */
+int moe_get_status(const void *ws, void *stream, int *device_status);
+
+/* Static string for a return code.  Never NULL. */
+const char *moe_error_string(int code);
+
+/* Per-kernel timing.  While enabled, every launch made by the library is
+ * bracketed by two CUDA events on its stream.  moe_profile_read synchronises
+ * the recorded events and returns, per kernel kind (0 <= kind < n_kinds), the
+ * summed device milliseconds and the launch count since the last reset, then
+ * resets.  moe_kernel_name names a kind ("route_topk", "gemm_gateup_fwd" ...),
+ * or returns NULL past the last kind.  Host-side bookkeeping only. */
+int moe_profile_enable(int on);
+int moe_profile_read(double *ms, int64_t *launches, int n_kinds);
+const char *moe_kernel_name(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

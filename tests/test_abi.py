@@ -1,0 +1,86 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry
+point, sizes its buffers, and rejects bad arguments on the host before any GPU
+work (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from grouped_gemm_route_b200 import build as B
+from grouped_gemm_route_b200 import moe as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return M.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(M.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_sizes_for_the_30b_shape(lib):
+    sh = M.make_shape(16384, 2048, 128, 8, 768)
+    sizes, p_cap = M.saved_sizes(sh)
+    P = 16384 * 8
+    assert p_cap % 128 == 0 and P <= p_cap <= P + 128 * 128
+    assert sizes[0] == P * 4 and sizes[8] == p_cap * 2 * 768 * 2 and sizes[9] == p_cap * 768 * 2
+    f, b = M.workspace_size(sh)
+    assert f >= P * 2048 * 2 and b >= p_cap * 2 * 768 * 2
+
+
+@pytest.mark.parametrize("T,d,E,k,I,dtype,code", [
+    (0, 256, 8, 2, 128, 0, M.MOE_ERR_ARG),
+    (16, 256, 8, 0, 128, 0, M.MOE_ERR_ARG),
+    (16, 256, 8, 9, 128, 0, M.MOE_ERR_ARG),
+    (16, 200, 8, 2, 128, 0, M.MOE_ERR_SHAPE),
+    (16, 256, 8, 2, 96, 0, M.MOE_ERR_SHAPE),
+    (16, 256, 1024, 2, 128, 0, M.MOE_ERR_SHAPE),
+    (16, 256, 128, 65, 128, 0, M.MOE_ERR_SHAPE),
+    (16, 256, 8, 2, 128, 1, M.MOE_ERR_UNSUPPORTED),
+    (16, 256, 8, 2, 128, 7, M.MOE_ERR_ARG),
+])
+def test_invalid_shapes_are_rejected(lib, T, d, E, k, I, dtype, code):
+    sh = M.make_shape(T, d, E, k, I, dtype)
+    f = ctypes.c_size_t()
+    assert lib.moe_workspace_size(ctypes.byref(sh), ctypes.byref(f), None) == code
+    assert lib.moe_fwd(ctypes.byref(sh), None, None, None, None, None, None, None, 0, None) == code
+
+
+def test_null_and_misaligned_pointers_are_rejected_before_launch(lib):
+    sh = M.make_shape(256, 256, 8, 2, 128)
+    saved = M.MoeSaved(*([16] * len(M.SAVED_FIELDS)))
+    # null x
+    assert lib.moe_fwd(ctypes.byref(sh), None, 16, 16, 16, 16, ctypes.byref(saved), 16, 1 << 40, None) == M.MOE_ERR_ARG
+    # misaligned out
+    assert lib.moe_fwd(ctypes.byref(sh), 16, 16, 16, 16, 17, ctypes.byref(saved), 16, 1 << 40, None) == M.MOE_ERR_ARG
+    # misaligned saved field
+    bad = M.MoeSaved(*([16] * (len(M.SAVED_FIELDS) - 1) + [24]))
+    assert lib.moe_fwd(ctypes.byref(sh), 16, 16, 16, 16, 16, ctypes.byref(bad), 16, 1 << 40, None) == M.MOE_ERR_ARG
+    # workspace too small
+    assert lib.moe_fwd(ctypes.byref(sh), 16, 16, 16, 16, 16, ctypes.byref(saved), 16, 64, None) == M.MOE_ERR_WS
+    assert lib.moe_bwd(ctypes.byref(sh), 16, 16, 16, 16, ctypes.byref(saved), 16, 16, 16, 16, None, 16, 64,
+                       None) == M.MOE_ERR_WS
+
+
+def test_error_strings_and_kernel_names(lib):
+    for code in range(-8, 1):
+        assert M.error_string(code)
+    assert M.error_string(-99) == "unknown error code"
+    names = M.kernel_names()
+    assert names[0] == "route_topk" and "gemm_gateup_fwd" in names and names[-1] == "route_bwd"

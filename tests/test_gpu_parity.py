@@ -1,0 +1,136 @@
+"""GPU parity: the CUDA layer (through the C ABI) against the fp64 CPU oracle.
+
+Routing indices, counts, offsets, permutation and inverse must match bit for
+bit; out, h, aw and every gradient must match within the normwise relative
+tolerance TOL_BF16 (bf16 operands, fp32 accumulation).  Small cases are
+checked element by element in full; the full-size workloads are checked on
+sampled tokens and experts, which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import TOL_BF16, check_routing, f64, make, normwise, run_layer, sorted_rows
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def full_check(cfg, inp, backward=True, check_h=True):
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    layer, res = run_layer(inp, T, d, E, k, I, backward=backward)
+    assert res["status"] == 0
+    logits = inp["logits"].numpy()
+    check_routing(res["saved"], logits, k)
+    x, wgu, wd = f64(inp["x"]), f64(inp["wgu"]), f64(inp["wd"])
+    ref = O.forward(x, logits, wgu, wd, k)
+    errs = dict(out=normwise(f64(res["out"]), ref["out"]))
+    if check_h:
+        errs["h"] = normwise(sorted_rows(res["saved"], "h"), ref["h"])
+        errs["aw"] = normwise(sorted_rows(res["saved"], "aw"), ref["w"].reshape(-1, 1) * ref["a"])
+    if backward:
+        g = O.backward(x, logits, wgu, wd, k, f64(inp["gout"]), ref)
+        for name in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
+            errs[name] = normwise(f64(res[name]), g[name])
+        # experts without tokens: exact-zero weight gradients
+        empty = np.nonzero(ref["counts"] == 0)[0]
+        for e in empty:
+            assert torch.count_nonzero(res["dwgu"][e]) == 0 and torch.count_nonzero(res["dwd"][e]) == 0
+    bad = {n: v for n, v in errs.items() if not v <= TOL_BF16}
+    assert not bad, f"normwise errors above {TOL_BF16}: {bad} (all: {errs})"
+    return errs
+
+
+def test_tiny_workload():
+    cfg, inp = make("tiny")
+    full_check(cfg, inp)
+
+
+@pytest.mark.parametrize("sizes", [
+    dict(T=1000, d=384, E=16, k=4, I=384),   # 128-wide N tiles, ragged groups
+    dict(T=700, d=512, E=12, k=3, I=256),    # 256-wide N tiles
+    dict(T=333, d=256, E=4, k=1, I=128),     # k = 1
+    dict(T=130, d=256, E=8, k=8, I=128),     # k = E
+    dict(T=1, d=256, E=8, k=2, I=128),       # a single token
+])
+def test_multi_tile_ragged(sizes):
+    cfg, inp = make(sizes, seed=3)
+    full_check(cfg, inp)
+
+
+def test_empty_and_dominant_experts():
+    cfg, inp = make(dict(T=600, d=256, E=16, k=2, I=256), seed=5)
+    lg = inp["logits"]
+    lg[:, 5] = -100.0   # never chosen
+    lg[:, 9] = -100.0
+    lg[:, 3] += 100.0   # chosen first by every token
+    full_check(cfg, inp)
+
+
+def test_tied_logits():
+    cfg, inp = make(dict(T=512, d=256, E=16, k=4, I=128), seed=7)
+    lg = inp["logits"]
+    lg.copy_(torch.round(lg * 2) / 2)
+    lg[::7] = 0.25       # fully tied rows -> experts 0..k-1
+    full_check(cfg, inp)
+
+
+def test_deterministic_bitwise():
+    cfg, inp = make(dict(T=900, d=256, E=16, k=4, I=256), seed=11)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    layer, r1 = run_layer(inp, T, d, E, k, I)
+    _, r2 = run_layer(inp, T, d, E, k, I, layer=layer)
+    for name in ("out", "dx", "dwgu", "dwd", "dscore", "dlogits"):
+        assert torch.equal(r1[name], r2[name]), name
+
+
+def _sampled_check(name, seed=0, n_tokens=48, experts=None):
+    cfg, inp = make(name, seed=seed)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    layer, res = run_layer(inp, T, d, E, k, I)
+    assert res["status"] == 0
+    logits = inp["logits"].numpy()
+    idx_ref, _ = check_routing(res["saved"], logits, k)
+    rng = np.random.default_rng(seed + 1)
+    toks = np.sort(rng.choice(T, size=n_tokens, replace=False))
+    toks[0], toks[-1] = 0, T - 1
+    x, gout = inp["x"].float().numpy(), inp["gout"].float().numpy()
+    wgu, wd = inp["wgu"], inp["wd"]
+    wgu_np, wd_np = wgu.float().numpy(), wd.float().numpy()
+    ft = O.forward_tokens(x, logits, wgu_np, wd_np, k, toks)
+    errs = dict(out=normwise(f64(res["out"])[toks], ft["out"]))
+    bt = O.backward_tokens(x, logits, wgu_np, wd_np, k, gout, toks)
+    for n in ("dx", "dscore", "dlogits"):
+        errs[n] = normwise(f64(res[n])[toks], bt[n])
+    counts = np.bincount(idx_ref.reshape(-1), minlength=E)
+    if experts is None:
+        experts = [int(np.argmin(np.abs(counts - np.median(counts)))), E - 1]
+    be = O.backward_experts(x, logits, wgu_np, wd_np, k, gout, experts)
+    for e in experts:
+        errs[f"dwgu[{e}]"] = normwise(f64(res["dwgu"][e]), be[e][0])
+        errs[f"dwd[{e}]"] = normwise(f64(res["dwd"][e]), be[e][1])
+    for e in np.nonzero(counts == 0)[0]:
+        assert torch.count_nonzero(res["dwgu"][e]) == 0 and torch.count_nonzero(res["dwd"][e]) == 0
+    bad = {n: v for n, v in errs.items() if not v <= TOL_BF16}
+    assert not bad, f"normwise errors above {TOL_BF16}: {bad} (all: {errs})"
+    return errs
+
+
+def test_qwen3_30b_shape_sampled():
+    _sampled_check("qwen3_30b_a3b")
+
+
+def test_qwen3_30b_skewed_routing_sampled():
+    from grouped_gemm_route_b200 import inputs as IN
+    cfg = IN.WORKLOADS["qwen3_30b_a3b_skew"]
+    lg = IN.make_logits(cfg["T"], cfg["E"], seed=0, zipf_s=cfg["zipf_s"]).numpy()
+    idx, _ = O.route(lg, cfg["k"])
+    counts = np.bincount(idx.reshape(-1), minlength=cfg["E"])
+    assert (counts == 0).sum() >= 8
+    order = np.argsort(counts)
+    medium = int(order[np.searchsorted(counts[order], 2000)])  # a busy but not the busiest expert
+    _sampled_check("qwen3_30b_a3b_skew", experts=[medium, int(np.argmax(counts == 0))])
+
+
+def test_qwen3_235b_shape_sampled():
+    _sampled_check("qwen3_235b_a22b", n_tokens=24)
