@@ -164,15 +164,16 @@ def oracle_weights(inp):
 
 
 def cpu_baseline(cfg, inp, n_tokens=0, budget_s=15.0):
+    """Oracle fwd+bwd throughput on the first n tokens; n grows until one pass takes ~budget_s/2."""
     from grouped_gemm_route_b200 import inputs as IN
     wgu64, wd64 = oracle_weights(inp)
-    n = n_tokens or 64
+    n = n_tokens or 256
     dt = time_oracle_step(cfg, inp, wgu64, wd64, n)
-    if not n_tokens:  # grow the sample to about budget_s of work
-        n = int(min(cfg["T"], max(64, n * budget_s / max(dt, 1e-3) * 0.8)))
+    while not n_tokens and dt < budget_s / 2 and n < cfg["T"]:
+        n = min(cfg["T"], n * 2)
         dt = time_oracle_step(cfg, inp, wgu64, wd64, n)
-    flops = IN.flops_fwd(T=n, **{k: cfg[k] for k in ("d", "E", "k", "I")}) + \
-        IN.flops_bwd(T=n, **{k: cfg[k] for k in ("d", "E", "k", "I")})
+    dims = {k: cfg[k] for k in ("d", "E", "k", "I")}
+    flops = IN.flops_fwd(T=n, **dims) + IN.flops_bwd(T=n, **dims)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
             "sample": f"fp64 numpy oracle, forward+backward of the first {n} of {cfg['T']} tokens "
                       f"(all experts' weights), {dt:.2f} s"}, n, dt

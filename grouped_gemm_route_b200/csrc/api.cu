@@ -441,6 +441,14 @@ int moe_get_status(const void *ws, void *stream, int *device_status) {
     return MOE_OK;
 }
 
+int moe_selftest_wait_timeout(void *ws, void *stream) {
+    if (!aligned16(ws)) return MOE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int *status = static_cast<int *>(ws);  // the status word is the first field of every workspace
+    if (cudaMemsetAsync(status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    return launch_expire_wait(status, st) == cudaSuccess ? MOE_OK : MOE_ERR_LAUNCH;
+}
+
 const char *moe_error_string(int code) {
     switch (code) {
         case MOE_OK: return "ok";

@@ -75,6 +75,8 @@ cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int
 cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t *idx, const int32_t *inv,
                              const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s);
 
+cudaError_t launch_expire_wait(int *status, cudaStream_t s);
+
 cudaError_t launch_gemm(GemmMode mode, int bn, const GemmArgs &args, const CUtensorMap &tmA,
                         const CUtensorMap &tmB, int grid, cudaStream_t s);
 

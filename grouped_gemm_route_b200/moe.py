@@ -23,7 +23,8 @@ MOE_ERR_LAUNCH, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE, MOE_ERR_UNSUPPORTED = -5, -6, -
 
 SAVED_FIELDS = ("topk_idx", "topk_w", "counts", "offsets", "group_start", "tile_expert", "perm", "inv", "h", "aw")
 EXPORTS = ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
-           "moe_error_string", "moe_profile_enable", "moe_profile_read", "moe_kernel_name")
+           "moe_error_string", "moe_profile_enable", "moe_profile_read", "moe_kernel_name",
+           "moe_selftest_wait_timeout")
 
 
 class MoeShape(ctypes.Structure):
@@ -63,6 +64,8 @@ def lib() -> ctypes.CDLL:
     L.moe_error_string.restype = ctypes.c_char_p
     L.moe_profile_enable.argtypes = [ctypes.c_int]
     L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
+    L.moe_selftest_wait_timeout.argtypes = [P, P]
+    L.moe_selftest_wait_timeout.restype = ctypes.c_int
     L.moe_kernel_name.argtypes = [ctypes.c_int]
     L.moe_kernel_name.restype = ctypes.c_char_p
     for name in ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
@@ -138,6 +141,11 @@ def get_status(ws, stream=None) -> int:
     s = ctypes.c_int()
     _check(lib().moe_get_status(_ptr(ws), _stream(stream), ctypes.byref(s)), "moe_get_status")
     return int(s.value)
+
+
+def selftest_wait_timeout(ws, stream=None):
+    """Launch the kernel whose bounded wait must expire (see include/moe.h)."""
+    _check(lib().moe_selftest_wait_timeout(_ptr(ws), _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def kernel_names():

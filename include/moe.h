@@ -138,6 +138,14 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x,
  * or MOE_ERR_LAUNCH if the copy itself failed. */
 int moe_get_status(const void *ws, void *stream, int *device_status);
 
+/* Failure-path self-test.  Launches one small kernel whose bounded wait on an
+ * mbarrier that nothing arrives at must expire (after about 2 s); the kernel then
+ * records MOE_ERR_TIMEOUT in the status word of `ws` (at least 16 bytes, device
+ * memory) and returns, leaving nothing in flight.  moe_get_status(ws, ...)
+ * afterwards reports MOE_ERR_TIMEOUT; later calls on the same context work
+ * normally.  Returns MOE_OK once launched. */
+int moe_selftest_wait_timeout(void *ws, void *stream);
+
 /* Static string for a return code.  Never NULL. */
 const char *moe_error_string(int code);
 
