@@ -460,6 +460,7 @@ const char *moe_error_string(int code) {
         case MOE_ERR_TIMEOUT: return "a device-side bounded wait expired";
         case MOE_ERR_DEVICE: return "a device-side index check failed";
         case MOE_ERR_UNSUPPORTED: return "dtype not implemented";
+        case MOE_ERR_SCRATCH_LIMIT: return "shape exceeds the fixed scratch of moe_route_noalloc (ceil(T/64)*E > 131072)";
         default: return "unknown error code";
     }
 }

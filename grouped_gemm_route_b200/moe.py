@@ -20,11 +20,12 @@ MOE_BF16, MOE_MXFP8 = 0, 1
 MOE_OK = 0
 MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_WS, MOE_ERR_ARCH = -1, -2, -3, -4
 MOE_ERR_LAUNCH, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE, MOE_ERR_UNSUPPORTED = -5, -6, -7, -8
+MOE_ERR_SCRATCH_LIMIT = -9
 
 SAVED_FIELDS = ("topk_idx", "topk_w", "counts", "offsets", "group_start", "tile_expert", "perm", "inv", "h", "aw")
 EXPORTS = ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
            "moe_error_string", "moe_profile_enable", "moe_profile_read", "moe_kernel_name",
-           "moe_selftest_wait_timeout")
+           "moe_selftest_wait_timeout", "moe_route_noalloc")
 
 
 class MoeShape(ctypes.Structure):
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.moe_error_string.restype = ctypes.c_char_p
     L.moe_profile_enable.argtypes = [ctypes.c_int]
     L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
+    L.moe_route_noalloc.argtypes = [S, P, ctypes.POINTER(MoeSaved), P]
+    L.moe_route_noalloc.restype = ctypes.c_int
     L.moe_selftest_wait_timeout.argtypes = [P, P]
     L.moe_selftest_wait_timeout.restype = ctypes.c_int
     L.moe_kernel_name.argtypes = [ctypes.c_int]
@@ -122,6 +125,15 @@ def route(shape, logits, saved: dict, ws, stream=None):
     st = saved_struct(saved)
     _check(lib().moe_route(ctypes.byref(shape), _ptr(logits), ctypes.byref(st), _ptr(ws), ws.numel(),
                            _stream(stream)), "moe_route")
+
+
+def route_noalloc(shape, logits, saved: dict, stream=None):
+    """Routing for callers that cannot allocate device memory: same results as
+    route(), with the kernels' scratch in a fixed array inside the library
+    instead of a caller workspace (see moe_route_noalloc in include/moe.h)."""
+    st = saved_struct(saved)
+    _check(lib().moe_route_noalloc(ctypes.byref(shape), _ptr(logits), ctypes.byref(st), _stream(stream)),
+           "moe_route_noalloc")
 
 
 def fwd(shape, x, logits, wgu, wd, out, saved: dict, ws, stream=None):

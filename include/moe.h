@@ -64,6 +64,7 @@ extern "C" {
 #define MOE_ERR_TIMEOUT (-6)     /* a device-side bounded wait expired (moe_get_status) */
 #define MOE_ERR_DEVICE (-7)      /* a device-side index check failed (moe_get_status) */
 #define MOE_ERR_UNSUPPORTED (-8) /* dtype not implemented */
+#define MOE_ERR_SCRATCH_LIMIT (-9) /* moe_route_noalloc: ceil(T/64)*E above its fixed scratch capacity */
 
 /* Operand precision of the expert GEMMs. */
 typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_dtype_t;
@@ -131,6 +132,38 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x,
             const void *w_gate_up, const void *w_down, const moe_saved_t *saved,
             void *dx, void *dw_gate_up, void *dw_down, float *dscore, float *dlogits,
             void *ws, size_t ws_bytes, void *stream);
+
+/* Routing and dispatch for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for users of
+ * the library that are not allowed to call cudaMalloc: for example code running
+ * inside a host program whose memory manager owns all of the GPU's memory and
+ * gives none to plug-ins, or code on a latency-critical path where an
+ * allocation (which may synchronise the whole device) is not acceptable.
+ *
+ * Same results as moe_route (same kernels), but the per-block histograms and
+ * bases that moe_route keeps in the caller's workspace live instead in a fixed
+ * 1 MiB __device__ array inside the library, which every GPU that loads the
+ * library holds until the process exits.  The caller still allocates and
+ * passes the logits and every moe_saved_t routing field (topk_idx, topk_w,
+ * counts, offsets, group_start, tile_expert, perm, inv); h and aw are not used.
+ * Nothing is allocated or freed: no cudaMalloc, no cudaFree, no allocating
+ * library routine.
+ *
+ * Limit: 2 * ceil(T/64) * E * 4 bytes must fit in 1 MiB, i.e. ceil(T/64) * E <=
+ * 131072 (e.g. T = 16384 with E <= 512, or T = 65536 with E <= 128); larger
+ * shapes return MOE_ERR_SCRATCH_LIMIT before anything is launched.  Other shape
+ * rules and error codes are those of moe_route.
+ *
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress (with that device current) and caches it; make that
+ * first call before any stream capture.  All calls share the one array and it
+ * keeps the last call's contents; every word a call reads is written earlier in
+ * the same call, so nothing needs clearing.  Calls that overlap on the GPU (on
+ * different streams, or from different host threads) race on the array and
+ * must be serialised by the caller.  Device-side index checks are not
+ * reported by this entry point (it has no status word). */
+int moe_route_noalloc(const moe_shape_t *shape, const float *logits, moe_saved_t *saved, void *stream);
 
 /* Synchronises `stream`, then reads the device status word of `ws` written by
  * the most recent moe_route / moe_fwd / moe_bwd on that workspace:
