@@ -330,9 +330,8 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
 
-    CUtensorMap tm_x, tm_wgu, tm_aw, tm_wd;
-    if (!make_map(&tm_x, x, pl.T, pl.d, 1) ||
-        !make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 128) ||
+    CUtensorMap tm_wgu, tm_aw, tm_wd;
+    if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 128) ||
         !make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) ||
         !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
         return MOE_ERR_LAUNCH;
@@ -344,9 +343,10 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.I / 128;
     a.num_k_blocks = pl.d / kTileK;
+    a.gsrc = static_cast<const __nv_bfloat16 *>(x);  // token rows gathered through perm (A operand)
     {
         Launch L(kKindGemmGateUpFwd, st);
-        if ((rc = L.done(launch_gemm(kGateUpFwd, 256, a, tm_x, tm_wgu, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kGateUpFwd, 256, a, tm_wgu, tm_wgu, grid, st)))) return rc;
     }
     a.n_tiles = pl.d / pl.bn_d;
     a.num_k_blocks = pl.I / kTileK;
@@ -377,14 +377,15 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     __nv_bfloat16 *dh = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_dh);
     float *dpart = reinterpret_cast<float *>(w8 + pl.ws_dpart);
 
-    CUtensorMap tm_gout_rows, tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn, tm_x_rows;
+    CUtensorMap tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn;
     const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I;
     const int64_t Ed = static_cast<int64_t>(pl.E) * pl.d;
-    if (!make_map(&tm_gout_rows, grad_out, pl.T, pl.d, 1) || !make_map(&tm_wd_mn, w_down, Ed, pl.I, 64) ||
-        !make_map(&tm_dh_rows, dh, pl.p_cap, 2 * pl.I, 128) || !make_map(&tm_wgu_mn, w_gate_up, EI2, pl.d, 64) ||
-        !make_map(&tm_aw_mn, saved->aw, pl.p_cap, pl.I, 64) || !make_map(&tm_dh_mn, dh, pl.p_cap, 2 * pl.I, 64) ||
-        !make_map(&tm_x_rows, x, pl.T, pl.d, 1))
+    if (!make_map(&tm_wd_mn, w_down, Ed, pl.I, 64) || !make_map(&tm_dh_rows, dh, pl.p_cap, 2 * pl.I, 128) ||
+        !make_map(&tm_wgu_mn, w_gate_up, EI2, pl.d, 64) || !make_map(&tm_aw_mn, saved->aw, pl.p_cap, pl.I, 64) ||
+        !make_map(&tm_dh_mn, dh, pl.p_cap, 2 * pl.I, 64))
         return MOE_ERR_LAUNCH;
+    const __nv_bfloat16 *gout_rows = static_cast<const __nv_bfloat16 *>(grad_out);
+    const __nv_bfloat16 *x_rows = static_cast<const __nv_bfloat16 *>(x);
 
     if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
     const int grid = grid_for(shape, dev);
@@ -395,9 +396,10 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     // b1: down dgrad, dscore partials, SwiGLU backward -> dh; zeroes the dx counters
     a.n_tiles = pl.I / pl.bn_i;
     a.num_k_blocks = pl.d / kTileK;
+    a.gsrc = gout_rows;  // A operand: grad_out rows gathered through perm
     {
         Launch L(kKindGemmDownDgrad, st);
-        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, a, tm_gout_rows, tm_wd_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, a, tm_wd_mn, tm_wd_mn, grid, st)))) return rc;
     }
     // b3: down wgrad  dW_down[e] = sum_p gout[t] (x) aw_p
     a.m_tiles = pl.d / kTileM;
@@ -405,7 +407,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dw = static_cast<__nv_bfloat16 *>(dw_down);
     {
         Launch L(kKindGemmDownWgrad, st);
-        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, a, tm_gout_rows, tm_aw_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, a, tm_aw_mn, tm_aw_mn, grid, st)))) return rc;
     }
     // b4: gate/up dgrad + ordered scatter-sum into dx
     a.n_tiles = pl.d / pl.bn_d;
@@ -419,9 +421,10 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.m_tiles = 2 * pl.I / kTileM;
     a.n_tiles = pl.d / pl.bn_d;
     a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
+    a.gsrc = x_rows;  // B operand: x rows gathered through perm
     {
         Launch L(kKindGemmGateUpWgrad, st);
-        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, a, tm_dh_mn, tm_x_rows, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, a, tm_dh_mn, tm_dh_mn, grid, st)))) return rc;
     }
     // b6: dscore (ordered sum of partials) and dlogits
     {

@@ -3,10 +3,14 @@
 // One kernel template serves the six expert GEMMs of the layer (two forward,
 // four backward).  Each CTA owns one SM and walks a static list of output
 // tiles.  Inside a CTA the work is split by warp:
-//   warp 0      producer: TMA loads of A and B K-blocks into a 4- or 6-stage
-//               shared-memory ring.  Token rows are fetched with the TMA row
-//               gather (tile::gather4) straight from x or grad_out through the
-//               dispatch permutation, so no permuted copy of the tokens exists.
+//   warp 0      TMA producer: bulk tensor loads of the dense operand (expert
+//               weights, or the sorted-layout activations) into a 4- or
+//               6-stage shared-memory ring, 128-byte swizzled.
+//   warps 6, 7  gather producers (modes that read token rows): 16-byte
+//               cp.async copies of x / grad_out rows picked through the
+//               dispatch permutation, written with the same 128-byte swizzle.
+//               The dispatch is fused into the operand load: no permuted copy
+//               of the tokens is ever written to memory.
 //   warp 1      allocates tensor memory and issues tcgen05.mma (one thread),
 //               accumulating a 128 x BN fp32 tile in TMEM; two TMEM buffers
 //               let the epilogue of one tile overlap the mainloop of the next.
@@ -23,8 +27,8 @@
 //
 // The combine and the scatter are deterministic: each (token, slot) row writes
 // its tile slice to a slot-addressed staging buffer and bumps a per-(token,
-// column tile) counter; the row that brings the counter to k sums the k slots
-// in slot order.  No thread ever waits on another CTA.
+// column tile) counter; the warp holding the row that brings the counter to k
+// sums the k slots in slot order.  No thread ever waits on another CTA.
 //
 // Every wait on an mbarrier is bounded in time.  On expiry the kernel records
 // a timeout in the status word, stops issuing work, waits (bounded) for its own
@@ -41,7 +45,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
+constexpr int kGatherWarp0 = 6;               // warps 6 and 7 gather token rows
+constexpr int kGatherThreads = 64;
 constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr int kChunkBytes = 64 * kTileK * 2;  // 8 KB: one 64-wide MN chunk of an MN-major K-block
 constexpr uint32_t kSbo = 1024;               // 8 rows x 128 B swizzle atom
@@ -59,13 +65,21 @@ struct Cfg {
 
 template <int MODE>
 struct ModeTraits {
-    static constexpr bool kMTiled = MODE <= kGateUpDgrad;            // M = sorted rows
+    static constexpr bool kMTiled = MODE <= kGateUpDgrad;  // M = sorted rows
     static constexpr bool kAGather = MODE == kGateUpFwd || MODE == kDownDgrad || MODE == kDownWgrad;
-    static constexpr bool kBGather = MODE == kGateUpWgrad;  // only the gate/up wgrad gathers B
+    static constexpr bool kBGather = MODE == kGateUpWgrad;
+    static constexpr bool kGather = kAGather || kBGather;
     static constexpr bool kAMn = MODE == kDownWgrad || MODE == kGateUpWgrad;
     static constexpr bool kBMn = MODE == kDownDgrad || MODE == kGateUpDgrad || MODE == kDownWgrad ||
                                  MODE == kGateUpWgrad;
 };
+
+// Bytes of one stage that arrive by TMA (the gathered operand arrives by cp.async).
+template <int MODE, int BN>
+__host__ __device__ constexpr uint32_t tma_stage_bytes() {
+    return ModeTraits<MODE>::kAGather ? Cfg<BN>::kBBytes
+                                      : (ModeTraits<MODE>::kBGather ? kABytes : Cfg<BN>::kStageBytes);
+}
 
 struct Tile {
     int e;      // expert
@@ -149,25 +163,18 @@ __device__ __forceinline__ void raise_abort(volatile int *abort_flag, int *statu
 }
 
 // ---------------------------------------------------------------------------
-// producer (warp 0)
+// TMA producer (warp 0): the operand(s) that are not gathered
 // ---------------------------------------------------------------------------
 template <int MODE, int BN>
 __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, const GemmArgs &a, uint8_t *smem,
                               uint64_t *full, uint64_t *empty, volatile int *abort_flag) {
     using C = Cfg<BN>;
-    using TR = ModeTraits<MODE>;
     const int lane = threadIdx.x & 31;
     const int total = total_tiles<MODE>(a);
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const Tile t = decode_tile<MODE>(tile, a);
-        int tok[4] = {0, 0, 0, 0};
-        if constexpr (TR::kMTiled && TR::kAGather) {
-            const int pos = t.mt * kTileM + 4 * lane;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) tok[i] = token_of(a, pos + i);
-        }
         for (int kb = 0; kb < t.nkb; ++kb) {
             const int s = it % C::kStages;
             const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
@@ -175,20 +182,12 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
                 ok = false;
                 break;
             }
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], tma_stage_bytes<MODE, BN>());
             __syncwarp();
             uint8_t *As = smem + s * C::kStageBytes;
             uint8_t *Bs = As + kABytes;
             const int k0 = kb * kTileK;
-            if constexpr (!TR::kMTiled) {
-                // wgrad: the K block is 64 sorted rows of expert e; 16 groups of 4
-                const int g = lane & 15;
-                const int pos = t.kpos0 + k0 + 4 * g;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) tok[i] = TR::kAGather || TR::kBGather ? token_of(a, pos + i) : 0;
-            }
             if constexpr (MODE == kGateUpFwd) {
-                tma_gather4(As + lane * 512, tmA, &full[s], k0, tok[0], tok[1], tok[2], tok[3]);
                 if (lane == 0) {
                     const int row = t.e * 2 * a.I + t.nt * (BN / 2);
                     tma_load_2d(Bs, tmB, &full[s], k0, row);                         // gate rows
@@ -200,23 +199,18 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
                     tma_load_2d(Bs, tmB, &full[s], k0, t.e * a.d + t.nt * BN);
                 }
             } else if constexpr (MODE == kDownDgrad) {
-                tma_gather4(As + lane * 512, tmA, &full[s], k0, tok[0], tok[1], tok[2], tok[3]);
-                if (lane < BN / 64) tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.e * a.d + k0);
+                if (lane < BN / 64)
+                    tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.e * a.d + k0);
             } else if constexpr (MODE == kGateUpDgrad) {
                 if (lane == 0) tma_load_2d(As, tmA, &full[s], k0, t.mt * kTileM);
                 if (lane < BN / 64)
                     tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.e * 2 * a.I + k0);
             } else if constexpr (MODE == kDownWgrad) {
-                const int c = lane >> 4, g = lane & 15;
-                tma_gather4(As + c * kChunkBytes + g * 512, tmA, &full[s], t.mt * kTileM + 64 * c, tok[0], tok[1],
-                            tok[2], tok[3]);
-                if (lane < BN / 64) tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.kpos0 + k0);
+                if (lane < BN / 64)
+                    tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.kpos0 + k0);
             } else {  // kGateUpWgrad
-                if (lane < 2) tma_load_2d(As + lane * kChunkBytes, tmA, &full[s], t.mt * kTileM + 64 * lane, t.kpos0 + k0);
-                const int g = lane & 15;
-                for (int c = lane >> 4; c < BN / 64; c += 2)
-                    tma_gather4(Bs + c * kChunkBytes + g * 512, tmB, &full[s], t.nt * BN + 64 * c, tok[0], tok[1],
-                                tok[2], tok[3]);
+                if (lane < 2)
+                    tma_load_2d(As + lane * kChunkBytes, tmA, &full[s], t.mt * kTileM + 64 * lane, t.kpos0 + k0);
             }
             ++it;
         }
@@ -230,6 +224,106 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
         }
         __syncwarp();
     }
+}
+
+// ---------------------------------------------------------------------------
+// gather producers (warps 6, 7): token rows through the dispatch permutation
+// ---------------------------------------------------------------------------
+// Thread g (0..63) copies 16-byte piece (g & 7) of the 128-byte rows
+// r = (g >> 3) + 8 i.  A row r of a 128-byte-swizzled stage lives at byte
+// r * 128, with its 16-byte piece c stored at position c ^ (r & 7).
+template <int MODE, int BN>
+__device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty,
+                            volatile int *abort_flag) {
+    using C = Cfg<BN>;
+    using TR = ModeTraits<MODE>;
+    const int g = threadIdx.x - kGatherWarp0 * 32;
+    const int piece = g & 7;
+    const int rg = g >> 3;
+    const size_t d = static_cast<size_t>(a.d);
+    const int total = total_tiles<MODE>(a);
+    int it = 0;
+    bool ok = true;
+    if constexpr (TR::kMTiled) {
+        // 16 rows of the 128-row tile per thread; K-major, one 128-byte row per K block
+        int tok[16], nxt[16];
+        int tile = blockIdx.x;
+        if (tile < total) {
+            const int mt = tile / a.n_tiles;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tok[i] = token_of(a, mt * kTileM + rg + 8 * i);
+        }
+        for (; tile < total && ok; tile += gridDim.x) {
+            const Tile t = decode_tile<MODE>(tile, a);
+            const int next = tile + gridDim.x;
+            if (next < total) {  // prefetch the next tile's token rows
+                const int mt = next / a.n_tiles;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) nxt[i] = token_of(a, mt * kTileM + rg + 8 * i);
+            }
+            const __nv_bfloat16 *rows[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) rows[i] = a.gsrc + static_cast<size_t>(tok[i]) * d + piece * 8;
+            for (int kb = 0; kb < t.nkb; ++kb) {
+                const int s = it % C::kStages;
+                const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
+                if (!warp_wait(&empty[s], ph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t As = smem_u32(smem + s * C::kStageBytes);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = rg + 8 * i;
+                    cp_async_16(As + r * 128 + ((piece ^ (r & 7)) << 4), rows[i] + kb * kTileK);
+                }
+                cp_async_arrive_noinc(&full[s]);
+                ++it;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tok[i] = nxt[i];
+        }
+    } else {
+        // wgrad: 64 K rows (tokens) per K block, MN-major; 8 rows per thread
+        constexpr int kChunks = MODE == kDownWgrad ? 2 : BN / 64;  // 64-wide MN chunks of the gathered operand
+        constexpr uint32_t kRegion = MODE == kDownWgrad ? 0u : static_cast<uint32_t>(kABytes);
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const Tile t = decode_tile<MODE>(tile, a);
+            const int col0 = MODE == kDownWgrad ? t.mt * kTileM : t.nt * BN;
+            int tok[8], nxt[8];
+            if (t.nkb > 0) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) tok[i] = token_of(a, t.kpos0 + rg + 8 * i);
+            }
+            for (int kb = 0; kb < t.nkb; ++kb) {
+                if (kb + 1 < t.nkb) {  // prefetch the next K block's tokens
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) nxt[i] = token_of(a, t.kpos0 + (kb + 1) * kTileK + rg + 8 * i);
+                }
+                const int s = it % C::kStages;
+                const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
+                if (!warp_wait(&empty[s], ph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t base = smem_u32(smem + s * C::kStageBytes) + kRegion;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = rg + 8 * i;
+                    const __nv_bfloat16 *src = a.gsrc + static_cast<size_t>(tok[i]) * d + col0 + piece * 8;
+                    const uint32_t dst = base + r * 128 + ((piece ^ (r & 7)) << 4);
+#pragma unroll
+                    for (int cc = 0; cc < kChunks; ++cc) cp_async_16(dst + cc * kChunkBytes, src + cc * 64);
+                }
+                cp_async_arrive_noinc(&full[s]);
+                ++it;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) tok[i] = nxt[i];
+            }
+        }
+    }
+    if (!ok) raise_abort(abort_flag, a.status);
+    cp_async_wait_all();  // our copies land before the CTA can exit
 }
 
 // ---------------------------------------------------------------------------
@@ -261,6 +355,7 @@ __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint6
                 ok = false;
                 break;
             }
+            if constexpr (TR::kGather) fence_proxy_async_smem();  // cp.async data -> tensor-core reads
             tc_fence_after_sync();
             const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
             const uint32_t b_base = a_base + kABytes;
@@ -287,7 +382,6 @@ __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint6
 // ---------------------------------------------------------------------------
 // epilogues (warps 2..5; thread = one accumulator row)
 // ---------------------------------------------------------------------------
-template <int BN>
 __device__ __forceinline__ void release_accumulator(uint64_t *tempty_acc) {
     tc_fence_before_sync();
     __syncwarp();
@@ -313,17 +407,12 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
         tmem_load_wait();
         tmem_regs_ready(gr);
         tmem_regs_ready(ur);
-        float g[32], u[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            g[i] = __uint_as_float(gr[i]);
-            u[i] = __uint_as_float(ur[i]);
-        }
         uint32_t pg[16], pu[16], pa[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             if (valid) {
-                const float g0 = g[2 * i], g1 = g[2 * i + 1], u0 = u[2 * i], u1 = u[2 * i + 1];
+                const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
+                const float u0 = __uint_as_float(ur[2 * i]), u1 = __uint_as_float(ur[2 * i + 1]);
                 const float s0 = __fdividef(1.f, 1.f + __expf(-g0));
                 const float s1 = __fdividef(1.f, 1.f + __expf(-g1));
                 pg[i] = pack_bf16x2(g0, g1);
@@ -337,13 +426,15 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
         store_row32(hrow + a.I + c * 32, pu);
         store_row32(arow + c * 32, pa);
     }
-    release_accumulator<BN>(tempty_acc);
+    release_accumulator(tempty_acc);
 }
 
-// down forward / gate-up dgrad: stage the slot's row slice, last arriver sums slots in order
+// down forward / gate-up dgrad: stage the slot's row slice; the warp holding the
+// last of a token's k slots sums the k staging rows in slot order
 template <int BN>
 __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                            uint64_t *tempty_acc) {
+    const int lane = threadIdx.x & 31;
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
@@ -360,35 +451,56 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
             store_row32(srow + c * 32, pv);
         }
     }
-    release_accumulator<BN>(tempty_acc);
-    if (!valid) return;
-    const int tok = p / a.k;
-    __threadfence();
-    int *ctr = a.cnt + static_cast<size_t>(tok) * a.cnt_stride + t.nt;
-    const int arrived = atomicAdd(ctr, 1);
-    if (arrived != a.k - 1) return;
-    __threadfence();
-    const __nv_bfloat16 *slots = a.stage + static_cast<size_t>(tok) * a.k * a.d + col0;
-    __nv_bfloat16 *orow = a.out + static_cast<size_t>(tok) * a.d + col0;
-#pragma unroll 1
-    for (int col = 0; col < BN; col += 8) {
-        float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < a.k; ++j) {  // slot order
-            const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(slots + static_cast<size_t>(j) * a.d + col));
-            acc8[0] += bf16_lo(u.x);
-            acc8[1] += bf16_hi(u.x);
-            acc8[2] += bf16_lo(u.y);
-            acc8[3] += bf16_hi(u.y);
-            acc8[4] += bf16_lo(u.z);
-            acc8[5] += bf16_hi(u.z);
-            acc8[6] += bf16_lo(u.w);
-            acc8[7] += bf16_hi(u.w);
-        }
-        *reinterpret_cast<uint4 *>(orow + col) =
-            make_uint4(pack_bf16x2(acc8[0], acc8[1]), pack_bf16x2(acc8[2], acc8[3]), pack_bf16x2(acc8[4], acc8[5]),
-                       pack_bf16x2(acc8[6], acc8[7]));
+    release_accumulator(tempty_acc);
+
+    const int tok = valid ? p / a.k : 0;
+    bool last = false;
+    if (valid) {
+        __threadfence();
+        last = atomicAdd(a.cnt + static_cast<size_t>(tok) * a.cnt_stride + t.nt, 1) == a.k - 1;
     }
-    *ctr = 0;  // ready for the next call
+    unsigned mask = __ballot_sync(0xffffffffu, last);
+    if (mask == 0u) return;
+    __threadfence();
+    constexpr int kCols = BN / 32;  // columns per lane
+    while (mask != 0u) {
+        const int src = __ffs(static_cast<int>(mask)) - 1;
+        mask &= mask - 1u;
+        const int tk = __shfl_sync(0xffffffffu, tok, src);
+        const __nv_bfloat16 *slot0 = a.stage + static_cast<size_t>(tk) * a.k * a.d + col0 + lane * kCols;
+        float acc[kCols];
+#pragma unroll
+        for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < a.k; ++j) {  // slot order
+            const __nv_bfloat16 *sp = slot0 + static_cast<size_t>(j) * a.d;
+            if constexpr (kCols == 8) {
+                const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(sp));
+                acc[0] += bf16_lo(u.x);
+                acc[1] += bf16_hi(u.x);
+                acc[2] += bf16_lo(u.y);
+                acc[3] += bf16_hi(u.y);
+                acc[4] += bf16_lo(u.z);
+                acc[5] += bf16_hi(u.z);
+                acc[6] += bf16_lo(u.w);
+                acc[7] += bf16_hi(u.w);
+            } else {
+                const uint2 u = __ldcg(reinterpret_cast<const uint2 *>(sp));
+                acc[0] += bf16_lo(u.x);
+                acc[1] += bf16_hi(u.x);
+                acc[2] += bf16_lo(u.y);
+                acc[3] += bf16_hi(u.y);
+            }
+        }
+        __nv_bfloat16 *orow = a.out + static_cast<size_t>(tk) * a.d + col0 + lane * kCols;
+        if constexpr (kCols == 8) {
+            *reinterpret_cast<uint4 *>(orow) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                          pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+        } else {
+            *reinterpret_cast<uint2 *>(orow) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+        }
+        if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + t.nt] = 0;  // ready for the next call
+    }
 }
 
 // down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh
@@ -436,7 +548,7 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
         store_row32(dhrow + c * 32, pdg);
         store_row32(dhrow + a.I + c * 32, pdu);
     }
-    release_accumulator<BN>(tempty_acc);
+    release_accumulator(tempty_acc);
     a.dpart[static_cast<size_t>(pos) * a.dpart_stride + t.nt] = valid ? ds : 0.f;
     if (valid && t.nt == 0) {  // counters of the dx scatter that follows
         const int tok = p / a.k;
@@ -466,7 +578,7 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
         }
         store_row32(row + c * 32, pv);
     }
-    release_accumulator<BN>(tempty_acc);
+    release_accumulator(tempty_acc);
 }
 
 template <int MODE, int BN>
@@ -504,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmArgs args) {
     using C = Cfg<BN>;
+    using TR = ModeTraits<MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
@@ -517,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1 + (TR::kGather ? kGatherThreads : 0));
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -543,8 +656,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((threadIdx.x & 31) == 0)
             mma_loop<MODE, BN>(args, smem, full, empty, tfull, tempty, drain, tmem_base, abort_flag);
         __syncwarp();
-    } else {
+    } else if (warp < kGatherWarp0) {
         epilogue_loop<MODE, BN>(args, tfull, tempty, tmem_base, abort_flag);
+    } else if constexpr (TR::kGather) {
+        gather_loop<MODE, BN>(args, smem, full, empty, abort_flag);
     }
 
     tc_fence_before_sync();

@@ -53,6 +53,7 @@ struct GemmArgs {
     const int *group_start;
     const int *tile_expert;
     const float *topk_w;
+    const __nv_bfloat16 *gsrc;  // token rows the gather warps read: x or grad_out [T, d]
     __nv_bfloat16 *h;
     __nv_bfloat16 *aw;
     __nv_bfloat16 *stage;
