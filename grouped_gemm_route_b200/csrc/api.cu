@@ -35,7 +35,7 @@ struct Plan {
     int dpart_stride;   // I / bn_i
     // workspace layout (byte offsets)
     size_t ws_status, ws_cnt, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
-    size_t ws_dh, ws_dpart, bwd_bytes;
+    size_t ws_dh, ws_dpart, ws_xs, ws_gs, bwd_bytes;
     size_t saved[MOE_SAVED_FIELDS];
 };
 
@@ -83,6 +83,10 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     off = align_up(off + static_cast<size_t>(p_cap) * 2 * s->I * 2);
     p->ws_dpart = off;
     off = align_up(off + static_cast<size_t>(p_cap) * p->dpart_stride * 4);
+    p->ws_xs = off;
+    off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
+    p->ws_gs = off;
+    off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
     p->bwd_bytes = off;
 
     const size_t Tk = static_cast<size_t>(P);
@@ -202,7 +206,8 @@ struct Launch {
 
 const char *kKindNames[kNumKernelKinds] = {
     "route_topk",       "route_scan",       "route_perm",           "gemm_gateup_fwd",      "gemm_down_fwd_combine",
-    "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd"};
+    "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd",
+    "sort_rows"};
 
 struct Saved {
     int32_t *idx;
@@ -377,15 +382,16 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     __nv_bfloat16 *dh = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_dh);
     float *dpart = reinterpret_cast<float *>(w8 + pl.ws_dpart);
 
-    CUtensorMap tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn;
+    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_xs);
+    __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_gs);
+    CUtensorMap tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn, tm_gs_rows, tm_gs_mn, tm_xs_mn;
     const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I;
     const int64_t Ed = static_cast<int64_t>(pl.E) * pl.d;
     if (!make_map(&tm_wd_mn, w_down, Ed, pl.I, 64) || !make_map(&tm_dh_rows, dh, pl.p_cap, 2 * pl.I, 128) ||
         !make_map(&tm_wgu_mn, w_gate_up, EI2, pl.d, 64) || !make_map(&tm_aw_mn, saved->aw, pl.p_cap, pl.I, 64) ||
-        !make_map(&tm_dh_mn, dh, pl.p_cap, 2 * pl.I, 64))
+        !make_map(&tm_dh_mn, dh, pl.p_cap, 2 * pl.I, 64) || !make_map(&tm_gs_rows, gs, pl.p_cap, pl.d, 128) ||
+        !make_map(&tm_gs_mn, gs, pl.p_cap, pl.d, 64) || !make_map(&tm_xs_mn, xs, pl.p_cap, pl.d, 64))
         return MOE_ERR_LAUNCH;
-    const __nv_bfloat16 *gout_rows = static_cast<const __nv_bfloat16 *>(grad_out);
-    const __nv_bfloat16 *x_rows = static_cast<const __nv_bfloat16 *>(x);
 
     if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
     const int grid = grid_for(shape, dev);
@@ -393,13 +399,20 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dh = dh;
     a.dpart = dpart;
 
+    // b0: x and grad_out in the expert-sorted layout (operands of the K = tokens wgrads)
+    {
+        Launch L(kKindSortRows, st);
+        if ((rc = L.done(launch_sort_rows(saved->perm, saved->group_start, pl.E, pl.k, static_cast<int>(pl.T), pl.d,
+                                          static_cast<const __nv_bfloat16 *>(x),
+                                          static_cast<const __nv_bfloat16 *>(grad_out), xs, gs, dev.sms, st))))
+            return rc;
+    }
     // b1: down dgrad, dscore partials, SwiGLU backward -> dh; zeroes the dx counters
     a.n_tiles = pl.I / pl.bn_i;
     a.num_k_blocks = pl.d / kTileK;
-    a.gsrc = gout_rows;  // A operand: grad_out rows gathered through perm
     {
         Launch L(kKindGemmDownDgrad, st);
-        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, a, tm_wd_mn, tm_wd_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, a, tm_gs_rows, tm_wd_mn, grid, st)))) return rc;
     }
     // b3: down wgrad  dW_down[e] = sum_p gout[t] (x) aw_p
     a.m_tiles = pl.d / kTileM;
@@ -407,7 +420,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dw = static_cast<__nv_bfloat16 *>(dw_down);
     {
         Launch L(kKindGemmDownWgrad, st);
-        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, a, tm_aw_mn, tm_aw_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, a, tm_gs_mn, tm_aw_mn, grid, st)))) return rc;
     }
     // b4: gate/up dgrad + ordered scatter-sum into dx
     a.n_tiles = pl.d / pl.bn_d;
@@ -421,10 +434,9 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.m_tiles = 2 * pl.I / kTileM;
     a.n_tiles = pl.d / pl.bn_d;
     a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
-    a.gsrc = x_rows;  // B operand: x rows gathered through perm
     {
         Launch L(kKindGemmGateUpWgrad, st);
-        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, a, tm_dh_mn, tm_dh_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, a, tm_dh_mn, tm_xs_mn, grid, st)))) return rc;
     }
     // b6: dscore (ordered sum of partials) and dlogits
     {

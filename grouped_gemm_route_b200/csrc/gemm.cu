@@ -6,11 +6,13 @@
 //   warp 0      TMA producer: bulk tensor loads of the dense operand (expert
 //               weights, or the sorted-layout activations) into a 4- or
 //               6-stage shared-memory ring, 128-byte swizzled.
-//   warps 6, 7  gather producers (modes that read token rows): 16-byte
-//               cp.async copies of x / grad_out rows picked through the
-//               dispatch permutation, written with the same 128-byte swizzle.
-//               The dispatch is fused into the operand load: no permuted copy
-//               of the tokens is ever written to memory.
+//   warps 6, 7  gather producers (forward gate/up GEMM): 16-byte cp.async
+//               copies of the x rows picked through the dispatch permutation,
+//               written with the same 128-byte swizzle.  The dispatch is fused
+//               into the operand load: the forward never writes a permuted
+//               copy of the tokens.  (The backward reads x and grad_out from
+//               expert-sorted copies made by sort_rows, so that its wgrads,
+//               whose K dimension is the tokens, run on plain TMA tiles.)
 //   warp 1      allocates tensor memory and issues tcgen05.mma (one thread),
 //               accumulating a 128 x BN fp32 tile in TMEM; two TMEM buffers
 //               let the epilogue of one tile overlap the mainloop of the next.
@@ -52,23 +54,26 @@ constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr int kChunkBytes = 64 * kTileK * 2;  // 8 KB: one 64-wide MN chunk of an MN-major K-block
 constexpr uint32_t kSbo = 1024;               // 8 rows x 128 B swizzle atom
 constexpr uint32_t kMnLbo = kChunkBytes;      // MN-major: distance between 64-wide chunks
+constexpr int kXposeBytes = 32 * 64;          // per epilogue warp: 32 rows x 64 bytes
+constexpr int kTailCap = 2048;                // finished (token, column tile) pairs a CTA defers to its tail
 
 template <int BN>
 struct Cfg {
     static constexpr int kStages = BN == 256 ? 4 : 6;
     static constexpr int kBBytes = BN * kTileK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kBarOffset = kStages * kStageBytes;
-    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1 KB alignment slack
+    static constexpr int kBarOffset = kStages * kStageBytes;      // mbarriers, TMEM slot, abort flag
+    static constexpr int kOrderOffset = kBarOffset + 512;         // wgrad expert order
+    static constexpr int kXposeOffset = kOrderOffset + 2 * kMaxExperts * 4;   // 4 x 2 KB epilogue transposes
+    static constexpr int kTailOffset = kXposeOffset + 4 * kXposeBytes;        // combine: finished tokens
+    static constexpr int kSmemBytes = kTailOffset + 4 * (kTailCap + 4) + 1024;  // + 1 KB alignment slack
     static constexpr uint32_t kTmemCols = 2 * BN;
 };
 
 template <int MODE>
 struct ModeTraits {
     static constexpr bool kMTiled = MODE <= kGateUpDgrad;  // M = sorted rows
-    static constexpr bool kAGather = MODE == kGateUpFwd || MODE == kDownDgrad || MODE == kDownWgrad;
-    static constexpr bool kBGather = MODE == kGateUpWgrad;
-    static constexpr bool kGather = kAGather || kBGather;
+    static constexpr bool kGather = MODE == kGateUpFwd;  // x rows gathered through the dispatch permutation
     static constexpr bool kAMn = MODE == kDownWgrad || MODE == kGateUpWgrad;
     static constexpr bool kBMn = MODE == kDownDgrad || MODE == kGateUpDgrad || MODE == kDownWgrad ||
                                  MODE == kGateUpWgrad;
@@ -77,8 +82,7 @@ struct ModeTraits {
 // Bytes of one stage that arrive by TMA (the gathered operand arrives by cp.async).
 template <int MODE, int BN>
 __host__ __device__ constexpr uint32_t tma_stage_bytes() {
-    return ModeTraits<MODE>::kAGather ? Cfg<BN>::kBBytes
-                                      : (ModeTraits<MODE>::kBGather ? kABytes : Cfg<BN>::kStageBytes);
+    return ModeTraits<MODE>::kGather ? Cfg<BN>::kBBytes : Cfg<BN>::kStageBytes;
 }
 
 struct Tile {
@@ -89,8 +93,10 @@ struct Tile {
     int kpos0;  // wgrad: first sorted row of the expert's group
 };
 
+// Wgrad tiles are walked expert by expert, busiest expert first (`order`, a
+// per-CTA copy in shared memory), so that long-K tiles are spread evenly.
 template <int MODE>
-__device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a) {
+__device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const int *order) {
     Tile t;
     if constexpr (ModeTraits<MODE>::kMTiled) {
         t.mt = tile / a.n_tiles;
@@ -100,8 +106,9 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a) {
         t.kpos0 = 0;
     } else {
         const int per = a.m_tiles * a.n_tiles;
-        t.e = tile / per;
-        const int r = tile - t.e * per;
+        const int rank = tile / per;
+        const int r = tile - rank * per;
+        t.e = order[rank];
         t.mt = r / a.n_tiles;
         t.nt = r - t.mt * a.n_tiles;
         const int gs = __ldg(a.group_start + t.e), ge = __ldg(a.group_start + t.e + 1);
@@ -132,22 +139,59 @@ __device__ __forceinline__ int token_of(const GemmArgs &a, int pos) {
     return p / a.k;
 }
 
-__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const uint32_t (&p)[16]) {
-    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+// Row transposes through a per-warp 32 x 64-byte shared buffer.  Thread r of
+// the epilogue owns accumulator row r; a transpose turns its 64-byte piece of
+// row r into global accesses where 4 lanes cover one row's 64 contiguous
+// bytes (8 rows per instruction).  16-byte pieces are XOR-swizzled by bits
+// 1..2 of the row so that neither pass has bank conflicts beyond the minimum.
+__device__ __forceinline__ uint32_t xpose_off(int row, int piece) {
+    return static_cast<uint32_t>(row * 64 + ((piece ^ ((row >> 1) & 3)) << 4));
 }
 
-__device__ __forceinline__ void load_row32(const __nv_bfloat16 *src, uint32_t (&p)[16]) {
-    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+// Store each lane's 64 bytes v to rowptr (nullptr: that row is skipped).
+__device__ __forceinline__ void warp_store_rows(uint8_t *buf, const uint32_t (&v)[16], void *rowptr) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint4 v = s4[i];
-        p[4 * i] = v.x;
-        p[4 * i + 1] = v.y;
-        p[4 * i + 2] = v.z;
-        p[4 * i + 3] = v.w;
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(buf + xpose_off(lane, q)) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    __syncwarp();
+    const int piece = lane & 3;
+    const unsigned long long mine = reinterpret_cast<unsigned long long>(rowptr);
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        const int row = rr * 8 + (lane >> 2);
+        const uint4 val = *reinterpret_cast<const uint4 *>(buf + xpose_off(row, piece));
+        char *dst = reinterpret_cast<char *>(__shfl_sync(0xffffffffu, mine, row));
+        if (dst != nullptr) *reinterpret_cast<uint4 *>(dst + piece * 16) = val;
     }
+    __syncwarp();
+}
+
+// Load 64 bytes of each lane's row from rowptr (nullptr: zeros).
+__device__ __forceinline__ void warp_load_rows(uint8_t *buf, uint32_t (&v)[16], const void *rowptr) {
+    const int lane = threadIdx.x & 31;
+    const int piece = lane & 3;
+    const unsigned long long mine = reinterpret_cast<unsigned long long>(rowptr);
+    uint4 got[4];
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        const int row = rr * 8 + (lane >> 2);
+        const char *src = reinterpret_cast<const char *>(__shfl_sync(0xffffffffu, mine, row));
+        got[rr] = src != nullptr ? *reinterpret_cast<const uint4 *>(src + piece * 16) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+        *reinterpret_cast<uint4 *>(buf + xpose_off(rr * 8 + (lane >> 2), piece)) = got[rr];
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 val = *reinterpret_cast<const uint4 *>(buf + xpose_off(lane, q));
+        v[4 * q] = val.x;
+        v[4 * q + 1] = val.y;
+        v[4 * q + 2] = val.z;
+        v[4 * q + 3] = val.w;
+    }
+    __syncwarp();
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
@@ -167,14 +211,14 @@ __device__ __forceinline__ void raise_abort(volatile int *abort_flag, int *statu
 // ---------------------------------------------------------------------------
 template <int MODE, int BN>
 __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, const GemmArgs &a, uint8_t *smem,
-                              uint64_t *full, uint64_t *empty, volatile int *abort_flag) {
+                              uint64_t *full, uint64_t *empty, const int *order, volatile int *abort_flag) {
     using C = Cfg<BN>;
     const int lane = threadIdx.x & 31;
     const int total = total_tiles<MODE>(a);
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const Tile t = decode_tile<MODE>(tile, a);
+        const Tile t = decode_tile<MODE>(tile, a, order);
         for (int kb = 0; kb < t.nkb; ++kb) {
             const int s = it % C::kStages;
             const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
@@ -199,6 +243,7 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
                     tma_load_2d(Bs, tmB, &full[s], k0, t.e * a.d + t.nt * BN);
                 }
             } else if constexpr (MODE == kDownDgrad) {
+                if (lane == 0) tma_load_2d(As, tmA, &full[s], k0, t.mt * kTileM);  // sorted grad_out rows
                 if (lane < BN / 64)
                     tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.e * a.d + k0);
             } else if constexpr (MODE == kGateUpDgrad) {
@@ -206,11 +251,15 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
                 if (lane < BN / 64)
                     tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.e * 2 * a.I + k0);
             } else if constexpr (MODE == kDownWgrad) {
-                if (lane < BN / 64)
-                    tma_load_2d(Bs + lane * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * lane, t.kpos0 + k0);
+                if (lane < 2)  // sorted grad_out rows, MN-major
+                    tma_load_2d(As + lane * kChunkBytes, tmA, &full[s], t.mt * kTileM + 64 * lane, t.kpos0 + k0);
+                if (lane >= 2 && lane < 2 + BN / 64)
+                    tma_load_2d(Bs + (lane - 2) * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * (lane - 2), t.kpos0 + k0);
             } else {  // kGateUpWgrad
                 if (lane < 2)
                     tma_load_2d(As + lane * kChunkBytes, tmA, &full[s], t.mt * kTileM + 64 * lane, t.kpos0 + k0);
+                if (lane >= 2 && lane < 2 + BN / 64)  // sorted x rows, MN-major
+                    tma_load_2d(Bs + (lane - 2) * kChunkBytes, tmB, &full[s], t.nt * BN + 64 * (lane - 2), t.kpos0 + k0);
             }
             ++it;
         }
@@ -233,10 +282,9 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
 // r = (g >> 3) + 8 i.  A row r of a 128-byte-swizzled stage lives at byte
 // r * 128, with its 16-byte piece c stored at position c ^ (r & 7).
 template <int MODE, int BN>
-__device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty,
+__device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty, const int *order,
                             volatile int *abort_flag) {
     using C = Cfg<BN>;
-    using TR = ModeTraits<MODE>;
     const int g = threadIdx.x - kGatherWarp0 * 32;
     const int piece = g & 7;
     const int rg = g >> 3;
@@ -244,7 +292,7 @@ __device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, ui
     const int total = total_tiles<MODE>(a);
     int it = 0;
     bool ok = true;
-    if constexpr (TR::kMTiled) {
+    {
         // 16 rows of the 128-row tile per thread; K-major, one 128-byte row per K block
         int tok[16], nxt[16];
         int tile = blockIdx.x;
@@ -254,7 +302,7 @@ __device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, ui
             for (int i = 0; i < 16; ++i) tok[i] = token_of(a, mt * kTileM + rg + 8 * i);
         }
         for (; tile < total && ok; tile += gridDim.x) {
-            const Tile t = decode_tile<MODE>(tile, a);
+            const Tile t = decode_tile<MODE>(tile, a, order);
             const int next = tile + gridDim.x;
             if (next < total) {  // prefetch the next tile's token rows
                 const int mt = next / a.n_tiles;
@@ -283,44 +331,6 @@ __device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, ui
 #pragma unroll
             for (int i = 0; i < 16; ++i) tok[i] = nxt[i];
         }
-    } else {
-        // wgrad: 64 K rows (tokens) per K block, MN-major; 8 rows per thread
-        constexpr int kChunks = MODE == kDownWgrad ? 2 : BN / 64;  // 64-wide MN chunks of the gathered operand
-        constexpr uint32_t kRegion = MODE == kDownWgrad ? 0u : static_cast<uint32_t>(kABytes);
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-            const Tile t = decode_tile<MODE>(tile, a);
-            const int col0 = MODE == kDownWgrad ? t.mt * kTileM : t.nt * BN;
-            int tok[8], nxt[8];
-            if (t.nkb > 0) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) tok[i] = token_of(a, t.kpos0 + rg + 8 * i);
-            }
-            for (int kb = 0; kb < t.nkb; ++kb) {
-                if (kb + 1 < t.nkb) {  // prefetch the next K block's tokens
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) nxt[i] = token_of(a, t.kpos0 + (kb + 1) * kTileK + rg + 8 * i);
-                }
-                const int s = it % C::kStages;
-                const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
-                if (!warp_wait(&empty[s], ph ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t base = smem_u32(smem + s * C::kStageBytes) + kRegion;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int r = rg + 8 * i;
-                    const __nv_bfloat16 *src = a.gsrc + static_cast<size_t>(tok[i]) * d + col0 + piece * 8;
-                    const uint32_t dst = base + r * 128 + ((piece ^ (r & 7)) << 4);
-#pragma unroll
-                    for (int cc = 0; cc < kChunks; ++cc) cp_async_16(dst + cc * kChunkBytes, src + cc * 64);
-                }
-                cp_async_arrive_noinc(&full[s]);
-                ++it;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) tok[i] = nxt[i];
-            }
-        }
     }
     if (!ok) raise_abort(abort_flag, a.status);
     cp_async_wait_all();  // our copies land before the CTA can exit
@@ -331,7 +341,8 @@ __device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, ui
 // ---------------------------------------------------------------------------
 template <int MODE, int BN>
 __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty, uint64_t *tfull,
-                         uint64_t *tempty, uint64_t *drain, uint32_t tmem_base, volatile int *abort_flag) {
+                         uint64_t *tempty, uint64_t *drain, uint32_t tmem_base, const int *order,
+                         volatile int *abort_flag) {
     using C = Cfg<BN>;
     using TR = ModeTraits<MODE>;
     constexpr uint32_t kIdesc = instr_desc_bf16(kTileM, BN, TR::kAMn, TR::kBMn);
@@ -339,7 +350,7 @@ __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint6
     int it = 0, local = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
-        const Tile t = decode_tile<MODE>(tile, a);
+        const Tile t = decode_tile<MODE>(tile, a, order);
         const int acc = local & 1;
         const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) {
@@ -388,10 +399,17 @@ __device__ __forceinline__ void release_accumulator(uint64_t *tempty_acc) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(tempty_acc);
 }
 
+// Per-CTA list of (token, column tile) pairs whose last slot this CTA wrote;
+// their slot-ordered sums run after the CTA's last tile (see combine_tail).
+struct TailList {
+    int *items;  // token * n_tiles + column tile
+    int *count;
+};
+
 // gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up
 template <int BN>
 __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
-                                               uint64_t *tempty_acc) {
+                                               uint64_t *tempty_acc, uint8_t *xbuf) {
     constexpr int kHalf = BN / 2;
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
@@ -407,6 +425,7 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
         tmem_load_wait();
         tmem_regs_ready(gr);
         tmem_regs_ready(ur);
+        if (c + 1 == kHalf / 32) release_accumulator(tempty_acc);  // TMEM no longer needed
         uint32_t pg[16], pu[16], pa[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -422,91 +441,173 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
                 pg[i] = pu[i] = pa[i] = 0u;
             }
         }
-        store_row32(hrow + c * 32, pg);
-        store_row32(hrow + a.I + c * 32, pu);
-        store_row32(arow + c * 32, pa);
+        warp_store_rows(xbuf, pg, hrow + c * 32);
+        warp_store_rows(xbuf, pu, hrow + a.I + c * 32);
+        warp_store_rows(xbuf, pa, arow + c * 32);
     }
-    release_accumulator(tempty_acc);
 }
 
-// down forward / gate-up dgrad: stage the slot's row slice; the warp holding the
-// last of a token's k slots sums the k staging rows in slot order
+// Slot-ordered sum of one finished (token, column tile): the warp reads the k
+// staging rows (coalesced, all slots in flight), writes out[token] and resets
+// the counter for the next call.
+template <int BN>
+__device__ __forceinline__ void combine_token(const GemmArgs &a, int tk, int nt) {
+    constexpr int kCols = BN / 32;  // columns per lane
+    const int lane = threadIdx.x & 31;
+    const int col0 = nt * BN;
+    const __nv_bfloat16 *slot0 = a.stage + static_cast<size_t>(tk) * a.k * a.d + col0 + lane * kCols;
+    float acc[kCols];
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < a.k; ++j) {  // slot order
+        const __nv_bfloat16 *sp = slot0 + static_cast<size_t>(j) * a.d;
+        if constexpr (kCols == 8) {
+            const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(sp));
+            acc[0] += bf16_lo(u.x);
+            acc[1] += bf16_hi(u.x);
+            acc[2] += bf16_lo(u.y);
+            acc[3] += bf16_hi(u.y);
+            acc[4] += bf16_lo(u.z);
+            acc[5] += bf16_hi(u.z);
+            acc[6] += bf16_lo(u.w);
+            acc[7] += bf16_hi(u.w);
+        } else {
+            const uint2 u = __ldcg(reinterpret_cast<const uint2 *>(sp));
+            acc[0] += bf16_lo(u.x);
+            acc[1] += bf16_hi(u.x);
+            acc[2] += bf16_lo(u.y);
+            acc[3] += bf16_hi(u.y);
+        }
+    }
+    __nv_bfloat16 *orow = a.out + static_cast<size_t>(tk) * a.d + col0 + lane * kCols;
+    if constexpr (kCols == 8) {
+        *reinterpret_cast<uint4 *>(orow) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                      pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    } else {
+        *reinterpret_cast<uint2 *>(orow) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+    }
+    if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + nt] = 0;
+}
+
+// down forward / gate-up dgrad: stage the slot's row slice, count the slot; a
+// (token, column tile) whose k-th slot lands here is queued for the tail
 template <int BN>
 __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
-                                           uint64_t *tempty_acc) {
+                                           uint64_t *tempty_acc, uint8_t *xbuf, const TailList &tail) {
     const int lane = threadIdx.x & 31;
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
-    const int col0 = t.nt * BN;
-    __nv_bfloat16 *srow = a.stage + static_cast<size_t>(valid ? p : 0) * a.d + col0;
+    __nv_bfloat16 *srow = valid ? a.stage + static_cast<size_t>(p) * a.d + t.nt * BN : nullptr;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_load32_sync(taddr + c * 32, v);
-        if (valid) {
-            uint32_t pv[16];
+        if (c + 1 == BN / 32) release_accumulator(tempty_acc);
+        uint32_t pv[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-            store_row32(srow + c * 32, pv);
-        }
+        for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        warp_store_rows(xbuf, pv, srow != nullptr ? srow + c * 32 : nullptr);
     }
-    release_accumulator(tempty_acc);
-
     const int tok = valid ? p / a.k : 0;
     bool last = false;
-    if (valid) {
-        __threadfence();
-        last = atomicAdd(a.cnt + static_cast<size_t>(tok) * a.cnt_stride + t.nt, 1) == a.k - 1;
-    }
+    __threadfence();  // this warp's staging rows before its counts
+    if (valid) last = atomicAdd(a.cnt + static_cast<size_t>(tok) * a.cnt_stride + t.nt, 1) == a.k - 1;
     unsigned mask = __ballot_sync(0xffffffffu, last);
     if (mask == 0u) return;
-    __threadfence();
-    constexpr int kCols = BN / 32;  // columns per lane
-    while (mask != 0u) {
-        const int src = __ffs(static_cast<int>(mask)) - 1;
-        mask &= mask - 1u;
-        const int tk = __shfl_sync(0xffffffffu, tok, src);
-        const __nv_bfloat16 *slot0 = a.stage + static_cast<size_t>(tk) * a.k * a.d + col0 + lane * kCols;
-        float acc[kCols];
+    __threadfence();  // the other slots' staging rows after their counts
+    const int n_last = __popc(mask);
+    int base = 0;
+    if (lane == 0) base = atomicAdd(tail.count, n_last);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const int my = __popc(mask & ((1u << lane) - 1u));
+    if (last && base + my < kTailCap) tail.items[base + my] = tok * a.n_tiles + t.nt;
+    // no room left in the tail list: reduce those tokens now
+    if (base + n_last > kTailCap) {
+        while (mask != 0u) {
+            const int src = __ffs(static_cast<int>(mask)) - 1;
+            const int idx = __popc(mask & ((1u << src) - 1u)) + (n_last - __popc(mask));
+            mask &= mask - 1u;
+            const int tk = __shfl_sync(0xffffffffu, tok, src);
+            if (base + idx >= kTailCap) combine_token<BN>(a, tk, t.nt);
+        }
+    }
+}
+
+// Slot-ordered sums of up to four finished (token, column tile) items at once
+// (independent accumulators, so four tokens' slot loads are in flight).
+template <int BN>
+__device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *items, int n) {
+    constexpr int kCols = BN / 32;
+    const int lane = threadIdx.x & 31;
+    const __nv_bfloat16 *base[4];
+    float acc[4][kCols];
 #pragma unroll
-        for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < a.k; ++j) {  // slot order
-            const __nv_bfloat16 *sp = slot0 + static_cast<size_t>(j) * a.d;
-            if constexpr (kCols == 8) {
-                const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(sp));
-                acc[0] += bf16_lo(u.x);
-                acc[1] += bf16_hi(u.x);
-                acc[2] += bf16_lo(u.y);
-                acc[3] += bf16_hi(u.y);
-                acc[4] += bf16_lo(u.z);
-                acc[5] += bf16_hi(u.z);
-                acc[6] += bf16_lo(u.w);
-                acc[7] += bf16_hi(u.w);
-            } else {
-                const uint2 u = __ldcg(reinterpret_cast<const uint2 *>(sp));
-                acc[0] += bf16_lo(u.x);
-                acc[1] += bf16_hi(u.x);
-                acc[2] += bf16_lo(u.y);
-                acc[3] += bf16_hi(u.y);
+    for (int u = 0; u < 4; ++u) {
+        const int item = items[u < n ? u : 0];
+        const int tk = item / a.n_tiles, nt = item - tk * a.n_tiles;
+        base[u] = a.stage + static_cast<size_t>(tk) * a.k * a.d + nt * BN + lane * kCols;
+#pragma unroll
+        for (int i = 0; i < kCols; ++i) acc[u][i] = 0.f;
+    }
+#pragma unroll 2
+    for (int j = 0; j < a.k; ++j) {  // slot order
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (u < n) {
+                const __nv_bfloat16 *sp = base[u] + static_cast<size_t>(j) * a.d;
+                if constexpr (kCols == 8) {
+                    const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(sp));
+                    acc[u][0] += bf16_lo(v.x);
+                    acc[u][1] += bf16_hi(v.x);
+                    acc[u][2] += bf16_lo(v.y);
+                    acc[u][3] += bf16_hi(v.y);
+                    acc[u][4] += bf16_lo(v.z);
+                    acc[u][5] += bf16_hi(v.z);
+                    acc[u][6] += bf16_lo(v.w);
+                    acc[u][7] += bf16_hi(v.w);
+                } else {
+                    const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(sp));
+                    acc[u][0] += bf16_lo(v.x);
+                    acc[u][1] += bf16_hi(v.x);
+                    acc[u][2] += bf16_lo(v.y);
+                    acc[u][3] += bf16_hi(v.y);
+                }
             }
         }
-        __nv_bfloat16 *orow = a.out + static_cast<size_t>(tk) * a.d + col0 + lane * kCols;
-        if constexpr (kCols == 8) {
-            *reinterpret_cast<uint4 *>(orow) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                                          pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-        } else {
-            *reinterpret_cast<uint2 *>(orow) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
-        }
-        if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + t.nt] = 0;  // ready for the next call
     }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (u < n) {
+            const int item = items[u];
+            const int tk = item / a.n_tiles, nt = item - tk * a.n_tiles;
+            __nv_bfloat16 *orow = a.out + static_cast<size_t>(tk) * a.d + nt * BN + lane * kCols;
+            if constexpr (kCols == 8) {
+                *reinterpret_cast<uint4 *>(orow) =
+                    make_uint4(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
+                               pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
+            } else {
+                *reinterpret_cast<uint2 *>(orow) =
+                    make_uint2(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]));
+            }
+            if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + nt] = 0;  // ready for the next call
+        }
+    }
+}
+
+// after the CTA's last tile: slot-ordered sums of its queued tokens, all warps
+template <int BN>
+__device__ __forceinline__ void combine_tail(const GemmArgs &a, const TailList &tail) {
+    const int n = min(*tail.count, kTailCap);
+    const int warp = threadIdx.x >> 5;
+    for (int i = warp * 4; i < n; i += (kThreads / 32) * 4) combine_tokens4<BN>(a, tail.items + i, min(4, n - i));
 }
 
 // down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh
 template <int BN>
 __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
-                                               uint64_t *tempty_acc) {
+                                               uint64_t *tempty_acc, uint8_t *xbuf) {
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
@@ -516,39 +617,34 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
     float ds = 0.f;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
+        uint32_t hg[16], hu[16];
+        warp_load_rows(xbuf, hg, valid ? hrow + c * 32 : nullptr);
+        warp_load_rows(xbuf, hu, valid ? hrow + a.I + c * 32 : nullptr);
         float G[32];
         tmem_load32_sync(taddr + c * 32, G);
+        if (c + 1 == BN / 32) release_accumulator(tempty_acc);
         uint32_t pdg[16], pdu[16];
-        if (valid) {
-            uint32_t hg[16], hu[16];
-            load_row32(hrow + c * 32, hg);
-            load_row32(hrow + a.I + c * 32, hu);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float dgv[2], duv[2];
+        for (int i = 0; i < 16; ++i) {
+            float dgv[2], duv[2];
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const float g = h2 ? bf16_hi(hg[i]) : bf16_lo(hg[i]);
-                    const float u = h2 ? bf16_hi(hu[i]) : bf16_lo(hu[i]);
-                    const float gr = G[2 * i + h2];
-                    const float sg = __fdividef(1.f, 1.f + __expf(-g));
-                    const float sl = g * sg;
-                    ds += gr * (sl * u);
-                    const float da = wv * gr;
-                    dgv[h2] = da * u * sg * (1.f + g * (1.f - sg));
-                    duv[h2] = da * sl;
-                }
-                pdg[i] = pack_bf16x2(dgv[0], dgv[1]);
-                pdu[i] = pack_bf16x2(duv[0], duv[1]);
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const float g = h2 ? bf16_hi(hg[i]) : bf16_lo(hg[i]);
+                const float u = h2 ? bf16_hi(hu[i]) : bf16_lo(hu[i]);
+                const float gr = G[2 * i + h2];
+                const float sg = __fdividef(1.f, 1.f + __expf(-g));
+                const float sl = g * sg;
+                ds += gr * (sl * u);
+                const float da = wv * gr;
+                dgv[h2] = da * u * sg * (1.f + g * (1.f - sg));
+                duv[h2] = da * sl;
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pdg[i] = pdu[i] = 0u;
+            pdg[i] = valid ? pack_bf16x2(dgv[0], dgv[1]) : 0u;
+            pdu[i] = valid ? pack_bf16x2(duv[0], duv[1]) : 0u;
         }
-        store_row32(dhrow + c * 32, pdg);
-        store_row32(dhrow + a.I + c * 32, pdu);
+        warp_store_rows(xbuf, pdg, dhrow + c * 32);
+        warp_store_rows(xbuf, pdu, dhrow + a.I + c * 32);
     }
-    release_accumulator(tempty_acc);
     a.dpart[static_cast<size_t>(pos) * a.dpart_stride + t.nt] = valid ? ds : 0.f;
     if (valid && t.nt == 0) {  // counters of the dx scatter that follows
         const int tok = p / a.k;
@@ -559,7 +655,7 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
 // weight gradients: store the tile (zeros for an expert without tokens)
 template <int MODE, int BN>
 __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
-                                          uint64_t *tempty_acc) {
+                                          uint64_t *tempty_acc, uint8_t *xbuf) {
     const int Mtot = MODE == kDownWgrad ? a.d : 2 * a.I;
     const int Ntot = MODE == kDownWgrad ? a.I : a.d;
     __nv_bfloat16 *row =
@@ -576,21 +672,21 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
 #pragma unroll
             for (int i = 0; i < 16; ++i) pv[i] = 0u;
         }
-        store_row32(row + c * 32, pv);
+        if (c + 1 == BN / 32) release_accumulator(tempty_acc);
+        warp_store_rows(xbuf, pv, row + c * 32);
     }
-    release_accumulator(tempty_acc);
 }
 
 template <int MODE, int BN>
 __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *tempty, uint32_t tmem_base,
-                              volatile int *abort_flag) {
+                              const int *order, uint8_t *xbuf, const TailList &tail, volatile int *abort_flag) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quad = warp & 3;  // TMEM lanes this warp may access: 32*quad .. 32*quad+31
     const int r = quad * 32 + lane;
     const int total = total_tiles<MODE>(a);
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
-        const Tile t = decode_tile<MODE>(tile, a);
+        const Tile t = decode_tile<MODE>(tile, a, order);
         const int acc = local & 1;
         const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
         if (!warp_wait(&tfull[acc], aph, abort_flag)) {
@@ -600,13 +696,13 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
         tc_fence_after_sync();
         const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
         if constexpr (MODE == kGateUpFwd) {
-            epi_gateup_fwd<BN>(a, t, r, taddr, &tempty[acc]);
+            epi_gateup_fwd<BN>(a, t, r, taddr, &tempty[acc], xbuf);
         } else if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
-            epi_combine<BN>(a, t, r, taddr, &tempty[acc]);
+            epi_combine<BN>(a, t, r, taddr, &tempty[acc], xbuf, tail);
         } else if constexpr (MODE == kDownDgrad) {
-            epi_down_dgrad<BN>(a, t, r, taddr, &tempty[acc]);
+            epi_down_dgrad<BN>(a, t, r, taddr, &tempty[acc], xbuf);
         } else {
-            epi_wgrad<MODE, BN>(a, t, r, taddr, &tempty[acc]);
+            epi_wgrad<MODE, BN>(a, t, r, taddr, &tempty[acc], xbuf);
         }
     }
 }
@@ -626,8 +722,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *drain = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const TailList tail{reinterpret_cast<int *>(smem + C::kTailOffset),
+                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap};
+    int *s_count = reinterpret_cast<int *>(smem + C::kOrderOffset);
+    int *order = s_count + kMaxExperts;
 
     const int warp = threadIdx.x >> 5;
+    if constexpr (!TR::kMTiled) {  // busiest expert first: rank by padded row count, ties to lower index
+        for (int e = threadIdx.x; e < args.E; e += kThreads)
+            s_count[e] = __ldg(args.group_start + e + 1) - __ldg(args.group_start + e);
+        __syncthreads();
+        for (int e = threadIdx.x; e < args.E; e += kThreads) {
+            const int c = s_count[e];
+            int rank = 0;
+            for (int f = 0; f < args.E; ++f) {
+                const int cf = s_count[f];
+                rank += (cf > c || (cf == c && f < e)) ? 1 : 0;
+            }
+            order[rank] = e;
+        }
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1 + (TR::kGather ? kGatherThreads : 0));
@@ -639,6 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
+        *tail.count = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -651,21 +766,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        producer_loop<MODE, BN>(&tmA, &tmB, args, smem, full, empty, abort_flag);
+        producer_loop<MODE, BN>(&tmA, &tmB, args, smem, full, empty, order, abort_flag);
     } else if (warp == 1) {
         if ((threadIdx.x & 31) == 0)
-            mma_loop<MODE, BN>(args, smem, full, empty, tfull, tempty, drain, tmem_base, abort_flag);
+            mma_loop<MODE, BN>(args, smem, full, empty, tfull, tempty, drain, tmem_base, order, abort_flag);
         __syncwarp();
     } else if (warp < kGatherWarp0) {
-        epilogue_loop<MODE, BN>(args, tfull, tempty, tmem_base, abort_flag);
+        epilogue_loop<MODE, BN>(args, tfull, tempty, tmem_base, order,
+                                smem + C::kXposeOffset + (warp - 2) * kXposeBytes, tail, abort_flag);
     } else if constexpr (TR::kGather) {
-        gather_loop<MODE, BN>(args, smem, full, empty, abort_flag);
+        gather_loop<MODE, BN>(args, smem, full, empty, order, abort_flag);
     }
 
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
+        if (!*abort_flag) combine_tail<BN>(args, tail);
+    }
 }
 
 template <int MODE, int BN>

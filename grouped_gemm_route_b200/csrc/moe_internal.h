@@ -29,6 +29,7 @@ enum KernelKind : int {
     kKindGemmGateUpDgrad,
     kKindGemmGateUpWgrad,
     kKindRouteBwd,
+    kKindSortRows,
     kNumKernelKinds
 };
 
@@ -36,10 +37,10 @@ enum KernelKind : int {
 enum GemmMode : int {
     kGateUpFwd = 0,    // h = x[perm] W_gu[e]^T ; epilogue SwiGLU -> h, aw
     kDownFwd = 1,      // y = aw W_down[e]^T   ; epilogue slot-ordered combine -> out
-    kDownDgrad = 2,    // G = gout[perm] W_down[e] ; epilogue dscore partials, SwiGLU bwd -> dh
+    kDownDgrad = 2,    // G = gout_sorted W_down[e] ; epilogue dscore partials, SwiGLU bwd -> dh
     kGateUpDgrad = 3,  // dx_p = dh W_gu[e]     ; epilogue slot-ordered scatter-sum -> dx
-    kDownWgrad = 4,    // dW_down[e] = gout[perm]^T aw
-    kGateUpWgrad = 5,  // dW_gu[e] = dh^T x[perm]
+    kDownWgrad = 4,    // dW_down[e] = gout_sorted^T aw
+    kGateUpWgrad = 5,  // dW_gu[e] = dh^T x_sorted
 };
 
 struct GemmArgs {
@@ -73,6 +74,9 @@ cudaError_t launch_route_scan(int T, int E, int n_chunks, const int32_t *chunk_c
                               int32_t *perm, int64_t p_cap, int *status, cudaStream_t s);
 cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int32_t *chunk_base, int32_t *perm,
                               int32_t *inv, int64_t p_cap, int *status, cudaStream_t s);
+cudaError_t launch_sort_rows(const int32_t *perm, const int32_t *group_start, int E, int k, int T, int d,
+                             const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs, __nv_bfloat16 *gs,
+                             int sms, cudaStream_t s);
 cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t *idx, const int32_t *inv,
                              const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s);
 
