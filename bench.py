@@ -328,33 +328,56 @@ def main():
     launches = int(sum(v[1] for v in per_kernel.values()))
 
     # ---- end-to-end through the public API with host buffers ----
+    # Every step copies its inputs (x, logits, grad_out) from pinned host memory,
+    # runs forward + backward, and copies its results (out, dx, dscore) back.
+    # Two layer instances alternate so that the copies of one step overlap the
+    # compute of the next (H2D and D2H on their own streams).
     e2e = None
     if not args.no_e2e:
+        nb = 2
+        layers = [layer] + [M.MoELayer(T, d, E, k, I, device=str(dev)) for _ in range(nb - 1)]
         hx, hlg, hg = (host[n].pin_memory() for n in ("x", "logits", "gout"))
-        hout = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
-        hdx = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
-        hds = torch.empty(T, k, dtype=torch.float32).pin_memory()
-        dx_, dlg_, dg_ = torch.empty_like(x), torch.empty_like(lg), torch.empty_like(gout)
+        hout = [torch.empty(T, d, dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+        hdx = [torch.empty(T, d, dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+        hds = [torch.empty(T, k, dtype=torch.float32).pin_memory() for _ in range(nb)]
+        dins = [(torch.empty_like(x), torch.empty_like(lg), torch.empty_like(gout)) for _ in range(nb)]
+        h2d = torch.cuda.Stream(dev)
+        d2h = torch.cuda.Stream(dev)
+        copied = [torch.cuda.Event() for _ in range(nb)]
+        computed = [torch.cuda.Event() for _ in range(nb)]
+        drained = [torch.cuda.Event() for _ in range(nb)]
 
-        def e2e_step():
-            dx_.copy_(hx, non_blocking=True)
-            dlg_.copy_(hlg, non_blocking=True)
-            dg_.copy_(hg, non_blocking=True)
-            layer.forward(dx_, dlg_, wgu, wd, stream)
-            layer.backward(dg_, dx_, wgu, wd, True, stream)
-            hout.copy_(layer.out, non_blocking=True)
-            hdx.copy_(layer.dx, non_blocking=True)
-            hds.copy_(layer.dscore, non_blocking=True)
+        def e2e_run(n_steps):
+            for i in range(n_steps):
+                b = i % nb
+                with torch.cuda.stream(h2d):
+                    h2d.wait_event(computed[b])  # step i - nb finished reading these inputs
+                    for dst, src in zip(dins[b], (hx, hlg, hg)):
+                        dst.copy_(src, non_blocking=True)
+                    copied[b].record(h2d)
+                stream.wait_event(copied[b])
+                stream.wait_event(drained[b])  # step i - nb's results have left the device
+                ly = layers[b]
+                ly.forward(dins[b][0], dins[b][1], wgu, wd, stream)
+                ly.backward(dins[b][2], dins[b][0], wgu, wd, True, stream)
+                computed[b].record(stream)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(computed[b])
+                    hout[b].copy_(ly.out, non_blocking=True)
+                    hdx[b].copy_(ly.dx, non_blocking=True)
+                    hds[b].copy_(ly.dscore, non_blocking=True)
+                    drained[b].record(d2h)
 
-        for _ in range(3):
-            e2e_step()
-        barrier()
+        e2e_run(3)
         torch.cuda.synchronize(dev)
+        barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        e0.record(h2d)
+        stream.wait_event(e0)
+        d2h.wait_event(e0)
+        e2e_run(args.e2e_steps)
+        stream.wait_stream(d2h)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
@@ -364,9 +387,11 @@ def main():
             pg.all_reduce(t, op=pg.ReduceOp.MAX)
             e_ms = float(t.item())
         bi = sum(t.numel() * t.element_size() for t in (hx, hlg, hg))
-        bo = sum(t.numel() * t.element_size() for t in (hout, hdx, hds))
+        bo = sum(t.numel() * t.element_size() for t in (hout[0], hdx[0], hds[0]))
         e2e = {"value": flops_step * world / (e_ms / args.e2e_steps * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": args.e2e_steps}
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": args.e2e_steps,
+               "overlap": "copies of step i+1 / i-1 overlap compute of step i (two layer buffers)"}
+        del layers
 
     # ---- CPU baseline (rank 0, N = 1 only) ----
     cpu = None

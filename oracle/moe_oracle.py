@@ -349,3 +349,158 @@ def backward_experts(x, logits, wgu, wd, k, gout, experts):
                                                 wf[pairs], wgu_e, wd_e)
         res[e] = (dwgu_e, dwd_e)
     return res
+
+
+# ----------------------------------------------------------------------------
+# MXFP8 operands: E4M3 elements with one UE8M0 (power-of-two) scale per block of
+# 32 consecutive elements along a GEMM's K dimension ("Prime Intellect's Prime
+# Mega MoE Trains Giant AI Models 55% Faster", section "Precision and hardware
+# support": MXFP8 on Blackwell uses small microscaling groups).
+#
+# Readings (the pages give no formula):
+#   * block scale X = 2^s with s the smallest integer such that amax <= 448 * 2^s
+#     (448 is the largest E4M3 magnitude), clamped to [-127, 127]; an all-zero
+#     block has s = 0.
+#   * element code = v / X rounded to the nearest E4M3 value, ties to the even
+#     code, magnitudes above 448 saturating to 448; the dequantised value is
+#     code * X.
+#   * the operands quantised are those of the library's six GEMMs, each along
+#     that GEMM's K (see forward_mx / backward_mx); for the two weight-gradient
+#     GEMMs K runs over an expert's tokens in sorted order, in blocks of 32
+#     starting at the expert's first pair.
+# ----------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_round(y):
+    """Nearest E4M3 value (ties to even code), saturating at +-448.
+
+    E4M3: 3 mantissa bits, exponent bias 7, normal binades from 2^-6 up to
+    448 = 1.75 * 2^8, subnormal spacing 2^-9.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    out = np.zeros_like(a)
+    nz = a > 0
+    e = np.floor(np.log2(np.where(nz, a, 1.0)))
+    # guard against log2 rounding: enforce 2^e <= a < 2^(e+1)
+    e = np.where(np.exp2(e) > a, e - 1, e)
+    e = np.where(np.exp2(e + 1) <= a, e + 1, e)
+    e = np.maximum(e, -6.0)                  # below 2^-6 the spacing stays 2^-9
+    q = np.exp2(e - 3.0)                     # spacing of the binade
+    r = np.round(a / q) * q                  # a / q is exact; np.round is ties-to-even
+    r = np.minimum(r, E4M3_MAX)
+    out[nz] = r[nz]
+    return np.copysign(out, y)
+
+
+def mx_scale_exponent(amax):
+    """Smallest integer s with amax <= 448 * 2^s (0 for amax = 0), clamped to [-127, 127]."""
+    amax = np.asarray(amax, dtype=np.float64)
+    s = np.zeros_like(amax)
+    nz = amax > 0
+    est = np.ceil(np.log2(np.where(nz, amax, 1.0) / E4M3_MAX))
+    # exact correction of the estimate with exact comparisons
+    est = np.where(amax > E4M3_MAX * np.exp2(est), est + 1, est)
+    est = np.where(amax <= E4M3_MAX * np.exp2(est - 1), est - 1, est)
+    s[nz] = est[nz]
+    return np.clip(s, -127, 127)
+
+
+def mx_qdq_blocks(v, axis):
+    """Quantise-dequantise v in blocks of 32 consecutive elements along `axis`."""
+    v = np.asarray(v, dtype=np.float64)
+    v = np.moveaxis(v, axis, -1)
+    n = v.shape[-1]
+    pad = (-n) % 32
+    if pad:
+        v = np.concatenate([v, np.zeros(v.shape[:-1] + (pad,))], axis=-1)
+    blk = v.reshape(v.shape[:-1] + (-1, 32))
+    s = mx_scale_exponent(np.max(np.abs(blk), axis=-1, keepdims=True))
+    X = np.exp2(s)
+    out = (e4m3_round(blk / X) * X).reshape(v.shape)[..., :n]
+    return np.moveaxis(out, -1, axis)
+
+
+def forward_mx(x, logits, wgu, wd, k):
+    """Forward with MXFP8 GEMM operands.
+
+    Gate/up GEMM: x and W_gate_up quantised along d.  Down GEMM: its operand
+    aw = w * silu(gate) * up (the routing weight folded into the activation)
+    and W_down quantised along I; out[t] = sum over slots of the down products.
+    Returns the same dict as forward, plus aw (per flat pair).
+    """
+    x, wgu, wd = _f64(x), _f64(wgu), _f64(wd)
+    T, d = x.shape
+    E, twoI, _ = wgu.shape
+    I = twoI // 2
+    idx, w = route(logits, k)
+    counts, offsets, perm, inv = dispatch(idx, E)
+    xq = mx_qdq_blocks(x, axis=1)
+    wguq = mx_qdq_blocks(wgu, axis=2)
+    wdq = mx_qdq_blocks(wd, axis=2)
+    wf = w.reshape(-1)
+    h = np.zeros((T * k, twoI))
+    aw = np.zeros((T * k, I))
+    y = np.zeros((T * k, d))
+    for e in range(E):
+        pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
+        if pairs.size == 0:
+            continue
+        he = xq[pairs // k] @ wguq[e].T
+        ae = wf[pairs][:, None] * (silu(he[:, :I]) * he[:, I:])
+        h[pairs], aw[pairs] = he, ae
+        y[pairs] = mx_qdq_blocks(ae, axis=1) @ wdq[e].T
+    out = np.zeros((T, d))
+    yk = y.reshape(T, k, d)
+    for j in range(k):
+        out += yk[:, j, :]
+    return dict(out=out, idx=idx, w=w, counts=counts, offsets=offsets, perm=perm, inv=inv, h=h, aw=aw, y=y)
+
+
+def backward_mx(x, logits, wgu, wd, k, gout, fwd):
+    """Backward with MXFP8 GEMM operands (fwd = forward_mx's result).
+
+    Down dgrad: grad_out rows and W_down along d.  Gate/up dgrad: dh and
+    W_gate_up along 2I.  Weight gradients: both operands along the expert's
+    tokens (sorted order, blocks of 32 from the expert's first pair).  The
+    SwiGLU backward and dscore use the unquantised h.
+    """
+    x, wgu, wd, gout = _f64(x), _f64(wgu), _f64(wd), _f64(gout)
+    T, d = x.shape
+    E, twoI, _ = wgu.shape
+    I = twoI // 2
+    idx, w, offsets, perm = fwd["idx"], fwd["w"], fwd["offsets"], fwd["perm"]
+    wf = w.reshape(-1)
+    goutq_d = mx_qdq_blocks(gout, axis=1)
+    wdq_d = mx_qdq_blocks(wd, axis=1)        # W_down[e] is [d, I]: blocks along d
+    wguq_2i = mx_qdq_blocks(wgu, axis=1)     # W_gate_up[e] is [2I, d]: blocks along 2I
+    dx_pair = np.zeros((T * k, d))
+    dscore = np.zeros(T * k)
+    dwgu = np.zeros_like(wgu)
+    dwd = np.zeros_like(wd)
+    for e in range(E):
+        pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
+        if pairs.size == 0:
+            continue
+        t = pairs // k
+        he = fwd["h"][pairs]
+        g, u = he[:, :I], he[:, I:]
+        a = silu(g) * u
+        G = goutq_d[t] @ wdq_d[e]
+        dscore[pairs] = np.sum(G * a, axis=1)
+        da = wf[pairs][:, None] * G
+        dh = np.concatenate([da * u * silu_grad(g), da * silu(g)], axis=1)
+        dx_pair[pairs] = mx_qdq_blocks(dh, axis=1) @ wguq_2i[e]
+        # K = the expert's tokens in sorted order, blocks of 32 from its first pair
+        dwd[e] = mx_qdq_blocks(gout[t], axis=0).T @ mx_qdq_blocks(fwd["aw"][pairs], axis=0)
+        dwgu[e] = mx_qdq_blocks(dh, axis=0).T @ mx_qdq_blocks(x[t], axis=0)
+    dx = np.zeros((T, d))
+    dxk = dx_pair.reshape(T, k, d)
+    for j in range(k):
+        dx += dxk[:, j, :]
+    dscore = dscore.reshape(T, k)
+    dl_slots = routing_backward(w, dscore)
+    dlogits = np.zeros((T, E))
+    np.put_along_axis(dlogits, idx.astype(np.int64), dl_slots, axis=1)
+    return dict(dx=dx, dwgu=dwgu, dwd=dwd, dscore=dscore, dlogits=dlogits)

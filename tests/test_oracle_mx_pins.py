@@ -1,0 +1,132 @@
+"""Pins for the oracle's MXFP8 operand quantisation and its MXFP8 layer.
+
+* the E4M3 grid is rebuilt from the format's bit fields (sign, 4 exponent
+  bits with bias 7, 3 mantissa bits, subnormals, 448 as the largest finite
+  magnitude): every code is a fixed point of e4m3_round, midpoints go to the
+  even code, larger magnitudes saturate;
+* the block scale exponent is checked against a brute-force search;
+* qdq is idempotent, scale-equivariant by powers of two and block-local;
+* with quantisation switched off, forward_mx / backward_mx reproduce the
+  pinned bf16 forward / backward (so their GEMM decomposition is right).
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def e4m3_codes():
+    """All finite non-negative E4M3 values from the bit fields (S.EEEE.MMM, bias 7)."""
+    vals = set()
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue  # the NaN code
+            if e == 0:
+                v = (m / 8.0) * 2.0 ** (1 - 7)
+            else:
+                v = (1 + m / 8.0) * 2.0 ** (e - 7)
+            vals.add(v)
+    return sorted(vals)
+
+
+def test_e4m3_codes_are_fixed_points_and_max_is_448():
+    codes = e4m3_codes()
+    assert max(codes) == 448.0 and len(codes) == 127
+    arr = np.array(codes + [-c for c in codes])
+    assert np.array_equal(O.e4m3_round(arr), arr)
+
+
+def test_e4m3_midpoints_round_to_even_code():
+    codes = e4m3_codes()
+    for lo, hi in zip(codes[:-1], codes[1:]):
+        mid = (lo + hi) / 2.0
+        # even code = even mantissa field; consecutive codes alternate parity
+        lo_code = codes.index(lo)
+        expect = lo if lo_code % 2 == 0 else hi
+        assert O.e4m3_round(np.array([mid]))[0] == expect, (lo, hi)
+        assert O.e4m3_round(np.array([math.nextafter(mid, 0)]))[0] == lo
+        assert O.e4m3_round(np.array([math.nextafter(mid, 1e9)]))[0] == hi
+
+
+def test_e4m3_saturates():
+    assert np.array_equal(O.e4m3_round(np.array([449.0, 1e6, -500.0])), [448.0, 448.0, -448.0])
+
+
+def test_scale_exponent_bruteforce():
+    rng = np.random.default_rng(1)
+    amax = np.concatenate([rng.lognormal(0, 6, 500), [448.0, 448.0 * 2 ** 3, 448.0 * 2 ** -5, 1e-30, 0.0]])
+    got = O.mx_scale_exponent(amax)
+    for a, s in zip(amax, got):
+        if a == 0:
+            assert s == 0
+            continue
+        best = next(t for t in range(-127, 128) if a <= 448.0 * 2.0 ** t)
+        assert s == best, (a, s, best)
+
+
+def test_qdq_idempotent_equivariant_blocklocal():
+    rng = np.random.default_rng(2)
+    v = rng.standard_normal((6, 96)) * np.exp(rng.standard_normal((6, 1)) * 3)
+    q = O.mx_qdq_blocks(v, axis=1)
+    assert np.array_equal(O.mx_qdq_blocks(q, axis=1), q)
+    assert np.array_equal(O.mx_qdq_blocks(v * 2.0 ** 5, axis=1), q * 2.0 ** 5)
+    v2 = v.copy()
+    v2[:, 32:64] *= 1000.0  # only the middle block's scale changes
+    q2 = O.mx_qdq_blocks(v2, axis=1)
+    assert np.array_equal(q2[:, :32], q[:, :32]) and np.array_equal(q2[:, 64:], q[:, 64:])
+    # the block maximum of a block whose amax is 448 * 2^s is kept exactly
+    w = rng.standard_normal(32) * 0.1
+    w[7] = 448.0 * 2.0 ** -6
+    assert O.mx_qdq_blocks(w[None, :], axis=1)[0, 7] == w[7]
+    # relative error per element is at most half an E4M3 spacing (2^-4) above the subnormal range
+    big = np.abs(v) > 2.0 ** -6 * np.max(np.abs(v))
+    assert np.max(np.abs(q - v)[big] / np.abs(v)[big]) <= 2.0 ** -4 + 1e-12
+
+
+def test_mx_layer_without_quantisation_is_the_bf16_layer(monkeypatch):
+    rng = np.random.default_rng(3)
+    T, d, E, k, I = 20, 64, 5, 2, 32
+    x = rng.standard_normal((T, d))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    wgu = rng.standard_normal((E, 2 * I, d)) * 0.2
+    wd = rng.standard_normal((E, d, I)) * 0.2
+    gout = rng.standard_normal((T, d))
+    ref_f = O.forward(x, logits, wgu, wd, k)
+    ref_b = O.backward(x, logits, wgu, wd, k, gout, ref_f)
+    monkeypatch.setattr(O, "mx_qdq_blocks", lambda v, axis: np.asarray(v, dtype=np.float64))
+    f = O.forward_mx(x, logits, wgu, wd, k)
+    b = O.backward_mx(x, logits, wgu, wd, k, gout, f)
+    assert np.allclose(f["out"], ref_f["out"], rtol=1e-12, atol=1e-12)
+    for key in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
+        assert np.allclose(b[key], ref_b[key], rtol=1e-11, atol=1e-12), key
+
+
+def test_mx_layer_close_to_bf16_layer():
+    rng = np.random.default_rng(4)
+    T, d, E, k, I = 40, 64, 4, 2, 32
+    x = rng.standard_normal((T, d))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    wgu = rng.standard_normal((E, 2 * I, d)) * 0.1
+    wd = rng.standard_normal((E, d, I)) * 0.1
+    gout = rng.standard_normal((T, d))
+    f = O.forward_mx(x, logits, wgu, wd, k)
+    ref = O.forward(x, logits, wgu, wd, k)
+    rel = np.linalg.norm(f["out"] - ref["out"]) / np.linalg.norm(ref["out"])
+    assert 1e-3 < rel < 0.1  # quantised, but only at E4M3 precision
+    b = O.backward_mx(x, logits, wgu, wd, k, gout, f)
+    rb = O.backward(x, logits, wgu, wd, k, gout, ref)
+    for key in ("dx", "dwgu", "dwd"):
+        rel = np.linalg.norm(b[key] - rb[key]) / np.linalg.norm(rb[key])
+        assert rel < 0.1, key
+
+
+def test_planted_mistake_scale_off_by_one(monkeypatch):
+    real = O.mx_scale_exponent
+    monkeypatch.setattr(O, "mx_scale_exponent", lambda a: real(a) - 1)  # would saturate block maxima
+    with pytest.raises(AssertionError):
+        test_scale_exponent_bruteforce()
