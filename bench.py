@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true", help="skip sampling nvidia-smi during the timed region")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0 = auto)")
     ap.add_argument("--override", default="", help="comma list of size overrides, e.g. T=4096,E=32 "
@@ -264,8 +265,9 @@ def main():
     M.profile_read()
     M.profile_enable(True)
     clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
+    if not args.no_clocks:
+        clocks.start()
+        time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)

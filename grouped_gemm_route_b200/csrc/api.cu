@@ -36,6 +36,11 @@ struct Plan {
     // workspace layout (byte offsets)
     size_t ws_status, ws_cnt, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
     size_t ws_dh, ws_dpart, ws_xs, ws_gs, bwd_bytes;
+    // MXFP8 operands: E4M3 codes and their scale atoms (forward, then backward)
+    bool mx;
+    size_t mx_x8, mx_xsf, mx_wgu8, mx_wgusf, mx_wd8, mx_wdsf, mx_aw8, mx_awsf;
+    size_t mx_gs8, mx_gssf, mx_wdt8, mx_wdtsf, mx_gsc8, mx_gscsf, mx_awc8, mx_awcsf, mx_wgut8, mx_wgutsf, mx_dh8,
+        mx_dhsf, mx_dhc8, mx_dhcsf, mx_xsc8, mx_xscsf;
     size_t saved[MOE_SAVED_FIELDS];
 };
 
@@ -45,7 +50,7 @@ int make_plan(const moe_shape_t *s, Plan *p) {
         return MOE_ERR_ARG;
     if (s->E > kMaxExperts || s->k > kMaxTopK) return MOE_ERR_SHAPE;
     if (s->d % 128 != 0 || s->I % 128 != 0) return MOE_ERR_SHAPE;
-    if (s->dtype != MOE_BF16) return s->dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_ARG;
+    if (s->dtype != MOE_BF16 && s->dtype != MOE_MXFP8) return MOE_ERR_ARG;
     const int64_t P = s->T * s->k;
     const int64_t widest = s->d > 2 * s->I ? s->d : 2 * static_cast<int64_t>(s->I);
     const int64_t nonempty = s->E < P ? s->E : P;
@@ -60,8 +65,9 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     p->p_cap = p_cap;
     p->m_tiles = p_cap / 128;
     p->n_chunks = static_cast<int>((s->T + kRouteChunk - 1) / kRouteChunk);
-    p->bn_d = s->d % 256 == 0 ? 256 : 128;
-    p->bn_i = s->I % 256 == 0 ? 256 : 128;
+    p->mx = s->dtype == MOE_MXFP8;
+    p->bn_d = !p->mx && s->d % 256 == 0 ? 256 : 128;  // MXFP8 GEMMs use 128-wide N tiles
+    p->bn_i = !p->mx && s->I % 256 == 0 ? 256 : 128;
     p->cnt_stride = s->d / p->bn_d;
     p->dpart_stride = s->I / p->bn_i;
 
@@ -77,6 +83,24 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     off = align_up(off + static_cast<size_t>(p->n_chunks) * s->E * 4);
     p->ws_chunk_base = off;
     off = align_up(off + static_cast<size_t>(p->n_chunks) * s->E * 4);
+    auto take = [&off](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes);
+        return at;
+    };
+    const size_t Td = static_cast<size_t>(s->T) * s->d, Pd = static_cast<size_t>(p_cap) * s->d;
+    const size_t PI = static_cast<size_t>(p_cap) * s->I, P2I = 2 * PI;
+    const size_t W2Id = static_cast<size_t>(s->E) * 2 * s->I * s->d, WdI = static_cast<size_t>(s->E) * s->d * s->I;
+    if (p->mx) {  // one scale byte per 32 elements
+        p->mx_x8 = take(Td);
+        p->mx_xsf = take(Td / 32);
+        p->mx_wgu8 = take(W2Id);
+        p->mx_wgusf = take(W2Id / 32);
+        p->mx_wd8 = take(WdI);
+        p->mx_wdsf = take(WdI / 32);
+        p->mx_aw8 = take(PI);
+        p->mx_awsf = take(PI / 32);
+    }
     p->fwd_bytes = off;
     off = common;
     p->ws_dh = off;
@@ -87,6 +111,24 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
     p->ws_gs = off;
     off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
+    if (p->mx) {
+        p->mx_gs8 = take(Pd);
+        p->mx_gssf = take(Pd / 32);
+        p->mx_wdt8 = take(WdI);
+        p->mx_wdtsf = take(WdI / 32);
+        p->mx_gsc8 = take(Pd);
+        p->mx_gscsf = take(Pd / 32);
+        p->mx_awc8 = take(PI);
+        p->mx_awcsf = take(PI / 32);
+        p->mx_wgut8 = take(W2Id);
+        p->mx_wgutsf = take(W2Id / 32);
+        p->mx_dh8 = take(P2I);
+        p->mx_dhsf = take(P2I / 32);
+        p->mx_dhc8 = take(P2I);
+        p->mx_dhcsf = take(P2I / 32);
+        p->mx_xsc8 = take(Pd);
+        p->mx_xscsf = take(Pd / 32);
+    }
     p->bwd_bytes = off;
 
     const size_t Tk = static_cast<size_t>(P);
@@ -157,6 +199,18 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint
     return r == CUDA_SUCCESS;
 }
 
+// 2-d E4M3 tensor [rows, cols] (row-major bytes), box = box_rows x 128 columns, 128-byte swizzle.
+bool make_map8(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint32_t box_rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // per-kernel timing (host bookkeeping only)
 // ---------------------------------------------------------------------------
@@ -207,7 +261,7 @@ struct Launch {
 const char *kKindNames[kNumKernelKinds] = {
     "route_topk",       "route_scan",       "route_perm",           "gemm_gateup_fwd",      "gemm_down_fwd_combine",
     "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd",
-    "sort_rows"};
+    "sort_rows", "mx_quant"};
 
 struct Saved {
     int32_t *idx;
@@ -270,6 +324,7 @@ GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
     a.I = pl.I;
     a.cnt_stride = pl.cnt_stride;
     a.dpart_stride = pl.dpart_stride;
+    a.k_elems = pl.mx ? 128 : kTileK;
     a.perm = sv->perm;
     a.group_start = sv->group_start;
     a.tile_expert = sv->tile_expert;
@@ -280,6 +335,139 @@ GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
     a.cnt = reinterpret_cast<int *>(ws + pl.ws_cnt);
     a.status = reinterpret_cast<int *>(ws + pl.ws_status);
     return a;
+}
+
+
+// MXFP8 forward after routing: quantise x (per-row scale bytes, for the
+// gather), W_gate_up (atoms in the tile's gate/up row order) and W_down, then
+// the two block-scaled GEMMs.  The gate/up epilogue writes aw's codes and scales.
+int fwd_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,
+           const void *w_down, void *out, moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
+    int rc;
+    const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I, Ed = static_cast<int64_t>(pl.E) * pl.d;
+    uint8_t *x8 = w8 + pl.mx_x8, *xsf = w8 + pl.mx_xsf, *wgu8 = w8 + pl.mx_wgu8, *wgusf = w8 + pl.mx_wgusf;
+    uint8_t *wd8 = w8 + pl.mx_wd8, *wdsf = w8 + pl.mx_wdsf, *aw8 = w8 + pl.mx_aw8, *awsf = w8 + pl.mx_awsf;
+    {
+        Launch L(kKindMxQuant, st);
+        if ((rc = L.done(launch_mx_quant_rows(static_cast<const __nv_bfloat16 *>(x), pl.T, pl.d, x8, xsf,
+                                              kMxSfRowBytes, pl.I, nullptr, dev.sms, st))))
+            return rc;
+    }
+    {
+        Launch L(kKindMxQuant, st);
+        if ((rc = L.done(launch_mx_quant_rows(static_cast<const __nv_bfloat16 *>(w_gate_up), EI2, pl.d, wgu8, wgusf,
+                                              kMxSfGateUp, pl.I, nullptr, dev.sms, st))))
+            return rc;
+    }
+    {
+        Launch L(kKindMxQuant, st);
+        if ((rc = L.done(launch_mx_quant_rows(static_cast<const __nv_bfloat16 *>(w_down), Ed, pl.I, wd8, wdsf,
+                                              kMxSfAtoms, pl.I, nullptr, dev.sms, st))))
+            return rc;
+    }
+    CUtensorMap tm_wgu8, tm_aw8, tm_wd8;
+    if (!make_map8(&tm_wgu8, wgu8, EI2, pl.d, 64) || !make_map8(&tm_aw8, aw8, pl.p_cap, pl.I, 128) ||
+        !make_map8(&tm_wd8, wd8, Ed, pl.I, 128))
+        return MOE_ERR_LAUNCH;
+    const int grid = grid_for(shape, dev);
+    GemmArgs a = base_args(pl, saved, w8);
+    a.n_tiles = pl.I / 64;
+    a.num_k_blocks = pl.d / 128;
+    a.gsrc = x8;
+    a.gsf = xsf;
+    a.sfb = wgusf;
+    a.mx_codes = aw8;
+    a.mx_sf = awsf;
+    {
+        Launch L(kKindGemmGateUpFwd, st);
+        if ((rc = L.done(launch_gemm(kGateUpFwd, 128, true, a, tm_wgu8, tm_wgu8, grid, st)))) return rc;
+    }
+    a.n_tiles = pl.d / 128;
+    a.num_k_blocks = pl.I / 128;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.sfa = awsf;
+    a.sfb = wdsf;
+    Launch L(kKindGemmDownFwd, st);
+    return L.done(launch_gemm(kDownFwd, 128, true, a, tm_aw8, tm_wd8, grid, st));
+}
+
+// MXFP8 backward after sort_rows: every GEMM operand quantised along that
+// GEMM's K (grad_out and W_down along d for the down dgrad, dh and W_gate_up
+// along 2I for the gate/up dgrad, both operands of each wgrad along the
+// expert's sorted rows); the down-dgrad epilogue writes dh's codes along 2I.
+int bwd_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *w_gate_up, const void *w_down,
+           const moe_saved_t *saved, void *dx, void *dw_gate_up, void *dw_down, GemmArgs a,
+           const __nv_bfloat16 *xs, const __nv_bfloat16 *gs, uint8_t *w8, cudaStream_t st) {
+    int rc;
+    const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I, Ed = static_cast<int64_t>(pl.E) * pl.d;
+    const int32_t *used = saved->group_start + pl.E;  // sorted rows in use
+    uint8_t *gs8 = w8 + pl.mx_gs8, *gssf = w8 + pl.mx_gssf, *wdt8 = w8 + pl.mx_wdt8, *wdtsf = w8 + pl.mx_wdtsf;
+    uint8_t *gsc8 = w8 + pl.mx_gsc8, *gscsf = w8 + pl.mx_gscsf, *awc8 = w8 + pl.mx_awc8, *awcsf = w8 + pl.mx_awcsf;
+    uint8_t *wgut8 = w8 + pl.mx_wgut8, *wgutsf = w8 + pl.mx_wgutsf, *dh8 = w8 + pl.mx_dh8, *dhsf = w8 + pl.mx_dhsf;
+    uint8_t *dhc8 = w8 + pl.mx_dhc8, *dhcsf = w8 + pl.mx_dhcsf, *xsc8 = w8 + pl.mx_xsc8, *xscsf = w8 + pl.mx_xscsf;
+    const __nv_bfloat16 *wd = static_cast<const __nv_bfloat16 *>(w_down);
+    const __nv_bfloat16 *wgu = static_cast<const __nv_bfloat16 *>(w_gate_up);
+    auto quant = [&](bool along_rows_of_src, const __nv_bfloat16 *src, int64_t rows, int cols, uint8_t *codes,
+                     uint8_t *sf, const int32_t *rows_used) {
+        Launch L(kKindMxQuant, st);
+        return along_rows_of_src
+                   ? L.done(launch_mx_quant_cols(src, rows, cols, codes, sf, rows_used, dev.sms, st))
+                   : L.done(launch_mx_quant_rows(src, rows, cols, codes, sf, kMxSfAtoms, pl.I, rows_used, dev.sms, st));
+    };
+    CUtensorMap tm_gs8, tm_wdt8, tm_gsc8, tm_awc8, tm_dh8, tm_wgut8, tm_dhc8, tm_xsc8;
+    if (!make_map8(&tm_gs8, gs8, pl.p_cap, pl.d, 128) || !make_map8(&tm_wdt8, wdt8, Ed, pl.I, 128) ||
+        !make_map8(&tm_gsc8, gsc8, pl.p_cap, pl.d, 128) || !make_map8(&tm_awc8, awc8, pl.p_cap, pl.I, 128) ||
+        !make_map8(&tm_dh8, dh8, pl.p_cap, 2 * pl.I, 128) || !make_map8(&tm_wgut8, wgut8, EI2, pl.d, 128) ||
+        !make_map8(&tm_dhc8, dhc8, pl.p_cap, 2 * pl.I, 128) || !make_map8(&tm_xsc8, xsc8, pl.p_cap, pl.d, 128))
+        return MOE_ERR_LAUNCH;
+    const int grid = grid_for(shape, dev);
+    // b1: down dgrad (K = d)
+    if ((rc = quant(false, gs, pl.p_cap, pl.d, gs8, gssf, used))) return rc;
+    if ((rc = quant(true, wd, Ed, pl.I, wdt8, wdtsf, nullptr))) return rc;
+    a.n_tiles = pl.I / 128;
+    a.num_k_blocks = pl.d / 128;
+    a.sfa = gssf;
+    a.sfb = wdtsf;
+    a.mx_codes = dh8;
+    a.mx_sf = dhsf;
+    {
+        Launch L(kKindGemmDownDgrad, st);
+        if ((rc = L.done(launch_gemm(kDownDgrad, 128, true, a, tm_gs8, tm_wdt8, grid, st)))) return rc;
+    }
+    // b3: down wgrad (K = sorted rows)
+    if ((rc = quant(true, gs, pl.p_cap, pl.d, gsc8, gscsf, used))) return rc;
+    if ((rc = quant(true, reinterpret_cast<const __nv_bfloat16 *>(saved->aw), pl.p_cap, pl.I, awc8, awcsf, used)))
+        return rc;
+    a.m_tiles = pl.d / 128;
+    a.n_tiles = pl.I / 128;
+    a.dw = static_cast<__nv_bfloat16 *>(dw_down);
+    a.sfa = gscsf;
+    a.sfb = awcsf;
+    {
+        Launch L(kKindGemmDownWgrad, st);
+        if ((rc = L.done(launch_gemm(kDownWgrad, 128, true, a, tm_gsc8, tm_awc8, grid, st)))) return rc;
+    }
+    // b4: gate/up dgrad + scatter (K = 2I)
+    if ((rc = quant(true, wgu, EI2, pl.d, wgut8, wgutsf, nullptr))) return rc;
+    a.n_tiles = pl.d / 128;
+    a.num_k_blocks = 2 * pl.I / 128;
+    a.out = static_cast<__nv_bfloat16 *>(dx);
+    a.sfa = dhsf;
+    a.sfb = wgutsf;
+    {
+        Launch L(kKindGemmGateUpDgrad, st);
+        if ((rc = L.done(launch_gemm(kGateUpDgrad, 128, true, a, tm_dh8, tm_wgut8, grid, st)))) return rc;
+    }
+    // b5: gate/up wgrad (K = sorted rows)
+    if ((rc = quant(true, a.dh, pl.p_cap, 2 * pl.I, dhc8, dhcsf, used))) return rc;
+    if ((rc = quant(true, xs, pl.p_cap, pl.d, xsc8, xscsf, used))) return rc;
+    a.m_tiles = 2 * pl.I / 128;
+    a.n_tiles = pl.d / 128;
+    a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
+    a.sfa = dhcsf;
+    a.sfb = xscsf;
+    Launch L(kKindGemmGateUpWgrad, st);
+    return L.done(launch_gemm(kGateUpWgrad, 128, true, a, tm_dhc8, tm_xsc8, grid, st));
 }
 
 }  // namespace
@@ -343,6 +531,7 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
 
     if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
     if ((rc = run_route(shape, pl, logits, saved, w8, st))) return rc;
+    if (pl.mx) return fwd_mx(pl, dev, shape, x, w_gate_up, w_down, out, saved, w8, st);
     const int grid = grid_for(shape, dev);
 
     GemmArgs a = base_args(pl, saved, w8);
@@ -351,14 +540,14 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
     a.gsrc = static_cast<const __nv_bfloat16 *>(x);  // token rows gathered through perm (A operand)
     {
         Launch L(kKindGemmGateUpFwd, st);
-        if ((rc = L.done(launch_gemm(kGateUpFwd, 256, a, tm_wgu, tm_wgu, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kGateUpFwd, 256, false, a, tm_wgu, tm_wgu, grid, st)))) return rc;
     }
     a.n_tiles = pl.d / pl.bn_d;
     a.num_k_blocks = pl.I / kTileK;
     a.out = static_cast<__nv_bfloat16 *>(out);
     {
         Launch L(kKindGemmDownFwd, st);
-        rc = L.done(launch_gemm(kDownFwd, pl.bn_d, a, tm_aw, tm_wd, grid, st));
+        rc = L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid, st));
     }
     return rc;
 }
@@ -407,12 +596,19 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
                                           static_cast<const __nv_bfloat16 *>(grad_out), xs, gs, dev.sms, st))))
             return rc;
     }
+    if (pl.mx) {
+        if ((rc = bwd_mx(pl, dev, shape, w_gate_up, w_down, saved, dx, dw_gate_up, dw_down, a, xs, gs, w8, st)))
+            return rc;
+        Launch L(kKindRouteBwd, st);
+        return L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_w, saved->topk_idx,
+                                       saved->inv, dpart, pl.dpart_stride, dscore, dlogits, st));
+    }
     // b1: down dgrad, dscore partials, SwiGLU backward -> dh; zeroes the dx counters
     a.n_tiles = pl.I / pl.bn_i;
     a.num_k_blocks = pl.d / kTileK;
     {
         Launch L(kKindGemmDownDgrad, st);
-        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, a, tm_gs_rows, tm_wd_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, false, a, tm_gs_rows, tm_wd_mn, grid, st)))) return rc;
     }
     // b3: down wgrad  dW_down[e] = sum_p gout[t] (x) aw_p
     a.m_tiles = pl.d / kTileM;
@@ -420,7 +616,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dw = static_cast<__nv_bfloat16 *>(dw_down);
     {
         Launch L(kKindGemmDownWgrad, st);
-        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, a, tm_gs_mn, tm_aw_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st)))) return rc;
     }
     // b4: gate/up dgrad + ordered scatter-sum into dx
     a.n_tiles = pl.d / pl.bn_d;
@@ -428,7 +624,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.out = static_cast<__nv_bfloat16 *>(dx);
     {
         Launch L(kKindGemmGateUpDgrad, st);
-        if ((rc = L.done(launch_gemm(kGateUpDgrad, pl.bn_d, a, tm_dh_rows, tm_wgu_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kGateUpDgrad, pl.bn_d, false, a, tm_dh_rows, tm_wgu_mn, grid, st)))) return rc;
     }
     // b5: gate/up wgrad  dW_gu[e] = sum_p dh_p (x) x[t]
     a.m_tiles = 2 * pl.I / kTileM;
@@ -436,7 +632,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
     {
         Launch L(kKindGemmGateUpWgrad, st);
-        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, a, tm_dh_mn, tm_xs_mn, grid, st)))) return rc;
+        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st)))) return rc;
     }
     // b6: dscore (ordered sum of partials) and dlogits
     {

@@ -41,6 +41,7 @@
 #include <stdint.h>
 
 #include "moe_internal.h"
+#include "mx.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -57,17 +58,26 @@ constexpr uint32_t kMnLbo = kChunkBytes;      // MN-major: distance between 64-w
 constexpr int kXposeBytes = 32 * 64;          // per epilogue warp: 32 rows x 64 bytes
 constexpr int kTailCap = 2048;                // finished (token, column tile) pairs a CTA defers to its tail
 
-template <int BN>
+// Pipeline geometry.  A stage holds one K block of both operands: 128-byte
+// operand rows, i.e. 64 bf16 or 128 E4M3 elements.  MXFP8 stages also carry
+// the A and B scale atoms (512 bytes each) and use BN = 128 so that the two
+// 128-column accumulators leave tensor-memory columns for the scales.
+template <int BN, bool MX = false>
 struct Cfg {
     static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kKElems = MX ? 128 : 64;                  // K elements per stage
     static constexpr int kBBytes = BN * kTileK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kBarOffset = kStages * kStageBytes;      // mbarriers, TMEM slot, abort flag
+    static constexpr int kSfBytes = MX ? 2 * kMxAtomBytes : 0;     // scale atoms per stage
+    static constexpr int kSfOffset = kStages * kStageBytes;
+    static constexpr int kBarOffset = kSfOffset + kStages * kSfBytes;  // mbarriers, TMEM slot, abort flag
     static constexpr int kOrderOffset = kBarOffset + 512;         // wgrad expert order
     static constexpr int kXposeOffset = kOrderOffset + 2 * kMaxExperts * 4;   // 4 x 2 KB epilogue transposes
     static constexpr int kTailOffset = kXposeOffset + 4 * kXposeBytes;        // combine: finished tokens
     static constexpr int kSmemBytes = kTailOffset + 4 * (kTailCap + 4) + 1024;  // + 1 KB alignment slack
-    static constexpr uint32_t kTmemCols = 2 * BN;
+    static constexpr uint32_t kTmemCols = MX ? 512 : 2 * BN;
+    static constexpr uint32_t kSfaCol = 2 * BN;                    // MXFP8 scale columns after the accumulators
+    static constexpr uint32_t kSfbCol = 2 * BN + 8;
 };
 
 template <int MODE>
@@ -80,9 +90,10 @@ struct ModeTraits {
 };
 
 // Bytes of one stage that arrive by TMA (the gathered operand arrives by cp.async).
-template <int MODE, int BN>
+template <int MODE, int BN, bool MX>
 __host__ __device__ constexpr uint32_t tma_stage_bytes() {
-    return ModeTraits<MODE>::kGather ? Cfg<BN>::kBBytes : Cfg<BN>::kStageBytes;
+    return (ModeTraits<MODE>::kGather ? Cfg<BN, MX>::kBBytes : Cfg<BN, MX>::kStageBytes) +
+           (MX ? (ModeTraits<MODE>::kGather ? kMxAtomBytes : 2 * kMxAtomBytes) : 0);
 }
 
 struct Tile {
@@ -112,7 +123,7 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const i
         t.mt = r / a.n_tiles;
         t.nt = r - t.mt * a.n_tiles;
         const int gs = __ldg(a.group_start + t.e), ge = __ldg(a.group_start + t.e + 1);
-        t.nkb = (ge - gs) / kTileK;
+        t.nkb = (ge - gs) / a.k_elems;
         t.kpos0 = gs;
     }
     if (t.e < 0 || t.e >= a.E) {  // corrupted routing state: do no work for this tile
@@ -209,10 +220,10 @@ __device__ __forceinline__ void raise_abort(volatile int *abort_flag, int *statu
 // ---------------------------------------------------------------------------
 // TMA producer (warp 0): the operand(s) that are not gathered
 // ---------------------------------------------------------------------------
-template <int MODE, int BN>
+template <int MODE, int BN, bool MX>
 __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, const GemmArgs &a, uint8_t *smem,
                               uint64_t *full, uint64_t *empty, const int *order, volatile int *abort_flag) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, MX>;
     const int lane = threadIdx.x & 31;
     const int total = total_tiles<MODE>(a);
     int it = 0;
@@ -226,12 +237,58 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
                 ok = false;
                 break;
             }
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], tma_stage_bytes<MODE, BN>());
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], tma_stage_bytes<MODE, BN, MX>());
             __syncwarp();
             uint8_t *As = smem + s * C::kStageBytes;
             uint8_t *Bs = As + kABytes;
-            const int k0 = kb * kTileK;
-            if constexpr (MODE == kGateUpFwd) {
+            const int k0 = kb * C::kKElems;
+            if constexpr (MX) {
+                // E4M3 operands (one 128 x 128-byte box each) and their scale atoms
+                uint8_t *sfs = smem + C::kSfOffset + s * C::kSfBytes;  // [A atom | B atom]
+                const int64_t kblk = kb;                               // K block of 128
+                if (lane == 0) {
+                    if constexpr (MODE == kGateUpFwd) {
+                        const int row = t.e * 2 * a.I + t.nt * 64;
+                        tma_load_2d(Bs, tmB, &full[s], k0, row);                   // 64 gate rows
+                        tma_load_2d(Bs + 64 * 128, tmB, &full[s], k0, row + a.I);  // 64 up rows
+                        bulk_load(sfs + kMxAtomBytes,
+                                  a.sfb + ((static_cast<int64_t>(t.e) * (a.I / 64) + t.nt) * (a.d / 128) + kblk) * kMxAtomBytes,
+                                  kMxAtomBytes, &full[s]);
+                    } else if constexpr (MODE == kDownFwd) {
+                        tma_load_2d(As, tmA, &full[s], k0, t.mt * kTileM);
+                        tma_load_2d(Bs, tmB, &full[s], k0, t.e * a.d + t.nt * 128);
+                        bulk_load(sfs, a.sfa + (static_cast<int64_t>(t.mt) * (a.I / 128) + kblk) * kMxAtomBytes,
+                                  kMxAtomBytes, &full[s]);
+                        bulk_load(sfs + kMxAtomBytes,
+                                  a.sfb + ((static_cast<int64_t>(t.e) * a.d + t.nt * 128) / 128 * (a.I / 128) + kblk) * kMxAtomBytes,
+                                  kMxAtomBytes, &full[s]);
+                    } else if constexpr (MODE == kDownDgrad) {
+                        tma_load_2d(As, tmA, &full[s], k0, t.mt * kTileM);
+                        tma_load_2d(Bs, tmB, &full[s], t.nt * 128, t.e * a.d + k0);
+                        bulk_load(sfs, a.sfa + (static_cast<int64_t>(t.mt) * (a.d / 128) + kblk) * kMxAtomBytes,
+                                  kMxAtomBytes, &full[s]);
+                        bulk_load(sfs + kMxAtomBytes,
+                                  a.sfb + ((static_cast<int64_t>(t.e) * a.d + k0) / 128 * (a.I / 128) + t.nt) * kMxAtomBytes,
+                                  kMxAtomBytes, &full[s]);
+                    } else if constexpr (MODE == kGateUpDgrad) {
+                        tma_load_2d(As, tmA, &full[s], k0, t.mt * kTileM);
+                        tma_load_2d(Bs, tmB, &full[s], t.nt * 128, t.e * 2 * a.I + k0);
+                        bulk_load(sfs, a.sfa + (static_cast<int64_t>(t.mt) * (2 * a.I / 128) + kblk) * kMxAtomBytes,
+                                  kMxAtomBytes, &full[s]);
+                        bulk_load(sfs + kMxAtomBytes,
+                                  a.sfb + ((static_cast<int64_t>(t.e) * 2 * a.I + k0) / 128 * (a.d / 128) + t.nt) * kMxAtomBytes,
+                                  kMxAtomBytes, &full[s]);
+                    } else {  // wgrads: K = the expert's sorted rows, both operands MN-major
+                        const int64_t kr = (static_cast<int64_t>(t.kpos0) + k0) / 128;
+                        const int mw = MODE == kDownWgrad ? a.d / 128 : 2 * a.I / 128;  // M extent in 128-blocks
+                        const int nw = MODE == kDownWgrad ? a.I / 128 : a.d / 128;      // N extent in 128-blocks
+                        tma_load_2d(As, tmA, &full[s], t.mt * kTileM, t.kpos0 + k0);
+                        tma_load_2d(Bs, tmB, &full[s], t.nt * 128, t.kpos0 + k0);
+                        bulk_load(sfs, a.sfa + (kr * mw + t.mt) * kMxAtomBytes, kMxAtomBytes, &full[s]);
+                        bulk_load(sfs + kMxAtomBytes, a.sfb + (kr * nw + t.nt) * kMxAtomBytes, kMxAtomBytes, &full[s]);
+                    }
+                }
+            } else if constexpr (MODE == kGateUpFwd) {
                 if (lane == 0) {
                     const int row = t.e * 2 * a.I + t.nt * (BN / 2);
                     tma_load_2d(Bs, tmB, &full[s], k0, row);                         // gate rows
@@ -281,56 +338,67 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
 // Thread g (0..63) copies 16-byte piece (g & 7) of the 128-byte rows
 // r = (g >> 3) + 8 i.  A row r of a 128-byte-swizzled stage lives at byte
 // r * 128, with its 16-byte piece c stored at position c ^ (r & 7).
-template <int MODE, int BN>
+template <int MODE, int BN, bool MX>
 __device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty, const int *order,
                             volatile int *abort_flag) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, MX>;
     const int g = threadIdx.x - kGatherWarp0 * 32;
     const int piece = g & 7;
     const int rg = g >> 3;
-    const size_t d = static_cast<size_t>(a.d);
+    const size_t row_bytes = static_cast<size_t>(a.d) * (MX ? 1 : 2);  // E4M3 codes or bf16
+    const uint8_t *src = static_cast<const uint8_t *>(a.gsrc);
     const int total = total_tiles<MODE>(a);
     int it = 0;
     bool ok = true;
-    {
-        // 16 rows of the 128-row tile per thread; K-major, one 128-byte row per K block
-        int tok[16], nxt[16];
-        int tile = blockIdx.x;
-        if (tile < total) {
-            const int mt = tile / a.n_tiles;
+    // 16 rows of the 128-row tile per thread; K-major, one 128-byte row piece per K block.
+    // MXFP8: the 8 piece-0 threads also copy each row's 4 scale bytes of the K block
+    // into the A scale atom of the stage.
+    int tok[16], nxt[16];
+    int tile = blockIdx.x;
+    if (tile < total) {
+        const int mt = tile / a.n_tiles;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) tok[i] = token_of(a, mt * kTileM + rg + 8 * i);
+        for (int i = 0; i < 16; ++i) tok[i] = token_of(a, mt * kTileM + rg + 8 * i);
+    }
+    for (; tile < total && ok; tile += gridDim.x) {
+        const Tile t = decode_tile<MODE>(tile, a, order);
+        const int next = tile + gridDim.x;
+        if (next < total) {  // prefetch the next tile's token rows
+            const int mt = next / a.n_tiles;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) nxt[i] = token_of(a, mt * kTileM + rg + 8 * i);
         }
-        for (; tile < total && ok; tile += gridDim.x) {
-            const Tile t = decode_tile<MODE>(tile, a, order);
-            const int next = tile + gridDim.x;
-            if (next < total) {  // prefetch the next tile's token rows
-                const int mt = next / a.n_tiles;
+        const uint8_t *rows[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) nxt[i] = token_of(a, mt * kTileM + rg + 8 * i);
+        for (int i = 0; i < 16; ++i) rows[i] = src + static_cast<size_t>(tok[i]) * row_bytes + piece * 16;
+        for (int kb = 0; kb < t.nkb; ++kb) {
+            const int s = it % C::kStages;
+            const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
+            if (!warp_wait(&empty[s], ph ^ 1u, abort_flag)) {
+                ok = false;
+                break;
             }
-            const __nv_bfloat16 *rows[16];
+            const uint32_t As = smem_u32(smem + s * C::kStageBytes);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) rows[i] = a.gsrc + static_cast<size_t>(tok[i]) * d + piece * 8;
-            for (int kb = 0; kb < t.nkb; ++kb) {
-                const int s = it % C::kStages;
-                const uint32_t ph = static_cast<uint32_t>(it / C::kStages) & 1u;
-                if (!warp_wait(&empty[s], ph ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t As = smem_u32(smem + s * C::kStageBytes);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int r = rg + 8 * i;
-                    cp_async_16(As + r * 128 + ((piece ^ (r & 7)) << 4), rows[i] + kb * kTileK);
-                }
-                cp_async_arrive_noinc(&full[s]);
-                ++it;
+            for (int i = 0; i < 16; ++i) {
+                const int r = rg + 8 * i;
+                cp_async_16(As + r * 128 + ((piece ^ (r & 7)) << 4), rows[i] + kb * 128);
             }
+            if constexpr (MX) {
+                if (piece == 0) {
+                    const uint32_t sfa = smem_u32(smem + C::kSfOffset + s * C::kSfBytes);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) tok[i] = nxt[i];
+                    for (int i = 0; i < 16; ++i) {
+                        const int r = rg + 8 * i;
+                        cp_async_4(sfa + mx_atom_byte(r, 0), a.gsf + static_cast<size_t>(tok[i]) * (a.d / kMxBlock) + kb * 4);
+                    }
+                }
+            }
+            cp_async_arrive_noinc(&full[s]);
+            ++it;
         }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) tok[i] = nxt[i];
     }
     if (!ok) raise_abort(abort_flag, a.status);
     cp_async_wait_all();  // our copies land before the CTA can exit
@@ -339,11 +407,11 @@ __device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, ui
 // ---------------------------------------------------------------------------
 // MMA issuer (warp 1, one thread)
 // ---------------------------------------------------------------------------
-template <int MODE, int BN>
+template <int MODE, int BN, bool MX>
 __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty, uint64_t *tfull,
                          uint64_t *tempty, uint64_t *drain, uint32_t tmem_base, const int *order,
                          volatile int *abort_flag) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, MX>;
     using TR = ModeTraits<MODE>;
     constexpr uint32_t kIdesc = instr_desc_bf16(kTileM, BN, TR::kAMn, TR::kBMn);
     const int total = total_tiles<MODE>(a);
@@ -370,13 +438,32 @@ __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint6
             tc_fence_after_sync();
             const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
             const uint32_t b_base = a_base + kABytes;
+            if constexpr (MX) {
+                // scale atoms -> tensor memory (ordered before the MMAs that read them),
+                // then four K=32 block-scaled MMAs; sf_id k picks scale byte k
+                const uint32_t sf_base = smem_u32(smem + C::kSfOffset + s * C::kSfBytes);
+                const uint32_t sfa_t = tmem_base + C::kSfaCol, sfb_t = tmem_base + C::kSfbCol;
+                tmem_copy_32x128b_x4(sfa_t, smem_desc_plain(sf_base, 128));
+                tmem_copy_32x128b_x4(sfb_t, smem_desc_plain(sf_base + kMxAtomBytes, 128));
 #pragma unroll
-            for (int kk = 0; kk < kTileK / 16; ++kk) {
-                const uint64_t ad = TR::kAMn ? smem_desc_sw128(a_base + kk * 2048, kMnLbo, kSbo)
-                                             : smem_desc_sw128(a_base + kk * 32, 16, kSbo);
-                const uint64_t bd = TR::kBMn ? smem_desc_sw128(b_base + kk * 2048, kMnLbo, kSbo)
-                                             : smem_desc_sw128(b_base + kk * 32, 16, kSbo);
-                mma_bf16(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = TR::kAMn ? smem_desc_sw128(a_base + kk * 4096, 16384, kSbo)
+                                                 : smem_desc_sw128(a_base + kk * 32, 16, kSbo);
+                    const uint64_t bd = TR::kBMn ? smem_desc_sw128(b_base + kk * 4096, 16384, kSbo)
+                                                 : smem_desc_sw128(b_base + kk * 32, 16, kSbo);
+                    mma_mxf8(d_tmem, ad, bd, instr_desc_mxf8(kTileM, BN, TR::kAMn, TR::kBMn, kk),
+                             sfa_t | (static_cast<uint32_t>(kk) << 30), sfb_t | (static_cast<uint32_t>(kk) << 30),
+                             (kb | kk) != 0 ? 1u : 0u);
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < kTileK / 16; ++kk) {
+                    const uint64_t ad = TR::kAMn ? smem_desc_sw128(a_base + kk * 2048, kMnLbo, kSbo)
+                                                 : smem_desc_sw128(a_base + kk * 32, 16, kSbo);
+                    const uint64_t bd = TR::kBMn ? smem_desc_sw128(b_base + kk * 2048, kMnLbo, kSbo)
+                                                 : smem_desc_sw128(b_base + kk * 32, 16, kSbo);
+                    mma_bf16(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                }
             }
             mma_commit(&empty[s]);  // frees the stage once these MMAs have read it
         }
@@ -406,8 +493,9 @@ struct TailList {
     int *count;
 };
 
-// gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up
-template <int BN>
+// gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up.
+// MXFP8: also aw's E4M3 codes and scale atoms along I (the down GEMM's K).
+template <int BN, bool MX>
 __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                                uint64_t *tempty_acc, uint8_t *xbuf) {
     constexpr int kHalf = BN / 2;
@@ -427,23 +515,32 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
         tmem_regs_ready(ur);
         if (c + 1 == kHalf / 32) release_accumulator(tempty_acc);  // TMEM no longer needed
         uint32_t pg[16], pu[16], pa[16];
+        float av[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float g = __uint_as_float(gr[i]), u = __uint_as_float(ur[i]);
+            av[i] = valid ? wv * g * __fdividef(1.f, 1.f + __expf(-g)) * u : 0.f;
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            if (valid) {
-                const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
-                const float u0 = __uint_as_float(ur[2 * i]), u1 = __uint_as_float(ur[2 * i + 1]);
-                const float s0 = __fdividef(1.f, 1.f + __expf(-g0));
-                const float s1 = __fdividef(1.f, 1.f + __expf(-g1));
-                pg[i] = pack_bf16x2(g0, g1);
-                pu[i] = pack_bf16x2(u0, u1);
-                pa[i] = pack_bf16x2(wv * g0 * s0 * u0, wv * g1 * s1 * u1);
-            } else {
-                pg[i] = pu[i] = pa[i] = 0u;
-            }
+            pg[i] = valid ? pack_bf16x2(__uint_as_float(gr[2 * i]), __uint_as_float(gr[2 * i + 1])) : 0u;
+            pu[i] = valid ? pack_bf16x2(__uint_as_float(ur[2 * i]), __uint_as_float(ur[2 * i + 1])) : 0u;
+            pa[i] = pack_bf16x2(av[2 * i], av[2 * i + 1]);
         }
         warp_store_rows(xbuf, pg, hrow + c * 32);
         warp_store_rows(xbuf, pu, hrow + a.I + c * 32);
         warp_store_rows(xbuf, pa, arow + c * 32);
+        if constexpr (MX) {
+            const int col = t.nt * kHalf + c * 32;
+            const int sc = mx_scale_exp(amax32(av));
+            uint32_t codes[8];
+            mx_encode32(av, sc, codes);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.mx_codes + static_cast<size_t>(pos) * a.I + col);
+            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            const int64_t atom = static_cast<int64_t>(t.mt) * (a.I / 128) + col / 128;
+            a.mx_sf[atom * kMxAtomBytes + mx_atom_byte(r, col / 32)] = static_cast<uint8_t>(sc + 127);
+        }
     }
 }
 
@@ -604,8 +701,9 @@ __device__ __forceinline__ void combine_tail(const GemmArgs &a, const TailList &
     for (int i = warp * 4; i < n; i += (kThreads / 32) * 4) combine_tokens4<BN>(a, tail.items + i, min(4, n - i));
 }
 
-// down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh
-template <int BN>
+// down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh.
+// MXFP8: also dh's E4M3 codes and scale atoms along 2I (the gate/up dgrad's K).
+template <int BN, bool MX>
 __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                                uint64_t *tempty_acc, uint8_t *xbuf) {
     const int pos = t.mt * kTileM + r;
@@ -623,27 +721,41 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
         float G[32];
         tmem_load32_sync(taddr + c * 32, G);
         if (c + 1 == BN / 32) release_accumulator(tempty_acc);
+        float dg[32], du[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float g = (i & 1) ? bf16_hi(hg[i >> 1]) : bf16_lo(hg[i >> 1]);
+            const float u = (i & 1) ? bf16_hi(hu[i >> 1]) : bf16_lo(hu[i >> 1]);
+            const float gr = G[i];
+            const float sg = __fdividef(1.f, 1.f + __expf(-g));
+            const float sl = g * sg;
+            ds += gr * (sl * u);
+            const float da = wv * gr;
+            dg[i] = valid ? da * u * sg * (1.f + g * (1.f - sg)) : 0.f;
+            du[i] = valid ? da * sl : 0.f;
+        }
         uint32_t pdg[16], pdu[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            float dgv[2], duv[2];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const float g = h2 ? bf16_hi(hg[i]) : bf16_lo(hg[i]);
-                const float u = h2 ? bf16_hi(hu[i]) : bf16_lo(hu[i]);
-                const float gr = G[2 * i + h2];
-                const float sg = __fdividef(1.f, 1.f + __expf(-g));
-                const float sl = g * sg;
-                ds += gr * (sl * u);
-                const float da = wv * gr;
-                dgv[h2] = da * u * sg * (1.f + g * (1.f - sg));
-                duv[h2] = da * sl;
-            }
-            pdg[i] = valid ? pack_bf16x2(dgv[0], dgv[1]) : 0u;
-            pdu[i] = valid ? pack_bf16x2(duv[0], duv[1]) : 0u;
+            pdg[i] = pack_bf16x2(dg[2 * i], dg[2 * i + 1]);
+            pdu[i] = pack_bf16x2(du[2 * i], du[2 * i + 1]);
         }
         warp_store_rows(xbuf, pdg, dhrow + c * 32);
         warp_store_rows(xbuf, pdu, dhrow + a.I + c * 32);
+        if constexpr (MX) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int col = (half ? a.I : 0) + t.nt * BN + c * 32;
+                const int sc = mx_scale_exp(amax32(half ? du : dg));
+                uint32_t codes[8];
+                mx_encode32(half ? du : dg, sc, codes);
+                uint4 *dst = reinterpret_cast<uint4 *>(a.mx_codes + static_cast<size_t>(pos) * 2 * a.I + col);
+                dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                const int64_t atom = static_cast<int64_t>(t.mt) * (2 * a.I / 128) + col / 128;
+                a.mx_sf[atom * kMxAtomBytes + mx_atom_byte(r, col / 32)] = static_cast<uint8_t>(sc + 127);
+            }
+        }
     }
     a.dpart[static_cast<size_t>(pos) * a.dpart_stride + t.nt] = valid ? ds : 0.f;
     if (valid && t.nt == 0) {  // counters of the dx scatter that follows
@@ -677,7 +789,7 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
     }
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool MX>
 __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *tempty, uint32_t tmem_base,
                               const int *order, uint8_t *xbuf, const TailList &tail, volatile int *abort_flag) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -696,22 +808,22 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
         tc_fence_after_sync();
         const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
         if constexpr (MODE == kGateUpFwd) {
-            epi_gateup_fwd<BN>(a, t, r, taddr, &tempty[acc], xbuf);
+            epi_gateup_fwd<BN, MX>(a, t, r, taddr, &tempty[acc], xbuf);
         } else if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
             epi_combine<BN>(a, t, r, taddr, &tempty[acc], xbuf, tail);
         } else if constexpr (MODE == kDownDgrad) {
-            epi_down_dgrad<BN>(a, t, r, taddr, &tempty[acc], xbuf);
+            epi_down_dgrad<BN, MX>(a, t, r, taddr, &tempty[acc], xbuf);
         } else {
             epi_wgrad<MODE, BN>(a, t, r, taddr, &tempty[acc], xbuf);
         }
     }
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmArgs args) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, MX>;
     using TR = ModeTraits<MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -766,16 +878,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        producer_loop<MODE, BN>(&tmA, &tmB, args, smem, full, empty, order, abort_flag);
+        producer_loop<MODE, BN, MX>(&tmA, &tmB, args, smem, full, empty, order, abort_flag);
     } else if (warp == 1) {
         if ((threadIdx.x & 31) == 0)
-            mma_loop<MODE, BN>(args, smem, full, empty, tfull, tempty, drain, tmem_base, order, abort_flag);
+            mma_loop<MODE, BN, MX>(args, smem, full, empty, tfull, tempty, drain, tmem_base, order, abort_flag);
         __syncwarp();
     } else if (warp < kGatherWarp0) {
-        epilogue_loop<MODE, BN>(args, tfull, tempty, tmem_base, order,
+        epilogue_loop<MODE, BN, MX>(args, tfull, tempty, tmem_base, order,
                                 smem + C::kXposeOffset + (warp - 2) * kXposeBytes, tail, abort_flag);
     } else if constexpr (TR::kGather) {
-        gather_loop<MODE, BN>(args, smem, full, empty, order, abort_flag);
+        gather_loop<MODE, BN, MX>(args, smem, full, empty, order, abort_flag);
     }
 
     tc_fence_before_sync();
@@ -787,39 +899,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool MX>
 cudaError_t launch_one(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
                        cudaStream_t s) {
     static bool attr_set = false;  // per instantiation; the attribute is per function and process-wide
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN, MX>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN, MX>::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    grouped_gemm_kernel<MODE, BN><<<grid, kThreads, Cfg<BN>::kSmemBytes, s>>>(tmA, tmB, args);
+    grouped_gemm_kernel<MODE, BN, MX><<<grid, kThreads, Cfg<BN, MX>::kSmemBytes, s>>>(tmA, tmB, args);
     return cudaGetLastError();
 }
 
 template <int MODE>
-cudaError_t launch_mode(int bn, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
-                        cudaStream_t s) {
-    if (bn == 256) return launch_one<MODE, 256>(args, tmA, tmB, grid, s);
-    if (bn == 128) return launch_one<MODE, 128>(args, tmA, tmB, grid, s);
+cudaError_t launch_mode(int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        int grid, cudaStream_t s) {
+    if (mx) return bn == 128 ? launch_one<MODE, 128, true>(args, tmA, tmB, grid, s) : cudaErrorInvalidValue;
+    if (bn == 256) return launch_one<MODE, 256, false>(args, tmA, tmB, grid, s);
+    if (bn == 128) return launch_one<MODE, 128, false>(args, tmA, tmB, grid, s);
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(GemmMode mode, int bn, const GemmArgs &args, const CUtensorMap &tmA,
+cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA,
                         const CUtensorMap &tmB, int grid, cudaStream_t s) {
     switch (mode) {
-        case kGateUpFwd: return launch_mode<kGateUpFwd>(bn, args, tmA, tmB, grid, s);
-        case kDownFwd: return launch_mode<kDownFwd>(bn, args, tmA, tmB, grid, s);
-        case kDownDgrad: return launch_mode<kDownDgrad>(bn, args, tmA, tmB, grid, s);
-        case kGateUpDgrad: return launch_mode<kGateUpDgrad>(bn, args, tmA, tmB, grid, s);
-        case kDownWgrad: return launch_mode<kDownWgrad>(bn, args, tmA, tmB, grid, s);
-        case kGateUpWgrad: return launch_mode<kGateUpWgrad>(bn, args, tmA, tmB, grid, s);
+        case kGateUpFwd: return launch_mode<kGateUpFwd>(bn, mx, args, tmA, tmB, grid, s);
+        case kDownFwd: return launch_mode<kDownFwd>(bn, mx, args, tmA, tmB, grid, s);
+        case kDownDgrad: return launch_mode<kDownDgrad>(bn, mx, args, tmA, tmB, grid, s);
+        case kGateUpDgrad: return launch_mode<kGateUpDgrad>(bn, mx, args, tmA, tmB, grid, s);
+        case kDownWgrad: return launch_mode<kDownWgrad>(bn, mx, args, tmA, tmB, grid, s);
+        case kGateUpWgrad: return launch_mode<kGateUpWgrad>(bn, mx, args, tmA, tmB, grid, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -17,6 +17,9 @@ constexpr int kRouteChunk = 64;   // tokens per routing block
 constexpr int kMaxExperts = 512;
 constexpr int kMaxTopK = 64;
 
+// Where the MXFP8 quantiser puts the block scales.
+enum MxSfMode : int { kMxSfAtoms = 0, kMxSfRowBytes = 1, kMxSfGateUp = 2 };
+
 // Kernel kinds, for per-kernel timing.
 enum KernelKind : int {
     kKindRouteTopk = 0,
@@ -30,6 +33,7 @@ enum KernelKind : int {
     kKindGemmGateUpWgrad,
     kKindRouteBwd,
     kKindSortRows,
+    kKindMxQuant,
     kNumKernelKinds
 };
 
@@ -48,13 +52,19 @@ struct GemmArgs {
     int n_tiles;          // tiles along N
     int m_tiles;          // wgrad: tiles along M of one expert's weight
     int num_k_blocks;     // M-tiled modes: K / 64
+    int k_elems;          // K elements per pipeline stage: 64 (bf16) or 128 (MXFP8)
     int cnt_stride;       // combine counters per token
     int dpart_stride;     // dscore partials per sorted row
     const int *perm;
     const int *group_start;
     const int *tile_expert;
     const float *topk_w;
-    const __nv_bfloat16 *gsrc;  // token rows the gather warps read: x or grad_out [T, d]
+    const void *gsrc;           // token rows the gather warps read (x: bf16, or its E4M3 codes)
+    const uint8_t *gsf;         // MXFP8: per-row scale bytes of the gathered rows [T, d/32]
+    const uint8_t *sfa;         // MXFP8: scale atoms of the A operand (TMA-fed)
+    const uint8_t *sfb;         // MXFP8: scale atoms of the B operand
+    uint8_t *mx_codes;          // MXFP8 epilogue output codes (aw or dh)
+    uint8_t *mx_sf;             // and their scale atoms
     __nv_bfloat16 *h;
     __nv_bfloat16 *aw;
     __nv_bfloat16 *stage;
@@ -82,7 +92,12 @@ cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t 
 
 cudaError_t launch_expire_wait(int *status, cudaStream_t s);
 
-cudaError_t launch_gemm(GemmMode mode, int bn, const GemmArgs &args, const CUtensorMap &tmA,
+cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA,
                         const CUtensorMap &tmB, int grid, cudaStream_t s);
+
+cudaError_t launch_mx_quant_rows(const __nv_bfloat16 *src, int64_t R, int K, uint8_t *dst, uint8_t *sf, int sf_mode,
+                                 int I, const int32_t *rows_used, int sms, cudaStream_t s);
+cudaError_t launch_mx_quant_cols(const __nv_bfloat16 *src, int64_t Kr, int N, uint8_t *dst, uint8_t *sf,
+                                 const int32_t *rows_used, int sms, cudaStream_t s);
 
 }  // namespace moe

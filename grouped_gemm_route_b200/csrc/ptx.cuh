@@ -93,6 +93,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Contiguous bytes global -> shared (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Four rows (r0..r3) of a 2-d tensor, columns [x, x + box width), written to
 // shared memory as four consecutive rows.  The tensor map's box is one row high.
 __device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int r0,
@@ -115,6 +123,11 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void *src) 
 // (the arrival is counted in the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 4-byte variant (L1-allocating form; the 16-byte form above bypasses L1).
+__device__ __forceinline__ void cp_async_4(uint32_t dst_smem, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
@@ -158,6 +171,25 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// MXFP8 MMA: D (+)= (A * 2^sfa) (B * 2^sfb)^T with E4M3 A and B and UE8M0
+// scales in tensor memory (one per 32 K elements per row; idesc selects the
+// byte of each scale word).
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// 32 rows x 16 bytes of shared memory into 4 tensor-memory columns of lanes
+// 0..31, replicated to the other three lane quadrants.
+__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far has completed.
@@ -219,6 +251,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
     d |= static_cast<uint64_t>(2) << 61;  // layout: 128-byte swizzle
     return d;
+}
+
+// Unswizzled K-major descriptor for tcgen05.cp sources: rows of 16 bytes,
+// 8-row core matrices `sbo` bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;  // leading offset (unused: one 16-byte column)
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100; layout 0 = no swizzle
+    return d;
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: E4M3 A and B,
+// fp32 accumulator, UE8M0 scales; sf_id picks the byte of the scale words.
+__host__ __device__ constexpr uint32_t instr_desc_mxf8(int M, int N, bool a_mn_major, bool b_mn_major, int sf_id) {
+    return (static_cast<uint32_t>(sf_id & 3) << 4)      // B scale byte
+           | ((a_mn_major ? 1u : 0u) << 15)              // A major (formats 0 = E4M3)
+           | ((b_mn_major ? 1u : 0u) << 16)              // B major
+           | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
+           | (1u << 23)                                  // scale format: UE8M0
+           | (static_cast<uint32_t>(M >> 4) << 24)       // M / 16
+           | (static_cast<uint32_t>(sf_id & 3) << 29);   // A scale byte
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, dense.

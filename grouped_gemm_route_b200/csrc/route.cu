@@ -257,31 +257,44 @@ __global__ void __launch_bounds__(kBwdThreads) route_bwd_kernel(int T, int E, in
 }
 
 // Backward only: copies of x and grad_out in the expert-sorted layout (row pos
-// = token of perm[pos]; padding rows are zero), one warp per row.
+// = token of perm[pos]; padding rows are zero).  Flat over (row, 16-byte
+// piece), four independent pieces per thread per step.
 __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restrict__ perm,
                                                         const int32_t *__restrict__ group_start, int E, int k,
                                                         int TK, int d, const __nv_bfloat16 *__restrict__ x,
                                                         const __nv_bfloat16 *__restrict__ g,
                                                         __nv_bfloat16 *__restrict__ xs, __nv_bfloat16 *__restrict__ gs) {
-    const int rows = group_start[E];
-    const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (blockDim.x / 32);
     const int n16 = d / 8;  // 16-byte pieces per row
+    const int total = group_start[E] * n16;
+    const int stride = gridDim.x * blockDim.x;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); row < rows; row += warps) {
-        const int p = perm[row];
-        const bool valid = p >= 0 && p < TK;
-        const size_t src = static_cast<size_t>(valid ? p / k : 0) * d;
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + src);
-        const uint4 *gr = reinterpret_cast<const uint4 *>(g + src);
-        uint4 *xo = reinterpret_cast<uint4 *>(xs + static_cast<size_t>(row) * d);
-        uint4 *go = reinterpret_cast<uint4 *>(gs + static_cast<size_t>(row) * d);
-#pragma unroll 4
-        for (int c = lane; c < n16; c += 32) {
-            const uint4 xv = valid ? __ldg(xr + c) : zero;
-            const uint4 gv = valid ? __ldg(gr + c) : zero;
-            xo[c] = xv;
-            go[c] = gv;
+    const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
+    const uint4 *g4 = reinterpret_cast<const uint4 *>(g);
+    uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
+    uint4 *gs4 = reinterpret_cast<uint4 *>(gs);
+    for (int base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += 4 * stride) {
+        uint4 xv[4], gv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * stride;
+            xv[u] = gv[u] = zero;
+            if (i < total) {
+                const int row = i / n16, piece = i - row * n16;
+                const int p = __ldg(perm + row);
+                if (p >= 0 && p < TK) {
+                    const size_t src = static_cast<size_t>(p / k) * n16 + piece;
+                    xv[u] = __ldg(x4 + src);
+                    gv[u] = __ldg(g4 + src);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * stride;
+            if (i < total) {
+                xs4[i] = xv[u];
+                gs4[i] = gv[u];
+            }
         }
     }
 }
@@ -291,7 +304,7 @@ __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restric
 cudaError_t launch_sort_rows(const int32_t *perm, const int32_t *group_start, int E, int k, int T, int d,
                              const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs, __nv_bfloat16 *gs,
                              int sms, cudaStream_t s) {
-    sort_rows_kernel<<<sms * 8, 256, 0, s>>>(perm, group_start, E, k, T * k, d, x, g, xs, gs);
+    sort_rows_kernel<<<sms * 8, 256, 0, s>>>(perm, group_start, E, k, T * k, d, x, g, xs, gs);  // 8 x 256 threads per SM
     return cudaGetLastError();
 }
 

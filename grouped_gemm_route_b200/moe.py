@@ -219,11 +219,12 @@ class MoELayer:
     I: int
     device: str = "cuda"
     max_sms: int = 0
+    dtype: int = MOE_BF16  # MOE_BF16 or MOE_MXFP8 (GEMM operand precision)
 
     def __post_init__(self):
         if not torch.cuda.is_available():
             raise RuntimeError("the fused MoE layer needs a CUDA device (sm_100)")
-        self.shape = make_shape(self.T, self.d, self.E, self.k, self.I, MOE_BF16, self.max_sms)
+        self.shape = make_shape(self.T, self.d, self.E, self.k, self.I, self.dtype, self.max_sms)
         self.saved = alloc_saved(self.shape, self.device)
         self.ws = alloc_workspace(self.shape, self.device)
         dev = self.device

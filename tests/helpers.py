@@ -8,8 +8,10 @@ from grouped_gemm_route_b200 import inputs as IN
 from grouped_gemm_route_b200 import moe as M
 from oracle import moe_oracle as O
 
-# Normwise relative tolerance for bf16 GEMM operands (fp32 accumulation).
+# Normwise relative tolerances (fp32 accumulation): bf16 GEMM operands, and
+# MXFP8 operands checked against the oracle that applies the same quantisation.
 TOL_BF16 = 1e-2
+TOL_MXFP8 = 3e-2
 
 
 def normwise(gpu, ref) -> float:
@@ -26,12 +28,12 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def run_layer(inp: dict, T, d, E, k, I, backward=True, layer=None):
+def run_layer(inp: dict, T, d, E, k, I, backward=True, layer=None, dtype=M.MOE_BF16):
     """Run fwd (+bwd) on the GPU; returns the layer and host copies of everything."""
     dev = "cuda"
     x, lg, wgu, wd = (inp[n].to(dev) for n in ("x", "logits", "wgu", "wd"))
     if layer is None:
-        layer = M.MoELayer(T, d, E, k, I, device=dev)
+        layer = M.MoELayer(T, d, E, k, I, device=dev, dtype=dtype)
     layer.forward(x, lg, wgu, wd)
     res = dict(out=layer.out.clone())
     if backward:
@@ -85,5 +87,6 @@ def make(cfg_or_sizes, seed=0, **over):
     else:
         cfg = dict(cfg_or_sizes)
     cfg.update(over)
+    cfg.pop("dtype", None)
     inp = IN.make_inputs(seed=seed, **cfg)
     return cfg, inp

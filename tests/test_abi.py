@@ -52,7 +52,7 @@ def test_sizes_for_the_30b_shape(lib):
     (16, 256, 8, 2, 96, 0, M.MOE_ERR_SHAPE),
     (16, 256, 1024, 2, 128, 0, M.MOE_ERR_SHAPE),
     (16, 256, 128, 65, 128, 0, M.MOE_ERR_SHAPE),
-    (16, 256, 8, 2, 128, 1, M.MOE_ERR_UNSUPPORTED),
+    (16, 256, 8, 2, 128, 2, M.MOE_ERR_ARG),
     (16, 256, 8, 2, 128, 7, M.MOE_ERR_ARG),
 ])
 def test_invalid_shapes_are_rejected(lib, T, d, E, k, I, dtype, code):
@@ -60,6 +60,14 @@ def test_invalid_shapes_are_rejected(lib, T, d, E, k, I, dtype, code):
     f = ctypes.c_size_t()
     assert lib.moe_workspace_size(ctypes.byref(sh), ctypes.byref(f), None) == code
     assert lib.moe_fwd(ctypes.byref(sh), None, None, None, None, None, None, None, 0, None) == code
+
+
+def test_mxfp8_sizes(lib):
+    sh = M.make_shape(16384, 2048, 128, 8, 768, M.MOE_MXFP8)
+    f_mx, b_mx = M.workspace_size(sh)
+    f_bf, b_bf = M.workspace_size(M.make_shape(16384, 2048, 128, 8, 768))
+    assert f_mx > f_bf and b_mx > b_bf  # room for E4M3 codes and scales
+    assert M.saved_sizes(sh) == M.saved_sizes(M.make_shape(16384, 2048, 128, 8, 768))
 
 
 def test_null_and_misaligned_pointers_are_rejected_before_launch(lib):
@@ -83,4 +91,5 @@ def test_error_strings_and_kernel_names(lib):
         assert M.error_string(code)
     assert M.error_string(-99) == "unknown error code"
     names = M.kernel_names()
-    assert names[0] == "route_topk" and "gemm_gateup_fwd" in names and names[-1] == "route_bwd"
+    assert names[0] == "route_topk" and "gemm_gateup_fwd" in names
+    assert {"route_bwd", "sort_rows", "mx_quant"} <= set(names)
