@@ -504,3 +504,97 @@ def backward_mx(x, logits, wgu, wd, k, gout, fwd):
     dlogits = np.zeros((T, E))
     np.put_along_axis(dlogits, idx.astype(np.int64), dl_slots, axis=1)
     return dict(dx=dx, dwgu=dwgu, dwd=dwd, dscore=dscore, dlogits=dlogits)
+
+
+# ----------------------------------------------------------------------------
+# sampled MXFP8 variants (same quantisation as forward_mx / backward_mx)
+# ----------------------------------------------------------------------------
+class _MxWeights:
+    """Per-expert quantised weights, computed on first use."""
+
+    def __init__(self, wgu, wd):
+        self.wgu, self.wd, self.cache = wgu, wd, {}
+
+    def get(self, e):
+        if e not in self.cache:
+            wgu_e, wd_e = _f64(self.wgu[e]), _f64(self.wd[e])
+            self.cache[e] = dict(gu_d=mx_qdq_blocks(wgu_e, axis=1), d_i=mx_qdq_blocks(wd_e, axis=1),
+                                 d_d=mx_qdq_blocks(wd_e, axis=0), gu_2i=mx_qdq_blocks(wgu_e, axis=0))
+        return self.cache[e]
+
+
+def forward_tokens_mx(x, logits, wgu, wd, k, tokens, weights=None):
+    """out rows of forward_mx for the listed tokens only."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    idx, w = route(np.asarray(logits)[tokens], k)
+    W = weights or _MxWeights(wgu, wd)
+    xq = mx_qdq_blocks(_f64(np.asarray(x)[tokens]), axis=1)
+    I = np.asarray(wd).shape[2]
+    out = np.zeros((tokens.size, xq.shape[1]))
+    for r in range(tokens.size):
+        for j in range(k):
+            q = W.get(int(idx[r, j]))
+            h = xq[r:r + 1] @ q["gu_d"].T
+            aw = w[r, j] * silu(h[:, :I]) * h[:, I:]
+            out[r] += (mx_qdq_blocks(aw, axis=1) @ q["d_i"].T)[0]
+    return dict(out=out, idx=idx, w=w)
+
+
+def backward_tokens_mx(x, logits, wgu, wd, k, gout, tokens, weights=None):
+    """dx, dscore and dlogits rows of backward_mx for the listed tokens only."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    logits = np.asarray(logits)
+    E = logits.shape[1]
+    idx, w = route(logits[tokens], k)
+    W = weights or _MxWeights(wgu, wd)
+    I = np.asarray(wd).shape[2]
+    xq = mx_qdq_blocks(_f64(np.asarray(x)[tokens]), axis=1)
+    gq = mx_qdq_blocks(_f64(np.asarray(gout)[tokens]), axis=1)
+    dx = np.zeros_like(xq)
+    dscore = np.zeros((tokens.size, k))
+    for r in range(tokens.size):
+        for j in range(k):
+            q = W.get(int(idx[r, j]))
+            h = xq[r:r + 1] @ q["gu_d"].T
+            g, u = h[:, :I], h[:, I:]
+            G = gq[r:r + 1] @ q["d_d"]
+            dscore[r, j] = np.sum(G * silu(g) * u)
+            da = w[r, j] * G
+            dh = np.concatenate([da * u * silu_grad(g), da * silu(g)], axis=1)
+            dx[r] += (mx_qdq_blocks(dh, axis=1) @ q["gu_2i"])[0]
+    dl_slots = routing_backward(w, dscore)
+    dlogits = np.zeros((tokens.size, E))
+    np.put_along_axis(dlogits, idx.astype(np.int64), dl_slots, axis=1)
+    return dict(dx=dx, dscore=dscore, dlogits=dlogits, idx=idx, w=w)
+
+
+def backward_experts_mx(x, logits, wgu, wd, k, gout, experts, weights=None):
+    """dW_gate_up[e] and dW_down[e] of backward_mx for the listed experts only."""
+    logits = np.asarray(logits)
+    E = logits.shape[1]
+    idx, w = route(logits, k)
+    counts, offsets, perm, inv = dispatch(idx, E)
+    wf = w.reshape(-1)
+    W = weights or _MxWeights(wgu, wd)
+    I = np.asarray(wd).shape[2]
+    res = {}
+    for e in experts:
+        e = int(e)
+        pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
+        if pairs.size == 0:
+            res[e] = (np.zeros(np.asarray(wgu[e]).shape), np.zeros(np.asarray(wd[e]).shape))
+            continue
+        q = W.get(e)
+        t = pairs // k
+        xr = _f64(np.asarray(x)[t])
+        gr = _f64(np.asarray(gout)[t])
+        h = mx_qdq_blocks(xr, axis=1) @ q["gu_d"].T
+        g, u = h[:, :I], h[:, I:]
+        aw = wf[pairs][:, None] * silu(g) * u
+        G = mx_qdq_blocks(gr, axis=1) @ q["d_d"]
+        da = wf[pairs][:, None] * G
+        dh = np.concatenate([da * u * silu_grad(g), da * silu(g)], axis=1)
+        dwd_e = mx_qdq_blocks(gr, axis=0).T @ mx_qdq_blocks(aw, axis=0)
+        dwgu_e = mx_qdq_blocks(dh, axis=0).T @ mx_qdq_blocks(xr, axis=0)
+        res[e] = (dwgu_e, dwd_e)
+    return res

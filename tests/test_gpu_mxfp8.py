@@ -57,3 +57,32 @@ def test_mxfp8_empty_expert():
     inp["logits"][:, 4] = -100.0
     errs = mx_check(cfg, inp)
     assert np.isfinite(list(errs.values())).all()
+
+
+def test_qwen3_30b_mxfp8_sampled():
+    """The MXFP8 30B workload at full size: routing bit-exact over all tokens;
+    out / dx / dscore / dlogits on sampled tokens and dW on sampled experts."""
+    cfg, inp = make("qwen3_30b_a3b_mxfp8", seed=0)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    layer, res = run_layer(inp, T, d, E, k, I, dtype=M.MOE_MXFP8)
+    assert res["status"] == 0
+    logits = inp["logits"].numpy()
+    idx_ref, _ = check_routing(res["saved"], logits, k)
+    rng = np.random.default_rng(1)
+    toks = np.sort(rng.choice(T, size=24, replace=False))
+    x, gout = inp["x"].float().numpy(), inp["gout"].float().numpy()
+    wgu, wd = inp["wgu"].float().numpy(), inp["wd"].float().numpy()
+    W = O._MxWeights(wgu, wd)
+    ft = O.forward_tokens_mx(x, logits, wgu, wd, k, toks, weights=W)
+    errs = dict(out=normwise(f64(res["out"])[toks], ft["out"]))
+    bt = O.backward_tokens_mx(x, logits, wgu, wd, k, gout, toks, weights=W)
+    for n in ("dx", "dscore", "dlogits"):
+        errs[n] = normwise(f64(res[n])[toks], bt[n])
+    counts = np.bincount(idx_ref.reshape(-1), minlength=E)
+    experts = [int(np.argmin(np.abs(counts - np.median(counts))))]
+    be = O.backward_experts_mx(x, logits, wgu, wd, k, gout, experts, weights=W)
+    for e in experts:
+        errs[f"dwgu[{e}]"] = normwise(f64(res["dwgu"][e]), be[e][0])
+        errs[f"dwd[{e}]"] = normwise(f64(res["dwd"][e]), be[e][1])
+    bad = {n: v for n, v in errs.items() if not v <= TOL_MXFP8}
+    assert not bad, f"normwise errors above {TOL_MXFP8}: {bad} (all: {errs})"

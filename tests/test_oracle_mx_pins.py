@@ -130,3 +130,25 @@ def test_planted_mistake_scale_off_by_one(monkeypatch):
     monkeypatch.setattr(O, "mx_scale_exponent", lambda a: real(a) - 1)  # would saturate block maxima
     with pytest.raises(AssertionError):
         test_scale_exponent_bruteforce()
+
+
+def test_sampled_mx_variants_agree_with_full():
+    rng = np.random.default_rng(6)
+    T, d, E, k, I = 48, 64, 5, 3, 32
+    x = rng.standard_normal((T, d))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    wgu = rng.standard_normal((E, 2 * I, d)) * 0.2
+    wd = rng.standard_normal((E, d, I)) * 0.2
+    gout = rng.standard_normal((T, d))
+    f = O.forward_mx(x, logits, wgu, wd, k)
+    b = O.backward_mx(x, logits, wgu, wd, k, gout, f)
+    toks = [0, 5, 47]
+    ft = O.forward_tokens_mx(x, logits, wgu, wd, k, toks)
+    assert np.allclose(ft["out"], f["out"][toks], rtol=1e-12, atol=1e-12)
+    bt = O.backward_tokens_mx(x, logits, wgu, wd, k, gout, toks)
+    for key in ("dx", "dscore", "dlogits"):
+        assert np.allclose(bt[key], b[key][toks], rtol=1e-11, atol=1e-12), key
+    be = O.backward_experts_mx(x, logits, wgu, wd, k, gout, [0, 3])
+    for e in (0, 3):
+        assert np.allclose(be[e][0], b["dwgu"][e], rtol=1e-11, atol=1e-12)
+        assert np.allclose(be[e][1], b["dwd"][e], rtol=1e-11, atol=1e-12)
