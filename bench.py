@@ -65,6 +65,26 @@ def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(ms, pg, device):
+    """The slowest rank's time (every rank calls this, in the same order)."""
+    if pg is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step_per_rank, world, ms_per_step):
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return flops_per_step_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
+def l2_note(cfg):
+    wbytes = cfg["E"] * 3 * cfg["d"] * cfg["I"] * 2
+    return f"inputs larger than L2 (expert weights {wbytes / 1e9:.2f} GB), no flush"
+
+
 def workload_config(name, cfg, extra=None):
     c = {"workload": name, "T": cfg["T"], "d": cfg["d"], "E": cfg["E"], "top_k": cfg["k"], "I": cfg["I"]}
     if "zipf_s" in cfg:
@@ -286,13 +306,10 @@ def main():
     elapsed_ms = t_start.elapsed_time(t_end)
     if layer.status(stream) != 0:
         raise SystemExit("device status error in the timed region")
-    if pg is not None:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, pg, dev)
     ms_per_step = elapsed_ms / args.steps
     flops_step = IN.flops_fwd(**cfg) + IN.flops_bwd(**cfg)
-    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(flops_step, world, ms_per_step)
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
@@ -389,14 +406,10 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if pg is not None:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
         bi = sum(t.numel() * t.element_size() for t in (hx, hlg, hg))
         bo = sum(t.numel() * t.element_size() for t in (hout[0], hdx[0], hds[0]))
-        e2e = {"value": flops_step * world / (e_ms / args.e2e_steps * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_tflops(flops_step, world, e_ms / args.e2e_steps), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": args.e2e_steps,
                "overlap": "copies of step i+1 / i-1 overlap compute of step i (two layer buffers)"}
         del layers
@@ -415,9 +428,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "mxfp8 (e4m3, ue8m0/32)" if mx else "bf16", "data": "synthetic",
-        "config": workload_config(args.workload, cfg, {"parallelism": f"replicas{world}",
-                                                       "l2": "inputs larger than L2 (expert weights 1.15 GB at "
-                                                             "the 30B shape), no flush"}),
+        "config": workload_config(args.workload, cfg, {"parallelism": f"replicas{world}", "l2": l2_note(cfg)}),
         "frac_of_peak": {"step": value / world / peak, "gemm_only": (flops_step / (gemm_ms * 1e-3) / 1e12) / peak
                               if gemm_ms else None, "peak": peak, "peak_source": roofline["peak_source"]},
         "roofline": roofline, "routing": routing, "kernels": breakdown, "gpu_launches": launches,

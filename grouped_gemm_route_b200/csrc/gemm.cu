@@ -40,6 +40,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "moe_internal.h"
 #include "mx.cuh"
 #include "ptx.cuh"
@@ -56,7 +58,8 @@ constexpr int kChunkBytes = 64 * kTileK * 2;  // 8 KB: one 64-wide MN chunk of a
 constexpr uint32_t kSbo = 1024;               // 8 rows x 128 B swizzle atom
 constexpr uint32_t kMnLbo = kChunkBytes;      // MN-major: distance between 64-wide chunks
 constexpr int kXposeBytes = 32 * 64;          // per epilogue warp: 32 rows x 64 bytes
-constexpr int kTailCap = 2048;                // finished (token, column tile) pairs a CTA defers to its tail
+constexpr int kTailCap = 4096;                // finished (token, column tile) pairs a CTA queues
+constexpr int kEpiWarps = 4;
 
 // Pipeline geometry.  A stage holds one K block of both operands: 128-byte
 // operand rows, i.e. 64 bf16 or 128 E4M3 elements.  MXFP8 stages also carry
@@ -71,10 +74,14 @@ struct Cfg {
     static constexpr int kSfBytes = MX ? 2 * kMxAtomBytes : 0;     // scale atoms per stage
     static constexpr int kSfOffset = kStages * kStageBytes;
     static constexpr int kBarOffset = kSfOffset + kStages * kSfBytes;  // mbarriers, TMEM slot, abort flag
-    static constexpr int kOrderOffset = kBarOffset + 512;         // wgrad expert order
-    static constexpr int kXposeOffset = kOrderOffset + 2 * kMaxExperts * 4;   // 4 x 2 KB epilogue transposes
-    static constexpr int kTailOffset = kXposeOffset + 4 * kXposeBytes;        // combine: finished tokens
-    static constexpr int kSmemBytes = kTailOffset + 4 * (kTailCap + 4) + 1024;  // + 1 KB alignment slack
+    // one region, used by the wgrads for their expert order and by the
+    // combine modes for their queue of finished tokens
+    static constexpr int kOrderOffset = kBarOffset + 512;
+    static constexpr int kTailOffset = kOrderOffset;
+    static constexpr int kUnionBytes = 4 * (kTailCap + 4) > 8 * kMaxExperts ? 4 * (kTailCap + 4) : 8 * kMaxExperts;
+    static constexpr int kXposeOffset = kOrderOffset + kUnionBytes;            // 4 x 2 KB epilogue transposes
+    static constexpr int kSmemBytes = kXposeOffset + 4 * kXposeBytes + 1024;  // + 1 KB alignment slack
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = MX ? 512 : 2 * BN;
     static constexpr uint32_t kSfaCol = 2 * BN;                    // MXFP8 scale columns after the accumulators
     static constexpr uint32_t kSfbCol = 2 * BN + 8;
@@ -486,11 +493,17 @@ __device__ __forceinline__ void release_accumulator(uint64_t *tempty_acc) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(tempty_acc);
 }
 
-// Per-CTA list of (token, column tile) pairs whose last slot this CTA wrote;
-// their slot-ordered sums run after the CTA's last tile (see combine_tail).
+// Per-CTA queue of (token, column tile) pairs whose last slot this CTA wrote.
+// The epilogue warps reserve entries (count) and publish them (an entry holds
+// -1 until written).  Workers claim batches of four entries (claim): warps 6
+// and 7 from the start, so that the sums overlap the mainloop, and every other
+// warp once its own loop is over (combine_worker).  `done` counts epilogue
+// warps that have finished, after which no entry is added.
 struct TailList {
     int *items;  // token * n_tiles + column tile
     int *count;
+    int *done;
+    int *claim;
 };
 
 // gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up.
@@ -619,7 +632,7 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
     if (lane == 0) base = atomicAdd(tail.count, n_last);
     base = __shfl_sync(0xffffffffu, base, 0);
     const int my = __popc(mask & ((1u << lane) - 1u));
-    if (last && base + my < kTailCap) tail.items[base + my] = tok * a.n_tiles + t.nt;
+    if (last && base + my < kTailCap) reinterpret_cast<volatile int *>(tail.items)[base + my] = tok * a.n_tiles + t.nt;
     // no room left in the tail list: reduce those tokens now
     if (base + n_last > kTailCap) {
         while (mask != 0u) {
@@ -632,11 +645,13 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
     }
 }
 
-// Slot-ordered sums of up to four finished (token, column tile) items at once
-// (independent accumulators, so four tokens' slot loads are in flight).
+// Slot-ordered sums of up to four finished (token, column tile) items at once:
+// the loads of eight slots of all four tokens are issued before any is summed,
+// so 32 row pieces per lane are in flight.
 template <int BN>
 __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *items, int n) {
-    constexpr int kCols = BN / 32;
+    constexpr int kCols = BN / 32;  // columns per lane: 8 (16 bytes) or 4 (8 bytes)
+    using Piece = typename std::conditional<kCols == 8, uint4, uint2>::type;
     const int lane = threadIdx.x & 31;
     const __nv_bfloat16 *base[4];
     float acc[4][kCols];
@@ -648,28 +663,27 @@ __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *it
 #pragma unroll
         for (int i = 0; i < kCols; ++i) acc[u][i] = 0.f;
     }
-#pragma unroll 2
-    for (int j = 0; j < a.k; ++j) {  // slot order
+    for (int j0 = 0; j0 < a.k; j0 += 8) {  // slot order
+        Piece pc[8][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (u < n) {
-                const __nv_bfloat16 *sp = base[u] + static_cast<size_t>(j) * a.d;
-                if constexpr (kCols == 8) {
-                    const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(sp));
-                    acc[u][0] += bf16_lo(v.x);
-                    acc[u][1] += bf16_hi(v.x);
-                    acc[u][2] += bf16_lo(v.y);
-                    acc[u][3] += bf16_hi(v.y);
-                    acc[u][4] += bf16_lo(v.z);
-                    acc[u][5] += bf16_hi(v.z);
-                    acc[u][6] += bf16_lo(v.w);
-                    acc[u][7] += bf16_hi(v.w);
-                } else {
-                    const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(sp));
-                    acc[u][0] += bf16_lo(v.x);
-                    acc[u][1] += bf16_hi(v.x);
-                    acc[u][2] += bf16_lo(v.y);
-                    acc[u][3] += bf16_hi(v.y);
+        for (int jj = 0; jj < 8; ++jj) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (u < n && j0 + jj < a.k)
+                    pc[jj][u] = __ldcg(reinterpret_cast<const Piece *>(base[u] + static_cast<size_t>(j0 + jj) * a.d));
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (u < n && j0 + jj < a.k) {
+                    const uint32_t *w = reinterpret_cast<const uint32_t *>(&pc[jj][u]);
+#pragma unroll
+                    for (int q = 0; q < kCols / 2; ++q) {
+                        acc[u][2 * q] += bf16_lo(w[q]);
+                        acc[u][2 * q + 1] += bf16_hi(w[q]);
+                    }
                 }
             }
         }
@@ -693,12 +707,58 @@ __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *it
     }
 }
 
-// after the CTA's last tile: slot-ordered sums of its queued tokens, all warps
+// A combine worker (one warp): claims batches of four queue entries until the
+// queue is drained (the epilogue warps are done and every reserved entry has
+// been claimed) and sums them.  Every wait is bounded; progress restarts the
+// clock.
 template <int BN>
-__device__ __forceinline__ void combine_tail(const GemmArgs &a, const TailList &tail) {
-    const int n = min(*tail.count, kTailCap);
-    const int warp = threadIdx.x >> 5;
-    for (int i = warp * 4; i < n; i += (kThreads / 32) * 4) combine_tokens4<BN>(a, tail.items + i, min(4, n - i));
+__device__ void combine_worker(const GemmArgs &a, const TailList &tail, volatile int *abort_flag) {
+    const int lane = threadIdx.x & 31;
+    volatile int *vcount = tail.count, *vdone = tail.done, *vitems = tail.items;
+    uint64_t t0 = global_timer_ns();
+    for (;;) {
+        // lane 0 claims a batch and decides how many of its entries exist (0:
+        // queue drained, or the wait gave up)
+        int n = 0, lo = 0;
+        if (lane == 0) {
+            lo = atomicAdd(tail.claim, 4);
+            bool fail = false;
+            while (lo < kTailCap) {
+                if (*vcount >= lo + 4) {
+                    n = 4;
+                    break;
+                }
+                if (*vdone == kEpiWarps) {
+                    __threadfence_block();
+                    n = max(0, min(*vcount, kTailCap) - lo);
+                    break;
+                }
+                if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) {
+                    fail = true;
+                    break;
+                }
+                __nanosleep(64);
+            }
+            for (int u = 0; u < n && !fail; ++u) {  // reserved entries are published shortly after
+                while (vitems[lo + u] < 0) {
+                    if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) {
+                        fail = true;
+                        break;
+                    }
+                }
+            }
+            if (fail) {
+                if (!*abort_flag) raise_abort(abort_flag, a.status);
+                n = 0;
+            }
+            __threadfence_block();
+        }
+        n = __shfl_sync(0xffffffffu, n, 0);
+        lo = __shfl_sync(0xffffffffu, lo, 0);
+        if (n <= 0) return;
+        combine_tokens4<BN>(a, tail.items + lo, n);
+        t0 = global_timer_ns();
+    }
 }
 
 // down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh.
@@ -835,11 +895,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const TailList tail{reinterpret_cast<int *>(smem + C::kTailOffset),
-                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap};
+                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap,
+                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap + 1,
+                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap + 2};
+    constexpr bool kCombine = MODE == kDownFwd || MODE == kGateUpDgrad;
     int *s_count = reinterpret_cast<int *>(smem + C::kOrderOffset);
     int *order = s_count + kMaxExperts;
 
     const int warp = threadIdx.x >> 5;
+    if constexpr (kCombine) {
+        for (int i = threadIdx.x; i < kTailCap; i += kThreads) tail.items[i] = -1;
+    }
     if constexpr (!TR::kMTiled) {  // busiest expert first: rank by padded row count, ties to lower index
         for (int e = threadIdx.x; e < args.E; e += kThreads)
             s_count[e] = __ldg(args.group_start + e + 1) - __ldg(args.group_start + e);
@@ -865,7 +931,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        *tail.count = 0;
+        if constexpr (kCombine) {
+            *tail.count = 0;
+            *tail.done = 0;
+            *tail.claim = 0;
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -886,17 +956,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kGatherWarp0) {
         epilogue_loop<MODE, BN, MX>(args, tfull, tempty, tmem_base, order,
                                 smem + C::kXposeOffset + (warp - 2) * kXposeBytes, tail, abort_flag);
+        if constexpr (kCombine) {  // this warp's queue entries are written: count it as done
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) {
+                __threadfence_block();
+                atomicAdd(tail.done, 1);
+            }
+        }
     } else if constexpr (TR::kGather) {
         gather_loop<MODE, BN, MX>(args, smem, full, empty, order, abort_flag);
     }
+    // combine modes: warps 6 and 7 from the start, the others after their loops
+    if constexpr (kCombine) combine_worker<BN>(args, tail, abort_flag);
 
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
-    if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
-        if (!*abort_flag) combine_tail<BN>(args, tail);
-    }
 }
 
 template <int MODE, int BN, bool MX>

@@ -36,19 +36,25 @@ __device__ __forceinline__ int mx_scale_exp(float amax) {
 // Byte offset of scale (row m, K block j) inside its 512-byte atom.
 __device__ __forceinline__ int mx_atom_byte(int m, int j) { return (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3); }
 
+// 2^-s as a float multiplier pair (f1 * f2), exact for every s in [-127, 127]:
+// 2^-127 is below the normal range, so it is applied as 2^-64 * 2^-63.  A
+// multiplication by an exact power of two is exact unless the product leaves
+// the normal range, where the E4M3 rounding is 0 or saturation either way.
+__device__ __forceinline__ float mx_pow2_neg(int s) { return __uint_as_float(static_cast<uint32_t>(127 - s) << 23); }
+
+// E4M3 code pair (lo = a, hi = b) of a * 2^-s and b * 2^-s (round to nearest
+// even, saturating at 448).
+__device__ __forceinline__ uint32_t mx_code2(float a, float b, float f1, float f2) {
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a * f1 * f2, b * f1 * f2), __NV_SATFINITE,
+                                                          __NV_E4M3));
+}
+
 // E4M3 codes of 32 values scaled by 2^-s, packed little-endian into 8 words.
 __device__ __forceinline__ void mx_encode32(const float (&v)[32], int s, uint32_t (&codes)[8]) {
+    const float f1 = mx_pow2_neg(s < 127 ? s : 64), f2 = s < 127 ? 1.f : mx_pow2_neg(63);
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const float y = ldexpf(v[4 * w + b], -s);
-            const uint32_t c = static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
-            word |= c << (8 * b);
-        }
-        codes[w] = word;
-    }
+    for (int w = 0; w < 8; ++w)
+        codes[w] = mx_code2(v[4 * w], v[4 * w + 1], f1, f2) | (mx_code2(v[4 * w + 2], v[4 * w + 3], f1, f2) << 16);
 }
 
 __device__ __forceinline__ float amax32(const float (&v)[32]) {

@@ -70,39 +70,58 @@ __global__ void mx_quant_rows_kernel(const __nv_bfloat16 *__restrict__ src, int6
 }
 
 // src [Kr, N] quantised along its rows (K = rows) per column, blocks of 32
-// rows; one thread per (32-row block, column pair).  Codes keep the [Kr, N]
-// layout (an MN-major GEMM operand); atoms are indexed (k / 128, n / 128) of a
-// [Kr/128][N/128] atom array.  Only the first rows_used rows when given.
-__global__ void mx_quant_cols_kernel(const __nv_bfloat16 *__restrict__ src, int64_t Kr, int N,
+// rows; one thread per (32-row block, 4 adjacent columns): 8-byte loads and
+// 4-byte code stores, so a warp moves 256 contiguous bytes of a row.  Codes
+// keep the [Kr, N] layout (an MN-major GEMM operand); atoms are indexed
+// (k / 128, n / 128) of a [Kr/128][N/128] atom array.  Only the first
+// rows_used rows when given.
+__global__ void __launch_bounds__(128) mx_quant_cols_kernel(const __nv_bfloat16 *__restrict__ src, int64_t Kr, int N,
                                      uint8_t *__restrict__ dst, uint8_t *__restrict__ sf,
                                      const int32_t *__restrict__ rows_used) {
     int64_t rows = Kr;
     if (rows_used != nullptr) rows = min(rows, static_cast<int64_t>(*rows_used));
-    const int npairs = N / 2;
-    const int64_t total = (rows / kMxBlock) * npairs;
+    const int nquads = N / 4;
+    const int64_t total = (rows / kMxBlock) * nquads;
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t kb = i / npairs;
-        const int n = static_cast<int>(i - kb * npairs) * 2;
-        float a[32], b[32];
-        const uint32_t *s2 = reinterpret_cast<const uint32_t *>(src + kb * kMxBlock * N + n);
+        const int64_t kb = i / nquads;
+        const int n = static_cast<int>(i - kb * nquads) * 4;
+        const uint2 *s4 = reinterpret_cast<const uint2 *>(src + kb * kMxBlock * N + n);
+        uint2 raw[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) raw[rr] = __ldg(s4 + static_cast<int64_t>(rr) * (N / 4));
+        float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
-            const uint32_t w = __ldg(s2 + static_cast<int64_t>(rr) * (N / 2));
-            a[rr] = __uint_as_float(w << 16);
-            b[rr] = __uint_as_float(w & 0xFFFF0000u);
+            m[0] = fmaxf(m[0], fabsf(__uint_as_float(raw[rr].x << 16)));
+            m[1] = fmaxf(m[1], fabsf(__uint_as_float(raw[rr].x & 0xFFFF0000u)));
+            m[2] = fmaxf(m[2], fabsf(__uint_as_float(raw[rr].y << 16)));
+            m[3] = fmaxf(m[3], fabsf(__uint_as_float(raw[rr].y & 0xFFFF0000u)));
         }
-        const int sa = mx_scale_exp(amax32(a)), sbx = mx_scale_exp(amax32(b));
+        int sc[4];
+        float f1[4], f2[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            sc[c] = mx_scale_exp(m[c]);
+            f1[c] = mx_pow2_neg(sc[c] < 127 ? sc[c] : 64);
+            f2[c] = sc[c] < 127 ? 1.f : mx_pow2_neg(63);
+        }
+        uint32_t *d32 = reinterpret_cast<uint32_t *>(dst + kb * kMxBlock * N + n);
 #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
-            const uint32_t ca = __nv_cvt_float_to_fp8(ldexpf(a[rr], -sa), __NV_SATFINITE, __NV_E4M3);
-            const uint32_t cb = __nv_cvt_float_to_fp8(ldexpf(b[rr], -sbx), __NV_SATFINITE, __NV_E4M3);
-            *reinterpret_cast<uint16_t *>(dst + (kb * kMxBlock + rr) * N + n) = static_cast<uint16_t>(ca | (cb << 8));
+            const float v0 = __uint_as_float(raw[rr].x << 16), v1 = __uint_as_float(raw[rr].x & 0xFFFF0000u);
+            const float v2 = __uint_as_float(raw[rr].y << 16), v3 = __uint_as_float(raw[rr].y & 0xFFFF0000u);
+            const uint32_t lo = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+                make_float2(v0 * f1[0] * f2[0], v1 * f1[1] * f2[1]), __NV_SATFINITE, __NV_E4M3));
+            const uint32_t hi = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+                make_float2(v2 * f1[2] * f2[2], v3 * f1[3] * f2[3]), __NV_SATFINITE, __NV_E4M3));
+            d32[static_cast<int64_t>(rr) * (N / 4)] = lo | (hi << 16);
         }
         const int64_t atom = (kb * kMxBlock / 128) * (N / 128) + n / 128;
         const int j = static_cast<int>(kb & 3);
-        sf[atom * kMxAtomBytes + mx_atom_byte(n & 127, j)] = static_cast<uint8_t>(sa + 127);
-        sf[atom * kMxAtomBytes + mx_atom_byte((n + 1) & 127, j)] = static_cast<uint8_t>(sbx + 127);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            sf[atom * kMxAtomBytes + mx_atom_byte((n + c) & 127, j)] = static_cast<uint8_t>(sc[c] + 127);
     }
 }
 
@@ -116,7 +135,7 @@ cudaError_t launch_mx_quant_rows(const __nv_bfloat16 *src, int64_t R, int K, uin
 
 cudaError_t launch_mx_quant_cols(const __nv_bfloat16 *src, int64_t Kr, int N, uint8_t *dst, uint8_t *sf,
                                  const int32_t *rows_used, int sms, cudaStream_t s) {
-    mx_quant_cols_kernel<<<sms * 8, 256, 0, s>>>(src, Kr, N, dst, sf, rows_used);
+    mx_quant_cols_kernel<<<sms * 24, 128, 0, s>>>(src, Kr, N, dst, sf, rows_used);
     return cudaGetLastError();
 }
 
