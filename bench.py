@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="skip sampling nvidia-smi during the timed region")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-routing-sweep", action="store_true",
+                    help="skip the routing-only timing over token counts")
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0 = auto)")
     ap.add_argument("--override", default="", help="comma list of size overrides, e.g. T=4096,E=32 "
                                                      "(smaller profiling cases; not a bench workload)")
@@ -83,6 +85,43 @@ def job_tflops(flops_per_step_per_rank, world, ms_per_step):
 def l2_note(cfg):
     wbytes = cfg["E"] * 3 * cfg["d"] * cfg["I"] * 2
     return f"inputs larger than L2 (expert weights {wbytes / 1e9:.2f} GB), no flush"
+
+
+def routing_sweep(M, IN, dev, stream, peak_gbs, E, k, Ts=(16384, 65536, 262144, 524288), reps=10):
+    """Routing alone (moe_route: top-k, histogram, scan, permutation) at growing
+    token counts, each call timed by itself with L2 flushed before it (a 256 MiB
+    write), so that the logits come from HBM.  The activation buffers that
+    routing does not touch are left out (alloc_saved_routing) and the hidden
+    sizes are small, so that the workspace stays small."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    for T in Ts:
+        sh = M.make_shape(T, 128, E, k, 128)
+        saved = M.alloc_saved_routing(sh, dev)
+        f, _ = M.workspace_size(sh)
+        ws = torch.empty(f, dtype=torch.uint8, device=dev)
+        g = torch.Generator(device="cpu").manual_seed(1000 + T)
+        logits = torch.randn(T, E, generator=g, dtype=torch.float32).to(dev)
+        for _ in range(3):
+            M.route(sh, logits, saved, ws, stream)
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            e0.record(stream)
+            M.route(sh, logits, saved, ws, stream)
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        if M.get_status(ws, stream) != 0:
+            raise SystemExit(f"device status {M.get_status(ws, stream)} in the routing sweep (T={T})")
+        us = statistics.median(times) * 1e3
+        nbytes = IN.routing_bytes(T, E, k)
+        out.append({"T": T, "us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
+                    "frac": nbytes / (us * 1e-6) / 1e9 / peak_gbs})
+        del saved, ws, logits
+    return out
 
 
 def workload_config(name, cfg, extra=None):
@@ -149,15 +188,26 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # oracle timing (CPU baseline and the reference arm)
 # ----------------------------------------------------------------------------
-def oracle_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+def oracle_threads(cfg):
+    """Threads the oracle step uses: the C++ oracle splits the experts over the
+    host's hardware threads; the numpy MXFP8 oracle uses the BLAS pool."""
+    if cfg.get("dtype") == "mxfp8":
+        try:
+            from threadpoolctl import threadpool_info
+            n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+            if n:
+                return int(max(n))
+        except Exception:
+            pass
+        return os.cpu_count() or 1
+    from oracle import cpp_oracle as C
+    return max(1, min(cfg["E"], C.hardware_threads()))
+
+
+def oracle_kind(cfg):
+    if cfg.get("dtype") == "mxfp8":
+        return "fp64 numpy MXFP8 oracle"
+    return "fp64 C++ oracle (experts split over std::threads; its backward recomputes h)"
 
 
 def oracle_sample(cfg, inp, n_tokens):
@@ -171,11 +221,19 @@ def oracle_sample(cfg, inp, n_tokens):
 
 
 def time_oracle_step(cfg, inp, wgu64, wd64, n_tokens):
-    from oracle import moe_oracle as O
     x, lg, gout = oracle_sample(cfg, inp, n_tokens)
+    k = cfg["k"]
+    if cfg.get("dtype") == "mxfp8":
+        from oracle import moe_oracle as O
+        t0 = time.perf_counter()
+        f = O.forward_mx(x, lg, wgu64, wd64, k)
+        O.backward_mx(x, lg, wgu64, wd64, k, gout, f)
+        return time.perf_counter() - t0
+    from oracle import cpp_oracle as C
+    nt = oracle_threads(cfg)
     t0 = time.perf_counter()
-    f = O.forward(x, lg, wgu64, wd64, cfg["k"])
-    O.backward(x, lg, wgu64, wd64, cfg["k"], gout, f)
+    C.forward(x, lg, wgu64, wd64, k, nthreads=nt, keep_intermediates=False)
+    C.backward(x, lg, wgu64, wd64, k, gout, nthreads=nt)
     return time.perf_counter() - t0
 
 
@@ -195,8 +253,8 @@ def cpu_baseline(cfg, inp, n_tokens=0, budget_s=15.0):
         dt = time_oracle_step(cfg, inp, wgu64, wd64, n)
     dims = {k: cfg[k] for k in ("d", "E", "k", "I")}
     flops = IN.flops_fwd(T=n, **dims) + IN.flops_bwd(T=n, **dims)
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle, forward+backward of the first {n} of {cfg['T']} tokens "
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle_threads(cfg), "kind": "oracle",
+            "sample": f"{oracle_kind(cfg)}, forward+backward of the first {n} of {cfg['T']} tokens "
                       f"(all experts' weights), {dt:.2f} s"}, n, dt
 
 
@@ -219,12 +277,12 @@ def run_reference(args, rank, world):
     dims = {k: cfg[k] for k in ("d", "E", "k", "I")}
     flops = (IN.flops_fwd(T=n, **dims) + IN.flops_bwd(T=n, **dims)) * args.steps
     value = flops / total / 1e12
-    sample = f"fp64 numpy oracle, forward+backward of the first {n} of {cfg['T']} tokens per step"
+    sample = f"{oracle_kind(cfg)}, forward+backward of the first {n} of {cfg['T']} tokens per step"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(args.workload, cfg, {"oracle_tokens_per_step": n}),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(cfg), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -335,7 +393,7 @@ def main():
             with open(tpath) as f:
                 tr = json.load(f)
             ent = tr.get(dom, {})
-            if ent.get("source_hash") == B.source_hash() and ent.get("workload") == args.workload:
+            if ent.get("source_hash") == B.source_hash(B.GEMM_SOURCES) and ent.get("workload") == args.workload:
                 traffic = ent.get("dram_bytes_per_launch")
         except Exception:
             traffic = None
@@ -343,11 +401,15 @@ def main():
                 "frac": achieved / peak, "traffic": traffic,
                 "peak_source": peak_note}
     gemm_ms = sum(per_kernel.get(n, (0.0, 0))[0] for n in gemm_flops) / args.steps
-    route_names = ("route_topk", "route_scan", "route_perm")
+    route_names = ("route_topk", "route_scan", "route_perm", "route_fused")
     route_ms = sum(per_kernel.get(n, (0.0, 0))[0] for n in route_names) / args.steps
     routing = {"bytes_per_step": IN.routing_bytes(T, E, k), "ms_per_step": route_ms,
                "achieved_gbs": IN.routing_bytes(T, E, k) / (route_ms * 1e-3) / 1e9 if route_ms else None,
                "peak_gbs": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))}
+    if not args.no_routing_sweep:
+        routing["sweep"] = routing_sweep(M, IN, dev, stream, routing["peak_gbs"], E, k)
+        routing["sweep_note"] = ("moe_route alone, E and top_k of this workload, one call per timing with L2 "
+                                 "flushed before it; median of 10")
     breakdown = {n: {"ms_per_step": v[0] / args.steps, "share": v[0] / total_kernel_ms,
                      "launches": v[1]} for n, v in per_kernel.items() if v[1]}
     launches = int(sum(v[1] for v in per_kernel.values()))

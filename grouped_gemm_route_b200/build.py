@@ -77,11 +77,18 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     return LIB
 
 
-def source_hash() -> str:
-    """sha256 over the library's sources (identifies which kernels a profile describes)."""
+# Files that define the grouped-GEMM kernels (a profile of those kernels stays
+# valid while these are unchanged).
+GEMM_SOURCES = ("gemm.cu", "ptx.cuh", "mx.cuh", "moe_internal.h")
+
+
+def source_hash(names=None) -> str:
+    """sha256 over the library's sources, or over the named csrc files only
+    (identifies which kernels a profile describes)."""
     import hashlib
     h = hashlib.sha256()
-    for p in sorted(_deps()):
+    paths = sorted(_deps()) if names is None else [os.path.join(CSRC, n) for n in sorted(names)]
+    for p in paths:
         if p == os.path.abspath(__file__):
             continue
         h.update(os.path.basename(p).encode())

@@ -261,7 +261,7 @@ struct Launch {
 const char *kKindNames[kNumKernelKinds] = {
     "route_topk",       "route_scan",       "route_perm",           "gemm_gateup_fwd",      "gemm_down_fwd_combine",
     "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd",
-    "sort_rows", "mx_quant"};
+    "sort_rows", "mx_quant", "route_fused"};
 
 struct Saved {
     int32_t *idx;
@@ -285,33 +285,23 @@ int grid_for(const moe_shape_t *s, const DeviceInfo &dev) {
     return g;
 }
 
-int run_route(const moe_shape_t *shape, const Plan &pl, const float *logits, moe_saved_t *saved, uint8_t *ws,
-              cudaStream_t st) {
+// Routing and dispatch in one cooperative launch.  The status word and the
+// grid-barrier counter (the 16 bytes at ws_status) are zeroed by the caller.
+int run_route(const moe_shape_t *shape, const Plan &pl, const DeviceInfo &dev, const float *logits,
+              moe_saved_t *saved, uint8_t *ws, cudaStream_t st) {
     int *status = reinterpret_cast<int *>(ws + pl.ws_status);
-    int32_t *chunk_counts = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_counts);
-    int32_t *chunk_base = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_base);
+    unsigned *barrier = reinterpret_cast<unsigned *>(ws + pl.ws_status + 8);
+    int32_t *blk_hist = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_counts);
+    int32_t *blk_base = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_base);
     int32_t *cnt = reinterpret_cast<int32_t *>(ws + pl.ws_cnt);
     (void)shape;
-    int rc;
-    {
-        Launch L(kKindRouteTopk, st);
-        rc = L.done(launch_route_topk(logits, static_cast<int>(pl.T), pl.E, pl.k, saved->topk_idx, saved->topk_w,
-                                      chunk_counts, cnt, pl.cnt_stride, st));
-        if (rc) return rc;
-    }
-    {
-        Launch L(kKindRouteScan, st);
-        rc = L.done(launch_route_scan(static_cast<int>(pl.T), pl.E, pl.n_chunks, chunk_counts, chunk_base,
-                                      saved->counts, saved->offsets, saved->group_start, saved->tile_expert,
-                                      saved->perm, pl.p_cap, status, st));
-        if (rc) return rc;
-    }
-    {
-        Launch L(kKindRoutePerm, st);
-        rc = L.done(launch_route_perm(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_idx, chunk_base, saved->perm,
-                                      saved->inv, pl.p_cap, status, st));
-    }
-    return rc;
+    const int grid = route_fused_grid(static_cast<int>(pl.T), pl.E, pl.k, dev.sms, pl.n_chunks);
+    if (grid < 1) return MOE_ERR_LAUNCH;
+    Launch L(kKindRouteFused, st);
+    return L.done(launch_route_fused(logits, static_cast<int>(pl.T), pl.E, pl.k, saved->topk_idx, saved->topk_w,
+                                     blk_hist, blk_base, saved->counts, saved->offsets, saved->group_start,
+                                     saved->tile_expert, saved->perm, saved->inv, cnt, pl.cnt_stride, pl.p_cap,
+                                     barrier, status, grid, st));
 }
 
 GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
@@ -504,8 +494,8 @@ int moe_route(const moe_shape_t *shape, const float *logits, moe_saved_t *saved,
     if ((rc = device_info(&dev))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
-    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
-    return run_route(shape, pl, logits, saved, w8, st);
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 16, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    return run_route(shape, pl, dev, logits, saved, w8, st);
 }
 
 int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const void *w_gate_up, const void *w_down,
@@ -529,8 +519,8 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
         !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
         return MOE_ERR_LAUNCH;
 
-    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
-    if ((rc = run_route(shape, pl, logits, saved, w8, st))) return rc;
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 16, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    if ((rc = run_route(shape, pl, dev, logits, saved, w8, st))) return rc;
     if (pl.mx) return fwd_mx(pl, dev, shape, x, w_gate_up, w_down, out, saved, w8, st);
     const int grid = grid_for(shape, dev);
 
@@ -591,7 +581,8 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     // b0: x and grad_out in the expert-sorted layout (operands of the K = tokens wgrads)
     {
         Launch L(kKindSortRows, st);
-        if ((rc = L.done(launch_sort_rows(saved->perm, saved->group_start, pl.E, pl.k, static_cast<int>(pl.T), pl.d,
+        if ((rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
+                                          static_cast<int>(pl.T), pl.d,
                                           static_cast<const __nv_bfloat16 *>(x),
                                           static_cast<const __nv_bfloat16 *>(grad_out), xs, gs, dev.sms, st))))
             return rc;

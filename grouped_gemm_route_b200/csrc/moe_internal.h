@@ -34,6 +34,7 @@ enum KernelKind : int {
     kKindRouteBwd,
     kKindSortRows,
     kKindMxQuant,
+    kKindRouteFused,
     kNumKernelKinds
 };
 
@@ -82,11 +83,19 @@ cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t 
 cudaError_t launch_route_scan(int T, int E, int n_chunks, const int32_t *chunk_counts, int32_t *chunk_base,
                               int32_t *counts, int32_t *offsets, int32_t *group_start, int32_t *tile_expert,
                               int32_t *perm, int64_t p_cap, int *status, cudaStream_t s);
+// Fused routing (one cooperative launch; see route.cu).  route_fused_grid
+// returns the grid (all blocks resident, at most n_chunks), 0 on failure.
+size_t route_fused_smem(int E, int k);
+int route_fused_grid(int T, int E, int k, int sms, int n_chunks);
+cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t *idx, float *w, int32_t *blk_hist,
+                               int32_t *blk_base, int32_t *counts, int32_t *offsets, int32_t *group_start,
+                               int32_t *tile_expert, int32_t *perm, int32_t *inv, int32_t *cnt, int cnt_per_token,
+                               int64_t p_cap, unsigned *barrier, int *status, int grid, cudaStream_t s);
 cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int32_t *chunk_base, int32_t *perm,
                               int32_t *inv, int64_t p_cap, int *status, cudaStream_t s);
-cudaError_t launch_sort_rows(const int32_t *perm, const int32_t *group_start, int E, int k, int T, int d,
-                             const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs, __nv_bfloat16 *gs,
-                             int sms, cudaStream_t s);
+cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
+                             int T, int d, const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs,
+                             __nv_bfloat16 *gs, int sms, cudaStream_t s);
 cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t *idx, const int32_t *inv,
                              const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s);
 

@@ -223,6 +223,283 @@ __global__ void route_perm_kernel(int T, int E, int k, const int32_t *__restrict
     if (bad) report_status(status, kStatusBadIndex);
 }
 
+// ---------------------------------------------------------------------------
+// Fused routing: the three steps above in one cooperative launch.  Block b of
+// G owns the contiguous tokens [T*b/G, T*(b+1)/G), and warp w of the block a
+// contiguous sub-range of those, so (block, warp, token, slot) order is token
+// order.  Phases, separated by grid barriers (every block resident: the launch
+// is cooperative; every wait is bounded):
+//   1  per token top-k, weights, combine counters; per-warp expert histograms;
+//      the block's histogram to blk_hist[b]
+//   2  block b scans expert e = b, b+G, ... over the G blocks: blk_base[.][e],
+//      counts[e]
+//   3  every block: padded exclusive scan of counts (group starts); block 0
+//      publishes it; each block writes the tile table and padding rows of its
+//      experts and the sorted position of each of its pairs, walking each
+//      warp's tokens in order with one lane per slot (a token's k experts are
+//      distinct, so the lanes never update the same counter).
+// ---------------------------------------------------------------------------
+constexpr int kFusedThreads = 512;
+constexpr int kFusedWarps = kFusedThreads / 32;
+static_assert(kFusedThreads >= kMaxExperts, "phase 3 scans one expert per thread");
+
+struct RouteFusedArgs {
+    const float *logits;
+    int T, E, k;
+    int32_t *idx;
+    float *w;
+    int32_t *blk_hist;  // [G, E]
+    int32_t *blk_base;  // [G, E]
+    int32_t *counts, *offsets, *group_start, *tile_expert, *perm, *inv;
+    int32_t *cnt;
+    int cnt_per_token;
+    int64_t p_cap;
+    unsigned *barrier;  // zero before the launch
+    int *status;
+};
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// All blocks of the grid arrive, then wait (bounded) until `target` arrivals
+// are counted.  Returns false for every thread of a block whose wait expired
+// (the status word then holds a timeout).
+__device__ bool grid_barrier(unsigned *ctr, unsigned target, int *status) {
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        const uint64_t t0 = global_timer_ns();
+        int ok = 1;
+        while (ld_acquire_gpu(ctr) < target) {
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                report_status(status, kStatusTimeout);
+                ok = 0;
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+// Exclusive scan of one int per thread over the block; returns the block total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int &excl, int *warp_sums) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    __syncthreads();  // warp_sums free from any earlier use
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int base = 0, total = 0;
+    for (int i = 0; i < kFusedWarps; ++i) {
+        const int ws = warp_sums[i];
+        if (i < warp) base += ws;
+        total += ws;
+    }
+    excl = base + incl - v;
+    return total;
+}
+
+// Top-k key of a logit: the high word orders fp32 values (-0 and +0 equal,
+// finite values assumed), the low word is ~expert so that among equal values
+// the lower expert index is larger.  0 is below every real key.
+__device__ __forceinline__ uint64_t topk_key(float v, int e) {
+    const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    const uint32_t hi = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (static_cast<uint64_t>(hi) << 32) | static_cast<uint32_t>(~e);
+}
+
+__device__ __forceinline__ float topk_value(uint32_t hi) {
+    return __uint_as_float((hi & 0x80000000u) ? (hi & 0x7FFFFFFFu) : ~hi);
+}
+
+template <int NV>
+__global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteFusedArgs a) {
+    extern __shared__ int smem_i[];
+    const int E = a.E, k = a.k, G = gridDim.x, b = blockIdx.x;
+    int *wcnt = smem_i;                          // [kFusedWarps][E] per-warp counts, then bases
+    int *gst = wcnt + kFusedWarps * E;           // [E + 1] padded group starts
+    int *warp_sums = gst + E + 1;                // [kFusedWarps]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = static_cast<int>(static_cast<int64_t>(a.T) * b / G);
+    const int t1 = static_cast<int>(static_cast<int64_t>(a.T) * (b + 1) / G);
+    const int nb = t1 - t0;
+    const int wt0 = t0 + nb * warp / kFusedWarps, wt1 = t0 + nb * (warp + 1) / kFusedWarps;
+    for (int i = threadIdx.x; i < kFusedWarps * E; i += kFusedThreads) wcnt[i] = 0;
+    __syncthreads();
+
+    // ---- phase 1: top-k of each token, kTokPar tokens at a time per warp ----
+    constexpr int kTokPar = NV <= 4 ? 2 : 1;
+    for (int t = wt0; t < wt1; t += kTokPar) {
+        uint64_t c[kTokPar][NV];  // this lane's (value, expert) keys, sorted descending
+        uint64_t sel[kTokPar][2];  // slots lane and lane + 32 after the rounds
+        uint32_t vmax[kTokPar];
+#pragma unroll
+        for (int u = 0; u < kTokPar; ++u) {
+            const bool live = t + u < wt1;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                const int e = lane + 32 * i;
+                c[u][i] = live && e < E ? topk_key(__ldg(a.logits + static_cast<size_t>(t + u) * E + e), e) : 0ull;
+            }
+#pragma unroll
+            for (int i = 1; i < NV; ++i)
+#pragma unroll
+                for (int q = i; q > 0; --q) {
+                    const uint64_t x0 = c[u][q - 1], x1 = c[u][q];
+                    const bool sw = x1 > x0;
+                    c[u][q - 1] = sw ? x1 : x0;
+                    c[u][q] = sw ? x0 : x1;
+                }
+            sel[u][0] = sel[u][1] = 0ull;
+        }
+        // round j: the warp's largest head key is slot j; its lane pops it
+        for (int j = 0; j < k; ++j) {
+#pragma unroll
+            for (int u = 0; u < kTokPar; ++u) {
+                const uint32_t hi = static_cast<uint32_t>(c[u][0] >> 32), lo = static_cast<uint32_t>(c[u][0]);
+                const uint32_t m_hi = __reduce_max_sync(0xffffffffu, hi);
+                const uint32_t m_lo = __reduce_max_sync(0xffffffffu, hi == m_hi ? lo : 0u);
+                if (j == 0) vmax[u] = m_hi;
+                if (hi == m_hi && lo == m_lo) {
+#pragma unroll
+                    for (int i = 0; i + 1 < NV; ++i) c[u][i] = c[u][i + 1];
+                    c[u][NV - 1] = 0ull;
+                }
+                const uint64_t key = (static_cast<uint64_t>(m_hi) << 32) | m_lo;
+                if (lane == (j & 31)) {
+                    if (j < 32)
+                        sel[u][0] = key;
+                    else
+                        sel[u][1] = key;
+                }
+            }
+        }
+        // weights: exp(l_j - l_max) over the chosen k, normalised by their sum
+        // (a fixed shuffle tree over the slots)
+#pragma unroll
+        for (int u = 0; u < kTokPar; ++u) {
+            const int tt = t + u;
+            const float m = topk_value(vmax[u]);
+            float p[2], sum = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int j = lane + 32 * h;
+                p[h] = j < k ? expf(topk_value(static_cast<uint32_t>(sel[u][h] >> 32)) - m) : 0.f;
+                sum += p[h];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (tt < wt1) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int j = lane + 32 * h;
+                    if (j < k) {
+                        const int e = static_cast<int>(~static_cast<uint32_t>(sel[u][h]));
+                        a.idx[static_cast<size_t>(tt) * k + j] = e;
+                        a.w[static_cast<size_t>(tt) * k + j] = p[h] / sum;
+                        wcnt[warp * E + e] += 1;  // the k experts of a token are distinct
+                    }
+                }
+                for (int cc = lane; cc < a.cnt_per_token; cc += 32)
+                    a.cnt[static_cast<size_t>(tt) * a.cnt_per_token + cc] = 0;
+            }
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kFusedThreads) {
+        int sum = 0;
+        for (int q = 0; q < kFusedWarps; ++q) sum += wcnt[q * E + e];
+        a.blk_hist[static_cast<size_t>(b) * E + e] = sum;
+    }
+    if (!grid_barrier(a.barrier, G, a.status)) return;
+
+    // ---- phase 2: per expert, exclusive scan over the blocks ----
+    for (int e = b; e < E; e += G) {
+        int carry = 0;
+        for (int c0 = 0; c0 < G; c0 += kFusedThreads) {
+            const int bb = c0 + threadIdx.x;
+            const int v = bb < G ? __ldcg(a.blk_hist + static_cast<size_t>(bb) * E + e) : 0;
+            int excl;
+            const int tot = block_exclusive_scan(v, excl, warp_sums);
+            if (bb < G) a.blk_base[static_cast<size_t>(bb) * E + e] = carry + excl;
+            carry += tot;
+        }
+        if (threadIdx.x == 0) a.counts[e] = carry;
+    }
+    if (!grid_barrier(a.barrier, 2u * G, a.status)) return;
+
+    // ---- phase 3: group starts, tile table, padding, positions ----
+    int c_excl = 0, p_excl = 0, c_tot = 0, p_tot = 0;
+    {
+        // E <= kMaxExperts = kFusedThreads: one expert per thread
+        const int e = threadIdx.x;
+        const int c = e < E ? __ldcg(a.counts + e) : 0;
+        const int padded = (c + kTileM - 1) / kTileM * kTileM;
+        c_tot = block_exclusive_scan(c, c_excl, warp_sums);
+        p_tot = block_exclusive_scan(padded, p_excl, warp_sums);
+        if (e < E) gst[e] = p_excl;
+        if (e == 0) gst[E] = p_tot;
+        if (b == 0 && e < E) {
+            a.group_start[e] = p_excl;
+            a.offsets[e] = c_excl;
+        }
+        if (b == 0 && e == 0) {
+            a.group_start[E] = p_tot;
+            a.offsets[E] = c_tot;
+            if (p_tot > a.p_cap) report_status(a.status, kStatusBadIndex);
+        }
+    }
+    __syncthreads();
+    if (gst[E] > a.p_cap) return;
+    for (int e = b; e < E; e += G) {
+        const int gs = gst[e], ge = gst[e + 1], c = __ldcg(a.counts + e);
+        for (int mt = gs / kTileM + threadIdx.x; mt < ge / kTileM; mt += kFusedThreads) a.tile_expert[mt] = e;
+        for (int q = gs + c + threadIdx.x; q < ge; q += kFusedThreads) a.perm[q] = -1;
+    }
+    // per-warp first position of each expert: group start + earlier blocks +
+    // earlier warps of this block
+    for (int e = threadIdx.x; e < E; e += kFusedThreads) {
+        int run = gst[e] + __ldcg(a.blk_base + static_cast<size_t>(b) * E + e);
+        for (int q = 0; q < kFusedWarps; ++q) {
+            const int c = wcnt[q * E + e];
+            wcnt[q * E + e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    bool bad = false;
+    for (int t = wt0; t < wt1; ++t) {
+        for (int j = lane; j < k; j += 32) {
+            const int p = t * k + j;
+            const int e = a.idx[p];  // written by this thread in phase 1
+            const int pos = wcnt[warp * E + e];
+            wcnt[warp * E + e] = pos + 1;
+            if (pos >= 0 && pos < gst[e + 1]) {
+                a.perm[pos] = p;
+                a.inv[p] = pos;
+            } else {
+                bad = true;
+            }
+        }
+        __syncwarp();
+    }
+    if (bad) report_status(a.status, kStatusBadIndex);
+}
+
 constexpr int kBwdThreads = 256;
 
 __global__ void __launch_bounds__(kBwdThreads) route_bwd_kernel(int T, int E, int k, const float *__restrict__ w,
@@ -257,54 +534,72 @@ __global__ void __launch_bounds__(kBwdThreads) route_bwd_kernel(int T, int E, in
 }
 
 // Backward only: copies of x and grad_out in the expert-sorted layout (row pos
-// = token of perm[pos]; padding rows are zero).  Flat over (row, 16-byte
-// piece), four independent pieces per thread per step.
-__global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restrict__ perm,
-                                                        const int32_t *__restrict__ group_start, int E, int k,
-                                                        int TK, int d, const __nv_bfloat16 *__restrict__ x,
+// holds the token of pair perm[pos]; padding rows are zero).  Walked in token
+// order: each 16-byte piece of a token's x and grad_out rows is read once and
+// stored to the sorted rows of the token's k pairs (inv), so the sources stream
+// from HBM once instead of once per pair.  A second loop zeroes the padding
+// rows at the end of each expert's group (fewer than kTileM per expert).
+__global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restrict__ inv,
+                                                        const int32_t *__restrict__ counts,
+                                                        const int32_t *__restrict__ group_start, int T, int E, int k,
+                                                        int d, const __nv_bfloat16 *__restrict__ x,
                                                         const __nv_bfloat16 *__restrict__ g,
                                                         __nv_bfloat16 *__restrict__ xs, __nv_bfloat16 *__restrict__ gs) {
     const int n16 = d / 8;  // 16-byte pieces per row
-    const int total = group_start[E] * n16;
-    const int stride = gridDim.x * blockDim.x;
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    const int rows_used = group_start[E];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
     const uint4 *g4 = reinterpret_cast<const uint4 *>(g);
     uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
     uint4 *gs4 = reinterpret_cast<uint4 *>(gs);
-    for (int base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += 4 * stride) {
-        uint4 xv[4], gv[4];
+    const int64_t total = static_cast<int64_t>(T) * n16;
+    for (int64_t i = tid; i < total; i += 2 * stride) {
+        uint4 xv[2], gv[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = base + u * stride;
-            xv[u] = gv[u] = zero;
-            if (i < total) {
-                const int row = i / n16, piece = i - row * n16;
-                const int p = __ldg(perm + row);
-                if (p >= 0 && p < TK) {
-                    const size_t src = static_cast<size_t>(p / k) * n16 + piece;
-                    xv[u] = __ldg(x4 + src);
-                    gv[u] = __ldg(g4 + src);
-                }
+        for (int u = 0; u < 2; ++u) {
+            const int64_t ii = i + u * stride;
+            if (ii < total) {
+                xv[u] = __ldg(x4 + ii);
+                gv[u] = __ldg(g4 + ii);
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = base + u * stride;
-            if (i < total) {
-                xs4[i] = xv[u];
-                gs4[i] = gv[u];
+        for (int u = 0; u < 2; ++u) {
+            const int64_t ii = i + u * stride;
+            if (ii < total) {
+                const int t = static_cast<int>(ii / n16), piece = static_cast<int>(ii - static_cast<int64_t>(t) * n16);
+                for (int j = 0; j < k; ++j) {
+                    const int pos = __ldg(inv + static_cast<int64_t>(t) * k + j);
+                    if (pos >= 0 && pos < rows_used) {
+                        xs4[static_cast<int64_t>(pos) * n16 + piece] = xv[u];
+                        gs4[static_cast<int64_t>(pos) * n16 + piece] = gv[u];
+                    }
+                }
             }
+        }
+    }
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    const int64_t per_expert = static_cast<int64_t>(kTileM - 1) * n16;
+    const int64_t pad_total = static_cast<int64_t>(E) * per_expert;
+    for (int64_t i = tid; i < pad_total; i += stride) {
+        const int e = static_cast<int>(i / per_expert);
+        const int64_t rem = i - e * per_expert;
+        const int r = static_cast<int>(rem / n16), piece = static_cast<int>(rem - static_cast<int64_t>(r) * n16);
+        const int row = __ldg(group_start + e) + __ldg(counts + e) + r;
+        if (row < __ldg(group_start + e + 1) && row < rows_used) {
+            xs4[static_cast<int64_t>(row) * n16 + piece] = zero;
+            gs4[static_cast<int64_t>(row) * n16 + piece] = zero;
         }
     }
 }
 
 }  // namespace
 
-cudaError_t launch_sort_rows(const int32_t *perm, const int32_t *group_start, int E, int k, int T, int d,
-                             const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs, __nv_bfloat16 *gs,
-                             int sms, cudaStream_t s) {
-    sort_rows_kernel<<<sms * 8, 256, 0, s>>>(perm, group_start, E, k, T * k, d, x, g, xs, gs);  // 8 x 256 threads per SM
+cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
+                             int T, int d, const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs,
+                             __nv_bfloat16 *gs, int sms, cudaStream_t s) {
+    sort_rows_kernel<<<sms * 8, 256, 0, s>>>(inv, counts, group_start, T, E, k, d, x, g, xs, gs);  // 8 x 256 threads per SM
     return cudaGetLastError();
 }
 
@@ -348,6 +643,50 @@ cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t 
     const int blocks = (T + per_block - 1) / per_block;
     route_bwd_kernel<<<blocks, kBwdThreads, 0, s>>>(T, E, k, w, idx, inv, dpart, dpart_stride, dscore, dlogits);
     return cudaGetLastError();
+}
+
+int route_fused_grid(int T, int E, int k, int sms, int n_chunks) {
+    const int nv = (E + 31) / 32;
+    const size_t smem = route_fused_smem(E, k);
+    int per_sm = 0;
+    cudaError_t e;
+    if (nv <= 1)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<1>, kFusedThreads, smem);
+    else if (nv <= 2)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<2>, kFusedThreads, smem);
+    else if (nv <= 4)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<4>, kFusedThreads, smem);
+    else if (nv <= 8)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<8>, kFusedThreads, smem);
+    else
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<16>, kFusedThreads, smem);
+    (void)T;
+    (void)k;
+    if (e != cudaSuccess || per_sm < 1) return 0;
+    const int g = per_sm * sms;
+    return g < n_chunks ? g : n_chunks;
+}
+
+size_t route_fused_smem(int E, int k) {
+    (void)k;
+    return (static_cast<size_t>(kFusedWarps) * E + E + 1 + kFusedWarps) * 4;
+}
+
+cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t *idx, float *w, int32_t *blk_hist,
+                               int32_t *blk_base, int32_t *counts, int32_t *offsets, int32_t *group_start,
+                               int32_t *tile_expert, int32_t *perm, int32_t *inv, int32_t *cnt, int cnt_per_token,
+                               int64_t p_cap, unsigned *barrier, int *status, int grid, cudaStream_t s) {
+    RouteFusedArgs a{logits, T, E, k, idx, w, blk_hist, blk_base, counts, offsets, group_start,
+                     tile_expert, perm, inv, cnt, cnt_per_token, p_cap, barrier, status};
+    void *params[] = {&a};
+    const size_t smem = route_fused_smem(E, k);
+    const int nv = (E + 31) / 32;
+    const void *fn = nv <= 1   ? reinterpret_cast<const void *>(route_fused_kernel<1>)
+                     : nv <= 2 ? reinterpret_cast<const void *>(route_fused_kernel<2>)
+                     : nv <= 4 ? reinterpret_cast<const void *>(route_fused_kernel<4>)
+                     : nv <= 8 ? reinterpret_cast<const void *>(route_fused_kernel<8>)
+                               : reinterpret_cast<const void *>(route_fused_kernel<16>);
+    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kFusedThreads), params, smem, s);
 }
 
 }  // namespace moe

@@ -204,6 +204,16 @@ def alloc_saved(shape: MoeShape, device) -> dict:
     return out
 
 
+def alloc_saved_routing(shape: MoeShape, device) -> dict:
+    """Saved buffers for moe_route alone: the routing fields at full size, and
+    16-byte placeholders for h and aw, which routing does not touch."""
+    sizes, p_cap = saved_sizes(shape)
+    T, E, k = shape.T, shape.E, shape.k
+    shapes = dict(topk_idx=(T, k), topk_w=(T, k), counts=(E,), offsets=(E + 1,), group_start=(E + 1,),
+                  tile_expert=(p_cap // 128,), perm=(p_cap,), inv=(T, k), h=(8,), aw=(8,))
+    return {name: torch.empty(shapes[name], dtype=_SAVED_DTYPES[name], device=device) for name in SAVED_FIELDS}
+
+
 def alloc_workspace(shape: MoeShape, device) -> torch.Tensor:
     f, b = workspace_size(shape)
     return torch.empty(max(f, b), dtype=torch.uint8, device=device)
