@@ -328,15 +328,15 @@ GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
 }
 
 
-// MXFP8 forward after routing: quantise x (per-row scale bytes, for the
-// gather), W_gate_up (atoms in the tile's gate/up row order) and W_down, then
-// the two block-scaled GEMMs.  The gate/up epilogue writes aw's codes and scales.
-int fwd_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,
-           const void *w_down, void *out, moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
+// MXFP8 gate/up GEMM after routing: quantise x (per-row scale bytes, for the
+// gather) and W_gate_up (atoms in the tile's gate/up row order), then the
+// block-scaled GEMM, whose epilogue writes h, aw and aw's codes and scales.
+int gateup_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,
+              moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
     int rc;
-    const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I, Ed = static_cast<int64_t>(pl.E) * pl.d;
+    const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I;
     uint8_t *x8 = w8 + pl.mx_x8, *xsf = w8 + pl.mx_xsf, *wgu8 = w8 + pl.mx_wgu8, *wgusf = w8 + pl.mx_wgusf;
-    uint8_t *wd8 = w8 + pl.mx_wd8, *wdsf = w8 + pl.mx_wdsf, *aw8 = w8 + pl.mx_aw8, *awsf = w8 + pl.mx_awsf;
+    uint8_t *aw8 = w8 + pl.mx_aw8, *awsf = w8 + pl.mx_awsf;
     {
         Launch L(kKindMxQuant, st);
         if ((rc = L.done(launch_mx_quant_rows(static_cast<const __nv_bfloat16 *>(x), pl.T, pl.d, x8, xsf,
@@ -349,17 +349,8 @@ int fwd_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, cons
                                               kMxSfGateUp, pl.I, nullptr, dev.sms, st))))
             return rc;
     }
-    {
-        Launch L(kKindMxQuant, st);
-        if ((rc = L.done(launch_mx_quant_rows(static_cast<const __nv_bfloat16 *>(w_down), Ed, pl.I, wd8, wdsf,
-                                              kMxSfAtoms, pl.I, nullptr, dev.sms, st))))
-            return rc;
-    }
-    CUtensorMap tm_wgu8, tm_aw8, tm_wd8;
-    if (!make_map8(&tm_wgu8, wgu8, EI2, pl.d, 64) || !make_map8(&tm_aw8, aw8, pl.p_cap, pl.I, 128) ||
-        !make_map8(&tm_wd8, wd8, Ed, pl.I, 128))
-        return MOE_ERR_LAUNCH;
-    const int grid = grid_for(shape, dev);
+    CUtensorMap tm_wgu8;
+    if (!make_map8(&tm_wgu8, wgu8, EI2, pl.d, 64)) return MOE_ERR_LAUNCH;
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.I / 64;
     a.num_k_blocks = pl.d / 128;
@@ -368,17 +359,49 @@ int fwd_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, cons
     a.sfb = wgusf;
     a.mx_codes = aw8;
     a.mx_sf = awsf;
+    Launch L(kKindGemmGateUpFwd, st);
+    return L.done(launch_gemm(kGateUpFwd, 128, true, a, tm_wgu8, tm_wgu8, grid_for(shape, dev), st));
+}
+
+// MXFP8 down GEMM + combine: quantise W_down along I, then the block-scaled
+// GEMM on aw's codes (written by the gate/up epilogue).
+int down_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *w_down, void *out,
+            moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
+    int rc;
+    const int64_t Ed = static_cast<int64_t>(pl.E) * pl.d;
+    uint8_t *wd8 = w8 + pl.mx_wd8, *wdsf = w8 + pl.mx_wdsf, *aw8 = w8 + pl.mx_aw8, *awsf = w8 + pl.mx_awsf;
     {
-        Launch L(kKindGemmGateUpFwd, st);
-        if ((rc = L.done(launch_gemm(kGateUpFwd, 128, true, a, tm_wgu8, tm_wgu8, grid, st)))) return rc;
+        Launch L(kKindMxQuant, st);
+        if ((rc = L.done(launch_mx_quant_rows(static_cast<const __nv_bfloat16 *>(w_down), Ed, pl.I, wd8, wdsf,
+                                              kMxSfAtoms, pl.I, nullptr, dev.sms, st))))
+            return rc;
     }
+    CUtensorMap tm_aw8, tm_wd8;
+    if (!make_map8(&tm_aw8, aw8, pl.p_cap, pl.I, 128) || !make_map8(&tm_wd8, wd8, Ed, pl.I, 128))
+        return MOE_ERR_LAUNCH;
+    GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.d / 128;
     a.num_k_blocks = pl.I / 128;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.sfa = awsf;
     a.sfb = wdsf;
     Launch L(kKindGemmDownFwd, st);
-    return L.done(launch_gemm(kDownFwd, 128, true, a, tm_aw8, tm_wd8, grid, st));
+    return L.done(launch_gemm(kDownFwd, 128, true, a, tm_aw8, tm_wd8, grid_for(shape, dev), st));
+}
+
+// The gate/up GEMM with its SwiGLU epilogue (h, aw into `saved`), for the
+// routing already in `saved`: bf16 or MXFP8 operands.
+int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,
+               moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
+    if (pl.mx) return gateup_mx(pl, dev, shape, x, w_gate_up, saved, w8, st);
+    CUtensorMap tm_wgu;
+    if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 128)) return MOE_ERR_LAUNCH;
+    GemmArgs a = base_args(pl, saved, w8);
+    a.n_tiles = pl.I / 128;
+    a.num_k_blocks = pl.d / kTileK;
+    a.gsrc = static_cast<const __nv_bfloat16 *>(x);  // token rows gathered through perm (A operand)
+    Launch L(kKindGemmGateUpFwd, st);
+    return L.done(launch_gemm(kGateUpFwd, 256, false, a, tm_wgu, tm_wgu, grid_for(shape, dev), st));
 }
 
 // MXFP8 backward after sort_rows: every GEMM operand quantised along that
@@ -513,33 +536,36 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
 
-    CUtensorMap tm_wgu, tm_aw, tm_wd;
-    if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 128) ||
-        !make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) ||
-        !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
-        return MOE_ERR_LAUNCH;
-
     if (cudaMemsetAsync(w8 + pl.ws_status, 0, 16, st) != cudaSuccess) return MOE_ERR_LAUNCH;
     if ((rc = run_route(shape, pl, dev, logits, saved, w8, st))) return rc;
-    if (pl.mx) return fwd_mx(pl, dev, shape, x, w_gate_up, w_down, out, saved, w8, st);
-    const int grid = grid_for(shape, dev);
-
+    if ((rc = gateup_fwd(pl, dev, shape, x, w_gate_up, saved, w8, st))) return rc;
+    if (pl.mx) return down_mx(pl, dev, shape, w_down, out, saved, w8, st);
+    CUtensorMap tm_aw, tm_wd;
+    if (!make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) ||
+        !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
+        return MOE_ERR_LAUNCH;
     GemmArgs a = base_args(pl, saved, w8);
-    a.n_tiles = pl.I / 128;
-    a.num_k_blocks = pl.d / kTileK;
-    a.gsrc = static_cast<const __nv_bfloat16 *>(x);  // token rows gathered through perm (A operand)
-    {
-        Launch L(kKindGemmGateUpFwd, st);
-        if ((rc = L.done(launch_gemm(kGateUpFwd, 256, false, a, tm_wgu, tm_wgu, grid, st)))) return rc;
-    }
     a.n_tiles = pl.d / pl.bn_d;
     a.num_k_blocks = pl.I / kTileK;
     a.out = static_cast<__nv_bfloat16 *>(out);
-    {
-        Launch L(kKindGemmDownFwd, st);
-        rc = L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid, st));
-    }
-    return rc;
+    Launch L(kKindGemmDownFwd, st);
+    return L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid_for(shape, dev), st));
+}
+
+int moe_recompute(const moe_shape_t *shape, const void *x, const void *w_gate_up, moe_saved_t *saved, void *ws,
+                  size_t ws_bytes, void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(x) || !aligned16(w_gate_up) || !aligned16(ws)) return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    if (ws_bytes < pl.fwd_bytes) return MOE_ERR_WS;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 16, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    return gateup_fwd(pl, dev, shape, x, w_gate_up, saved, w8, st);
 }
 
 int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const void *w_gate_up, const void *w_down,

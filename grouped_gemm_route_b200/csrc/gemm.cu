@@ -185,18 +185,25 @@ __device__ __forceinline__ void warp_store_rows(uint8_t *buf, const uint32_t (&v
     __syncwarp();
 }
 
-// Load 64 bytes of each lane's row from rowptr (nullptr: zeros).
-__device__ __forceinline__ void warp_load_rows(uint8_t *buf, uint32_t (&v)[16], const void *rowptr) {
+// Row loads in two halves, so that a caller can have the next piece's loads
+// in flight while it works on the current one: warp_load_issue starts the
+// global loads (64 bytes of each lane's row from rowptr; nullptr: zeros),
+// warp_load_finish turns them around through the shared buffer.
+__device__ __forceinline__ void warp_load_issue(uint4 (&got)[4], const void *rowptr) {
     const int lane = threadIdx.x & 31;
     const int piece = lane & 3;
     const unsigned long long mine = reinterpret_cast<unsigned long long>(rowptr);
-    uint4 got[4];
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr) {
         const int row = rr * 8 + (lane >> 2);
         const char *src = reinterpret_cast<const char *>(__shfl_sync(0xffffffffu, mine, row));
         got[rr] = src != nullptr ? *reinterpret_cast<const uint4 *>(src + piece * 16) : make_uint4(0u, 0u, 0u, 0u);
     }
+}
+
+__device__ __forceinline__ void warp_load_finish(uint8_t *buf, const uint4 (&got)[4], uint32_t (&v)[16]) {
+    const int lane = threadIdx.x & 31;
+    const int piece = lane & 3;
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr)
         *reinterpret_cast<uint4 *>(buf + xpose_off(rr * 8 + (lane >> 2), piece)) = got[rr];
@@ -622,11 +629,11 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
     }
     const int tok = valid ? p / a.k : 0;
     bool last = false;
-    __threadfence();  // this warp's staging rows before its counts
+    fence_acq_rel_gpu();  // this warp's staging rows (ordered by the transposes' __syncwarp) before its counts
     if (valid) last = atomicAdd(a.cnt + static_cast<size_t>(tok) * a.cnt_stride + t.nt, 1) == a.k - 1;
     unsigned mask = __ballot_sync(0xffffffffu, last);
     if (mask == 0u) return;
-    __threadfence();  // the other slots' staging rows after their counts
+    fence_acq_rel_gpu();  // the other slots' staging rows after their counts
     const int n_last = __popc(mask);
     int base = 0;
     if (lane == 0) base = atomicAdd(tail.count, n_last);
@@ -776,8 +783,11 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
         uint32_t hg[16], hu[16];
-        warp_load_rows(xbuf, hg, valid ? hrow + c * 32 : nullptr);
-        warp_load_rows(xbuf, hu, valid ? hrow + a.I + c * 32 : nullptr);
+        uint4 cg[4], cu[4];
+        warp_load_issue(cg, valid ? hrow + c * 32 : nullptr);
+        warp_load_issue(cu, valid ? hrow + a.I + c * 32 : nullptr);
+        warp_load_finish(xbuf, cg, hg);
+        warp_load_finish(xbuf, cu, hu);
         float G[32];
         tmem_load32_sync(taddr + c * 32, G);
         if (c + 1 == BN / 32) release_accumulator(tempty_acc);

@@ -26,6 +26,10 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// Release/acquire fence at GPU scope (orders this thread's, and through a
+// preceding __syncwarp its warp's, earlier accesses against later ones).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // Record the first device-side error of a call (later ones are dropped).
 __device__ __forceinline__ void report_status(int *status, int code) {
     if (status) atomicCAS(status, kStatusOk, code);

@@ -303,13 +303,80 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int &excl, int *warp_
     if (lane == 31) warp_sums[warp] = incl;
     __syncthreads();
     int base = 0, total = 0;
-    for (int i = 0; i < kFusedWarps; ++i) {
+    const int nwarps = static_cast<int>(blockDim.x >> 5);
+    for (int i = 0; i < nwarps; ++i) {
         const int ws = warp_sums[i];
         if (i < warp) base += ws;
         total += ws;
     }
     excl = base + incl - v;
     return total;
+}
+
+// Phase 2 of both routing kernels: block b scans expert e = b, b+G, ... over
+// the G blocks' histograms (blk_base[.][e] exclusive, counts[e] the total).
+__device__ void route_scan_experts(const RouteFusedArgs &a, int *warp_sums) {
+    const int E = a.E, G = gridDim.x;
+    for (int e = blockIdx.x; e < E; e += G) {
+        int carry = 0;
+        for (int c0 = 0; c0 < G; c0 += blockDim.x) {
+            const int bb = c0 + threadIdx.x;
+            const int v = bb < G ? __ldcg(a.blk_hist + static_cast<size_t>(bb) * E + e) : 0;
+            int excl;
+            const int tot = block_exclusive_scan(v, excl, warp_sums);
+            if (bb < G) a.blk_base[static_cast<size_t>(bb) * E + e] = carry + excl;
+            carry += tot;
+        }
+        if (threadIdx.x == 0) a.counts[e] = carry;
+    }
+}
+
+// Phase 3 start of both routing kernels (E <= blockDim.x: one expert per
+// thread): padded group starts into gst[0..E] (block 0 also publishes them
+// with the unpadded offsets), then the tile table and padding rows of experts
+// b, b+G, ...  Returns false when the groups exceed the sorted capacity.
+__device__ bool route_group_layout(const RouteFusedArgs &a, int *gst, int *warp_sums) {
+    const int E = a.E, b = blockIdx.x, G = gridDim.x;
+    int c_excl = 0, p_excl = 0;
+    const int e = threadIdx.x;
+    const int c = e < E ? __ldcg(a.counts + e) : 0;
+    const int padded = (c + kTileM - 1) / kTileM * kTileM;
+    const int c_tot = block_exclusive_scan(c, c_excl, warp_sums);
+    const int p_tot = block_exclusive_scan(padded, p_excl, warp_sums);
+    if (e < E) gst[e] = p_excl;
+    if (e == 0) gst[E] = p_tot;
+    if (b == 0 && e < E) {
+        a.group_start[e] = p_excl;
+        a.offsets[e] = c_excl;
+    }
+    if (b == 0 && e == 0) {
+        a.group_start[E] = p_tot;
+        a.offsets[E] = c_tot;
+        if (p_tot > a.p_cap) report_status(a.status, kStatusBadIndex);
+    }
+    __syncthreads();
+    if (gst[E] > a.p_cap) return false;
+    for (int x = b; x < E; x += G) {
+        const int gs = gst[x], ge = gst[x + 1], cx = __ldcg(a.counts + x);
+        for (int mt = gs / kTileM + threadIdx.x; mt < ge / kTileM; mt += blockDim.x) a.tile_expert[mt] = x;
+        for (int q = gs + cx + threadIdx.x; q < ge; q += blockDim.x) a.perm[q] = -1;
+    }
+    return true;
+}
+
+// Turns per-warp expert counts wcnt[nwarps][E] into each warp's first sorted
+// position per expert: group start + earlier blocks + earlier warps.
+__device__ void route_warp_bases(const RouteFusedArgs &a, int *wcnt, const int *gst, int nwarps) {
+    const int E = a.E;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = gst[e] + __ldcg(a.blk_base + static_cast<size_t>(blockIdx.x) * E + e);
+        for (int q = 0; q < nwarps; ++q) {
+            const int c = wcnt[q * E + e];
+            wcnt[q * E + e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
 }
 
 // Top-k key of a logit: the high word orders fp32 values (-0 and +0 equal,
@@ -428,59 +495,12 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
     if (!grid_barrier(a.barrier, G, a.status)) return;
 
     // ---- phase 2: per expert, exclusive scan over the blocks ----
-    for (int e = b; e < E; e += G) {
-        int carry = 0;
-        for (int c0 = 0; c0 < G; c0 += kFusedThreads) {
-            const int bb = c0 + threadIdx.x;
-            const int v = bb < G ? __ldcg(a.blk_hist + static_cast<size_t>(bb) * E + e) : 0;
-            int excl;
-            const int tot = block_exclusive_scan(v, excl, warp_sums);
-            if (bb < G) a.blk_base[static_cast<size_t>(bb) * E + e] = carry + excl;
-            carry += tot;
-        }
-        if (threadIdx.x == 0) a.counts[e] = carry;
-    }
+    route_scan_experts(a, warp_sums);
     if (!grid_barrier(a.barrier, 2u * G, a.status)) return;
 
     // ---- phase 3: group starts, tile table, padding, positions ----
-    int c_excl = 0, p_excl = 0, c_tot = 0, p_tot = 0;
-    {
-        // E <= kMaxExperts = kFusedThreads: one expert per thread
-        const int e = threadIdx.x;
-        const int c = e < E ? __ldcg(a.counts + e) : 0;
-        const int padded = (c + kTileM - 1) / kTileM * kTileM;
-        c_tot = block_exclusive_scan(c, c_excl, warp_sums);
-        p_tot = block_exclusive_scan(padded, p_excl, warp_sums);
-        if (e < E) gst[e] = p_excl;
-        if (e == 0) gst[E] = p_tot;
-        if (b == 0 && e < E) {
-            a.group_start[e] = p_excl;
-            a.offsets[e] = c_excl;
-        }
-        if (b == 0 && e == 0) {
-            a.group_start[E] = p_tot;
-            a.offsets[E] = c_tot;
-            if (p_tot > a.p_cap) report_status(a.status, kStatusBadIndex);
-        }
-    }
-    __syncthreads();
-    if (gst[E] > a.p_cap) return;
-    for (int e = b; e < E; e += G) {
-        const int gs = gst[e], ge = gst[e + 1], c = __ldcg(a.counts + e);
-        for (int mt = gs / kTileM + threadIdx.x; mt < ge / kTileM; mt += kFusedThreads) a.tile_expert[mt] = e;
-        for (int q = gs + c + threadIdx.x; q < ge; q += kFusedThreads) a.perm[q] = -1;
-    }
-    // per-warp first position of each expert: group start + earlier blocks +
-    // earlier warps of this block
-    for (int e = threadIdx.x; e < E; e += kFusedThreads) {
-        int run = gst[e] + __ldcg(a.blk_base + static_cast<size_t>(b) * E + e);
-        for (int q = 0; q < kFusedWarps; ++q) {
-            const int c = wcnt[q * E + e];
-            wcnt[q * E + e] = run;
-            run += c;
-        }
-    }
-    __syncthreads();
+    if (!route_group_layout(a, gst, warp_sums)) return;
+    route_warp_bases(a, wcnt, gst, kFusedWarps);
     bool bad = false;
     for (int t = wt0; t < wt1; ++t) {
         for (int j = lane; j < k; j += 32) {
@@ -498,6 +518,216 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
         __syncwarp();
     }
     if (bad) report_status(a.status, kStatusBadIndex);
+}
+
+// ---------------------------------------------------------------------------
+// Fused routing, lane-per-token form, for E <= 128 with E a multiple of 4k and
+// k <= 8.  Same phases and the same results as route_fused_kernel; phase 1 and
+// the positions of phase 3 give each lane one token:
+//   * a warp stages 32 consecutive tokens' logits in shared memory (cp.async;
+//     rows padded by 4 words so that one-row-per-lane reads do not conflict),
+//     and each lane turns its row into order keys in place;
+//   * tau = the smallest of k group maxima (k disjoint groups of E/k values):
+//     at least k values are >= tau, so every one of the k largest is; the lane
+//     lists the positions of its values >= tau;
+//   * the listed values go through a sorted insertion into k registers of
+//     (value key, ~expert) -- larger value first, lower expert on ties -- which
+//     leaves the k largest in slot order;
+//   * weights as in route_fused_kernel, the sum taken in slot order.
+// Positions: per batch of 32 tokens, each expert's set of lanes (a bitmask
+// built with atomicOr) gives a pair's rank among the batch's earlier tokens;
+// the highest of those lanes then advances the warp's running position.
+// ---------------------------------------------------------------------------
+constexpr int kLaneThreads = 256;
+constexpr int kLaneWarps = kLaneThreads / 32;
+constexpr int kLaneMaxE = 128;
+constexpr int kLaneMaxK = 8;
+
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int K>
+__global__ void __launch_bounds__(kLaneThreads, 1) route_lane_kernel(const RouteFusedArgs a) {
+    extern __shared__ __align__(16) uint32_t sm_u[];
+    const int E = a.E, G = gridDim.x, b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int stride = E + 4;                                   // words per staged row
+    uint32_t *stage = sm_u + warp * 32 * stride;                // [32][stride] this warp's rows
+    uint8_t *lists = reinterpret_cast<uint8_t *>(sm_u + kLaneWarps * 32 * stride) + warp * 32 * E;  // [32][E]
+    int *wcnt = reinterpret_cast<int *>(sm_u + kLaneWarps * 32 * stride + kLaneWarps * 8 * E);     // [warps][E]
+    uint32_t *emask = reinterpret_cast<uint32_t *>(wcnt + kLaneWarps * E);                         // [warps][E]
+    int *gst = reinterpret_cast<int *>(emask + kLaneWarps * E);                                    // [E + 1]
+    int *warp_sums = gst + E + 1;                                                                  // [warps]
+    const int t0 = static_cast<int>(static_cast<int64_t>(a.T) * b / G);
+    const int t1 = static_cast<int>(static_cast<int64_t>(a.T) * (b + 1) / G);
+    const int nb = t1 - t0;
+    const int wt0 = t0 + nb * warp / kLaneWarps, wt1 = t0 + nb * (warp + 1) / kLaneWarps;
+    for (int i = threadIdx.x; i < kLaneWarps * E; i += kLaneThreads) {
+        wcnt[i] = 0;
+        emask[i] = 0u;
+    }
+    __syncthreads();
+
+    // ---- phase 1: top-k, one token per lane ----
+    const int P4 = E / 4, gsz = E / K;
+    uint32_t *myrow = stage + lane * stride;
+    uint8_t *mylist = lists + lane * E;
+    if (lane == 0 && wt0 < wt1)
+        prefetch_l2(a.logits + static_cast<size_t>(wt0) * E,
+                    static_cast<uint32_t>(min(32, wt1 - wt0)) * static_cast<uint32_t>(E) * 4u);
+    for (int tb = wt0; tb < wt1; tb += 32) {
+        const int rows = min(32, wt1 - tb);
+        const float *src = a.logits + static_cast<size_t>(tb) * E;
+        for (int q = lane; q < rows * P4; q += 32) {
+            const int r = q / P4, c4 = q - r * P4;
+            cp_async_16(smem_u32(stage + r * stride + 4 * c4), src + static_cast<size_t>(r) * E + 4 * c4);
+        }
+        if (lane == 0 && tb + 32 < wt1)  // the next batch's rows on their way to L2
+            prefetch_l2(src + static_cast<size_t>(32) * E,
+                        static_cast<uint32_t>(min(32, wt1 - tb - 32)) * static_cast<uint32_t>(E) * 4u);
+        cp_async_wait_all();
+        __syncwarp();
+        const bool live = lane < rows;
+        int n = 0;
+        if (live) {
+            uint32_t tau = 0xFFFFFFFFu;
+#pragma unroll 1
+            for (int g = 0; g < K; ++g) {
+                uint32_t gm = 0u;
+                for (int i = g * gsz; i < (g + 1) * gsz; i += 4) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(myrow + i);
+                    const uint4 kk = make_uint4(order_key(__uint_as_float(v.x)), order_key(__uint_as_float(v.y)),
+                                                order_key(__uint_as_float(v.z)), order_key(__uint_as_float(v.w)));
+                    *reinterpret_cast<uint4 *>(myrow + i) = kk;
+                    gm = max(gm, max(max(kk.x, kk.y), max(kk.z, kk.w)));
+                }
+                tau = min(tau, gm);
+            }
+            for (int i = 0; i < E; i += 4) {
+                const uint4 kk = *reinterpret_cast<const uint4 *>(myrow + i);
+                if (kk.x >= tau) mylist[n++] = static_cast<uint8_t>(i);
+                if (kk.y >= tau) mylist[n++] = static_cast<uint8_t>(i + 1);
+                if (kk.z >= tau) mylist[n++] = static_cast<uint8_t>(i + 2);
+                if (kk.w >= tau) mylist[n++] = static_cast<uint8_t>(i + 3);
+            }
+        }
+        uint64_t top[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) top[j] = 0ull;
+        const int nmax = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(n));
+        for (int c = 0; c < nmax; ++c) {
+            if (c < n) {
+                const int i = mylist[c];
+                const uint64_t x = (static_cast<uint64_t>(myrow[i]) << 32) | static_cast<uint32_t>(~i);
+                if (x > top[K - 1]) {
+#pragma unroll
+                    for (int j = K - 1; j > 0; --j) top[j] = x > top[j - 1] ? top[j - 1] : (x > top[j] ? x : top[j]);
+                    top[0] = x > top[0] ? x : top[0];
+                }
+            }
+        }
+        if (live) {
+            const int t = tb + lane;
+            const float m = topk_value(static_cast<uint32_t>(top[0] >> 32));
+            float p[K], sum = 0.f;
+            int e[K];
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                e[j] = static_cast<int>(~static_cast<uint32_t>(top[j]));
+                p[j] = expf(topk_value(static_cast<uint32_t>(top[j] >> 32)) - m);
+                sum += p[j];  // slot order
+            }
+            int32_t *irow = a.idx + static_cast<size_t>(t) * K;
+            float *wrow = a.w + static_cast<size_t>(t) * K;
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                irow[j] = e[j];
+                wrow[j] = p[j] / sum;
+                atomicAdd(&wcnt[warp * E + e[j]], 1);
+            }
+            for (int cc = 0; cc < a.cnt_per_token; ++cc) a.cnt[static_cast<size_t>(t) * a.cnt_per_token + cc] = 0;
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kLaneThreads) {
+        int sum = 0;
+        for (int q = 0; q < kLaneWarps; ++q) sum += wcnt[q * E + e];
+        a.blk_hist[static_cast<size_t>(b) * E + e] = sum;
+    }
+    if (!grid_barrier(a.barrier, G, a.status)) return;
+
+    // ---- phase 2: per expert, exclusive scan over the blocks ----
+    route_scan_experts(a, warp_sums);
+    if (!grid_barrier(a.barrier, 2u * G, a.status)) return;
+
+    // ---- phase 3: group starts, tile table, padding, positions ----
+    if (!route_group_layout(a, gst, warp_sums)) return;
+    route_warp_bases(a, wcnt, gst, kLaneWarps);
+    bool bad = false;
+    const uint32_t below = (1u << lane) - 1u;
+    int *run = wcnt + warp * E;
+    uint32_t *msk = emask + warp * E;
+    for (int tb = wt0; tb < wt1; tb += 32) {
+        const int t = tb + lane;
+        const bool live = t < wt1;
+        int e[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            e[j] = live ? a.idx[static_cast<size_t>(t) * K + j] : 0;  // written by this thread in phase 1
+            if (live) atomicOr(&msk[e[j]], 1u << lane);
+        }
+        __syncwarp();
+        if (live) {
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                const int pos = run[e[j]] + __popc(msk[e[j]] & below);
+                const int pair = t * K + j;
+                if (pos >= 0 && pos < gst[e[j] + 1]) {
+                    a.perm[pos] = pair;
+                    a.inv[pair] = pos;
+                } else {
+                    bad = true;
+                }
+            }
+        }
+        __syncwarp();
+        if (live) {
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                const uint32_t mm = msk[e[j]];
+                if (lane == 31 - __clz(mm)) {  // one lane per expert advances its position
+                    run[e[j]] += __popc(mm);
+                    msk[e[j]] = 0u;
+                }
+            }
+        }
+        __syncwarp();
+    }
+    if (bad) report_status(a.status, kStatusBadIndex);
+}
+
+size_t route_lane_smem(int E) {
+    return (static_cast<size_t>(kLaneWarps) * 32 * (E + 4) + static_cast<size_t>(kLaneWarps) * 8 * E +
+            2 * static_cast<size_t>(kLaneWarps) * E + E + 1 + kLaneWarps) *
+           4;
+}
+
+bool route_lane_ok(int E, int k) { return E <= kLaneMaxE && k <= kLaneMaxK && E % (4 * k) == 0; }
+
+const void *route_lane_fn(int k) {
+    switch (k) {
+        case 1: return reinterpret_cast<const void *>(route_lane_kernel<1>);
+        case 2: return reinterpret_cast<const void *>(route_lane_kernel<2>);
+        case 3: return reinterpret_cast<const void *>(route_lane_kernel<3>);
+        case 4: return reinterpret_cast<const void *>(route_lane_kernel<4>);
+        case 5: return reinterpret_cast<const void *>(route_lane_kernel<5>);
+        case 6: return reinterpret_cast<const void *>(route_lane_kernel<6>);
+        case 7: return reinterpret_cast<const void *>(route_lane_kernel<7>);
+        default: return reinterpret_cast<const void *>(route_lane_kernel<8>);
+    }
 }
 
 constexpr int kBwdThreads = 256;
@@ -646,22 +876,28 @@ cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t 
 }
 
 int route_fused_grid(int T, int E, int k, int sms, int n_chunks) {
-    const int nv = (E + 31) / 32;
-    const size_t smem = route_fused_smem(E, k);
+    (void)T;
     int per_sm = 0;
     cudaError_t e;
-    if (nv <= 1)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<1>, kFusedThreads, smem);
-    else if (nv <= 2)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<2>, kFusedThreads, smem);
-    else if (nv <= 4)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<4>, kFusedThreads, smem);
-    else if (nv <= 8)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<8>, kFusedThreads, smem);
-    else
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<16>, kFusedThreads, smem);
-    (void)T;
-    (void)k;
+    if (route_lane_ok(E, k)) {
+        const void *fn = route_lane_fn(k);
+        const size_t smem = route_lane_smem(E);
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kLaneThreads, smem);
+    } else {
+        const int nv = (E + 31) / 32;
+        const size_t smem = route_fused_smem(E, k);
+        if (nv <= 1)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<1>, kFusedThreads, smem);
+        else if (nv <= 2)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<2>, kFusedThreads, smem);
+        else if (nv <= 4)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<4>, kFusedThreads, smem);
+        else if (nv <= 8)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<8>, kFusedThreads, smem);
+        else
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<16>, kFusedThreads, smem);
+    }
     if (e != cudaSuccess || per_sm < 1) return 0;
     const int g = per_sm * sms;
     return g < n_chunks ? g : n_chunks;
@@ -679,6 +915,9 @@ cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t
     RouteFusedArgs a{logits, T, E, k, idx, w, blk_hist, blk_base, counts, offsets, group_start,
                      tile_expert, perm, inv, cnt, cnt_per_token, p_cap, barrier, status};
     void *params[] = {&a};
+    if (route_lane_ok(E, k))
+        return cudaLaunchCooperativeKernel(route_lane_fn(k), dim3(grid), dim3(kLaneThreads), params,
+                                           route_lane_smem(E), s);
     const size_t smem = route_fused_smem(E, k);
     const int nv = (E + 31) / 32;
     const void *fn = nv <= 1   ? reinterpret_cast<const void *>(route_fused_kernel<1>)

@@ -25,7 +25,7 @@ MOE_ERR_SCRATCH_LIMIT = -9
 SAVED_FIELDS = ("topk_idx", "topk_w", "counts", "offsets", "group_start", "tile_expert", "perm", "inv", "h", "aw")
 EXPORTS = ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
            "moe_error_string", "moe_profile_enable", "moe_profile_read", "moe_kernel_name",
-           "moe_selftest_wait_timeout", "moe_route_noalloc")
+           "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_recompute")
 
 
 class MoeShape(ctypes.Structure):
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
     L.moe_profile_enable.argtypes = [ctypes.c_int]
     L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
     L.moe_route_noalloc.argtypes = [S, P, ctypes.POINTER(MoeSaved), P]
+    L.moe_recompute.argtypes = [S, P, P, ctypes.POINTER(MoeSaved), P, ctypes.c_size_t, P]
+    L.moe_recompute.restype = ctypes.c_int
     L.moe_route_noalloc.restype = ctypes.c_int
     L.moe_selftest_wait_timeout.argtypes = [P, P]
     L.moe_selftest_wait_timeout.restype = ctypes.c_int
@@ -147,6 +149,14 @@ def bwd(shape, gout, x, wgu, wd, saved: dict, dx, dwgu, dwd, dscore, dlogits, ws
     _check(lib().moe_bwd(ctypes.byref(shape), _ptr(gout), _ptr(x), _ptr(wgu), _ptr(wd), ctypes.byref(st),
                          _ptr(dx), _ptr(dwgu), _ptr(dwd), _ptr(dscore), _ptr(dlogits), _ptr(ws), ws.numel(),
                          _stream(stream)), "moe_bwd")
+
+
+def recompute(shape, x, wgu, saved: dict, ws, stream=None):
+    """Rewrite saved h and aw from x and W_gate_up for the routing in `saved`
+    (the gate/up GEMM again, for a backward whose forward dropped them)."""
+    st = saved_struct(saved)
+    _check(lib().moe_recompute(ctypes.byref(shape), _ptr(x), _ptr(wgu), ctypes.byref(st), _ptr(ws), ws.numel(),
+                               _stream(stream)), "moe_recompute")
 
 
 def get_status(ws, stream=None) -> int:

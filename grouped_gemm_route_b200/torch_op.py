@@ -1,6 +1,6 @@
 """PyTorch custom ops and autograd for the fused MoE layer.
 
-    out = moe_layer(x, logits, w_gate_up, w_down, top_k)     # bf16 [T, d]
+    out = moe_layer(x, logits, w_gate_up, w_down, top_k)     # [T, d], x.dtype
     out.backward(g)   # x.grad, logits.grad, w_gate_up.grad, w_down.grad
 
 The integration surface that "Mario/overlap moe kernel integration (prime-rl
@@ -13,7 +13,9 @@ where every step of the layer runs.  They are registered with torch.library
 (`ggr_b200::moe_forward`, `ggr_b200::moe_backward`) together with fake
 implementations, so torch.compile(fullgraph=True) traces through the layer
 without a graph break.  The saved routing state and activations are extra
-outputs of the forward op, kept by autograd for the backward op.
+outputs of the forward op, kept by autograd for the backward op.  A second
+pair (`moe_forward_ckpt`, `moe_backward_ckpt`) is the recompute mode: only the
+routing state is kept, and the backward regenerates h and aw (moe_recompute).
 """
 from __future__ import annotations
 
@@ -21,7 +23,7 @@ import torch
 
 from . import moe as M
 
-__all__ = ["moe_layer", "moe_forward", "moe_backward"]
+__all__ = ["moe_layer", "moe_forward", "moe_backward", "moe_forward_ckpt", "moe_backward_ckpt"]
 
 _SAVED_SHAPES = {
     "topk_idx": lambda T, E, k, I, p: (T, k), "topk_w": lambda T, E, k, I, p: (T, k),
@@ -131,13 +133,88 @@ def _backward(ctx, grad_out, *_unused_saved_grads):
 moe_forward.register_autograd(_backward, setup_context=_setup_context)
 
 
-def moe_layer(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor, top_k: int,
-              mxfp8: bool = False) -> torch.Tensor:
-    """The fused MoE layer as a differentiable function: bf16 out [T, d].
+_ROUTING_FIELDS = M.SAVED_FIELDS[:8]  # the saved fields without h and aw
 
-    x bf16 [T, d]; logits fp32 [T, E]; w_gate_up bf16 [E, 2I, d] (rows 0..I-1
-    gate, I..2I-1 up); w_down bf16 [E, d, I].  mxfp8=True runs the expert GEMMs
-    on MXFP8 operands (E4M3 with one UE8M0 scale per 32 elements along K).
+
+@torch.library.custom_op("ggr_b200::moe_forward_ckpt", mutates_args=(), device_types="cuda")
+def moe_forward_ckpt(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
+                     top_k: int, dtype: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
+                                                      torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
+                                                      torch.Tensor]:
+    """Recompute mode: out plus the routing state only; h and aw are dropped
+    when the op returns and regenerated by the backward op."""
+    outs = moe_forward(x, logits, w_gate_up, w_down, top_k, dtype)
+    return outs[:9]
+
+
+@moe_forward_ckpt.register_fake
+def _moe_forward_ckpt_fake(x, logits, w_gate_up, w_down, top_k, dtype):
+    return _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype)[:9]
+
+
+@torch.library.custom_op("ggr_b200::moe_backward_ckpt", mutates_args=(), device_types="cuda")
+def moe_backward_ckpt(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
+                      topk_idx: torch.Tensor, topk_w: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
+                      group_start: torch.Tensor, tile_expert: torch.Tensor, perm: torch.Tensor, inv: torch.Tensor,
+                      top_k: int,
+                      dtype: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Recompute mode backward: moe_recompute regenerates h and aw, then moe_bwd."""
+    T, d, E, I = _dims(x, w_gate_up)
+    shape = M.make_shape(T, d, E, top_k, I, dtype)
+    _, p_cap = M.saved_sizes(shape)
+    dev = x.device
+    h = torch.empty(p_cap, 2 * I, dtype=torch.bfloat16, device=dev)
+    aw = torch.empty(p_cap, I, dtype=torch.bfloat16, device=dev)
+    saved = dict(zip(M.SAVED_FIELDS, (topk_idx, topk_w, counts, offsets, group_start, tile_expert, perm, inv, h,
+                                      aw)))
+    f, _ = M.workspace_size(shape)
+    ws = torch.empty(f, dtype=torch.uint8, device=dev)
+    M.recompute(shape, x.contiguous(), w_gate_up.contiguous(), saved, ws, torch.cuda.current_stream(dev))
+    del ws
+    return moe_backward(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start, tile_expert,
+                        perm, inv, h, aw, top_k, dtype)
+
+
+@moe_backward_ckpt.register_fake
+def _moe_backward_ckpt_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
+                            tile_expert, perm, inv, top_k, dtype):
+    return _moe_backward_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
+                              tile_expert, perm, inv, None, None, top_k, dtype)
+
+
+def _setup_context_ckpt(ctx, inputs, output):
+    x, logits, w_gate_up, w_down, top_k, dtype = inputs
+    routing = output[1:]
+    ctx.save_for_backward(x, w_gate_up, w_down, *routing)
+    ctx.top_k, ctx.dtype = top_k, dtype
+    ctx.mark_non_differentiable(*routing)
+
+
+def _backward_ckpt(ctx, grad_out, *_unused_routing_grads):
+    x, w_gate_up, w_down, *routing = ctx.saved_tensors
+    dx, dlogits, dwgu, dwd, _ = moe_backward_ckpt(grad_out.to(torch.bfloat16), x, w_gate_up, w_down, *routing,
+                                                  ctx.top_k, ctx.dtype)
+    return dx, dlogits, dwgu, dwd, None, None
+
+
+moe_forward_ckpt.register_autograd(_backward_ckpt, setup_context=_setup_context_ckpt)
+
+
+def moe_layer(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor, top_k: int,
+              mxfp8: bool = False, recompute: bool = False) -> torch.Tensor:
+    """The fused MoE layer as a differentiable function: out [T, d] in x's dtype.
+
+    x [T, d]; logits [T, E]; w_gate_up [E, 2I, d] (rows 0..I-1 gate, I..2I-1
+    up); w_down [E, d, I].  The layer runs on bf16 tokens and weights and fp32
+    logits: other floating dtypes are cast on the way in, and autograd returns
+    each gradient in its input's dtype.  mxfp8=True runs the expert GEMMs on
+    MXFP8 operands (E4M3 with one UE8M0 scale per 32 elements along K).
+    recompute=True keeps only the routing state between forward and backward
+    (h and aw, 0.6 GB at the Qwen3-30B-A3B layer shape, are regenerated by one
+    more gate/up GEMM in the backward); the results are bit-identical.
     """
     dtype = M.MOE_MXFP8 if mxfp8 else M.MOE_BF16
-    return moe_forward(x, logits, w_gate_up, w_down, int(top_k), dtype)[0]
+    op = moe_forward_ckpt if recompute else moe_forward
+    out = op(x.to(torch.bfloat16), logits.to(torch.float32), w_gate_up.to(torch.bfloat16),
+             w_down.to(torch.bfloat16), int(top_k), dtype)[0]
+    return out.to(x.dtype)

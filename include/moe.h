@@ -115,7 +115,8 @@ int moe_route(const moe_shape_t *shape, const float *logits, moe_saved_t *saved,
 
 /* Forward.  x: bf16 [T,d]; logits: fp32 [T,E]; w_gate_up: bf16 [E,2I,d];
  * w_down: bf16 [E,d,I]; out: bf16 [T,d].  Runs moe_route, then the gate/up
- * grouped GEMM (tokens gathered by TMA from x, SwiGLU in the epilogue; writes
+ * grouped GEMM (token rows gathered from x through the dispatch permutation
+ * straight into the GEMM's operand tiles, SwiGLU in the epilogue; writes
  * saved->h and saved->aw), then the down grouped GEMM whose epilogue performs
  * the weighted combine as a deterministic slot-ordered reduction into out. */
 int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits,
@@ -133,6 +134,18 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x,
             void *dx, void *dw_gate_up, void *dw_down, float *dscore, float *dlogits,
             void *ws, size_t ws_bytes, void *stream);
 
+/* Recompute mode ("Mario/overlap moe kernel integration (prime-rl PR #3651)",
+ * the custom-op commit note: under activation checkpointing the op saves only
+ * its own inputs and the forward runs again before the backward).  Rewrites
+ * saved->h and saved->aw from x and w_gate_up for the routing already in
+ * `saved` (topk_w, group_start, tile_expert, perm from moe_fwd or moe_route):
+ * the gate/up grouped GEMM and its SwiGLU epilogue only, bit-identical to what
+ * moe_fwd wrote.  A caller may therefore drop h and aw after the forward and
+ * call this before moe_bwd.  Workspace: fwd_bytes of moe_workspace_size.
+ * Arguments and errors as moe_fwd. */
+int moe_recompute(const moe_shape_t *shape, const void *x, const void *w_gate_up, moe_saved_t *saved,
+                  void *ws, size_t ws_bytes, void *stream);
+
 /* Routing and dispatch for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this entry point; it exists for users of
@@ -141,8 +154,9 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x,
  * gives none to plug-ins, or code on a latency-critical path where an
  * allocation (which may synchronise the whole device) is not acceptable.
  *
- * Same results as moe_route (same kernels), but the per-block histograms and
- * bases that moe_route keeps in the caller's workspace live instead in a fixed
+ * Same results as moe_route, bit for bit (it runs the three-launch form of
+ * the same routing: top-k, scan, permutation), but the per-block histograms and
+ * bases that it keeps in a workspace live instead in a fixed
  * 1 MiB __device__ array inside the library, which every GPU that loads the
  * library holds until the process exits.  The caller still allocates and
  * passes the logits and every moe_saved_t routing field (topk_idx, topk_w,

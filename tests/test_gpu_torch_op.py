@@ -50,3 +50,37 @@ def test_compile_fullgraph_matches_eager():
     torch.cuda.synchronize()
     for a, b in zip(eager, comp):
         assert torch.equal(a.grad, b.grad)
+
+
+def test_caller_dtypes_in_and_out():
+    cfg, inp = IN.make_workload("tiny", seed=5, device="cpu")
+    k = cfg["k"]
+    dev = "cuda:0"
+    x = inp["x"].to(dev).float().requires_grad_()
+    lg = inp["logits"].to(dev).double().requires_grad_()
+    wgu = inp["wgu"].to(dev).float().requires_grad_()
+    wd = inp["wd"].to(dev).requires_grad_()
+    out = TO.moe_layer(x, lg, wgu, wd, k)
+    assert out.dtype == torch.float32
+    out.backward(inp["gout"].to(dev).float())
+    assert x.grad.dtype == torch.float32 and lg.grad.dtype == torch.float64
+    assert wgu.grad.dtype == torch.float32 and wd.grad.dtype == torch.bfloat16
+    # same numbers as the all-bf16 call
+    ref = leaves(inp, dev)
+    TO.moe_layer(*ref, k).backward(inp["gout"].to(dev))
+    assert torch.equal(x.grad.to(torch.bfloat16), ref[0].grad)
+    assert torch.equal(wd.grad, ref[3].grad)
+
+
+def test_recompute_mode_same_bits():
+    cfg, inp = IN.make_workload("tiny", seed=6, device="cpu")
+    k = cfg["k"]
+    dev = "cuda:0"
+    gout = inp["gout"].to(dev)
+    a = leaves(inp, dev)
+    TO.moe_layer(*a, k).backward(gout)
+    b = leaves(inp, dev)
+    TO.moe_layer(*b, k, recompute=True).backward(gout)
+    torch.cuda.synchronize()
+    for p, q in zip(a, b):
+        assert torch.equal(p.grad, q.grad)
