@@ -55,6 +55,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="skip sampling nvidia-smi during the timed region")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-recompute", action="store_true", help="skip the recompute-mode timing")
     ap.add_argument("--no-routing-sweep", action="store_true",
                     help="skip the routing-only timing over token counts")
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0 = auto)")
@@ -414,6 +415,35 @@ def main():
                      "launches": v[1]} for n, v in per_kernel.items() if v[1]}
     launches = int(sum(v[1] for v in per_kernel.values()))
 
+    # ---- recompute mode: forward, h and aw regenerated, backward ----
+    # (the layer cost under activation checkpointing: the gate/up GEMM runs
+    # twice; same results as the plain step, tested bit for bit)
+    recompute = None
+    if not args.no_recompute:
+        def step_recompute():
+            layer.forward(x, lg, wgu, wd, stream)
+            M.recompute(layer.shape, x, wgu, layer.saved, layer.ws, stream)
+            layer.backward(gout, x, wgu, wd, True, stream)
+
+        for _ in range(3):
+            step_recompute()
+        n_rc = max(3, args.steps // 4)
+        barrier()
+        torch.cuda.synchronize(dev)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(n_rc):
+            step_recompute()
+        r1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        rc_ms = max_over_ranks(r0.elapsed_time(r1), pg, dev) / n_rc
+        if layer.status(stream) != 0:
+            raise SystemExit("device status error in the recompute-mode loop")
+        recompute = {"ms_per_step": rc_ms, "value": job_tflops(flops_step, world, rc_ms), "unit": UNIT,
+                     "steps": n_rc, "note": "forward + moe_recompute (gate/up GEMM again) + backward; value counts "
+                                            "the layer's fwd+bwd FLOPs only"}
+
     # ---- end-to-end through the public API with host buffers ----
     # Every step copies its inputs (x, logits, grad_out) from pinned host memory,
     # runs forward + backward, and copies its results (out, dx, dscore) back.
@@ -494,7 +524,7 @@ def main():
         "frac_of_peak": {"step": value / world / peak, "gemm_only": (flops_step / (gemm_ms * 1e-3) / 1e12) / peak
                               if gemm_ms else None, "peak": peak, "peak_source": roofline["peak_source"]},
         "roofline": roofline, "routing": routing, "kernels": breakdown, "gpu_launches": launches,
-        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        "clocks": clk, "e2e": e2e, "recompute": recompute, "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
     return 0
