@@ -500,6 +500,44 @@ __device__ __forceinline__ void release_accumulator(uint64_t *tempty_acc) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(tempty_acc);
 }
 
+// One 32-column chunk of this warp's accumulator rows (fp32 in registers) as
+// bf16 to row (nullptr: skipped).
+__device__ __forceinline__ void store_chunk_bf16(uint8_t *xbuf, const uint32_t (&v)[32], __nv_bfloat16 *row) {
+    uint32_t pv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+    warp_store_rows(xbuf, pv, row);
+}
+
+// Streams this warp's 32 accumulator rows (BN fp32 columns) to bf16 rows at
+// row (nullptr: skipped), 32 columns at a time, with the tensor-memory load of
+// chunk c + 1 in flight while chunk c is converted and stored.  Releases the
+// accumulator as soon as its last chunk is in registers.
+template <int BN>
+__device__ __forceinline__ void store_accumulator_bf16(uint32_t taddr, uint8_t *xbuf, __nv_bfloat16 *row,
+                                                       uint64_t *tempty_acc) {
+    uint32_t ra[32], rb[32];
+    tmem_load32(taddr, ra);
+    tmem_load_wait();
+    tmem_regs_ready(ra);
+#pragma unroll
+    for (int c = 0; c < BN / 32; c += 2) {
+        tmem_load32(taddr + (c + 1) * 32, rb);
+        store_chunk_bf16(xbuf, ra, row != nullptr ? row + c * 32 : nullptr);
+        tmem_load_wait();
+        tmem_regs_ready(rb);
+        if (c + 2 < BN / 32)
+            tmem_load32(taddr + (c + 2) * 32, ra);
+        else
+            release_accumulator(tempty_acc);
+        store_chunk_bf16(xbuf, rb, row != nullptr ? row + (c + 1) * 32 : nullptr);
+        if (c + 2 < BN / 32) {
+            tmem_load_wait();
+            tmem_regs_ready(ra);
+        }
+    }
+}
+
 // Per-CTA queue of (token, column tile) pairs whose last slot this CTA wrote.
 // The epilogue warps reserve entries (count) and publish them (an entry holds
 // -1 until written).  Workers claim batches of four entries (claim): warps 6
@@ -515,51 +553,79 @@ struct TailList {
 
 // gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up.
 // MXFP8: also aw's E4M3 codes and scale atoms along I (the down GEMM's K).
+// One 32-column chunk c of gate (gr) and up (ur) accumulator values.
+template <int BN, bool MX>
+__device__ __forceinline__ void gateup_chunk(const GemmArgs &a, const Tile &t, int r, int pos, bool valid, float wv,
+                                             int c, const uint32_t (&gr)[32], const uint32_t (&ur)[32],
+                                             __nv_bfloat16 *hrow, __nv_bfloat16 *arow, uint8_t *xbuf) {
+    constexpr int kHalf = BN / 2;
+    uint32_t pg[16], pu[16], pa[16];
+    float av[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float g = __uint_as_float(gr[i]), u = __uint_as_float(ur[i]);
+        av[i] = valid ? wv * g * __fdividef(1.f, 1.f + __expf(-g)) * u : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        pg[i] = valid ? pack_bf16x2(__uint_as_float(gr[2 * i]), __uint_as_float(gr[2 * i + 1])) : 0u;
+        pu[i] = valid ? pack_bf16x2(__uint_as_float(ur[2 * i]), __uint_as_float(ur[2 * i + 1])) : 0u;
+        pa[i] = pack_bf16x2(av[2 * i], av[2 * i + 1]);
+    }
+    warp_store_rows(xbuf, pg, hrow + c * 32);
+    warp_store_rows(xbuf, pu, hrow + a.I + c * 32);
+    warp_store_rows(xbuf, pa, arow + c * 32);
+    if constexpr (MX) {
+        const int col = t.nt * kHalf + c * 32;
+        const int sc = mx_scale_exp(amax32(av));
+        uint32_t codes[8];
+        mx_encode32(av, sc, codes);
+        uint4 *dst = reinterpret_cast<uint4 *>(a.mx_codes + static_cast<size_t>(pos) * a.I + col);
+        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        const int64_t atom = static_cast<int64_t>(t.mt) * (a.I / 128) + col / 128;
+        a.mx_sf[atom * kMxAtomBytes + mx_atom_byte(r, col / 32)] = static_cast<uint8_t>(sc + 127);
+    }
+}
+
+// The tensor-memory loads of chunk c + 1 are in flight while chunk c is worked on.
 template <int BN, bool MX>
 __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                                uint64_t *tempty_acc, uint8_t *xbuf) {
     constexpr int kHalf = BN / 2;
+    constexpr int kChunks = kHalf / 32;
+    static_assert(kChunks % 2 == 0, "chunks are taken in pairs");
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
     const float wv = valid ? __ldg(a.topk_w + p) : 0.f;
     __nv_bfloat16 *hrow = a.h + static_cast<size_t>(pos) * 2 * a.I + t.nt * kHalf;
     __nv_bfloat16 *arow = a.aw + static_cast<size_t>(pos) * a.I + t.nt * kHalf;
-#pragma unroll 1
-    for (int c = 0; c < kHalf / 32; ++c) {
-        uint32_t gr[32], ur[32];
-        tmem_load32(taddr + c * 32, gr);
-        tmem_load32(taddr + kHalf + c * 32, ur);
+    uint32_t ga[32], ua[32], gb[32], ub[32];
+    tmem_load32(taddr, ga);
+    tmem_load32(taddr + kHalf, ua);
+    tmem_load_wait();
+    tmem_regs_ready(ga);
+    tmem_regs_ready(ua);
+#pragma unroll
+    for (int c = 0; c < kChunks; c += 2) {
+        tmem_load32(taddr + (c + 1) * 32, gb);
+        tmem_load32(taddr + kHalf + (c + 1) * 32, ub);
+        gateup_chunk<BN, MX>(a, t, r, pos, valid, wv, c, ga, ua, hrow, arow, xbuf);
         tmem_load_wait();
-        tmem_regs_ready(gr);
-        tmem_regs_ready(ur);
-        if (c + 1 == kHalf / 32) release_accumulator(tempty_acc);  // TMEM no longer needed
-        uint32_t pg[16], pu[16], pa[16];
-        float av[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float g = __uint_as_float(gr[i]), u = __uint_as_float(ur[i]);
-            av[i] = valid ? wv * g * __fdividef(1.f, 1.f + __expf(-g)) * u : 0.f;
+        tmem_regs_ready(gb);
+        tmem_regs_ready(ub);
+        if (c + 2 < kChunks) {
+            tmem_load32(taddr + (c + 2) * 32, ga);
+            tmem_load32(taddr + kHalf + (c + 2) * 32, ua);
+        } else {
+            release_accumulator(tempty_acc);  // TMEM no longer needed
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            pg[i] = valid ? pack_bf16x2(__uint_as_float(gr[2 * i]), __uint_as_float(gr[2 * i + 1])) : 0u;
-            pu[i] = valid ? pack_bf16x2(__uint_as_float(ur[2 * i]), __uint_as_float(ur[2 * i + 1])) : 0u;
-            pa[i] = pack_bf16x2(av[2 * i], av[2 * i + 1]);
-        }
-        warp_store_rows(xbuf, pg, hrow + c * 32);
-        warp_store_rows(xbuf, pu, hrow + a.I + c * 32);
-        warp_store_rows(xbuf, pa, arow + c * 32);
-        if constexpr (MX) {
-            const int col = t.nt * kHalf + c * 32;
-            const int sc = mx_scale_exp(amax32(av));
-            uint32_t codes[8];
-            mx_encode32(av, sc, codes);
-            uint4 *dst = reinterpret_cast<uint4 *>(a.mx_codes + static_cast<size_t>(pos) * a.I + col);
-            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-            const int64_t atom = static_cast<int64_t>(t.mt) * (a.I / 128) + col / 128;
-            a.mx_sf[atom * kMxAtomBytes + mx_atom_byte(r, col / 32)] = static_cast<uint8_t>(sc + 127);
+        gateup_chunk<BN, MX>(a, t, r, pos, valid, wv, c + 1, gb, ub, hrow, arow, xbuf);
+        if (c + 2 < kChunks) {
+            tmem_load_wait();
+            tmem_regs_ready(ga);
+            tmem_regs_ready(ua);
         }
     }
 }
@@ -617,16 +683,7 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
     __nv_bfloat16 *srow = valid ? a.stage + static_cast<size_t>(p) * a.d + t.nt * BN : nullptr;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_load32_sync(taddr + c * 32, v);
-        if (c + 1 == BN / 32) release_accumulator(tempty_acc);
-        uint32_t pv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        warp_store_rows(xbuf, pv, srow != nullptr ? srow + c * 32 : nullptr);
-    }
+    store_accumulator_bf16<BN>(taddr, xbuf, srow, tempty_acc);
     const int tok = valid ? p / a.k : 0;
     bool last = false;
     fence_acq_rel_gpu();  // this warp's staging rows (ordered by the transposes' __syncwarp) before its counts
@@ -842,21 +899,16 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
     const int Ntot = MODE == kDownWgrad ? a.I : a.d;
     __nv_bfloat16 *row =
         a.dw + (static_cast<size_t>(t.e) * Mtot + t.mt * kTileM + r) * static_cast<size_t>(Ntot) + t.nt * BN;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pv[16];
-        if (t.nkb > 0) {
-            float v[32];
-            tmem_load32_sync(taddr + c * 32, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pv[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pv[i] = 0u;
-        }
-        if (c + 1 == BN / 32) release_accumulator(tempty_acc);
-        warp_store_rows(xbuf, pv, row + c * 32);
+    if (t.nkb > 0) {
+        store_accumulator_bf16<BN>(taddr, xbuf, row, tempty_acc);
+        return;
     }
+    release_accumulator(tempty_acc);  // an expert without tokens: exact zeros, the accumulator is not read
+    uint32_t zero[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) zero[i] = 0u;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) warp_store_rows(xbuf, zero, row + c * 32);
 }
 
 template <int MODE, int BN, bool MX>
