@@ -31,8 +31,8 @@ struct Plan {
     int n_chunks;       // routing blocks
     int bn_d;           // N tile of the GEMMs whose N is d
     int bn_i;           // N tile of the GEMMs whose N is I
-    int cnt_stride;     // d / bn_d
-    int dpart_stride;   // I / bn_i
+    int cnt_stride;     // d / bn_d: combine counters per token, one per column tile
+    int dpart_stride;   // 2 I / bn_i: dscore partials per sorted row, one per column half-tile
     // workspace layout (byte offsets)
     size_t ws_status, ws_cnt, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
     size_t ws_dh, ws_dpart, ws_xs, ws_gs, bwd_bytes;
@@ -69,7 +69,8 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     p->bn_d = !p->mx && s->d % 256 == 0 ? 256 : 128;  // MXFP8 GEMMs use 128-wide N tiles
     p->bn_i = !p->mx && s->I % 256 == 0 ? 256 : 128;
     p->cnt_stride = s->d / p->bn_d;
-    p->dpart_stride = s->I / p->bn_i;
+    p->dpart_stride = 2 * s->I / p->bn_i;  // the down dgrad's two epilogue warps per row each write a partial
+                                           // (the kernel's kSplit for that mode)
 
     size_t off = 0;
     p->ws_status = off;

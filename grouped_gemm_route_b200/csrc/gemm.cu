@@ -3,21 +3,26 @@
 // One kernel template serves the six expert GEMMs of the layer (two forward,
 // four backward).  Each CTA owns one SM and walks a static list of output
 // tiles.  Inside a CTA the work is split by warp:
-//   warp 0      TMA producer: bulk tensor loads of the dense operand (expert
-//               weights, or the sorted-layout activations) into a 4- or
-//               6-stage shared-memory ring, 128-byte swizzled.
-//   warps 6, 7  gather producers (forward gate/up GEMM): 16-byte cp.async
-//               copies of the x rows picked through the dispatch permutation,
-//               written with the same 128-byte swizzle.  The dispatch is fused
-//               into the operand load: the forward never writes a permuted
-//               copy of the tokens.  (The backward reads x and grad_out from
-//               expert-sorted copies made by sort_rows, so that its wgrads,
-//               whose K dimension is the tokens, run on plain TMA tiles.)
-//   warp 1      allocates tensor memory and issues tcgen05.mma (one thread),
-//               accumulating a 128 x BN fp32 tile in TMEM; two TMEM buffers
-//               let the epilogue of one tile overlap the mainloop of the next.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               output row per thread) and the fused per-mode epilogue.
+//   warp 0       TMA producer: bulk tensor loads of the dense operand (expert
+//                weights, or the sorted-layout activations) into a 4- or
+//                6-stage shared-memory ring, 128-byte swizzled.
+//   warp 1       allocates tensor memory and issues tcgen05.mma (one thread),
+//                accumulating a 128 x BN fp32 tile in TMEM; two TMEM buffers
+//                let the epilogue of one tile overlap the mainloop of the next.
+//   warps 2..5   epilogue, one warp per tensor-memory lane quadrant (its 32
+//                rows; tcgen05.ld, one output row per thread) and the mode's
+//                fused epilogue.  The down dgrad, whose epilogue waits on loads
+//                of h, runs eight: warps 2..9, two per quadrant, each taking
+//                half of the tile's columns.
+//   next two     forward gate/up GEMM: gather producers, 16-byte cp.async
+//                copies of the x rows picked through the dispatch permutation,
+//                written with the same 128-byte swizzle.  The dispatch is fused
+//                into the operand load: the forward never writes a permuted
+//                copy of the tokens.  (The backward reads x and grad_out from
+//                expert-sorted copies made by sort_rows, so that its wgrads,
+//                whose K dimension is the tokens, run on plain TMA tiles.)
+//                Combine GEMMs: combine workers (below).  Idle in the other
+//                modes.
 //
 // Modes (see GemmMode): the expert MLP of "Prime Intellect Fused MoE Kernel:
 // 3.11x MoE Training Speed", section "What a mixture-of-experts layer actually
@@ -29,8 +34,9 @@
 //
 // The combine and the scatter are deterministic: each (token, slot) row writes
 // its tile slice to a slot-addressed staging buffer and bumps a per-(token,
-// column tile) counter; the warp holding the row that brings the counter to k
-// sums the k slots in slot order.  No thread ever waits on another CTA.
+// column tile) counter; the CTA holding the row that brings the counter to k
+// queues it, and its combine workers sum the k slots in slot order.  No thread
+// ever waits on another CTA.
 //
 // Every wait on an mbarrier is bounded in time.  On expiry the kernel records
 // a timeout in the status word, stops issuing work, waits (bounded) for its own
@@ -50,16 +56,14 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kGatherWarp0 = 6;               // warps 6 and 7 gather token rows
+constexpr int kEpiWarp0 = 2;                  // epilogue warps start here (one or two per TMEM lane quadrant)
+constexpr int kMaxEpiWarps = 8;
 constexpr int kGatherThreads = 64;
 constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr int kChunkBytes = 64 * kTileK * 2;  // 8 KB: one 64-wide MN chunk of an MN-major K-block
 constexpr uint32_t kSbo = 1024;               // 8 rows x 128 B swizzle atom
 constexpr uint32_t kMnLbo = kChunkBytes;      // MN-major: distance between 64-wide chunks
 constexpr int kXposeBytes = 32 * 64;          // per epilogue warp: 32 rows x 64 bytes
-constexpr int kTailCap = 4096;                // finished (token, column tile) pairs a CTA queues
-constexpr int kEpiWarps = 4;
 
 // Pipeline geometry.  A stage holds one K block of both operands: 128-byte
 // operand rows, i.e. 64 bf16 or 128 E4M3 elements.  MXFP8 stages also carry
@@ -76,12 +80,14 @@ struct Cfg {
     static constexpr int kBarOffset = kSfOffset + kStages * kSfBytes;  // mbarriers, TMEM slot, abort flag
     // one region, used by the wgrads for their expert order and by the
     // combine modes for their queue of finished tokens
+    static constexpr int kTailCap = MX ? 2048 : 4096;  // finished (token, column half-tile) pairs a CTA queues
     static constexpr int kOrderOffset = kBarOffset + 512;
     static constexpr int kTailOffset = kOrderOffset;
     static constexpr int kUnionBytes = 4 * (kTailCap + 4) > 8 * kMaxExperts ? 4 * (kTailCap + 4) : 8 * kMaxExperts;
-    static constexpr int kXposeOffset = kOrderOffset + kUnionBytes;            // 4 x 2 KB epilogue transposes
-    static constexpr int kSmemBytes = kXposeOffset + 4 * kXposeBytes + 1024;  // + 1 KB alignment slack
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static constexpr int kXposeOffset = kOrderOffset + kUnionBytes;  // one 2 KB transpose per epilogue warp
+    // + 1 KB alignment slack; the largest layout must fit 227 KB
+    static constexpr int smem_bytes(int epi_warps) { return kXposeOffset + epi_warps * kXposeBytes + 1024; }
+    static_assert(smem_bytes(kMaxEpiWarps) <= 227 * 1024, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = MX ? 512 : 2 * BN;
     static constexpr uint32_t kSfaCol = 2 * BN;                    // MXFP8 scale columns after the accumulators
     static constexpr uint32_t kSfbCol = 2 * BN + 8;
@@ -94,6 +100,14 @@ struct ModeTraits {
     static constexpr bool kAMn = MODE == kDownWgrad || MODE == kGateUpWgrad;
     static constexpr bool kBMn = MODE == kDownDgrad || MODE == kGateUpDgrad || MODE == kDownWgrad ||
                                  MODE == kGateUpWgrad;
+    static constexpr bool kCombine = MODE == kDownFwd || MODE == kGateUpDgrad;
+    // Epilogue warps per TMEM lane quadrant: the down dgrad's epilogue (h
+    // loads, dh stores) is latency bound and splits each tile's columns
+    // between two warps; elsewhere one warp takes all of its 32 rows.
+    static constexpr int kSplit = MODE == kDownDgrad ? 2 : 1;
+    static constexpr int kEpiWarps = 4 * kSplit;
+    static constexpr int kGatherWarp0 = kEpiWarp0 + kEpiWarps;  // two more warps: gather, or combine workers
+    static constexpr int kThreads = 32 * (kGatherWarp0 + 2);  // the two last warps idle where unused
 };
 
 // Bytes of one stage that arrive by TMA (the gathered operand arrives by cp.async).
@@ -356,7 +370,7 @@ template <int MODE, int BN, bool MX>
 __device__ void gather_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty, const int *order,
                             volatile int *abort_flag) {
     using C = Cfg<BN, MX>;
-    const int g = threadIdx.x - kGatherWarp0 * 32;
+    const int g = threadIdx.x - ModeTraits<MODE>::kGatherWarp0 * 32;
     const int piece = g & 7;
     const int rg = g >> 3;
     const size_t row_bytes = static_cast<size_t>(a.d) * (MX ? 1 : 2);  // E4M3 codes or bf16
@@ -549,6 +563,7 @@ struct TailList {
     int *count;
     int *done;
     int *claim;
+    int cap;     // entries
 };
 
 // gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up.
@@ -630,51 +645,12 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
     }
 }
 
-// Slot-ordered sum of one finished (token, column tile): the warp reads the k
-// staging rows (coalesced, all slots in flight), writes out[token] and resets
-// the counter for the next call.
 template <int BN>
-__device__ __forceinline__ void combine_token(const GemmArgs &a, int tk, int nt) {
-    constexpr int kCols = BN / 32;  // columns per lane
-    const int lane = threadIdx.x & 31;
-    const int col0 = nt * BN;
-    const __nv_bfloat16 *slot0 = a.stage + static_cast<size_t>(tk) * a.k * a.d + col0 + lane * kCols;
-    float acc[kCols];
-#pragma unroll
-    for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < a.k; ++j) {  // slot order
-        const __nv_bfloat16 *sp = slot0 + static_cast<size_t>(j) * a.d;
-        if constexpr (kCols == 8) {
-            const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(sp));
-            acc[0] += bf16_lo(u.x);
-            acc[1] += bf16_hi(u.x);
-            acc[2] += bf16_lo(u.y);
-            acc[3] += bf16_hi(u.y);
-            acc[4] += bf16_lo(u.z);
-            acc[5] += bf16_hi(u.z);
-            acc[6] += bf16_lo(u.w);
-            acc[7] += bf16_hi(u.w);
-        } else {
-            const uint2 u = __ldcg(reinterpret_cast<const uint2 *>(sp));
-            acc[0] += bf16_lo(u.x);
-            acc[1] += bf16_hi(u.x);
-            acc[2] += bf16_lo(u.y);
-            acc[3] += bf16_hi(u.y);
-        }
-    }
-    __nv_bfloat16 *orow = a.out + static_cast<size_t>(tk) * a.d + col0 + lane * kCols;
-    if constexpr (kCols == 8) {
-        *reinterpret_cast<uint4 *>(orow) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                                      pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-    } else {
-        *reinterpret_cast<uint2 *>(orow) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
-    }
-    if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + nt] = 0;
-}
+__device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *items, int n);
 
-// down forward / gate-up dgrad: stage the slot's row slice, count the slot; a
-// (token, column tile) whose k-th slot lands here is queued for the tail
+// down forward / gate-up dgrad: stage the slot's row slice and count it; a
+// (token, column tile) whose k-th slot lands here is queued for the combine
+// workers
 template <int BN>
 __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                            uint64_t *tempty_acc, uint8_t *xbuf, const TailList &tail) {
@@ -682,12 +658,13 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
-    __nv_bfloat16 *srow = valid ? a.stage + static_cast<size_t>(p) * a.d + t.nt * BN : nullptr;
+    const int nh = t.nt;
+    __nv_bfloat16 *srow = valid ? a.stage + static_cast<size_t>(p) * a.d + nh * BN : nullptr;
     store_accumulator_bf16<BN>(taddr, xbuf, srow, tempty_acc);
     const int tok = valid ? p / a.k : 0;
     bool last = false;
     fence_acq_rel_gpu();  // this warp's staging rows (ordered by the transposes' __syncwarp) before its counts
-    if (valid) last = atomicAdd(a.cnt + static_cast<size_t>(tok) * a.cnt_stride + t.nt, 1) == a.k - 1;
+    if (valid) last = atomicAdd(a.cnt + static_cast<size_t>(tok) * a.cnt_stride + nh, 1) == a.k - 1;
     unsigned mask = __ballot_sync(0xffffffffu, last);
     if (mask == 0u) return;
     fence_acq_rel_gpu();  // the other slots' staging rows after their counts
@@ -696,34 +673,40 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
     if (lane == 0) base = atomicAdd(tail.count, n_last);
     base = __shfl_sync(0xffffffffu, base, 0);
     const int my = __popc(mask & ((1u << lane) - 1u));
-    if (last && base + my < kTailCap) reinterpret_cast<volatile int *>(tail.items)[base + my] = tok * a.n_tiles + t.nt;
-    // no room left in the tail list: reduce those tokens now
-    if (base + n_last > kTailCap) {
+    const int item = tok * a.n_tiles + nh;
+    if (last && base + my < tail.cap) reinterpret_cast<volatile int *>(tail.items)[base + my] = item;
+    // no room left in the queue: sum those tokens now
+    if (base + n_last > tail.cap) {
         while (mask != 0u) {
             const int src = __ffs(static_cast<int>(mask)) - 1;
             const int idx = __popc(mask & ((1u << src) - 1u)) + (n_last - __popc(mask));
             mask &= mask - 1u;
-            const int tk = __shfl_sync(0xffffffffu, tok, src);
-            if (base + idx >= kTailCap) combine_token<BN>(a, tk, t.nt);
+            const int it = __shfl_sync(0xffffffffu, item, src);
+            if (base + idx >= tail.cap) combine_tokens4<BN>(a, &it, 1);
         }
     }
 }
 
 // Slot-ordered sums of up to four finished (token, column tile) items at once:
 // the loads of eight slots of all four tokens are issued before any is summed,
-// so 32 row pieces per lane are in flight.
+// so 32 row pieces per lane are in flight.  BN columns per item, BN / 32 per
+// lane (8 or 4: a 16- or 8-byte piece).
 template <int BN>
 __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *items, int n) {
-    constexpr int kCols = BN / 32;  // columns per lane: 8 (16 bytes) or 4 (8 bytes)
-    using Piece = typename std::conditional<kCols == 8, uint4, uint2>::type;
+    constexpr int BH = BN;
+    constexpr int kCols = BH / 32;
+    constexpr int kWords = kCols / 2;
+    using Piece = typename std::conditional<kCols == 8, uint4,
+                                            typename std::conditional<kCols == 4, uint2, uint32_t>::type>::type;
     const int lane = threadIdx.x & 31;
+    const int n2 = a.n_tiles;
     const __nv_bfloat16 *base[4];
     float acc[4][kCols];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         const int item = items[u < n ? u : 0];
-        const int tk = item / a.n_tiles, nt = item - tk * a.n_tiles;
-        base[u] = a.stage + static_cast<size_t>(tk) * a.k * a.d + nt * BN + lane * kCols;
+        const int tk = item / n2, nh = item - tk * n2;
+        base[u] = a.stage + static_cast<size_t>(tk) * a.k * a.d + nh * BH + lane * kCols;
 #pragma unroll
         for (int i = 0; i < kCols; ++i) acc[u][i] = 0.f;
     }
@@ -744,7 +727,7 @@ __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *it
                 if (u < n && j0 + jj < a.k) {
                     const uint32_t *w = reinterpret_cast<const uint32_t *>(&pc[jj][u]);
 #pragma unroll
-                    for (int q = 0; q < kCols / 2; ++q) {
+                    for (int q = 0; q < kWords; ++q) {
                         acc[u][2 * q] += bf16_lo(w[q]);
                         acc[u][2 * q + 1] += bf16_hi(w[q]);
                     }
@@ -756,17 +739,13 @@ __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *it
     for (int u = 0; u < 4; ++u) {
         if (u < n) {
             const int item = items[u];
-            const int tk = item / a.n_tiles, nt = item - tk * a.n_tiles;
-            __nv_bfloat16 *orow = a.out + static_cast<size_t>(tk) * a.d + nt * BN + lane * kCols;
-            if constexpr (kCols == 8) {
-                *reinterpret_cast<uint4 *>(orow) =
-                    make_uint4(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
-                               pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
-            } else {
-                *reinterpret_cast<uint2 *>(orow) =
-                    make_uint2(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]));
-            }
-            if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + nt] = 0;  // ready for the next call
+            const int tk = item / n2, nh = item - tk * n2;
+            Piece outv;
+            uint32_t *ow = reinterpret_cast<uint32_t *>(&outv);
+#pragma unroll
+            for (int q = 0; q < kWords; ++q) ow[q] = pack_bf16x2(acc[u][2 * q], acc[u][2 * q + 1]);
+            *reinterpret_cast<Piece *>(a.out + static_cast<size_t>(tk) * a.d + nh * BH + lane * kCols) = outv;
+            if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + nh] = 0;  // ready for the next call
         }
     }
 }
@@ -776,7 +755,7 @@ __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *it
 // been claimed) and sums them.  Every wait is bounded; progress restarts the
 // clock.
 template <int BN>
-__device__ void combine_worker(const GemmArgs &a, const TailList &tail, volatile int *abort_flag) {
+__device__ void combine_worker(const GemmArgs &a, const TailList &tail, volatile int *abort_flag, int n_epi) {
     const int lane = threadIdx.x & 31;
     volatile int *vcount = tail.count, *vdone = tail.done, *vitems = tail.items;
     uint64_t t0 = global_timer_ns();
@@ -787,14 +766,14 @@ __device__ void combine_worker(const GemmArgs &a, const TailList &tail, volatile
         if (lane == 0) {
             lo = atomicAdd(tail.claim, 4);
             bool fail = false;
-            while (lo < kTailCap) {
+            while (lo < tail.cap) {
                 if (*vcount >= lo + 4) {
                     n = 4;
                     break;
                 }
-                if (*vdone == kEpiWarps) {
+                if (*vdone == n_epi) {
                     __threadfence_block();
-                    n = max(0, min(*vcount, kTailCap) - lo);
+                    n = max(0, min(*vcount, tail.cap) - lo);
                     break;
                 }
                 if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) {
@@ -828,7 +807,7 @@ __device__ void combine_worker(const GemmArgs &a, const TailList &tail, volatile
 // down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh.
 // MXFP8: also dh's E4M3 codes and scale atoms along 2I (the gate/up dgrad's K).
 template <int BN, bool MX>
-__device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
+__device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t, int r, int ch, uint32_t taddr,
                                                uint64_t *tempty_acc, uint8_t *xbuf) {
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
@@ -837,8 +816,10 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
     const __nv_bfloat16 *hrow = a.h + static_cast<size_t>(pos) * 2 * a.I + t.nt * BN;
     __nv_bfloat16 *dhrow = a.dh + static_cast<size_t>(pos) * 2 * a.I + t.nt * BN;
     float ds = 0.f;
+    constexpr int kSplit = ModeTraits<kDownDgrad>::kSplit;  // epilogue warps per row
+    constexpr int kMine = BN / 32 / kSplit;                  // 32-column chunks per epilogue warp
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = ch * kMine; c < (ch + 1) * kMine; ++c) {
         uint32_t hg[16], hu[16];
         uint4 cg[4], cu[4];
         warp_load_issue(cg, valid ? hrow + c * 32 : nullptr);
@@ -847,7 +828,7 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
         warp_load_finish(xbuf, cu, hu);
         float G[32];
         tmem_load32_sync(taddr + c * 32, G);
-        if (c + 1 == BN / 32) release_accumulator(tempty_acc);
+        if (c + 1 == (ch + 1) * kMine) release_accumulator(tempty_acc);
         float dg[32], du[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -884,8 +865,8 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
             }
         }
     }
-    a.dpart[static_cast<size_t>(pos) * a.dpart_stride + t.nt] = valid ? ds : 0.f;
-    if (valid && t.nt == 0) {  // counters of the dx scatter that follows
+    a.dpart[static_cast<size_t>(pos) * a.dpart_stride + kSplit * t.nt + ch] = valid ? ds : 0.f;
+    if (valid && t.nt == 0 && ch == 0) {  // counters of the dx scatter that follows
         const int tok = p / a.k;
         for (int c = 0; c < a.cnt_stride; ++c) a.cnt[static_cast<size_t>(tok) * a.cnt_stride + c] = 0;
     }
@@ -897,10 +878,11 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
                                           uint64_t *tempty_acc, uint8_t *xbuf) {
     const int Mtot = MODE == kDownWgrad ? a.d : 2 * a.I;
     const int Ntot = MODE == kDownWgrad ? a.I : a.d;
-    __nv_bfloat16 *row =
-        a.dw + (static_cast<size_t>(t.e) * Mtot + t.mt * kTileM + r) * static_cast<size_t>(Ntot) + t.nt * BN;
+    constexpr int BH = BN;
+    __nv_bfloat16 *row = a.dw + (static_cast<size_t>(t.e) * Mtot + t.mt * kTileM + r) * static_cast<size_t>(Ntot) +
+                         t.nt * BN;
     if (t.nkb > 0) {
-        store_accumulator_bf16<BN>(taddr, xbuf, row, tempty_acc);
+        store_accumulator_bf16<BH>(taddr, xbuf, row, tempty_acc);
         return;
     }
     release_accumulator(tempty_acc);  // an expert without tokens: exact zeros, the accumulator is not read
@@ -908,7 +890,7 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
 #pragma unroll
     for (int i = 0; i < 16; ++i) zero[i] = 0u;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) warp_store_rows(xbuf, zero, row + c * 32);
+    for (int c = 0; c < BH / 32; ++c) warp_store_rows(xbuf, zero, row + c * 32);
 }
 
 template <int MODE, int BN, bool MX>
@@ -916,6 +898,7 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
                               const int *order, uint8_t *xbuf, const TailList &tail, volatile int *abort_flag) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quad = warp & 3;  // TMEM lanes this warp may access: 32*quad .. 32*quad+31
+    const int ch = (warp - kEpiWarp0) >> 2;  // down dgrad: which half of the tile's columns
     const int r = quad * 32 + lane;
     const int total = total_tiles<MODE>(a);
     int local = 0;
@@ -934,7 +917,7 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
         } else if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
             epi_combine<BN>(a, t, r, taddr, &tempty[acc], xbuf, tail);
         } else if constexpr (MODE == kDownDgrad) {
-            epi_down_dgrad<BN, MX>(a, t, r, taddr, &tempty[acc], xbuf);
+            epi_down_dgrad<BN, MX>(a, t, r, ch, taddr, &tempty[acc], xbuf);
         } else {
             epi_wgrad<MODE, BN>(a, t, r, taddr, &tempty[acc], xbuf);
         }
@@ -942,7 +925,7 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
 }
 
 template <int MODE, int BN, bool MX>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmArgs args) {
     using C = Cfg<BN, MX>;
@@ -957,22 +940,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const TailList tail{reinterpret_cast<int *>(smem + C::kTailOffset),
-                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap,
-                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap + 1,
-                        reinterpret_cast<int *>(smem + C::kTailOffset) + kTailCap + 2};
-    constexpr bool kCombine = MODE == kDownFwd || MODE == kGateUpDgrad;
+                        reinterpret_cast<int *>(smem + C::kTailOffset) + C::kTailCap,
+                        reinterpret_cast<int *>(smem + C::kTailOffset) + C::kTailCap + 1,
+                        reinterpret_cast<int *>(smem + C::kTailOffset) + C::kTailCap + 2, C::kTailCap};
+    constexpr bool kCombine = TR::kCombine;
     int *s_count = reinterpret_cast<int *>(smem + C::kOrderOffset);
     int *order = s_count + kMaxExperts;
 
     const int warp = threadIdx.x >> 5;
     if constexpr (kCombine) {
-        for (int i = threadIdx.x; i < kTailCap; i += kThreads) tail.items[i] = -1;
+        for (int i = threadIdx.x; i < C::kTailCap; i += TR::kThreads) tail.items[i] = -1;
     }
     if constexpr (!TR::kMTiled) {  // busiest expert first: rank by padded row count, ties to lower index
-        for (int e = threadIdx.x; e < args.E; e += kThreads)
+        for (int e = threadIdx.x; e < args.E; e += TR::kThreads)
             s_count[e] = __ldg(args.group_start + e + 1) - __ldg(args.group_start + e);
         __syncthreads();
-        for (int e = threadIdx.x; e < args.E; e += kThreads) {
+        for (int e = threadIdx.x; e < args.E; e += TR::kThreads) {
             const int c = s_count[e];
             int rank = 0;
             for (int f = 0; f < args.E; ++f) {
@@ -989,7 +972,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], TR::kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -1015,9 +998,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((threadIdx.x & 31) == 0)
             mma_loop<MODE, BN, MX>(args, smem, full, empty, tfull, tempty, drain, tmem_base, order, abort_flag);
         __syncwarp();
-    } else if (warp < kGatherWarp0) {
+    } else if (warp < TR::kGatherWarp0) {
         epilogue_loop<MODE, BN, MX>(args, tfull, tempty, tmem_base, order,
-                                smem + C::kXposeOffset + (warp - 2) * kXposeBytes, tail, abort_flag);
+                                smem + C::kXposeOffset + (warp - kEpiWarp0) * kXposeBytes, tail, abort_flag);
         if constexpr (kCombine) {  // this warp's queue entries are written: count it as done
             __syncwarp();
             if ((threadIdx.x & 31) == 0) {
@@ -1029,7 +1012,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         gather_loop<MODE, BN, MX>(args, smem, full, empty, order, abort_flag);
     }
     // combine modes: warps 6 and 7 from the start, the others after their loops
-    if constexpr (kCombine) combine_worker<BN>(args, tail, abort_flag);
+    if constexpr (kCombine) combine_worker<BN>(args, tail, abort_flag, TR::kEpiWarps);
 
     tc_fence_before_sync();
     __syncthreads();
@@ -1040,14 +1023,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int MODE, int BN, bool MX>
 cudaError_t launch_one(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
                        cudaStream_t s) {
+    constexpr int kSmem = Cfg<BN, MX>::smem_bytes(ModeTraits<MODE>::kEpiWarps);
     static bool attr_set = false;  // per instantiation; the attribute is per function and process-wide
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN, MX>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN, MX>::kSmemBytes);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    grouped_gemm_kernel<MODE, BN, MX><<<grid, kThreads, Cfg<BN, MX>::kSmemBytes, s>>>(tmA, tmB, args);
+    grouped_gemm_kernel<MODE, BN, MX><<<grid, ModeTraits<MODE>::kThreads, kSmem, s>>>(tmA, tmB, args);
     return cudaGetLastError();
 }
 
