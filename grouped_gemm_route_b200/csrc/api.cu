@@ -634,7 +634,10 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dw = static_cast<__nv_bfloat16 *>(dw_down);
     {
         Launch L(kKindGemmDownWgrad, st);
-        if ((rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st)))) return rc;
+        if ((rc = L.done(gemm_pair_ok(kDownWgrad, pl.bn_i, false, a.m_tiles, grid)
+                             ? launch_gemm_pair(kDownWgrad, a, tm_gs_mn, tm_aw_mn, grid, st)
+                             : launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st))))
+            return rc;
     }
     // b4: gate/up dgrad + ordered scatter-sum into dx
     a.n_tiles = pl.d / pl.bn_d;
@@ -650,7 +653,10 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
     {
         Launch L(kKindGemmGateUpWgrad, st);
-        if ((rc = L.done(launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st)))) return rc;
+        if ((rc = L.done(gemm_pair_ok(kGateUpWgrad, pl.bn_d, false, a.m_tiles, grid)
+                             ? launch_gemm_pair(kGateUpWgrad, a, tm_dh_mn, tm_xs_mn, grid, st)
+                             : launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st))))
+            return rc;
     }
     // b6: dscore (ordered sum of partials) and dlogits
     {

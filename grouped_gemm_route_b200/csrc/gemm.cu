@@ -514,6 +514,18 @@ __device__ __forceinline__ void release_accumulator(uint64_t *tempty_acc) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(tempty_acc);
 }
 
+// CTA pairs: the accumulator barrier is the leader's, whichever CTA releases.
+template <bool PAIR>
+__device__ __forceinline__ void release_acc(uint64_t *tempty_acc) {
+    if constexpr (PAIR) {
+        tc_fence_before_sync();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(cluster_addr(tempty_acc, 0));
+    } else {
+        release_accumulator(tempty_acc);
+    }
+}
+
 // One 32-column chunk of this warp's accumulator rows (fp32 in registers) as
 // bf16 to row (nullptr: skipped).
 __device__ __forceinline__ void store_chunk_bf16(uint8_t *xbuf, const uint32_t (&v)[32], __nv_bfloat16 *row) {
@@ -527,7 +539,7 @@ __device__ __forceinline__ void store_chunk_bf16(uint8_t *xbuf, const uint32_t (
 // row (nullptr: skipped), 32 columns at a time, with the tensor-memory load of
 // chunk c + 1 in flight while chunk c is converted and stored.  Releases the
 // accumulator as soon as its last chunk is in registers.
-template <int BN>
+template <int BN, bool PAIR = false>
 __device__ __forceinline__ void store_accumulator_bf16(uint32_t taddr, uint8_t *xbuf, __nv_bfloat16 *row,
                                                        uint64_t *tempty_acc) {
     uint32_t ra[32], rb[32];
@@ -543,7 +555,7 @@ __device__ __forceinline__ void store_accumulator_bf16(uint32_t taddr, uint8_t *
         if (c + 2 < BN / 32)
             tmem_load32(taddr + (c + 2) * 32, ra);
         else
-            release_accumulator(tempty_acc);
+            release_acc<PAIR>(tempty_acc);
         store_chunk_bf16(xbuf, rb, row != nullptr ? row + (c + 1) * 32 : nullptr);
         if (c + 2 < BN / 32) {
             tmem_load_wait();
@@ -873,7 +885,7 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
 }
 
 // weight gradients: store the tile (zeros for an expert without tokens)
-template <int MODE, int BN>
+template <int MODE, int BN, bool PAIR = false>
 __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                           uint64_t *tempty_acc, uint8_t *xbuf) {
     const int Mtot = MODE == kDownWgrad ? a.d : 2 * a.I;
@@ -882,10 +894,10 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
     __nv_bfloat16 *row = a.dw + (static_cast<size_t>(t.e) * Mtot + t.mt * kTileM + r) * static_cast<size_t>(Ntot) +
                          t.nt * BN;
     if (t.nkb > 0) {
-        store_accumulator_bf16<BH>(taddr, xbuf, row, tempty_acc);
+        store_accumulator_bf16<BH, PAIR>(taddr, xbuf, row, tempty_acc);
         return;
     }
-    release_accumulator(tempty_acc);  // an expert without tokens: exact zeros, the accumulator is not read
+    release_acc<PAIR>(tempty_acc);  // an expert without tokens: exact zeros, the accumulator is not read
     uint32_t zero[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) zero[i] = 0u;
@@ -1020,6 +1032,210 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Weight gradients on CTA pairs (bf16, BN = 256).  A cluster of two CTAs
+// computes one 256 x 256 tile with tcgen05.mma.cta_group::2: each CTA loads
+// its own 128 M rows of A and one half (128 columns) of B, so a CTA moves half
+// the B bytes per MMA it takes part in; six 32 KB stages instead of four of
+// 48 KB.  The leader (rank 0) arms the stage barriers for both CTAs' bytes and
+// issues the MMAs; commits arrive on the barriers of both CTAs; the epilogue
+// warps of both CTAs release an accumulator on the leader's barrier.  No load
+// is multicast.  Every wait is bounded, and both CTAs always reach the final
+// cluster barrier (no early exit), after which the pair frees its tensor
+// memory.
+// ---------------------------------------------------------------------------
+template <int BN>
+struct PairCfg {
+    static constexpr int kBHalfBytes = (BN / 2) * kTileK * 2;  // this CTA's half of a B stage
+    static constexpr int kStageBytes = kABytes + kBHalfBytes;
+    static constexpr int kStages = (192 * 1024) / kStageBytes;
+    static constexpr int kBarOffset = kStages * kStageBytes;
+    static constexpr int kOrderOffset = kBarOffset + 512;
+    static constexpr int kXposeOffset = kOrderOffset + 8 * kMaxExperts;
+    static constexpr int kSmemBytes = kXposeOffset + 4 * kXposeBytes + 1024;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static constexpr uint32_t kTmemCols = 2 * BN;
+};
+
+// Pair tile = (expert rank in LPT order, pair of 128-row M tiles, N tile).
+template <int MODE>
+__device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, const int *order, uint32_t rank) {
+    Tile t;
+    const int mp_tiles = a.m_tiles / 2;
+    const int per = mp_tiles * a.n_tiles;
+    const int er = tile / per;
+    const int rr = tile - er * per;
+    t.e = order[er];
+    const int mp = rr / a.n_tiles;
+    t.nt = rr - mp * a.n_tiles;
+    t.mt = 2 * mp + static_cast<int>(rank);
+    const int gs = __ldg(a.group_start + t.e), ge = __ldg(a.group_start + t.e + 1);
+    t.nkb = (ge - gs) / a.k_elems;
+    t.kpos0 = gs;
+    if (t.e < 0 || t.e >= a.E) {
+        t.e = 0;
+        t.nkb = 0;
+    }
+    return t;
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(256, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const GemmArgs args) {
+    static_assert(MODE == kDownWgrad || MODE == kGateUpWgrad, "pairs serve the weight gradients");
+    using P = PairCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + P::kBarOffset);
+    uint64_t *empty = full + P::kStages;
+    uint64_t *tfull = empty + P::kStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *s_count = reinterpret_cast<int *>(smem + P::kOrderOffset);
+    int *order = s_count + kMaxExperts;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const GemmArgs &a = args;
+
+    // busiest expert first (the same order in both CTAs)
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+        s_count[e] = __ldg(a.group_start + e + 1) - __ldg(a.group_start + e);
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        const int c = s_count[e];
+        int rk = 0;
+        for (int f = 0; f < a.E; ++f) {
+            const int cf = s_count[f];
+            rk += (cf > c || (cf == c && f < e)) ? 1 : 0;
+        }
+        order[rk] = e;
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P::kStages; ++s) {
+            mbar_init(&full[s], 1);   // the leader's producer; both CTAs' bytes
+            mbar_init(&empty[s], 1);  // one commit per use
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 8);  // four epilogue warps in each CTA (leader's barrier)
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, P::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync();  // both CTAs' barriers initialised and tensor memory allocated
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = a.E * (a.m_tiles / 2) * a.n_tiles;
+
+    if (warp == 0) {
+        // ---- producer: this CTA's A rows and B half, counted on the leader's barrier ----
+        int it = 0;
+        bool ok = true;
+        for (int tile = pair; tile < total && ok; tile += npairs) {
+            const Tile t = decode_pair_tile<MODE>(tile, a, order, rank);
+            for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+                const int s = it % P::kStages;
+                const uint32_t ph = static_cast<uint32_t>(it / P::kStages) & 1u;
+                if (!warp_wait(&empty[s], ph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (leader && lane == 0) mbar_arrive_expect_tx(&full[s], 2u * P::kStageBytes);
+                __syncwarp();
+                const uint32_t fb = cluster_addr(&full[s], 0);
+                uint8_t *As = smem + s * P::kStageBytes;
+                uint8_t *Bs = As + kABytes;
+                const int k0 = kb * kTileK;
+                if (lane < 2)  // A: 128 M rows, MN-major, two 64-wide chunks
+                    tma_load_2d_pair(As + lane * kChunkBytes, &tmA, fb, t.mt * kTileM + 64 * lane, t.kpos0 + k0);
+                if (lane >= 2 && lane < 2 + BN / 128)  // this CTA's half of B, MN-major
+                    tma_load_2d_pair(Bs + (lane - 2) * kChunkBytes, &tmB, fb,
+                                     t.nt * BN + static_cast<int>(rank) * (BN / 2) + 64 * (lane - 2), t.kpos0 + k0);
+            }
+        }
+        if (!ok) raise_abort(abort_flag, a.status);
+    } else if (warp == 1) {
+        // ---- MMA (leader, one thread): M = 256 over the pair ----
+        if (leader && lane == 0) {
+            constexpr uint32_t kIdesc = instr_desc_bf16(2 * kTileM, BN, true, true);
+            int it = 0, local = 0;
+            bool ok = true;
+            for (int tile = pair; tile < total && ok; tile += npairs, ++local) {
+                const Tile t = decode_pair_tile<MODE>(tile, a, order, rank);
+                const int acc = local & 1;
+                const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
+                if (!mbar_wait_cluster(&tempty[acc], aph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+                    const int s = it % P::kStages;
+                    const uint32_t ph = static_cast<uint32_t>(it / P::kStages) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_base = smem_u32(smem + s * P::kStageBytes);
+                    const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kTileK / 16; ++kk)
+                        mma_bf16_pair(d_tmem, smem_desc_sw128(a_base + kk * 2048, kMnLbo, kSbo),
+                                      smem_desc_sw128(b_base + kk * 2048, kMnLbo, kSbo), kIdesc,
+                                      (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit_pair(&empty[s], 0x3);  // frees the stage in both CTAs
+                }
+                if (!ok) break;
+                mma_commit_pair(&tfull[acc], 0x3);
+            }
+            if (!ok) {
+                raise_abort(abort_flag, a.status);
+                mma_commit_pair(drain, 0x1);
+                mbar_wait(drain, 0u, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ---- epilogue: this CTA's 128 rows of the tile ----
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        uint8_t *xbuf = smem + P::kXposeOffset + (warp - 2) * kXposeBytes;
+        int local = 0;
+        for (int tile = pair; tile < total; tile += npairs, ++local) {
+            const Tile t = decode_pair_tile<MODE>(tile, a, order, rank);
+            const int acc = local & 1;
+            const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
+            if (!warp_wait(&tfull[acc], aph, abort_flag)) {
+                raise_abort(abort_flag, a.status);
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t taddr =
+                tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
+            epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while its peer may still signal into it
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, P::kTmemCols);
+}
+
 template <int MODE, int BN, bool MX>
 cudaError_t launch_one(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
                        cudaStream_t s) {
@@ -1044,6 +1260,40 @@ cudaError_t launch_mode(int bn, bool mx, const GemmArgs &args, const CUtensorMap
     return cudaErrorInvalidValue;
 }
 
+// Launch of a CTA-pair kernel: clusters of two, as many pairs as the GPU holds
+// at once (capped by the grid the caller offers).
+template <int MODE>
+cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
+                        cudaStream_t s) {
+    using P = PairCfg<256>;
+    auto *fn = grouped_gemm_pair_kernel<MODE, 256>;
+    static int max_pairs = -1;  // per instantiation: resident clusters of two
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = P::kSmemBytes;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_pairs < 0) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3(grid & ~1);
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
+        if (e != cudaSuccess) return e;
+        max_pairs = n;
+    }
+    const int pairs = (grid / 2) < max_pairs ? grid / 2 : max_pairs;
+    if (pairs < 1) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3(2 * pairs);
+    return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, args);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA,
@@ -1056,6 +1306,17 @@ cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, co
         case kDownWgrad: return launch_mode<kDownWgrad>(bn, mx, args, tmA, tmB, grid, s);
         case kGateUpWgrad: return launch_mode<kGateUpWgrad>(bn, mx, args, tmA, tmB, grid, s);
     }
+    return cudaErrorInvalidValue;
+}
+
+bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid) {
+    return !mx && bn == 256 && (mode == kDownWgrad || mode == kGateUpWgrad) && m_tiles % 2 == 0 && grid >= 2;
+}
+
+cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                             int grid, cudaStream_t s) {
+    if (mode == kDownWgrad) return launch_pair<kDownWgrad>(args, tmA, tmB, grid, s);
+    if (mode == kGateUpWgrad) return launch_pair<kGateUpWgrad>(args, tmA, tmB, grid, s);
     return cudaErrorInvalidValue;
 }
 

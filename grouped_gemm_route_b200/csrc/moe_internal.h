@@ -103,6 +103,11 @@ cudaError_t launch_expire_wait(int *status, cudaStream_t s);
 
 cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA,
                         const CUtensorMap &tmB, int grid, cudaStream_t s);
+// Weight gradients on CTA pairs (tcgen05 cta_group::2, bf16, BN = 256): used
+// where gemm_pair_ok holds; same arguments and results as launch_gemm.
+bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid);
+cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                             int grid, cudaStream_t s);
 
 cudaError_t launch_mx_quant_rows(const __nv_bfloat16 *src, int64_t R, int K, uint8_t *dst, uint8_t *sf, int sf_mode,
                                  int I, const int32_t *rows_used, int sms, cudaStream_t s);
