@@ -296,13 +296,13 @@ int run_route(const moe_shape_t *shape, const Plan &pl, const DeviceInfo &dev, c
     int32_t *blk_base = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_base);
     int32_t *cnt = reinterpret_cast<int32_t *>(ws + pl.ws_cnt);
     (void)shape;
-    const int grid = route_fused_grid(static_cast<int>(pl.T), pl.E, pl.k, dev.sms, pl.n_chunks);
+    const int grid = route_fused_grid(logits, static_cast<int>(pl.T), pl.E, pl.k, dev.sms, pl.n_chunks);
     if (grid < 1) return MOE_ERR_LAUNCH;
     Launch L(kKindRouteFused, st);
     return L.done(launch_route_fused(logits, static_cast<int>(pl.T), pl.E, pl.k, saved->topk_idx, saved->topk_w,
                                      blk_hist, blk_base, saved->counts, saved->offsets, saved->group_start,
                                      saved->tile_expert, saved->perm, saved->inv, cnt, pl.cnt_stride, pl.p_cap,
-                                     barrier, status, grid, st));
+                                     barrier, status, dev.sms, grid, st));
 }
 
 GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
@@ -645,7 +645,10 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.out = static_cast<__nv_bfloat16 *>(dx);
     {
         Launch L(kKindGemmGateUpDgrad, st);
-        if ((rc = L.done(launch_gemm(kGateUpDgrad, pl.bn_d, false, a, tm_dh_rows, tm_wgu_mn, grid, st)))) return rc;
+        if ((rc = L.done(gemm_pair_ok(kGateUpDgrad, pl.bn_d, false, 0, grid)
+                             ? launch_gemm_pair(kGateUpDgrad, a, tm_dh_rows, tm_wgu_mn, grid, st)
+                             : launch_gemm(kGateUpDgrad, pl.bn_d, false, a, tm_dh_rows, tm_wgu_mn, grid, st))))
+            return rc;
     }
     // b5: gate/up wgrad  dW_gu[e] = sum_p dh_p (x) x[t]
     a.m_tiles = 2 * pl.I / kTileM;

@@ -123,6 +123,7 @@ struct Tile {
     int nt;     // N tile
     int nkb;    // K blocks
     int kpos0;  // wgrad: first sorted row of the expert's group
+    bool skip;  // CTA pairs: this CTA's M tile lies past its expert's group (computed, not stored)
 };
 
 // Wgrad tiles are walked expert by expert, busiest expert first (`order`, a
@@ -130,6 +131,7 @@ struct Tile {
 template <int MODE>
 __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const int *order) {
     Tile t;
+    t.skip = false;
     if constexpr (ModeTraits<MODE>::kMTiled) {
         t.mt = tile / a.n_tiles;
         t.nt = tile - t.mt * a.n_tiles;
@@ -663,7 +665,7 @@ __device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *it
 // down forward / gate-up dgrad: stage the slot's row slice and count it; a
 // (token, column tile) whose k-th slot lands here is queued for the combine
 // workers
-template <int BN>
+template <int BN, bool PAIR = false>
 __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                            uint64_t *tempty_acc, uint8_t *xbuf, const TailList &tail) {
     const int lane = threadIdx.x & 31;
@@ -672,7 +674,7 @@ __device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, in
     const bool valid = p >= 0 && p < a.T * a.k;
     const int nh = t.nt;
     __nv_bfloat16 *srow = valid ? a.stage + static_cast<size_t>(p) * a.d + nh * BN : nullptr;
-    store_accumulator_bf16<BN>(taddr, xbuf, srow, tempty_acc);
+    store_accumulator_bf16<BN, PAIR>(taddr, xbuf, srow, tempty_acc);
     const int tok = valid ? p / a.k : 0;
     bool last = false;
     fence_acq_rel_gpu();  // this warp's staging rows (ordered by the transposes' __syncwarp) before its counts
@@ -1033,58 +1035,101 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Weight gradients on CTA pairs (bf16, BN = 256).  A cluster of two CTAs
-// computes one 256 x 256 tile with tcgen05.mma.cta_group::2: each CTA loads
-// its own 128 M rows of A and one half (128 columns) of B, so a CTA moves half
-// the B bytes per MMA it takes part in; six 32 KB stages instead of four of
-// 48 KB.  The leader (rank 0) arms the stage barriers for both CTAs' bytes and
-// issues the MMAs; commits arrive on the barriers of both CTAs; the epilogue
-// warps of both CTAs release an accumulator on the leader's barrier.  No load
-// is multicast.  Every wait is bounded, and both CTAs always reach the final
-// cluster barrier (no early exit), after which the pair frees its tensor
+// GEMMs on CTA pairs (bf16, BN = 256): the weight gradients and the gate/up
+// dgrad.  A cluster of two CTAs computes one 256 x 256 tile with
+// tcgen05.mma.cta_group::2: each CTA loads its own 128 M rows of A and one
+// half (128 columns) of B, so a CTA moves half the B bytes per MMA it takes
+// part in; 32 KB stages instead of 48 KB.  The leader (rank 0) arms the stage
+// barriers for both CTAs' bytes and issues the MMAs; commits arrive on the
+// barriers of both CTAs; the epilogue warps of both CTAs release an
+// accumulator on the leader's barrier.  Each CTA's epilogue works on its own
+// 128 rows exactly as in the one-CTA kernel (same functions, same outputs).
+//
+// M-tiled modes pair two consecutive 128-row tiles of one expert (both use the
+// expert's B).  An expert with an odd number of tiles has a last pair whose
+// second tile lies past its group: the peer loads those rows (or zeros past
+// the end of the sorted buffer), the MMA computes them, and the peer's
+// epilogue only releases the accumulator.  Pair rows are numbered expert by
+// expert from a per-CTA table of their starts.
+//
+// No load is multicast.  Every wait is bounded, and both CTAs always reach the
+// final cluster barrier (no early exit), after which the pair frees its tensor
 // memory.
 // ---------------------------------------------------------------------------
-template <int BN>
+template <int MODE, int BN>
 struct PairCfg {
+    using TR = ModeTraits<MODE>;
     static constexpr int kBHalfBytes = (BN / 2) * kTileK * 2;  // this CTA's half of a B stage
     static constexpr int kStageBytes = kABytes + kBHalfBytes;
-    static constexpr int kStages = (192 * 1024) / kStageBytes;
+    static constexpr int kTailCap = TR::kCombine ? 4096 : 0;
+    static constexpr int kOrderBytes = 8 * kMaxExperts;  // wgrads: counts + order; M-tiled: pair-row starts
+    static constexpr int kTailBytes = TR::kCombine ? 4 * (kTailCap + 4) : 0;
+    static constexpr int kXposeTotal = TR::kEpiWarps * kXposeBytes;
+    static constexpr int kFixed = 512 + kOrderBytes + kTailBytes + kXposeTotal + 1024;
+    static constexpr int kFit = (227 * 1024 - kFixed) / kStageBytes;
+    static constexpr int kStages = kFit < 6 ? kFit : 6;
     static constexpr int kBarOffset = kStages * kStageBytes;
     static constexpr int kOrderOffset = kBarOffset + 512;
-    static constexpr int kXposeOffset = kOrderOffset + 8 * kMaxExperts;
-    static constexpr int kSmemBytes = kXposeOffset + 4 * kXposeBytes + 1024;
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static constexpr int kTailOffset = kOrderOffset + kOrderBytes;
+    static constexpr int kXposeOffset = kTailOffset + kTailBytes;
+    static constexpr int kSmemBytes = kXposeOffset + kXposeTotal + 1024;
+    static_assert(kStages >= 4 && kSmemBytes <= 227 * 1024, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = 2 * BN;
 };
 
-// Pair tile = (expert rank in LPT order, pair of 128-row M tiles, N tile).
+// Pair tile.  Wgrads: (expert rank in LPT order, pair of 128-row M tiles, N
+// tile).  M-tiled modes: (pair row, N tile), the pair row's expert found in
+// pstart (pstart[e] = first pair row of expert e, pstart[E] = their number).
 template <int MODE>
-__device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, const int *order, uint32_t rank) {
+__device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, const int *tbl, uint32_t rank) {
     Tile t;
-    const int mp_tiles = a.m_tiles / 2;
-    const int per = mp_tiles * a.n_tiles;
-    const int er = tile / per;
-    const int rr = tile - er * per;
-    t.e = order[er];
-    const int mp = rr / a.n_tiles;
-    t.nt = rr - mp * a.n_tiles;
-    t.mt = 2 * mp + static_cast<int>(rank);
-    const int gs = __ldg(a.group_start + t.e), ge = __ldg(a.group_start + t.e + 1);
-    t.nkb = (ge - gs) / a.k_elems;
-    t.kpos0 = gs;
-    if (t.e < 0 || t.e >= a.E) {
-        t.e = 0;
-        t.nkb = 0;
+    t.skip = false;
+    if constexpr (ModeTraits<MODE>::kMTiled) {
+        const int pr = tile / a.n_tiles;
+        t.nt = tile - pr * a.n_tiles;
+        int lo = 0, hi = a.E;  // the last expert whose first pair row is <= pr
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tbl[mid] <= pr)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        t.e = lo;
+        const int g0 = __ldg(a.group_start + lo) / kTileM, g1 = __ldg(a.group_start + lo + 1) / kTileM;
+        t.mt = g0 + 2 * (pr - tbl[lo]) + static_cast<int>(rank);
+        t.skip = t.mt >= g1;
+        t.nkb = a.num_k_blocks;
+        t.kpos0 = 0;
+    } else {
+        const int mp_tiles = a.m_tiles / 2;
+        const int per = mp_tiles * a.n_tiles;
+        const int er = tile / per;
+        const int rr = tile - er * per;
+        t.e = tbl[er];
+        const int mp = rr / a.n_tiles;
+        t.nt = rr - mp * a.n_tiles;
+        t.mt = 2 * mp + static_cast<int>(rank);
+        const int gs = __ldg(a.group_start + t.e), ge = __ldg(a.group_start + t.e + 1);
+        t.nkb = (ge - gs) / a.k_elems;
+        t.kpos0 = gs;
+        if (t.e < 0 || t.e >= a.E) {
+            t.e = 0;
+            t.nkb = 0;
+        }
     }
     return t;
 }
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const GemmArgs args) {
-    static_assert(MODE == kDownWgrad || MODE == kGateUpWgrad, "pairs serve the weight gradients");
-    using P = PairCfg<BN>;
+    static_assert(MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad,
+                  "the modes where pairs measured faster than one CTA");
+    using P = PairCfg<MODE, BN>;
+    using TR = ModeTraits<MODE>;
+    constexpr bool kCombine = TR::kCombine;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + P::kBarOffset);
@@ -1095,25 +1140,54 @@ __global__ void __launch_bounds__(256, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_count = reinterpret_cast<int *>(smem + P::kOrderOffset);
-    int *order = s_count + kMaxExperts;
+    int *tbl = TR::kMTiled ? s_count : s_count + kMaxExperts;  // pair-row starts, or the expert order
+    const TailList tail{reinterpret_cast<int *>(smem + P::kTailOffset),
+                        reinterpret_cast<int *>(smem + P::kTailOffset) + P::kTailCap,
+                        reinterpret_cast<int *>(smem + P::kTailOffset) + P::kTailCap + 1,
+                        reinterpret_cast<int *>(smem + P::kTailOffset) + P::kTailCap + 2, P::kTailCap};
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const GemmArgs &a = args;
 
-    // busiest expert first (the same order in both CTAs)
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-        s_count[e] = __ldg(a.group_start + e + 1) - __ldg(a.group_start + e);
-    __syncthreads();
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-        const int c = s_count[e];
-        int rk = 0;
-        for (int f = 0; f < a.E; ++f) {
-            const int cf = s_count[f];
-            rk += (cf > c || (cf == c && f < e)) ? 1 : 0;
+    if constexpr (kCombine) {
+        for (int i = threadIdx.x; i < P::kTailCap; i += TR::kThreads) tail.items[i] = -1;
+    }
+    if constexpr (TR::kMTiled) {
+        // pair rows per expert: ceil(tiles / 2), numbered expert by expert (warp 0 scans)
+        if (warp == 0) {
+            int carry = 0;
+            for (int e0 = 0; e0 < a.E; e0 += 32) {
+                const int e = e0 + lane;
+                int np = 0;
+                if (e < a.E)
+                    np = ((__ldg(a.group_start + e + 1) - __ldg(a.group_start + e)) / kTileM + 1) >> 1;
+                int incl = np;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += o;
+                }
+                if (e < a.E) tbl[e] = carry + incl - np;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) tbl[a.E] = carry;
         }
-        order[rk] = e;
+    } else {
+        // busiest expert first (the same order in both CTAs)
+        for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+            s_count[e] = __ldg(a.group_start + e + 1) - __ldg(a.group_start + e);
+        __syncthreads();
+        for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+            const int c = s_count[e];
+            int rk = 0;
+            for (int f = 0; f < a.E; ++f) {
+                const int cf = s_count[f];
+                rk += (cf > c || (cf == c && f < e)) ? 1 : 0;
+            }
+            tbl[rk] = e;
+        }
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < P::kStages; ++s) {
@@ -1122,10 +1196,15 @@ __global__ void __launch_bounds__(256, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 8);  // four epilogue warps in each CTA (leader's barrier)
+            mbar_init(&tempty[i], 2 * TR::kEpiWarps);  // the epilogue warps of both CTAs (leader's barrier)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
+        if constexpr (kCombine) {
+            *tail.count = 0;
+            *tail.done = 0;
+            *tail.claim = 0;
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -1133,17 +1212,17 @@ __global__ void __launch_bounds__(256, 1)
         tmem_relinquish_pair();
     }
     tc_fence_before_sync();
-    cluster_sync();  // both CTAs' barriers initialised and tensor memory allocated
+    cluster_sync();  // both CTAs' tables and barriers initialised and tensor memory allocated
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = a.E * (a.m_tiles / 2) * a.n_tiles;
+    const int total = TR::kMTiled ? tbl[a.E] * a.n_tiles : a.E * (a.m_tiles / 2) * a.n_tiles;
 
     if (warp == 0) {
         // ---- producer: this CTA's A rows and B half, counted on the leader's barrier ----
         int it = 0;
         bool ok = true;
         for (int tile = pair; tile < total && ok; tile += npairs) {
-            const Tile t = decode_pair_tile<MODE>(tile, a, order, rank);
+            const Tile t = decode_pair_tile<MODE>(tile, a, tbl, rank);
             for (int kb = 0; kb < t.nkb; ++kb, ++it) {
                 const int s = it % P::kStages;
                 const uint32_t ph = static_cast<uint32_t>(it / P::kStages) & 1u;
@@ -1157,22 +1236,32 @@ __global__ void __launch_bounds__(256, 1)
                 uint8_t *As = smem + s * P::kStageBytes;
                 uint8_t *Bs = As + kABytes;
                 const int k0 = kb * kTileK;
-                if (lane < 2)  // A: 128 M rows, MN-major, two 64-wide chunks
-                    tma_load_2d_pair(As + lane * kChunkBytes, &tmA, fb, t.mt * kTileM + 64 * lane, t.kpos0 + k0);
-                if (lane >= 2 && lane < 2 + BN / 128)  // this CTA's half of B, MN-major
-                    tma_load_2d_pair(Bs + (lane - 2) * kChunkBytes, &tmB, fb,
-                                     t.nt * BN + static_cast<int>(rank) * (BN / 2) + 64 * (lane - 2), t.kpos0 + k0);
+                const int bcol = t.nt * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B columns
+                if constexpr (TR::kMTiled) {
+                    // A: 128 sorted rows of dh, K-major; B: this CTA's half of W_gate_up[e], MN-major
+                    const int brow = t.e * 2 * a.I + k0;
+                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.mt * kTileM);
+                    if (lane >= 1 && lane < 1 + BN / 128)
+                        tma_load_2d_pair(Bs + (lane - 1) * kChunkBytes, &tmB, fb, bcol + 64 * (lane - 1), brow);
+                } else {
+                    if (lane < 2)  // A: 128 M rows, MN-major, two 64-wide chunks
+                        tma_load_2d_pair(As + lane * kChunkBytes, &tmA, fb, t.mt * kTileM + 64 * lane,
+                                         t.kpos0 + k0);
+                    if (lane >= 2 && lane < 2 + BN / 128)  // this CTA's half of B, MN-major
+                        tma_load_2d_pair(Bs + (lane - 2) * kChunkBytes, &tmB, fb, bcol + 64 * (lane - 2),
+                                         t.kpos0 + k0);
+                }
             }
         }
         if (!ok) raise_abort(abort_flag, a.status);
     } else if (warp == 1) {
         // ---- MMA (leader, one thread): M = 256 over the pair ----
         if (leader && lane == 0) {
-            constexpr uint32_t kIdesc = instr_desc_bf16(2 * kTileM, BN, true, true);
+            constexpr uint32_t kIdesc = instr_desc_bf16(2 * kTileM, BN, TR::kAMn, TR::kBMn);
             int it = 0, local = 0;
             bool ok = true;
             for (int tile = pair; tile < total && ok; tile += npairs, ++local) {
-                const Tile t = decode_pair_tile<MODE>(tile, a, order, rank);
+                const Tile t = decode_pair_tile<MODE>(tile, a, tbl, rank);
                 const int acc = local & 1;
                 const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
                 if (!mbar_wait_cluster(&tempty[acc], aph ^ 1u, abort_flag)) {
@@ -1192,10 +1281,13 @@ __global__ void __launch_bounds__(256, 1)
                     const uint32_t a_base = smem_u32(smem + s * P::kStageBytes);
                     const uint32_t b_base = a_base + kABytes;
 #pragma unroll
-                    for (int kk = 0; kk < kTileK / 16; ++kk)
-                        mma_bf16_pair(d_tmem, smem_desc_sw128(a_base + kk * 2048, kMnLbo, kSbo),
-                                      smem_desc_sw128(b_base + kk * 2048, kMnLbo, kSbo), kIdesc,
-                                      (kb | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kTileK / 16; ++kk) {
+                        const uint64_t ad = TR::kAMn ? smem_desc_sw128(a_base + kk * 2048, kMnLbo, kSbo)
+                                                     : smem_desc_sw128(a_base + kk * 32, 16, kSbo);
+                        const uint64_t bd = TR::kBMn ? smem_desc_sw128(b_base + kk * 2048, kMnLbo, kSbo)
+                                                     : smem_desc_sw128(b_base + kk * 32, 16, kSbo);
+                        mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
                     mma_commit_pair(&empty[s], 0x3);  // frees the stage in both CTAs
                 }
                 if (!ok) break;
@@ -1208,14 +1300,14 @@ __global__ void __launch_bounds__(256, 1)
             }
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp < TR::kGatherWarp0) {
         // ---- epilogue: this CTA's 128 rows of the tile ----
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
-        uint8_t *xbuf = smem + P::kXposeOffset + (warp - 2) * kXposeBytes;
+        uint8_t *xbuf = smem + P::kXposeOffset + (warp - kEpiWarp0) * kXposeBytes;
         int local = 0;
         for (int tile = pair; tile < total; tile += npairs, ++local) {
-            const Tile t = decode_pair_tile<MODE>(tile, a, order, rank);
+            const Tile t = decode_pair_tile<MODE>(tile, a, tbl, rank);
             const int acc = local & 1;
             const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
             if (!warp_wait(&tfull[acc], aph, abort_flag)) {
@@ -1225,9 +1317,24 @@ __global__ void __launch_bounds__(256, 1)
             tc_fence_after_sync();
             const uint32_t taddr =
                 tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-            epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
+            if (t.skip) {
+                release_acc<true>(&tempty[acc]);
+            } else if constexpr (kCombine) {
+                epi_combine<BN, true>(a, t, r, taddr, &tempty[acc], xbuf, tail);
+            } else {
+                epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
+            }
+        }
+        if constexpr (kCombine) {  // this warp's queue entries are written: count it as done
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                atomicAdd(tail.done, 1);
+            }
         }
     }
+    // combine mode: the two last warps from the start, the others after their loops
+    if constexpr (kCombine) combine_worker<BN>(a, tail, abort_flag, TR::kEpiWarps);
 
     tc_fence_before_sync();
     __syncthreads();
@@ -1265,7 +1372,7 @@ cudaError_t launch_mode(int bn, bool mx, const GemmArgs &args, const CUtensorMap
 template <int MODE>
 cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
                         cudaStream_t s) {
-    using P = PairCfg<256>;
+    using P = PairCfg<MODE, 256>;
     auto *fn = grouped_gemm_pair_kernel<MODE, 256>;
     static int max_pairs = -1;  // per instantiation: resident clusters of two
     cudaLaunchAttribute attr[1];
@@ -1274,7 +1381,7 @@ cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUte
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(ModeTraits<MODE>::kThreads);
     cfg.dynamicSmemBytes = P::kSmemBytes;
     cfg.stream = s;
     cfg.attrs = attr;
@@ -1310,14 +1417,19 @@ cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, co
 }
 
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid) {
-    return !mx && bn == 256 && (mode == kDownWgrad || mode == kGateUpWgrad) && m_tiles % 2 == 0 && grid >= 2;
+    if (mx || bn != 256 || grid < 2) return false;
+    if (mode == kDownWgrad || mode == kGateUpWgrad) return m_tiles % 2 == 0;
+    return mode == kGateUpDgrad;
 }
 
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
                              int grid, cudaStream_t s) {
-    if (mode == kDownWgrad) return launch_pair<kDownWgrad>(args, tmA, tmB, grid, s);
-    if (mode == kGateUpWgrad) return launch_pair<kGateUpWgrad>(args, tmA, tmB, grid, s);
-    return cudaErrorInvalidValue;
+    switch (mode) {
+        case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, grid, s);
+        case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, grid, s);
+        case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace moe

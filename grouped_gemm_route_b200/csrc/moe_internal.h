@@ -84,13 +84,16 @@ cudaError_t launch_route_scan(int T, int E, int n_chunks, const int32_t *chunk_c
                               int32_t *counts, int32_t *offsets, int32_t *group_start, int32_t *tile_expert,
                               int32_t *perm, int64_t p_cap, int *status, cudaStream_t s);
 // Fused routing (one cooperative launch; see route.cu).  route_fused_grid
-// returns the grid (all blocks resident, at most n_chunks), 0 on failure.
+// returns the grid (all blocks resident, at most n_chunks), 0 on failure;
+// launch_route_fused takes the same SM count, from which it picks the same
+// kernel configuration.
 size_t route_fused_smem(int E, int k);
-int route_fused_grid(int T, int E, int k, int sms, int n_chunks);
+int route_fused_grid(const float *logits, int T, int E, int k, int sms, int n_chunks);
 cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t *idx, float *w, int32_t *blk_hist,
                                int32_t *blk_base, int32_t *counts, int32_t *offsets, int32_t *group_start,
                                int32_t *tile_expert, int32_t *perm, int32_t *inv, int32_t *cnt, int cnt_per_token,
-                               int64_t p_cap, unsigned *barrier, int *status, int grid, cudaStream_t s);
+                               int64_t p_cap, unsigned *barrier, int *status, int sms, int grid,
+                               cudaStream_t s);
 cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int32_t *chunk_base, int32_t *perm,
                               int32_t *inv, int64_t p_cap, int *status, cudaStream_t s);
 cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
@@ -103,8 +106,9 @@ cudaError_t launch_expire_wait(int *status, cudaStream_t s);
 
 cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA,
                         const CUtensorMap &tmB, int grid, cudaStream_t s);
-// Weight gradients on CTA pairs (tcgen05 cta_group::2, bf16, BN = 256): used
-// where gemm_pair_ok holds; same arguments and results as launch_gemm.
+// GEMMs on CTA pairs (tcgen05 cta_group::2, bf16, BN = 256): the weight
+// gradients and the gate/up dgrad; used where gemm_pair_ok holds, with the same
+// arguments and results as launch_gemm.
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid);
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
                              int grid, cudaStream_t s);

@@ -256,6 +256,7 @@ struct RouteFusedArgs {
     int64_t p_cap;
     unsigned *barrier;  // zero before the launch
     int *status;
+    int lane_stages;    // lane form: ring depth per warp
 };
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
@@ -521,140 +522,264 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
 }
 
 // ---------------------------------------------------------------------------
-// Fused routing, lane-per-token form, for E <= 128 with E a multiple of 4k and
-// k <= 8.  Same phases and the same results as route_fused_kernel; phase 1 and
-// the positions of phase 3 give each lane one token:
-//   * a warp stages 32 consecutive tokens' logits in shared memory (cp.async;
-//     rows padded by 4 words so that one-row-per-lane reads do not conflict),
-//     and each lane turns its row into order keys in place;
-//   * tau = the smallest of k group maxima (k disjoint groups of E/k values):
-//     at least k values are >= tau, so every one of the k largest is; the lane
-//     lists the positions of its values >= tau;
-//   * the listed values go through a sorted insertion into k registers of
-//     (value key, ~expert) -- larger value first, lower expert on ties -- which
-//     leaves the k largest in slot order;
+// Fused routing, lane-per-token form, for E <= 128 with E a multiple of 4k,
+// k <= 8 and 16-byte aligned logits.  Same phases and the same results as
+// route_fused_kernel; phase 1 and the positions of phase 3 give each lane one
+// token:
+//   * each lane copies its token's logit row into shared memory with one bulk
+//     copy (rows padded by 4 words, so that one-row-per-lane reads do not
+//     conflict); a warp's buffers form a ring of `stages` batches of 32 rows,
+//     the next batch in flight while the current one is processed;
+//   * tau, a lower bound on the k-th largest logit: the row is split into NG
+//     disjoint groups of consecutive experts (NG = 2k when E is a multiple of
+//     8k, else k) and tau is the k-th largest group maximum -- k groups have a
+//     maximum >= tau, so at least k logits are >= tau and each of the k
+//     largest is;
+//   * the logits >= tau (a bitmask) are visited in expert order and inserted
+//     into k sorted registers of (order key, expert): a strictly larger key
+//     moves ahead, an equal key stays behind the lower experts already there,
+//     which leaves the k largest in slot order (value descending, lower
+//     expert first on ties);
 //   * weights as in route_fused_kernel, the sum taken in slot order.
 // Positions: per batch of 32 tokens, each expert's set of lanes (a bitmask
 // built with atomicOr) gives a pair's rank among the batch's earlier tokens;
 // the highest of those lanes then advances the warp's running position.
 // ---------------------------------------------------------------------------
-constexpr int kLaneThreads = 256;
-constexpr int kLaneWarps = kLaneThreads / 32;
+constexpr int kLaneMaxWarps = 16;
 constexpr int kLaneMaxE = 128;
 constexpr int kLaneMaxK = 8;
+constexpr size_t kLaneSmemLimit = 227u * 1024u;
+
+// Byte offsets of the lane kernel's shared memory.
+struct LaneSmem {
+    int stride;  // words per staged row
+    size_t bars, wcnt, emask, gst, wsum, total;
+};
+
+__host__ __device__ inline LaneSmem lane_smem_layout(int E, int warps, int stages) {
+    LaneSmem L;
+    L.stride = E + 4;
+    L.bars = static_cast<size_t>(warps) * stages * 32 * L.stride * 4;  // staged rows first
+    L.wcnt = L.bars + static_cast<size_t>(warps) * stages * 8;        // [warps][stages] mbarriers
+    L.emask = L.wcnt + static_cast<size_t>(warps) * E * 4;            // [warps][E] counts, then bases
+    L.gst = L.emask + static_cast<size_t>(warps) * E * 4;             // [warps][E] lane masks
+    L.wsum = L.gst + static_cast<size_t>(E + 1) * 4;                  // [E + 1] group starts
+    L.total = L.wsum + static_cast<size_t>(warps) * 4;                // [warps] scan scratch
+    return L;
+}
 
 __device__ __forceinline__ uint32_t order_key(float v) {
     const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
 }
 
-template <int K>
-__global__ void __launch_bounds__(kLaneThreads, 1) route_lane_kernel(const RouteFusedArgs a) {
-    extern __shared__ __align__(16) uint32_t sm_u[];
-    const int E = a.E, G = gridDim.x, b = blockIdx.x;
+// The k-th largest of g[0 .. NGM*K): the minimum when NGM == 1; for NGM == 2
+// each half is sorted (descending, odd-even transposition) and the k-th
+// largest of two sorted lists A, B is max over i of min(A_i, B_(k-i)), A_i the
+// i-th largest of A and A_0 = +inf.
+template <int K, int NGM>
+__device__ __forceinline__ float kth_largest(float (&g)[NGM * K]) {
+    if constexpr (NGM == 1) {
+        float t = g[0];
+#pragma unroll
+        for (int j = 1; j < K; ++j) t = fminf(t, g[j]);
+        return t;
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int r = 0; r < K; ++r) {
+#pragma unroll
+                for (int i = h * K + (r & 1); i + 1 < (h + 1) * K; i += 2) {
+                    const float hi = fmaxf(g[i], g[i + 1]), lo = fminf(g[i], g[i + 1]);
+                    g[i] = hi;
+                    g[i + 1] = lo;
+                }
+            }
+        }
+        float t = fmaxf(g[K - 1], g[2 * K - 1]);
+#pragma unroll
+        for (int i = 1; i < K; ++i) t = fmaxf(t, fminf(g[i - 1], g[2 * K - 1 - i]));
+        return t;
+    }
+}
+
+template <int K, int NGM>
+__global__ void __launch_bounds__(kLaneMaxWarps * 32, 1) route_lane_kernel(const RouteFusedArgs a) {
+    extern __shared__ __align__(16) uint8_t sm_b[];
+    constexpr int NG = NGM * K;
+    const int E = a.E, G = gridDim.x, b = blockIdx.x, S = a.lane_stages;
+    const int nw = static_cast<int>(blockDim.x >> 5);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int stride = E + 4;                                   // words per staged row
-    uint32_t *stage = sm_u + warp * 32 * stride;                // [32][stride] this warp's rows
-    uint8_t *lists = reinterpret_cast<uint8_t *>(sm_u + kLaneWarps * 32 * stride) + warp * 32 * E;  // [32][E]
-    int *wcnt = reinterpret_cast<int *>(sm_u + kLaneWarps * 32 * stride + kLaneWarps * 8 * E);     // [warps][E]
-    uint32_t *emask = reinterpret_cast<uint32_t *>(wcnt + kLaneWarps * E);                         // [warps][E]
-    int *gst = reinterpret_cast<int *>(emask + kLaneWarps * E);                                    // [E + 1]
-    int *warp_sums = gst + E + 1;                                                                  // [warps]
+    const LaneSmem L = lane_smem_layout(E, nw, S);
+    const int stride = L.stride;
+    const float *stage = reinterpret_cast<const float *>(sm_b) + static_cast<size_t>(warp) * S * 32 * stride;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_b + L.bars) + warp * S;
+    int *wcnt = reinterpret_cast<int *>(sm_b + L.wcnt);
+    uint32_t *emask = reinterpret_cast<uint32_t *>(sm_b + L.emask);
+    int *gst = reinterpret_cast<int *>(sm_b + L.gst);
+    int *warp_sums = reinterpret_cast<int *>(sm_b + L.wsum);
     const int t0 = static_cast<int>(static_cast<int64_t>(a.T) * b / G);
     const int t1 = static_cast<int>(static_cast<int64_t>(a.T) * (b + 1) / G);
     const int nb = t1 - t0;
-    const int wt0 = t0 + nb * warp / kLaneWarps, wt1 = t0 + nb * (warp + 1) / kLaneWarps;
-    for (int i = threadIdx.x; i < kLaneWarps * E; i += kLaneThreads) {
+    const int wt0 = t0 + nb * warp / nw, wt1 = t0 + nb * (warp + 1) / nw;
+    const int nbatch = (wt1 - wt0 + 31) / 32;
+    const bool vec_k = (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.idx) | reinterpret_cast<uintptr_t>(a.w)) & 15u) == 0;
+    const bool vec_cnt = (a.cnt_per_token % 4 == 0) && (reinterpret_cast<uintptr_t>(a.cnt) & 15u) == 0;
+    for (int i = threadIdx.x; i < nw * E; i += blockDim.x) {
         wcnt[i] = 0;
         emask[i] = 0u;
     }
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
+        fence_barrier_init();
+    }
     __syncthreads();
 
-    // ---- phase 1: top-k, one token per lane ----
-    const int P4 = E / 4, gsz = E / K;
-    uint32_t *myrow = stage + lane * stride;
-    uint8_t *mylist = lists + lane * E;
-    if (lane == 0 && wt0 < wt1)
-        prefetch_l2(a.logits + static_cast<size_t>(wt0) * E,
-                    static_cast<uint32_t>(min(32, wt1 - wt0)) * static_cast<uint32_t>(E) * 4u);
-    for (int tb = wt0; tb < wt1; tb += 32) {
-        const int rows = min(32, wt1 - tb);
-        const float *src = a.logits + static_cast<size_t>(tb) * E;
-        for (int q = lane; q < rows * P4; q += 32) {
-            const int r = q / P4, c4 = q - r * P4;
-            cp_async_16(smem_u32(stage + r * stride + 4 * c4), src + static_cast<size_t>(r) * E + 4 * c4);
-        }
-        if (lane == 0 && tb + 32 < wt1)  // the next batch's rows on their way to L2
-            prefetch_l2(src + static_cast<size_t>(32) * E,
-                        static_cast<uint32_t>(min(32, wt1 - tb - 32)) * static_cast<uint32_t>(E) * 4u);
-        cp_async_wait_all();
+    // Batch `it` of this warp (32 rows from token wt0 + 32*it) into ring slot it % S.
+    auto issue = [&](int it) {
+        const int tb = wt0 + 32 * it, rows = min(32, wt1 - tb), s = it % S;
+        fence_proxy_async_smem();  // this lane's earlier reads of the slot come first
         __syncwarp();
-        const bool live = lane < rows;
-        int n = 0;
-        if (live) {
-            uint32_t tau = 0xFFFFFFFFu;
-#pragma unroll 1
-            for (int g = 0; g < K; ++g) {
-                uint32_t gm = 0u;
-                for (int i = g * gsz; i < (g + 1) * gsz; i += 4) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(myrow + i);
-                    const uint4 kk = make_uint4(order_key(__uint_as_float(v.x)), order_key(__uint_as_float(v.y)),
-                                                order_key(__uint_as_float(v.z)), order_key(__uint_as_float(v.w)));
-                    *reinterpret_cast<uint4 *>(myrow + i) = kk;
-                    gm = max(gm, max(max(kk.x, kk.y), max(kk.z, kk.w)));
-                }
-                tau = min(tau, gm);
-            }
-            for (int i = 0; i < E; i += 4) {
-                const uint4 kk = *reinterpret_cast<const uint4 *>(myrow + i);
-                if (kk.x >= tau) mylist[n++] = static_cast<uint8_t>(i);
-                if (kk.y >= tau) mylist[n++] = static_cast<uint8_t>(i + 1);
-                if (kk.z >= tau) mylist[n++] = static_cast<uint8_t>(i + 2);
-                if (kk.w >= tau) mylist[n++] = static_cast<uint8_t>(i + 3);
-            }
+        if (lane == 0) mbar_arrive_expect_tx(&bar[s], static_cast<uint32_t>(rows * E) * 4u);
+        __syncwarp();
+        if (lane < rows)
+            bulk_load(const_cast<float *>(stage) + static_cast<size_t>(s * 32 + lane) * stride,
+                      a.logits + static_cast<size_t>(tb + lane) * E, static_cast<uint32_t>(E) * 4u, &bar[s]);
+    };
+
+    // ---- phase 1: top-k, one token per lane ----
+    const int E4 = E / 4, gq = E / (4 * NG);  // float4s per row, per group
+    bool wait_ok = true;
+    int it = 0;
+    for (int p = 0; p < S && p < nbatch; ++p) issue(p);
+    for (; it < nbatch; ++it) {
+        const int tb = wt0 + 32 * it, rows = min(32, wt1 - tb), s = it % S;
+        const bool arrived = mbar_wait(&bar[s], static_cast<uint32_t>(it / S) & 1u, nullptr);
+        if (!__all_sync(0xffffffffu, arrived)) {
+            wait_ok = false;
+            break;
         }
-        uint64_t top[K];
+        const bool live = lane < rows;
+        const float4 *r4 = reinterpret_cast<const float4 *>(stage + static_cast<size_t>(s * 32 + lane) * stride);
+        uint64_t mlo = 0ull, mhi = 0ull;  // logits >= tau: experts 0..63, 64..127
+        int ncand = 0;
+        if (live) {
+            float gm[NG];
 #pragma unroll
-        for (int j = 0; j < K; ++j) top[j] = 0ull;
-        const int nmax = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(n));
-        for (int c = 0; c < nmax; ++c) {
-            if (c < n) {
-                const int i = mylist[c];
-                const uint64_t x = (static_cast<uint64_t>(myrow[i]) << 32) | static_cast<uint32_t>(~i);
-                if (x > top[K - 1]) {
+            for (int g = 0; g < NG; ++g) {
+                float mx = -INFINITY;
 #pragma unroll
-                    for (int j = K - 1; j > 0; --j) top[j] = x > top[j - 1] ? top[j - 1] : (x > top[j] ? x : top[j]);
-                    top[0] = x > top[0] ? x : top[0];
+                for (int q = 0; q < 32 / NG; ++q) {
+                    if (q < gq) {
+                        const float4 v = r4[g * gq + q];
+                        mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+                    }
                 }
+                gm[g] = mx;
+            }
+            const float tau = kth_largest<K, NGM>(gm);
+            uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (8 * wd + j < E4) {
+                        const float4 v = r4[8 * wd + j];
+                        uint32_t bits = 0u;
+                        if (v.x >= tau) bits |= 1u << (4 * j);
+                        if (v.y >= tau) bits |= 2u << (4 * j);
+                        if (v.z >= tau) bits |= 4u << (4 * j);
+                        if (v.w >= tau) bits |= 8u << (4 * j);
+                        m[wd] |= bits;
+                    }
+                }
+            }
+            mlo = (static_cast<uint64_t>(m[1]) << 32) | m[0];
+            mhi = (static_cast<uint64_t>(m[3]) << 32) | m[2];
+            ncand = __popcll(mlo) + __popcll(mhi);
+        }
+        uint32_t tk[K];
+        int ti[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            tk[j] = 0u;  // below every real key
+            ti[j] = 0;
+        }
+        const float *row = reinterpret_cast<const float *>(r4);
+        const int cmax = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(ncand)));
+        for (int c = 0; c < cmax; ++c) {
+            if (c < ncand) {
+                const bool in_lo = mlo != 0ull;
+                const uint64_t cur = in_lo ? mlo : mhi;
+                const int e = __ffsll(static_cast<long long>(cur)) - 1 + (in_lo ? 0 : 64);
+                const uint64_t rest = cur & (cur - 1ull);
+                if (in_lo)
+                    mlo = rest;
+                else
+                    mhi = rest;
+                const uint32_t xk = order_key(row[e]);
+                bool gt[K];
+#pragma unroll
+                for (int j = 0; j < K; ++j) gt[j] = xk > tk[j];
+#pragma unroll
+                for (int j = K - 1; j > 0; --j) {
+                    tk[j] = gt[j - 1] ? tk[j - 1] : (gt[j] ? xk : tk[j]);
+                    ti[j] = gt[j - 1] ? ti[j - 1] : (gt[j] ? e : ti[j]);
+                }
+                tk[0] = gt[0] ? xk : tk[0];
+                ti[0] = gt[0] ? e : ti[0];
             }
         }
         if (live) {
             const int t = tb + lane;
-            const float m = topk_value(static_cast<uint32_t>(top[0] >> 32));
+            const float mx = topk_value(tk[0]);
             float p[K], sum = 0.f;
-            int e[K];
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                e[j] = static_cast<int>(~static_cast<uint32_t>(top[j]));
-                p[j] = expf(topk_value(static_cast<uint32_t>(top[j] >> 32)) - m);
+                p[j] = expf(topk_value(tk[j]) - mx);
                 sum += p[j];  // slot order
             }
+            float wv[K];
+#pragma unroll
+            for (int j = 0; j < K; ++j) wv[j] = p[j] / sum;
             int32_t *irow = a.idx + static_cast<size_t>(t) * K;
             float *wrow = a.w + static_cast<size_t>(t) * K;
+            if (vec_k) {
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-                irow[j] = e[j];
-                wrow[j] = p[j] / sum;
-                atomicAdd(&wcnt[warp * E + e[j]], 1);
+                for (int j = 0; j < K; j += 4) {
+                    *reinterpret_cast<int4 *>(irow + j) = make_int4(ti[j], ti[j + 1], ti[j + 2], ti[j + 3]);
+                    *reinterpret_cast<float4 *>(wrow + j) = make_float4(wv[j], wv[j + 1], wv[j + 2], wv[j + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    irow[j] = ti[j];
+                    wrow[j] = wv[j];
+                }
             }
-            for (int cc = 0; cc < a.cnt_per_token; ++cc) a.cnt[static_cast<size_t>(t) * a.cnt_per_token + cc] = 0;
+#pragma unroll
+            for (int j = 0; j < K; ++j) atomicAdd(&wcnt[warp * E + ti[j]], 1);
+            int32_t *crow = a.cnt + static_cast<size_t>(t) * a.cnt_per_token;
+            if (vec_cnt) {
+                for (int cc = 0; cc < a.cnt_per_token; cc += 4)
+                    *reinterpret_cast<int4 *>(crow + cc) = make_int4(0, 0, 0, 0);
+            } else {
+                for (int cc = 0; cc < a.cnt_per_token; ++cc) crow[cc] = 0;
+            }
         }
         __syncwarp();
+        if (it + S < nbatch) issue(it + S);
+    }
+    if (!wait_ok) {
+        if (lane == 0) report_status(a.status, kStatusTimeout);
+        for (int q = it; q < it + S && q < nbatch; ++q)  // copies still in flight land before the exit
+            (void)mbar_wait(&bar[q % S], static_cast<uint32_t>(q / S) & 1u, nullptr);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kLaneThreads) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int sum = 0;
-        for (int q = 0; q < kLaneWarps; ++q) sum += wcnt[q * E + e];
+        for (int q = 0; q < nw; ++q) sum += wcnt[q * E + e];
         a.blk_hist[static_cast<size_t>(b) * E + e] = sum;
     }
     if (!grid_barrier(a.barrier, G, a.status)) return;
@@ -665,7 +790,8 @@ __global__ void __launch_bounds__(kLaneThreads, 1) route_lane_kernel(const Route
 
     // ---- phase 3: group starts, tile table, padding, positions ----
     if (!route_group_layout(a, gst, warp_sums)) return;
-    route_warp_bases(a, wcnt, gst, kLaneWarps);
+    route_warp_bases(a, wcnt, gst, nw);
+    if (!wait_ok) return;  // this warp's idx rows are incomplete
     bool bad = false;
     const uint32_t below = (1u << lane) - 1u;
     int *run = wcnt + warp * E;
@@ -674,10 +800,23 @@ __global__ void __launch_bounds__(kLaneThreads, 1) route_lane_kernel(const Route
         const int t = tb + lane;
         const bool live = t < wt1;
         int e[K];
+        if (live) {
+            const int32_t *irow = a.idx + static_cast<size_t>(t) * K;  // written by this thread in phase 1
+            if (vec_k) {
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
-            e[j] = live ? a.idx[static_cast<size_t>(t) * K + j] : 0;  // written by this thread in phase 1
-            if (live) atomicOr(&msk[e[j]], 1u << lane);
+                for (int j = 0; j < K; j += 4) {
+                    const int4 v = *reinterpret_cast<const int4 *>(irow + j);
+                    e[j] = v.x;
+                    e[j + 1] = v.y;
+                    e[j + 2] = v.z;
+                    e[j + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < K; ++j) e[j] = irow[j];
+            }
+#pragma unroll
+            for (int j = 0; j < K; ++j) atomicOr(&msk[e[j]], 1u << lane);
         }
         __syncwarp();
         if (live) {
@@ -709,25 +848,46 @@ __global__ void __launch_bounds__(kLaneThreads, 1) route_lane_kernel(const Route
     if (bad) report_status(a.status, kStatusBadIndex);
 }
 
-size_t route_lane_smem(int E) {
-    return (static_cast<size_t>(kLaneWarps) * 32 * (E + 4) + static_cast<size_t>(kLaneWarps) * 8 * E +
-            2 * static_cast<size_t>(kLaneWarps) * E + E + 1 + kLaneWarps) *
-           4;
+// Warps and ring depth of the lane kernel, as many warps as fit in shared
+// memory (at least E / 32, since phase 3 gives one expert to each thread).
+// With at most 384 tokens per SM a warp has one or two batches, and a ring of
+// two batches per warp (fewer, fuller warps) finishes first; with more tokens
+// one batch per warp and twice the warps hide more latency (measured at E =
+// 128: 16 K tokens 24.6 against 26.6 us, 512 K tokens 185 against 155 us).
+struct LaneCfg {
+    int warps, stages;
+    size_t smem;
+};
+
+LaneCfg lane_cfg(int E, int T, int sms) {
+    LaneCfg c{kLaneMaxWarps, static_cast<int64_t>(T) <= 384ll * sms ? 2 : 1, 0};
+    while (c.warps > 1 && lane_smem_layout(E, c.warps, c.stages).total > kLaneSmemLimit) --c.warps;
+    c.smem = lane_smem_layout(E, c.warps, c.stages).total;
+    return c;
 }
 
-bool route_lane_ok(int E, int k) { return E <= kLaneMaxE && k <= kLaneMaxK && E % (4 * k) == 0; }
+bool route_lane_ok(int E, int k, const float *logits) {
+    return E <= kLaneMaxE && k >= 1 && k <= kLaneMaxK && E % (4 * k) == 0 &&
+           (reinterpret_cast<uintptr_t>(logits) & 15u) == 0 && lane_cfg(E, 0, 1).warps * 32 >= E &&
+           lane_cfg(E, 1 << 30, 1).warps * 32 >= E;
+}
 
-const void *route_lane_fn(int k) {
+template <int NGM>
+const void *route_lane_fn_k(int k) {
     switch (k) {
-        case 1: return reinterpret_cast<const void *>(route_lane_kernel<1>);
-        case 2: return reinterpret_cast<const void *>(route_lane_kernel<2>);
-        case 3: return reinterpret_cast<const void *>(route_lane_kernel<3>);
-        case 4: return reinterpret_cast<const void *>(route_lane_kernel<4>);
-        case 5: return reinterpret_cast<const void *>(route_lane_kernel<5>);
-        case 6: return reinterpret_cast<const void *>(route_lane_kernel<6>);
-        case 7: return reinterpret_cast<const void *>(route_lane_kernel<7>);
-        default: return reinterpret_cast<const void *>(route_lane_kernel<8>);
+        case 1: return reinterpret_cast<const void *>(route_lane_kernel<1, NGM>);
+        case 2: return reinterpret_cast<const void *>(route_lane_kernel<2, NGM>);
+        case 3: return reinterpret_cast<const void *>(route_lane_kernel<3, NGM>);
+        case 4: return reinterpret_cast<const void *>(route_lane_kernel<4, NGM>);
+        case 5: return reinterpret_cast<const void *>(route_lane_kernel<5, NGM>);
+        case 6: return reinterpret_cast<const void *>(route_lane_kernel<6, NGM>);
+        case 7: return reinterpret_cast<const void *>(route_lane_kernel<7, NGM>);
+        default: return reinterpret_cast<const void *>(route_lane_kernel<8, NGM>);
     }
+}
+
+const void *route_lane_fn(int E, int k) {
+    return E % (8 * k) == 0 ? route_lane_fn_k<2>(k) : route_lane_fn_k<1>(k);
 }
 
 constexpr int kBwdThreads = 256;
@@ -875,15 +1035,14 @@ cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t 
     return cudaGetLastError();
 }
 
-int route_fused_grid(int T, int E, int k, int sms, int n_chunks) {
-    (void)T;
+int route_fused_grid(const float *logits, int T, int E, int k, int sms, int n_chunks) {
     int per_sm = 0;
     cudaError_t e;
-    if (route_lane_ok(E, k)) {
-        const void *fn = route_lane_fn(k);
-        const size_t smem = route_lane_smem(E);
-        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kLaneThreads, smem);
+    if (route_lane_ok(E, k, logits)) {
+        const void *fn = route_lane_fn(E, k);
+        const LaneCfg c = lane_cfg(E, T, sms);
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, c.warps * 32, c.smem);
     } else {
         const int nv = (E + 31) / 32;
         const size_t smem = route_fused_smem(E, k);
@@ -911,13 +1070,15 @@ size_t route_fused_smem(int E, int k) {
 cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t *idx, float *w, int32_t *blk_hist,
                                int32_t *blk_base, int32_t *counts, int32_t *offsets, int32_t *group_start,
                                int32_t *tile_expert, int32_t *perm, int32_t *inv, int32_t *cnt, int cnt_per_token,
-                               int64_t p_cap, unsigned *barrier, int *status, int grid, cudaStream_t s) {
+                               int64_t p_cap, unsigned *barrier, int *status, int sms, int grid, cudaStream_t s) {
     RouteFusedArgs a{logits, T, E, k, idx, w, blk_hist, blk_base, counts, offsets, group_start,
-                     tile_expert, perm, inv, cnt, cnt_per_token, p_cap, barrier, status};
+                     tile_expert, perm, inv, cnt, cnt_per_token, p_cap, barrier, status, 0};
     void *params[] = {&a};
-    if (route_lane_ok(E, k))
-        return cudaLaunchCooperativeKernel(route_lane_fn(k), dim3(grid), dim3(kLaneThreads), params,
-                                           route_lane_smem(E), s);
+    if (route_lane_ok(E, k, logits)) {
+        const LaneCfg c = lane_cfg(E, T, sms);
+        a.lane_stages = c.stages;
+        return cudaLaunchCooperativeKernel(route_lane_fn(E, k), dim3(grid), dim3(c.warps * 32), params, c.smem, s);
+    }
     const size_t smem = route_fused_smem(E, k);
     const int nv = (E + 31) / 32;
     const void *fn = nv <= 1   ? reinterpret_cast<const void *>(route_fused_kernel<1>)

@@ -12,6 +12,7 @@ import torch
 
 from helpers import TOL_BF16, check_routing, f64, make, normwise, run_layer, sorted_rows
 from oracle import moe_oracle as O
+from grouped_gemm_route_b200 import moe as M
 
 pytestmark = pytest.mark.gpu
 
@@ -134,3 +135,23 @@ def test_qwen3_30b_skewed_routing_sampled():
 
 def test_qwen3_235b_shape_sampled():
     _sampled_check("qwen3_235b_a22b", n_tokens=24)
+
+
+@pytest.mark.parametrize("max_sms", [7, 3])
+def test_results_do_not_depend_on_the_grid(max_sms):
+    # every tile (or CTA-pair tile) is computed whole by one CTA or pair and every
+    # reduction has a fixed order, so a layer on a few SMs gives the same bits
+    cfg, inp = make(dict(T=700, d=512, E=12, k=3, I=256), seed=13)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    x, lg, wgu, wd, gout = (inp[n].cuda() for n in ("x", "logits", "wgu", "wd", "gout"))
+    outs = []
+    for sms in (0, max_sms):
+        layer = M.MoELayer(T, d, E, k, I, max_sms=sms)
+        o = layer.forward(x, lg, wgu, wd).clone()
+        g = {n: t.clone() for n, t in layer.backward(gout, x, wgu, wd).items()}
+        torch.cuda.synchronize()
+        assert layer.status() == 0
+        outs.append((o, g))
+    assert torch.equal(outs[0][0], outs[1][0])
+    for n in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
+        assert torch.equal(outs[0][1][n], outs[1][1][n]), n

@@ -1,7 +1,8 @@
 """Routing alone (moe_route) against the oracle, bit-exact, on shapes that
 reach both routing kernels: the lane-per-token form (E <= 128, E a multiple of
-4k, k <= 8) and the warp-per-token form (everything else), with and without
-tied logits, and on token counts that leave ragged per-warp batches."""
+4k, k <= 8; both of its ring depths and both group counts) and the
+warp-per-token form (everything else), with and without tied logits, and on
+token counts that leave ragged per-warp batches."""
 import numpy as np
 import pytest
 import torch
@@ -17,6 +18,11 @@ pytestmark = pytest.mark.gpu
     (16384, 128, 8, False),  # lane form at the workload's size
     (2048, 96, 4, False),    # lane form, E not a power of two
     (77, 32, 8, True),       # lane form, fewer tokens than one warp batch per warp
+    (50000, 128, 8, False),  # lane form, two-batch ring per warp, both slots used
+    (70000, 128, 8, True),   # lane form, one batch per warp (more than 384 tokens per SM), ties
+    (131072, 128, 8, False), # lane form, one batch per warp, several batches each
+    (3000, 120, 5, True),    # lane form, 2k groups of 12 experts
+    (3000, 64, 8, False),    # lane form, 2k groups of 4 experts
     (3000, 160, 8, False),   # warp form: E > 128
     (777, 20, 3, True),      # warp form: E not a multiple of 4k
     (4096, 64, 6, False),    # warp form: 64 is not a multiple of 24
