@@ -77,8 +77,8 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     off = align_up(off + 16);
     p->ws_cnt = off;
     off = align_up(off + static_cast<size_t>(s->T) * p->cnt_stride * 4);
-    p->ws_stage = off;
-    off = align_up(off + static_cast<size_t>(P) * s->d * 2);
+    p->ws_stage = off;  // combine staging [P, d]; before it, the bf16 forward's sorted x [p_cap, d]
+    off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
     const size_t common = off;
     p->ws_chunk_counts = off;
     off = align_up(off + static_cast<size_t>(p->n_chunks) * s->E * 4);
@@ -262,7 +262,7 @@ struct Launch {
 const char *kKindNames[kNumKernelKinds] = {
     "route_topk",       "route_scan",       "route_perm",           "gemm_gateup_fwd",      "gemm_down_fwd_combine",
     "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd",
-    "sort_rows", "mx_quant", "route_fused"};
+    "sort_rows", "mx_quant", "route_fused", "sort_x"};
 
 struct Saved {
     int32_t *idx;
@@ -400,9 +400,27 @@ int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, 
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.I / 128;
     a.num_k_blocks = pl.d / kTileK;
+    const int grid = grid_for(shape, dev);
+    if (gemm_pair_ok(kGateUpFwd, 256, false, 0, grid)) {
+        // x in the sorted layout (in the combine's staging space, unused until the
+        // down GEMM), then plain TMA tiles on CTA pairs
+        __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_stage);
+        {
+            Launch L(kKindSortX, st);
+            const int rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
+                                                   static_cast<int>(pl.T), pl.d,
+                                                   static_cast<const __nv_bfloat16 *>(x), nullptr, xs, nullptr,
+                                                   false, dev.sms, st));
+            if (rc) return rc;
+        }
+        CUtensorMap tm_xs;
+        if (!make_map(&tm_xs, xs, pl.p_cap, pl.d, 128)) return MOE_ERR_LAUNCH;
+        Launch L(kKindGemmGateUpFwd, st);
+        return L.done(launch_gemm_pair(kGateUpFwd, a, tm_xs, tm_wgu, grid, st));
+    }
     a.gsrc = static_cast<const __nv_bfloat16 *>(x);  // token rows gathered through perm (A operand)
     Launch L(kKindGemmGateUpFwd, st);
-    return L.done(launch_gemm(kGateUpFwd, 256, false, a, tm_wgu, tm_wgu, grid_for(shape, dev), st));
+    return L.done(launch_gemm(kGateUpFwd, 256, false, a, tm_wgu, tm_wgu, grid, st));
 }
 
 // MXFP8 backward after sort_rows: every GEMM operand quantised along that
@@ -611,7 +629,8 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
         if ((rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
                                           static_cast<int>(pl.T), pl.d,
                                           static_cast<const __nv_bfloat16 *>(x),
-                                          static_cast<const __nv_bfloat16 *>(grad_out), xs, gs, dev.sms, st))))
+                                          static_cast<const __nv_bfloat16 *>(grad_out), xs, gs, true, dev.sms,
+                                          st))))
             return rc;
     }
     if (pl.mx) {

@@ -618,7 +618,7 @@ __device__ __forceinline__ void gateup_chunk(const GemmArgs &a, const Tile &t, i
 }
 
 // The tensor-memory loads of chunk c + 1 are in flight while chunk c is worked on.
-template <int BN, bool MX>
+template <int BN, bool MX, bool PAIR = false>
 __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                                uint64_t *tempty_acc, uint8_t *xbuf) {
     constexpr int kHalf = BN / 2;
@@ -648,7 +648,7 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
             tmem_load32(taddr + (c + 2) * 32, ga);
             tmem_load32(taddr + kHalf + (c + 2) * 32, ua);
         } else {
-            release_accumulator(tempty_acc);  // TMEM no longer needed
+            release_acc<PAIR>(tempty_acc);  // TMEM no longer needed
         }
         gateup_chunk<BN, MX>(a, t, r, pos, valid, wv, c + 1, gb, ub, hrow, arow, xbuf);
         if (c + 2 < kChunks) {
@@ -1035,8 +1035,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// GEMMs on CTA pairs (bf16, BN = 256): the weight gradients and the gate/up
-// dgrad.  A cluster of two CTAs computes one 256 x 256 tile with
+// GEMMs on CTA pairs (bf16, BN = 256): the gate/up forward (on x gathered into
+// the sorted layout first), the gate/up dgrad and the weight gradients.  A cluster of two CTAs computes one 256 x 256 tile with
 // tcgen05.mma.cta_group::2: each CTA loads its own 128 M rows of A and one
 // half (128 columns) of B, so a CTA moves half the B bytes per MMA it takes
 // part in; 32 KB stages instead of 48 KB.  The leader (rank 0) arms the stage
@@ -1125,7 +1125,7 @@ template <int MODE, int BN>
 __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const GemmArgs args) {
-    static_assert(MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad,
+    static_assert(MODE == kGateUpFwd || MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad,
                   "the modes where pairs measured faster than one CTA");
     using P = PairCfg<MODE, BN>;
     using TR = ModeTraits<MODE>;
@@ -1237,7 +1237,15 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 uint8_t *Bs = As + kABytes;
                 const int k0 = kb * kTileK;
                 const int bcol = t.nt * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B columns
-                if constexpr (TR::kMTiled) {
+                if constexpr (MODE == kGateUpFwd) {
+                    // A: 128 sorted rows of x; B: the leader loads the tile's 128 gate rows of
+                    // W_gate_up[e], the peer its 128 up rows (both K-major), so that accumulator
+                    // columns [0, 128) hold gate and [128, 256) up, as in the one-CTA kernel
+                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.mt * kTileM);
+                    if (lane == 1)
+                        tma_load_2d_pair(Bs, &tmB, fb, k0,
+                                         t.e * 2 * a.I + static_cast<int>(rank) * a.I + t.nt * (BN / 2));
+                } else if constexpr (TR::kMTiled) {
                     // A: 128 sorted rows of dh, K-major; B: this CTA's half of W_gate_up[e], MN-major
                     const int brow = t.e * 2 * a.I + k0;
                     if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.mt * kTileM);
@@ -1319,6 +1327,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
             if (t.skip) {
                 release_acc<true>(&tempty[acc]);
+            } else if constexpr (MODE == kGateUpFwd) {
+                epi_gateup_fwd<BN, false, true>(a, t, r, taddr, &tempty[acc], xbuf);
             } else if constexpr (kCombine) {
                 epi_combine<BN, true>(a, t, r, taddr, &tempty[acc], xbuf, tail);
             } else {
@@ -1419,7 +1429,7 @@ cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, co
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid) {
     if (mx || bn != 256 || grid < 2) return false;
     if (mode == kDownWgrad || mode == kGateUpWgrad) return m_tiles % 2 == 0;
-    return mode == kGateUpDgrad;
+    return mode == kGateUpFwd || mode == kGateUpDgrad;
 }
 
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
@@ -1427,6 +1437,7 @@ cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensor
     switch (mode) {
         case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, grid, s);
         case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, grid, s);
+        case kGateUpFwd: return launch_pair<kGateUpFwd>(args, tmA, tmB, grid, s);
         case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, grid, s);
         default: return cudaErrorInvalidValue;
     }

@@ -35,6 +35,7 @@ enum KernelKind : int {
     kKindSortRows,
     kKindMxQuant,
     kKindRouteFused,
+    kKindSortX,
     kNumKernelKinds
 };
 
@@ -96,9 +97,11 @@ cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t
                                cudaStream_t s);
 cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int32_t *chunk_base, int32_t *perm,
                               int32_t *inv, int64_t p_cap, int *status, cudaStream_t s);
+// x (and grad_out, when g is not null) in the expert-sorted layout; zero_pad
+// also zeroes each group's padding rows (the wgrads sum over them).
 cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
                              int T, int d, const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs,
-                             __nv_bfloat16 *gs, int sms, cudaStream_t s);
+                             __nv_bfloat16 *gs, bool zero_pad, int sms, cudaStream_t s);
 cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t *idx, const int32_t *inv,
                              const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s);
 

@@ -923,18 +923,21 @@ __global__ void __launch_bounds__(kBwdThreads) route_bwd_kernel(int T, int E, in
     }
 }
 
-// Backward only: copies of x and grad_out in the expert-sorted layout (row pos
-// holds the token of pair perm[pos]; padding rows are zero).  Walked in token
-// order: each 16-byte piece of a token's x and grad_out rows is read once and
-// stored to the sorted rows of the token's k pairs (inv), so the sources stream
-// from HBM once instead of once per pair.  A second loop zeroes the padding
-// rows at the end of each expert's group (fewer than kTileM per expert).
+// Copies of x and grad_out in the expert-sorted layout (row pos holds the
+// token of pair perm[pos]): both for the backward, x alone (g and gs null) for
+// the forward's gate/up GEMM.  Walked in token order: each 16-byte piece of a
+// token's rows is read once and stored to the sorted rows of the token's k
+// pairs (inv), so the sources stream from HBM once instead of once per pair.
+// With zero_pad a second loop zeroes the padding rows at the end of each
+// expert's group (fewer than kTileM per expert): the wgrads sum over them,
+// while the forward GEMM discards those rows' products.
 __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restrict__ inv,
                                                         const int32_t *__restrict__ counts,
                                                         const int32_t *__restrict__ group_start, int T, int E, int k,
                                                         int d, const __nv_bfloat16 *__restrict__ x,
                                                         const __nv_bfloat16 *__restrict__ g,
-                                                        __nv_bfloat16 *__restrict__ xs, __nv_bfloat16 *__restrict__ gs) {
+                                                        __nv_bfloat16 *__restrict__ xs, __nv_bfloat16 *__restrict__ gs,
+                                                        bool zero_pad) {
     const int n16 = d / 8;  // 16-byte pieces per row
     const int rows_used = group_start[E];
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -945,13 +948,13 @@ __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restric
     uint4 *gs4 = reinterpret_cast<uint4 *>(gs);
     const int64_t total = static_cast<int64_t>(T) * n16;
     for (int64_t i = tid; i < total; i += 2 * stride) {
-        uint4 xv[2], gv[2];
+        uint4 xv[2], gv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int64_t ii = i + u * stride;
             if (ii < total) {
                 xv[u] = __ldg(x4 + ii);
-                gv[u] = __ldg(g4 + ii);
+                if (g4 != nullptr) gv[u] = __ldg(g4 + ii);
             }
         }
 #pragma unroll
@@ -963,12 +966,13 @@ __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restric
                     const int pos = __ldg(inv + static_cast<int64_t>(t) * k + j);
                     if (pos >= 0 && pos < rows_used) {
                         xs4[static_cast<int64_t>(pos) * n16 + piece] = xv[u];
-                        gs4[static_cast<int64_t>(pos) * n16 + piece] = gv[u];
+                        if (gs4 != nullptr) gs4[static_cast<int64_t>(pos) * n16 + piece] = gv[u];
                     }
                 }
             }
         }
     }
+    if (!zero_pad) return;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     const int64_t per_expert = static_cast<int64_t>(kTileM - 1) * n16;
     const int64_t pad_total = static_cast<int64_t>(E) * per_expert;
@@ -979,7 +983,7 @@ __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restric
         const int row = __ldg(group_start + e) + __ldg(counts + e) + r;
         if (row < __ldg(group_start + e + 1) && row < rows_used) {
             xs4[static_cast<int64_t>(row) * n16 + piece] = zero;
-            gs4[static_cast<int64_t>(row) * n16 + piece] = zero;
+            if (gs4 != nullptr) gs4[static_cast<int64_t>(row) * n16 + piece] = zero;
         }
     }
 }
@@ -988,8 +992,9 @@ __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restric
 
 cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
                              int T, int d, const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs,
-                             __nv_bfloat16 *gs, int sms, cudaStream_t s) {
-    sort_rows_kernel<<<sms * 8, 256, 0, s>>>(inv, counts, group_start, T, E, k, d, x, g, xs, gs);  // 8 x 256 threads per SM
+                             __nv_bfloat16 *gs, bool zero_pad, int sms, cudaStream_t s) {
+    // 8 x 256 threads per SM
+    sort_rows_kernel<<<sms * 8, 256, 0, s>>>(inv, counts, group_start, T, E, k, d, x, g, xs, gs, zero_pad);
     return cudaGetLastError();
 }
 
