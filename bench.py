@@ -88,7 +88,7 @@ def l2_note(cfg):
     return f"inputs larger than L2 (expert weights {wbytes / 1e9:.2f} GB), no flush"
 
 
-def routing_sweep(M, IN, dev, stream, peak_gbs, E, k, Ts=(16384, 65536, 262144, 524288), reps=10):
+def routing_sweep(M, IN, dev, stream, peak_gbs, E, k, Ts=(16384, 65536, 262144, 524288, 1048576), reps=10):
     """Routing alone (moe_route: top-k, histogram, scan, permutation) at growing
     token counts, each call timed by itself with L2 flushed before it (a 256 MiB
     write), so that the logits come from HBM.  The activation buffers that

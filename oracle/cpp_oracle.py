@@ -49,8 +49,9 @@ def lib() -> ctypes.CDLL:
         i64, i32, p = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
         L.moe_oracle_route.argtypes = [i64, i32, i32, p, p, p]
         L.moe_oracle_dispatch.argtypes = [i64, i32, i32, p, p, p, p, p]
-        L.moe_oracle_forward.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p, p, p, i32]
-        L.moe_oracle_backward.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p, p, p, p, i32]
+        f64 = ctypes.c_double
+        L.moe_oracle_forward.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p, p, p, i32, f64]
+        L.moe_oracle_backward.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p, p, p, p, i32, f64]
         L.moe_oracle_hardware_threads.restype = ctypes.c_uint
         for f in (L.moe_oracle_route, L.moe_oracle_dispatch, L.moe_oracle_forward, L.moe_oracle_backward):
             f.restype = ctypes.c_int
@@ -99,7 +100,7 @@ def dispatch(idx, E):
     return counts, offsets, perm, inv.reshape(T, k)
 
 
-def forward(x, logits, wgu, wd, k, nthreads: int = 1, keep_intermediates: bool = True):
+def forward(x, logits, wgu, wd, k, nthreads: int = 1, keep_intermediates: bool = True, limit: float = 0.0):
     x, lg, wgu, wd = _f64(x), _f32(logits), _f64(wgu), _f64(wd)
     T, d = x.shape
     E, twoI, _ = wgu.shape
@@ -110,12 +111,13 @@ def forward(x, logits, wgu, wd, k, nthreads: int = 1, keep_intermediates: bool =
     h = np.empty((T * k, twoI)) if keep_intermediates else None
     a = np.empty((T * k, I)) if keep_intermediates else None
     rc = lib().moe_oracle_forward(T, d, E, k, I, _p(x), _p(lg), _p(wgu), _p(wd), _p(out), _p(idx), _p(w),
-                                  _p(h) if h is not None else None, _p(a) if a is not None else None, nthreads)
+                                  _p(h) if h is not None else None, _p(a) if a is not None else None, nthreads,
+                                  float(limit))
     _ok(rc, "forward")
     return dict(out=out, idx=idx, w=w, h=h, a=a)
 
 
-def backward(x, logits, wgu, wd, k, gout, nthreads: int = 1):
+def backward(x, logits, wgu, wd, k, gout, nthreads: int = 1, limit: float = 0.0):
     x, lg, wgu, wd, gout = _f64(x), _f32(logits), _f64(wgu), _f64(wd), _f64(gout)
     T, d = x.shape
     E, twoI, _ = wgu.shape
@@ -126,6 +128,6 @@ def backward(x, logits, wgu, wd, k, gout, nthreads: int = 1):
     dscore = np.empty((T, k))
     dlogits = np.empty((T, E))
     rc = lib().moe_oracle_backward(T, d, E, k, I, _p(x), _p(lg), _p(wgu), _p(wd), _p(gout), _p(dx), _p(dwgu),
-                                   _p(dwd), _p(dscore), _p(dlogits), nthreads)
+                                   _p(dwd), _p(dscore), _p(dlogits), nthreads, float(limit))
     _ok(rc, "backward")
     return dict(dx=dx, dwgu=dwgu, dwd=dwd, dscore=dscore, dlogits=dlogits)

@@ -25,7 +25,12 @@
 //    over the kept k; slot j = the j-th choice.
 //  * dispatch: experts ascending, tokens ascending inside an expert.
 //  * expert: W_gate_up[e] is [2I, d] (rows 0..I-1 gate, I..2I-1 up),
-//    W_down[e] is [d, I]; a = silu(gate) * up; no bias, no clamp.
+//    W_down[e] is [d, I]; a = silu(gate) * up; no bias.
+//  * clamped SwiGLU (the DeepSeek V4 `ClampedSilu` that the review note of
+//    "Mario/overlap moe kernel integration (prime-rl PR #3651)" says the kernel
+//    computes; no formula on the pages): with limit L > 0,
+//    a = silu(min(gate, L)) * clip(up, -L, L), the gradient passing where the
+//    input lies in the closed interval; limit 0 is the plain SwiGLU.
 //  * combine and dx scatter: sums over slots j = 0..k-1 in slot order.
 //  * dscore[t, j] = dL/dw[t, j]; dlogits through the renormalised softmax.
 //
@@ -49,6 +54,26 @@ double silu(double z) { return z * sigmoid(z); }
 double silu_grad(double z) {
     const double s = sigmoid(z);
     return s * (1.0 + z * (1.0 - s));
+}
+
+// The activation: plain SwiGLU for L <= 0, clamped SwiGLU for L > 0.
+double act(double g, double u, double L) {
+    if (L > 0) {
+        g = std::min(g, L);
+        u = std::min(std::max(u, -L), L);
+    }
+    return silu(g) * u;
+}
+
+// (dg, du) of act for dL/da = da; a clamp stops the gradient outside its interval.
+void act_grad(double g, double u, double L, double da, double *dg, double *du) {
+    double gc = g, uc = u;
+    if (L > 0) {
+        gc = std::min(g, L);
+        uc = std::min(std::max(u, -L), L);
+    }
+    *dg = (L > 0 && g > L) ? 0.0 : da * uc * silu_grad(gc);
+    *du = (L > 0 && std::fabs(u) > L) ? 0.0 : da * silu(gc);
 }
 
 // Run fn(e) for every expert e, experts dealt round-robin to n threads.
@@ -124,10 +149,10 @@ int moe_oracle_dispatch(int64_t T, int E, int k, const int32_t *idx, int32_t *co
 
 // Forward.  x [T, d], wgu [E, 2I, d], wd [E, d, I] (doubles); logits fp32
 // [T, E].  Writes out [T, d], idx [T, k], w [T, k]; h [T*k, 2I] and a [T*k, I]
-// per flat pair when not null.
+// per flat pair when not null.  limit > 0: clamped SwiGLU.
 int moe_oracle_forward(int64_t T, int d, int E, int k, int I, const double *x, const float *logits,
                        const double *wgu, const double *wd, double *out, int32_t *idx, double *w, double *h,
-                       double *a, int nthreads) {
+                       double *a, int nthreads, double limit) {
     if (moe_oracle_route(T, E, k, logits, idx, w) != 0) return -1;
     const int64_t P = T * k;
     std::vector<int32_t> counts(E), offsets(E + 1), perm(P), inv(P);
@@ -145,7 +170,7 @@ int moe_oracle_forward(int64_t T, int d, int E, int k, int I, const double *x, c
                 for (int c = 0; c < d; ++c) s += Wg[static_cast<size_t>(r) * d + c] * xt[c];
                 hh[r] = s;
             }
-            for (int i = 0; i < I; ++i) aa[i] = silu(hh[i]) * hh[I + i];
+            for (int i = 0; i < I; ++i) aa[i] = act(hh[i], hh[I + i], limit);
             double *yq = y.data() + q * d;
             for (int o = 0; o < d; ++o) {
                 double s = 0.0;
@@ -170,9 +195,10 @@ int moe_oracle_forward(int64_t T, int d, int E, int k, int I, const double *x, c
 
 // Backward for dL/dout = gout [T, d].  Writes dx [T, d], dwgu [E, 2I, d],
 // dwd [E, d, I], dscore [T, k] and dlogits [T, E] (zero outside the chosen k).
+// limit > 0: clamped SwiGLU.
 int moe_oracle_backward(int64_t T, int d, int E, int k, int I, const double *x, const float *logits,
                         const double *wgu, const double *wd, const double *gout, double *dx, double *dwgu,
-                        double *dwd, double *dscore, double *dlogits, int nthreads) {
+                        double *dwd, double *dscore, double *dlogits, int nthreads, double limit) {
     const int64_t P = T * k;
     std::vector<int32_t> idx(P), counts(E), offsets(E + 1), perm(P), inv(P);
     std::vector<double> w(P);
@@ -197,7 +223,7 @@ int moe_oracle_backward(int64_t T, int d, int E, int k, int I, const double *x, 
                 for (int c = 0; c < d; ++c) s += Wg[static_cast<size_t>(r) * d + c] * xt[c];
                 hh[r] = s;
             }
-            for (int i = 0; i < I; ++i) aa[i] = silu(hh[i]) * hh[I + i];
+            for (int i = 0; i < I; ++i) aa[i] = act(hh[i], hh[I + i], limit);
             // G = W_down[e]^T gout[t] (each G[i] summed over o = 0..d-1 in order,
             // rows of W_down read contiguously); dscore = <G, a>
             std::fill(G.begin(), G.end(), 0.0);
@@ -207,11 +233,7 @@ int moe_oracle_backward(int64_t T, int d, int E, int k, int I, const double *x, 
             for (int i = 0; i < I; ++i) ds += G[i] * aa[i];
             dscore[q] = ds;
             // SwiGLU backward of da = w G
-            for (int i = 0; i < I; ++i) {
-                const double da = wq * G[i];
-                dh[i] = da * hh[I + i] * silu_grad(hh[i]);
-                dh[I + i] = da * silu(hh[i]);
-            }
+            for (int i = 0; i < I; ++i) act_grad(hh[i], hh[I + i], limit, wq * G[i], &dh[i], &dh[I + i]);
             // dW_down[e] += (w gout[t]) (x) a
             for (int o = 0; o < d; ++o) {
                 const double go = wq * gt[o];

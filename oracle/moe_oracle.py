@@ -30,7 +30,14 @@ Readings taken where the pages are silent (each one is listed in the design doc):
   (a stable counting sort of the flattened choices t*k + j).
 * expert MLP: W_gate_up[e] is [2I, d] with rows 0..I-1 the gate and rows
   I..2I-1 the up projection; W_down[e] is [d, I].  h = W_gate_up[e] x,
-  a = silu(h_gate) * h_up, y = W_down[e] a.  No bias, no clamp.
+  a = silu(h_gate) * h_up, y = W_down[e] a.  No bias.
+* clamped SwiGLU ("Mario/overlap moe kernel integration (prime-rl PR #3651)",
+  the review note on the DeepSeek V4 clamped SwiGLU, `ClampedSilu`, which the
+  kernel computes, as opposed to the variant with sigmoid * 1.702 and up + 1,
+  which it does not): the pages give no formula.  Reading: with a limit
+  L > 0, a = silu(min(h_gate, L)) * clip(h_up, -L, L); the gradient passes
+  where the input lies in the closed interval (h_gate <= L, |h_up| <= L) and
+  is zero outside it.  limit = 0 is the plain SwiGLU above.
 * combine: out[t] = sum over slots j = 0..k-1, in slot order, of w[t,j] y_(t,j).
 * dscore[t,j] is the gradient with respect to the renormalised weight w[t,j];
   dlogits is the gradient with respect to the router logits through the
@@ -44,7 +51,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "route", "dispatch", "silu", "sigmoid", "expert_forward",
+    "route", "dispatch", "silu", "sigmoid", "swiglu", "swiglu_backward", "expert_forward",
     "combine_forward", "forward", "backward", "dense_forward",
     "forward_tokens", "backward_tokens", "backward_experts",
 ]
@@ -70,6 +77,37 @@ def silu_grad(z):
     """d silu / dz = sigma(z) * (1 + z * (1 - sigma(z)))."""
     s = sigmoid(z)
     return s * (1.0 + z * (1.0 - s))
+
+
+def _clamps(g, u, limit):
+    """(gate, up) after the clamp of the clamped SwiGLU; unchanged for limit = 0."""
+    g, u = np.asarray(g, dtype=np.float64), np.asarray(u, dtype=np.float64)
+    if limit > 0:
+        return np.minimum(g, limit), np.clip(u, -limit, limit)
+    return g, u
+
+
+def swiglu(g, u, limit=0.0):
+    """a = silu(g) * u; with limit > 0, silu(min(g, limit)) * clip(u, -limit, limit)."""
+    gc, uc = _clamps(g, u, limit)
+    return silu(gc) * uc
+
+
+def swiglu_backward(g, u, da, limit=0.0):
+    """(dg, du) of a = swiglu(g, u, limit) for dL/da = da.
+
+    Inside the clamps: dg = da * uc * silu'(gc), du = da * silu(gc).  A clamp
+    passes the gradient where its input lies in the closed interval and stops
+    it outside (g > limit, |u| > limit).
+    """
+    gc, uc = _clamps(g, u, limit)
+    da = np.asarray(da, dtype=np.float64)
+    dg = da * uc * silu_grad(gc)
+    du = da * silu(gc)
+    if limit > 0:
+        dg = np.where(np.asarray(g) <= limit, dg, 0.0)
+        du = np.where(np.abs(np.asarray(u)) <= limit, du, 0.0)
+    return dg, du
 
 
 # ----------------------------------------------------------------------------
@@ -124,15 +162,15 @@ def dispatch(idx, E):
 # ----------------------------------------------------------------------------
 # one expert's MLP
 # ----------------------------------------------------------------------------
-def expert_forward(xe, wgu_e, wd_e):
-    """SwiGLU expert on a block of rows.
+def expert_forward(xe, wgu_e, wd_e, limit=0.0):
+    """SwiGLU expert on a block of rows (clamped SwiGLU for limit > 0).
 
     xe [n, d]; wgu_e [2I, d]; wd_e [d, I].  Returns (h [n, 2I], a [n, I], y [n, d]).
     """
     I = wd_e.shape[1]
     h = xe @ wgu_e.T
     g, u = h[:, :I], h[:, I:]
-    a = silu(g) * u
+    a = swiglu(g, u, limit)
     y = a @ wd_e.T
     return h, a, y
 
@@ -144,7 +182,7 @@ def _f64(a):
 # ----------------------------------------------------------------------------
 # forward
 # ----------------------------------------------------------------------------
-def combine_forward(x, idx, w, wgu, wd):
+def combine_forward(x, idx, w, wgu, wd, limit=0.0):
     """Layer output for a given routing (idx, w): out[t] = sum_j w[t,j] y_(t,j)."""
     x, w, wgu, wd = _f64(x), _f64(w), _f64(wgu), _f64(wd)
     T, k = idx.shape
@@ -156,7 +194,7 @@ def combine_forward(x, idx, w, wgu, wd):
         pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
         if pairs.size == 0:
             continue
-        _, _, y = expert_forward(x[pairs // k], wgu[e], wd[e])
+        _, _, y = expert_forward(x[pairs // k], wgu[e], wd[e], limit)
         y_pair[pairs] = y
     y_pair = y_pair.reshape(T, k, d)
     out = np.zeros((T, d))
@@ -165,8 +203,8 @@ def combine_forward(x, idx, w, wgu, wd):
     return out
 
 
-def forward(x, logits, wgu, wd, k):
-    """Full forward.  Returns a dict with out and every intermediate.
+def forward(x, logits, wgu, wd, k, limit=0.0):
+    """Full forward (clamped SwiGLU for limit > 0).  Returns a dict with out and every intermediate.
 
     h, a, y are stored per flat pair index (t*k + j) so that they do not depend
     on any particular sorted layout.
@@ -184,7 +222,7 @@ def forward(x, logits, wgu, wd, k):
         pairs = perm[offsets[e]:offsets[e + 1]].astype(np.int64)
         if pairs.size == 0:
             continue
-        he, ae, ye = expert_forward(x[pairs // k], wgu[e], wd[e])
+        he, ae, ye = expert_forward(x[pairs // k], wgu[e], wd[e], limit)
         h[pairs], a[pairs], y[pairs] = he, ae, ye
     out = np.zeros((T, d))
     yk = y.reshape(T, k, d)
@@ -194,7 +232,7 @@ def forward(x, logits, wgu, wd, k):
                 perm=perm, inv=inv, h=h, a=a, y=y)
 
 
-def dense_forward(x, logits, wgu, wd, k):
+def dense_forward(x, logits, wgu, wd, k, limit=0.0):
     """Brute force: every expert on every token, masked by the routing.
 
     M[t, e] = w[t, j] if expert e is token t's j-th choice, else 0;
@@ -210,7 +248,7 @@ def dense_forward(x, logits, wgu, wd, k):
             M[t, idx[t, j]] = w[t, j]
     out = np.zeros((T, d))
     for e in range(E):
-        _, _, ye = expert_forward(x, wgu[e], wd[e])
+        _, _, ye = expert_forward(x, wgu[e], wd[e], limit)
         out += M[:, e:e + 1] * ye
     return out
 
@@ -218,7 +256,7 @@ def dense_forward(x, logits, wgu, wd, k):
 # ----------------------------------------------------------------------------
 # backward
 # ----------------------------------------------------------------------------
-def _pair_backward(x_rows, gout_rows, w_rows, wgu_e, wd_e):
+def _pair_backward(x_rows, gout_rows, w_rows, wgu_e, wd_e, limit=0.0):
     """Backward of one expert's block of pairs.
 
     Returns (dx_rows [n,d] unscaled contribution to dx[t], dscore [n],
@@ -227,12 +265,11 @@ def _pair_backward(x_rows, gout_rows, w_rows, wgu_e, wd_e):
     I = wd_e.shape[1]
     h = x_rows @ wgu_e.T
     g, u = h[:, :I], h[:, I:]
-    a = silu(g) * u
+    a = swiglu(g, u, limit)
     G = gout_rows @ wd_e                    # W_down[e]^T gout[t]   [n, I]
     dscore = np.sum(G * a, axis=1)          # <G, a> = <gout[t], y_p>
     da = w_rows[:, None] * G
-    dg = da * u * silu_grad(g)
-    du = da * silu(g)
+    dg, du = swiglu_backward(g, u, da, limit)
     dh = np.concatenate([dg, du], axis=1)   # [n, 2I]
     dwd_e = (w_rows[:, None] * gout_rows).T @ a   # sum_p (w gout) (x) a
     dx_rows = dh @ wgu_e                    # W_gate_up[e]^T dh      [n, d]
@@ -251,7 +288,7 @@ def routing_backward(w, dscore):
     return w * (dscore - s)
 
 
-def backward(x, logits, wgu, wd, k, gout, fwd=None):
+def backward(x, logits, wgu, wd, k, gout, fwd=None, limit=0.0):
     """Full backward for loss L with dL/dout = gout.
 
     Returns dict(dx [T,d], dwgu [E,2I,d], dwd [E,d,I], dscore [T,k],
@@ -276,7 +313,7 @@ def backward(x, logits, wgu, wd, k, gout, fwd=None):
         if pairs.size == 0:
             continue
         t = pairs // k
-        dxr, ds, dwgu[e], dwd[e], dhe = _pair_backward(x[t], gout[t], wf[pairs], wgu[e], wd[e])
+        dxr, ds, dwgu[e], dwd[e], dhe = _pair_backward(x[t], gout[t], wf[pairs], wgu[e], wd[e], limit)
         dx_pair[pairs], dscore[pairs], dh[pairs] = dxr, ds, dhe
     dx = np.zeros((T, d))
     dxk = dx_pair.reshape(T, k, d)
@@ -292,7 +329,7 @@ def backward(x, logits, wgu, wd, k, gout, fwd=None):
 # ----------------------------------------------------------------------------
 # sampled variants, for checking very large layers one output at a time
 # ----------------------------------------------------------------------------
-def forward_tokens(x, logits, wgu, wd, k, tokens):
+def forward_tokens(x, logits, wgu, wd, k, tokens, limit=0.0):
     """out rows for the listed tokens only (same arithmetic as forward)."""
     tokens = np.asarray(tokens, dtype=np.int64)
     idx, w = route(np.asarray(logits)[tokens], k)
@@ -301,12 +338,12 @@ def forward_tokens(x, logits, wgu, wd, k, tokens):
     for j in range(k):
         for r in range(tokens.size):
             e = int(idx[r, j])
-            _, _, y = expert_forward(xt[r:r + 1], _f64(wgu[e]), _f64(wd[e]))
+            _, _, y = expert_forward(xt[r:r + 1], _f64(wgu[e]), _f64(wd[e]), limit)
             out[r] += w[r, j] * y[0]
     return dict(out=out, idx=idx, w=w)
 
 
-def backward_tokens(x, logits, wgu, wd, k, gout, tokens):
+def backward_tokens(x, logits, wgu, wd, k, gout, tokens, limit=0.0):
     """dx, dscore and dlogits rows for the listed tokens only."""
     tokens = np.asarray(tokens, dtype=np.int64)
     logits = np.asarray(logits)
@@ -320,7 +357,7 @@ def backward_tokens(x, logits, wgu, wd, k, gout, tokens):
         for r in range(tokens.size):
             e = int(idx[r, j])
             dxr, ds, _, _, _ = _pair_backward(xt[r:r + 1], gt[r:r + 1], w[r, j:j + 1],
-                                              _f64(wgu[e]), _f64(wd[e]))
+                                              _f64(wgu[e]), _f64(wd[e]), limit)
             dx[r] += dxr[0]
             dscore[r, j] = ds[0]
     dl_slots = routing_backward(w, dscore)
@@ -329,7 +366,7 @@ def backward_tokens(x, logits, wgu, wd, k, gout, tokens):
     return dict(dx=dx, dscore=dscore, dlogits=dlogits, idx=idx, w=w)
 
 
-def backward_experts(x, logits, wgu, wd, k, gout, experts):
+def backward_experts(x, logits, wgu, wd, k, gout, experts, limit=0.0):
     """dW_gate_up[e] and dW_down[e] for the listed experts only."""
     logits = np.asarray(logits)
     E = logits.shape[1]
@@ -346,7 +383,7 @@ def backward_experts(x, logits, wgu, wd, k, gout, experts):
             continue
         t = pairs // k
         _, _, dwgu_e, dwd_e, _ = _pair_backward(_f64(np.asarray(x)[t]), _f64(np.asarray(gout)[t]),
-                                                wf[pairs], wgu_e, wd_e)
+                                                wf[pairs], wgu_e, wd_e, limit)
         res[e] = (dwgu_e, dwd_e)
     return res
 
@@ -422,7 +459,7 @@ def mx_qdq_blocks(v, axis):
     return np.moveaxis(out, -1, axis)
 
 
-def forward_mx(x, logits, wgu, wd, k):
+def forward_mx(x, logits, wgu, wd, k, limit=0.0):
     """Forward with MXFP8 GEMM operands.
 
     Gate/up GEMM: x and W_gate_up quantised along d.  Down GEMM: its operand
@@ -448,7 +485,7 @@ def forward_mx(x, logits, wgu, wd, k):
         if pairs.size == 0:
             continue
         he = xq[pairs // k] @ wguq[e].T
-        ae = wf[pairs][:, None] * (silu(he[:, :I]) * he[:, I:])
+        ae = wf[pairs][:, None] * swiglu(he[:, :I], he[:, I:], limit)
         h[pairs], aw[pairs] = he, ae
         y[pairs] = mx_qdq_blocks(ae, axis=1) @ wdq[e].T
     out = np.zeros((T, d))
@@ -458,7 +495,7 @@ def forward_mx(x, logits, wgu, wd, k):
     return dict(out=out, idx=idx, w=w, counts=counts, offsets=offsets, perm=perm, inv=inv, h=h, aw=aw, y=y)
 
 
-def backward_mx(x, logits, wgu, wd, k, gout, fwd):
+def backward_mx(x, logits, wgu, wd, k, gout, fwd, limit=0.0):
     """Backward with MXFP8 GEMM operands (fwd = forward_mx's result).
 
     Down dgrad: grad_out rows and W_down along d.  Gate/up dgrad: dh and
@@ -486,11 +523,11 @@ def backward_mx(x, logits, wgu, wd, k, gout, fwd):
         t = pairs // k
         he = fwd["h"][pairs]
         g, u = he[:, :I], he[:, I:]
-        a = silu(g) * u
+        a = swiglu(g, u, limit)
         G = goutq_d[t] @ wdq_d[e]
         dscore[pairs] = np.sum(G * a, axis=1)
         da = wf[pairs][:, None] * G
-        dh = np.concatenate([da * u * silu_grad(g), da * silu(g)], axis=1)
+        dh = np.concatenate(swiglu_backward(g, u, da, limit), axis=1)
         dx_pair[pairs] = mx_qdq_blocks(dh, axis=1) @ wguq_2i[e]
         # K = the expert's tokens in sorted order, blocks of 32 from its first pair
         dwd[e] = mx_qdq_blocks(gout[t], axis=0).T @ mx_qdq_blocks(fwd["aw"][pairs], axis=0)
@@ -523,7 +560,7 @@ class _MxWeights:
         return self.cache[e]
 
 
-def forward_tokens_mx(x, logits, wgu, wd, k, tokens, weights=None):
+def forward_tokens_mx(x, logits, wgu, wd, k, tokens, weights=None, limit=0.0):
     """out rows of forward_mx for the listed tokens only."""
     tokens = np.asarray(tokens, dtype=np.int64)
     idx, w = route(np.asarray(logits)[tokens], k)
@@ -535,12 +572,12 @@ def forward_tokens_mx(x, logits, wgu, wd, k, tokens, weights=None):
         for j in range(k):
             q = W.get(int(idx[r, j]))
             h = xq[r:r + 1] @ q["gu_d"].T
-            aw = w[r, j] * silu(h[:, :I]) * h[:, I:]
+            aw = w[r, j] * swiglu(h[:, :I], h[:, I:], limit)
             out[r] += (mx_qdq_blocks(aw, axis=1) @ q["d_i"].T)[0]
     return dict(out=out, idx=idx, w=w)
 
 
-def backward_tokens_mx(x, logits, wgu, wd, k, gout, tokens, weights=None):
+def backward_tokens_mx(x, logits, wgu, wd, k, gout, tokens, weights=None, limit=0.0):
     """dx, dscore and dlogits rows of backward_mx for the listed tokens only."""
     tokens = np.asarray(tokens, dtype=np.int64)
     logits = np.asarray(logits)
@@ -558,9 +595,9 @@ def backward_tokens_mx(x, logits, wgu, wd, k, gout, tokens, weights=None):
             h = xq[r:r + 1] @ q["gu_d"].T
             g, u = h[:, :I], h[:, I:]
             G = gq[r:r + 1] @ q["d_d"]
-            dscore[r, j] = np.sum(G * silu(g) * u)
+            dscore[r, j] = np.sum(G * swiglu(g, u, limit))
             da = w[r, j] * G
-            dh = np.concatenate([da * u * silu_grad(g), da * silu(g)], axis=1)
+            dh = np.concatenate(swiglu_backward(g, u, da, limit), axis=1)
             dx[r] += (mx_qdq_blocks(dh, axis=1) @ q["gu_2i"])[0]
     dl_slots = routing_backward(w, dscore)
     dlogits = np.zeros((tokens.size, E))
@@ -568,7 +605,7 @@ def backward_tokens_mx(x, logits, wgu, wd, k, gout, tokens, weights=None):
     return dict(dx=dx, dscore=dscore, dlogits=dlogits, idx=idx, w=w)
 
 
-def backward_experts_mx(x, logits, wgu, wd, k, gout, experts, weights=None):
+def backward_experts_mx(x, logits, wgu, wd, k, gout, experts, weights=None, limit=0.0):
     """dW_gate_up[e] and dW_down[e] of backward_mx for the listed experts only."""
     logits = np.asarray(logits)
     E = logits.shape[1]
@@ -590,10 +627,10 @@ def backward_experts_mx(x, logits, wgu, wd, k, gout, experts, weights=None):
         gr = _f64(np.asarray(gout)[t])
         h = mx_qdq_blocks(xr, axis=1) @ q["gu_d"].T
         g, u = h[:, :I], h[:, I:]
-        aw = wf[pairs][:, None] * silu(g) * u
+        aw = wf[pairs][:, None] * swiglu(g, u, limit)
         G = mx_qdq_blocks(gr, axis=1) @ q["d_d"]
         da = wf[pairs][:, None] * G
-        dh = np.concatenate([da * u * silu_grad(g), da * silu(g)], axis=1)
+        dh = np.concatenate(swiglu_backward(g, u, da, limit), axis=1)
         dwd_e = mx_qdq_blocks(gr, axis=0).T @ mx_qdq_blocks(aw, axis=0)
         dwgu_e = mx_qdq_blocks(dh, axis=0).T @ mx_qdq_blocks(xr, axis=0)
         res[e] = (dwgu_e, dwd_e)

@@ -121,3 +121,22 @@ def test_central_differences_pin_cpp_backward():
         vp[e, o, i] += h
         vm[e, o, i] -= h
         assert abs((L(x, wgu, vp) - L(x, wgu, vm)) / (2 * h) - b["dwd"][e, o, i]) < 1e-7
+
+
+@pytest.mark.parametrize("limit", [0.3, 1.0])
+def test_clamped_swiglu_agrees_with_numpy_oracle(limit):
+    rng = np.random.default_rng(31)
+    T, d, E, k, I = 40, 32, 6, 2, 16
+    x = rng.standard_normal((T, d))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    wgu = rng.standard_normal((E, 2 * I, d)) * 0.3
+    wd = rng.standard_normal((E, d, I)) * 0.3
+    gout = rng.standard_normal((T, d))
+    ref_f = O.forward(x, logits, wgu, wd, k, limit=limit)
+    assert np.any(ref_f["h"][:, :I] > limit) and np.any(np.abs(ref_f["h"][:, I:]) > limit)
+    f = C.forward(x, logits, wgu, wd, k, nthreads=3, limit=limit)
+    assert np.allclose(f["out"], ref_f["out"], rtol=1e-12, atol=1e-12)
+    ref_b = O.backward(x, logits, wgu, wd, k, gout, limit=limit)
+    b = C.backward(x, logits, wgu, wd, k, gout, nthreads=3, limit=limit)
+    for key in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
+        assert np.allclose(b[key], ref_b[key], rtol=1e-11, atol=1e-12), key

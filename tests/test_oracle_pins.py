@@ -334,7 +334,7 @@ def test_planted_mistake_silu_grad(monkeypatch, fd_case):
 
 
 def test_planted_mistake_gate_up_swap(monkeypatch):
-    def swapped(xe, wgu_e, wd_e):
+    def swapped(xe, wgu_e, wd_e, limit=0.0):
         I = wd_e.shape[1]
         h = xe @ wgu_e.T
         a = O.silu(h[:, I:]) * h[:, :I]
