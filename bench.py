@@ -88,10 +88,11 @@ def l2_note(cfg):
     return f"inputs larger than L2 (expert weights {wbytes / 1e9:.2f} GB), no flush"
 
 
-def routing_sweep(M, IN, dev, stream, peak_gbs, E, k, Ts=(16384, 65536, 262144, 524288, 1048576), reps=10):
+def routing_sweep(M, IN, dev, stream, peak_gbs, E, k, Ts=(16384, 65536, 262144, 524288, 1000000), reps=10):
     """Routing alone (moe_route: top-k, histogram, scan, permutation) at growing
     token counts, each call timed by itself with L2 flushed before it (a 256 MiB
-    write), so that the logits come from HBM.  The activation buffers that
+    write), so that the logits come from HBM.  The largest count, 10^6 tokens,
+    is near the most the library's 32-bit sorted-layout indices allow at k = 8.  The activation buffers that
     routing does not touch are left out (alloc_saved_routing) and the hidden
     sizes are small, so that the workspace stays small."""
     import torch

@@ -8,6 +8,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <cmath>
 #include <mutex>
 #include <vector>
 
@@ -33,6 +34,7 @@ struct Plan {
     int bn_i;           // N tile of the GEMMs whose N is I
     int cnt_stride;     // d / bn_d: combine counters per token, one per column tile
     int dpart_stride;   // 2 I / bn_i: dscore partials per sorted row, one per column half-tile
+    float limit;        // clamped SwiGLU limit, +inf for the plain SwiGLU
     // workspace layout (byte offsets)
     size_t ws_status, ws_cnt, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
     size_t ws_dh, ws_dpart, ws_xs, ws_gs, bwd_bytes;
@@ -51,6 +53,7 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     if (s->E > kMaxExperts || s->k > kMaxTopK) return MOE_ERR_SHAPE;
     if (s->d % 128 != 0 || s->I % 128 != 0) return MOE_ERR_SHAPE;
     if (s->dtype != MOE_BF16 && s->dtype != MOE_MXFP8) return MOE_ERR_ARG;
+    if (!(s->swiglu_limit >= 0.f) || std::isinf(s->swiglu_limit)) return MOE_ERR_ARG;  // NaN fails the first test
     const int64_t P = s->T * s->k;
     const int64_t widest = s->d > 2 * s->I ? s->d : 2 * static_cast<int64_t>(s->I);
     const int64_t nonempty = s->E < P ? s->E : P;
@@ -66,6 +69,7 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     p->m_tiles = p_cap / 128;
     p->n_chunks = static_cast<int>((s->T + kRouteChunk - 1) / kRouteChunk);
     p->mx = s->dtype == MOE_MXFP8;
+    p->limit = s->swiglu_limit > 0.f ? s->swiglu_limit : INFINITY;  // +inf: no clamp, min / clamp are exact no-ops
     p->bn_d = !p->mx && s->d % 256 == 0 ? 256 : 128;  // MXFP8 GEMMs use 128-wide N tiles
     p->bn_i = !p->mx && s->I % 256 == 0 ? 256 : 128;
     p->cnt_stride = s->d / p->bn_d;
@@ -315,6 +319,7 @@ GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
     a.I = pl.I;
     a.cnt_stride = pl.cnt_stride;
     a.dpart_stride = pl.dpart_stride;
+    a.limit = pl.limit;
     a.k_elems = pl.mx ? 128 : kTileK;
     a.perm = sv->perm;
     a.group_start = sv->group_start;

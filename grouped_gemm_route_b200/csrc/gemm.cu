@@ -580,7 +580,9 @@ struct TailList {
     int cap;     // entries
 };
 
-// gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up.
+// gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up,
+// or with the clamped SwiGLU aw = w * silu(min(gate, L)) * clamp(up, -L, L)
+// (a.limit = L; +inf leaves gate and up unchanged, bit for bit).
 // MXFP8: also aw's E4M3 codes and scale atoms along I (the down GEMM's K).
 // One 32-column chunk c of gate (gr) and up (ur) accumulator values.
 template <int BN, bool MX>
@@ -592,7 +594,8 @@ __device__ __forceinline__ void gateup_chunk(const GemmArgs &a, const Tile &t, i
     float av[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-        const float g = __uint_as_float(gr[i]), u = __uint_as_float(ur[i]);
+        const float g = fminf(__uint_as_float(gr[i]), a.limit);
+        const float u = fminf(fmaxf(__uint_as_float(ur[i]), -a.limit), a.limit);
         av[i] = valid ? wv * g * __fdividef(1.f, 1.f + __expf(-g)) * u : 0.f;
     }
 #pragma unroll
@@ -818,7 +821,9 @@ __device__ void combine_worker(const GemmArgs &a, const TailList &tail, volatile
     }
 }
 
-// down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh.
+// down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh
+// (clamped SwiGLU: gate and up clamped as in the forward, and each clamp stops
+// its gradient where h lies outside its interval).
 // MXFP8: also dh's E4M3 codes and scale atoms along 2I (the gate/up dgrad's K).
 template <int BN, bool MX>
 __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t, int r, int ch, uint32_t taddr,
@@ -846,15 +851,16 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
         float dg[32], du[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float g = (i & 1) ? bf16_hi(hg[i >> 1]) : bf16_lo(hg[i >> 1]);
-            const float u = (i & 1) ? bf16_hi(hu[i >> 1]) : bf16_lo(hu[i >> 1]);
+            const float g0 = (i & 1) ? bf16_hi(hg[i >> 1]) : bf16_lo(hg[i >> 1]);
+            const float u0 = (i & 1) ? bf16_hi(hu[i >> 1]) : bf16_lo(hu[i >> 1]);
+            const float g = fminf(g0, a.limit), u = fminf(fmaxf(u0, -a.limit), a.limit);
             const float gr = G[i];
             const float sg = __fdividef(1.f, 1.f + __expf(-g));
             const float sl = g * sg;
             ds += gr * (sl * u);
             const float da = wv * gr;
-            dg[i] = valid ? da * u * sg * (1.f + g * (1.f - sg)) : 0.f;
-            du[i] = valid ? da * sl : 0.f;
+            dg[i] = valid && g0 <= a.limit ? da * u * sg * (1.f + g * (1.f - sg)) : 0.f;
+            du[i] = valid && fabsf(u0) <= a.limit ? da * sl : 0.f;
         }
         uint32_t pdg[16], pdu[16];
 #pragma unroll

@@ -57,6 +57,7 @@ struct GemmArgs {
     int k_elems;          // K elements per pipeline stage: 64 (bf16) or 128 (MXFP8)
     int cnt_stride;       // combine counters per token
     int dpart_stride;     // dscore partials per sorted row
+    float limit;          // clamped SwiGLU limit; +inf for the plain SwiGLU
     const int *perm;
     const int *group_start;
     const int *tile_expert;

@@ -30,7 +30,8 @@ EXPORTS = ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe
 
 class MoeShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
-                ("I", ctypes.c_int32), ("dtype", ctypes.c_int32), ("max_sms", ctypes.c_int32)]
+                ("I", ctypes.c_int32), ("dtype", ctypes.c_int32), ("max_sms", ctypes.c_int32),
+                ("swiglu_limit", ctypes.c_float)]
 
 
 class MoeSaved(ctypes.Structure):
@@ -92,8 +93,9 @@ def _check(rc: int, where: str):
         raise MoeError(rc, where)
 
 
-def make_shape(T, d, E, k, I, dtype=MOE_BF16, max_sms=0) -> MoeShape:
-    return MoeShape(int(T), int(d), int(E), int(k), int(I), int(dtype), int(max_sms))
+def make_shape(T, d, E, k, I, dtype=MOE_BF16, max_sms=0, swiglu_limit=0.0) -> MoeShape:
+    """swiglu_limit: 0 for SwiGLU, L > 0 for the clamped SwiGLU (see include/moe.h)."""
+    return MoeShape(int(T), int(d), int(E), int(k), int(I), int(dtype), int(max_sms), float(swiglu_limit))
 
 
 def saved_sizes(shape: MoeShape):
@@ -240,11 +242,12 @@ class MoELayer:
     device: str = "cuda"
     max_sms: int = 0
     dtype: int = MOE_BF16  # MOE_BF16 or MOE_MXFP8 (GEMM operand precision)
+    swiglu_limit: float = 0.0  # 0: SwiGLU; L > 0: clamped SwiGLU
 
     def __post_init__(self):
         if not torch.cuda.is_available():
             raise RuntimeError("the fused MoE layer needs a CUDA device (sm_100)")
-        self.shape = make_shape(self.T, self.d, self.E, self.k, self.I, self.dtype, self.max_sms)
+        self.shape = make_shape(self.T, self.d, self.E, self.k, self.I, self.dtype, self.max_sms, self.swiglu_limit)
         self.saved = alloc_saved(self.shape, self.device)
         self.ws = alloc_workspace(self.shape, self.device)
         dev = self.device

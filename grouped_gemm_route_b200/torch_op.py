@@ -57,15 +57,16 @@ def _check_inputs(x, logits, w_gate_up, w_down, top_k):
 
 @torch.library.custom_op("ggr_b200::moe_forward", mutates_args=(), device_types="cuda")
 def moe_forward(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
-                top_k: int, dtype: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
-                                                 torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
-                                                 torch.Tensor, torch.Tensor, torch.Tensor]:
+                top_k: int, dtype: int, swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor,
+                                                                      torch.Tensor, torch.Tensor, torch.Tensor,
+                                                                      torch.Tensor, torch.Tensor, torch.Tensor,
+                                                                      torch.Tensor, torch.Tensor]:
     """out plus the saved state (topk_idx, topk_w, counts, offsets, group_start,
     tile_expert, perm, inv, h, aw), in the field order of moe_saved_t."""
     _check_inputs(x, logits, w_gate_up, w_down, top_k)
     T, d, E, I = _dims(x, w_gate_up)
     x, logits, w_gate_up, w_down = (t.contiguous() for t in (x, logits, w_gate_up, w_down))
-    shape = M.make_shape(T, d, E, top_k, I, dtype)
+    shape = M.make_shape(T, d, E, top_k, I, dtype, swiglu_limit=swiglu_limit)
     saved = M.alloc_saved(shape, x.device)
     f, _ = M.workspace_size(shape)
     ws = torch.empty(f, dtype=torch.uint8, device=x.device)
@@ -75,7 +76,7 @@ def moe_forward(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, 
 
 
 @moe_forward.register_fake
-def _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype):
+def _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit):
     T, d, E, I = _dims(x, w_gate_up)
     _, p_cap = M.saved_sizes(M.make_shape(T, d, E, top_k, I, dtype))  # host-side shape rule of the library
     saved = tuple(x.new_empty(_SAVED_SHAPES[n](T, E, top_k, I, p_cap), dtype=_SAVED_DTYPES[n])
@@ -87,11 +88,11 @@ def _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype):
 def moe_backward(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
                  topk_idx: torch.Tensor, topk_w: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
                  group_start: torch.Tensor, tile_expert: torch.Tensor, perm: torch.Tensor, inv: torch.Tensor,
-                 h: torch.Tensor, aw: torch.Tensor, top_k: int,
-                 dtype: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+                 h: torch.Tensor, aw: torch.Tensor, top_k: int, dtype: int,
+                 swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
     """(dx, dlogits, dw_gate_up, dw_down, dscore) for dL/dout = grad_out."""
     T, d, E, I = _dims(x, w_gate_up)
-    shape = M.make_shape(T, d, E, top_k, I, dtype)
+    shape = M.make_shape(T, d, E, top_k, I, dtype, swiglu_limit=swiglu_limit)
     saved = dict(zip(M.SAVED_FIELDS, (topk_idx, topk_w, counts, offsets, group_start, tile_expert, perm, inv, h,
                                       aw)))
     _, b = M.workspace_size(shape)
@@ -109,25 +110,25 @@ def moe_backward(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.Tenso
 
 @moe_backward.register_fake
 def _moe_backward_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
-                       tile_expert, perm, inv, h, aw, top_k, dtype):
+                       tile_expert, perm, inv, h, aw, top_k, dtype, swiglu_limit):
     T, d, E, I = _dims(x, w_gate_up)
     return (x.new_empty(T, d), x.new_empty(T, E, dtype=torch.float32), w_gate_up.new_empty(E, 2 * I, d),
             w_down.new_empty(E, d, I), x.new_empty(T, top_k, dtype=torch.float32))
 
 
 def _setup_context(ctx, inputs, output):
-    x, logits, w_gate_up, w_down, top_k, dtype = inputs
+    x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit = inputs
     saved = output[1:]
     ctx.save_for_backward(x, w_gate_up, w_down, *saved)
-    ctx.top_k, ctx.dtype = top_k, dtype
+    ctx.top_k, ctx.dtype, ctx.swiglu_limit = top_k, dtype, swiglu_limit
     ctx.mark_non_differentiable(*saved)
 
 
 def _backward(ctx, grad_out, *_unused_saved_grads):
     x, w_gate_up, w_down, *saved = ctx.saved_tensors
     dx, dlogits, dwgu, dwd, _ = moe_backward(grad_out.to(torch.bfloat16), x, w_gate_up, w_down, *saved,
-                                             ctx.top_k, ctx.dtype)
-    return dx, dlogits, dwgu, dwd, None, None
+                                             ctx.top_k, ctx.dtype, ctx.swiglu_limit)
+    return dx, dlogits, dwgu, dwd, None, None, None
 
 
 moe_forward.register_autograd(_backward, setup_context=_setup_context)
@@ -138,29 +139,30 @@ _ROUTING_FIELDS = M.SAVED_FIELDS[:8]  # the saved fields without h and aw
 
 @torch.library.custom_op("ggr_b200::moe_forward_ckpt", mutates_args=(), device_types="cuda")
 def moe_forward_ckpt(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
-                     top_k: int, dtype: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
-                                                      torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
-                                                      torch.Tensor]:
+                     top_k: int, dtype: int, swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor,
+                                                                           torch.Tensor, torch.Tensor, torch.Tensor,
+                                                                           torch.Tensor, torch.Tensor, torch.Tensor]:
     """Recompute mode: out plus the routing state only; h and aw are dropped
     when the op returns and regenerated by the backward op."""
-    outs = moe_forward(x, logits, w_gate_up, w_down, top_k, dtype)
+    outs = moe_forward(x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit)
     return outs[:9]
 
 
 @moe_forward_ckpt.register_fake
-def _moe_forward_ckpt_fake(x, logits, w_gate_up, w_down, top_k, dtype):
-    return _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype)[:9]
+def _moe_forward_ckpt_fake(x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit):
+    return _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit)[:9]
 
 
 @torch.library.custom_op("ggr_b200::moe_backward_ckpt", mutates_args=(), device_types="cuda")
 def moe_backward_ckpt(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
                       topk_idx: torch.Tensor, topk_w: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
                       group_start: torch.Tensor, tile_expert: torch.Tensor, perm: torch.Tensor, inv: torch.Tensor,
-                      top_k: int,
-                      dtype: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+                      top_k: int, dtype: int,
+                      swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
+                                                    torch.Tensor]:
     """Recompute mode backward: moe_recompute regenerates h and aw, then moe_bwd."""
     T, d, E, I = _dims(x, w_gate_up)
-    shape = M.make_shape(T, d, E, top_k, I, dtype)
+    shape = M.make_shape(T, d, E, top_k, I, dtype, swiglu_limit=swiglu_limit)
     _, p_cap = M.saved_sizes(shape)
     dev = x.device
     h = torch.empty(p_cap, 2 * I, dtype=torch.bfloat16, device=dev)
@@ -172,36 +174,36 @@ def moe_backward_ckpt(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.
     M.recompute(shape, x.contiguous(), w_gate_up.contiguous(), saved, ws, torch.cuda.current_stream(dev))
     del ws
     return moe_backward(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start, tile_expert,
-                        perm, inv, h, aw, top_k, dtype)
+                        perm, inv, h, aw, top_k, dtype, swiglu_limit)
 
 
 @moe_backward_ckpt.register_fake
 def _moe_backward_ckpt_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
-                            tile_expert, perm, inv, top_k, dtype):
+                            tile_expert, perm, inv, top_k, dtype, swiglu_limit):
     return _moe_backward_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
-                              tile_expert, perm, inv, None, None, top_k, dtype)
+                              tile_expert, perm, inv, None, None, top_k, dtype, swiglu_limit)
 
 
 def _setup_context_ckpt(ctx, inputs, output):
-    x, logits, w_gate_up, w_down, top_k, dtype = inputs
+    x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit = inputs
     routing = output[1:]
     ctx.save_for_backward(x, w_gate_up, w_down, *routing)
-    ctx.top_k, ctx.dtype = top_k, dtype
+    ctx.top_k, ctx.dtype, ctx.swiglu_limit = top_k, dtype, swiglu_limit
     ctx.mark_non_differentiable(*routing)
 
 
 def _backward_ckpt(ctx, grad_out, *_unused_routing_grads):
     x, w_gate_up, w_down, *routing = ctx.saved_tensors
     dx, dlogits, dwgu, dwd, _ = moe_backward_ckpt(grad_out.to(torch.bfloat16), x, w_gate_up, w_down, *routing,
-                                                  ctx.top_k, ctx.dtype)
-    return dx, dlogits, dwgu, dwd, None, None
+                                                  ctx.top_k, ctx.dtype, ctx.swiglu_limit)
+    return dx, dlogits, dwgu, dwd, None, None, None
 
 
 moe_forward_ckpt.register_autograd(_backward_ckpt, setup_context=_setup_context_ckpt)
 
 
 def moe_layer(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor, top_k: int,
-              mxfp8: bool = False, recompute: bool = False) -> torch.Tensor:
+              mxfp8: bool = False, recompute: bool = False, swiglu_limit: float = 0.0) -> torch.Tensor:
     """The fused MoE layer as a differentiable function: out [T, d] in x's dtype.
 
     x [T, d]; logits [T, E]; w_gate_up [E, 2I, d] (rows 0..I-1 gate, I..2I-1
@@ -212,9 +214,11 @@ def moe_layer(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_
     recompute=True keeps only the routing state between forward and backward
     (h and aw, 0.6 GB at the Qwen3-30B-A3B layer shape, are regenerated by one
     more gate/up GEMM in the backward); the results are bit-identical.
+    swiglu_limit=L > 0 selects the clamped SwiGLU, silu(min(gate, L)) *
+    clamp(up, -L, L) (0: the plain SwiGLU).
     """
     dtype = M.MOE_MXFP8 if mxfp8 else M.MOE_BF16
     op = moe_forward_ckpt if recompute else moe_forward
     out = op(x.to(torch.bfloat16), logits.to(torch.float32), w_gate_up.to(torch.bfloat16),
-             w_down.to(torch.bfloat16), int(top_k), dtype)[0]
+             w_down.to(torch.bfloat16), int(top_k), dtype, float(swiglu_limit))[0]
     return out.to(x.dtype)

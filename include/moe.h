@@ -70,12 +70,21 @@ extern "C" {
 typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_dtype_t;
 
 /* Layer shape.  T tokens, hidden size d, E experts, top-k, expert width I.
- * max_sms caps the persistent grids (0 = every SM). */
+ * max_sms caps the persistent grids (0 = every SM).
+ *
+ * swiglu_limit selects the expert activation.  0: SwiGLU, a = silu(gate) * up.
+ * L > 0: the clamped SwiGLU that the review note of "Mario/overlap moe kernel
+ * integration (prime-rl PR #3651)" says the fused kernel computes (DeepSeek V4
+ * ClampedSilu; the pages give no formula, this is the library's reading):
+ * a = silu(min(gate, L)) * clamp(up, -L, L), whose gradient passes where the
+ * input lies inside the closed interval and is zero outside it.  Negative,
+ * infinite or NaN limits are rejected with MOE_ERR_ARG. */
 typedef struct {
     int64_t T;
     int32_t d, E, k, I;
     int32_t dtype;   /* moe_dtype_t */
     int32_t max_sms;
+    float swiglu_limit;
 } moe_shape_t;
 
 /* State written by moe_fwd (and moe_route) and read by moe_bwd.  Every field

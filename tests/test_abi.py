@@ -62,6 +62,22 @@ def test_invalid_shapes_are_rejected(lib, T, d, E, k, I, dtype, code):
     assert lib.moe_fwd(ctypes.byref(sh), None, None, None, None, None, None, None, 0, None) == code
 
 
+@pytest.mark.parametrize("limit", [-1.0, float("inf"), float("nan")])
+def test_invalid_swiglu_limits_are_rejected(lib, limit):
+    sh = M.make_shape(256, 256, 8, 2, 128, swiglu_limit=limit)
+    f = ctypes.c_size_t()
+    assert lib.moe_workspace_size(ctypes.byref(sh), ctypes.byref(f), None) == M.MOE_ERR_ARG
+    assert lib.moe_fwd(ctypes.byref(sh), None, None, None, None, None, None, None, 0, None) == M.MOE_ERR_ARG
+
+
+def test_swiglu_limit_changes_no_size(lib):
+    plain = M.make_shape(16384, 2048, 128, 8, 768)
+    clamped = M.make_shape(16384, 2048, 128, 8, 768, swiglu_limit=7.0)
+    assert M.saved_sizes(plain) == M.saved_sizes(clamped)
+    assert M.workspace_size(plain) == M.workspace_size(clamped)
+    assert ctypes.sizeof(M.MoeShape) == 40  # int64 T, six int32, float swiglu_limit: 36 bytes, padded to 8
+
+
 def test_mxfp8_sizes(lib):
     sh = M.make_shape(16384, 2048, 128, 8, 768, M.MOE_MXFP8)
     f_mx, b_mx = M.workspace_size(sh)

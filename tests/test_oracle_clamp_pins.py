@@ -6,6 +6,9 @@
 * a limit above every pre-activation gives the plain layer bit for bit;
 * central finite differences of the clamped forward for every gradient, on
   inputs whose pre-activations stay well away from the clamps' corners;
+* the side of a clamp is decided on h rounded to bfloat16: bf16_round is
+  pinned against torch's float32 -> bfloat16 conversion and hand-worked ties,
+  and swiglu_backward against points just inside and outside a clamp;
 * a planted mistake (the gate clamped from below instead of above) fails the
   closed form.
 """
@@ -44,8 +47,10 @@ def py_act_grad(v, L):
     return dg + du
 
 
-def identity_layer(rng, T=14, d=7, E=5):
+def identity_layer(rng, L, T=14, d=7, E=5):
     x = rng.standard_normal((T, d)) * 2.5
+    near = np.abs(np.abs(x) - L) < 0.05  # keep |x| clear of L by more than a bf16 spacing
+    x[near] += 0.1
     logits = rng.standard_normal((T, E)).astype(np.float32)
     eye = np.eye(d)
     wgu = np.stack([np.concatenate([eye, eye])] * E)
@@ -56,7 +61,7 @@ def identity_layer(rng, T=14, d=7, E=5):
 @pytest.mark.parametrize("L", [0.5, 1.5, 3.0])
 def test_identity_experts_closed_form(L):
     rng = np.random.default_rng(int(L * 10))
-    x, logits, wgu, wd = identity_layer(rng)
+    x, logits, wgu, wd = identity_layer(rng, L)
     assert np.any(x > L) and np.any(x < -L)  # both clamps active somewhere
     out = O.forward(x, logits, wgu, wd, 3, limit=L)["out"]
     ref = np.array([[py_act(v, L) for v in row] for row in x])
@@ -165,3 +170,28 @@ def test_planted_mistake_gate_clamped_from_below(monkeypatch):
     monkeypatch.setattr(O, "_clamps", wrong)
     with pytest.raises(AssertionError):
         test_identity_experts_closed_form(1.5)
+
+
+def test_bf16_round_matches_torch_conversion():
+    import torch
+    rng = np.random.default_rng(11)
+    v = np.concatenate([rng.standard_normal(4000) * np.exp(rng.uniform(-20, 20, 4000)),
+                        [0.0, -0.0, 1.0, 0.2, 0.1875, -3.75e-3]]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.bf16_round(v.astype(np.float64)), ref)
+    # hand-worked ties: halfway values go to the even 8-bit significand
+    assert O.bf16_round(1.0 + 2.0 ** -8) == 1.0
+    assert O.bf16_round(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert O.bf16_round(-(1.0 + 3 * 2.0 ** -8)) == -(1.0 + 2.0 ** -6)
+
+
+def test_clamp_side_is_decided_on_bf16_h():
+    L = 0.25  # a bfloat16 value; the bf16 spacing just above it is 2^-9
+    g = np.array([L + 1e-6, L + 2.0 ** -9, L - 1e-6, 0.1])
+    u = np.array([0.1, 0.1, 0.1, -(L + 1e-6)])
+    dg, du = O.swiglu_backward(g, u, np.ones(4), L)
+    assert dg[0] != 0.0  # rounds to L: inside
+    assert dg[1] == 0.0  # the next bf16 value: outside
+    assert dg[2] != 0.0 and dg[3] != 0.0
+    assert du[3] != 0.0  # -(L + 1e-6) rounds to -L: inside
+    assert np.all(du[:3] != 0.0)

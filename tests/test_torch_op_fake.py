@@ -15,12 +15,12 @@ def test_forward_and_backward_fakes_match_the_library_sizes():
         lg = torch.empty(T, E, dtype=torch.float32, device="cuda")
         wgu = torch.empty(E, 2 * I, d, dtype=torch.bfloat16, device="cuda")
         wd = torch.empty(E, d, I, dtype=torch.bfloat16, device="cuda")
-        outs = TO.moe_forward(x, lg, wgu, wd, k, M.MOE_BF16)
+        outs = TO.moe_forward(x, lg, wgu, wd, k, M.MOE_BF16, 0.0)
         assert tuple(outs[0].shape) == (T, d) and outs[0].dtype == torch.bfloat16
         for name, t, nbytes in zip(M.SAVED_FIELDS, outs[1:], sizes):
             assert t.numel() * t.element_size() == nbytes, name
         assert outs[M.SAVED_FIELDS.index("perm") + 1].shape[0] == p_cap
-        g = TO.moe_backward(outs[0], x, wgu, wd, *outs[1:], k, M.MOE_BF16)
+        g = TO.moe_backward(outs[0], x, wgu, wd, *outs[1:], k, M.MOE_BF16, 0.0)
         assert [tuple(t.shape) for t in g] == [(T, d), (T, E), (E, 2 * I, d), (E, d, I), (T, k)]
         assert [t.dtype for t in g] == [torch.bfloat16, torch.float32, torch.bfloat16, torch.bfloat16,
                                         torch.float32]
