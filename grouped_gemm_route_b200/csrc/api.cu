@@ -32,11 +32,10 @@ struct Plan {
     int n_chunks;       // routing blocks
     int bn_d;           // N tile of the GEMMs whose N is d
     int bn_i;           // N tile of the GEMMs whose N is I
-    int cnt_stride;     // d / bn_d: combine counters per token, one per column tile
     int dpart_stride;   // 2 I / bn_i: dscore partials per sorted row, one per column half-tile
     float limit;        // clamped SwiGLU limit, +inf for the plain SwiGLU
     // workspace layout (byte offsets)
-    size_t ws_status, ws_cnt, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
+    size_t ws_status, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
     size_t ws_dh, ws_dpart, ws_xs, ws_gs, bwd_bytes;
     // MXFP8 operands: E4M3 codes and their scale atoms (forward, then backward)
     bool mx;
@@ -72,15 +71,12 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     p->limit = s->swiglu_limit > 0.f ? s->swiglu_limit : INFINITY;  // +inf: no clamp, min / clamp are exact no-ops
     p->bn_d = !p->mx && s->d % 256 == 0 ? 256 : 128;  // MXFP8 GEMMs use 128-wide N tiles
     p->bn_i = !p->mx && s->I % 256 == 0 ? 256 : 128;
-    p->cnt_stride = s->d / p->bn_d;
     p->dpart_stride = 2 * s->I / p->bn_i;  // the down dgrad's two epilogue warps per row each write a partial
                                            // (the kernel's kSplit for that mode)
 
     size_t off = 0;
     p->ws_status = off;
     off = align_up(off + 16);
-    p->ws_cnt = off;
-    off = align_up(off + static_cast<size_t>(s->T) * p->cnt_stride * 4);
     p->ws_stage = off;  // combine staging [P, d]; before it, the bf16 forward's sorted x [p_cap, d]
     off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
     const size_t common = off;
@@ -266,7 +262,7 @@ struct Launch {
 const char *kKindNames[kNumKernelKinds] = {
     "route_topk",       "route_scan",       "route_perm",           "gemm_gateup_fwd",      "gemm_down_fwd_combine",
     "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd",
-    "sort_rows", "mx_quant", "route_fused", "sort_x"};
+    "sort_rows", "mx_quant", "route_fused", "sort_x", "combine"};
 
 struct Saved {
     int32_t *idx;
@@ -298,15 +294,23 @@ int run_route(const moe_shape_t *shape, const Plan &pl, const DeviceInfo &dev, c
     unsigned *barrier = reinterpret_cast<unsigned *>(ws + pl.ws_status + 8);
     int32_t *blk_hist = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_counts);
     int32_t *blk_base = reinterpret_cast<int32_t *>(ws + pl.ws_chunk_base);
-    int32_t *cnt = reinterpret_cast<int32_t *>(ws + pl.ws_cnt);
     (void)shape;
     const int grid = route_fused_grid(logits, static_cast<int>(pl.T), pl.E, pl.k, dev.sms, pl.n_chunks);
     if (grid < 1) return MOE_ERR_LAUNCH;
     Launch L(kKindRouteFused, st);
     return L.done(launch_route_fused(logits, static_cast<int>(pl.T), pl.E, pl.k, saved->topk_idx, saved->topk_w,
                                      blk_hist, blk_base, saved->counts, saved->offsets, saved->group_start,
-                                     saved->tile_expert, saved->perm, saved->inv, cnt, pl.cnt_stride, pl.p_cap,
+                                     saved->tile_expert, saved->perm, saved->inv, pl.p_cap,
                                      barrier, status, dev.sms, grid, st));
+}
+
+// The slot-ordered sum of the k staged rows of every token (the combine after
+// the down GEMM, the scatter into dx after the gate/up dgrad).
+int run_combine(const Plan &pl, const DeviceInfo &dev, const uint8_t *ws, void *dst, cudaStream_t st) {
+    Launch L(kKindCombine, st);
+    return L.done(launch_combine_rows(reinterpret_cast<const __nv_bfloat16 *>(ws + pl.ws_stage),
+                                      static_cast<int>(pl.T), pl.k, pl.d, static_cast<__nv_bfloat16 *>(dst), dev.sms,
+                                      st));
 }
 
 GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
@@ -317,7 +321,6 @@ GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
     a.E = pl.E;
     a.k = pl.k;
     a.I = pl.I;
-    a.cnt_stride = pl.cnt_stride;
     a.dpart_stride = pl.dpart_stride;
     a.limit = pl.limit;
     a.k_elems = pl.mx ? 128 : kTileK;
@@ -328,7 +331,6 @@ GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
     a.h = reinterpret_cast<__nv_bfloat16 *>(sv->h);
     a.aw = reinterpret_cast<__nv_bfloat16 *>(sv->aw);
     a.stage = reinterpret_cast<__nv_bfloat16 *>(ws + pl.ws_stage);
-    a.cnt = reinterpret_cast<int *>(ws + pl.ws_cnt);
     a.status = reinterpret_cast<int *>(ws + pl.ws_status);
     return a;
 }
@@ -388,11 +390,14 @@ int down_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, con
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.d / 128;
     a.num_k_blocks = pl.I / 128;
-    a.out = static_cast<__nv_bfloat16 *>(out);
     a.sfa = awsf;
     a.sfb = wdsf;
-    Launch L(kKindGemmDownFwd, st);
-    return L.done(launch_gemm(kDownFwd, 128, true, a, tm_aw8, tm_wd8, grid_for(shape, dev), st));
+    {
+        Launch L(kKindGemmDownFwd, st);
+        const int rc = L.done(launch_gemm(kDownFwd, 128, true, a, tm_aw8, tm_wd8, grid_for(shape, dev), st));
+        if (rc) return rc;
+    }
+    return run_combine(pl, dev, w8, out, st);
 }
 
 // The gate/up GEMM with its SwiGLU epilogue (h, aw into `saved`), for the
@@ -488,13 +493,13 @@ int bwd_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, cons
     if ((rc = quant(true, wgu, EI2, pl.d, wgut8, wgutsf, nullptr))) return rc;
     a.n_tiles = pl.d / 128;
     a.num_k_blocks = 2 * pl.I / 128;
-    a.out = static_cast<__nv_bfloat16 *>(dx);
     a.sfa = dhsf;
     a.sfb = wgutsf;
     {
         Launch L(kKindGemmGateUpDgrad, st);
         if ((rc = L.done(launch_gemm(kGateUpDgrad, 128, true, a, tm_dh8, tm_wgut8, grid, st)))) return rc;
     }
+    if ((rc = run_combine(pl, dev, w8, dx, st))) return rc;
     // b5: gate/up wgrad (K = sorted rows)
     if ((rc = quant(true, a.dh, pl.p_cap, 2 * pl.I, dhc8, dhcsf, used))) return rc;
     if ((rc = quant(true, xs, pl.p_cap, pl.d, xsc8, xscsf, used))) return rc;
@@ -571,9 +576,12 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.d / pl.bn_d;
     a.num_k_blocks = pl.I / kTileK;
-    a.out = static_cast<__nv_bfloat16 *>(out);
-    Launch L(kKindGemmDownFwd, st);
-    return L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid_for(shape, dev), st));
+    {
+        Launch L(kKindGemmDownFwd, st);
+        const int rc = L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid_for(shape, dev), st));
+        if (rc) return rc;
+    }
+    return run_combine(pl, dev, w8, out, st);
 }
 
 int moe_recompute(const moe_shape_t *shape, const void *x, const void *w_gate_up, moe_saved_t *saved, void *ws,
@@ -645,7 +653,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
         return L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_w, saved->topk_idx,
                                        saved->inv, dpart, pl.dpart_stride, dscore, dlogits, st));
     }
-    // b1: down dgrad, dscore partials, SwiGLU backward -> dh; zeroes the dx counters
+    // b1: down dgrad, dscore partials, SwiGLU backward -> dh
     a.n_tiles = pl.I / pl.bn_i;
     a.num_k_blocks = pl.d / kTileK;
     {
@@ -666,7 +674,6 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     // b4: gate/up dgrad + ordered scatter-sum into dx
     a.n_tiles = pl.d / pl.bn_d;
     a.num_k_blocks = 2 * pl.I / kTileK;
-    a.out = static_cast<__nv_bfloat16 *>(dx);
     {
         Launch L(kKindGemmGateUpDgrad, st);
         if ((rc = L.done(gemm_pair_ok(kGateUpDgrad, pl.bn_d, false, 0, grid)
@@ -674,6 +681,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
                              : launch_gemm(kGateUpDgrad, pl.bn_d, false, a, tm_dh_rows, tm_wgu_mn, grid, st))))
             return rc;
     }
+    if ((rc = run_combine(pl, dev, w8, dx, st))) return rc;
     // b5: gate/up wgrad  dW_gu[e] = sum_p dh_p (x) x[t]
     a.m_tiles = 2 * pl.I / kTileM;
     a.n_tiles = pl.d / pl.bn_d;

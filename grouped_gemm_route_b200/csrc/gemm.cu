@@ -14,15 +14,12 @@
 //                fused epilogue.  The down dgrad, whose epilogue waits on loads
 //                of h, runs eight: warps 2..9, two per quadrant, each taking
 //                half of the tile's columns.
-//   next two     forward gate/up GEMM: gather producers, 16-byte cp.async
-//                copies of the x rows picked through the dispatch permutation,
-//                written with the same 128-byte swizzle.  The dispatch is fused
-//                into the operand load: the forward never writes a permuted
-//                copy of the tokens.  (The backward reads x and grad_out from
-//                expert-sorted copies made by sort_rows, so that its wgrads,
-//                whose K dimension is the tokens, run on plain TMA tiles.)
-//                Combine GEMMs: combine workers (below).  Idle in the other
-//                modes.
+//   next two     MXFP8 forward gate/up GEMM: gather producers, 16-byte
+//                cp.async copies of the x rows picked through the dispatch
+//                permutation, written with the same 128-byte swizzle.  Idle in
+//                the other modes.  (The bf16 forward and the backward read x,
+//                and the backward grad_out, from expert-sorted copies made by
+//                sort_rows, so that their GEMMs run on plain TMA tiles.)
 //
 // Modes (see GemmMode): the expert MLP of "Prime Intellect Fused MoE Kernel:
 // 3.11x MoE Training Speed", section "What a mixture-of-experts layer actually
@@ -32,11 +29,13 @@
 // "Where MoE training loses time") the two dgrads, the two wgrads and the
 // scatter of token gradients back to token order.
 //
-// The combine and the scatter are deterministic: each (token, slot) row writes
-// its tile slice to a slot-addressed staging buffer and bumps a per-(token,
-// column tile) counter; the CTA holding the row that brings the counter to k
-// queues it, and its combine workers sum the k slots in slot order.  No thread
-// ever waits on another CTA.
+// The combine and the scatter are deterministic: the down forward and the
+// gate/up dgrad store each (token, slot) row of their output, rounded to bf16,
+// to a slot-addressed staging buffer, and a bandwidth-bound kernel
+// (combine_rows) then sums every token's k staged rows in slot order.  Summing
+// inside the GEMM (per-row counters, a last-arriver queue and worker warps)
+// measured slower: the workers competed with the mainloop for the SM and the
+// memory system.
 //
 // Every wait on an mbarrier is bounded in time.  On expiry the kernel records
 // a timeout in the status word, stops issuing work, waits (bounded) for its own
@@ -78,13 +77,8 @@ struct Cfg {
     static constexpr int kSfBytes = MX ? 2 * kMxAtomBytes : 0;     // scale atoms per stage
     static constexpr int kSfOffset = kStages * kStageBytes;
     static constexpr int kBarOffset = kSfOffset + kStages * kSfBytes;  // mbarriers, TMEM slot, abort flag
-    // one region, used by the wgrads for their expert order and by the
-    // combine modes for their queue of finished tokens
-    static constexpr int kTailCap = MX ? 2048 : 4096;  // finished (token, column half-tile) pairs a CTA queues
-    static constexpr int kOrderOffset = kBarOffset + 512;
-    static constexpr int kTailOffset = kOrderOffset;
-    static constexpr int kUnionBytes = 4 * (kTailCap + 4) > 8 * kMaxExperts ? 4 * (kTailCap + 4) : 8 * kMaxExperts;
-    static constexpr int kXposeOffset = kOrderOffset + kUnionBytes;  // one 2 KB transpose per epilogue warp
+    static constexpr int kOrderOffset = kBarOffset + 512;              // the wgrads' expert order
+    static constexpr int kXposeOffset = kOrderOffset + 8 * kMaxExperts;  // one 2 KB transpose per epilogue warp
     // + 1 KB alignment slack; the largest layout must fit 227 KB
     static constexpr int smem_bytes(int epi_warps) { return kXposeOffset + epi_warps * kXposeBytes + 1024; }
     static_assert(smem_bytes(kMaxEpiWarps) <= 227 * 1024, "shared memory per CTA");
@@ -100,14 +94,15 @@ struct ModeTraits {
     static constexpr bool kAMn = MODE == kDownWgrad || MODE == kGateUpWgrad;
     static constexpr bool kBMn = MODE == kDownDgrad || MODE == kGateUpDgrad || MODE == kDownWgrad ||
                                  MODE == kGateUpWgrad;
-    static constexpr bool kCombine = MODE == kDownFwd || MODE == kGateUpDgrad;
+    // rows staged per (token, slot) for the slot-ordered sum that follows the GEMM
+    static constexpr bool kStage = MODE == kDownFwd || MODE == kGateUpDgrad;
     // Epilogue warps per TMEM lane quadrant: the down dgrad's epilogue (h
     // loads, dh stores) is latency bound and splits each tile's columns
     // between two warps; elsewhere one warp takes all of its 32 rows.
     static constexpr int kSplit = MODE == kDownDgrad ? 2 : 1;
     static constexpr int kEpiWarps = 4 * kSplit;
-    static constexpr int kGatherWarp0 = kEpiWarp0 + kEpiWarps;  // two more warps: gather, or combine workers
-    static constexpr int kThreads = 32 * (kGatherWarp0 + 2);  // the two last warps idle where unused
+    static constexpr int kGatherWarp0 = kEpiWarp0 + kEpiWarps;  // two more warps: the gather producers
+    static constexpr int kThreads = 32 * (kGatherWarp0 + 2);  // the two last warps idle where nothing is gathered
 };
 
 // Bytes of one stage that arrive by TMA (the gathered operand arrives by cp.async).
@@ -566,20 +561,6 @@ __device__ __forceinline__ void store_accumulator_bf16(uint32_t taddr, uint8_t *
     }
 }
 
-// Per-CTA queue of (token, column tile) pairs whose last slot this CTA wrote.
-// The epilogue warps reserve entries (count) and publish them (an entry holds
-// -1 until written).  Workers claim batches of four entries (claim): warps 6
-// and 7 from the start, so that the sums overlap the mainloop, and every other
-// warp once its own loop is over (combine_worker).  `done` counts epilogue
-// warps that have finished, after which no entry is added.
-struct TailList {
-    int *items;  // token * n_tiles + column tile
-    int *count;
-    int *done;
-    int *claim;
-    int cap;     // entries
-};
-
 // gate/up forward: SwiGLU; writes h (gate, up) and aw = w * silu(gate) * up,
 // or with the clamped SwiGLU aw = w * silu(min(gate, L)) * clamp(up, -L, L)
 // (a.limit = L; +inf leaves gate and up unchanged, bit for bit).
@@ -662,163 +643,18 @@ __device__ __forceinline__ void epi_gateup_fwd(const GemmArgs &a, const Tile &t,
     }
 }
 
-template <int BN>
-__device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *items, int n);
-
-// down forward / gate-up dgrad: stage the slot's row slice and count it; a
-// (token, column tile) whose k-th slot lands here is queued for the combine
-// workers
+// down forward / gate-up dgrad: this CTA's rows of the tile, rounded to bf16, to
+// the staging row of their (token, slot) pair; the slot-ordered sum over a
+// token's k staged rows runs as its own bandwidth-bound kernel afterwards
+// (combine_rows).  Padding rows store nothing.
 template <int BN, bool PAIR = false>
-__device__ __forceinline__ void epi_combine(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
-                                           uint64_t *tempty_acc, uint8_t *xbuf, const TailList &tail) {
-    const int lane = threadIdx.x & 31;
+__device__ __forceinline__ void epi_stage(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
+                                          uint64_t *tempty_acc, uint8_t *xbuf) {
     const int pos = t.mt * kTileM + r;
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
-    const int nh = t.nt;
-    __nv_bfloat16 *srow = valid ? a.stage + static_cast<size_t>(p) * a.d + nh * BN : nullptr;
+    __nv_bfloat16 *srow = valid ? a.stage + static_cast<size_t>(p) * a.d + t.nt * BN : nullptr;
     store_accumulator_bf16<BN, PAIR>(taddr, xbuf, srow, tempty_acc);
-    const int tok = valid ? p / a.k : 0;
-    bool last = false;
-    fence_acq_rel_gpu();  // this warp's staging rows (ordered by the transposes' __syncwarp) before its counts
-    if (valid) last = atomicAdd(a.cnt + static_cast<size_t>(tok) * a.cnt_stride + nh, 1) == a.k - 1;
-    unsigned mask = __ballot_sync(0xffffffffu, last);
-    if (mask == 0u) return;
-    fence_acq_rel_gpu();  // the other slots' staging rows after their counts
-    const int n_last = __popc(mask);
-    int base = 0;
-    if (lane == 0) base = atomicAdd(tail.count, n_last);
-    base = __shfl_sync(0xffffffffu, base, 0);
-    const int my = __popc(mask & ((1u << lane) - 1u));
-    const int item = tok * a.n_tiles + nh;
-    if (last && base + my < tail.cap) reinterpret_cast<volatile int *>(tail.items)[base + my] = item;
-    // no room left in the queue: sum those tokens now
-    if (base + n_last > tail.cap) {
-        while (mask != 0u) {
-            const int src = __ffs(static_cast<int>(mask)) - 1;
-            const int idx = __popc(mask & ((1u << src) - 1u)) + (n_last - __popc(mask));
-            mask &= mask - 1u;
-            const int it = __shfl_sync(0xffffffffu, item, src);
-            if (base + idx >= tail.cap) combine_tokens4<BN>(a, &it, 1);
-        }
-    }
-}
-
-// Slot-ordered sums of up to four finished (token, column tile) items at once:
-// the loads of eight slots of all four tokens are issued before any is summed,
-// so 32 row pieces per lane are in flight.  BN columns per item, BN / 32 per
-// lane (8 or 4: a 16- or 8-byte piece).
-template <int BN>
-__device__ __forceinline__ void combine_tokens4(const GemmArgs &a, const int *items, int n) {
-    constexpr int BH = BN;
-    constexpr int kCols = BH / 32;
-    constexpr int kWords = kCols / 2;
-    using Piece = typename std::conditional<kCols == 8, uint4,
-                                            typename std::conditional<kCols == 4, uint2, uint32_t>::type>::type;
-    const int lane = threadIdx.x & 31;
-    const int n2 = a.n_tiles;
-    const __nv_bfloat16 *base[4];
-    float acc[4][kCols];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int item = items[u < n ? u : 0];
-        const int tk = item / n2, nh = item - tk * n2;
-        base[u] = a.stage + static_cast<size_t>(tk) * a.k * a.d + nh * BH + lane * kCols;
-#pragma unroll
-        for (int i = 0; i < kCols; ++i) acc[u][i] = 0.f;
-    }
-    for (int j0 = 0; j0 < a.k; j0 += 8) {  // slot order
-        Piece pc[8][4];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (u < n && j0 + jj < a.k)
-                    pc[jj][u] = __ldcg(reinterpret_cast<const Piece *>(base[u] + static_cast<size_t>(j0 + jj) * a.d));
-            }
-        }
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (u < n && j0 + jj < a.k) {
-                    const uint32_t *w = reinterpret_cast<const uint32_t *>(&pc[jj][u]);
-#pragma unroll
-                    for (int q = 0; q < kWords; ++q) {
-                        acc[u][2 * q] += bf16_lo(w[q]);
-                        acc[u][2 * q + 1] += bf16_hi(w[q]);
-                    }
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        if (u < n) {
-            const int item = items[u];
-            const int tk = item / n2, nh = item - tk * n2;
-            Piece outv;
-            uint32_t *ow = reinterpret_cast<uint32_t *>(&outv);
-#pragma unroll
-            for (int q = 0; q < kWords; ++q) ow[q] = pack_bf16x2(acc[u][2 * q], acc[u][2 * q + 1]);
-            *reinterpret_cast<Piece *>(a.out + static_cast<size_t>(tk) * a.d + nh * BH + lane * kCols) = outv;
-            if (lane == 0) a.cnt[static_cast<size_t>(tk) * a.cnt_stride + nh] = 0;  // ready for the next call
-        }
-    }
-}
-
-// A combine worker (one warp): claims batches of four queue entries until the
-// queue is drained (the epilogue warps are done and every reserved entry has
-// been claimed) and sums them.  Every wait is bounded; progress restarts the
-// clock.
-template <int BN>
-__device__ void combine_worker(const GemmArgs &a, const TailList &tail, volatile int *abort_flag, int n_epi) {
-    const int lane = threadIdx.x & 31;
-    volatile int *vcount = tail.count, *vdone = tail.done, *vitems = tail.items;
-    uint64_t t0 = global_timer_ns();
-    for (;;) {
-        // lane 0 claims a batch and decides how many of its entries exist (0:
-        // queue drained, or the wait gave up)
-        int n = 0, lo = 0;
-        if (lane == 0) {
-            lo = atomicAdd(tail.claim, 4);
-            bool fail = false;
-            while (lo < tail.cap) {
-                if (*vcount >= lo + 4) {
-                    n = 4;
-                    break;
-                }
-                if (*vdone == n_epi) {
-                    __threadfence_block();
-                    n = max(0, min(*vcount, tail.cap) - lo);
-                    break;
-                }
-                if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) {
-                    fail = true;
-                    break;
-                }
-                __nanosleep(64);
-            }
-            for (int u = 0; u < n && !fail; ++u) {  // reserved entries are published shortly after
-                while (vitems[lo + u] < 0) {
-                    if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) {
-                        fail = true;
-                        break;
-                    }
-                }
-            }
-            if (fail) {
-                if (!*abort_flag) raise_abort(abort_flag, a.status);
-                n = 0;
-            }
-            __threadfence_block();
-        }
-        n = __shfl_sync(0xffffffffu, n, 0);
-        lo = __shfl_sync(0xffffffffu, lo, 0);
-        if (n <= 0) return;
-        combine_tokens4<BN>(a, tail.items + lo, n);
-        t0 = global_timer_ns();
-    }
 }
 
 // down dgrad: G = W_down^T gout; dscore partial <G, a>; SwiGLU backward -> dh
@@ -886,10 +722,6 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
         }
     }
     a.dpart[static_cast<size_t>(pos) * a.dpart_stride + kSplit * t.nt + ch] = valid ? ds : 0.f;
-    if (valid && t.nt == 0 && ch == 0) {  // counters of the dx scatter that follows
-        const int tok = p / a.k;
-        for (int c = 0; c < a.cnt_stride; ++c) a.cnt[static_cast<size_t>(tok) * a.cnt_stride + c] = 0;
-    }
 }
 
 // weight gradients: store the tile (zeros for an expert without tokens)
@@ -915,7 +747,7 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
 
 template <int MODE, int BN, bool MX>
 __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *tempty, uint32_t tmem_base,
-                              const int *order, uint8_t *xbuf, const TailList &tail, volatile int *abort_flag) {
+                              const int *order, uint8_t *xbuf, volatile int *abort_flag) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quad = warp & 3;  // TMEM lanes this warp may access: 32*quad .. 32*quad+31
     const int ch = (warp - kEpiWarp0) >> 2;  // down dgrad: which half of the tile's columns
@@ -935,7 +767,7 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
         if constexpr (MODE == kGateUpFwd) {
             epi_gateup_fwd<BN, MX>(a, t, r, taddr, &tempty[acc], xbuf);
         } else if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
-            epi_combine<BN>(a, t, r, taddr, &tempty[acc], xbuf, tail);
+            epi_stage<BN>(a, t, r, taddr, &tempty[acc], xbuf);
         } else if constexpr (MODE == kDownDgrad) {
             epi_down_dgrad<BN, MX>(a, t, r, ch, taddr, &tempty[acc], xbuf);
         } else {
@@ -959,18 +791,10 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     uint64_t *drain = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    const TailList tail{reinterpret_cast<int *>(smem + C::kTailOffset),
-                        reinterpret_cast<int *>(smem + C::kTailOffset) + C::kTailCap,
-                        reinterpret_cast<int *>(smem + C::kTailOffset) + C::kTailCap + 1,
-                        reinterpret_cast<int *>(smem + C::kTailOffset) + C::kTailCap + 2, C::kTailCap};
-    constexpr bool kCombine = TR::kCombine;
     int *s_count = reinterpret_cast<int *>(smem + C::kOrderOffset);
     int *order = s_count + kMaxExperts;
 
     const int warp = threadIdx.x >> 5;
-    if constexpr (kCombine) {
-        for (int i = threadIdx.x; i < C::kTailCap; i += TR::kThreads) tail.items[i] = -1;
-    }
     if constexpr (!TR::kMTiled) {  // busiest expert first: rank by padded row count, ties to lower index
         for (int e = threadIdx.x; e < args.E; e += TR::kThreads)
             s_count[e] = __ldg(args.group_start + e + 1) - __ldg(args.group_start + e);
@@ -996,11 +820,6 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        if constexpr (kCombine) {
-            *tail.count = 0;
-            *tail.done = 0;
-            *tail.claim = 0;
-        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -1020,19 +839,10 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         __syncwarp();
     } else if (warp < TR::kGatherWarp0) {
         epilogue_loop<MODE, BN, MX>(args, tfull, tempty, tmem_base, order,
-                                smem + C::kXposeOffset + (warp - kEpiWarp0) * kXposeBytes, tail, abort_flag);
-        if constexpr (kCombine) {  // this warp's queue entries are written: count it as done
-            __syncwarp();
-            if ((threadIdx.x & 31) == 0) {
-                __threadfence_block();
-                atomicAdd(tail.done, 1);
-            }
-        }
+                                smem + C::kXposeOffset + (warp - kEpiWarp0) * kXposeBytes, abort_flag);
     } else if constexpr (TR::kGather) {
         gather_loop<MODE, BN, MX>(args, smem, full, empty, order, abort_flag);
     }
-    // combine modes: warps 6 and 7 from the start, the others after their loops
-    if constexpr (kCombine) combine_worker<BN>(args, tail, abort_flag, TR::kEpiWarps);
 
     tc_fence_before_sync();
     __syncthreads();
@@ -1067,17 +877,14 @@ struct PairCfg {
     using TR = ModeTraits<MODE>;
     static constexpr int kBHalfBytes = (BN / 2) * kTileK * 2;  // this CTA's half of a B stage
     static constexpr int kStageBytes = kABytes + kBHalfBytes;
-    static constexpr int kTailCap = TR::kCombine ? 4096 : 0;
     static constexpr int kOrderBytes = 8 * kMaxExperts;  // wgrads: counts + order; M-tiled: pair-row starts
-    static constexpr int kTailBytes = TR::kCombine ? 4 * (kTailCap + 4) : 0;
     static constexpr int kXposeTotal = TR::kEpiWarps * kXposeBytes;
-    static constexpr int kFixed = 512 + kOrderBytes + kTailBytes + kXposeTotal + 1024;
+    static constexpr int kFixed = 512 + kOrderBytes + kXposeTotal + 1024;
     static constexpr int kFit = (227 * 1024 - kFixed) / kStageBytes;
     static constexpr int kStages = kFit < 6 ? kFit : 6;
     static constexpr int kBarOffset = kStages * kStageBytes;
     static constexpr int kOrderOffset = kBarOffset + 512;
-    static constexpr int kTailOffset = kOrderOffset + kOrderBytes;
-    static constexpr int kXposeOffset = kTailOffset + kTailBytes;
+    static constexpr int kXposeOffset = kOrderOffset + kOrderBytes;
     static constexpr int kSmemBytes = kXposeOffset + kXposeTotal + 1024;
     static_assert(kStages >= 4 && kSmemBytes <= 227 * 1024, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = 2 * BN;
@@ -1135,7 +942,6 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                   "the modes where pairs measured faster than one CTA");
     using P = PairCfg<MODE, BN>;
     using TR = ModeTraits<MODE>;
-    constexpr bool kCombine = TR::kCombine;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + P::kBarOffset);
@@ -1147,19 +953,12 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_count = reinterpret_cast<int *>(smem + P::kOrderOffset);
     int *tbl = TR::kMTiled ? s_count : s_count + kMaxExperts;  // pair-row starts, or the expert order
-    const TailList tail{reinterpret_cast<int *>(smem + P::kTailOffset),
-                        reinterpret_cast<int *>(smem + P::kTailOffset) + P::kTailCap,
-                        reinterpret_cast<int *>(smem + P::kTailOffset) + P::kTailCap + 1,
-                        reinterpret_cast<int *>(smem + P::kTailOffset) + P::kTailCap + 2, P::kTailCap};
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const GemmArgs &a = args;
 
-    if constexpr (kCombine) {
-        for (int i = threadIdx.x; i < P::kTailCap; i += TR::kThreads) tail.items[i] = -1;
-    }
     if constexpr (TR::kMTiled) {
         // pair rows per expert: ceil(tiles / 2), numbered expert by expert (warp 0 scans)
         if (warp == 0) {
@@ -1206,11 +1005,6 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        if constexpr (kCombine) {
-            *tail.count = 0;
-            *tail.done = 0;
-            *tail.claim = 0;
-        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -1335,22 +1129,13 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 release_acc<true>(&tempty[acc]);
             } else if constexpr (MODE == kGateUpFwd) {
                 epi_gateup_fwd<BN, false, true>(a, t, r, taddr, &tempty[acc], xbuf);
-            } else if constexpr (kCombine) {
-                epi_combine<BN, true>(a, t, r, taddr, &tempty[acc], xbuf, tail);
+            } else if constexpr (TR::kStage) {
+                epi_stage<BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
             } else {
                 epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
             }
         }
-        if constexpr (kCombine) {  // this warp's queue entries are written: count it as done
-            __syncwarp();
-            if (lane == 0) {
-                __threadfence_block();
-                atomicAdd(tail.done, 1);
-            }
-        }
     }
-    // combine mode: the two last warps from the start, the others after their loops
-    if constexpr (kCombine) combine_worker<BN>(a, tail, abort_flag, TR::kEpiWarps);
 
     tc_fence_before_sync();
     __syncthreads();

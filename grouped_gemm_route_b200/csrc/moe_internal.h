@@ -36,13 +36,14 @@ enum KernelKind : int {
     kKindMxQuant,
     kKindRouteFused,
     kKindSortX,
+    kKindCombine,
     kNumKernelKinds
 };
 
 // Which GEMM of the layer a launch computes; selects operand loading and epilogue.
 enum GemmMode : int {
     kGateUpFwd = 0,    // h = x[perm] W_gu[e]^T ; epilogue SwiGLU -> h, aw
-    kDownFwd = 1,      // y = aw W_down[e]^T   ; epilogue slot-ordered combine -> out
+    kDownFwd = 1,      // y = aw W_down[e]^T   ; epilogue stages y per (token, slot) for combine_rows
     kDownDgrad = 2,    // G = gout_sorted W_down[e] ; epilogue dscore partials, SwiGLU bwd -> dh
     kGateUpDgrad = 3,  // dx_p = dh W_gu[e]     ; epilogue slot-ordered scatter-sum -> dx
     kDownWgrad = 4,    // dW_down[e] = gout_sorted^T aw
@@ -55,7 +56,6 @@ struct GemmArgs {
     int m_tiles;          // wgrad: tiles along M of one expert's weight
     int num_k_blocks;     // M-tiled modes: K / 64
     int k_elems;          // K elements per pipeline stage: 64 (bf16) or 128 (MXFP8)
-    int cnt_stride;       // combine counters per token
     int dpart_stride;     // dscore partials per sorted row
     float limit;          // clamped SwiGLU limit; +inf for the plain SwiGLU
     const int *perm;
@@ -70,9 +70,7 @@ struct GemmArgs {
     uint8_t *mx_sf;             // and their scale atoms
     __nv_bfloat16 *h;
     __nv_bfloat16 *aw;
-    __nv_bfloat16 *stage;
-    int *cnt;
-    __nv_bfloat16 *out;   // out (fwd) or dx (bwd)
+    __nv_bfloat16 *stage;  // staged rows [T*k, d] of the down forward and the gate/up dgrad (row t*k + j)
     __nv_bfloat16 *dh;
     float *dpart;
     __nv_bfloat16 *dw;    // weight gradient (wgrad modes)
@@ -81,7 +79,7 @@ struct GemmArgs {
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
-                              int32_t *chunk_counts, int32_t *cnt, int cnt_per_token, cudaStream_t s);
+                              int32_t *chunk_counts, cudaStream_t s);
 cudaError_t launch_route_scan(int T, int E, int n_chunks, const int32_t *chunk_counts, int32_t *chunk_base,
                               int32_t *counts, int32_t *offsets, int32_t *group_start, int32_t *tile_expert,
                               int32_t *perm, int64_t p_cap, int *status, cudaStream_t s);
@@ -93,11 +91,14 @@ size_t route_fused_smem(int E, int k);
 int route_fused_grid(const float *logits, int T, int E, int k, int sms, int n_chunks);
 cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t *idx, float *w, int32_t *blk_hist,
                                int32_t *blk_base, int32_t *counts, int32_t *offsets, int32_t *group_start,
-                               int32_t *tile_expert, int32_t *perm, int32_t *inv, int32_t *cnt, int cnt_per_token,
-                               int64_t p_cap, unsigned *barrier, int *status, int sms, int grid,
+                               int32_t *tile_expert, int32_t *perm, int32_t *inv, int64_t p_cap, unsigned *barrier, int *status, int sms, int grid,
                                cudaStream_t s);
 cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int32_t *chunk_base, int32_t *perm,
                               int32_t *inv, int64_t p_cap, int *status, cudaStream_t s);
+// out[t] = slot-ordered fp32 sum of the staged rows t*k + j (bf16 in, bf16 out):
+// the down forward's combine and the gate/up dgrad's scatter into dx.
+cudaError_t launch_combine_rows(const __nv_bfloat16 *stage, int T, int k, int d, __nv_bfloat16 *out, int sms,
+                                cudaStream_t s);
 // x (and grad_out, when g is not null) in the expert-sorted layout; zero_pad
 // also zeroes each group's padding rows (the wgrads sum over them).
 cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
@@ -110,9 +111,9 @@ cudaError_t launch_expire_wait(int *status, cudaStream_t s);
 
 cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA,
                         const CUtensorMap &tmB, int grid, cudaStream_t s);
-// GEMMs on CTA pairs (tcgen05 cta_group::2, bf16, BN = 256): the weight
-// gradients and the gate/up dgrad; used where gemm_pair_ok holds, with the same
-// arguments and results as launch_gemm.
+// GEMMs on CTA pairs (tcgen05 cta_group::2, bf16, BN = 256): the gate/up
+// forward, the gate/up dgrad and the weight gradients; used where gemm_pair_ok
+// holds, with the same arguments and results as launch_gemm.
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid);
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
                              int grid, cudaStream_t s);

@@ -32,8 +32,7 @@ template <int NV>
 __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const float *__restrict__ logits, int T, int E,
                                                                   int k, int32_t *__restrict__ idx,
                                                                   float *__restrict__ w,
-                                                                  int32_t *__restrict__ chunk_counts,
-                                                                  int32_t *__restrict__ cnt, int cnt_per_token) {
+                                                                  int32_t *__restrict__ chunk_counts) {
     __shared__ int hist[kMaxExperts];
     __shared__ float sel_v[kTopkWarps][kMaxTopK];
     __shared__ int sel_e[kTopkWarps][kMaxTopK];
@@ -99,7 +98,6 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const float *_
             w[static_cast<size_t>(t) * k + j] = expf(sel_v[warp][j] - m) / s;
             atomicAdd(&hist[e], 1);
         }
-        for (int c = lane; c < cnt_per_token; c += 32) cnt[static_cast<size_t>(t) * cnt_per_token + c] = 0;
         __syncwarp();
     }
     __syncthreads();
@@ -229,7 +227,7 @@ __global__ void route_perm_kernel(int T, int E, int k, const int32_t *__restrict
 // contiguous sub-range of those, so (block, warp, token, slot) order is token
 // order.  Phases, separated by grid barriers (every block resident: the launch
 // is cooperative; every wait is bounded):
-//   1  per token top-k, weights, combine counters; per-warp expert histograms;
+//   1  per token top-k and weights; per-warp expert histograms;
 //      the block's histogram to blk_hist[b]
 //   2  block b scans expert e = b, b+G, ... over the G blocks: blk_base[.][e],
 //      counts[e]
@@ -251,8 +249,6 @@ struct RouteFusedArgs {
     int32_t *blk_hist;  // [G, E]
     int32_t *blk_base;  // [G, E]
     int32_t *counts, *offsets, *group_start, *tile_expert, *perm, *inv;
-    int32_t *cnt;
-    int cnt_per_token;
     int64_t p_cap;
     unsigned *barrier;  // zero before the launch
     int *status;
@@ -481,8 +477,6 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
                         wcnt[warp * E + e] += 1;  // the k experts of a token are distinct
                     }
                 }
-                for (int cc = lane; cc < a.cnt_per_token; cc += 32)
-                    a.cnt[static_cast<size_t>(tt) * a.cnt_per_token + cc] = 0;
             }
         }
         __syncwarp();
@@ -625,7 +619,6 @@ __global__ void __launch_bounds__(kLaneMaxWarps * 32, 1) route_lane_kernel(const
     const int wt0 = t0 + nb * warp / nw, wt1 = t0 + nb * (warp + 1) / nw;
     const int nbatch = (wt1 - wt0 + 31) / 32;
     const bool vec_k = (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.idx) | reinterpret_cast<uintptr_t>(a.w)) & 15u) == 0;
-    const bool vec_cnt = (a.cnt_per_token % 4 == 0) && (reinterpret_cast<uintptr_t>(a.cnt) & 15u) == 0;
     for (int i = threadIdx.x; i < nw * E; i += blockDim.x) {
         wcnt[i] = 0;
         emask[i] = 0u;
@@ -760,13 +753,6 @@ __global__ void __launch_bounds__(kLaneMaxWarps * 32, 1) route_lane_kernel(const
             }
 #pragma unroll
             for (int j = 0; j < K; ++j) atomicAdd(&wcnt[warp * E + ti[j]], 1);
-            int32_t *crow = a.cnt + static_cast<size_t>(t) * a.cnt_per_token;
-            if (vec_cnt) {
-                for (int cc = 0; cc < a.cnt_per_token; cc += 4)
-                    *reinterpret_cast<int4 *>(crow + cc) = make_int4(0, 0, 0, 0);
-            } else {
-                for (int cc = 0; cc < a.cnt_per_token; ++cc) crow[cc] = 0;
-            }
         }
         __syncwarp();
         if (it + S < nbatch) issue(it + S);
@@ -988,7 +974,55 @@ __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restric
     }
 }
 
+// The combine and the dx scatter-sum: out[t] = sum over slots j = 0..k-1, in
+// slot order, of the staged bf16 rows t*k + j, summed in fp32 and rounded to
+// bf16 once.  One thread per 16-byte piece of a token's row (consecutive
+// threads read consecutive pieces of the same row); the loads of eight slots
+// are issued before any is added.  Reads each staged row once and streams it
+// (evict-first): k*d*2 bytes in, d*2 out per token.
+__global__ void __launch_bounds__(256) combine_rows_kernel(const __nv_bfloat16 *__restrict__ stage, int T, int k,
+                                                           int d, __nv_bfloat16 *__restrict__ out) {
+    const int n16 = d / 8;
+    const int64_t total = static_cast<int64_t>(T) * n16;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const uint4 *src = reinterpret_cast<const uint4 *>(stage);
+    uint4 *dst = reinterpret_cast<uint4 *>(out);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t t = i / n16;
+        const int64_t piece = i - t * n16;
+        const uint4 *row0 = src + t * k * n16 + piece;
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        for (int j0 = 0; j0 < k; j0 += 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                if (j0 + jj < k) v[jj] = __ldcs(row0 + static_cast<int64_t>(j0 + jj) * n16);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                if (j0 + jj < k) {  // slot order
+                    const uint32_t w[4] = {v[jj].x, v[jj].y, v[jj].z, v[jj].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[2 * q] += bf16_lo(w[q]);
+                        acc[2 * q + 1] += bf16_hi(w[q]);
+                    }
+                }
+            }
+        }
+        dst[i] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                            pack_bf16x2(acc[6], acc[7]));
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_combine_rows(const __nv_bfloat16 *stage, int T, int k, int d, __nv_bfloat16 *out, int sms,
+                                cudaStream_t s) {
+    combine_rows_kernel<<<sms * 8, 256, 0, s>>>(stage, T, k, d, out);  // 8 x 256 threads per SM
+    return cudaGetLastError();
+}
 
 cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
                              int T, int d, const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs,
@@ -999,19 +1033,19 @@ cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const in
 }
 
 cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
-                              int32_t *chunk_counts, int32_t *cnt, int cnt_per_token, cudaStream_t s) {
+                              int32_t *chunk_counts, cudaStream_t s) {
     const int blocks = (T + kRouteChunk - 1) / kRouteChunk;
     const int nv = (E + 31) / 32;
     if (nv <= 1)
-        route_topk_kernel<1><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts, cnt, cnt_per_token);
+        route_topk_kernel<1><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts);
     else if (nv <= 2)
-        route_topk_kernel<2><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts, cnt, cnt_per_token);
+        route_topk_kernel<2><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts);
     else if (nv <= 4)
-        route_topk_kernel<4><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts, cnt, cnt_per_token);
+        route_topk_kernel<4><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts);
     else if (nv <= 8)
-        route_topk_kernel<8><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts, cnt, cnt_per_token);
+        route_topk_kernel<8><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts);
     else
-        route_topk_kernel<16><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts, cnt, cnt_per_token);
+        route_topk_kernel<16><<<blocks, kTopkThreads, 0, s>>>(logits, T, E, k, idx, w, chunk_counts);
     return cudaGetLastError();
 }
 
@@ -1074,10 +1108,9 @@ size_t route_fused_smem(int E, int k) {
 
 cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t *idx, float *w, int32_t *blk_hist,
                                int32_t *blk_base, int32_t *counts, int32_t *offsets, int32_t *group_start,
-                               int32_t *tile_expert, int32_t *perm, int32_t *inv, int32_t *cnt, int cnt_per_token,
-                               int64_t p_cap, unsigned *barrier, int *status, int sms, int grid, cudaStream_t s) {
+                               int32_t *tile_expert, int32_t *perm, int32_t *inv, int64_t p_cap, unsigned *barrier, int *status, int sms, int grid, cudaStream_t s) {
     RouteFusedArgs a{logits, T, E, k, idx, w, blk_hist, blk_base, counts, offsets, group_start,
-                     tile_expert, perm, inv, cnt, cnt_per_token, p_cap, barrier, status, 0};
+                     tile_expert, perm, inv, p_cap, barrier, status, 0};
     void *params[] = {&a};
     if (route_lane_ok(E, k, logits)) {
         const LaneCfg c = lane_cfg(E, T, sms);

@@ -83,7 +83,7 @@ extern "C" int moe_route_noalloc(const moe_shape_t *shape, const float *logits, 
     // Every scratch word read below is written earlier in this same call
     // (route_topk writes all histograms, route_scan all bases), so nothing in
     // the shared array has to be cleared first.
-    if (launch_route_topk(logits, T, E, k, saved->topk_idx, saved->topk_w, chunk_counts, nullptr, 0, st) !=
+    if (launch_route_topk(logits, T, E, k, saved->topk_idx, saved->topk_w, chunk_counts, st) !=
         cudaSuccess)
         return MOE_ERR_LAUNCH;
     if (launch_route_scan(T, E, static_cast<int>(n_chunks), chunk_counts, chunk_base, saved->counts, saved->offsets,

@@ -124,9 +124,10 @@ int moe_route(const moe_shape_t *shape, const float *logits, moe_saved_t *saved,
 
 /* Forward.  x: bf16 [T,d]; logits: fp32 [T,E]; w_gate_up: bf16 [E,2I,d];
  * w_down: bf16 [E,d,I]; out: bf16 [T,d].  Runs moe_route, then the gate/up
- * grouped GEMM (token rows gathered from x through the dispatch permutation
- * straight into the GEMM's operand tiles, SwiGLU in the epilogue; writes
- * saved->h and saved->aw), then the down grouped GEMM whose epilogue performs
+ * grouped GEMM (bf16: on x copied into the expert-sorted layout; MXFP8: token
+ * rows gathered through the dispatch permutation straight into the GEMM's
+ * operand tiles; SwiGLU in the epilogue; writes saved->h and saved->aw), then
+ * the down grouped GEMM, whose epilogue stages each (token, slot) product, and
  * the weighted combine as a deterministic slot-ordered reduction into out. */
 int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits,
             const void *w_gate_up, const void *w_down, void *out,
