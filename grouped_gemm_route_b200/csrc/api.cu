@@ -143,6 +143,7 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     p->saved[7] = Tk * 4;                                   // inv
     p->saved[8] = static_cast<size_t>(p_cap) * 2 * s->I * 2;  // h
     p->saved[9] = static_cast<size_t>(p_cap) * s->I * 2;      // aw
+    p->saved[10] = static_cast<size_t>(p_cap) * s->d * 2;     // xs (optional)
     return MOE_OK;
 }
 
@@ -273,10 +274,11 @@ struct Saved {
 
 int check_saved(const moe_saved_t *s) {
     if (!s) return MOE_ERR_ARG;
-    const void *ptrs[MOE_SAVED_FIELDS] = {s->topk_idx, s->topk_w, s->counts, s->offsets, s->group_start,
-                                         s->tile_expert, s->perm, s->inv, s->h, s->aw};
+    const void *ptrs[MOE_SAVED_FIELDS - 1] = {s->topk_idx, s->topk_w, s->counts, s->offsets, s->group_start,
+                                             s->tile_expert, s->perm, s->inv, s->h, s->aw};
     for (const void *q : ptrs)
         if (!aligned16(q)) return MOE_ERR_ARG;
+    if (s->xs != nullptr && !aligned16(s->xs)) return MOE_ERR_ARG;  // optional
     return MOE_OK;
 }
 
@@ -402,27 +404,34 @@ int down_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, con
 
 // The gate/up GEMM with its SwiGLU epilogue (h, aw into `saved`), for the
 // routing already in `saved`: bf16 or MXFP8 operands.
+// x in the expert-sorted layout, into saved->xs (padding rows zeroed, for the
+// backward's gate/up wgrad) when the caller keeps it, else into the combine's
+// staging space (unused until the down GEMM; padding rows left as they are).
+int sort_x(const Plan &pl, const DeviceInfo &dev, const void *x, const moe_saved_t *saved, uint8_t *w8,
+           cudaStream_t st, __nv_bfloat16 **dst) {
+    *dst = saved->xs != nullptr ? static_cast<__nv_bfloat16 *>(saved->xs)
+                                : reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_stage);
+    Launch L(kKindSortX, st);
+    return L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k, static_cast<int>(pl.T),
+                                   pl.d, static_cast<const __nv_bfloat16 *>(x), nullptr, *dst, nullptr,
+                                   saved->xs != nullptr, dev.sms, st));
+}
+
 int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,
                moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
+    int rc;
+    const int grid = grid_for(shape, dev);
+    const bool pair = !pl.mx && gemm_pair_ok(kGateUpFwd, 256, false, 0, grid);
+    __nv_bfloat16 *xs = nullptr;
+    if (pair || saved->xs != nullptr)
+        if ((rc = sort_x(pl, dev, x, saved, w8, st, &xs))) return rc;
     if (pl.mx) return gateup_mx(pl, dev, shape, x, w_gate_up, saved, w8, st);
     CUtensorMap tm_wgu;
     if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 128)) return MOE_ERR_LAUNCH;
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.I / 128;
     a.num_k_blocks = pl.d / kTileK;
-    const int grid = grid_for(shape, dev);
-    if (gemm_pair_ok(kGateUpFwd, 256, false, 0, grid)) {
-        // x in the sorted layout (in the combine's staging space, unused until the
-        // down GEMM), then plain TMA tiles on CTA pairs
-        __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_stage);
-        {
-            Launch L(kKindSortX, st);
-            const int rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
-                                                   static_cast<int>(pl.T), pl.d,
-                                                   static_cast<const __nv_bfloat16 *>(x), nullptr, xs, nullptr,
-                                                   false, dev.sms, st));
-            if (rc) return rc;
-        }
+    if (pair) {  // plain TMA tiles of the sorted x on CTA pairs
         CUtensorMap tm_xs;
         if (!make_map(&tm_xs, xs, pl.p_cap, pl.d, 128)) return MOE_ERR_LAUNCH;
         Launch L(kKindGemmGateUpFwd, st);
@@ -619,7 +628,10 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     __nv_bfloat16 *dh = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_dh);
     float *dpart = reinterpret_cast<float *>(w8 + pl.ws_dpart);
 
-    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_xs);
+    // x in the sorted layout: the forward's copy when the caller kept it, else sorted here
+    const bool have_xs = saved->xs != nullptr;
+    __nv_bfloat16 *xs = have_xs ? static_cast<__nv_bfloat16 *>(saved->xs)
+                                : reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_xs);
     __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_gs);
     CUtensorMap tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn, tm_gs_rows, tm_gs_mn, tm_xs_mn;
     const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I;
@@ -636,15 +648,18 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     a.dh = dh;
     a.dpart = dpart;
 
-    // b0: x and grad_out in the expert-sorted layout (operands of the K = tokens wgrads)
+    // b0: grad_out (and x, unless the forward kept it) in the expert-sorted layout,
+    // padding rows zero (operands of the K = tokens wgrads)
     {
         Launch L(kKindSortRows, st);
-        if ((rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
-                                          static_cast<int>(pl.T), pl.d,
-                                          static_cast<const __nv_bfloat16 *>(x),
-                                          static_cast<const __nv_bfloat16 *>(grad_out), xs, gs, true, dev.sms,
-                                          st))))
-            return rc;
+        const auto *g = static_cast<const __nv_bfloat16 *>(grad_out);
+        rc = have_xs ? L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
+                                               static_cast<int>(pl.T), pl.d, g, nullptr, gs, nullptr, true, dev.sms,
+                                               st))
+                     : L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
+                                               static_cast<int>(pl.T), pl.d, static_cast<const __nv_bfloat16 *>(x),
+                                               g, xs, gs, true, dev.sms, st));
+        if (rc) return rc;
     }
     if (pl.mx) {
         if ((rc = bwd_mx(pl, dev, shape, w_gate_up, w_down, saved, dx, dw_gate_up, dw_down, a, xs, gs, w8, st)))

@@ -22,7 +22,8 @@ MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_WS, MOE_ERR_ARCH = -1, -2, -3, -4
 MOE_ERR_LAUNCH, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE, MOE_ERR_UNSUPPORTED = -5, -6, -7, -8
 MOE_ERR_SCRATCH_LIMIT = -9
 
-SAVED_FIELDS = ("topk_idx", "topk_w", "counts", "offsets", "group_start", "tile_expert", "perm", "inv", "h", "aw")
+SAVED_FIELDS = ("topk_idx", "topk_w", "counts", "offsets", "group_start", "tile_expert", "perm", "inv", "h", "aw",
+                "xs")
 EXPORTS = ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
            "moe_error_string", "moe_profile_enable", "moe_profile_read", "moe_kernel_name",
            "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_recompute")
@@ -122,7 +123,7 @@ def _stream(stream):
 
 
 def saved_struct(saved: dict) -> MoeSaved:
-    return MoeSaved(*[saved[n].data_ptr() for n in SAVED_FIELDS])
+    return MoeSaved(*[saved[n].data_ptr() if saved.get(n) is not None else None for n in SAVED_FIELDS])
 
 
 def route(shape, logits, saved: dict, ws, stream=None):
@@ -200,16 +201,22 @@ def profile_read():
 # ----------------------------------------------------------------------------
 _SAVED_DTYPES = dict(topk_idx=torch.int32, topk_w=torch.float32, counts=torch.int32, offsets=torch.int32,
                      group_start=torch.int32, tile_expert=torch.int32, perm=torch.int32, inv=torch.int32,
-                     h=torch.bfloat16, aw=torch.bfloat16)
+                     h=torch.bfloat16, aw=torch.bfloat16, xs=torch.bfloat16)
 
 
-def alloc_saved(shape: MoeShape, device) -> dict:
+def alloc_saved(shape: MoeShape, device, keep_sorted_x: bool = True) -> dict:
+    """Every saved buffer; keep_sorted_x=False leaves the optional xs out (None):
+    the backward then sorts x itself, 2 * P_cap * d bytes less between the passes."""
     sizes, p_cap = saved_sizes(shape)
     T, E, k, I = shape.T, shape.E, shape.k, shape.I
     shapes = dict(topk_idx=(T, k), topk_w=(T, k), counts=(E,), offsets=(E + 1,), group_start=(E + 1,),
-                  tile_expert=(p_cap // 128,), perm=(p_cap,), inv=(T, k), h=(p_cap, 2 * I), aw=(p_cap, I))
+                  tile_expert=(p_cap // 128,), perm=(p_cap,), inv=(T, k), h=(p_cap, 2 * I), aw=(p_cap, I),
+                  xs=(p_cap, shape.d))
     out = {}
     for name, nbytes in zip(SAVED_FIELDS, sizes):
+        if name == "xs" and not keep_sorted_x:
+            out[name] = None
+            continue
         t = torch.empty(shapes[name], dtype=_SAVED_DTYPES[name], device=device)
         assert t.numel() * t.element_size() == nbytes, name
         out[name] = t
@@ -217,13 +224,15 @@ def alloc_saved(shape: MoeShape, device) -> dict:
 
 
 def alloc_saved_routing(shape: MoeShape, device) -> dict:
-    """Saved buffers for moe_route alone: the routing fields at full size, and
-    16-byte placeholders for h and aw, which routing does not touch."""
+    """Saved buffers for moe_route alone: the routing fields at full size,
+    16-byte placeholders for h and aw, which routing does not touch, and no xs."""
     sizes, p_cap = saved_sizes(shape)
     T, E, k = shape.T, shape.E, shape.k
     shapes = dict(topk_idx=(T, k), topk_w=(T, k), counts=(E,), offsets=(E + 1,), group_start=(E + 1,),
                   tile_expert=(p_cap // 128,), perm=(p_cap,), inv=(T, k), h=(8,), aw=(8,))
-    return {name: torch.empty(shapes[name], dtype=_SAVED_DTYPES[name], device=device) for name in SAVED_FIELDS}
+    out = {name: torch.empty(shapes[name], dtype=_SAVED_DTYPES[name], device=device) for name in SAVED_FIELDS[:-1]}
+    out["xs"] = None
+    return out
 
 
 def alloc_workspace(shape: MoeShape, device) -> torch.Tensor:
@@ -243,12 +252,13 @@ class MoELayer:
     max_sms: int = 0
     dtype: int = MOE_BF16  # MOE_BF16 or MOE_MXFP8 (GEMM operand precision)
     swiglu_limit: float = 0.0  # 0: SwiGLU; L > 0: clamped SwiGLU
+    keep_sorted_x: bool = True  # keep x's sorted copy from forward to backward (saves re-sorting it)
 
     def __post_init__(self):
         if not torch.cuda.is_available():
             raise RuntimeError("the fused MoE layer needs a CUDA device (sm_100)")
         self.shape = make_shape(self.T, self.d, self.E, self.k, self.I, self.dtype, self.max_sms, self.swiglu_limit)
-        self.saved = alloc_saved(self.shape, self.device)
+        self.saved = alloc_saved(self.shape, self.device, self.keep_sorted_x)
         self.ws = alloc_workspace(self.shape, self.device)
         dev = self.device
         self.out = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=dev)

@@ -26,15 +26,16 @@ from . import moe as M
 __all__ = ["moe_layer", "moe_forward", "moe_backward", "moe_forward_ckpt", "moe_backward_ckpt"]
 
 _SAVED_SHAPES = {
-    "topk_idx": lambda T, E, k, I, p: (T, k), "topk_w": lambda T, E, k, I, p: (T, k),
-    "counts": lambda T, E, k, I, p: (E,), "offsets": lambda T, E, k, I, p: (E + 1,),
-    "group_start": lambda T, E, k, I, p: (E + 1,), "tile_expert": lambda T, E, k, I, p: (p // 128,),
-    "perm": lambda T, E, k, I, p: (p,), "inv": lambda T, E, k, I, p: (T, k),
-    "h": lambda T, E, k, I, p: (p, 2 * I), "aw": lambda T, E, k, I, p: (p, I),
+    "topk_idx": lambda T, d, E, k, I, p: (T, k), "topk_w": lambda T, d, E, k, I, p: (T, k),
+    "counts": lambda T, d, E, k, I, p: (E,), "offsets": lambda T, d, E, k, I, p: (E + 1,),
+    "group_start": lambda T, d, E, k, I, p: (E + 1,), "tile_expert": lambda T, d, E, k, I, p: (p // 128,),
+    "perm": lambda T, d, E, k, I, p: (p,), "inv": lambda T, d, E, k, I, p: (T, k),
+    "h": lambda T, d, E, k, I, p: (p, 2 * I), "aw": lambda T, d, E, k, I, p: (p, I),
+    "xs": lambda T, d, E, k, I, p: (p, d),
 }
 _SAVED_DTYPES = dict(topk_idx=torch.int32, topk_w=torch.float32, counts=torch.int32, offsets=torch.int32,
                      group_start=torch.int32, tile_expert=torch.int32, perm=torch.int32, inv=torch.int32,
-                     h=torch.bfloat16, aw=torch.bfloat16)
+                     h=torch.bfloat16, aw=torch.bfloat16, xs=torch.bfloat16)
 
 
 def _dims(x, w_gate_up):
@@ -60,9 +61,9 @@ def moe_forward(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, 
                 top_k: int, dtype: int, swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor,
                                                                       torch.Tensor, torch.Tensor, torch.Tensor,
                                                                       torch.Tensor, torch.Tensor, torch.Tensor,
-                                                                      torch.Tensor, torch.Tensor]:
+                                                                      torch.Tensor, torch.Tensor, torch.Tensor]:
     """out plus the saved state (topk_idx, topk_w, counts, offsets, group_start,
-    tile_expert, perm, inv, h, aw), in the field order of moe_saved_t."""
+    tile_expert, perm, inv, h, aw, xs), in the field order of moe_saved_t."""
     _check_inputs(x, logits, w_gate_up, w_down, top_k)
     T, d, E, I = _dims(x, w_gate_up)
     x, logits, w_gate_up, w_down = (t.contiguous() for t in (x, logits, w_gate_up, w_down))
@@ -79,7 +80,7 @@ def moe_forward(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, 
 def _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit):
     T, d, E, I = _dims(x, w_gate_up)
     _, p_cap = M.saved_sizes(M.make_shape(T, d, E, top_k, I, dtype))  # host-side shape rule of the library
-    saved = tuple(x.new_empty(_SAVED_SHAPES[n](T, E, top_k, I, p_cap), dtype=_SAVED_DTYPES[n])
+    saved = tuple(x.new_empty(_SAVED_SHAPES[n](T, d, E, top_k, I, p_cap), dtype=_SAVED_DTYPES[n])
                   for n in M.SAVED_FIELDS)
     return (x.new_empty(T, d),) + saved
 
@@ -88,13 +89,13 @@ def _moe_forward_fake(x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit):
 def moe_backward(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
                  topk_idx: torch.Tensor, topk_w: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
                  group_start: torch.Tensor, tile_expert: torch.Tensor, perm: torch.Tensor, inv: torch.Tensor,
-                 h: torch.Tensor, aw: torch.Tensor, top_k: int, dtype: int,
+                 h: torch.Tensor, aw: torch.Tensor, xs: torch.Tensor, top_k: int, dtype: int,
                  swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
     """(dx, dlogits, dw_gate_up, dw_down, dscore) for dL/dout = grad_out."""
     T, d, E, I = _dims(x, w_gate_up)
     shape = M.make_shape(T, d, E, top_k, I, dtype, swiglu_limit=swiglu_limit)
     saved = dict(zip(M.SAVED_FIELDS, (topk_idx, topk_w, counts, offsets, group_start, tile_expert, perm, inv, h,
-                                      aw)))
+                                      aw, xs)))
     _, b = M.workspace_size(shape)
     ws = torch.empty(b, dtype=torch.uint8, device=x.device)
     dev = x.device
@@ -110,7 +111,7 @@ def moe_backward(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.Tenso
 
 @moe_backward.register_fake
 def _moe_backward_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
-                       tile_expert, perm, inv, h, aw, top_k, dtype, swiglu_limit):
+                       tile_expert, perm, inv, h, aw, xs, top_k, dtype, swiglu_limit):
     T, d, E, I = _dims(x, w_gate_up)
     return (x.new_empty(T, d), x.new_empty(T, E, dtype=torch.float32), w_gate_up.new_empty(E, 2 * I, d),
             w_down.new_empty(E, d, I), x.new_empty(T, top_k, dtype=torch.float32))
@@ -134,7 +135,7 @@ def _backward(ctx, grad_out, *_unused_saved_grads):
 moe_forward.register_autograd(_backward, setup_context=_setup_context)
 
 
-_ROUTING_FIELDS = M.SAVED_FIELDS[:8]  # the saved fields without h and aw
+_ROUTING_FIELDS = M.SAVED_FIELDS[:8]  # the saved fields without h, aw and xs
 
 
 @torch.library.custom_op("ggr_b200::moe_forward_ckpt", mutates_args=(), device_types="cuda")
@@ -142,8 +143,8 @@ def moe_forward_ckpt(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Ten
                      top_k: int, dtype: int, swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor,
                                                                            torch.Tensor, torch.Tensor, torch.Tensor,
                                                                            torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Recompute mode: out plus the routing state only; h and aw are dropped
-    when the op returns and regenerated by the backward op."""
+    """Recompute mode: out plus the routing state only; h, aw and xs are
+    dropped when the op returns and regenerated by the backward op."""
     outs = moe_forward(x, logits, w_gate_up, w_down, top_k, dtype, swiglu_limit)
     return outs[:9]
 
@@ -160,28 +161,29 @@ def moe_backward_ckpt(grad_out: torch.Tensor, x: torch.Tensor, w_gate_up: torch.
                       top_k: int, dtype: int,
                       swiglu_limit: float) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor,
                                                     torch.Tensor]:
-    """Recompute mode backward: moe_recompute regenerates h and aw, then moe_bwd."""
+    """Recompute mode backward: moe_recompute regenerates h, aw and xs, then moe_bwd."""
     T, d, E, I = _dims(x, w_gate_up)
     shape = M.make_shape(T, d, E, top_k, I, dtype, swiglu_limit=swiglu_limit)
     _, p_cap = M.saved_sizes(shape)
     dev = x.device
     h = torch.empty(p_cap, 2 * I, dtype=torch.bfloat16, device=dev)
     aw = torch.empty(p_cap, I, dtype=torch.bfloat16, device=dev)
+    xs = torch.empty(p_cap, d, dtype=torch.bfloat16, device=dev)
     saved = dict(zip(M.SAVED_FIELDS, (topk_idx, topk_w, counts, offsets, group_start, tile_expert, perm, inv, h,
-                                      aw)))
+                                      aw, xs)))
     f, _ = M.workspace_size(shape)
     ws = torch.empty(f, dtype=torch.uint8, device=dev)
     M.recompute(shape, x.contiguous(), w_gate_up.contiguous(), saved, ws, torch.cuda.current_stream(dev))
     del ws
     return moe_backward(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start, tile_expert,
-                        perm, inv, h, aw, top_k, dtype, swiglu_limit)
+                        perm, inv, h, aw, xs, top_k, dtype, swiglu_limit)
 
 
 @moe_backward_ckpt.register_fake
 def _moe_backward_ckpt_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
                             tile_expert, perm, inv, top_k, dtype, swiglu_limit):
     return _moe_backward_fake(grad_out, x, w_gate_up, w_down, topk_idx, topk_w, counts, offsets, group_start,
-                              tile_expert, perm, inv, None, None, top_k, dtype, swiglu_limit)
+                              tile_expert, perm, inv, None, None, None, top_k, dtype, swiglu_limit)
 
 
 def _setup_context_ckpt(ctx, inputs, output):
@@ -212,8 +214,9 @@ def moe_layer(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_
     each gradient in its input's dtype.  mxfp8=True runs the expert GEMMs on
     MXFP8 operands (E4M3 with one UE8M0 scale per 32 elements along K).
     recompute=True keeps only the routing state between forward and backward
-    (h and aw, 0.6 GB at the Qwen3-30B-A3B layer shape, are regenerated by one
-    more gate/up GEMM in the backward); the results are bit-identical.
+    (h, aw and the sorted copy of x, 1.2 GB at the Qwen3-30B-A3B layer shape,
+    are regenerated by one more gate/up GEMM in the backward); the results are
+    bit-identical.
     swiglu_limit=L > 0 selects the clamped SwiGLU, silu(min(gate, L)) *
     clamp(up, -L, L) (0: the plain SwiGLU).
     """

@@ -104,9 +104,12 @@ typedef struct {
     int32_t *inv;         /* [T,k]   pair -> sorted row                                */
     void *h;              /* bf16 [P_cap, 2I] gate/up pre-activations, sorted layout   */
     void *aw;             /* bf16 [P_cap, I]  w[t,j] * silu(gate) * up, sorted layout  */
+    void *xs;             /* bf16 [P_cap, d]  x in the sorted layout, padding rows 0; OPTIONAL:
+                           * when not NULL, moe_fwd and moe_recompute write it and moe_bwd reads
+                           * it instead of sorting x again (NULL: moe_bwd sorts x itself) */
 } moe_saved_t;
 
-#define MOE_SAVED_FIELDS 10
+#define MOE_SAVED_FIELDS 11
 
 /* Bytes of each moe_saved_t field (in declaration order) and the sorted-layout
  * row capacity.  Pure host function; touches no GPU. */

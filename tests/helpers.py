@@ -41,7 +41,7 @@ def run_layer(inp: dict, T, d, E, k, I, backward=True, layer=None, dtype=M.MOE_B
         res.update({n: v.clone() for n, v in g.items() if v is not None})
     torch.cuda.synchronize()
     status = layer.status()
-    res["saved"] = {n: v.clone() for n, v in layer.saved.items()}
+    res["saved"] = {n: v.clone() if v is not None else None for n, v in layer.saved.items()}
     res["status"] = status
     return layer, res
 

@@ -40,6 +40,7 @@ def test_sizes_for_the_30b_shape(lib):
     P = 16384 * 8
     assert p_cap % 128 == 0 and P <= p_cap <= P + 128 * 128
     assert sizes[0] == P * 4 and sizes[8] == p_cap * 2 * 768 * 2 and sizes[9] == p_cap * 768 * 2
+    assert sizes[10] == p_cap * 2048 * 2  # the optional sorted copy of x
     f, b = M.workspace_size(sh)
     assert f >= P * 2048 * 2 and b >= p_cap * 2 * 768 * 2
 
@@ -96,6 +97,9 @@ def test_null_and_misaligned_pointers_are_rejected_before_launch(lib):
     # misaligned saved field
     bad = M.MoeSaved(*([16] * (len(M.SAVED_FIELDS) - 1) + [24]))
     assert lib.moe_fwd(ctypes.byref(sh), 16, 16, 16, 16, 16, ctypes.byref(bad), 16, 1 << 40, None) == M.MOE_ERR_ARG
+    # the optional sorted x: NULL is accepted (the misaligned field above was it)
+    no_xs = M.MoeSaved(*([16] * (len(M.SAVED_FIELDS) - 1) + [None]))
+    assert lib.moe_fwd(ctypes.byref(sh), 16, 16, 16, 16, 16, ctypes.byref(no_xs), 16, 64, None) == M.MOE_ERR_WS
     # workspace too small
     assert lib.moe_fwd(ctypes.byref(sh), 16, 16, 16, 16, 16, ctypes.byref(saved), 16, 64, None) == M.MOE_ERR_WS
     assert lib.moe_bwd(ctypes.byref(sh), 16, 16, 16, 16, ctypes.byref(saved), 16, 16, 16, 16, None, 16, 64,

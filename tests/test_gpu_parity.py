@@ -155,3 +155,20 @@ def test_results_do_not_depend_on_the_grid(max_sms):
     assert torch.equal(outs[0][0], outs[1][0])
     for n in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
         assert torch.equal(outs[0][1][n], outs[1][1][n]), n
+
+
+@pytest.mark.parametrize("dtype", [M.MOE_BF16, M.MOE_MXFP8])
+def test_sorted_x_kept_or_not_gives_the_same_bits(dtype):
+    """With saved xs the forward keeps its sorted copy of x and the backward
+    skips sorting x; without it the backward sorts x itself: same results."""
+    cfg, inp = make(dict(T=700, d=512, E=12, k=3, I=256), seed=31)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    runs = []
+    for keep in (True, False):
+        layer = M.MoELayer(T, d, E, k, I, device="cuda", dtype=dtype, keep_sorted_x=keep)
+        _, res = run_layer(inp, T, d, E, k, I, layer=layer)
+        assert res["status"] == 0
+        assert (res["saved"]["xs"] is not None) == keep
+        runs.append(res)
+    for name in ("out", "dx", "dwgu", "dwd", "dscore", "dlogits"):
+        assert torch.equal(runs[0][name], runs[1][name]), name
