@@ -911,12 +911,15 @@ __global__ void __launch_bounds__(kBwdThreads) route_bwd_kernel(int T, int E, in
 
 // Copies of x and grad_out in the expert-sorted layout (row pos holds the
 // token of pair perm[pos]): both for the backward, x alone (g and gs null) for
-// the forward's gate/up GEMM.  Walked in token order: each 16-byte piece of a
-// token's rows is read once and stored to the sorted rows of the token's k
-// pairs (inv), so the sources stream from HBM once instead of once per pair.
-// With zero_pad a second loop zeroes the padding rows at the end of each
-// expert's group (fewer than kTileM per expert): the wgrads sum over them,
-// while the forward GEMM discards those rows' products.
+// the forward's gate/up GEMM.  One warp per token: its k sorted rows (inv) are
+// read once, each lane loads up to eight 16-byte pieces of the token's row(s)
+// before storing them to all k rows, so the sources stream from HBM once and
+// every store instruction writes 512 contiguous bytes of a sorted row.  With
+// zero_pad a second loop zeroes the padding rows at the end of each expert's
+// group (fewer than kTileM per expert): the wgrads sum over them, while the
+// forward GEMM discards those rows' products.
+constexpr int kSortPieces = 8;  // 16-byte pieces a lane holds at once, per source
+
 __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restrict__ inv,
                                                         const int32_t *__restrict__ counts,
                                                         const int32_t *__restrict__ group_start, int T, int E, int k,
@@ -926,33 +929,40 @@ __global__ void __launch_bounds__(256) sort_rows_kernel(const int32_t *__restric
                                                         bool zero_pad) {
     const int n16 = d / 8;  // 16-byte pieces per row
     const int rows_used = group_start[E];
+    const int lane = threadIdx.x & 31;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
     const uint4 *g4 = reinterpret_cast<const uint4 *>(g);
     uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
     uint4 *gs4 = reinterpret_cast<uint4 *>(gs);
-    const int64_t total = static_cast<int64_t>(T) * n16;
-    for (int64_t i = tid; i < total; i += 2 * stride) {
-        uint4 xv[2], gv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+    const int warps = static_cast<int>(stride >> 5);
+    for (int t = static_cast<int>(tid >> 5); t < T; t += warps) {
+        const int64_t src = static_cast<int64_t>(t) * n16;
+        for (int p0 = 0; p0 < n16; p0 += 32 * kSortPieces) {
+            uint4 xv[kSortPieces], gv[kSortPieces];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int64_t ii = i + u * stride;
-            if (ii < total) {
-                xv[u] = __ldg(x4 + ii);
-                if (g4 != nullptr) gv[u] = __ldg(g4 + ii);
+            for (int q = 0; q < kSortPieces; ++q) {
+                const int piece = p0 + 32 * q + lane;
+                if (piece < n16) {
+                    xv[q] = __ldcs(x4 + src + piece);
+                    if (g4 != nullptr) gv[q] = __ldcs(g4 + src + piece);
+                }
             }
-        }
+            for (int j0 = 0; j0 < k; j0 += 32) {
+                const int pos_l = j0 + lane < k ? __ldg(inv + static_cast<int64_t>(t) * k + j0 + lane) : -1;
+                const int nj = min(32, k - j0);
+                for (int jj = 0; jj < nj; ++jj) {
+                    const int pos = __shfl_sync(0xffffffffu, pos_l, jj);
+                    if (pos < 0 || pos >= rows_used) continue;  // warp-uniform
+                    const int64_t dst = static_cast<int64_t>(pos) * n16;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int64_t ii = i + u * stride;
-            if (ii < total) {
-                const int t = static_cast<int>(ii / n16), piece = static_cast<int>(ii - static_cast<int64_t>(t) * n16);
-                for (int j = 0; j < k; ++j) {
-                    const int pos = __ldg(inv + static_cast<int64_t>(t) * k + j);
-                    if (pos >= 0 && pos < rows_used) {
-                        xs4[static_cast<int64_t>(pos) * n16 + piece] = xv[u];
-                        if (gs4 != nullptr) gs4[static_cast<int64_t>(pos) * n16 + piece] = gv[u];
+                    for (int q = 0; q < kSortPieces; ++q) {
+                        const int piece = p0 + 32 * q + lane;
+                        if (piece < n16) {
+                            xs4[dst + piece] = xv[q];
+                            if (gs4 != nullptr) gs4[dst + piece] = gv[q];
+                        }
                     }
                 }
             }
