@@ -83,8 +83,6 @@ struct Cfg {
     static constexpr int smem_bytes(int epi_warps) { return kXposeOffset + epi_warps * kXposeBytes + 1024; }
     static_assert(smem_bytes(kMaxEpiWarps) <= 227 * 1024, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = MX ? 512 : 2 * BN;
-    static constexpr uint32_t kSfaCol = 2 * BN;                    // MXFP8 scale columns after the accumulators
-    static constexpr uint32_t kSfbCol = 2 * BN + 8;
 };
 
 template <int MODE>
@@ -467,7 +465,8 @@ __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint6
                 // scale atoms -> tensor memory (ordered before the MMAs that read them),
                 // then four K=32 block-scaled MMAs; sf_id k picks scale byte k
                 const uint32_t sf_base = smem_u32(smem + C::kSfOffset + s * C::kSfBytes);
-                const uint32_t sfa_t = tmem_base + C::kSfaCol, sfb_t = tmem_base + C::kSfbCol;
+                // the scale columns follow the two accumulators
+                const uint32_t sfa_t = tmem_base + 2u * BN, sfb_t = tmem_base + 2u * BN + 8u;
                 tmem_copy_32x128b_x4(sfa_t, smem_desc_plain(sf_base, 128));
                 tmem_copy_32x128b_x4(sfb_t, smem_desc_plain(sf_base + kMxAtomBytes, 128));
 #pragma unroll
@@ -764,10 +763,10 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
         }
         tc_fence_after_sync();
         const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-        if constexpr (MODE == kGateUpFwd) {
-            epi_gateup_fwd<BN, MX>(a, t, r, taddr, &tempty[acc], xbuf);
-        } else if constexpr (MODE == kDownFwd || MODE == kGateUpDgrad) {
+        if constexpr (ModeTraits<MODE>::kStage) {
             epi_stage<BN>(a, t, r, taddr, &tempty[acc], xbuf);
+        } else if constexpr (MODE == kGateUpFwd) {
+            epi_gateup_fwd<BN, MX>(a, t, r, taddr, &tempty[acc], xbuf);
         } else if constexpr (MODE == kDownDgrad) {
             epi_down_dgrad<BN, MX>(a, t, r, ch, taddr, &tempty[acc], xbuf);
         } else {
