@@ -159,6 +159,25 @@ def test_results_do_not_depend_on_the_grid(max_sms):
         assert torch.equal(outs[0][1][n], outs[1][1][n]), n
 
 
+def test_single_sm_runs_the_one_cta_kernels():
+    """On one SM no CTA pair fits: every GEMM runs on the one-CTA kernels (the
+    bf16 gate/up forward with its cp.async gather), checked against the oracle."""
+    cfg, inp = make(dict(T=300, d=256, E=8, k=2, I=256), seed=17)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    layer = M.MoELayer(T, d, E, k, I, device="cuda", max_sms=1)
+    _, res = run_layer(inp, T, d, E, k, I, layer=layer)
+    assert res["status"] == 0
+    logits = inp["logits"].numpy()
+    check_routing(res["saved"], logits, k)
+    x, wgu, wd = f64(inp["x"]), f64(inp["wgu"]), f64(inp["wd"])
+    ref = O.forward(x, logits, wgu, wd, k)
+    g = O.backward(x, logits, wgu, wd, k, f64(inp["gout"]), ref)
+    errs = dict(out=normwise(f64(res["out"]), ref["out"]))
+    for name in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
+        errs[name] = normwise(f64(res[name]), g[name])
+    assert all(v <= TOL_BF16 for v in errs.values()), errs
+
+
 @pytest.mark.parametrize("dtype", [M.MOE_BF16, M.MOE_MXFP8])
 def test_sorted_x_kept_or_not_gives_the_same_bits(dtype):
     """With saved xs the forward keeps its sorted copy of x and the backward
