@@ -38,7 +38,8 @@ struct Plan {
     size_t ws_status, ws_stage, ws_chunk_counts, ws_chunk_base, fwd_bytes;
     size_t ws_dh, ws_dpart, ws_xs, ws_gs, bwd_bytes;
     // MXFP8 operands: E4M3 codes and their scale atoms (forward, then backward)
-    bool mx;
+    bool mx;      // forward GEMMs on MXFP8 operands
+    bool mx_bwd;  // backward GEMMs on MXFP8 operands
     size_t mx_x8, mx_xsf, mx_wgu8, mx_wgusf, mx_wd8, mx_wdsf, mx_aw8, mx_awsf;
     size_t mx_gs8, mx_gssf, mx_wdt8, mx_wdtsf, mx_gsc8, mx_gscsf, mx_awc8, mx_awcsf, mx_wgut8, mx_wgutsf, mx_dh8,
         mx_dhsf, mx_dhc8, mx_dhcsf, mx_xsc8, mx_xscsf;
@@ -51,7 +52,7 @@ int make_plan(const moe_shape_t *s, Plan *p) {
         return MOE_ERR_ARG;
     if (s->E > kMaxExperts || s->k > kMaxTopK) return MOE_ERR_SHAPE;
     if (s->d % 128 != 0 || s->I % 128 != 0) return MOE_ERR_SHAPE;
-    if (s->dtype != MOE_BF16 && s->dtype != MOE_MXFP8) return MOE_ERR_ARG;
+    if (s->dtype != MOE_BF16 && s->dtype != MOE_MXFP8 && s->dtype != MOE_MXFP8_FWD) return MOE_ERR_ARG;
     if (!(s->swiglu_limit >= 0.f) || std::isinf(s->swiglu_limit)) return MOE_ERR_ARG;  // NaN fails the first test
     const int64_t P = s->T * s->k;
     const int64_t widest = s->d > 2 * s->I ? s->d : 2 * static_cast<int64_t>(s->I);
@@ -67,10 +68,12 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     p->p_cap = p_cap;
     p->m_tiles = p_cap / 128;
     p->n_chunks = static_cast<int>((s->T + kRouteChunk - 1) / kRouteChunk);
-    p->mx = s->dtype == MOE_MXFP8;
+    p->mx = s->dtype == MOE_MXFP8 || s->dtype == MOE_MXFP8_FWD;  // forward GEMMs on MXFP8 operands
+    p->mx_bwd = s->dtype == MOE_MXFP8;                            // backward GEMMs too
     p->limit = s->swiglu_limit > 0.f ? s->swiglu_limit : INFINITY;  // +inf: no clamp, min / clamp are exact no-ops
-    p->bn_d = !p->mx && s->d % 256 == 0 ? 256 : 128;  // MXFP8 GEMMs use 128-wide N tiles
-    p->bn_i = !p->mx && s->I % 256 == 0 ? 256 : 128;
+    // N tiles of the bf16 GEMMs (the MXFP8 GEMMs use 128-wide tiles of their own)
+    p->bn_d = !p->mx_bwd && s->d % 256 == 0 ? 256 : 128;
+    p->bn_i = !p->mx_bwd && s->I % 256 == 0 ? 256 : 128;
     p->dpart_stride = 2 * s->I / p->bn_i;  // the down dgrad's two epilogue warps per row each write a partial
                                            // (the kernel's kSplit for that mode)
 
@@ -112,7 +115,7 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
     p->ws_gs = off;
     off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
-    if (p->mx) {
+    if (p->mx_bwd) {
         p->mx_gs8 = take(Pd);
         p->mx_gssf = take(Pd / 32);
         p->mx_wdt8 = take(WdI);
@@ -325,7 +328,7 @@ GemmArgs base_args(const Plan &pl, const moe_saved_t *sv, uint8_t *ws) {
     a.I = pl.I;
     a.dpart_stride = pl.dpart_stride;
     a.limit = pl.limit;
-    a.k_elems = pl.mx ? 128 : kTileK;
+    a.k_elems = pl.mx_bwd ? 128 : kTileK;  // wgrad K rows per stage (backward only)
     a.perm = sv->perm;
     a.group_start = sv->group_start;
     a.tile_expert = sv->tile_expert;
@@ -661,7 +664,7 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
                                                g, xs, gs, true, dev.sms, st));
         if (rc) return rc;
     }
-    if (pl.mx) {
+    if (pl.mx_bwd) {
         if ((rc = bwd_mx(pl, dev, shape, w_gate_up, w_down, saved, dx, dw_gate_up, dw_down, a, xs, gs, w8, st)))
             return rc;
         Launch L(kKindRouteBwd, st);

@@ -17,6 +17,7 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 MOE_BF16, MOE_MXFP8 = 0, 1
+MOE_MXFP8_FWD = 2  # MXFP8 forward GEMMs, bf16 backward GEMMs
 MOE_OK = 0
 MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_WS, MOE_ERR_ARCH = -1, -2, -3, -4
 MOE_ERR_LAUNCH, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE, MOE_ERR_UNSUPPORTED = -5, -6, -7, -8
@@ -250,7 +251,7 @@ class MoELayer:
     I: int
     device: str = "cuda"
     max_sms: int = 0
-    dtype: int = MOE_BF16  # MOE_BF16 or MOE_MXFP8 (GEMM operand precision)
+    dtype: int = MOE_BF16  # MOE_BF16, MOE_MXFP8 or MOE_MXFP8_FWD (GEMM operand precision)
     swiglu_limit: float = 0.0  # 0: SwiGLU; L > 0: clamped SwiGLU
     keep_sorted_x: bool = True  # keep x's sorted copy from forward to backward (saves re-sorting it)
 

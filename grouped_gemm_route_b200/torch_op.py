@@ -205,7 +205,8 @@ moe_forward_ckpt.register_autograd(_backward_ckpt, setup_context=_setup_context_
 
 
 def moe_layer(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor, top_k: int,
-              mxfp8: bool = False, recompute: bool = False, swiglu_limit: float = 0.0) -> torch.Tensor:
+              mxfp8: bool = False, recompute: bool = False, swiglu_limit: float = 0.0,
+              fp8_bwd: bool = True) -> torch.Tensor:
     """The fused MoE layer as a differentiable function: out [T, d] in x's dtype.
 
     x [T, d]; logits [T, E]; w_gate_up [E, 2I, d] (rows 0..I-1 gate, I..2I-1
@@ -218,9 +219,10 @@ def moe_layer(x: torch.Tensor, logits: torch.Tensor, w_gate_up: torch.Tensor, w_
     are regenerated by one more gate/up GEMM in the backward); the results are
     bit-identical.
     swiglu_limit=L > 0 selects the clamped SwiGLU, silu(min(gate, L)) *
-    clamp(up, -L, L) (0: the plain SwiGLU).
+    clamp(up, -L, L) (0: the plain SwiGLU).  fp8_bwd=False (with mxfp8=True)
+    keeps the backward GEMMs in bf16.
     """
-    dtype = M.MOE_MXFP8 if mxfp8 else M.MOE_BF16
+    dtype = (M.MOE_MXFP8 if fp8_bwd else M.MOE_MXFP8_FWD) if mxfp8 else M.MOE_BF16
     op = moe_forward_ckpt if recompute else moe_forward
     out = op(x.to(torch.bfloat16), logits.to(torch.float32), w_gate_up.to(torch.bfloat16),
              w_down.to(torch.bfloat16), int(top_k), dtype, float(swiglu_limit))[0]

@@ -67,7 +67,11 @@ extern "C" {
 #define MOE_ERR_SCRATCH_LIMIT (-9) /* moe_route_noalloc: ceil(T/64)*E above its fixed scratch capacity */
 
 /* Operand precision of the expert GEMMs. */
-typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_dtype_t;
+/* MOE_MXFP8_FWD: MXFP8 forward GEMMs, bf16 backward GEMMs (the backward runs
+ * on the h and aw the MXFP8 forward saved) -- the pages' `fp8_bwd` switch
+ * ("Prime Intellect's Prime Mega MoE Trains Giant AI Models 55% Faster",
+ * section "Precision and hardware support") set off. */
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1, MOE_MXFP8_FWD = 2 } moe_dtype_t;
 
 /* Layer shape.  T tokens, hidden size d, E experts, top-k, expert width I.
  * max_sms caps the persistent grids (0 = every SM).

@@ -267,14 +267,15 @@ def dense_forward(x, logits, wgu, wd, k, limit=0.0):
 # ----------------------------------------------------------------------------
 # backward
 # ----------------------------------------------------------------------------
-def _pair_backward(x_rows, gout_rows, w_rows, wgu_e, wd_e, limit=0.0):
-    """Backward of one expert's block of pairs.
+def _pair_backward(x_rows, gout_rows, w_rows, wgu_e, wd_e, limit=0.0, h_rows=None):
+    """Backward of one expert's block of pairs (h_rows: the forward's h for
+    these pairs, else recomputed from x).
 
     Returns (dx_rows [n,d] unscaled contribution to dx[t], dscore [n],
     dwgu_e [2I,d], dwd_e [d,I], dh [n,2I]).
     """
     I = wd_e.shape[1]
-    h = x_rows @ wgu_e.T
+    h = x_rows @ wgu_e.T if h_rows is None else h_rows
     g, u = h[:, :I], h[:, I:]
     a = swiglu(g, u, limit)
     G = gout_rows @ wd_e                    # W_down[e]^T gout[t]   [n, I]
@@ -299,11 +300,13 @@ def routing_backward(w, dscore):
     return w * (dscore - s)
 
 
-def backward(x, logits, wgu, wd, k, gout, fwd=None, limit=0.0):
+def backward(x, logits, wgu, wd, k, gout, fwd=None, limit=0.0, h=None):
     """Full backward for loss L with dL/dout = gout.
 
-    Returns dict(dx [T,d], dwgu [E,2I,d], dwd [E,d,I], dscore [T,k],
-    dlogits [T,E], dh [T*k, 2I] per flat pair).
+    h: the gate/up pre-activations the forward saved, per flat pair
+    [T*k, 2I] (the MXFP8 forward's, for a bf16 backward after it); None
+    recomputes them from x.  Returns dict(dx [T,d], dwgu [E,2I,d],
+    dwd [E,d,I], dscore [T,k], dlogits [T,E], dh [T*k, 2I] per flat pair).
     """
     x, wgu, wd, gout = _f64(x), _f64(wgu), _f64(wd), _f64(gout)
     T, d = x.shape
@@ -324,7 +327,8 @@ def backward(x, logits, wgu, wd, k, gout, fwd=None, limit=0.0):
         if pairs.size == 0:
             continue
         t = pairs // k
-        dxr, ds, dwgu[e], dwd[e], dhe = _pair_backward(x[t], gout[t], wf[pairs], wgu[e], wd[e], limit)
+        dxr, ds, dwgu[e], dwd[e], dhe = _pair_backward(x[t], gout[t], wf[pairs], wgu[e], wd[e], limit,
+                                                        None if h is None else _f64(h)[pairs])
         dx_pair[pairs], dscore[pairs], dh[pairs] = dxr, ds, dhe
     dx = np.zeros((T, d))
     dxk = dx_pair.reshape(T, k, d)

@@ -53,7 +53,7 @@ def test_sizes_for_the_30b_shape(lib):
     (16, 256, 8, 2, 96, 0, M.MOE_ERR_SHAPE),
     (16, 256, 1024, 2, 128, 0, M.MOE_ERR_SHAPE),
     (16, 256, 128, 65, 128, 0, M.MOE_ERR_SHAPE),
-    (16, 256, 8, 2, 128, 2, M.MOE_ERR_ARG),
+    (16, 256, 8, 2, 128, 3, M.MOE_ERR_ARG),
     (16, 256, 8, 2, 128, 7, M.MOE_ERR_ARG),
 ])
 def test_invalid_shapes_are_rejected(lib, T, d, E, k, I, dtype, code):

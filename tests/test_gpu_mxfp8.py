@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 from grouped_gemm_route_b200 import moe as M
-from helpers import TOL_MXFP8, check_routing, f64, make, normwise, run_layer, sorted_rows
+from helpers import TOL_BF16, TOL_MXFP8, check_routing, f64, make, normwise, run_layer, sorted_rows
 from oracle import moe_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -86,3 +86,23 @@ def test_qwen3_30b_mxfp8_sampled():
         errs[f"dwd[{e}]"] = normwise(f64(res["dwd"][e]), be[e][1])
     bad = {n: v for n, v in errs.items() if not v <= TOL_MXFP8}
     assert not bad, f"normwise errors above {TOL_MXFP8}: {bad} (all: {errs})"
+
+
+@pytest.mark.parametrize("sizes", ["tiny", dict(T=700, d=512, E=12, k=3, I=256)])
+def test_mxfp8_forward_bf16_backward(sizes):
+    """MOE_MXFP8_FWD: the forward of the MXFP8 layer, then the bf16 backward on
+    the h and aw that forward saved (oracle: backward with the MXFP8 forward's h)."""
+    cfg, inp = make(sizes, seed=21)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    layer, res = run_layer(inp, T, d, E, k, I, dtype=M.MOE_MXFP8_FWD)
+    assert res["status"] == 0
+    logits = inp["logits"].numpy()
+    check_routing(res["saved"], logits, k)
+    x, wgu, wd, gout = f64(inp["x"]), f64(inp["wgu"]), f64(inp["wd"]), f64(inp["gout"])
+    ref = O.forward_mx(x, logits, wgu, wd, k)
+    g = O.backward(x, logits, wgu, wd, k, gout, ref, h=ref["h"])
+    errs = dict(h=normwise(sorted_rows(res["saved"], "h"), ref["h"]), out=normwise(f64(res["out"]), ref["out"]))
+    for name in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
+        errs[name] = normwise(f64(res[name]), g[name])
+    bad = {n: v for n, v in errs.items() if not v <= TOL_BF16}
+    assert not bad, f"normwise errors above {TOL_BF16}: {bad} (all: {errs})"

@@ -152,3 +152,25 @@ def test_sampled_mx_variants_agree_with_full():
     for e in (0, 3):
         assert np.allclose(be[e][0], b["dwgu"][e], rtol=1e-11, atol=1e-12)
         assert np.allclose(be[e][1], b["dwd"][e], rtol=1e-11, atol=1e-12)
+
+
+def test_backward_on_given_h():
+    """backward(h=...) uses the given pre-activations: the forward's own h gives
+    the plain backward bit for bit; the MXFP8 forward's h gives the bf16 backward
+    that follows an MXFP8 forward (and differs from the plain one)."""
+    rng = np.random.default_rng(8)
+    T, d, E, k, I = 24, 64, 5, 2, 32
+    x = rng.standard_normal((T, d))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    wgu = rng.standard_normal((E, 2 * I, d)) * 0.2
+    wd = rng.standard_normal((E, d, I)) * 0.2
+    gout = rng.standard_normal((T, d))
+    f = O.forward(x, logits, wgu, wd, k)
+    b = O.backward(x, logits, wgu, wd, k, gout, f)
+    bh = O.backward(x, logits, wgu, wd, k, gout, f, h=f["h"])
+    for key in ("dx", "dwgu", "dwd", "dscore", "dlogits"):
+        assert np.array_equal(b[key], bh[key]), key
+    fm = O.forward_mx(x, logits, wgu, wd, k)
+    bm = O.backward(x, logits, wgu, wd, k, gout, fm, h=fm["h"])
+    rel = np.linalg.norm(bm["dscore"] - b["dscore"]) / np.linalg.norm(b["dscore"])
+    assert 1e-4 < rel < 0.1
