@@ -1,5 +1,7 @@
-// Routing and dispatch kernels of the fused MoE layer, and the routing-score
-// backward.
+// Routing and dispatch kernels of the fused MoE layer, the routing-score
+// backward, and the two data-movement passes around the GEMMs: the copies of x
+// and grad_out in the expert-sorted layout (sort_rows) and the slot-ordered sum
+// of staged rows into out / dx (combine_rows).
 //
 // Routing rule (the layer's router, see include/moe.h): softmax over the E
 // router logits, keep the k largest, renormalise over the kept k.  The k
@@ -10,10 +12,13 @@
 // stable counting sort of the T*k choices by expert into a sorted layout whose
 // expert groups are padded to multiples of 128 rows (the GEMM tile height).
 //
-// Three launches: (1) per token top-k + weights + a per-block expert histogram,
-// (2) one block: totals, exclusive scans, per-block bases, tile table, padding,
-// (3) per block: each thread owns one expert and walks the block's tokens in
-// order, so positions inside an expert follow token order exactly.
+// The layer routes with one cooperative launch (route_fused, below: a
+// lane-per-token form for E <= 128 and a warp-per-token form otherwise).  The
+// three-launch form right below serves moe_route_noalloc: (1) per token top-k +
+// weights + a per-block expert histogram, (2) one block: totals, exclusive
+// scans, per-block bases, tile table, padding, (3) per block: each thread owns
+// one expert and walks the block's tokens in order, so positions inside an
+// expert follow token order exactly.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
