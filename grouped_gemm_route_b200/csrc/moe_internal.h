@@ -42,10 +42,10 @@ enum KernelKind : int {
 
 // Which GEMM of the layer a launch computes; selects operand loading and epilogue.
 enum GemmMode : int {
-    kGateUpFwd = 0,    // h = x[perm] W_gu[e]^T ; epilogue SwiGLU -> h, aw
+    kGateUpFwd = 0,    // h = x_sorted W_gu[e]^T ; epilogue SwiGLU -> h, aw (MXFP8: x rows gathered)
     kDownFwd = 1,      // y = aw W_down[e]^T   ; epilogue stages y per (token, slot) for combine_rows
     kDownDgrad = 2,    // G = gout_sorted W_down[e] ; epilogue dscore partials, SwiGLU bwd -> dh
-    kGateUpDgrad = 3,  // dx_p = dh W_gu[e]     ; epilogue slot-ordered scatter-sum -> dx
+    kGateUpDgrad = 3,  // dx_p = dh W_gu[e]     ; epilogue stages dx_p per (token, slot) for combine_rows
     kDownWgrad = 4,    // dW_down[e] = gout_sorted^T aw
     kGateUpWgrad = 5,  // dW_gu[e] = dh^T x_sorted
 };
