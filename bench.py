@@ -2,11 +2,12 @@
 """Benchmark of the fused MoE layer (forward + backward) on B200.
 
 One step = one full pass of the layer's hot path: routing (top-k, histogram,
-scan, permutation), the gate/up grouped GEMM with the TMA row-gather dispatch
-and the SwiGLU epilogue, the down grouped GEMM with the ordered combine, and
-the backward (down dgrad + SwiGLU backward, both weight gradients, gate/up
-dgrad with the ordered scatter, routing-score gradients), all through the C
-ABI of libmoe.so on device-resident synthetic inputs.
+scan, permutation), the dispatch (x copied into the expert-sorted layout; under
+MXFP8 gathered inside the GEMM), the gate/up grouped GEMM with the SwiGLU
+epilogue, the down grouped GEMM and the slot-ordered combine, and the backward
+(grad_out sorted, down dgrad + SwiGLU backward, both weight gradients, gate/up
+dgrad and the slot-ordered scatter into dx, routing-score gradients), all
+through the C ABI of libmoe.so on device-resident synthetic inputs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
