@@ -15,7 +15,8 @@ implementations, so torch.compile(fullgraph=True) traces through the layer
 without a graph break.  The saved routing state and activations are extra
 outputs of the forward op, kept by autograd for the backward op.  A second
 pair (`moe_forward_ckpt`, `moe_backward_ckpt`) is the recompute mode: only the
-routing state is kept, and the backward regenerates h and aw (moe_recompute).
+routing state is kept, and the backward regenerates h, aw and the sorted copy
+of x (moe_recompute).
 """
 from __future__ import annotations
 
