@@ -87,6 +87,16 @@ def test_mxfp8_sizes(lib):
     assert M.saved_sizes(sh) == M.saved_sizes(M.make_shape(16384, 2048, 128, 8, 768))
 
 
+def test_mxfp8_forward_bf16_backward_sizes(lib):
+    # MXFP8 operands in the forward workspace only; the backward's is the bf16 one
+    shape = (16384, 2048, 128, 8, 768)
+    f_bf, b_bf = M.workspace_size(M.make_shape(*shape))
+    f_mx, b_mx = M.workspace_size(M.make_shape(*shape, M.MOE_MXFP8))
+    f_mf, b_mf = M.workspace_size(M.make_shape(*shape, M.MOE_MXFP8_FWD))
+    assert f_mf == f_mx and b_mf == b_bf and b_mf < b_mx
+    assert M.saved_sizes(M.make_shape(*shape, M.MOE_MXFP8_FWD)) == M.saved_sizes(M.make_shape(*shape))
+
+
 def test_null_and_misaligned_pointers_are_rejected_before_launch(lib):
     sh = M.make_shape(256, 256, 8, 2, 128)
     saved = M.MoeSaved(*([16] * len(M.SAVED_FIELDS)))
