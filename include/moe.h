@@ -13,8 +13,9 @@
  * integration (prime-rl PR #3651)", Overview and the custom-op commit note:
  * the fused compute takes undispatched tokens plus their routing, runs in
  * bf16 and returns gradients in the inputs' dtypes.  Here the expert-parallel
- * network exchange of those pages becomes an on-GPU gather (dispatch) and an
- * ordered reduction (combine / scatter).
+ * network exchange of those pages becomes an on-GPU copy of the tokens into
+ * the expert-sorted layout (dispatch; under MXFP8 a gather inside the GEMM's
+ * operand load) and an ordered reduction (combine / scatter).
  *
  * Definitions (P = T*k token-slot pairs; pair (t,j) is flat index t*k+j):
  *   routing   idx[t,:] = the k largest logits[t,:] (ties -> lower expert index),
@@ -24,6 +25,7 @@
  *             pairs sorted by expert, tokens ascending inside an expert
  *   expert    h = W_gate_up[e] x[t]  (W_gate_up[e] is [2I,d]: gate rows then up rows)
  *             a = silu(h[0:I]) * h[I:2I];  y = W_down[e] a  (W_down[e] is [d,I])
+ *             (moe_shape_t.swiglu_limit selects the clamped form of a)
  *   combine   out[t] = sum_{j=0..k-1, in slot order} w[t,j] y_(t,j)
  *   backward  dscore[t,j] = <gout[t], y_(t,j)>,  dx, dW_gate_up, dW_down,
  *             dlogits[t,i] = w_i (dscore_i - sum_j w_j dscore_j) for chosen i, else 0
@@ -42,7 +44,9 @@
  *     out-of-range index) are recorded in a status word inside the workspace
  *     and reported by moe_get_status.
  *   - Shape limits: 1 <= k <= min(E, 64), E <= 512, d and I multiples of 128,
- *     T >= 1, T*k*max(d,2I) < 2^31.  Pointers must be 16-byte aligned.
+ *     T >= 1, P_cap*max(d,2I) < 2^31 (P_cap, the sorted-layout row capacity,
+ *     from moe_saved_sizes; about T*k + 127*E).  Pointers must be 16-byte
+ *     aligned.
  */
 #ifndef MOE_H_
 #define MOE_H_
