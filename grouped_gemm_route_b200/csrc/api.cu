@@ -54,11 +54,17 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     if (s->d % 128 != 0 || s->I % 128 != 0) return MOE_ERR_SHAPE;
     if (s->dtype != MOE_BF16 && s->dtype != MOE_MXFP8 && s->dtype != MOE_MXFP8_FWD) return MOE_ERR_ARG;
     if (!(s->swiglu_limit >= 0.f) || std::isinf(s->swiglu_limit)) return MOE_ERR_ARG;  // NaN fails the first test
+    // Element offsets inside the kernels are 32-bit: P_cap * max(d, 2I) < 2^31.
+    // T is bounded first so that no product below can overflow 64 bits.
+    constexpr int64_t kIndexLimit = int64_t(1) << 31;
+    if (s->T >= kIndexLimit) return MOE_ERR_SHAPE;
     const int64_t P = s->T * s->k;
-    const int64_t widest = s->d > 2 * s->I ? s->d : 2 * static_cast<int64_t>(s->I);
+    const int64_t widest = s->d > 2 * static_cast<int64_t>(s->I) ? s->d : 2 * static_cast<int64_t>(s->I);
     const int64_t nonempty = s->E < P ? s->E : P;
     const int64_t p_cap = (P + 127 * nonempty + 127) / 128 * 128;
-    if (p_cap * widest >= (int64_t(1) << 31) || P * s->d >= (int64_t(1) << 31)) return MOE_ERR_SHAPE;
+    if (p_cap >= (kIndexLimit + widest - 1) / widest) return MOE_ERR_SHAPE;  // p_cap * widest >= 2^31
+    // weight rows (E*2I of W_gate_up, E*d of W_down) are 32-bit tensor-map coordinates
+    if (static_cast<int64_t>(s->E) * widest >= kIndexLimit) return MOE_ERR_SHAPE;
     p->T = s->T;
     p->d = s->d;
     p->E = s->E;

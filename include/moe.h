@@ -44,8 +44,9 @@
  *     out-of-range index) are recorded in a status word inside the workspace
  *     and reported by moe_get_status.
  *   - Shape limits: 1 <= k <= min(E, 64), E <= 512, d and I multiples of 128,
- *     T >= 1, P_cap*max(d,2I) < 2^31 (P_cap, the sorted-layout row capacity,
- *     from moe_saved_sizes; about T*k + 127*E).  Pointers must be 16-byte
+ *     1 <= T < 2^31, P_cap*max(d,2I) < 2^31 (P_cap, the sorted-layout row
+ *     capacity, from moe_saved_sizes; about T*k + 127*E), E*max(d,2I) < 2^31.
+ *     Shapes past these limits return MOE_ERR_SHAPE.  Pointers must be 16-byte
  *     aligned.
  */
 #ifndef MOE_H_

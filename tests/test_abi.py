@@ -63,6 +63,30 @@ def test_invalid_shapes_are_rejected(lib, T, d, E, k, I, dtype, code):
     assert lib.moe_fwd(ctypes.byref(sh), None, None, None, None, None, None, None, 0, None) == code
 
 
+@pytest.mark.parametrize("T,d,E,k,I", [
+    (1 << 31, 128, 8, 1, 128),          # T past 2^31
+    (1 << 62, 128, 8, 8, 128),          # T * k would overflow 64 bits
+    (1 << 30, 1 << 30, 64, 64, 128),    # P_cap * d would overflow 64 bits
+    (1 << 20, 2048, 8, 8, 128),         # P_cap * d = 2^34
+    (1, (1 << 23) - 128, 512, 1, 128),  # P_cap * d just below 2^31, E * d past it (W_down rows)
+])
+def test_index_range_limits_are_rejected(lib, T, d, E, k, I):
+    sh = M.make_shape(T, d, E, k, I)
+    f = ctypes.c_size_t()
+    assert lib.moe_workspace_size(ctypes.byref(sh), ctypes.byref(f), None) == M.MOE_ERR_SHAPE
+    assert lib.moe_saved_sizes(ctypes.byref(sh), None, None) == M.MOE_ERR_SHAPE
+
+
+def test_index_range_limit_boundary(lib):
+    # P_cap * max(d, 2I) < 2^31 exactly at the edge: d = 2048, so P_cap < 2^20
+    d, E, k, I = 2048, 8, 1, 128
+    ok_T = (1 << 20) - 128 - 127 * E  # P_cap = T*k + 127*E rounded up to 128 = 2^20 - 128
+    sizes, p_cap = M.saved_sizes(M.make_shape(ok_T, d, E, k, I))
+    assert p_cap * d < (1 << 31) and p_cap == (1 << 20) - 128
+    bad = M.make_shape(ok_T + 1, d, E, k, I)  # P_cap = 2^20
+    assert lib.moe_saved_sizes(ctypes.byref(bad), None, None) == M.MOE_ERR_SHAPE
+
+
 @pytest.mark.parametrize("limit", [-1.0, float("inf"), float("nan")])
 def test_invalid_swiglu_limits_are_rejected(lib, limit):
     sh = M.make_shape(256, 256, 8, 2, 128, swiglu_limit=limit)
