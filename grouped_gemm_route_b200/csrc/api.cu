@@ -747,7 +747,9 @@ const char *moe_error_string(int code) {
     switch (code) {
         case MOE_OK: return "ok";
         case MOE_ERR_ARG: return "invalid argument (null or misaligned pointer, or k/T/E out of range)";
-        case MOE_ERR_SHAPE: return "unsupported shape (d and I must be multiples of 128; E <= 512; k <= 64)";
+        case MOE_ERR_SHAPE:
+            return "unsupported shape (d and I must be multiples of 128; E <= 512; k <= 64; T < 2^31; "
+                   "P_cap*max(d,2I) and E*max(d,2I) below 2^31)";
         case MOE_ERR_WS: return "workspace too small";
         case MOE_ERR_ARCH: return "device is not an sm_100 (B200-class) GPU";
         case MOE_ERR_LAUNCH: return "CUDA launch or runtime call failed";

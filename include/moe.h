@@ -62,7 +62,7 @@ extern "C" {
 /* Return codes. */
 #define MOE_OK 0
 #define MOE_ERR_ARG (-1)         /* null / misaligned pointer, k < 1, k > E, T < 1 ... */
-#define MOE_ERR_SHAPE (-2)       /* d or I not a multiple of 128, E or k above the limits */
+#define MOE_ERR_SHAPE (-2)       /* d or I not a multiple of 128, a size above the limits   */
 #define MOE_ERR_WS (-3)          /* workspace smaller than moe_workspace_size reports */
 #define MOE_ERR_ARCH (-4)        /* current device is not compute capability 10.0 */
 #define MOE_ERR_LAUNCH (-5)      /* a CUDA launch or runtime call failed */
