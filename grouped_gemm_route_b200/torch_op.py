@@ -55,6 +55,8 @@ def _check_inputs(x, logits, w_gate_up, w_down, top_k):
         raise ValueError("shapes: x [T,d], logits [T,E], w_gate_up [E,2I,d], w_down [E,d,I]")
     if not 1 <= top_k <= E:
         raise ValueError("need 1 <= top_k <= E")
+    if len({t.device for t in (x, logits, w_gate_up, w_down)}) != 1:
+        raise ValueError("x, logits, w_gate_up and w_down must be on one device")
 
 
 @torch.library.custom_op("ggr_b200::moe_forward", mutates_args=(), device_types="cuda")

@@ -24,3 +24,26 @@ def test_forward_and_backward_fakes_match_the_library_sizes():
         assert [tuple(t.shape) for t in g] == [(T, d), (T, E), (E, 2 * I, d), (E, d, I), (T, k)]
         assert [t.dtype for t in g] == [torch.bfloat16, torch.float32, torch.bfloat16, torch.bfloat16,
                                         torch.float32]
+
+
+def test_input_checks_reject_bad_dtypes_shapes_top_k_and_devices():
+    import pytest
+    T, d, E, I = 8, 256, 4, 128
+    x = torch.empty(T, d, dtype=torch.bfloat16)
+    lg = torch.empty(T, E, dtype=torch.float32)
+    wgu = torch.empty(E, 2 * I, d, dtype=torch.bfloat16)
+    wd = torch.empty(E, d, I, dtype=torch.bfloat16)
+    TO._check_inputs(x, lg, wgu, wd, 2)  # a valid set passes
+    with pytest.raises(TypeError):
+        TO._check_inputs(x.float(), lg, wgu, wd, 2)
+    with pytest.raises(TypeError):
+        TO._check_inputs(x, lg.double(), wgu, wd, 2)
+    with pytest.raises(ValueError):
+        TO._check_inputs(x, lg[:, :3], wgu, wd, 2)
+    with pytest.raises(ValueError):
+        TO._check_inputs(x, lg, wgu, wd.transpose(1, 2), 2)
+    for k in (0, E + 1):
+        with pytest.raises(ValueError):
+            TO._check_inputs(x, lg, wgu, wd, k)
+    with pytest.raises(ValueError, match="one device"):
+        TO._check_inputs(x, lg, wgu, wd.to("meta"), 2)
