@@ -19,7 +19,7 @@ What the layer computes (sources, by page and section):
   the routing (top scores, selected expert indices), runs in bf16 and returns
   gradients in the inputs' dtypes.
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 
 * routing: softmax over all E router logits, keep the k largest, renormalise
   over the kept k.  The k largest are chosen on the fp32 logits themselves
