@@ -45,6 +45,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <type_traits>
 
 #include "moe_internal.h"
@@ -1143,16 +1144,28 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     if (warp == 1) tmem_dealloc_pair(tmem_base, P::kTmemCols);
 }
 
+// The opt-in to more than 48 KB of dynamic shared memory belongs to a kernel
+// as loaded on one device (each device's context holds its own copy), so it,
+// and the occupancy measured with it, are cached per device.
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+    int d = -1;
+    return cudaGetDevice(&d) == cudaSuccess && d >= 0 && d < kMaxDevices ? d : -1;
+}
+
 template <int MODE, int BN, bool MX>
 cudaError_t launch_one(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
                        cudaStream_t s) {
     constexpr int kSmem = Cfg<BN, MX>::smem_bytes(ModeTraits<MODE>::kEpiWarps);
-    static bool attr_set = false;  // per instantiation; the attribute is per function and process-wide
-    if (!attr_set) {
+    static std::atomic<bool> attr_set[kMaxDevices];  // per instantiation and device
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN, MX>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     grouped_gemm_kernel<MODE, BN, MX><<<grid, ModeTraits<MODE>::kThreads, kSmem, s>>>(tmA, tmB, args);
     return cudaGetLastError();
@@ -1174,7 +1187,10 @@ cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUte
                         cudaStream_t s) {
     using P = PairCfg<MODE, 256>;
     auto *fn = grouped_gemm_pair_kernel<MODE, 256>;
-    static int max_pairs = -1;  // per instantiation: resident clusters of two
+    static std::atomic<int> max_pairs_plus1[kMaxDevices];  // per instantiation and device: resident
+                                                           // clusters of two, plus one (0: not measured)
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -1186,6 +1202,7 @@ cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUte
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    int max_pairs = max_pairs_plus1[dev].load(std::memory_order_acquire) - 1;
     if (max_pairs < 0) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes);
         if (e != cudaSuccess) return e;
@@ -1194,6 +1211,7 @@ cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUte
         e = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
         if (e != cudaSuccess) return e;
         max_pairs = n;
+        max_pairs_plus1[dev].store(n + 1, std::memory_order_release);
     }
     const int pairs = (grid / 2) < max_pairs ? grid / 2 : max_pairs;
     if (pairs < 1) return cudaErrorInvalidConfiguration;
