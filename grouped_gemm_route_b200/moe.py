@@ -117,10 +117,16 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, t):
+    """The stream to launch on: the given one, else the current stream of t's device."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(t.device)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(t):
+    """The library launches on the current CUDA device: make it t's device for the call."""
+    return torch.cuda.device(t.device)
 
 
 def saved_struct(saved: dict) -> MoeSaved:
@@ -129,8 +135,9 @@ def saved_struct(saved: dict) -> MoeSaved:
 
 def route(shape, logits, saved: dict, ws, stream=None):
     st = saved_struct(saved)
-    _check(lib().moe_route(ctypes.byref(shape), _ptr(logits), ctypes.byref(st), _ptr(ws), ws.numel(),
-                           _stream(stream)), "moe_route")
+    with _on(logits):
+        _check(lib().moe_route(ctypes.byref(shape), _ptr(logits), ctypes.byref(st), _ptr(ws), ws.numel(),
+                               _stream(stream, logits)), "moe_route")
 
 
 def route_noalloc(shape, logits, saved: dict, stream=None):
@@ -138,40 +145,46 @@ def route_noalloc(shape, logits, saved: dict, stream=None):
     route(), with the kernels' scratch in a fixed array inside the library
     instead of a caller workspace (see moe_route_noalloc in include/moe.h)."""
     st = saved_struct(saved)
-    _check(lib().moe_route_noalloc(ctypes.byref(shape), _ptr(logits), ctypes.byref(st), _stream(stream)),
-           "moe_route_noalloc")
+    with _on(logits):
+        _check(lib().moe_route_noalloc(ctypes.byref(shape), _ptr(logits), ctypes.byref(st),
+                                       _stream(stream, logits)), "moe_route_noalloc")
 
 
 def fwd(shape, x, logits, wgu, wd, out, saved: dict, ws, stream=None):
     st = saved_struct(saved)
-    _check(lib().moe_fwd(ctypes.byref(shape), _ptr(x), _ptr(logits), _ptr(wgu), _ptr(wd), _ptr(out),
-                         ctypes.byref(st), _ptr(ws), ws.numel(), _stream(stream)), "moe_fwd")
+    with _on(x):
+        _check(lib().moe_fwd(ctypes.byref(shape), _ptr(x), _ptr(logits), _ptr(wgu), _ptr(wd), _ptr(out),
+                             ctypes.byref(st), _ptr(ws), ws.numel(), _stream(stream, x)), "moe_fwd")
 
 
 def bwd(shape, gout, x, wgu, wd, saved: dict, dx, dwgu, dwd, dscore, dlogits, ws, stream=None):
     st = saved_struct(saved)
-    _check(lib().moe_bwd(ctypes.byref(shape), _ptr(gout), _ptr(x), _ptr(wgu), _ptr(wd), ctypes.byref(st),
-                         _ptr(dx), _ptr(dwgu), _ptr(dwd), _ptr(dscore), _ptr(dlogits), _ptr(ws), ws.numel(),
-                         _stream(stream)), "moe_bwd")
+    with _on(gout):
+        _check(lib().moe_bwd(ctypes.byref(shape), _ptr(gout), _ptr(x), _ptr(wgu), _ptr(wd), ctypes.byref(st),
+                             _ptr(dx), _ptr(dwgu), _ptr(dwd), _ptr(dscore), _ptr(dlogits), _ptr(ws), ws.numel(),
+                             _stream(stream, gout)), "moe_bwd")
 
 
 def recompute(shape, x, wgu, saved: dict, ws, stream=None):
     """Rewrite saved h and aw from x and W_gate_up for the routing in `saved`
     (the gate/up GEMM again, for a backward whose forward dropped them)."""
     st = saved_struct(saved)
-    _check(lib().moe_recompute(ctypes.byref(shape), _ptr(x), _ptr(wgu), ctypes.byref(st), _ptr(ws), ws.numel(),
-                               _stream(stream)), "moe_recompute")
+    with _on(x):
+        _check(lib().moe_recompute(ctypes.byref(shape), _ptr(x), _ptr(wgu), ctypes.byref(st), _ptr(ws),
+                                   ws.numel(), _stream(stream, x)), "moe_recompute")
 
 
 def get_status(ws, stream=None) -> int:
     s = ctypes.c_int()
-    _check(lib().moe_get_status(_ptr(ws), _stream(stream), ctypes.byref(s)), "moe_get_status")
+    with _on(ws):
+        _check(lib().moe_get_status(_ptr(ws), _stream(stream, ws), ctypes.byref(s)), "moe_get_status")
     return int(s.value)
 
 
 def selftest_wait_timeout(ws, stream=None):
     """Launch the kernel whose bounded wait must expire (see include/moe.h)."""
-    _check(lib().moe_selftest_wait_timeout(_ptr(ws), _stream(stream)), "moe_selftest_wait_timeout")
+    with _on(ws):
+        _check(lib().moe_selftest_wait_timeout(_ptr(ws), _stream(stream, ws)), "moe_selftest_wait_timeout")
 
 
 def kernel_names():
