@@ -31,8 +31,9 @@
  *             dlogits[t,i] = w_i (dscore_i - sum_j w_j dscore_j) for chosen i, else 0
  *
  * Conventions for every entry point:
- *   - All pointers are DEVICE pointers unless stated otherwise; every tensor is
- *     row-major and contiguous.  bf16 = IEEE bfloat16 (2 bytes).
+ *   - All pointers are DEVICE pointers unless stated otherwise, in memory of the
+ *     current CUDA device (cudaSetDevice), on which every call launches; every
+ *     tensor is row-major and contiguous.  bf16 = IEEE bfloat16 (2 bytes).
  *   - The caller owns and allocates every buffer (outputs, saved state and the
  *     workspace).  The library never allocates or frees device memory and keeps
  *     no state between calls except cached per-device properties.
