@@ -147,3 +147,43 @@ def test_error_strings_and_kernel_names(lib):
     names = M.kernel_names()
     assert names[0] == "route_topk" and "gemm_gateup_fwd" in names
     assert {"route_bwd", "sort_rows", "mx_quant"} <= set(names)
+
+
+def test_other_entry_points_reject_bad_arguments_on_the_host(lib):
+    sh = M.make_shape(256, 256, 8, 2, 128)
+    bad_shape = M.make_shape(256, 200, 8, 2, 128)
+    saved = M.MoeSaved(*([16] * len(M.SAVED_FIELDS)))
+    misaligned = M.MoeSaved(*([16] * 2 + [20] + [16] * (len(M.SAVED_FIELDS) - 3)))
+    # moe_route: shape, pointers, workspace size
+    assert lib.moe_route(ctypes.byref(bad_shape), 16, ctypes.byref(saved), 16, 1 << 40, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_route(ctypes.byref(sh), None, ctypes.byref(saved), 16, 1 << 40, None) == M.MOE_ERR_ARG
+    assert lib.moe_route(ctypes.byref(sh), 16, ctypes.byref(misaligned), 16, 1 << 40, None) == M.MOE_ERR_ARG
+    assert lib.moe_route(ctypes.byref(sh), 16, None, 16, 1 << 40, None) == M.MOE_ERR_ARG
+    assert lib.moe_route(ctypes.byref(sh), 16, ctypes.byref(saved), 16, 64, None) == M.MOE_ERR_WS
+    # moe_recompute
+    assert lib.moe_recompute(ctypes.byref(bad_shape), 16, 16, ctypes.byref(saved), 16, 1 << 40,
+                             None) == M.MOE_ERR_SHAPE
+    assert lib.moe_recompute(ctypes.byref(sh), 16, 24, ctypes.byref(saved), 16, 1 << 40, None) == M.MOE_ERR_ARG
+    assert lib.moe_recompute(ctypes.byref(sh), 16, 16, ctypes.byref(saved), 16, 64, None) == M.MOE_ERR_WS
+    # moe_route_noalloc: shape, pointers, and the fixed scratch's capacity (ceil(T/64) * E <= 131072)
+    assert lib.moe_route_noalloc(ctypes.byref(bad_shape), 16, ctypes.byref(saved), None) == M.MOE_ERR_SHAPE
+    assert lib.moe_route_noalloc(ctypes.byref(sh), 16, None, None) == M.MOE_ERR_ARG
+    assert lib.moe_route_noalloc(ctypes.byref(sh), 16, ctypes.byref(misaligned), None) == M.MOE_ERR_ARG
+    big = M.make_shape(64 * 1025, 128, 128, 1, 128)  # 1025 blocks x 128 experts > 131072
+    assert lib.moe_route_noalloc(ctypes.byref(big), 16, ctypes.byref(saved), None) == M.MOE_ERR_SCRATCH_LIMIT
+    # status word, self-test
+    st = ctypes.c_int()
+    assert lib.moe_get_status(None, None, ctypes.byref(st)) == M.MOE_ERR_ARG
+    assert lib.moe_get_status(16, None, None) == M.MOE_ERR_ARG
+    assert lib.moe_selftest_wait_timeout(None, None) == M.MOE_ERR_ARG
+    assert lib.moe_selftest_wait_timeout(20, None) == M.MOE_ERR_ARG
+
+
+def test_profile_read_without_records_returns_zeros(lib):
+    n = len(M.kernel_names())
+    assert lib.moe_profile_enable(0) == M.MOE_OK
+    ms = (ctypes.c_double * n)(*([7.0] * n))
+    cnt = (ctypes.c_int64 * n)(*([7] * n))
+    assert lib.moe_profile_read(ms, cnt, n) == M.MOE_OK
+    assert list(ms) == [0.0] * n and list(cnt) == [0] * n
+    assert lib.moe_kernel_name(-1) is None and lib.moe_kernel_name(n) is None
