@@ -224,7 +224,10 @@ const char *moe_error_string(int code);
  * the recorded events and returns, per kernel kind (0 <= kind < n_kinds), the
  * summed device milliseconds and the launch count since the last reset, then
  * resets.  moe_kernel_name names a kind ("route_topk", "gemm_gateup_fwd" ...),
- * or returns NULL past the last kind.  Host-side bookkeeping only. */
+ * or returns NULL past the last kind.  Host-side bookkeeping only.  The timing
+ * events are pooled for the whole process: profile one device per process (a
+ * launch timed on another device than the events' own makes moe_profile_read
+ * return MOE_ERR_LAUNCH; the layer's results are not affected). */
 int moe_profile_enable(int on);
 int moe_profile_read(double *ms, int64_t *launches, int n_kinds);
 const char *moe_kernel_name(int kind);
