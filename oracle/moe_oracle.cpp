@@ -30,9 +30,8 @@
 //    "Mario/overlap moe kernel integration (prime-rl PR #3651)" says the kernel
 //    computes; no formula on the pages): with limit L > 0,
 //    a = silu(min(gate, L)) * clip(up, -L, L), the gradient passing where the
-//    input lies in the closed interval; limit 0 is the plain SwiGLU.  The side
-//    of a clamp is decided on h rounded to bfloat16 (bf16_round), the precision
-//    in which the layer keeps h between forward and backward.
+//    input lies in the closed interval (end points inside), decided on the
+//    exact pre-activation; limit 0 is the plain SwiGLU.
 //  * combine and dx scatter: sums over slots j = 0..k-1 in slot order.
 //  * dscore[t, j] = dL/dw[t, j]; dlogits through the renormalised softmax.
 //
@@ -67,23 +66,16 @@ double act(double g, double u, double L) {
     return silu(g) * u;
 }
 
-// Nearest bfloat16 value (8 significant bits, ties to even), as a double.
-double bf16_round(double v) {
-    int e = 0;
-    const double m = std::frexp(v, &e);  // v = m * 2^e, 0.5 <= |m| < 1
-    return std::ldexp(std::nearbyint(m * 256.0), e - 8);  // default rounding: to nearest, ties to even
-}
-
 // (dg, du) of act for dL/da = da; a clamp stops the gradient outside its
-// interval, the side decided on the bfloat16-rounded input.
+// closed interval.
 void act_grad(double g, double u, double L, double da, double *dg, double *du) {
     double gc = g, uc = u;
     if (L > 0) {
         gc = std::min(g, L);
         uc = std::min(std::max(u, -L), L);
     }
-    *dg = (L > 0 && bf16_round(g) > L) ? 0.0 : da * uc * silu_grad(gc);
-    *du = (L > 0 && std::fabs(bf16_round(u)) > L) ? 0.0 : da * silu(gc);
+    *dg = (L > 0 && g > L) ? 0.0 : da * uc * silu_grad(gc);
+    *du = (L > 0 && std::fabs(u) > L) ? 0.0 : da * silu(gc);
 }
 
 // Run fn(e) for every expert e, experts dealt round-robin to n threads.

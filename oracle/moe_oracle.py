@@ -37,10 +37,10 @@ Readings taken where the pages are silent:
   which it does not): the pages give no formula.  Reading: with a limit
   L > 0, a = silu(min(h_gate, L)) * clip(h_up, -L, L); the gradient passes
   where the input lies in the closed interval (h_gate <= L, |h_up| <= L) and
-  is zero outside it.  limit = 0 is the plain SwiGLU above.  Which side of a
-  clamp an element lies on is a discrete decision taken by floating point, so
-  the backward takes it on h rounded to bfloat16, the precision in which the
-  layer keeps h between forward and backward (bf16_round).
+  is zero outside it.  limit = 0 is the plain SwiGLU above.  Both the clamp
+  and the side of it on which the gradient stops are taken on the exact
+  pre-activation (the definition's derivative, with the closed interval's
+  end points counted inside).
 * combine: out[t] = sum over slots j = 0..k-1, in slot order, of w[t,j] y_(t,j).
 * dscore[t,j] is the gradient with respect to the renormalised weight w[t,j];
   dlogits is the gradient with respect to the router logits through the
@@ -82,13 +82,6 @@ def silu_grad(z):
     return s * (1.0 + z * (1.0 - s))
 
 
-def bf16_round(v):
-    """Nearest bfloat16 value of v (8 significant bits, ties to even), in float64."""
-    v = np.asarray(v, dtype=np.float64)
-    m, e = np.frexp(v)  # v = m * 2^e, 0.5 <= |m| < 1
-    return np.ldexp(np.rint(m * 256.0), e - 8)  # np.rint rounds half to even
-
-
 def _clamps(g, u, limit):
     """(gate, up) after the clamp of the clamped SwiGLU; unchanged for limit = 0."""
     g, u = np.asarray(g, dtype=np.float64), np.asarray(u, dtype=np.float64)
@@ -108,16 +101,16 @@ def swiglu_backward(g, u, da, limit=0.0):
 
     Inside the clamps: dg = da * uc * silu'(gc), du = da * silu(gc).  A clamp
     passes the gradient where its input lies in the closed interval and stops
-    it outside (g > limit, |u| > limit), the side decided on bf16_round(g) and
-    bf16_round(u).
+    it outside (g > limit, |u| > limit), decided on g and u themselves.
     """
+    g, u = np.asarray(g, dtype=np.float64), np.asarray(u, dtype=np.float64)
     gc, uc = _clamps(g, u, limit)
     da = np.asarray(da, dtype=np.float64)
     dg = da * uc * silu_grad(gc)
     du = da * silu(gc)
     if limit > 0:
-        dg = np.where(bf16_round(g) <= limit, dg, 0.0)
-        du = np.where(np.abs(bf16_round(u)) <= limit, du, 0.0)
+        dg = np.where(g <= limit, dg, 0.0)
+        du = np.where(np.abs(u) <= limit, du, 0.0)
     return dg, du
 
 

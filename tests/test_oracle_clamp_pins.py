@@ -6,11 +6,13 @@
 * a limit above every pre-activation gives the plain layer bit for bit;
 * central finite differences of the clamped forward for every gradient, on
   inputs whose pre-activations stay well away from the clamps' corners;
-* the side of a clamp is decided on h rounded to bfloat16: bf16_round is
-  pinned against torch's float32 -> bfloat16 conversion and hand-worked ties,
-  and swiglu_backward against points just inside and outside a clamp;
-* a planted mistake (the gate clamped from below instead of above) fails the
-  closed form.
+* the side of a clamp is decided on the exact pre-activation, with the end
+  points of the closed interval inside: a closed form on experts whose gate
+  pre-activation lands exactly on the limit, or a quarter of a bfloat16 step
+  above it (where a rule that rounded h to bfloat16 first would put it
+  inside), written with scalar math;
+* planted mistakes fail the closed forms: the gate clamped from below instead
+  of above, the side decided on h rounded to bfloat16, and an open interval.
 """
 import math
 
@@ -172,26 +174,110 @@ def test_planted_mistake_gate_clamped_from_below(monkeypatch):
         test_identity_experts_closed_form(1.5)
 
 
-def test_bf16_round_matches_torch_conversion():
+def _bf16(v):
+    """float64 -> nearest bfloat16 -> float64, through torch (used only to plant a mistake)."""
     import torch
-    rng = np.random.default_rng(11)
-    v = np.concatenate([rng.standard_normal(4000) * np.exp(rng.uniform(-20, 20, 4000)),
-                        [0.0, -0.0, 1.0, 0.2, 0.1875, -3.75e-3]]).astype(np.float32)
-    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
-    assert np.array_equal(O.bf16_round(v.astype(np.float64)), ref)
-    # hand-worked ties: halfway values go to the even 8-bit significand
-    assert O.bf16_round(1.0 + 2.0 ** -8) == 1.0
-    assert O.bf16_round(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
-    assert O.bf16_round(-(1.0 + 3 * 2.0 ** -8)) == -(1.0 + 2.0 ** -6)
+    return torch.from_numpy(np.asarray(v, dtype=np.float64)).to(torch.bfloat16).to(torch.float64).numpy()
 
 
-def test_clamp_side_is_decided_on_bf16_h():
-    L = 0.25  # a bfloat16 value; the bf16 spacing just above it is 2^-9
-    g = np.array([L + 1e-6, L + 2.0 ** -9, L - 1e-6, 0.1])
-    u = np.array([0.1, 0.1, 0.1, -(L + 1e-6)])
-    dg, du = O.swiglu_backward(g, u, np.ones(4), L)
-    assert dg[0] != 0.0  # rounds to L: inside
-    assert dg[1] == 0.0  # the next bf16 value: outside
-    assert dg[2] != 0.0 and dg[3] != 0.0
-    assert du[3] != 0.0  # -(L + 1e-6) rounds to -L: inside
-    assert np.all(du[:3] != 0.0)
+SIDE_L = 0.5
+SIDE_EPS = 2.0 ** -10  # weight of the neighbouring input in the gate rows
+
+
+def side_layer():
+    """One expert (E = k = 1, so w = 1), d = I = 4: W_gate = Id + eps * S with S
+    the cyclic shift (g_i = x_i + eps * x_(i+1 mod 4)), W_up = Id, W_down = Id.
+
+    Token 0: g_0 = L + eps / 4 = L + 2^-12, a quarter of the bfloat16 spacing
+    (2^-8) above L: outside the gate's interval, although bfloat16 rounding
+    would give exactly L.  Token 1: g_0 = L exactly and u_2 = -L exactly: both
+    on the closed interval's end points, inside.  Token 2: u_1 = L + 2^-12,
+    just outside the up clamp (bfloat16 rounding would again give L)."""
+    L, eps, d = SIDE_L, SIDE_EPS, 4
+    x = np.array([[L, 0.25, 0.1, -0.3],
+                  [L, 0.0, -L, 0.2],
+                  [0.1, L + 2.0 ** -12, 0.0, 0.05]])
+    shift = np.roll(np.eye(d), 1, axis=1)  # (S x)_i = x_(i+1 mod d)
+    wgu = np.concatenate([np.eye(d) + eps * shift, np.eye(d)])[None]
+    wd = np.eye(d)[None]
+    logits = np.zeros((x.shape[0], 1), dtype=np.float32)
+    gout = np.array([[1.0, -0.5, 0.25, 2.0], [0.75, 1.5, -1.0, 0.5], [-2.0, 1.25, 0.3, 0.9]])
+    return x, logits, wgu, wd, gout
+
+
+def side_closed_form(x, gout):
+    """out and dx of side_layer by scalar math: gate g_i = x_i + eps x_(i+1),
+    up u_i = x_i; a_i = silu(min(g_i, L)) clip(u_i, -L, L); out = a;
+    dx_j = dg_j + eps dg_(j-1) + du_j, with dg_i = gout_i clip(u_i) silu'(min(g_i, L))
+    where g_i <= L (else 0) and du_i = gout_i silu(min(g_i, L)) where |u_i| <= L (else 0)."""
+    L, eps = SIDE_L, SIDE_EPS
+    T, d = x.shape
+    out = np.zeros((T, d))
+    dx = np.zeros((T, d))
+    for t in range(T):
+        dg, du = [0.0] * d, [0.0] * d
+        for i in range(d):
+            g = x[t, i] + eps * x[t, (i + 1) % d]
+            u = x[t, i]
+            gc = g if g <= L else L
+            uc = -L if u < -L else (L if u > L else u)
+            out[t, i] = py_silu(gc) * uc
+            s = py_sigmoid(gc)
+            dg[i] = gout[t, i] * uc * s * (1 + gc * (1 - s)) if g <= L else 0.0
+            du[i] = gout[t, i] * py_silu(gc) if -L <= u <= L else 0.0
+        for j in range(d):
+            dx[t, j] = dg[j] + eps * dg[(j - 1) % d] + du[j]
+    return out, dx
+
+
+def test_clamp_side_closed_form():
+    x, logits, wgu, wd, gout = side_layer()
+    ref_out, ref_dx = side_closed_form(x, gout)
+    f = O.forward(x, logits, wgu, wd, 1, limit=SIDE_L)
+    g = O.backward(x, logits, wgu, wd, 1, gout, f, limit=SIDE_L)
+    assert np.allclose(f["out"], ref_out, rtol=1e-13, atol=1e-15)
+    assert np.allclose(g["dx"], ref_dx, rtol=1e-13, atol=1e-15)
+    # the cases the layer was built for do occur in the oracle's own h
+    h = f["h"]
+    assert h[0, 0] > SIDE_L and _bf16(h[0, 0]) == SIDE_L
+    assert h[1, 0] == SIDE_L and h[1, 4 + 2] == -SIDE_L
+    assert h[2, 4 + 1] > SIDE_L and _bf16(h[2, 4 + 1]) == SIDE_L
+
+
+def test_clamp_side_closed_form_cpp():
+    from oracle import cpp_oracle as C
+    x, logits, wgu, wd, gout = side_layer()
+    _, ref_dx = side_closed_form(x, gout)
+    g = C.backward(x, logits, wgu, wd, 1, gout, nthreads=1, limit=SIDE_L)
+    assert np.allclose(g["dx"], ref_dx, rtol=1e-13, atol=1e-15)
+
+
+def _planted_backward(decide):
+    """swiglu_backward with the clamp side taken by `decide(g, u, limit)`."""
+    def backward(g, u, da, limit=0.0):
+        g, u = np.asarray(g, dtype=np.float64), np.asarray(u, dtype=np.float64)
+        gc, uc = O._clamps(g, u, limit)
+        da = np.asarray(da, dtype=np.float64)
+        dg, du = da * uc * O.silu_grad(gc), da * O.silu(gc)
+        if limit > 0:
+            keep_g, keep_u = decide(g, u, limit)
+            dg, du = np.where(keep_g, dg, 0.0), np.where(keep_u, du, 0.0)
+        return dg, du
+    return backward
+
+
+@pytest.mark.parametrize("rule", ["bf16_side", "open_interval"])
+def test_planted_wrong_side_rule_fails_closed_form(monkeypatch, rule):
+    if rule == "bf16_side":
+        decide = lambda g, u, L: (_bf16(g) <= L, np.abs(_bf16(u)) <= L)  # noqa: E731
+    else:
+        decide = lambda g, u, L: (g < L, np.abs(u) < L)  # noqa: E731
+    monkeypatch.setattr(O, "swiglu_backward", _planted_backward(decide))
+    with pytest.raises(AssertionError):
+        test_clamp_side_closed_form()
+
+
+def test_planted_right_side_rule_passes(monkeypatch):
+    """The planting harness itself: with the definition's rule it passes."""
+    monkeypatch.setattr(O, "swiglu_backward", _planted_backward(lambda g, u, L: (g <= L, np.abs(u) <= L)))
+    test_clamp_side_closed_form()
