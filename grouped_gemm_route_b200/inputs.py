@@ -82,6 +82,33 @@ def make_inputs(T, d, E, k, I, seed=0, device="cpu", zipf_s=None, with_grad=True
     return {name: t.to(device).contiguous() for name, t in out.items()}
 
 
+def make_grid_inputs(T, d, E, k, I, seed=0, device="cpu", **_):
+    """Inputs on coarse grids, for checks where a discrete decision taken on a
+    pre-activation must not depend on rounding (the sides of the clamped
+    SwiGLU's clamps).
+
+    x = n / 4 with n uniform in -4..4; W_gate_up and W_down = m / 64 with m
+    uniform in -3..3; grad_out ~ N(0,1) and router logits ~ N(0,1) as in
+    make_inputs.  Every product x * W is a multiple of 2^-8 and every gate/up
+    pre-activation h = W_gate_up x is an exact multiple of 2^-8 in float32
+    (|h| stays far below 2^16), exactly representable in bfloat16 while
+    |h| < 1, and E4M3 block quantisation leaves x and the weights unchanged.
+    A limit strictly between two multiples of 2^-8 is therefore on the same
+    side of every h whether h is taken exactly, in float32 or rounded to
+    bfloat16."""
+    def grid(shape, tensor, half_range, step):
+        n = torch.randint(-half_range, half_range + 1, shape, generator=_gen(seed, tensor))
+        return (n.to(torch.float32) * step).to(torch.bfloat16)
+    out = dict(
+        x=grid((T, d), "x", 4, 0.25),
+        logits=make_logits(T, E, seed),
+        wgu=grid((E, 2 * I, d), "wgu", 3, 1.0 / 64),
+        wd=grid((E, d, I), "wd", 3, 1.0 / 64),
+        gout=_randn((T, d), seed, "gout"),
+    )
+    return {name: t.to(device).contiguous() for name, t in out.items()}
+
+
 def make_workload(name: str, seed=0, device="cpu", with_grad=True):
     cfg = dict(WORKLOADS[name])
     return cfg, make_inputs(seed=seed, device=device, with_grad=with_grad, **cfg)

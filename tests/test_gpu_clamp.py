@@ -1,14 +1,23 @@
 """GPU parity of the clamped SwiGLU (swiglu_limit L > 0: a = silu(min(gate, L))
 * clamp(up, -L, L)) against the oracle, in bf16 and MXFP8, forward and
-backward.  The backward's clamp sides are decided on bf16 h on both sides.  h holds the unclamped pre-activations; aw the weighted clamped
+backward.  h holds the unclamped pre-activations; aw the weighted clamped
 activation.  A limit above every pre-activation must give the plain layer bit
-for bit, and recompute mode must give the clamped layer bit for bit."""
+for bit, and recompute mode must give the clamped layer bit for bit.
+
+The oracle decides each clamp's side on the exact pre-activation; the kernels
+decide on their float32 accumulator (forward) and on the bfloat16 h they saved
+(backward).  The parity cases therefore take their inputs on coarse grids
+(inputs.make_grid_inputs), where every pre-activation is an exact multiple of
+2^-8, and limits strictly between two such multiples: the three precisions put
+every element on the same side of every clamp, so the comparison measures the
+arithmetic, not a different set of decisions."""
 import numpy as np
 import pytest
 import torch
 
 from grouped_gemm_route_b200 import moe as M
 from grouped_gemm_route_b200 import torch_op as TO
+from grouped_gemm_route_b200 import inputs as IN
 from helpers import TOL_BF16, TOL_MXFP8, check_routing, f64, make, normwise, run_layer, sorted_rows
 from oracle import moe_oracle as O
 
@@ -47,20 +56,33 @@ def clamp_check(cfg, inp, L, dtype):
     return errs
 
 
-# limits are bfloat16 values, so that the kernel's float32 limit and the oracle's agree exactly
+def make_grid(sizes, seed):
+    cfg = dict(IN.WORKLOADS[sizes]) if isinstance(sizes, str) else dict(sizes)
+    cfg.pop("dtype", None)
+    return cfg, IN.make_grid_inputs(seed=seed, **cfg)
+
+
+def off_grid(L):
+    """The limit lies strictly between two multiples of 2^-8 (and is exact in float32)."""
+    return (L * 256) % 1 != 0 and float(np.float32(L)) == L
+
+
+# limits are odd multiples of 2^-9: between two grid values of h
 @pytest.mark.parametrize("sizes,L", [
-    ("tiny", 0.1875),
-    (dict(T=700, d=512, E=12, k=3, I=256), 0.3125),
-    (dict(T=1000, d=384, E=16, k=4, I=384), 0.25),
+    ("tiny", 155 / 512),
+    (dict(T=700, d=512, E=12, k=3, I=256), 181 / 512),
+    (dict(T=1000, d=384, E=16, k=4, I=384), 129 / 512),
 ])
 def test_clamped_bf16(sizes, L):
-    cfg, inp = make(sizes, seed=17)
+    assert off_grid(L)
+    cfg, inp = make_grid(sizes, seed=17)
     clamp_check(cfg, inp, L, M.MOE_BF16)
 
 
-@pytest.mark.parametrize("sizes,L", [("tiny", 0.1875), (dict(T=700, d=512, E=12, k=3, I=256), 0.3125)])
+@pytest.mark.parametrize("sizes,L", [("tiny", 155 / 512), (dict(T=700, d=512, E=12, k=3, I=256), 181 / 512)])
 def test_clamped_mxfp8(sizes, L):
-    cfg, inp = make(sizes, seed=19)
+    assert off_grid(L)
+    cfg, inp = make_grid(sizes, seed=19)
     clamp_check(cfg, inp, L, M.MOE_MXFP8)
 
 
@@ -77,8 +99,8 @@ def test_limit_above_every_preactivation_is_the_plain_layer_bitwise():
 
 
 def test_clamped_torch_op_recompute_is_bitwise_and_grads_in_input_dtype():
-    cfg, inp = make("tiny", seed=29)
-    k, L, dev = cfg["k"], 0.1875, "cuda:0"
+    cfg, inp = make_grid("tiny", seed=29)
+    k, L, dev = cfg["k"], 155 / 512, "cuda:0"
     gout = inp["gout"].to(dev)
     runs = []
     for recompute in (False, True):

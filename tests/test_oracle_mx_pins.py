@@ -174,3 +174,81 @@ def test_backward_on_given_h():
     bm = O.backward(x, logits, wgu, wd, k, gout, fm, h=fm["h"])
     rel = np.linalg.norm(bm["dscore"] - b["dscore"]) / np.linalg.norm(b["dscore"])
     assert 1e-4 < rel < 0.1
+
+
+# ----------------------------------------------------------------------------
+# Where the weight-gradient blocks start.  Reading: the K dimension of a weight
+# gradient is one expert's own tokens, in dispatch order (tokens ascending), and
+# its blocks of 32 start at that expert's first token -- a property of the
+# expert alone, not of where its group sits among the other experts' pairs.
+# ----------------------------------------------------------------------------
+def _block_origin_case(split):
+    """k = 1, E = 3.  Tokens 37..99 go to expert 1 in both variants; tokens
+    0..split-1 go to expert 0 and split..36 to expert 2, so expert 1's first
+    sorted position is `split` while its own token sequence stays the same."""
+    rng = np.random.default_rng(5)
+    T, d, E, I = 100, 64, 3, 32
+    x = rng.standard_normal((T, d))
+    gout = rng.standard_normal((T, d))
+    # a large row at expert 1's 29th token: which rows share its block (and so
+    # its scale) depends on where the blocks start
+    gout[37 + 28] *= 64.0
+    wgu = rng.standard_normal((E, 2 * I, d)) * 0.2
+    wd = rng.standard_normal((E, d, I)) * 0.2
+    choice = np.where(np.arange(T) < split, 0, np.where(np.arange(T) < 37, 2, 1))
+    logits = np.full((T, E), -4.0, dtype=np.float32)
+    logits[np.arange(T), choice] = 4.0
+    logits += rng.uniform(0, 0.5, (T, E)).astype(np.float32)  # weights vary per token
+    logits[np.arange(T), choice] += 4.0
+    return x, logits, wgu, wd, gout
+
+
+def _qdq32_loop(rows):
+    """Blocks of 32 consecutive rows, the first starting at row 0, each column
+    of a block quantised with its own scale: a plain loop over the blocks."""
+    rows = np.asarray(rows, dtype=np.float64)
+    out = np.zeros_like(rows)
+    for b0 in range(0, rows.shape[0], 32):
+        blk = rows[b0:b0 + 32]
+        for c in range(rows.shape[1]):
+            col = blk[:, c]
+            amax = float(np.max(np.abs(col)))
+            s = 0
+            if amax > 0:
+                s = -127
+                while amax > 448.0 * 2.0 ** s:
+                    s += 1
+            out[b0:b0 + 32, c] = O.e4m3_round(col / 2.0 ** s) * 2.0 ** s
+    return out
+
+
+def test_wgrad_blocks_start_at_the_experts_first_token():
+    dws = []
+    for split in (37, 30):
+        x, logits, wgu, wd, gout = _block_origin_case(split)
+        f = O.forward_mx(x, logits, wgu, wd, 1)
+        assert int(f["offsets"][1]) == split and int(f["counts"][1]) == 63
+        b = O.backward_mx(x, logits, wgu, wd, 1, gout, f)
+        dws.append(b["dwd"][1])
+        # brute force on expert 1's own token sequence (tokens 37..99 ascending)
+        pairs = f["perm"][f["offsets"][1]:f["offsets"][2]].astype(np.int64)
+        assert np.array_equal(pairs, np.arange(37, 100))
+        ref = _qdq32_loop(gout[pairs]).T @ _qdq32_loop(f["aw"][pairs])
+        assert np.allclose(b["dwd"][1], ref, rtol=1e-13, atol=1e-13)
+    # expert 1's gradient does not move when its group's start among the sorted pairs moves
+    assert np.array_equal(dws[0], dws[1])
+
+
+def test_wgrad_block_origin_pin_discriminates():
+    """Blocks aligned to the global sorted position instead (origin 0 of all
+    pairs) give a different dW_down for the expert that starts at 37."""
+    x, logits, wgu, wd, gout = _block_origin_case(37)
+    f = O.forward_mx(x, logits, wgu, wd, 1)
+    b = O.backward_mx(x, logits, wgu, wd, 1, gout, f)
+    lo, hi = int(f["offsets"][1]), int(f["offsets"][2])
+    pairs = f["perm"][lo:hi].astype(np.int64)
+    pad = lo % 32  # rows of the global block that belong to expert 0: zeros here
+    g = np.concatenate([np.zeros((pad, gout.shape[1])), gout[pairs]])
+    a = np.concatenate([np.zeros((pad, f["aw"].shape[1])), f["aw"][pairs]])
+    glob = _qdq32_loop(g).T @ _qdq32_loop(a)
+    assert not np.allclose(b["dwd"][1], glob, rtol=1e-6, atol=1e-9)
