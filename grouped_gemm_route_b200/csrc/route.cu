@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
             }
         }
         // weights: exp(l_j - l_max) over the chosen k, normalised by their sum
-        // (a fixed shuffle tree over the slots)
+        // taken in slot order (the same sum, bit for bit, as the lane form's)
 #pragma unroll
         for (int u = 0; u < kTokPar; ++u) {
             const int tt = t + u;
@@ -467,10 +467,8 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
             for (int h = 0; h < 2; ++h) {
                 const int j = lane + 32 * h;
                 p[h] = j < k ? expf(topk_value(static_cast<uint32_t>(sel[u][h] >> 32)) - m) : 0.f;
-                sum += p[h];
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, j < 32 ? p[0] : p[1], j & 31);
             if (tt < wt1) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {

@@ -13,8 +13,14 @@
 // GPU that loads the library keeps it until the process exits.  In host code
 // the array's name is only a host-side stand-in, so its device address is
 // looked up with cudaGetSymbolAddress once per device, with that device
-// current, on the first call made on that device.
+// current, on the first call made on that device.  The address is kept with
+// the identifier of the context it belongs to; a call that finds another
+// context current (cudaDeviceReset destroys the device's primary context and
+// the next runtime call creates a new one, with the module loaded anew) looks
+// the address up again.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -34,16 +40,45 @@ static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
 std::mutex g_scratch_mu;
 void *g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context identifier the address belongs to
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
 
-// Device address of g_route_scratch on the current device (looked up once).
+// Identifier of the current context (0: none current yet, or not available).
+unsigned long long current_context_id() {
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_route_scratch on the current device: looked up on the
+// first call on a device, and again whenever the current context is not the
+// one the cached address was taken in.
 int scratch_address(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_LAUNCH;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (g_ctx_current == nullptr || g_ctx_id == nullptr) {
+        void *f1 = nullptr, *f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 4000, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || f1 == nullptr ||
+            cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess || f2 == nullptr)
+            return MOE_ERR_LAUNCH;
+        g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+        g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
+    }
+    const unsigned long long ctx = current_context_id();
+    if (g_scratch_addr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_LAUNCH;
+        const unsigned long long now = current_context_id();  // the lookup makes the context current
+        if (now == 0) return MOE_ERR_LAUNCH;
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = now;
     }
     *out = g_scratch_addr[dev];
     return MOE_OK;

@@ -177,8 +177,10 @@ int moe_recompute(const moe_shape_t *shape, const void *x, const void *w_gate_up
  * gives none to plug-ins, or code on a latency-critical path where an
  * allocation (which may synchronise the whole device) is not acceptable.
  *
- * Same results as moe_route, bit for bit (it runs the three-launch form of
- * the same routing: top-k, scan, permutation), but the per-block histograms and
+ * Same results as moe_route, bit for bit: indices, weights, counts, offsets,
+ * group starts, tile table, permutation and its inverse (it runs the
+ * three-launch form of the same routing: top-k, scan, permutation; every form
+ * sums a token's k exponentials in slot order), but the per-block histograms and
  * bases that it keeps in a workspace live instead in a fixed
  * 1 MiB __device__ array inside the library, which every GPU that loads the
  * library holds until the process exits.  The caller still allocates and
@@ -193,8 +195,11 @@ int moe_recompute(const moe_shape_t *shape, const void *x, const void *w_gate_up
  * rules and error codes are those of moe_route.
  *
  * The first call on each device looks up the array's device address with
- * cudaGetSymbolAddress (with that device current) and caches it; make that
- * first call before any stream capture.  All calls share the one array and it
+ * cudaGetSymbolAddress (with that device current) and caches it together with
+ * the identifier of the current context; make that first call before any
+ * stream capture.  A call that finds a different context current (after
+ * cudaDeviceReset, for example) looks the address up again, so the first call
+ * after a reset must also come before any capture.  All calls share the one array and it
  * keeps the last call's contents; every word a call reads is written earlier in
  * the same call, so nothing needs clearing.  Calls that overlap on the GPU (on
  * different streams, or from different host threads) race on the array and
