@@ -32,6 +32,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "fused MoE layer fwd+bwd TFLOP/s & % of bf16 tensor peak (Qwen3-30B-A3B shape)"
 UNIT = "TFLOP/s"
+# workloads timed after the headline one and reported in the same JSON line
+OTHER_WORKLOADS = ("qwen3_235b_a22b", "qwen3_30b_a3b_skew", "qwen3_30b_a3b_mxfp8", "tiny")
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 
 
@@ -60,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-routing-sweep", action="store_true",
                     help="skip the routing-only timing over token counts")
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0 = auto)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other workloads (reported under 'configs')")
     ap.add_argument("--override", default="", help="comma list of size overrides, e.g. T=4096,E=32 "
                                                      "(smaller profiling cases; not a bench workload)")
     return ap.parse_args()
@@ -293,6 +297,120 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------
+# timing helpers (our arm)
+# ----------------------------------------------------------------------------
+def timed_loop(step, n_steps, stream, dev, barrier):
+    """Device time of n_steps calls of step(), CUDA events on the launching
+    stream, a barrier and a synchronize on both sides; ms per step."""
+    import torch
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(n_steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    return t0.elapsed_time(t1) / n_steps
+
+
+def profiled_loop(M, step, n_steps, stream, dev, barrier):
+    """The same steps with the library's per-kernel events on: returns
+    {kernel: (total ms, launches)} and the loop's ms per step."""
+    M.profile_read()
+    M.profile_enable(True)
+    try:
+        ms = timed_loop(step, n_steps, stream, dev, barrier)
+    finally:
+        M.profile_enable(False)
+    return M.profile_read(), ms
+
+
+def gemm_flops_per_launch(T, d, k, I):
+    """Algorithmic FLOPs of one launch of each grouped GEMM (P = T*k pairs)."""
+    P = T * k
+    return {"gemm_gateup_fwd": 4.0 * P * d * I, "gemm_down_fwd_combine": 2.0 * P * I * d,
+            "gemm_down_dgrad": 2.0 * P * d * I, "gemm_down_wgrad": 2.0 * P * d * I,
+            "gemm_gateup_dgrad_scatter": 4.0 * P * d * I, "gemm_gateup_wgrad": 4.0 * P * d * I}
+
+
+def kernel_breakdown(per_kernel, n_steps):
+    total = sum(v[0] for v in per_kernel.values()) or 1.0
+    return {n: {"ms_per_step": v[0] / n_steps, "share": v[0] / total, "launches": v[1]}
+            for n, v in per_kernel.items() if v[1]}
+
+
+def tensor_peaks(peaks, src, mx, clk):
+    """The tensor peak a GEMM is compared with, and the other one.
+
+    The measured burst figure (cuBLAS timed alone) applies when the timed
+    region ran at the maximum SM clock; the sustained one (a seconds-long loop
+    under the power cap) when the clock record shows the cap holding the clock
+    down.  MXFP8 runs at twice the bf16 rate (derived, not measured)."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    at_max = bool(clk) and clk.get("sm_mhz", 0) >= 0.97 * clk.get("sm_max_mhz", 1e9)
+    scale, tag = (2.0, "2 x ") if mx else (1.0, "")
+    note = " (derived FP8 rate)" if mx else ""
+    if at_max or not clk:
+        return (scale * burst, f"{tag}{src} bf16_tflops (burst; timed region at max SM clock){note}",
+                {"sustained": scale * sust})
+    return (scale * sust, f"{tag}{src} bf16_tflops_sustained (clock held below max){note}",
+            {"burst": scale * burst})
+
+
+def time_other_config(M, IN, name, n_steps, n_warmup, dev, stream, barrier, peaks, peak_src, seed, clk_gpu):
+    """ms per step, TFLOP/s, the GEMMs' share of the tensor peak and the clocks
+    of one more workload, timed the same way as the headline one (events off),
+    its breakdown from a second, profiled loop.  Frees its buffers on return."""
+    import torch
+    cfg = dict(IN.WORKLOADS[name])
+    host = IN.make_inputs(seed=seed, device="cpu", **cfg)
+    T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
+    x, lg, wgu, wd, gout = (host[n].to(dev) for n in ("x", "logits", "wgu", "wd", "gout"))
+    del host
+    mx = cfg.get("dtype") == "mxfp8"
+    layer = M.MoELayer(T, d, E, k, I, device=str(dev), dtype=M.MOE_MXFP8 if mx else M.MOE_BF16)
+
+    def step():
+        layer.forward(x, lg, wgu, wd, stream)
+        layer.backward(gout, x, wgu, wd, True, stream)
+
+    for _ in range(max(3, n_warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(clk_gpu)
+    if clk_gpu is not None:
+        clocks.start()
+        time.sleep(0.3)
+    ms = timed_loop(step, n_steps, stream, dev, barrier)
+    clk = clocks.stop() if clk_gpu is not None else None
+    per_kernel, _ = profiled_loop(M, step, n_steps, stream, dev, barrier)
+    status = layer.status(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status} in workload {name}")
+    flops = IN.flops_fwd(**cfg) + IN.flops_bwd(**cfg)
+    gf = gemm_flops_per_launch(T, d, k, I)
+    gemm_ms = sum(per_kernel.get(n, (0.0, 0))[0] for n in gf) / n_steps
+    peak, note, _ = tensor_peaks(peaks, peak_src, mx, clk)
+    tflops = flops / (ms * 1e-3) / 1e12
+    out = {"ms_per_step": ms, "value": tflops, "unit": UNIT, "steps": n_steps,
+           "frac_of_peak": tflops / peak,
+           "gemm_only_frac": (flops / (gemm_ms * 1e-3) / 1e12) / peak if gemm_ms else None,
+           "gemm_ms_per_step": gemm_ms, "peak": peak, "peak_source": note, "clocks": clk,
+           "config": workload_config(name, cfg), "dtype": "mxfp8 (e4m3, ue8m0/32)" if mx else "bf16",
+           "kernels": {n: v["ms_per_step"] for n, v in kernel_breakdown(per_kernel, n_steps).items()}}
+    if "zipf_s" in cfg:
+        counts = layer.saved["counts"].cpu()
+        out["routing_skew"] = {"max_count": int(counts.max()), "empty_experts": int((counts == 0).sum())}
+    del layer, x, lg, wgu, wd, gout
+    torch.cuda.empty_cache()
+    return out
+
+
+# ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
 def main():
@@ -344,50 +462,33 @@ def main():
         if pg is not None:
             pg.barrier()
 
-    # ---- device-resident timed region (per-kernel events enabled) ----
-    M.profile_read()
-    M.profile_enable(True)
+    # ---- device-resident timed region: the layer alone, no per-kernel events ----
     clocks = ClockSampler(local)
     if not args.no_clocks:
         clocks.start()
         time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize(dev)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for _ in range(args.steps):
-        step()
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
+    ms_per_step = timed_loop(step, args.steps, stream, dev, barrier)
     clk = clocks.stop()
-    M.profile_enable(False)
-    per_kernel = M.profile_read()
-    elapsed_ms = t_start.elapsed_time(t_end)
     if layer.status(stream) != 0:
         raise SystemExit("device status error in the timed region")
-    elapsed_ms = max_over_ranks(elapsed_ms, pg, dev)
-    ms_per_step = elapsed_ms / args.steps
+    ms_per_step = max_over_ranks(ms_per_step, pg, dev)
     flops_step = IN.flops_fwd(**cfg) + IN.flops_bwd(**cfg)
     value = job_tflops(flops_step, world, ms_per_step)
 
+    # ---- per-kernel breakdown: a second loop of the same steps, every launch
+    # bracketed by CUDA events on its stream ----
+    per_kernel, prof_ms = profiled_loop(M, step, args.steps, stream, dev, barrier)
+    if layer.status(stream) != 0:
+        raise SystemExit("device status error in the profiled loop")
+
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
-    P = T * k
-    gemm_flops = {"gemm_gateup_fwd": 4.0 * P * d * I, "gemm_down_fwd_combine": 2.0 * P * I * d,
-                  "gemm_down_dgrad": 2.0 * P * d * I, "gemm_down_wgrad": 2.0 * P * d * I,
-                  "gemm_gateup_dgrad_scatter": 4.0 * P * d * I, "gemm_gateup_wgrad": 4.0 * P * d * I}
-    total_kernel_ms = sum(v[0] for v in per_kernel.values()) or 1.0
+    gemm_flops = gemm_flops_per_launch(T, d, k, I)
     dom = max(gemm_flops, key=lambda n: per_kernel.get(n, (0.0, 0))[0])
     dom_ms, dom_n = per_kernel[dom]
     dom_avg_ms = dom_ms / max(dom_n, 1)
     achieved = gemm_flops[dom] / (dom_avg_ms * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    peak_note = f"{peak_src} bf16_tflops_sustained"
-    if mx:  # dense FP8 runs at twice the bf16 rate: derived from the measured bf16 figure
-        peak *= 2.0
-        peak_note = f"2 x {peak_src} bf16_tflops_sustained (derived FP8 rate)"
+    peak, peak_note, peak_alt = tensor_peaks(peaks, peak_src, mx, clk)
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if os.path.exists(tpath):
@@ -401,8 +502,9 @@ def main():
         except Exception:
             traffic = None
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "peak_source": peak_note}
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
+                "frac_other_peak": {k_: achieved / v for k_, v in peak_alt.items()},
+                "timing": "mean launch time from the per-kernel CUDA events of the profiled loop"}
     gemm_ms = sum(per_kernel.get(n, (0.0, 0))[0] for n in gemm_flops) / args.steps
     route_names = ("route_topk", "route_scan", "route_perm", "route_fused")
     route_ms = sum(per_kernel.get(n, (0.0, 0))[0] for n in route_names) / args.steps
@@ -413,9 +515,9 @@ def main():
         routing["sweep"] = routing_sweep(M, IN, dev, stream, routing["peak_gbs"], E, k)
         routing["sweep_note"] = ("moe_route alone, E and top_k of this workload, one call per timing with L2 "
                                  "flushed before it; median of 10")
-    breakdown = {n: {"ms_per_step": v[0] / args.steps, "share": v[0] / total_kernel_ms,
-                     "launches": v[1]} for n, v in per_kernel.items() if v[1]}
-    launches = int(sum(v[1] for v in per_kernel.values()))
+    breakdown = kernel_breakdown(per_kernel, args.steps)
+    launches_per_step = sum(v[1] for v in per_kernel.values()) / args.steps
+    launches = int(round(launches_per_step * args.steps))
 
     # ---- recompute mode: forward, h and aw regenerated, backward ----
     # (the layer cost under activation checkpointing: the gate/up GEMM runs
@@ -505,13 +607,28 @@ def main():
         bo = sum(t.numel() * t.element_size() for t in (hout[0], hdx[0], hds[0]))
         e2e = {"value": job_tflops(flops_step, world, e_ms / args.e2e_steps), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": args.e2e_steps,
-               "overlap": "copies of step i+1 / i-1 overlap compute of step i (two layer buffers)"}
+               "overlap": "copies of step i+1 / i-1 overlap compute of step i (two layer buffers)",
+               "note": "the step's result read back is out, dx and dscore; dW_gate_up and dW_down stay on the "
+                       "device, as in a training loop whose optimizer runs on the GPU"}
         del layers
 
     # ---- CPU baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, _, _ = cpu_baseline(cfg, host, args.cpu_tokens)
+
+    # ---- the other workloads (N = 1 only): same warm-up and steps, events off,
+    # breakdown from a profiled loop; the headline layer's buffers are freed first ----
+    others = None
+    if world == 1 and not args.no_configs:
+        del layer, x, lg, wgu, wd, gout
+        torch.cuda.empty_cache()
+        others = {}
+        for name in OTHER_WORKLOADS:
+            if name == args.workload:
+                continue
+            others[name] = time_other_config(M, IN, name, args.steps, args.warmup, dev, stream, barrier, peaks,
+                                             peak_src, args.seed, None if args.no_clocks else local)
 
     if pg is not None:
         pg.barrier()
@@ -527,6 +644,9 @@ def main():
                               if gemm_ms else None, "peak": peak, "peak_source": roofline["peak_source"]},
         "roofline": roofline, "routing": routing, "kernels": breakdown, "gpu_launches": launches,
         "clocks": clk, "e2e": e2e, "recompute": recompute, "cpu_baseline": cpu,
+        "timing": "value and ms_per_step from a loop without per-kernel events; kernels and roofline from a "
+                  f"second loop of the same steps with them ({prof_ms:.4f} ms per step there)",
+        "configs": others,
     }
     print(json.dumps(line), flush=True)
     return 0

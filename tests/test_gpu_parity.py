@@ -2,9 +2,11 @@
 
 Routing indices, counts, offsets, permutation and inverse must match bit for
 bit; out, h, aw and every gradient must match within the normwise relative
-tolerance TOL_BF16 (bf16 operands, fp32 accumulation).  Small cases are
-checked element by element in full; the full-size workloads are checked on
-sampled tokens and experts, which the oracle computes one by one.
+tolerance TOL_BF16 (bf16 operands, fp32 accumulation).  Small cases and the
+Qwen3-30B-A3B-shaped workloads (uniform and skewed routing) are checked in
+full, every token and every expert; the Qwen3-235B-A22B-shaped workload on
+sampled tokens and on experts spread over the load distribution (the busiest
+among them), which the oracle computes one by one.
 """
 import numpy as np
 import pytest
@@ -87,6 +89,19 @@ def test_deterministic_bitwise():
         assert torch.equal(r1[name], r2[name]), name
 
 
+def spread_experts(counts, n=8):
+    """The busiest expert, the least loaded non-empty one and experts at evenly
+    spaced ranks of the load in between (n in all when there are enough)."""
+    order = np.argsort(counts, kind="stable")
+    nonempty = order[counts[order] > 0]
+    pick = {int(order[-1]), int(nonempty[0])}
+    for q in np.linspace(0, len(nonempty) - 1, n):
+        if len(pick) >= n:
+            break
+        pick.add(int(nonempty[int(round(q))]))
+    return sorted(pick)
+
+
 def _sampled_check(name, seed=0, n_tokens=48, experts=None):
     cfg, inp = make(name, seed=seed)
     T, d, E, k, I = (cfg[n] for n in ("T", "d", "E", "k", "I"))
@@ -107,7 +122,8 @@ def _sampled_check(name, seed=0, n_tokens=48, experts=None):
         errs[n] = normwise(f64(res[n])[toks], bt[n])
     counts = np.bincount(idx_ref.reshape(-1), minlength=E)
     if experts is None:
-        experts = [int(np.argmin(np.abs(counts - np.median(counts)))), E - 1]
+        experts = spread_experts(counts)
+    assert int(np.argmax(counts)) in experts
     be = O.backward_experts(x, logits, wgu_np, wd_np, k, gout, experts)
     for e in experts:
         errs[f"dwgu[{e}]"] = normwise(f64(res["dwgu"][e]), be[e][0])
@@ -119,22 +135,30 @@ def _sampled_check(name, seed=0, n_tokens=48, experts=None):
     return errs
 
 
-def test_qwen3_30b_shape_sampled():
-    _sampled_check("qwen3_30b_a3b")
+@pytest.mark.slow
+def test_qwen3_30b_full_size_every_output():
+    """The 30B workload at full size: every token's out and dx, every pair's h
+    and aw, every expert's dW, all against the full fp64 oracle."""
+    cfg, inp = make("qwen3_30b_a3b", seed=0)
+    full_check(cfg, inp)
 
 
-def test_qwen3_30b_skewed_routing_sampled():
+@pytest.mark.slow
+def test_qwen3_30b_skewed_routing_full_size_every_output():
+    """The skewed 30B workload at full size, in full: the busiest expert
+    (about 16,000 pairs: the longest weight-gradient K loops) and the empty
+    ones (exact-zero weight gradients) included."""
     from grouped_gemm_route_b200 import inputs as IN
-    cfg = IN.WORKLOADS["qwen3_30b_a3b_skew"]
+    cfg = dict(IN.WORKLOADS["qwen3_30b_a3b_skew"])
     lg = IN.make_logits(cfg["T"], cfg["E"], seed=0, zipf_s=cfg["zipf_s"]).numpy()
     idx, _ = O.route(lg, cfg["k"])
     counts = np.bincount(idx.reshape(-1), minlength=cfg["E"])
-    assert (counts == 0).sum() >= 8
-    order = np.argsort(counts)
-    medium = int(order[np.searchsorted(counts[order], 2000)])  # a busy but not the busiest expert
-    _sampled_check("qwen3_30b_a3b_skew", experts=[medium, int(np.argmax(counts == 0))])
+    assert (counts == 0).sum() >= 8 and counts.max() > 10 * np.median(counts)
+    cfg, inp = make("qwen3_30b_a3b_skew", seed=0)
+    full_check(cfg, inp)
 
 
+@pytest.mark.slow
 def test_qwen3_235b_shape_sampled():
     _sampled_check("qwen3_235b_a22b", n_tokens=24)
 
