@@ -159,6 +159,22 @@ __device__ __forceinline__ int total_tiles(const GemmArgs &a) {
     }
 }
 
+// The i-th tile of CTA (or CTA pair) `first` of `count`.  The M-tiled modes,
+// whose tiles all cost the same, deal them round-robin.  The weight
+// gradients' tiles come busiest expert first (tiles of one expert cost the
+// same, and the cost falls along the list) and are dealt in snake order,
+// forwards in even rounds and backwards in odd ones, so that under skewed
+// routing every CTA's total stays close to the mean.  A CTA's tiles increase
+// with i in both orders.
+template <int MODE>
+__device__ __forceinline__ int nth_tile(int i, int first, int count) {
+    if constexpr (ModeTraits<MODE>::kMTiled) {
+        return first + i * count;
+    } else {
+        return i * count + ((i & 1) ? count - 1 - first : first);
+    }
+}
+
 // Token row of a sorted position (padding rows read token 0; their products
 // are masked or multiplied by zero rows of the other operand).
 __device__ __forceinline__ int token_of(const GemmArgs &a, int pos) {
@@ -252,7 +268,8 @@ __device__ void producer_loop(const CUtensorMap *tmA, const CUtensorMap *tmB, co
     const int total = total_tiles<MODE>(a);
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+    for (int i = 0, tile = nth_tile<MODE>(0, blockIdx.x, gridDim.x); tile < total && ok;
+         tile = nth_tile<MODE>(++i, blockIdx.x, gridDim.x)) {
         const Tile t = decode_tile<MODE>(tile, a, order);
         for (int kb = 0; kb < t.nkb; ++kb) {
             const int s = it % C::kStages;
@@ -441,7 +458,8 @@ __device__ void mma_loop(const GemmArgs &a, uint8_t *smem, uint64_t *full, uint6
     const int total = total_tiles<MODE>(a);
     int it = 0, local = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+    for (int tile = nth_tile<MODE>(0, blockIdx.x, gridDim.x); tile < total && ok;
+         tile = nth_tile<MODE>(++local, blockIdx.x, gridDim.x)) {
         const Tile t = decode_tile<MODE>(tile, a, order);
         const int acc = local & 1;
         const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
@@ -754,7 +772,8 @@ __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *temp
     const int r = quad * 32 + lane;
     const int total = total_tiles<MODE>(a);
     int local = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+    for (int tile = nth_tile<MODE>(0, blockIdx.x, gridDim.x); tile < total;
+         tile = nth_tile<MODE>(++local, blockIdx.x, gridDim.x)) {
         const Tile t = decode_tile<MODE>(tile, a, order);
         const int acc = local & 1;
         const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
@@ -1021,7 +1040,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         // ---- producer: this CTA's A rows and B half, counted on the leader's barrier ----
         int it = 0;
         bool ok = true;
-        for (int tile = pair; tile < total && ok; tile += npairs) {
+        for (int i = 0, tile = nth_tile<MODE>(0, pair, npairs); tile < total && ok;
+             tile = nth_tile<MODE>(++i, pair, npairs)) {
             const Tile t = decode_pair_tile<MODE>(tile, a, tbl, rank);
             for (int kb = 0; kb < t.nkb; ++kb, ++it) {
                 const int s = it % P::kStages;
@@ -1068,7 +1088,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
             constexpr uint32_t kIdesc = instr_desc_bf16(2 * kTileM, BN, TR::kAMn, TR::kBMn);
             int it = 0, local = 0;
             bool ok = true;
-            for (int tile = pair; tile < total && ok; tile += npairs, ++local) {
+            for (int tile = nth_tile<MODE>(0, pair, npairs); tile < total && ok;
+                 tile = nth_tile<MODE>(++local, pair, npairs)) {
                 const Tile t = decode_pair_tile<MODE>(tile, a, tbl, rank);
                 const int acc = local & 1;
                 const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
@@ -1114,7 +1135,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         const int r = quad * 32 + lane;
         uint8_t *xbuf = smem + P::kXposeOffset + (warp - kEpiWarp0) * kXposeBytes;
         int local = 0;
-        for (int tile = pair; tile < total; tile += npairs, ++local) {
+        for (int tile = nth_tile<MODE>(0, pair, npairs); tile < total;
+             tile = nth_tile<MODE>(++local, pair, npairs)) {
             const Tile t = decode_pair_tile<MODE>(tile, a, tbl, rank);
             const int acc = local & 1;
             const uint32_t aph = static_cast<uint32_t>(local >> 1) & 1u;
