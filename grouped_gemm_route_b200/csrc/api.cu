@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <cmath>
+#include <functional>
 #include <mutex>
 #include <vector>
 
@@ -89,9 +90,9 @@ int make_plan(const moe_shape_t *s, Plan *p) {
     p->ws_stage = off;  // combine staging [P, d]; before it, the bf16 forward's sorted x [p_cap, d]
     off = align_up(off + static_cast<size_t>(p_cap) * s->d * 2);
     const size_t common = off;
-    p->ws_chunk_counts = off;
+    p->ws_chunk_counts = off;  // routing: per-block expert histograms
     off = align_up(off + static_cast<size_t>(p->n_chunks) * s->E * 4);
-    p->ws_chunk_base = off;
+    p->ws_chunk_base = off;    // and their per-expert exclusive scans over the blocks
     off = align_up(off + static_cast<size_t>(p->n_chunks) * s->E * 4);
     auto take = [&off](size_t bytes) {
         const size_t at = off;
@@ -223,6 +224,41 @@ bool make_map8(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uin
 }
 
 // ---------------------------------------------------------------------------
+// one extra stream per device, for bandwidth-bound work that runs beside a
+// tensor-bound GEMM (with two events to fork from and join the caller's stream)
+// ---------------------------------------------------------------------------
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    bool tried = false;
+    std::mutex mu;  // an event's record and the wait on it stay together when host threads share the stream
+
+    // `to` waits for everything issued so far on `from` (through event ev).
+    bool link(cudaEvent_t ev, cudaStream_t from, cudaStream_t to) {
+        std::lock_guard<std::mutex> lock(mu);
+        return cudaEventRecord(ev, from) == cudaSuccess && cudaStreamWaitEvent(to, ev, 0) == cudaSuccess;
+    }
+};
+SideStream g_side[64];
+
+// The current device's side stream, created on first use; nullptr if it could
+// not be created (the caller then runs everything on its own stream).
+SideStream *side_stream() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    SideStream &ss = g_side[dev];
+    if (!ss.tried) {
+        ss.tried = true;
+        if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+            ss.s = nullptr;
+    }
+    return ss.s != nullptr && ss.fork != nullptr && ss.join != nullptr ? &ss : nullptr;
+}
+
+// ---------------------------------------------------------------------------
 // per-kernel timing (host bookkeeping only)
 // ---------------------------------------------------------------------------
 struct Timing {
@@ -272,7 +308,7 @@ struct Launch {
 const char *kKindNames[kNumKernelKinds] = {
     "route_topk",       "route_scan",       "route_perm",           "gemm_gateup_fwd",      "gemm_down_fwd_combine",
     "gemm_down_dgrad",  "gemm_down_wgrad",  "gemm_gateup_dgrad_scatter", "gemm_gateup_wgrad", "route_bwd",
-    "sort_rows", "mx_quant", "route_fused", "sort_x", "combine"};
+    "sort_rows", "mx_quant", "route_fused", "sort_x", "combine", "ep_layout", "ep_rows"};
 
 struct Saved {
     int32_t *idx;
@@ -426,6 +462,20 @@ int sort_x(const Plan &pl, const DeviceInfo &dev, const void *x, const moe_saved
                                    saved->xs != nullptr, dev.sms, st));
 }
 
+// The bf16 gate/up GEMM on CTA pairs over x already in the sorted layout.
+int gateup_pair_sorted(const Plan &pl, const moe_shape_t *shape, const DeviceInfo &dev, const void *xs,
+                       const void *w_gate_up, moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
+    CUtensorMap tm_wgu, tm_xs;  // the pair kernel loads W_gate_up in 64-row boxes (gate and up halves)
+    if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 64) ||
+        !make_map(&tm_xs, xs, pl.p_cap, pl.d, 128))
+        return MOE_ERR_LAUNCH;
+    GemmArgs a = base_args(pl, saved, w8);
+    a.n_tiles = pl.I / 128;
+    a.num_k_blocks = pl.d / kTileK;
+    Launch L(kKindGemmGateUpFwd, st);
+    return L.done(launch_gemm_pair(kGateUpFwd, a, tm_xs, tm_wgu, grid_for(shape, dev), st));
+}
+
 int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,
                moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
     int rc;
@@ -435,20 +485,31 @@ int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, 
     if (pair || saved->xs != nullptr)
         if ((rc = sort_x(pl, dev, x, saved, w8, st, &xs))) return rc;
     if (pl.mx) return gateup_mx(pl, dev, shape, x, w_gate_up, saved, w8, st);
+    if (pair) return gateup_pair_sorted(pl, shape, dev, xs, w_gate_up, saved, w8, st);  // plain TMA tiles
     CUtensorMap tm_wgu;
     if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 128)) return MOE_ERR_LAUNCH;
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.I / 128;
     a.num_k_blocks = pl.d / kTileK;
-    if (pair) {  // plain TMA tiles of the sorted x on CTA pairs
-        CUtensorMap tm_xs;
-        if (!make_map(&tm_xs, xs, pl.p_cap, pl.d, 128)) return MOE_ERR_LAUNCH;
-        Launch L(kKindGemmGateUpFwd, st);
-        return L.done(launch_gemm_pair(kGateUpFwd, a, tm_xs, tm_wgu, grid, st));
-    }
     a.gsrc = static_cast<const __nv_bfloat16 *>(x);  // token rows gathered through perm (A operand)
     Launch L(kKindGemmGateUpFwd, st);
     return L.done(launch_gemm(kGateUpFwd, 256, false, a, tm_wgu, tm_wgu, grid, st));
+}
+
+// The bf16 down GEMM; its epilogue writes each valid sorted row's product to
+// row perm[pos] of `stage` (NULL: the workspace's staging buffer).
+int down_fwd_staged(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *w_down,
+                    const moe_saved_t *saved, uint8_t *w8, void *stage, cudaStream_t st) {
+    CUtensorMap tm_aw, tm_wd;
+    if (!make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) ||
+        !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
+        return MOE_ERR_LAUNCH;
+    GemmArgs a = base_args(pl, saved, w8);
+    if (stage != nullptr) a.stage = static_cast<__nv_bfloat16 *>(stage);
+    a.n_tiles = pl.d / pl.bn_d;
+    a.num_k_blocks = pl.I / kTileK;
+    Launch L(kKindGemmDownFwd, st);
+    return L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid_for(shape, dev), st));
 }
 
 // MXFP8 backward after sort_rows: every GEMM operand quantised along that
@@ -530,6 +591,64 @@ int bwd_mx(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, cons
     return L.done(launch_gemm(kGateUpWgrad, 128, true, a, tm_dhc8, tm_xsc8, grid, st));
 }
 
+// The four bf16 backward GEMMs on sorted grad_out (gs) and sorted x (xs), both
+// with zero padding rows: b1 down dgrad (dscore partials, SwiGLU backward ->
+// dh), b3 down wgrad, b4 gate/up dgrad (each valid sorted row's dx product to
+// row perm[pos] of `stage`; NULL: the workspace's staging buffer), b5 gate/up
+// wgrad.  `a` carries the routing state, dh and the dscore partials.
+int bwd_gemms(const Plan &pl, const DeviceInfo &dev, int grid, GemmArgs a, const void *gs, const void *xs,
+              const void *w_gate_up, const void *w_down, const moe_saved_t *saved, void *dw_gate_up, void *dw_down,
+              void *stage, cudaStream_t st, const std::function<int()> &after_dgrad = nullptr) {
+    (void)dev;
+    int rc;
+    CUtensorMap tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn, tm_gs_rows, tm_gs_mn, tm_xs_mn;
+    const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I;
+    const int64_t Ed = static_cast<int64_t>(pl.E) * pl.d;
+    if (!make_map(&tm_wd_mn, w_down, Ed, pl.I, 64) || !make_map(&tm_dh_rows, a.dh, pl.p_cap, 2 * pl.I, 128) ||
+        !make_map(&tm_wgu_mn, w_gate_up, EI2, pl.d, 64) || !make_map(&tm_aw_mn, saved->aw, pl.p_cap, pl.I, 64) ||
+        !make_map(&tm_dh_mn, a.dh, pl.p_cap, 2 * pl.I, 64) || !make_map(&tm_gs_rows, gs, pl.p_cap, pl.d, 128) ||
+        !make_map(&tm_gs_mn, gs, pl.p_cap, pl.d, 64) || !make_map(&tm_xs_mn, xs, pl.p_cap, pl.d, 64))
+        return MOE_ERR_LAUNCH;
+    if (stage != nullptr) a.stage = static_cast<__nv_bfloat16 *>(stage);
+    // b1: down dgrad, dscore partials, SwiGLU backward -> dh
+    a.n_tiles = pl.I / pl.bn_i;
+    a.num_k_blocks = pl.d / kTileK;
+    {
+        Launch L(kKindGemmDownDgrad, st);
+        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, false, a, tm_gs_rows, tm_wd_mn, grid, st)))) return rc;
+    }
+    // b3: down wgrad  dW_down[e] = sum_p gout[t] (x) aw_p
+    a.m_tiles = pl.d / kTileM;
+    a.n_tiles = pl.I / pl.bn_i;
+    a.dw = static_cast<__nv_bfloat16 *>(dw_down);
+    {
+        Launch L(kKindGemmDownWgrad, st);
+        if ((rc = L.done(gemm_pair_ok(kDownWgrad, pl.bn_i, false, a.m_tiles, grid)
+                             ? launch_gemm_pair(kDownWgrad, a, tm_gs_mn, tm_aw_mn, grid, st)
+                             : launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st))))
+            return rc;
+    }
+    // b4: gate/up dgrad, rows staged for the ordered scatter-sum into dx
+    a.n_tiles = pl.d / pl.bn_d;
+    a.num_k_blocks = 2 * pl.I / kTileK;
+    {
+        Launch L(kKindGemmGateUpDgrad, st);
+        if ((rc = L.done(gemm_pair_ok(kGateUpDgrad, pl.bn_d, false, 0, grid)
+                             ? launch_gemm_pair(kGateUpDgrad, a, tm_dh_rows, tm_wgu_mn, grid, st)
+                             : launch_gemm(kGateUpDgrad, pl.bn_d, false, a, tm_dh_rows, tm_wgu_mn, grid, st))))
+            return rc;
+    }
+    if (after_dgrad && (rc = after_dgrad())) return rc;  // work that may run beside the gate/up wgrad
+    // b5: gate/up wgrad  dW_gu[e] = sum_p dh_p (x) x[t]
+    a.m_tiles = 2 * pl.I / kTileM;
+    a.n_tiles = pl.d / pl.bn_d;
+    a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
+    Launch L(kKindGemmGateUpWgrad, st);
+    return L.done(gemm_pair_ok(kGateUpWgrad, pl.bn_d, false, a.m_tiles, grid)
+                      ? launch_gemm_pair(kGateUpWgrad, a, tm_dh_mn, tm_xs_mn, grid, st)
+                      : launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -587,18 +706,7 @@ int moe_fwd(const moe_shape_t *shape, const void *x, const float *logits, const 
     if ((rc = run_route(shape, pl, dev, logits, saved, w8, st))) return rc;
     if ((rc = gateup_fwd(pl, dev, shape, x, w_gate_up, saved, w8, st))) return rc;
     if (pl.mx) return down_mx(pl, dev, shape, w_down, out, saved, w8, st);
-    CUtensorMap tm_aw, tm_wd;
-    if (!make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) ||
-        !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
-        return MOE_ERR_LAUNCH;
-    GemmArgs a = base_args(pl, saved, w8);
-    a.n_tiles = pl.d / pl.bn_d;
-    a.num_k_blocks = pl.I / kTileK;
-    {
-        Launch L(kKindGemmDownFwd, st);
-        const int rc = L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid_for(shape, dev), st));
-        if (rc) return rc;
-    }
+    if ((rc = down_fwd_staged(pl, dev, shape, w_down, saved, w8, nullptr, st))) return rc;
     return run_combine(pl, dev, w8, out, st);
 }
 
@@ -642,15 +750,6 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
     __nv_bfloat16 *xs = have_xs ? static_cast<__nv_bfloat16 *>(saved->xs)
                                 : reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_xs);
     __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_gs);
-    CUtensorMap tm_wd_mn, tm_dh_rows, tm_wgu_mn, tm_aw_mn, tm_dh_mn, tm_gs_rows, tm_gs_mn, tm_xs_mn;
-    const int64_t EI2 = static_cast<int64_t>(pl.E) * 2 * pl.I;
-    const int64_t Ed = static_cast<int64_t>(pl.E) * pl.d;
-    if (!make_map(&tm_wd_mn, w_down, Ed, pl.I, 64) || !make_map(&tm_dh_rows, dh, pl.p_cap, 2 * pl.I, 128) ||
-        !make_map(&tm_wgu_mn, w_gate_up, EI2, pl.d, 64) || !make_map(&tm_aw_mn, saved->aw, pl.p_cap, pl.I, 64) ||
-        !make_map(&tm_dh_mn, dh, pl.p_cap, 2 * pl.I, 64) || !make_map(&tm_gs_rows, gs, pl.p_cap, pl.d, 128) ||
-        !make_map(&tm_gs_mn, gs, pl.p_cap, pl.d, 64) || !make_map(&tm_xs_mn, xs, pl.p_cap, pl.d, 64))
-        return MOE_ERR_LAUNCH;
-
     if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
     const int grid = grid_for(shape, dev);
     GemmArgs a = base_args(pl, const_cast<moe_saved_t *>(saved), w8);
@@ -677,46 +776,22 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
         return L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_w, saved->topk_idx,
                                        saved->inv, dpart, pl.dpart_stride, dscore, dlogits, st));
     }
-    // b1: down dgrad, dscore partials, SwiGLU backward -> dh
-    a.n_tiles = pl.I / pl.bn_i;
-    a.num_k_blocks = pl.d / kTileK;
-    {
-        Launch L(kKindGemmDownDgrad, st);
-        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, false, a, tm_gs_rows, tm_wd_mn, grid, st)))) return rc;
-    }
-    // b3: down wgrad  dW_down[e] = sum_p gout[t] (x) aw_p
-    a.m_tiles = pl.d / kTileM;
-    a.n_tiles = pl.I / pl.bn_i;
-    a.dw = static_cast<__nv_bfloat16 *>(dw_down);
-    {
-        Launch L(kKindGemmDownWgrad, st);
-        if ((rc = L.done(gemm_pair_ok(kDownWgrad, pl.bn_i, false, a.m_tiles, grid)
-                             ? launch_gemm_pair(kDownWgrad, a, tm_gs_mn, tm_aw_mn, grid, st)
-                             : launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st))))
-            return rc;
-    }
-    // b4: gate/up dgrad + ordered scatter-sum into dx
-    a.n_tiles = pl.d / pl.bn_d;
-    a.num_k_blocks = 2 * pl.I / kTileK;
-    {
-        Launch L(kKindGemmGateUpDgrad, st);
-        if ((rc = L.done(gemm_pair_ok(kGateUpDgrad, pl.bn_d, false, 0, grid)
-                             ? launch_gemm_pair(kGateUpDgrad, a, tm_dh_rows, tm_wgu_mn, grid, st)
-                             : launch_gemm(kGateUpDgrad, pl.bn_d, false, a, tm_dh_rows, tm_wgu_mn, grid, st))))
-            return rc;
-    }
-    if ((rc = run_combine(pl, dev, w8, dx, st))) return rc;
-    // b5: gate/up wgrad  dW_gu[e] = sum_p dh_p (x) x[t]
-    a.m_tiles = 2 * pl.I / kTileM;
-    a.n_tiles = pl.d / pl.bn_d;
-    a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
-    {
-        Launch L(kKindGemmGateUpWgrad, st);
-        if ((rc = L.done(gemm_pair_ok(kGateUpWgrad, pl.bn_d, false, a.m_tiles, grid)
-                             ? launch_gemm_pair(kGateUpWgrad, a, tm_dh_mn, tm_xs_mn, grid, st)
-                             : launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st))))
-            return rc;
-    }
+    // The scatter-sum into dx (bandwidth bound) needs only the gate/up dgrad's
+    // staged rows: it runs on a second stream beside the gate/up wgrad (tensor
+    // bound; its persistent CTAs leave threads and registers free on every SM),
+    // joined back before the call's last kernel.
+    SideStream *side = side_stream();
+    bool forked = false;
+    auto fork_combine = [&]() -> int {
+        if (side != nullptr && side->link(side->fork, st, side->s)) {
+            forked = true;
+            return run_combine(pl, dev, w8, dx, side->s);
+        }
+        return run_combine(pl, dev, w8, dx, st);
+    };
+    rc = bwd_gemms(pl, dev, grid, a, gs, xs, w_gate_up, w_down, saved, dw_gate_up, dw_down, nullptr, st, fork_combine);
+    if (forked && !side->link(side->join, side->s, st)) return MOE_ERR_LAUNCH;
+    if (rc) return rc;
     // b6: dscore (ordered sum of partials) and dlogits
     {
         Launch L(kKindRouteBwd, st);
@@ -724,6 +799,170 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
                                      dpart, pl.dpart_stride, dscore, dlogits, st));
     }
     return rc;
+}
+
+// ---------------------------------------------------------------------------
+// expert parallelism (see include/moe.h and ep.cu)
+// ---------------------------------------------------------------------------
+int moe_ep_expert_layout(int G, int E_loc, const int32_t *recv_counts, int64_t *row_off, int64_t *cmp_off,
+                         int64_t *rows, int64_t *padded_rows) {
+    if (G < 1 || E_loc < 1 || E_loc > kMaxExperts || !recv_counts || !row_off || !cmp_off || !rows || !padded_rows)
+        return MOE_ERR_ARG;
+    int64_t cmp = 0, pad = 0;
+    for (int e = 0; e < E_loc; ++e) {
+        int64_t n_e = 0;
+        for (int s = 0; s < G; ++s) {
+            const int32_t c = recv_counts[static_cast<int64_t>(s) * E_loc + e];
+            if (c < 0) return MOE_ERR_ARG;
+            row_off[static_cast<int64_t>(s) * E_loc + e] = pad + n_e;
+            cmp_off[static_cast<int64_t>(s) * E_loc + e] = cmp + n_e;
+            n_e += c;
+        }
+        cmp += n_e;
+        pad += (n_e + kTileM - 1) / kTileM * kTileM;
+    }
+    *rows = cmp;
+    *padded_rows = pad;
+    return MOE_OK;
+}
+
+int moe_ep_dispatch(const moe_shape_t *shape, const void *src, const moe_saved_t *saved, void *dst, float *w_rows,
+                    void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(src) || !aligned16(dst) || (w_rows && !aligned16(w_rows))) return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    {
+        Launch L(kKindSortX, st);
+        if ((rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, pl.k,
+                                          static_cast<int>(pl.T), pl.d, static_cast<const __nv_bfloat16 *>(src),
+                                          nullptr, static_cast<__nv_bfloat16 *>(dst), nullptr, false, dev.sms, st))))
+            return rc;
+    }
+    if (w_rows == nullptr) return MOE_OK;
+    Launch L(kKindEpRows, st);
+    return L.done(launch_ep_row_weights(saved->perm, saved->tile_expert, saved->counts, saved->offsets,
+                                        saved->group_start, saved->topk_w, pl.E, pl.P, pl.p_cap, w_rows, dev.sms, st));
+}
+
+// Shape rules of the expert side: T = the rows received, k = 1, E = local experts, bf16 on CTA pairs.
+static int expert_side_checks(const moe_shape_t *shape, const Plan &pl, const DeviceInfo &dev) {
+    if (shape->k != 1 || shape->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!gemm_pair_ok(kGateUpFwd, 256, false, 0, grid_for(shape, dev))) return MOE_ERR_UNSUPPORTED;
+    (void)pl;
+    return MOE_OK;
+}
+
+int moe_expert_fwd(const moe_shape_t *shape, int G, const int32_t *recv_counts, void *xr, const void *w_gate_up,
+                   const void *w_down, void *y_rows, moe_saved_t *saved, void *ws, size_t ws_bytes, void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (G < 1 || !aligned16(recv_counts) || !aligned16(xr) || !aligned16(w_gate_up) || !aligned16(w_down) ||
+        !aligned16(y_rows) || !aligned16(ws))
+        return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    if (ws_bytes < pl.fwd_bytes) return MOE_ERR_WS;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    if ((rc = expert_side_checks(shape, pl, dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 16, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    {
+        Launch L(kKindEpLayout, st);
+        if ((rc = L.done(launch_ep_layout(G, pl.E, recv_counts, pl.p_cap, saved->counts, saved->offsets,
+                                          saved->group_start, saved->tile_expert, saved->perm, saved->inv,
+                                          reinterpret_cast<int *>(w8 + pl.ws_status), st))))
+            return rc;
+    }
+    {  // the received rows' padding rows to zero (no rows are copied: T = 0)
+        Launch L(kKindSortRows, st);
+        if ((rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, 1, 0, pl.d, nullptr,
+                                          nullptr, static_cast<__nv_bfloat16 *>(xr), nullptr, true, dev.sms, st))))
+            return rc;
+    }
+    if ((rc = gateup_pair_sorted(pl, shape, dev, xr, w_gate_up, saved, w8, st))) return rc;
+    return down_fwd_staged(pl, dev, shape, w_down, saved, w8, y_rows, st);
+}
+
+int moe_expert_bwd(const moe_shape_t *shape, void *gr, const void *xr, const void *w_gate_up, const void *w_down,
+                   const moe_saved_t *saved, void *dx_rows, void *dw_gate_up, void *dw_down, float *ds_rows,
+                   void *ws, size_t ws_bytes, void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(gr) || !aligned16(xr) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(dx_rows) ||
+        !aligned16(dw_gate_up) || !aligned16(dw_down) || !aligned16(ds_rows) || !aligned16(ws))
+        return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    if (ws_bytes < pl.bwd_bytes) return MOE_ERR_WS;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    if ((rc = expert_side_checks(shape, pl, dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    float *dpart = reinterpret_cast<float *>(w8 + pl.ws_dpart);
+    if (cudaMemsetAsync(w8 + pl.ws_status, 0, 4, st) != cudaSuccess) return MOE_ERR_LAUNCH;
+    {  // the received grad_out rows' padding rows to zero
+        Launch L(kKindSortRows, st);
+        if ((rc = L.done(launch_sort_rows(saved->inv, saved->counts, saved->group_start, pl.E, 1, 0, pl.d, nullptr,
+                                          nullptr, static_cast<__nv_bfloat16 *>(gr), nullptr, true, dev.sms, st))))
+            return rc;
+    }
+    GemmArgs a = base_args(pl, const_cast<moe_saved_t *>(saved), w8);
+    a.dh = reinterpret_cast<__nv_bfloat16 *>(w8 + pl.ws_dh);
+    a.dpart = dpart;
+    if ((rc = bwd_gemms(pl, dev, grid_for(shape, dev), a, gr, xr, w_gate_up, w_down, saved, dw_gate_up, dw_down,
+                        dx_rows, st)))
+        return rc;
+    // dscore of every received row (compact order): the ordered sum of its partials
+    Launch L(kKindRouteBwd, st);
+    return L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, 1, saved->topk_w, saved->topk_idx, saved->inv, dpart,
+                                   pl.dpart_stride, ds_rows, nullptr, st));
+}
+
+int moe_ep_combine(const moe_shape_t *shape, const moe_saved_t *saved, const void *rows, void *out, void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(rows) || !aligned16(out)) return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Launch L(kKindCombine, st);
+    return L.done(launch_ep_combine(static_cast<const __nv_bfloat16 *>(rows), saved->topk_idx, saved->inv,
+                                    saved->offsets, saved->group_start, static_cast<int>(pl.T), pl.E, pl.k, pl.d, pl.P,
+                                    static_cast<__nv_bfloat16 *>(out), nullptr, dev.sms, st));
+}
+
+int moe_ep_backward_finish(const moe_shape_t *shape, const moe_saved_t *saved, const void *dx_rows,
+                           const float *ds_rows, void *dx, float *dscore, float *dlogits, void *stream) {
+    Plan pl;
+    int rc = make_plan(shape, &pl);
+    if (rc) return rc;
+    if (!aligned16(dx_rows) || !aligned16(ds_rows) || !aligned16(dx) || !aligned16(dscore) ||
+        (dlogits && !aligned16(dlogits)))
+        return MOE_ERR_ARG;
+    if ((rc = check_saved(saved))) return rc;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    {
+        Launch L(kKindCombine, st);
+        if ((rc = L.done(launch_ep_combine(static_cast<const __nv_bfloat16 *>(dx_rows), saved->topk_idx, saved->inv,
+                                           saved->offsets, saved->group_start, static_cast<int>(pl.T), pl.E, pl.k,
+                                           pl.d, pl.P, static_cast<__nv_bfloat16 *>(dx), nullptr, dev.sms, st))))
+            return rc;
+    }
+    Launch L(kKindRouteBwd, st);
+    return L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_w, saved->topk_idx, saved->inv,
+                                   ds_rows, 1, dscore, dlogits, st, saved->group_start, saved->offsets));
 }
 
 int moe_get_status(const void *ws, void *stream, int *device_status) {

@@ -117,7 +117,10 @@ struct Tile {
     int nt;     // N tile
     int nkb;    // K blocks
     int kpos0;  // wgrad: first sorted row of the expert's group
-    bool skip;  // CTA pairs: this CTA's M tile lies past its expert's group (computed, not stored)
+    bool skip;  // CTA-pair gate/up dgrad: this CTA's M tile lies past its expert's group (computed, not stored)
+    bool half;  // CTA-pair gate/up forward: an expert's last, unpaired 128-row tile, computed by
+                // one M = 128 pair MMA (64 rows per CTA)
+    int row0;   // CTA pairs, M-tiled: first sorted row of this CTA's A rows
 };
 
 // Wgrad tiles are walked expert by expert, busiest expert first (`order`, a
@@ -126,6 +129,8 @@ template <int MODE>
 __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const int *order) {
     Tile t;
     t.skip = false;
+    t.half = false;
+    t.row0 = 0;
     if constexpr (ModeTraits<MODE>::kMTiled) {
         t.mt = tile / a.n_tiles;
         t.nt = tile - t.mt * a.n_tiles;
@@ -763,6 +768,60 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
     for (int c = 0; c < BH / 32; ++c) warp_store_rows(xbuf, zero, row + c * 32);
 }
 
+// Gate/up forward on CTA pairs (BN = 256): a tile covers gate/up columns
+// nt*128 .. +128, laid out in the accumulator as [gate 0..63 | up 0..63 |
+// gate 64..127 | up 64..127] (see the producer).  Output chunk c (32 gate
+// columns and the matching up columns) sits at TMEM column (c >> 1) * 128 +
+// (c & 1) * 32 (gate) and 64 further (up).  A full tile's thread owns row
+// quad * 32 + lane and all four chunks.  A half tile (M = 128 pair MMA) holds
+// this CTA's 64 rows in lanes 0..63 with columns [0, 128) of the tile and in
+// lanes 64..127 with columns [128, 256), both at TMEM columns [0, 128): the
+// thread owns row (quad & 1) * 32 + lane of its 64 and chunks 2h, 2h + 1 with
+// h = quad >> 1.  Same SwiGLU arithmetic as the one-CTA kernel.
+__device__ __forceinline__ void epi_gateup_fwd_pair(const GemmArgs &a, const Tile &t, int quad, int lane,
+                                                    uint32_t taddr, uint64_t *tempty_acc, uint8_t *xbuf) {
+    const int r = t.half ? (quad & 1) * 32 + lane : quad * 32 + lane;
+    const int pos = t.row0 + r;
+    const int p = __ldg(a.perm + pos);
+    const bool valid = p >= 0 && p < a.T * a.k;
+    const float wv = valid ? __ldg(a.topk_w + p) : 0.f;
+    __nv_bfloat16 *hrow = a.h + static_cast<size_t>(pos) * 2 * a.I + t.nt * 128;
+    __nv_bfloat16 *arow = a.aw + static_cast<size_t>(pos) * a.I + t.nt * 128;
+    const int c_first = t.half ? 2 * (quad >> 1) : 0;
+    const int n_chunks = t.half ? 2 : 4;
+    auto gate_col = [&](int c) -> uint32_t {
+        return static_cast<uint32_t>(t.half ? (c & 1) * 32 : (c >> 1) * 128 + (c & 1) * 32);
+    };
+    uint32_t ga[32], ua[32], gb[32], ub[32];
+    tmem_load32(taddr + gate_col(c_first), ga);
+    tmem_load32(taddr + gate_col(c_first) + 64, ua);
+    tmem_load_wait();
+    tmem_regs_ready(ga);
+    tmem_regs_ready(ua);
+#pragma unroll 1
+    for (int i = 0; i < n_chunks; i += 2) {
+        const int c = c_first + i;
+        tmem_load32(taddr + gate_col(c + 1), gb);
+        tmem_load32(taddr + gate_col(c + 1) + 64, ub);
+        gateup_chunk<256, false>(a, t, r, pos, valid, wv, c, ga, ua, hrow, arow, xbuf);
+        tmem_load_wait();
+        tmem_regs_ready(gb);
+        tmem_regs_ready(ub);
+        if (i + 2 < n_chunks) {
+            tmem_load32(taddr + gate_col(c + 2), ga);
+            tmem_load32(taddr + gate_col(c + 2) + 64, ua);
+        } else {
+            release_acc<true>(tempty_acc);  // TMEM no longer needed
+        }
+        gateup_chunk<256, false>(a, t, r, pos, valid, wv, c + 1, gb, ub, hrow, arow, xbuf);
+        if (i + 2 < n_chunks) {
+            tmem_load_wait();
+            tmem_regs_ready(ga);
+            tmem_regs_ready(ua);
+        }
+    }
+}
+
 template <int MODE, int BN, bool MX>
 __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *tempty, uint32_t tmem_base,
                               const int *order, uint8_t *xbuf, volatile int *abort_flag) {
@@ -881,11 +940,13 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
 // 128 rows exactly as in the one-CTA kernel (same functions, same outputs).
 //
 // M-tiled modes pair two consecutive 128-row tiles of one expert (both use the
-// expert's B).  An expert with an odd number of tiles has a last pair whose
-// second tile lies past its group: the peer loads those rows (or zeros past
-// the end of the sorted buffer), the MMA computes them, and the peer's
-// epilogue only releases the accumulator.  Pair rows are numbered expert by
-// expert from a per-CTA table of their starts.
+// expert's B).  An expert with an odd number of tiles ends with a half pair
+// row.  In the gate/up forward it is the last tile alone, computed by M = 128
+// pair MMAs: each CTA holds 64 of its rows, and the MMA runs at the same rate
+// per row as the M = 256 form.  In the gate/up dgrad the peer loads the rows
+// past the group (or zeros past the end of the sorted buffer), the MMA computes
+// them and the peer's epilogue only releases the accumulator.  Pair rows are
+// numbered expert by expert from a per-CTA table of their starts.
 //
 // No load is multicast.  Every wait is bounded, and both CTAs always reach the
 // final cluster barrier (no early exit), after which the pair frees its tensor
@@ -916,6 +977,8 @@ template <int MODE>
 __device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, const int *tbl, uint32_t rank) {
     Tile t;
     t.skip = false;
+    t.half = false;
+    t.row0 = 0;
     if constexpr (ModeTraits<MODE>::kMTiled) {
         const int pr = tile / a.n_tiles;
         t.nt = tile - pr * a.n_tiles;
@@ -929,8 +992,18 @@ __device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, co
         }
         t.e = lo;
         const int g0 = __ldg(a.group_start + lo) / kTileM, g1 = __ldg(a.group_start + lo + 1) / kTileM;
-        t.mt = g0 + 2 * (pr - tbl[lo]) + static_cast<int>(rank);
-        t.skip = t.mt >= g1;
+        const int t0 = g0 + 2 * (pr - tbl[lo]);  // the pair row's first tile (t0 < g1)
+        if constexpr (MODE == kGateUpFwd) {
+            t.half = t0 + 1 >= g1;  // the expert's last tile has no partner: M = 128 pair MMA
+            t.mt = t.half ? t0 : t0 + static_cast<int>(rank);
+            t.row0 = t.half ? t0 * kTileM + 64 * static_cast<int>(rank) : t.mt * kTileM;
+        } else {
+            // the gate/up dgrad computes the unpaired tile's partner rows and discards them (a
+            // half-row MMA measured 1.5 % slower here: its operand loads bound the pair row)
+            t.mt = t0 + static_cast<int>(rank);
+            t.skip = t.mt >= g1;
+            t.row0 = t.mt * kTileM;
+        }
         t.nkb = a.num_k_blocks;
         t.kpos0 = 0;
     } else {
@@ -1058,17 +1131,20 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 const int k0 = kb * kTileK;
                 const int bcol = t.nt * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B columns
                 if constexpr (MODE == kGateUpFwd) {
-                    // A: 128 sorted rows of x; B: the leader loads the tile's 128 gate rows of
-                    // W_gate_up[e], the peer its 128 up rows (both K-major), so that accumulator
-                    // columns [0, 128) hold gate and [128, 256) up, as in the one-CTA kernel
-                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.mt * kTileM);
-                    if (lane == 1)
-                        tma_load_2d_pair(Bs, &tmB, fb, k0,
-                                         t.e * 2 * a.I + static_cast<int>(rank) * a.I + t.nt * (BN / 2));
+                    // A: 128 sorted rows of x from row0 (a half tile's MMA reads the first 64);
+                    // B: the tile covers gate/up columns nt*128 .. +128; the leader loads 64 gate
+                    // rows and the 64 matching up rows for the first 64 of them, the peer for the
+                    // other 64 (64-row boxes, K-major), so that accumulator columns hold, per
+                    // 64-column group, gate then up of the same expert columns -- in a half tile
+                    // each TMEM lane half then holds whole (gate, up) pairs
+                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.row0);
+                    const int grow = t.e * 2 * a.I + t.nt * (BN / 2) + 64 * static_cast<int>(rank);
+                    if (lane == 1) tma_load_2d_pair(Bs, &tmB, fb, k0, grow);
+                    if (lane == 2) tma_load_2d_pair(Bs + 64 * 128, &tmB, fb, k0, grow + a.I);
                 } else if constexpr (TR::kMTiled) {
-                    // A: 128 sorted rows of dh, K-major; B: this CTA's half of W_gate_up[e], MN-major
+                    // A: 128 sorted rows of dh from row0, K-major; B: this CTA's half of W_gate_up[e], MN-major
                     const int brow = t.e * 2 * a.I + k0;
-                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.mt * kTileM);
+                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.row0);
                     if (lane >= 1 && lane < 1 + BN / 128)
                         tma_load_2d_pair(Bs + (lane - 1) * kChunkBytes, &tmB, fb, bcol + 64 * (lane - 1), brow);
                 } else {
@@ -1086,6 +1162,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         // ---- MMA (leader, one thread): M = 256 over the pair ----
         if (leader && lane == 0) {
             constexpr uint32_t kIdesc = instr_desc_bf16(2 * kTileM, BN, TR::kAMn, TR::kBMn);
+            constexpr uint32_t kIdescHalf = instr_desc_bf16(kTileM, BN, TR::kAMn, TR::kBMn);  // 64 rows per CTA
             int it = 0, local = 0;
             bool ok = true;
             for (int tile = nth_tile<MODE>(0, pair, npairs); tile < total && ok;
@@ -1115,7 +1192,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                                                      : smem_desc_sw128(a_base + kk * 32, 16, kSbo);
                         const uint64_t bd = TR::kBMn ? smem_desc_sw128(b_base + kk * 2048, kMnLbo, kSbo)
                                                      : smem_desc_sw128(b_base + kk * 32, 16, kSbo);
-                        mma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        mma_bf16_pair(d_tmem, ad, bd, t.half ? kIdescHalf : kIdesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[s], 0x3);  // frees the stage in both CTAs
                 }
@@ -1147,12 +1224,13 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
             tc_fence_after_sync();
             const uint32_t taddr =
                 tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-            if (t.skip) {
-                release_acc<true>(&tempty[acc]);
-            } else if constexpr (MODE == kGateUpFwd) {
-                epi_gateup_fwd<BN, false, true>(a, t, r, taddr, &tempty[acc], xbuf);
+            if constexpr (MODE == kGateUpFwd) {
+                epi_gateup_fwd_pair(a, t, quad, lane, taddr, &tempty[acc], xbuf);
             } else if constexpr (TR::kStage) {
-                epi_stage<BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
+                if (t.skip)
+                    release_acc<true>(&tempty[acc]);
+                else
+                    epi_stage<BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
             } else {
                 epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
             }

@@ -37,6 +37,8 @@ enum KernelKind : int {
     kKindRouteFused,
     kKindSortX,
     kKindCombine,
+    kKindEpLayout,
+    kKindEpRows,
     kNumKernelKinds
 };
 
@@ -104,8 +106,25 @@ cudaError_t launch_combine_rows(const __nv_bfloat16 *stage, int T, int k, int d,
 cudaError_t launch_sort_rows(const int32_t *inv, const int32_t *counts, const int32_t *group_start, int E, int k,
                              int T, int d, const __nv_bfloat16 *x, const __nv_bfloat16 *g, __nv_bfloat16 *xs,
                              __nv_bfloat16 *gs, bool zero_pad, int sms, cudaStream_t s);
+// dscore (ordered sums of the partials at each pair's row) and dlogits; with
+// compact_gs / compact_off the row of pair (t, j) is its compact sorted index
+// (expert-parallel path, see ep.cu).
 cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t *idx, const int32_t *inv,
-                             const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s);
+                             const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s,
+                             const int32_t *compact_gs = nullptr, const int32_t *compact_off = nullptr);
+
+// Expert-parallel path (ep.cu).  Routing weight of every sorted row in compact order.
+cudaError_t launch_ep_row_weights(const int32_t *perm, const int32_t *tile_expert, const int32_t *counts,
+                                  const int32_t *offsets, const int32_t *group_start, const float *topk_w, int E,
+                                  int64_t P, int64_t p_cap, float *w_rows, int sms, cudaStream_t s);
+// Expert side: routing state of the received rows from recv[G][E] (one block).
+cudaError_t launch_ep_layout(int G, int E, const int32_t *recv, int64_t p_cap, int32_t *counts, int32_t *offsets,
+                             int32_t *group_start, int32_t *tile_expert, int32_t *perm, int32_t *inv, int *status,
+                             cudaStream_t s);
+// out[t] = slot-ordered sum of the compact rows of token t's pairs.
+cudaError_t launch_ep_combine(const __nv_bfloat16 *rows, const int32_t *idx, const int32_t *inv,
+                              const int32_t *offsets, const int32_t *group_start, int T, int E, int k, int d,
+                              int64_t P, __nv_bfloat16 *out, int *status, int sms, cudaStream_t s);
 
 cudaError_t launch_expire_wait(int *status, cudaStream_t s);
 

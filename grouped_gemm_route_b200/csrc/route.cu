@@ -881,12 +881,18 @@ const void *route_lane_fn(int E, int k) {
 
 constexpr int kBwdThreads = 256;
 
+// dscore[t, j] = the ordered sum of the dscore partials of pair (t, j)'s row,
+// and dlogits through the renormalised softmax.  The row is inv[t, j] (the
+// sorted layout); with compact_gs / compact_off (expert-parallel path) it is
+// the pair's compact sorted index offsets[e] + inv[t, j] - group_start[e].
 __global__ void __launch_bounds__(kBwdThreads) route_bwd_kernel(int T, int E, int k, const float *__restrict__ w,
                                                                 const int32_t *__restrict__ idx,
                                                                 const int32_t *__restrict__ inv,
                                                                 const float *__restrict__ dpart, int dpart_stride,
                                                                 float *__restrict__ dscore,
-                                                                float *__restrict__ dlogits) {
+                                                                float *__restrict__ dlogits,
+                                                                const int32_t *__restrict__ compact_gs,
+                                                                const int32_t *__restrict__ compact_off) {
     __shared__ float s_ds[kBwdThreads / 32][kMaxTopK];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * (kBwdThreads / 32) + warp;
@@ -894,7 +900,11 @@ __global__ void __launch_bounds__(kBwdThreads) route_bwd_kernel(int T, int E, in
     if (dlogits)
         for (int e = lane; e < E; e += 32) dlogits[static_cast<size_t>(t) * E + e] = 0.f;
     for (int j = lane; j < k; j += 32) {
-        const int pos = inv[static_cast<size_t>(t) * k + j];
+        int pos = inv[static_cast<size_t>(t) * k + j];
+        if (compact_gs != nullptr) {
+            const int e = idx[static_cast<size_t>(t) * k + j];
+            pos = e >= 0 && e < E ? compact_off[e] + pos - compact_gs[e] : 0;
+        }
         float ds = 0.f;
         for (int n = 0; n < dpart_stride; ++n) ds += dpart[static_cast<size_t>(pos) * dpart_stride + n];
         dscore[static_cast<size_t>(t) * k + j] = ds;
@@ -1080,10 +1090,12 @@ cudaError_t launch_route_perm(int T, int E, int k, const int32_t *idx, const int
 }
 
 cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t *idx, const int32_t *inv,
-                             const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s) {
+                             const float *dpart, int dpart_stride, float *dscore, float *dlogits, cudaStream_t s,
+                             const int32_t *compact_gs, const int32_t *compact_off) {
     const int per_block = kBwdThreads / 32;
     const int blocks = (T + per_block - 1) / per_block;
-    route_bwd_kernel<<<blocks, kBwdThreads, 0, s>>>(T, E, k, w, idx, inv, dpart, dpart_stride, dscore, dlogits);
+    route_bwd_kernel<<<blocks, kBwdThreads, 0, s>>>(T, E, k, w, idx, inv, dpart, dpart_stride, dscore, dlogits,
+                                                    compact_gs, compact_off);
     return cudaGetLastError();
 }
 

@@ -27,7 +27,8 @@ SAVED_FIELDS = ("topk_idx", "topk_w", "counts", "offsets", "group_start", "tile_
                 "xs")
 EXPORTS = ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
            "moe_error_string", "moe_profile_enable", "moe_profile_read", "moe_kernel_name",
-           "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_recompute")
+           "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_recompute", "moe_ep_expert_layout",
+           "moe_ep_dispatch", "moe_expert_fwd", "moe_expert_bwd", "moe_ep_combine", "moe_ep_backward_finish")
 
 
 class MoeShape(ctypes.Structure):
@@ -76,6 +77,16 @@ def lib() -> ctypes.CDLL:
     L.moe_selftest_wait_timeout.restype = ctypes.c_int
     L.moe_kernel_name.argtypes = [ctypes.c_int]
     L.moe_kernel_name.restype = ctypes.c_char_p
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    L.moe_ep_expert_layout.argtypes = [ctypes.c_int, ctypes.c_int, P, i64p, i64p, i64p, i64p]
+    L.moe_ep_dispatch.argtypes = [S, P, ctypes.POINTER(MoeSaved), P, P, P]
+    L.moe_expert_fwd.argtypes = [S, ctypes.c_int, P, P, P, P, P, ctypes.POINTER(MoeSaved), P, ctypes.c_size_t, P]
+    L.moe_expert_bwd.argtypes = [S, P, P, P, P, ctypes.POINTER(MoeSaved), P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_ep_combine.argtypes = [S, ctypes.POINTER(MoeSaved), P, P, P]
+    L.moe_ep_backward_finish.argtypes = [S, ctypes.POINTER(MoeSaved), P, P, P, P, P, P]
+    for name in ("moe_ep_expert_layout", "moe_ep_dispatch", "moe_expert_fwd", "moe_expert_bwd", "moe_ep_combine",
+                 "moe_ep_backward_finish"):
+        getattr(L, name).restype = ctypes.c_int
     for name in ("moe_saved_sizes", "moe_workspace_size", "moe_route", "moe_fwd", "moe_bwd", "moe_get_status",
                  "moe_profile_enable", "moe_profile_read"):
         getattr(L, name).restype = ctypes.c_int
@@ -172,6 +183,67 @@ def recompute(shape, x, wgu, saved: dict, ws, stream=None):
     with _on(x):
         _check(lib().moe_recompute(ctypes.byref(shape), _ptr(x), _ptr(wgu), ctypes.byref(st), _ptr(ws),
                                    ws.numel(), _stream(stream, x)), "moe_recompute")
+
+
+# ----------------------------------------------------------------------------
+# expert parallelism (see include/moe.h): the device steps; grouped_gemm_route_b200.ep
+# runs the exchanges between them
+# ----------------------------------------------------------------------------
+def ep_expert_layout(G: int, E_loc: int, recv_counts):
+    """Host only.  recv_counts: int array-like [G, E_loc] (rows of local expert e
+    from source s).  Returns (row_off [G, E_loc], cmp_off [G, E_loc], rows,
+    padded_rows) as Python ints: where each (source, expert) segment lands in
+    the padded local layout and in compact order."""
+    flat = [int(c) for c in torch.as_tensor(recv_counts).reshape(-1).tolist()]
+    if len(flat) != G * E_loc:
+        raise ValueError("recv_counts must hold G * E_loc counts")
+    rc = (ctypes.c_int32 * len(flat))(*flat)
+    row_off = (ctypes.c_int64 * len(flat))()
+    cmp_off = (ctypes.c_int64 * len(flat))()
+    rows, padded = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().moe_ep_expert_layout(G, E_loc, rc, row_off, cmp_off, ctypes.byref(rows), ctypes.byref(padded)),
+           "moe_ep_expert_layout")
+    ro = [[row_off[s * E_loc + e] for e in range(E_loc)] for s in range(G)]
+    co = [[cmp_off[s * E_loc + e] for e in range(E_loc)] for s in range(G)]
+    return ro, co, int(rows.value), int(padded.value)
+
+
+def ep_dispatch(shape, src, saved: dict, dst, w_rows=None, stream=None):
+    st = saved_struct(saved)
+    with _on(src):
+        _check(lib().moe_ep_dispatch(ctypes.byref(shape), _ptr(src), ctypes.byref(st), _ptr(dst), _ptr(w_rows),
+                                     _stream(stream, src)), "moe_ep_dispatch")
+
+
+def expert_fwd(shape, G, recv_counts, xr, wgu, wd, y_rows, saved: dict, ws, stream=None):
+    st = saved_struct(saved)
+    with _on(xr):
+        _check(lib().moe_expert_fwd(ctypes.byref(shape), int(G), _ptr(recv_counts), _ptr(xr), _ptr(wgu), _ptr(wd),
+                                    _ptr(y_rows), ctypes.byref(st), _ptr(ws), ws.numel(), _stream(stream, xr)),
+               "moe_expert_fwd")
+
+
+def expert_bwd(shape, gr, xr, wgu, wd, saved: dict, dx_rows, dwgu, dwd, ds_rows, ws, stream=None):
+    st = saved_struct(saved)
+    with _on(gr):
+        _check(lib().moe_expert_bwd(ctypes.byref(shape), _ptr(gr), _ptr(xr), _ptr(wgu), _ptr(wd), ctypes.byref(st),
+                                    _ptr(dx_rows), _ptr(dwgu), _ptr(dwd), _ptr(ds_rows), _ptr(ws), ws.numel(),
+                                    _stream(stream, gr)), "moe_expert_bwd")
+
+
+def ep_combine(shape, saved: dict, rows, out, stream=None):
+    st = saved_struct(saved)
+    with _on(rows):
+        _check(lib().moe_ep_combine(ctypes.byref(shape), ctypes.byref(st), _ptr(rows), _ptr(out),
+                                    _stream(stream, rows)), "moe_ep_combine")
+
+
+def ep_backward_finish(shape, saved: dict, dx_rows, ds_rows, dx, dscore, dlogits, stream=None):
+    st = saved_struct(saved)
+    with _on(dx_rows):
+        _check(lib().moe_ep_backward_finish(ctypes.byref(shape), ctypes.byref(st), _ptr(dx_rows), _ptr(ds_rows),
+                                            _ptr(dx), _ptr(dscore), _ptr(dlogits), _stream(stream, dx_rows)),
+               "moe_ep_backward_finish")
 
 
 def get_status(ws, stream=None) -> int:

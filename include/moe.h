@@ -36,7 +36,11 @@
  *     tensor is row-major and contiguous.  bf16 = IEEE bfloat16 (2 bytes).
  *   - The caller owns and allocates every buffer (outputs, saved state and the
  *     workspace).  The library never allocates or frees device memory and keeps
- *     no state between calls except cached per-device properties.
+ *     no state between calls except cached per-device properties and, per
+ *     device, one extra stream with two events: moe_bwd forks bandwidth-bound
+ *     work onto it beside a tensor-bound GEMM and joins it back into `stream`
+ *     before its last kernel (ordering on `stream` is as if everything ran
+ *     there).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Calls that share a workspace must not overlap on the GPU.
  *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Arguments are
@@ -206,6 +210,98 @@ int moe_recompute(const moe_shape_t *shape, const void *x, const void *w_gate_up
  * must be serialised by the caller.  Device-side index checks are not
  * reported by this entry point (it has no status word). */
 int moe_route_noalloc(const moe_shape_t *shape, const float *logits, moe_saved_t *saved, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Expert parallelism (EP).  "Prime Intellect's Prime Mega MoE Trains Giant AI
+ * Models 55% Faster", sections "Where MoE training loses time" and "One kernel
+ * overlaps the pipeline": the experts are spread over G GPUs, every token
+ * travels to the GPUs that own its experts and the results travel back; the
+ * backward pass repeats the exchange for gradients.
+ *
+ * Rank q of G owns the E/G consecutive experts [q*E/G, (q+1)*E/G) (E a
+ * multiple of G).  Every rank holds its own T tokens and the weights of its
+ * own experts.  The exchanges are copies between the GPUs' own memories (NCCL
+ * send/receive, issued by the caller between these calls); no kernel here
+ * reads another GPU's memory.  One layer step on every rank:
+ *
+ *  source side   moe_route over all E experts, then moe_ep_dispatch: x rows in
+ *                the sorted layout (`xs`, group of expert e at group_start[e])
+ *                and the routing weight of every pair in compact sorted order
+ *                (`w_rows`: expert e's pairs at offsets[e] ..).  Because the
+ *                experts of one rank are consecutive, so are their groups.
+ *                For destination q and each of its experts e it sends
+ *                counts[e] rows of xs from row group_start[e] and counts[e]
+ *                weights of w_rows from offsets[e]; it sends counts[q*E/G ..
+ *                (q+1)*E/G - 1] first, so that q can size its buffers.
+ *  expert side   recv_counts[s][e] = rows of local expert e from source s.
+ *                moe_ep_expert_layout (host) gives where those land: xr row
+ *                row_off[s][e] (the local sorted layout, every local expert's
+ *                group padded to 128 rows, sources in rank order inside it)
+ *                and compact index cmp_off[s][e] (w_rows, results).
+ *                moe_expert_fwd runs the gate/up GEMM + SwiGLU and the down
+ *                GEMM on them; each received row's product w * y goes to its
+ *                compact index of y_rows, which the expert side sends back:
+ *                recv_counts[s][e] rows from cmp_off[s][e] to source s.
+ *  source side   receives them at compact index offsets[e] + ... (the mirror
+ *                of its sends) and moe_ep_combine sums each token's k rows in
+ *                slot order into out.
+ *  backward      source: moe_ep_dispatch of grad_out (no weights), sent like
+ *                x.  Expert: moe_expert_bwd -> dx rows and dscore rows
+ *                (compact, sent back like y) and the local experts' dW.
+ *                Source: moe_ep_backward_finish -> dx, dscore, dlogits.
+ *
+ * With G = 1 the results are those of moe_fwd / moe_bwd, bit for bit.  Only
+ * bf16 operands, and the gate/up GEMM on CTA pairs (max_sms != 1), are
+ * supported on the expert side; other shapes return MOE_ERR_UNSUPPORTED.
+ * The source-side calls take no workspace: their index checks skip a bad row
+ * without reporting it.
+ * ------------------------------------------------------------------------- */
+
+/* Host only.  recv_counts: host int32 [G][E_loc].  Writes row_off[G][E_loc]
+ * (first row of each (source, expert) segment in the expert side's padded
+ * sorted layout), cmp_off[G][E_loc] (first compact index), the number of rows
+ * received and the padded row count.  MOE_ERR_ARG on a negative count. */
+int moe_ep_expert_layout(int G, int E_loc, const int32_t *recv_counts, int64_t *row_off, int64_t *cmp_off,
+                         int64_t *rows, int64_t *padded_rows);
+
+/* Source side, after moe_route with the same shape: src (bf16 [T,d], x or
+ * grad_out) into dst (bf16 [P_cap, d], sorted layout; padding rows are not
+ * written) and, when w_rows is not NULL, w_rows (fp32 [T*k]) = the routing
+ * weight of each pair in compact sorted order. */
+int moe_ep_dispatch(const moe_shape_t *shape, const void *src, const moe_saved_t *saved, void *dst, float *w_rows,
+                    void *stream);
+
+/* Expert side, forward.  shape: T = rows received (from moe_ep_expert_layout),
+ * k = 1, E = E_loc, d, I as the layer's; every buffer sized by
+ * moe_saved_sizes / moe_workspace_size for that shape.  recv_counts: device
+ * int32 [G][E_loc].  xr: bf16 [P_cap, d], the received rows at row_off (its
+ * padding rows are zeroed here).  saved->topk_w: the received weights (compact
+ * order); the call fills the other routing fields of `saved` for the received
+ * layout (perm: padded row -> compact index, inv: compact index -> padded row)
+ * and h, aw.  w_gate_up, w_down: the local experts' weights [E_loc, ...].
+ * y_rows: bf16 [T, d], row i = w_i * (W_down a) of compact row i. */
+int moe_expert_fwd(const moe_shape_t *shape, int G, const int32_t *recv_counts, void *xr, const void *w_gate_up,
+                   const void *w_down, void *y_rows, moe_saved_t *saved, void *ws, size_t ws_bytes, void *stream);
+
+/* Expert side, backward, after moe_expert_fwd on the same `saved`.  gr: bf16
+ * [P_cap, d], the received grad_out rows at row_off (padding zeroed here).
+ * Writes dx_rows (bf16 [T, d], compact), ds_rows (fp32 [T], dL/dw of each
+ * received pair, compact) and the local experts' dw_gate_up, dw_down (an expert
+ * that received no row gets exact zeros). */
+int moe_expert_bwd(const moe_shape_t *shape, void *gr, const void *xr, const void *w_gate_up, const void *w_down,
+                   const moe_saved_t *saved, void *dx_rows, void *dw_gate_up, void *dw_down, float *ds_rows,
+                   void *ws, size_t ws_bytes, void *stream);
+
+/* Source side: out[t] (bf16 [T,d]) = sum over slots j = 0..k-1, in slot order,
+ * of rows (bf16 [T*k, d], compact sorted order, as received back) of token t's
+ * pairs; fp32 sum, one bf16 rounding. */
+int moe_ep_combine(const moe_shape_t *shape, const moe_saved_t *saved, const void *rows, void *out, void *stream);
+
+/* Source side, backward: dx (bf16 [T,d]) from dx_rows as moe_ep_combine does;
+ * dscore[t,j] (fp32 [T,k]) = ds_rows of the pair; dlogits (fp32 [T,E], or NULL)
+ * through the renormalised softmax, as moe_bwd computes them. */
+int moe_ep_backward_finish(const moe_shape_t *shape, const moe_saved_t *saved, const void *dx_rows,
+                           const float *ds_rows, void *dx, float *dscore, float *dlogits, void *stream);
 
 /* Synchronises `stream`, then reads the device status word of `ws` written by
  * the most recent moe_route / moe_fwd / moe_bwd on that workspace:
