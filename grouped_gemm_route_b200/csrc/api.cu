@@ -211,6 +211,19 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint
     return r == CUDA_SUCCESS;
 }
 
+// 2-d bf16 tensor [rows, cols], box = 128 rows x 32 columns (64-byte rows), 64-byte swizzle: the
+// chunks of h the down dgrad's loader warp moves into its ring.
+bool make_map_h(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {32, 128};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // 2-d E4M3 tensor [rows, cols] (row-major bytes), box = box_rows x 128 columns, 128-byte swizzle.
 bool make_map8(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint32_t box_rows) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -465,15 +478,17 @@ int sort_x(const Plan &pl, const DeviceInfo &dev, const void *x, const moe_saved
 // The bf16 gate/up GEMM on CTA pairs over x already in the sorted layout.
 int gateup_pair_sorted(const Plan &pl, const moe_shape_t *shape, const DeviceInfo &dev, const void *xs,
                        const void *w_gate_up, moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
-    CUtensorMap tm_wgu, tm_xs;  // the pair kernel loads W_gate_up in 64-row boxes (gate and up halves)
+    // the pair kernel loads W_gate_up in 64-row boxes (gate and up halves), and x in 128-row boxes
+    // (64-row boxes for an expert's unpaired last tile)
+    CUtensorMap tm_wgu, tm_xs, tm_xs64;
     if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 64) ||
-        !make_map(&tm_xs, xs, pl.p_cap, pl.d, 128))
+        !make_map(&tm_xs, xs, pl.p_cap, pl.d, 128) || !make_map(&tm_xs64, xs, pl.p_cap, pl.d, 64))
         return MOE_ERR_LAUNCH;
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.I / 128;
     a.num_k_blocks = pl.d / kTileK;
     Launch L(kKindGemmGateUpFwd, st);
-    return L.done(launch_gemm_pair(kGateUpFwd, a, tm_xs, tm_wgu, grid_for(shape, dev), st));
+    return L.done(launch_gemm_pair(kGateUpFwd, a, tm_xs, tm_wgu, grid_for(shape, dev), st, &tm_xs64));
 }
 
 int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,
@@ -610,12 +625,19 @@ int bwd_gemms(const Plan &pl, const DeviceInfo &dev, int grid, GemmArgs a, const
         !make_map(&tm_gs_mn, gs, pl.p_cap, pl.d, 64) || !make_map(&tm_xs_mn, xs, pl.p_cap, pl.d, 64))
         return MOE_ERR_LAUNCH;
     if (stage != nullptr) a.stage = static_cast<__nv_bfloat16 *>(stage);
-    // b1: down dgrad, dscore partials, SwiGLU backward -> dh
+    // b1: down dgrad, dscore partials, SwiGLU backward -> dh (CTA pairs: h streamed into a ring by TMA)
     a.n_tiles = pl.I / pl.bn_i;
     a.num_k_blocks = pl.d / kTileK;
     {
         Launch L(kKindGemmDownDgrad, st);
-        if ((rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, false, a, tm_gs_rows, tm_wd_mn, grid, st)))) return rc;
+        if (gemm_pair_ok(kDownDgrad, pl.bn_i, false, 0, grid)) {
+            CUtensorMap tm_h;
+            if (!make_map_h(&tm_h, saved->h, pl.p_cap, 2 * pl.I)) return MOE_ERR_LAUNCH;
+            rc = L.done(launch_gemm_pair(kDownDgrad, a, tm_gs_rows, tm_wd_mn, grid, st, &tm_h));
+        } else {
+            rc = L.done(launch_gemm(kDownDgrad, pl.bn_i, false, a, tm_gs_rows, tm_wd_mn, grid, st));
+        }
+        if (rc) return rc;
     }
     // b3: down wgrad  dW_down[e] = sum_p gout[t] (x) aw_p
     a.m_tiles = pl.d / kTileM;

@@ -747,6 +747,102 @@ __device__ __forceinline__ void epi_down_dgrad(const GemmArgs &a, const Tile &t,
     a.dpart[static_cast<size_t>(pos) * a.dpart_stride + kSplit * t.nt + ch] = valid ? ds : 0.f;
 }
 
+// Store each lane's 32 bytes v (16 bf16) to rowptr (nullptr: that row is
+// skipped) through the warp's shared buffer: a store instruction then covers
+// 16 rows x 32 contiguous bytes.  16-byte pieces are XOR-swizzled by bit 2 of
+// the row (no bank conflicts beyond the minimum in either pass).
+__device__ __forceinline__ uint32_t xpose16_off(int row, int piece) {
+    return static_cast<uint32_t>(row * 32 + ((piece ^ ((row >> 2) & 1)) << 4));
+}
+
+__device__ __forceinline__ void warp_store_rows16(uint8_t *buf, const uint32_t (&v)[8], void *rowptr) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+        *reinterpret_cast<uint4 *>(buf + xpose16_off(lane, q)) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    __syncwarp();
+    const int piece = lane & 1;
+    const unsigned long long mine = reinterpret_cast<unsigned long long>(rowptr);
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int row = rr * 16 + (lane >> 1);
+        const uint4 val = *reinterpret_cast<const uint4 *>(buf + xpose16_off(row, piece));
+        char *dst = reinterpret_cast<char *>(__shfl_sync(0xffffffffu, mine, row));
+        if (dst != nullptr) *reinterpret_cast<uint4 *>(dst + piece * 16) = val;
+    }
+    __syncwarp();
+}
+
+// Down dgrad on CTA pairs (BN = 256).  The h values of chunk c -- gate and up
+// columns nt * 256 + c * 32 .. +32 of this CTA's 128 rows -- arrive in ring
+// slot hit & 1: two TMA boxes of 128 rows x 64 bytes with the 64-byte swizzle
+// (16-byte piece q of row r at piece q ^ ((r >> 1) & 3)), loaded by the h
+// loader warp one chunk ahead.  The two warps of a tensor-memory lane quadrant
+// take 16 columns of each chunk each (ch).  Same arithmetic as
+// epi_down_dgrad; dpart gets one partial per (row, n tile, ch).  Returns false
+// when a bounded wait expired.
+__device__ __forceinline__ bool epi_down_dgrad_ring(const GemmArgs &a, const Tile &t, int r, int ch, uint32_t taddr,
+                                                    uint64_t *tempty_acc, uint8_t *xbuf, const uint8_t *ring,
+                                                    uint64_t *hfull, uint64_t *hempty, int &hit,
+                                                    volatile int *abort_flag) {
+    constexpr int BN = 256;
+    constexpr int kSlot = 2 * kTileM * 32 * 2;
+    constexpr int kSplit = ModeTraits<kDownDgrad>::kSplit;
+    const int lane = threadIdx.x & 31;
+    const int pos = t.row0 + r;
+    const int p = __ldg(a.perm + pos);
+    const bool valid = p >= 0 && p < a.T * a.k;
+    const float wv = valid ? __ldg(a.topk_w + p) : 0.f;
+    __nv_bfloat16 *dhrow = a.dh + static_cast<size_t>(pos) * 2 * a.I + t.nt * BN;
+    const int sw = (r >> 1) & 3;
+    float ds = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c, ++hit) {
+        const int slot = hit & 1;
+        if (!warp_wait(&hfull[slot], static_cast<uint32_t>(hit >> 1) & 1u, abort_flag)) return false;
+        const uint8_t *gbox = ring + slot * kSlot;
+        const uint8_t *ubox = gbox + kSlot / 2;
+        uint32_t hg[8], hu[8];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint32_t off = static_cast<uint32_t>(r * 64 + (((2 * ch + q) ^ sw) << 4));
+            const uint4 g = *reinterpret_cast<const uint4 *>(gbox + off);
+            const uint4 u = *reinterpret_cast<const uint4 *>(ubox + off);
+            hg[4 * q] = g.x; hg[4 * q + 1] = g.y; hg[4 * q + 2] = g.z; hg[4 * q + 3] = g.w;
+            hu[4 * q] = u.x; hu[4 * q + 1] = u.y; hu[4 * q + 2] = u.z; hu[4 * q + 3] = u.w;
+        }
+        float G[16];
+        tmem_load16_sync(taddr + c * 32 + ch * 16, G);
+        if (c + 1 == BN / 32) release_acc<true>(tempty_acc);  // tensor memory no longer needed
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&hempty[slot]);  // this warp is done with the slot
+        float dg[16], du[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float g0 = (i & 1) ? bf16_hi(hg[i >> 1]) : bf16_lo(hg[i >> 1]);
+            const float u0 = (i & 1) ? bf16_hi(hu[i >> 1]) : bf16_lo(hu[i >> 1]);
+            const float g = fminf(g0, a.limit), u = fminf(fmaxf(u0, -a.limit), a.limit);
+            const float gr = G[i];
+            const float sg = __fdividef(1.f, 1.f + __expf(-g));
+            const float sl = g * sg;
+            ds += gr * (sl * u);
+            const float da = wv * gr;
+            dg[i] = valid && g0 <= a.limit ? da * u * sg * (1.f + g * (1.f - sg)) : 0.f;
+            du[i] = valid && fabsf(u0) <= a.limit ? da * sl : 0.f;
+        }
+        uint32_t pdg[8], pdu[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            pdg[i] = pack_bf16x2(dg[2 * i], dg[2 * i + 1]);
+            pdu[i] = pack_bf16x2(du[2 * i], du[2 * i + 1]);
+        }
+        warp_store_rows16(xbuf, pdg, dhrow + c * 32 + ch * 16);
+        warp_store_rows16(xbuf, pdu, dhrow + a.I + c * 32 + ch * 16);
+    }
+    a.dpart[static_cast<size_t>(pos) * a.dpart_stride + kSplit * t.nt + ch] = valid ? ds : 0.f;
+    return true;
+}
+
 // weight gradients: store the tile (zeros for an expert without tokens)
 template <int MODE, int BN, bool PAIR = false>
 __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
@@ -959,10 +1055,14 @@ struct PairCfg {
     static constexpr int kStageBytes = kABytes + kBHalfBytes;
     static constexpr int kOrderBytes = 8 * kMaxExperts;  // wgrads: counts + order; M-tiled: pair-row starts
     static constexpr int kXposeTotal = TR::kEpiWarps * kXposeBytes;
-    static constexpr int kFixed = 512 + kOrderBytes + kXposeTotal + 1024;
+    // down dgrad: a ring of two h chunks (gate and up, 128 rows x 32 columns each)
+    static constexpr int kRingSlotBytes = 2 * kTileM * 32 * 2;
+    static constexpr int kRingBytes = MODE == kDownDgrad ? 2 * kRingSlotBytes : 0;
+    static constexpr int kFixed = 512 + kOrderBytes + kXposeTotal + kRingBytes + 1024;
     static constexpr int kFit = (227 * 1024 - kFixed) / kStageBytes;
     static constexpr int kStages = kFit < 6 ? kFit : 6;
-    static constexpr int kBarOffset = kStages * kStageBytes;
+    static constexpr int kRingOffset = kStages * kStageBytes;  // 1024-byte aligned (stages are 32 KB)
+    static constexpr int kBarOffset = kRingOffset + kRingBytes;
     static constexpr int kOrderOffset = kBarOffset + 512;
     static constexpr int kXposeOffset = kOrderOffset + kOrderBytes;
     static constexpr int kSmemBytes = kXposeOffset + kXposeTotal + 1024;
@@ -1029,8 +1129,9 @@ __device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, co
 template <int MODE, int BN>
 __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const GemmArgs args) {
-    static_assert(MODE == kGateUpFwd || MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad,
+                             const __grid_constant__ CUtensorMap tmA64, const GemmArgs args) {
+    static_assert(MODE == kGateUpFwd || MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad ||
+                      MODE == kDownDgrad,
                   "the modes where pairs measured faster than one CTA");
     using P = PairCfg<MODE, BN>;
     using TR = ModeTraits<MODE>;
@@ -1041,10 +1142,13 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     uint64_t *tfull = empty + P::kStages;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *hfull = drain + 1;   // down dgrad: h ring slots loaded (TMA bytes)
+    uint64_t *hempty = hfull + 2;  // down dgrad: h ring slots read by every epilogue warp
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(hempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_count = reinterpret_cast<int *>(smem + P::kOrderOffset);
     int *tbl = TR::kMTiled ? s_count : s_count + kMaxExperts;  // pair-row starts, or the expert order
+    uint8_t *ring = smem + P::kRingOffset;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1094,6 +1198,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], 2 * TR::kEpiWarps);  // the epilogue warps of both CTAs (leader's barrier)
+            mbar_init(&hfull[i], 1);                   // this CTA's h loader
+            mbar_init(&hempty[i], TR::kEpiWarps);      // this CTA's epilogue warps
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -1123,7 +1229,9 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                if (leader && lane == 0) mbar_arrive_expect_tx(&full[s], 2u * P::kStageBytes);
+                // a half tile's A is 64 rows (tmA64) in each CTA
+                if (leader && lane == 0)
+                    mbar_arrive_expect_tx(&full[s], t.half ? 2u * (P::kStageBytes - kABytes / 2) : 2u * P::kStageBytes);
                 __syncwarp();
                 const uint32_t fb = cluster_addr(&full[s], 0);
                 uint8_t *As = smem + s * P::kStageBytes;
@@ -1131,16 +1239,23 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 const int k0 = kb * kTileK;
                 const int bcol = t.nt * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B columns
                 if constexpr (MODE == kGateUpFwd) {
-                    // A: 128 sorted rows of x from row0 (a half tile's MMA reads the first 64);
+                    // A: 128 sorted rows of x from row0 (a half tile: 64 rows, all its MMA reads);
                     // B: the tile covers gate/up columns nt*128 .. +128; the leader loads 64 gate
                     // rows and the 64 matching up rows for the first 64 of them, the peer for the
                     // other 64 (64-row boxes, K-major), so that accumulator columns hold, per
                     // 64-column group, gate then up of the same expert columns -- in a half tile
                     // each TMEM lane half then holds whole (gate, up) pairs
-                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.row0);
+                    if (lane == 0) tma_load_2d_pair(As, t.half ? &tmA64 : &tmA, fb, k0, t.row0);
                     const int grow = t.e * 2 * a.I + t.nt * (BN / 2) + 64 * static_cast<int>(rank);
                     if (lane == 1) tma_load_2d_pair(Bs, &tmB, fb, k0, grow);
                     if (lane == 2) tma_load_2d_pair(Bs + 64 * 128, &tmB, fb, k0, grow + a.I);
+                } else if constexpr (MODE == kDownDgrad) {
+                    // A: 128 sorted rows of grad_out, K-major; B: this CTA's half of W_down[e]
+                    // (its N = I columns), MN-major
+                    const int brow = t.e * a.d + k0;
+                    if (lane == 0) tma_load_2d_pair(As, &tmA, fb, k0, t.row0);
+                    if (lane >= 1 && lane < 1 + BN / 128)
+                        tma_load_2d_pair(Bs + (lane - 1) * kChunkBytes, &tmB, fb, bcol + 64 * (lane - 1), brow);
                 } else if constexpr (TR::kMTiled) {
                     // A: 128 sorted rows of dh from row0, K-major; B: this CTA's half of W_gate_up[e], MN-major
                     const int brow = t.e * 2 * a.I + k0;
@@ -1211,6 +1326,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         uint8_t *xbuf = smem + P::kXposeOffset + (warp - kEpiWarp0) * kXposeBytes;
+        int hit = 0;  // down dgrad: h ring chunks consumed so far
         int local = 0;
         for (int tile = nth_tile<MODE>(0, pair, npairs); tile < total;
              tile = nth_tile<MODE>(++local, pair, npairs)) {
@@ -1226,6 +1342,14 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
             if constexpr (MODE == kGateUpFwd) {
                 epi_gateup_fwd_pair(a, t, quad, lane, taddr, &tempty[acc], xbuf);
+            } else if constexpr (MODE == kDownDgrad) {
+                if (t.skip) {
+                    release_acc<true>(&tempty[acc]);
+                } else if (!epi_down_dgrad_ring(a, t, r, (warp - kEpiWarp0) >> 2, taddr, &tempty[acc], xbuf, ring,
+                                                hfull, hempty, hit, abort_flag)) {
+                    raise_abort(abort_flag, a.status);
+                    break;
+                }
             } else if constexpr (TR::kStage) {
                 if (t.skip)
                     release_acc<true>(&tempty[acc]);
@@ -1235,6 +1359,37 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
             }
         }
+    }
+
+    if constexpr (MODE == kDownDgrad) {
+        if (warp == TR::kGatherWarp0 && lane == 0) {
+            // ---- h loader: this CTA's rows of h, chunk by chunk, one chunk ahead of the epilogue ----
+            int hit = 0;
+            bool ok = true;
+            for (int tile = nth_tile<MODE>(0, pair, npairs), i = 0; tile < total && ok;
+                 tile = nth_tile<MODE>(++i, pair, npairs)) {
+                const Tile t = decode_pair_tile<MODE>(tile, a, tbl, rank);
+                if (t.skip) continue;
+                for (int c = 0; c < BN / 32; ++c, ++hit) {
+                    const int slot = hit & 1;
+                    if (!mbar_wait(&hempty[slot], (static_cast<uint32_t>(hit >> 1) & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&hfull[slot], P::kRingSlotBytes);
+                    uint8_t *dst = ring + slot * P::kRingSlotBytes;
+                    const int col = t.nt * BN + c * 32;
+                    tma_load_2d(dst, &tmA64, &hfull[slot], col, t.row0);                        // gate
+                    tma_load_2d(dst + P::kRingSlotBytes / 2, &tmA64, &hfull[slot], a.I + col, t.row0);  // up
+                }
+            }
+            if (!ok) {
+                raise_abort(abort_flag, a.status);
+                for (int q = hit > 2 ? hit - 2 : 0; q < hit; ++q)  // its copies in flight land first
+                    mbar_wait(&hfull[q & 1], static_cast<uint32_t>(q >> 1) & 1u, nullptr);
+            }
+        }
+        __syncwarp();
     }
 
     tc_fence_before_sync();
@@ -1283,8 +1438,8 @@ cudaError_t launch_mode(int bn, bool mx, const GemmArgs &args, const CUtensorMap
 // Launch of a CTA-pair kernel: clusters of two, as many pairs as the GPU holds
 // at once (capped by the grid the caller offers).
 template <int MODE>
-cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid,
-                        cudaStream_t s) {
+cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        const CUtensorMap &tmA64, int grid, cudaStream_t s) {
     using P = PairCfg<MODE, 256>;
     auto *fn = grouped_gemm_pair_kernel<MODE, 256>;
     static std::atomic<int> max_pairs_plus1[kMaxDevices];  // per instantiation and device: resident
@@ -1316,7 +1471,7 @@ cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUte
     const int pairs = (grid / 2) < max_pairs ? grid / 2 : max_pairs;
     if (pairs < 1) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3(2 * pairs);
-    return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, args);
+    return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, tmA64, args);
 }
 
 }  // namespace
@@ -1337,16 +1492,20 @@ cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, co
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid) {
     if (mx || bn != 256 || grid < 2) return false;
     if (mode == kDownWgrad || mode == kGateUpWgrad) return m_tiles % 2 == 0;
-    return mode == kGateUpFwd || mode == kGateUpDgrad;
+    return mode == kGateUpFwd || mode == kGateUpDgrad || mode == kDownDgrad;
 }
 
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                             int grid, cudaStream_t s) {
+                             int grid, cudaStream_t s, const CUtensorMap *tmA64) {
+    const CUtensorMap &a64 = tmA64 != nullptr ? *tmA64 : tmA;
     switch (mode) {
-        case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, grid, s);
-        case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, grid, s);
-        case kGateUpFwd: return launch_pair<kGateUpFwd>(args, tmA, tmB, grid, s);
-        case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, grid, s);
+        case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, a64, grid, s);
+        case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, a64, grid, s);
+        case kGateUpFwd: return tmA64 != nullptr ? launch_pair<kGateUpFwd>(args, tmA, tmB, a64, grid, s)
+                                                 : cudaErrorInvalidValue;  // half tiles need the 64-row map
+        case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, a64, grid, s);
+        case kDownDgrad: return tmA64 != nullptr ? launch_pair<kDownDgrad>(args, tmA, tmB, a64, grid, s)
+                                                 : cudaErrorInvalidValue;  // needs the map of h
         default: return cudaErrorInvalidValue;
     }
 }

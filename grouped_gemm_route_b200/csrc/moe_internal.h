@@ -134,8 +134,10 @@ cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, co
 // forward, the gate/up dgrad and the weight gradients; used where gemm_pair_ok
 // holds, with the same arguments and results as launch_gemm.
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid);
+// tmA64: the gate/up forward's A operand in 64-row boxes (an expert's unpaired
+// last tile loads 64 rows per CTA); unused by the other modes.
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                             int grid, cudaStream_t s);
+                             int grid, cudaStream_t s, const CUtensorMap *tmA64 = nullptr);
 
 cudaError_t launch_mx_quant_rows(const __nv_bfloat16 *src, int64_t R, int K, uint8_t *dst, uint8_t *sf, int sf_mode,
                                  int I, const int32_t *rows_used, int sms, cudaStream_t s);
