@@ -515,16 +515,21 @@ int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, 
 // row perm[pos] of `stage` (NULL: the workspace's staging buffer).
 int down_fwd_staged(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *w_down,
                     const moe_saved_t *saved, uint8_t *w8, void *stage, cudaStream_t st) {
-    CUtensorMap tm_aw, tm_wd;
-    if (!make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) ||
-        !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pl.bn_d))
+    const int grid = grid_for(shape, dev);
+    // CTA pairs: each CTA loads 128 of the tile's 256 rows of W_down, and an expert's unpaired last
+    // tile loads 64-row boxes of aw
+    const bool pair = gemm_pair_ok(kDownFwd, pl.bn_d, false, 0, grid);
+    CUtensorMap tm_aw, tm_aw64, tm_wd;
+    if (!make_map(&tm_aw, saved->aw, pl.p_cap, pl.I, 128) || !make_map(&tm_aw64, saved->aw, pl.p_cap, pl.I, 64) ||
+        !make_map(&tm_wd, w_down, static_cast<int64_t>(pl.E) * pl.d, pl.I, pair ? 128 : pl.bn_d))
         return MOE_ERR_LAUNCH;
     GemmArgs a = base_args(pl, saved, w8);
     if (stage != nullptr) a.stage = static_cast<__nv_bfloat16 *>(stage);
     a.n_tiles = pl.d / pl.bn_d;
     a.num_k_blocks = pl.I / kTileK;
     Launch L(kKindGemmDownFwd, st);
-    return L.done(launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid_for(shape, dev), st));
+    return L.done(pair ? launch_gemm_pair(kDownFwd, a, tm_aw, tm_wd, grid, st, &tm_aw64)
+                       : launch_gemm(kDownFwd, pl.bn_d, false, a, tm_aw, tm_wd, grid, st));
 }
 
 // MXFP8 backward after sort_rows: every GEMM operand quantised along that

@@ -918,6 +918,20 @@ __device__ __forceinline__ void epi_gateup_fwd_pair(const GemmArgs &a, const Til
     }
 }
 
+// Staged rows on CTA pairs, half tile (M = 128 pair MMA): the thread owns row
+// (quad & 1) * 32 + lane of this CTA's 64 rows and output columns
+// [h * 128, h * 128 + 128) of the tile, h = quad >> 1, at tensor-memory
+// columns [0, 128); staged as in epi_stage.
+__device__ __forceinline__ void epi_stage_half(const GemmArgs &a, const Tile &t, int quad, int lane, uint32_t taddr,
+                                               uint64_t *tempty_acc, uint8_t *xbuf) {
+    const int pos = t.row0 + (quad & 1) * 32 + lane;
+    const int p = __ldg(a.perm + pos);
+    const bool valid = p >= 0 && p < a.T * a.k;
+    __nv_bfloat16 *srow =
+        valid ? a.stage + static_cast<size_t>(p) * a.d + t.nt * 256 + (quad >> 1) * 128 : nullptr;
+    store_accumulator_bf16<128, true>(taddr, xbuf, srow, tempty_acc);
+}
+
 template <int MODE, int BN, bool MX>
 __device__ void epilogue_loop(const GemmArgs &a, uint64_t *tfull, uint64_t *tempty, uint32_t tmem_base,
                               const int *order, uint8_t *xbuf, volatile int *abort_flag) {
@@ -1093,13 +1107,13 @@ __device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, co
         t.e = lo;
         const int g0 = __ldg(a.group_start + lo) / kTileM, g1 = __ldg(a.group_start + lo + 1) / kTileM;
         const int t0 = g0 + 2 * (pr - tbl[lo]);  // the pair row's first tile (t0 < g1)
-        if constexpr (MODE == kGateUpFwd) {
+        if constexpr (MODE == kGateUpFwd || MODE == kDownFwd) {
             t.half = t0 + 1 >= g1;  // the expert's last tile has no partner: M = 128 pair MMA
             t.mt = t.half ? t0 : t0 + static_cast<int>(rank);
             t.row0 = t.half ? t0 * kTileM + 64 * static_cast<int>(rank) : t.mt * kTileM;
         } else {
-            // the gate/up dgrad computes the unpaired tile's partner rows and discards them (a
-            // half-row MMA measured 1.5 % slower here: its operand loads bound the pair row)
+            // the dgrads compute the unpaired tile's partner rows and discard them (a half-row MMA
+            // measured 1.5 % slower in the gate/up dgrad: its operand loads bound the pair row)
             t.mt = t0 + static_cast<int>(rank);
             t.skip = t.mt >= g1;
             t.row0 = t.mt * kTileM;
@@ -1131,7 +1145,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmA64, const GemmArgs args) {
     static_assert(MODE == kGateUpFwd || MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad ||
-                      MODE == kDownDgrad,
+                      MODE == kDownDgrad || MODE == kDownFwd,
                   "the modes where pairs measured faster than one CTA");
     using P = PairCfg<MODE, BN>;
     using TR = ModeTraits<MODE>;
@@ -1249,6 +1263,11 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                     const int grow = t.e * 2 * a.I + t.nt * (BN / 2) + 64 * static_cast<int>(rank);
                     if (lane == 1) tma_load_2d_pair(Bs, &tmB, fb, k0, grow);
                     if (lane == 2) tma_load_2d_pair(Bs + 64 * 128, &tmB, fb, k0, grow + a.I);
+                } else if constexpr (MODE == kDownFwd) {
+                    // A: 128 sorted rows of aw from row0 (a half tile: 64 rows); B: this CTA's 128 of the
+                    // tile's 256 rows of W_down[e] (output columns), K-major
+                    if (lane == 0) tma_load_2d_pair(As, t.half ? &tmA64 : &tmA, fb, k0, t.row0);
+                    if (lane == 1) tma_load_2d_pair(Bs, &tmB, fb, k0, t.e * a.d + t.nt * BN + static_cast<int>(rank) * (BN / 2));
                 } else if constexpr (MODE == kDownDgrad) {
                     // A: 128 sorted rows of grad_out, K-major; B: this CTA's half of W_down[e]
                     // (its N = I columns), MN-major
@@ -1353,6 +1372,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
             } else if constexpr (TR::kStage) {
                 if (t.skip)
                     release_acc<true>(&tempty[acc]);
+                else if (t.half)
+                    epi_stage_half(a, t, quad, lane, taddr, &tempty[acc], xbuf);
                 else
                     epi_stage<BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
             } else {
@@ -1492,7 +1513,7 @@ cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, co
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid) {
     if (mx || bn != 256 || grid < 2) return false;
     if (mode == kDownWgrad || mode == kGateUpWgrad) return m_tiles % 2 == 0;
-    return mode == kGateUpFwd || mode == kGateUpDgrad || mode == kDownDgrad;
+    return mode == kGateUpFwd || mode == kGateUpDgrad || mode == kDownDgrad || mode == kDownFwd;
 }
 
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
@@ -1506,6 +1527,8 @@ cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensor
         case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, a64, grid, s);
         case kDownDgrad: return tmA64 != nullptr ? launch_pair<kDownDgrad>(args, tmA, tmB, a64, grid, s)
                                                  : cudaErrorInvalidValue;  // needs the map of h
+        case kDownFwd: return tmA64 != nullptr ? launch_pair<kDownFwd>(args, tmA, tmB, a64, grid, s)
+                                               : cudaErrorInvalidValue;  // half tiles need the 64-row map
         default: return cudaErrorInvalidValue;
     }
 }
