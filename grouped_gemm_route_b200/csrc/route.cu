@@ -12,8 +12,9 @@
 // stable counting sort of the T*k choices by expert into a sorted layout whose
 // expert groups are padded to multiples of 128 rows (the GEMM tile height).
 //
-// The layer routes with one cooperative launch (route_fused, below: a
-// lane-per-token form for E <= 128 and a warp-per-token form otherwise).  The
+// The layer routes with one cooperative launch (route_fused, below: a form
+// with four lanes per token and one grid barrier for E <= 128, a warp per token
+// and two grid barriers otherwise).  The
 // three-launch form right below serves moe_route_noalloc: (1) per token top-k +
 // weights + a per-block expert histogram, (2) one block: totals, exclusive
 // scans, per-block bases, tile table, padding, (3) per block: each thread owns
@@ -257,7 +258,6 @@ struct RouteFusedArgs {
     int64_t p_cap;
     unsigned *barrier;  // zero before the launch
     int *status;
-    int lane_stages;    // lane form: ring depth per warp
 };
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
@@ -519,49 +519,83 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
 }
 
 // ---------------------------------------------------------------------------
-// Fused routing, lane-per-token form, for E <= 128 with E a multiple of 4k,
-// k <= 8 and 16-byte aligned logits.  Same phases and the same results as
-// route_fused_kernel; phase 1 and the positions of phase 3 give each lane one
-// token:
-//   * each lane copies its token's logit row into shared memory with one bulk
-//     copy (rows padded by 4 words, so that one-row-per-lane reads do not
-//     conflict); a warp's buffers form a ring of `stages` batches of 32 rows,
-//     the next batch in flight while the current one is processed;
-//   * tau, a lower bound on the k-th largest logit: the row is split into NG
-//     disjoint groups of consecutive experts (NG = 2k when E is a multiple of
-//     8k, else k) and tau is the k-th largest group maximum -- k groups have a
-//     maximum >= tau, so at least k logits are >= tau and each of the k
-//     largest is;
-//   * the logits >= tau (a bitmask) are visited in expert order and inserted
-//     into k sorted registers of (order key, expert): a strictly larger key
-//     moves ahead, an equal key stays behind the lower experts already there,
-//     which leaves the k largest in slot order (value descending, lower
-//     expert first on ties);
-//   * weights as in route_fused_kernel, the sum taken in slot order.
-// Positions: per batch of 32 tokens, each expert's set of lanes (a bitmask
-// built with atomicOr) gives a pair's rank among the batch's earlier tokens;
-// the highest of those lanes then advances the warp's running position.
+// Fused routing, quad form: four lanes per token, for E <= 128 with E a
+// multiple of 4, E >= 4k, k <= 8 and 16-byte aligned logits.  Same results as
+// route_fused_kernel, with one grid barrier.  Block b of G owns the tokens
+// [T*b/G, T*(b+1)/G), warp w of the block a contiguous sub-range of those.
+//
+// Phase 1: a warp takes 8 tokens at a time; lane q of a token holds the
+// 16-byte pieces q, q+4, q+8, ... of the token's logit row in registers.
+//   * tau, a lower bound on the k-th largest logit, is the k-th largest of the
+//     E/4 piece maxima: k pieces have a maximum >= tau, so at least k logits
+//     are >= tau and each of the k largest is.  Each lane sorts its piece
+//     maxima; two butterfly steps merge the four lanes' lists (the k largest
+//     of two lists A, B sorted descending are max(A_i, B_(k-1-i)), i < k).
+//   * The logits >= tau (about 9 per token on Gaussian logits) are the
+//     candidates: each lane appends its own, as 64-bit keys (order key of the
+//     value, then ~expert), to the token's list in shared memory.
+//   * A candidate's slot is its rank, the number of candidates with a larger
+//     key, so the k largest land in slot order (value descending, lower expert
+//     first on ties).  A token with more than kQuadCap candidates (many exact
+//     ties) takes its k largest one per round instead: the four lanes compare
+//     their best remaining keys and the winner leaves.
+//   * Weights as in route_fused_kernel, the sum taken in slot order.  The
+//     block's expert histogram goes to blk_hist[b].
+// Grid barrier.
+// Phase 2, in every block: each expert's total over all blocks and its sum
+// over the blocks before b (all G histograms read from L2), the padded group
+// starts (block 0 publishes counts, offsets and group starts), the tile table
+// and padding rows of experts b, b+G, ...
+// Phase 3: the block's tokens in chunks of one token per thread.  A pair's
+// rank within its expert in the chunk comes from per-warp lane masks and a
+// scan over the warps; the chunk's pairs are counting-sorted by expert in
+// shared memory and written to perm one expert's run at a time (an expert's
+// pairs of one chunk are consecutive in perm), so the stores are coalesced.
 // ---------------------------------------------------------------------------
-constexpr int kLaneMaxWarps = 16;
-constexpr int kLaneMaxE = 128;
-constexpr int kLaneMaxK = 8;
-constexpr size_t kLaneSmemLimit = 227u * 1024u;
+constexpr int kQuadThreads = 768;  // at most; see quad_cfg
+constexpr int kQuadTok = 8;    // tokens per warp batch
+constexpr int kQuadCap = 16;   // candidates per token ranked at once
+constexpr int kQuadMaxE = 128;
+constexpr int kQuadMaxK = 8;
+constexpr size_t kQuadSmemLimit = 227u * 1024u;
 
-// Byte offsets of the lane kernel's shared memory.
-struct LaneSmem {
-    int stride;  // words per staged row
-    size_t bars, wcnt, emask, gst, wsum, total;
+// Byte offsets of the quad kernel's shared memory.  Phase 3 reuses the staged
+// rows' area for buf .. call.
+struct QuadSmem {
+    size_t cand, sval, sidx, msk, woff, gst, wsum, total;
+    size_t buf, ebuf, run, ccnt, pre, tot, call;
 };
 
-__host__ __device__ inline LaneSmem lane_smem_layout(int E, int warps, int stages) {
-    LaneSmem L;
-    L.stride = E + 4;
-    L.bars = static_cast<size_t>(warps) * stages * 32 * L.stride * 4;  // staged rows first
-    L.wcnt = L.bars + static_cast<size_t>(warps) * stages * 8;        // [warps][stages] mbarriers
-    L.emask = L.wcnt + static_cast<size_t>(warps) * E * 4;            // [warps][E] counts, then bases
-    L.gst = L.emask + static_cast<size_t>(warps) * E * 4;             // [warps][E] lane masks
-    L.wsum = L.gst + static_cast<size_t>(E + 1) * 4;                  // [E + 1] group starts
-    L.total = L.wsum + static_cast<size_t>(warps) * 4;                // [warps] scan scratch
+__host__ __device__ inline QuadSmem quad_smem_layout(int E, int warps) {
+    QuadSmem L;
+    const size_t rows = static_cast<size_t>(warps) * kQuadTok, threads = static_cast<size_t>(warps) * 32;
+    const size_t parts = threads / static_cast<size_t>(E);
+    size_t p3 = 0;
+    L.buf = p3;                                  // [threads * kQuadMaxK] pair of each chunk-sorted slot
+    p3 += threads * kQuadMaxK * 4;
+    L.ebuf = p3;                                 // [threads * kQuadMaxK] its expert (16 bit)
+    p3 += threads * kQuadMaxK * 2;
+    L.run = p3;                                  // [E] next sorted position of each expert
+    p3 += static_cast<size_t>(E) * 4;
+    L.ccnt = p3;                                 // [E] the chunk's pairs per expert
+    p3 += static_cast<size_t>(E) * 4;
+    L.pre = p3;                                  // [parts][E] partial sums over earlier blocks
+    p3 += parts * E * 4;
+    L.tot = p3;                                  // [parts][E] partial sums over all blocks
+    p3 += parts * E * 4;
+    L.call = p3;                                 // [E] expert totals, then position offsets
+    p3 += static_cast<size_t>(E) * 4;
+    const size_t staged = rows * E * 4;          // phase 1: [warps][8][E] logits (candidates' values)
+    L.cand = staged > p3 ? staged : p3;          // [warps][8][kQuadCap] candidate keys
+    L.sval = L.cand + rows * kQuadCap * 8;       // [warps][8][kQuadMaxK] order keys by slot
+    L.sidx = L.sval + rows * kQuadMaxK * 4;      // [warps][8][kQuadMaxK] experts by slot
+    // [E][warps + 1]: the row stride warps + 1 puts both a warp's lanes (random
+    // experts) and an expert's warps (one per lane) on distinct banks
+    L.msk = L.sidx + rows * kQuadMaxK * 4;                          // lane masks
+    L.woff = L.msk + static_cast<size_t>(E) * (warps + 1) * 4;      // phase 1 counts, phase 3 first ranks
+    L.gst = L.woff + static_cast<size_t>(E) * (warps + 1) * 4;      // [E + 1] padded group starts
+    L.wsum = L.gst + static_cast<size_t>(E + 4) * 4;          // [33] scan scratch
+    L.total = L.wsum + 68 * 4;
     return L;
 }
 
@@ -570,313 +604,492 @@ __device__ __forceinline__ uint32_t order_key(float v) {
     return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
 }
 
-// The k-th largest of g[0 .. NGM*K): the minimum when NGM == 1; for NGM == 2
-// each half is sorted (descending, odd-even transposition) and the k-th
-// largest of two sorted lists A, B is max over i of min(A_i, B_(k-i)), A_i the
-// i-th largest of A and A_0 = +inf.
-template <int K, int NGM>
-__device__ __forceinline__ float kth_largest(float (&g)[NGM * K]) {
-    if constexpr (NGM == 1) {
-        float t = g[0];
+__device__ __forceinline__ void cas_desc(float &a, float &b) {
+    const float hi = fmaxf(a, b), lo = fminf(a, b);
+    a = hi;
+    b = lo;
+}
+
+// Sorts g descending with Batcher's odd-even merge sort (the network of the
+// next power of two, comparators beyond N dropped).
+template <int N>
+__device__ __forceinline__ void sort_desc(float (&g)[N]) {
+    constexpr int P = N <= 1 ? 1 : N <= 2 ? 2 : N <= 4 ? 4 : 8;
+    static_assert(N <= 8, "up to 8 keys");
 #pragma unroll
-        for (int j = 1; j < K; ++j) t = fminf(t, g[j]);
-        return t;
-    } else {
+    for (int p = 1; p < P; p <<= 1) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int k = p; k >= 1; k >>= 1) {
 #pragma unroll
-            for (int r = 0; r < K; ++r) {
+            for (int j = k % p; j + k < P; j += 2 * k) {
 #pragma unroll
-                for (int i = h * K + (r & 1); i + 1 < (h + 1) * K; i += 2) {
-                    const float hi = fmaxf(g[i], g[i + 1]), lo = fminf(g[i], g[i + 1]);
-                    g[i] = hi;
-                    g[i + 1] = lo;
+                for (int i = 0; i < k; ++i) {
+                    if (i + j + k < N && (i + j) / (2 * p) == (i + j + k) / (2 * p)) cas_desc(g[i + j], g[i + j + k]);
                 }
             }
         }
-        float t = fmaxf(g[K - 1], g[2 * K - 1]);
-#pragma unroll
-        for (int i = 1; i < K; ++i) t = fmaxf(t, fminf(g[i - 1], g[2 * K - 1 - i]));
-        return t;
     }
 }
 
-template <int K, int NGM>
-__global__ void __launch_bounds__(kLaneMaxWarps * 32, 1) route_lane_kernel(const RouteFusedArgs a) {
+// Sorts a bitonic sequence descending (N a power of two), else any sequence.
+template <int N>
+__device__ __forceinline__ void sort_bitonic_desc(float (&c)[N]) {
+    if constexpr ((N & (N - 1)) == 0) {
+#pragma unroll
+        for (int s = N / 2; s >= 1; s >>= 1) {
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                if ((j & s) == 0) cas_desc(c[j], c[j + s]);
+            }
+        }
+    } else {
+        sort_desc<N>(c);
+    }
+}
+
+__device__ __forceinline__ uint64_t cand_key(float v, int e) {
+    return (static_cast<uint64_t>(order_key(v)) << 32) | static_cast<uint32_t>(~e);
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+    }
+    return v;
+}
+
+// Exclusive scans of two ints per thread over the block: warp scans, then
+// warp 0 scans the warps' totals.  tot gets the block totals; wsum holds 66
+// ints.
+__device__ __forceinline__ void block_scan2(int v0, int v1, int &x0, int &x1, int &tot0, int &tot1, int *wsum) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = static_cast<int>(blockDim.x >> 5);
+    const int i0 = warp_incl_scan(v0), i1 = warp_incl_scan(v1);
+    __syncthreads();  // wsum free from any earlier use
+    if (lane == 31) {
+        wsum[warp] = i0;
+        wsum[33 + warp] = i1;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int s0 = lane < nw ? wsum[lane] : 0, s1 = lane < nw ? wsum[33 + lane] : 0;
+        const int si0 = warp_incl_scan(s0), si1 = warp_incl_scan(s1);
+        if (lane < nw) {
+            wsum[lane] = si0 - s0;
+            wsum[33 + lane] = si1 - s1;
+        }
+        if (lane == 31) {
+            wsum[32] = si0;
+            wsum[65] = si1;
+        }
+    }
+    __syncthreads();
+    x0 = wsum[warp] + i0 - v0;
+    x1 = wsum[33 + warp] + i1 - v1;
+    tot0 = wsum[32];
+    tot1 = wsum[65];
+}
+
+template <int K, int NV>
+__global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const RouteFusedArgs a) {
     extern __shared__ __align__(16) uint8_t sm_b[];
-    constexpr int NG = NGM * K;
-    const int E = a.E, G = gridDim.x, b = blockIdx.x, S = a.lane_stages;
+    constexpr int SPL = (K + 3) / 4;  // slots per lane
+    constexpr unsigned kFull = 0xffffffffu;
+    const int E = a.E, E4 = E / 4, G = gridDim.x, b = blockIdx.x;
     const int nw = static_cast<int>(blockDim.x >> 5);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const LaneSmem L = lane_smem_layout(E, nw, S);
-    const int stride = L.stride;
-    const float *stage = reinterpret_cast<const float *>(sm_b) + static_cast<size_t>(warp) * S * 32 * stride;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_b + L.bars) + warp * S;
-    int *wcnt = reinterpret_cast<int *>(sm_b + L.wcnt);
-    uint32_t *emask = reinterpret_cast<uint32_t *>(sm_b + L.emask);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tq = lane >> 2, q = lane & 3;
+    const QuadSmem L = quad_smem_layout(E, nw);
+    const int row = warp * kQuadTok + tq;
+    float *srow = reinterpret_cast<float *>(sm_b) + static_cast<size_t>(row) * E;
+    uint64_t *cand = reinterpret_cast<uint64_t *>(sm_b + L.cand) + row * kQuadCap;
+    uint32_t *sval = reinterpret_cast<uint32_t *>(sm_b + L.sval) + row * kQuadMaxK;
+    int *sidx = reinterpret_cast<int *>(sm_b + L.sidx) + row * kQuadMaxK;
+    const int ws = nw + 1;  // row stride of wcnt, msk and woff
+    int *wcnt = reinterpret_cast<int *>(sm_b + L.woff);  // phase 1: [E][ws] per-warp expert counts
     int *gst = reinterpret_cast<int *>(sm_b + L.gst);
-    int *warp_sums = reinterpret_cast<int *>(sm_b + L.wsum);
+    int *wsum = reinterpret_cast<int *>(sm_b + L.wsum);
     const int t0 = static_cast<int>(static_cast<int64_t>(a.T) * b / G);
     const int t1 = static_cast<int>(static_cast<int64_t>(a.T) * (b + 1) / G);
     const int nb = t1 - t0;
     const int wt0 = t0 + nb * warp / nw, wt1 = t0 + nb * (warp + 1) / nw;
-    const int nbatch = (wt1 - wt0 + 31) / 32;
-    const bool vec_k = (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.idx) | reinterpret_cast<uintptr_t>(a.w)) & 15u) == 0;
-    for (int i = threadIdx.x; i < nw * E; i += blockDim.x) {
-        wcnt[i] = 0;
-        emask[i] = 0u;
-    }
-    if (lane == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
-        fence_barrier_init();
-    }
+    for (int i = threadIdx.x; i < E * ws; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
 
-    // Batch `it` of this warp (32 rows from token wt0 + 32*it) into ring slot it % S.
-    auto issue = [&](int it) {
-        const int tb = wt0 + 32 * it, rows = min(32, wt1 - tb), s = it % S;
-        fence_proxy_async_smem();  // this lane's earlier reads of the slot come first
-        __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(&bar[s], static_cast<uint32_t>(rows * E) * 4u);
-        __syncwarp();
-        if (lane < rows)
-            bulk_load(const_cast<float *>(stage) + static_cast<size_t>(s * 32 + lane) * stride,
-                      a.logits + static_cast<size_t>(tb + lane) * E, static_cast<uint32_t>(E) * 4u, &bar[s]);
-    };
-
-    // ---- phase 1: top-k, one token per lane ----
-    const int E4 = E / 4, gq = E / (4 * NG);  // float4s per row, per group
-    bool wait_ok = true;
-    int it = 0;
-    for (int p = 0; p < S && p < nbatch; ++p) issue(p);
-    for (; it < nbatch; ++it) {
-        const int tb = wt0 + 32 * it, rows = min(32, wt1 - tb), s = it % S;
-        const bool arrived = mbar_wait(&bar[s], static_cast<uint32_t>(it / S) & 1u, nullptr);
-        if (!__all_sync(0xffffffffu, arrived)) {
-            wait_ok = false;
-            break;
+    // ---- phase 1: top-k, four lanes per token ----
+    for (int tb = wt0; tb < wt1; tb += kQuadTok) {
+        const int t = tb + tq;
+        const bool live = t < wt1;
+        const float4 *src = reinterpret_cast<const float4 *>(a.logits) + static_cast<size_t>(live ? t : 0) * E4;
+        float4 v[NV];
+        float gm[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            if (live && q + 4 * i < E4) {
+                v[i] = __ldcs(src + q + 4 * i);
+                gm[i] = fmaxf(fmaxf(v[i].x, v[i].y), fmaxf(v[i].z, v[i].w));
+            } else {
+                v[i] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                gm[i] = -INFINITY;
+            }
         }
-        const bool live = lane < rows;
-        const float4 *r4 = reinterpret_cast<const float4 *>(stage + static_cast<size_t>(s * 32 + lane) * stride);
-        uint64_t mlo = 0ull, mhi = 0ull;  // logits >= tau: experts 0..63, 64..127
-        int ncand = 0;
+        // tau: the k-th largest piece maximum of the token's four lanes
+        sort_desc<NV>(gm);
+        float lst[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) lst[j] = j < NV ? gm[j] : -INFINITY;
+        float mrg[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) mrg[j] = fmaxf(lst[j], __shfl_xor_sync(kFull, lst[K - 1 - j], 1));
+        sort_bitonic_desc<K>(mrg);
+        float tau = INFINITY;
+#pragma unroll
+        for (int j = 0; j < K; ++j) tau = fminf(tau, fmaxf(mrg[j], __shfl_xor_sync(kFull, mrg[K - 1 - j], 2)));
+        // candidates: bit 4i + c of m is component c of piece q + 4i
+        uint32_t m = 0u;
         if (live) {
-            float gm[NG];
 #pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                float mx = -INFINITY;
+            for (int i = 0; i < NV; ++i) {
+                if (q + 4 * i >= E4) continue;
+                uint32_t bits = 0u;
+                if (v[i].x >= tau) bits |= 1u;
+                if (v[i].y >= tau) bits |= 2u;
+                if (v[i].z >= tau) bits |= 4u;
+                if (v[i].w >= tau) bits |= 8u;
+                m |= bits << (4 * i);
+                if (bits != 0u) reinterpret_cast<float4 *>(srow)[q + 4 * i] = v[i];
+            }
+        }
+        const int nc = __popc(m);
+        int incl = nc;
+        {
+            const int u1 = __shfl_up_sync(kFull, incl, 1, 4);
+            if (q >= 1) incl += u1;
+            const int u2 = __shfl_up_sync(kFull, incl, 2, 4);
+            if (q >= 2) incl += u2;
+        }
+        const int ncand = __shfl_sync(kFull, incl, 3, 4);
+        const bool ranked = live && ncand <= kQuadCap;
+        if (ranked) {
+            int pos = incl - nc;
+            for (uint32_t mm = m; mm != 0u; mm &= mm - 1u) {
+                const int bit = __ffs(static_cast<int>(mm)) - 1;
+                const int e = 16 * (bit >> 2) + 4 * q + (bit & 3);
+                cand[pos++] = cand_key(srow[e], e);
+            }
+        }
+        __syncwarp();
+        if (ranked) {
+            uint64_t own[4];
+            int rk[4];
 #pragma unroll
-                for (int q = 0; q < 32 / NG; ++q) {
-                    if (q < gq) {
-                        const float4 v = r4[g * gq + q];
-                        mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+            for (int u = 0; u < 4; ++u) {
+                own[u] = q + 4 * u < ncand ? cand[q + 4 * u] : ~0ull;
+                rk[u] = 0;
+            }
+            for (int j = 0; j < ncand; ++j) {
+                const uint64_t kj = cand[j];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) rk[u] += kj > own[u] ? 1 : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (q + 4 * u < ncand && rk[u] < K) {
+                    sval[rk[u]] = static_cast<uint32_t>(own[u] >> 32);
+                    sidx[rk[u]] = static_cast<int>(~static_cast<uint32_t>(own[u]));
+                }
+            }
+        }
+        if (__any_sync(kFull, live && !ranked)) {
+            // many ties: the k largest one per round
+            const bool mine = live && !ranked;
+            uint32_t rem = mine ? m : 0u;
+#pragma unroll 1
+            for (int s = 0; s < K; ++s) {
+                uint64_t best = 0ull;
+                for (uint32_t mm = rem; mm != 0u; mm &= mm - 1u) {
+                    const int bit = __ffs(static_cast<int>(mm)) - 1;
+                    const int e = 16 * (bit >> 2) + 4 * q + (bit & 3);
+                    const uint64_t key = cand_key(srow[e], e);
+                    best = key > best ? key : best;
+                }
+                uint64_t o = __shfl_xor_sync(kFull, best, 1);
+                best = o > best ? o : best;
+                o = __shfl_xor_sync(kFull, best, 2);
+                best = o > best ? o : best;
+                const int e = static_cast<int>(~static_cast<uint32_t>(best));
+                if (mine) {
+                    if (((e >> 2) & 3) == q) rem &= ~(1u << (4 * (e >> 4) + (e & 3)));
+                    if (q == 0) {
+                        sval[s] = static_cast<uint32_t>(best >> 32);
+                        sidx[s] = e;
                     }
                 }
-                gm[g] = mx;
-            }
-            const float tau = kth_largest<K, NGM>(gm);
-            uint32_t m[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (8 * wd + j < E4) {
-                        const float4 v = r4[8 * wd + j];
-                        uint32_t bits = 0u;
-                        if (v.x >= tau) bits |= 1u << (4 * j);
-                        if (v.y >= tau) bits |= 2u << (4 * j);
-                        if (v.z >= tau) bits |= 4u << (4 * j);
-                        if (v.w >= tau) bits |= 8u << (4 * j);
-                        m[wd] |= bits;
-                    }
-                }
-            }
-            mlo = (static_cast<uint64_t>(m[1]) << 32) | m[0];
-            mhi = (static_cast<uint64_t>(m[3]) << 32) | m[2];
-            ncand = __popcll(mlo) + __popcll(mhi);
-        }
-        uint32_t tk[K];
-        int ti[K];
-#pragma unroll
-        for (int j = 0; j < K; ++j) {
-            tk[j] = 0u;  // below every real key
-            ti[j] = 0;
-        }
-        const float *row = reinterpret_cast<const float *>(r4);
-        const int cmax = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(ncand)));
-        for (int c = 0; c < cmax; ++c) {
-            if (c < ncand) {
-                const bool in_lo = mlo != 0ull;
-                const uint64_t cur = in_lo ? mlo : mhi;
-                const int e = __ffsll(static_cast<long long>(cur)) - 1 + (in_lo ? 0 : 64);
-                const uint64_t rest = cur & (cur - 1ull);
-                if (in_lo)
-                    mlo = rest;
-                else
-                    mhi = rest;
-                const uint32_t xk = order_key(row[e]);
-                bool gt[K];
-#pragma unroll
-                for (int j = 0; j < K; ++j) gt[j] = xk > tk[j];
-#pragma unroll
-                for (int j = K - 1; j > 0; --j) {
-                    tk[j] = gt[j - 1] ? tk[j - 1] : (gt[j] ? xk : tk[j]);
-                    ti[j] = gt[j - 1] ? ti[j - 1] : (gt[j] ? e : ti[j]);
-                }
-                tk[0] = gt[0] ? xk : tk[0];
-                ti[0] = gt[0] ? e : ti[0];
             }
         }
+        __syncwarp();
         if (live) {
-            const int t = tb + lane;
-            const float mx = topk_value(tk[0]);
-            float p[K], sum = 0.f;
+            const float mx = topk_value(sval[0]);
+            float sum = 0.f;
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-                p[j] = expf(topk_value(tk[j]) - mx);
-                sum += p[j];  // slot order
+            for (int j = 0; j < K; ++j) sum += expf(topk_value(sval[j]) - mx);  // slot order
+            int ej[SPL];
+            float wj[SPL];
+#pragma unroll
+            for (int u = 0; u < SPL; ++u) {
+                const int j = q * SPL + u;
+                ej[u] = j < K ? sidx[j] : 0;
+                wj[u] = j < K ? expf(topk_value(sval[j]) - mx) / sum : 0.f;
             }
-            float wv[K];
-#pragma unroll
-            for (int j = 0; j < K; ++j) wv[j] = p[j] / sum;
-            int32_t *irow = a.idx + static_cast<size_t>(t) * K;
-            float *wrow = a.w + static_cast<size_t>(t) * K;
-            if (vec_k) {
-#pragma unroll
-                for (int j = 0; j < K; j += 4) {
-                    *reinterpret_cast<int4 *>(irow + j) = make_int4(ti[j], ti[j + 1], ti[j + 2], ti[j + 3]);
-                    *reinterpret_cast<float4 *>(wrow + j) = make_float4(wv[j], wv[j + 1], wv[j + 2], wv[j + 3]);
+            int32_t *irow = a.idx + static_cast<size_t>(t) * K + q * SPL;
+            float *wrow = a.w + static_cast<size_t>(t) * K + q * SPL;
+            if constexpr (SPL == 2 && K % 2 == 0) {
+                if (q * SPL < K) {
+                    *reinterpret_cast<int2 *>(irow) = make_int2(ej[0], ej[1]);
+                    *reinterpret_cast<float2 *>(wrow) = make_float2(wj[0], wj[1]);
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < K; ++j) {
-                    irow[j] = ti[j];
-                    wrow[j] = wv[j];
+                for (int u = 0; u < SPL; ++u) {
+                    if (q * SPL + u < K) {
+                        irow[u] = ej[u];
+                        wrow[u] = wj[u];
+                    }
                 }
             }
 #pragma unroll
-            for (int j = 0; j < K; ++j) atomicAdd(&wcnt[warp * E + ti[j]], 1);
+            for (int u = 0; u < SPL; ++u)
+                if (q * SPL + u < K) atomicAdd(&wcnt[ej[u] * ws + warp], 1);
         }
         __syncwarp();
-        if (it + S < nbatch) issue(it + S);
-    }
-    if (!wait_ok) {
-        if (lane == 0) report_status(a.status, kStatusTimeout);
-        for (int q = it; q < it + S && q < nbatch; ++q)  // copies still in flight land before the exit
-            (void)mbar_wait(&bar[q % S], static_cast<uint32_t>(q / S) & 1u, nullptr);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int sum = 0;
-        for (int q = 0; q < nw; ++q) sum += wcnt[q * E + e];
-        a.blk_hist[static_cast<size_t>(b) * E + e] = sum;
+    for (int x = threadIdx.x; x < E; x += blockDim.x) {
+        int c = 0;
+        for (int w = 0; w < nw; ++w) c += wcnt[x * ws + w];
+        a.blk_hist[static_cast<size_t>(b) * E + x] = c;
     }
     if (!grid_barrier(a.barrier, G, a.status)) return;
 
-    // ---- phase 2: per expert, exclusive scan over the blocks ----
-    route_scan_experts(a, warp_sums);
-    if (!grid_barrier(a.barrier, 2u * G, a.status)) return;
-
-    // ---- phase 3: group starts, tile table, padding, positions ----
-    if (!route_group_layout(a, gst, warp_sums)) return;
-    route_warp_bases(a, wcnt, gst, nw);
-    if (!wait_ok) return;  // this warp's idx rows are incomplete
-    bool bad = false;
-    const uint32_t below = (1u << lane) - 1u;
-    int *run = wcnt + warp * E;
-    uint32_t *msk = emask + warp * E;
-    for (int tb = wt0; tb < wt1; tb += 32) {
-        const int t = tb + lane;
-        const bool live = t < wt1;
-        int e[K];
-        if (live) {
-            const int32_t *irow = a.idx + static_cast<size_t>(t) * K;  // written by this thread in phase 1
-            if (vec_k) {
+    // ---- phase 2: totals, earlier blocks' sums, group layout ----
+    int *run = reinterpret_cast<int *>(sm_b + L.run);
+    int *ccnt = reinterpret_cast<int *>(sm_b + L.ccnt);
+    int *call = reinterpret_cast<int *>(sm_b + L.call);
+    {
+        int *pre = reinterpret_cast<int *>(sm_b + L.pre);
+        int *tot = reinterpret_cast<int *>(sm_b + L.tot);
+        const int parts = static_cast<int>(blockDim.x) / E;  // >= 1
+        const int x = threadIdx.x % E, p = threadIdx.x / E;
+        if (p < parts) {
+            // all of this thread's loads in flight at once (G <= 40 * parts in one round)
+            int sp = 0, st = 0;
+            for (int b0 = p; b0 < G; b0 += 40 * parts) {
+                int v[40];
 #pragma unroll
-                for (int j = 0; j < K; j += 4) {
-                    const int4 v = *reinterpret_cast<const int4 *>(irow + j);
-                    e[j] = v.x;
-                    e[j + 1] = v.y;
-                    e[j + 2] = v.z;
-                    e[j + 3] = v.w;
+                for (int i = 0; i < 40; ++i) {
+                    const int bb = b0 + i * parts;
+                    v[i] = bb < G ? __ldcg(a.blk_hist + static_cast<size_t>(bb) * E + x) : 0;
                 }
-            } else {
 #pragma unroll
-                for (int j = 0; j < K; ++j) e[j] = irow[j];
+                for (int i = 0; i < 40; ++i) {
+                    st += v[i];
+                    sp += b0 + i * parts < b ? v[i] : 0;
+                }
             }
-#pragma unroll
-            for (int j = 0; j < K; ++j) atomicOr(&msk[e[j]], 1u << lane);
+            pre[p * E + x] = sp;
+            tot[p * E + x] = st;
         }
-        __syncwarp();
+        __syncthreads();
+        int c = 0, before = 0;
+        if (threadIdx.x < E) {
+            for (int pp = 0; pp < parts; ++pp) {
+                c += tot[pp * E + threadIdx.x];
+                before += pre[pp * E + threadIdx.x];
+            }
+        }
+        const int padded = (c + kTileM - 1) / kTileM * kTileM;
+        int c_excl, p_excl, c_tot, p_tot;
+        block_scan2(c, padded, c_excl, p_excl, c_tot, p_tot, wsum);
+        if (threadIdx.x < E) {
+            gst[threadIdx.x] = p_excl;
+            run[threadIdx.x] = p_excl + before;
+            call[threadIdx.x] = c;
+            if (b == 0) {
+                a.counts[threadIdx.x] = c;
+                a.group_start[threadIdx.x] = p_excl;
+                a.offsets[threadIdx.x] = c_excl;
+            }
+        }
+        if (threadIdx.x == 0) {
+            gst[E] = p_tot;
+            if (b == 0) {
+                a.group_start[E] = p_tot;
+                a.offsets[E] = c_tot;
+                if (p_tot > a.p_cap) report_status(a.status, kStatusBadIndex);
+            }
+        }
+        __syncthreads();
+        if (gst[E] > a.p_cap) return;
+        for (int xx = b; xx < E; xx += G) {
+            const int gs = gst[xx], ge = gst[xx + 1], cx = call[xx];
+            for (int mt = gs / kTileM + threadIdx.x; mt < ge / kTileM; mt += blockDim.x) a.tile_expert[mt] = xx;
+            for (int qq = gs + cx + threadIdx.x; qq < ge; qq += blockDim.x) a.perm[qq] = -1;
+        }
+    }
+
+    // ---- phase 3: positions, one chunk of blockDim.x tokens at a time ----
+    uint32_t *msk = reinterpret_cast<uint32_t *>(sm_b + L.msk);
+    int *woff = reinterpret_cast<int *>(sm_b + L.woff);
+    int *buf = reinterpret_cast<int *>(sm_b + L.buf);
+    uint16_t *ebuf = reinterpret_cast<uint16_t *>(sm_b + L.ebuf);
+    int *dlt = call;  // sorted position minus chunk-local slot, per expert
+    const bool vec_k = (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.idx) | reinterpret_cast<uintptr_t>(a.inv)) & 15u) == 0;
+    const uint32_t below = (1u << lane) - 1u;
+    const int xper = (E + nw - 1) / nw, xw0 = warp * xper;  // this warp's experts in the scans
+    // the experts of token t (written in phase 1, before the barrier)
+    auto load_row = [&](int t, int (&e)[K]) {
+        const int32_t *irow = a.idx + static_cast<size_t>(t) * K;
+        if (vec_k) {
+#pragma unroll
+            for (int j = 0; j < K; j += 4) {
+                const int4 v4 = __ldcg(reinterpret_cast<const int4 *>(irow + j));
+                e[j] = v4.x;
+                e[j + 1] = v4.y;
+                e[j + 2] = v4.z;
+                e[j + 3] = v4.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < K; ++j) e[j] = __ldcg(irow + j);
+        }
+    };
+    for (int i = threadIdx.x; i < E * ws; i += blockDim.x) msk[i] = 0u;
+    bool bad = false;
+    int e[K];
+    if (t0 + static_cast<int>(threadIdx.x) < t1) load_row(t0 + static_cast<int>(threadIdx.x), e);
+    __syncthreads();
+    for (int c0 = t0; c0 < t1; c0 += static_cast<int>(blockDim.x)) {
+        const int t = c0 + static_cast<int>(threadIdx.x);
+        const bool live = t < t1;
         if (live) {
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                const int pos = run[e[j]] + __popc(msk[e[j]] & below);
-                const int pair = t * K + j;
-                if (pos >= 0 && pos < gst[e[j] + 1]) {
-                    a.perm[pos] = pair;
-                    a.inv[pair] = pos;
-                } else {
+                if (e[j] < 0 || e[j] >= E) {  // cannot happen for finite logits; keeps the indexing in bounds
+                    e[j] = 0;
                     bad = true;
                 }
+                atomicOr(&msk[e[j] * ws + warp], 1u << lane);
             }
         }
-        __syncwarp();
+        __syncthreads();
+        // the next chunk's rows in flight while this one is placed
+        int en[K] = {};
+        const int tn = t + static_cast<int>(blockDim.x);
+        if (tn < t1) load_row(tn, en);
+        // each of this warp's experts: its pairs per warp, scanned over the warps
+        int wt = 0;
+        for (int x = xw0; x < xw0 + xper && x < E; ++x) {
+            const int cw = lane < nw ? __popc(msk[x * ws + lane]) : 0;
+            const int ci = warp_incl_scan(cw);
+            if (lane < nw) woff[x * ws + lane] = ci - cw;
+            const int cx = __shfl_sync(0xffffffffu, ci, 31);
+            if (lane == 0) ccnt[x] = cx;
+            wt += cx;
+        }
+        if (lane == 0) wsum[warp] = wt;
+        __syncthreads();
+        // chunk-local starts: earlier warps' experts, then this warp's earlier experts
+        {
+            const int v = lane < nw ? wsum[lane] : 0;
+            const int vi = warp_incl_scan(v);
+            int base = __shfl_sync(0xffffffffu, vi - v, warp);
+            for (int x = xw0; x < xw0 + xper && x < E; ++x) {
+                if (lane < nw) woff[x * ws + lane] += base;
+                if (lane == 0) dlt[x] = run[x] - base;
+                base += ccnt[x];
+            }
+        }
+        __syncthreads();
         if (live) {
+            int pos[K];
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                const uint32_t mm = msk[e[j]];
-                if (lane == 31 - __clz(mm)) {  // one lane per expert advances its position
-                    run[e[j]] += __popc(mm);
-                    msk[e[j]] = 0u;
-                }
+                const int x = e[j];
+                const int lp = woff[x * ws + warp] + __popc(msk[x * ws + warp] & below);
+                buf[lp] = t * K + j;
+                ebuf[lp] = static_cast<uint16_t>(x);
+                pos[j] = lp + dlt[x];
+            }
+            int32_t *vrow = a.inv + static_cast<size_t>(t) * K;
+            if (vec_k) {
+#pragma unroll
+                for (int j = 0; j < K; j += 4)
+                    *reinterpret_cast<int4 *>(vrow + j) = make_int4(pos[j], pos[j + 1], pos[j + 2], pos[j + 3]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < K; ++j) vrow[j] = pos[j];
             }
         }
-        __syncwarp();
+        __syncthreads();
+        const int np = min(t1 - c0, static_cast<int>(blockDim.x)) * K;  // the chunk's pairs
+        for (int i = threadIdx.x; i < np; i += blockDim.x) {
+            const int x = ebuf[i];
+            const int p = i + dlt[x];
+            if (p >= 0 && p < gst[x + 1])
+                a.perm[p] = buf[i];
+            else
+                bad = true;
+        }
+        __syncthreads();
+        for (int x = threadIdx.x; x < E; x += blockDim.x) run[x] += ccnt[x];
+        for (int i = threadIdx.x; i < E * ws; i += blockDim.x) msk[i] = 0u;
+#pragma unroll
+        for (int j = 0; j < K; ++j) e[j] = en[j];
+        __syncthreads();
     }
     if (bad) report_status(a.status, kStatusBadIndex);
 }
 
-// Warps and ring depth of the lane kernel, as many warps as fit in shared
-// memory (at least E / 32, since phase 3 gives one expert to each thread).
-// With at most 384 tokens per SM a warp has one or two batches, and a ring of
-// two batches per warp (fewer, fuller warps) finishes first; with more tokens
-// one batch per warp and twice the warps hide more latency (measured at E =
-// 128: 16 K tokens 24.6 against 26.6 us, 512 K tokens 185 against 155 us).
-struct LaneCfg {
-    int warps, stages;
+// Warps of the quad kernel: 16 while an SM has at most 1024 tokens, else 24
+// (measured at E = 128, k = 8 against 16, 24 and 32 warps: 16 K tokens 22.5,
+// 24.5 and 26.6 us; 1 M tokens 266, 231 and 244 us); fewer if shared memory
+// runs out, at least E / 32 (phase 2 gives one expert to each thread).
+struct QuadCfg {
+    int warps;
     size_t smem;
 };
 
-LaneCfg lane_cfg(int E, int T, int sms) {
-    LaneCfg c{kLaneMaxWarps, static_cast<int64_t>(T) <= 384ll * sms ? 2 : 1, 0};
-    while (c.warps > 1 && lane_smem_layout(E, c.warps, c.stages).total > kLaneSmemLimit) --c.warps;
-    c.smem = lane_smem_layout(E, c.warps, c.stages).total;
+QuadCfg quad_cfg(int E, int T, int sms) {
+    QuadCfg c{static_cast<int64_t>(T) <= 1024ll * sms ? 16 : kQuadThreads / 32, 0};
+    while (c.warps > 1 && quad_smem_layout(E, c.warps).total > kQuadSmemLimit) --c.warps;
+    c.smem = quad_smem_layout(E, c.warps).total;
     return c;
 }
 
-bool route_lane_ok(int E, int k, const float *logits) {
-    return E <= kLaneMaxE && k >= 1 && k <= kLaneMaxK && E % (4 * k) == 0 &&
-           (reinterpret_cast<uintptr_t>(logits) & 15u) == 0 && lane_cfg(E, 0, 1).warps * 32 >= E &&
-           lane_cfg(E, 1 << 30, 1).warps * 32 >= E;
+bool route_quad_ok(int E, int k, const float *logits) {
+    return E <= kQuadMaxE && E % 4 == 0 && k >= 1 && k <= kQuadMaxK && E >= 4 * k &&
+           (reinterpret_cast<uintptr_t>(logits) & 15u) == 0 && quad_cfg(E, 0, 1).warps * 32 >= E &&
+           quad_cfg(E, 1 << 30, 1).warps * 32 >= E;
 }
 
-template <int NGM>
-const void *route_lane_fn_k(int k) {
+template <int NV>
+const void *route_quad_fn_k(int k) {
     switch (k) {
-        case 1: return reinterpret_cast<const void *>(route_lane_kernel<1, NGM>);
-        case 2: return reinterpret_cast<const void *>(route_lane_kernel<2, NGM>);
-        case 3: return reinterpret_cast<const void *>(route_lane_kernel<3, NGM>);
-        case 4: return reinterpret_cast<const void *>(route_lane_kernel<4, NGM>);
-        case 5: return reinterpret_cast<const void *>(route_lane_kernel<5, NGM>);
-        case 6: return reinterpret_cast<const void *>(route_lane_kernel<6, NGM>);
-        case 7: return reinterpret_cast<const void *>(route_lane_kernel<7, NGM>);
-        default: return reinterpret_cast<const void *>(route_lane_kernel<8, NGM>);
+        case 1: return reinterpret_cast<const void *>(route_quad_kernel<1, NV>);
+        case 2: return reinterpret_cast<const void *>(route_quad_kernel<2, NV>);
+        case 3: return reinterpret_cast<const void *>(route_quad_kernel<3, NV>);
+        case 4: return reinterpret_cast<const void *>(route_quad_kernel<4, NV>);
+        case 5: return reinterpret_cast<const void *>(route_quad_kernel<5, NV>);
+        case 6: return reinterpret_cast<const void *>(route_quad_kernel<6, NV>);
+        case 7: return reinterpret_cast<const void *>(route_quad_kernel<7, NV>);
+        default: return reinterpret_cast<const void *>(route_quad_kernel<8, NV>);
     }
 }
 
-const void *route_lane_fn(int E, int k) {
-    return E % (8 * k) == 0 ? route_lane_fn_k<2>(k) : route_lane_fn_k<1>(k);
+// NV: 16-byte pieces a lane holds, E/16 rounded up to a power of two.
+const void *route_quad_fn(int E, int k) {
+    return E <= 32 ? route_quad_fn_k<2>(k) : E <= 64 ? route_quad_fn_k<4>(k) : route_quad_fn_k<8>(k);
 }
 
 constexpr int kBwdThreads = 256;
@@ -1102,9 +1315,9 @@ cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t 
 int route_fused_grid(const float *logits, int T, int E, int k, int sms, int n_chunks) {
     int per_sm = 0;
     cudaError_t e;
-    if (route_lane_ok(E, k, logits)) {
-        const void *fn = route_lane_fn(E, k);
-        const LaneCfg c = lane_cfg(E, T, sms);
+    if (route_quad_ok(E, k, logits)) {
+        const void *fn = route_quad_fn(E, k);
+        const QuadCfg c = quad_cfg(E, T, sms);
         e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
         if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, c.warps * 32, c.smem);
     } else {
@@ -1135,12 +1348,11 @@ cudaError_t launch_route_fused(const float *logits, int T, int E, int k, int32_t
                                int32_t *blk_base, int32_t *counts, int32_t *offsets, int32_t *group_start,
                                int32_t *tile_expert, int32_t *perm, int32_t *inv, int64_t p_cap, unsigned *barrier, int *status, int sms, int grid, cudaStream_t s) {
     RouteFusedArgs a{logits, T, E, k, idx, w, blk_hist, blk_base, counts, offsets, group_start,
-                     tile_expert, perm, inv, p_cap, barrier, status, 0};
+                     tile_expert, perm, inv, p_cap, barrier, status};
     void *params[] = {&a};
-    if (route_lane_ok(E, k, logits)) {
-        const LaneCfg c = lane_cfg(E, T, sms);
-        a.lane_stages = c.stages;
-        return cudaLaunchCooperativeKernel(route_lane_fn(E, k), dim3(grid), dim3(c.warps * 32), params, c.smem, s);
+    if (route_quad_ok(E, k, logits)) {
+        const QuadCfg c = quad_cfg(E, T, sms);
+        return cudaLaunchCooperativeKernel(route_quad_fn(E, k), dim3(grid), dim3(c.warps * 32), params, c.smem, s);
     }
     const size_t smem = route_fused_smem(E, k);
     const int nv = (E + 31) / 32;

@@ -1,6 +1,7 @@
 """Routing alone (moe_route) against the oracle, bit-exact, on shapes that
-reach both routing kernels: the lane-per-token form (E <= 128, E a multiple of
-4k, k <= 8; both of its ring depths and both group counts) and the
+reach both routing kernels: the quad form (four lanes per token; E <= 128, E a
+multiple of 4, E >= 4k, k <= 8; 16 and 24 warps, one and several position
+chunks per block, the rank and the one-per-round selections) and the
 warp-per-token form (everything else), with and without tied logits, and on
 token counts that leave ragged per-warp batches."""
 import numpy as np
@@ -14,19 +15,23 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("T,E,k,ties", [
-    (5000, 128, 8, True),    # lane form, the 30B router shape, many exact ties
-    (16384, 128, 8, False),  # lane form at the workload's size
-    (2048, 96, 4, False),    # lane form, E not a power of two
-    (77, 32, 8, True),       # lane form, fewer tokens than one warp batch per warp
-    (50000, 128, 8, False),  # lane form, two-batch ring per warp, both slots used
-    (70000, 128, 8, True),   # lane form, one batch per warp (more than 384 tokens per SM), ties
-    (131072, 128, 8, False), # lane form, one batch per warp, several batches each
-    (3000, 120, 5, True),    # lane form, 2k groups of 12 experts
-    (3000, 64, 8, False),    # lane form, 2k groups of 4 experts
+    (5000, 128, 8, True),    # quad form, the 30B router shape, many exact ties (one per round)
+    (16384, 128, 8, False),  # quad form at the workload's size (16 warps)
+    (2048, 96, 4, False),    # quad form, E not a power of two
+    (77, 32, 8, True),       # quad form, fewer tokens than one batch per warp
+    (50000, 128, 8, False),  # quad form, 16 warps, one position chunk per block
+    (70000, 128, 8, True),   # quad form, ties
+    (131072, 128, 8, False), # quad form, 16 warps, two position chunks per block
+    (200000, 128, 8, True),  # quad form, 24 warps, two position chunks per block, ties
+    (3000, 120, 5, True),    # quad form, 30 pieces per row, odd k
+    (3000, 64, 8, False),    # quad form, E = 8k
+    (777, 20, 3, True),      # quad form, 5 pieces per row
+    (4096, 64, 6, False),    # quad form, k = 6
+    (1000, 8, 2, True),      # quad form, E = 4k
     (3000, 160, 8, False),   # warp form: E > 128
-    (777, 20, 3, True),      # warp form: E not a multiple of 4k
-    (4096, 64, 6, False),    # warp form: 64 is not a multiple of 24
     (300, 512, 16, True),    # warp form: largest E, k > 8
+    (1000, 130, 4, True),    # warp form: E not a multiple of 4
+    (500, 8, 4, True),       # warp form: E < 4k
 ])
 def test_routing_bit_exact(T, E, k, ties):
     g = torch.Generator().manual_seed(T * 31 + E)

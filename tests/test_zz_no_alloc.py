@@ -8,8 +8,8 @@ workspace.  This test checks, through the C ABI, that two calls in a row give
 the same routing state as the ordinary workspace-based moe_route, and that
 shapes beyond the fixed scratch are refused.  The comparison is bit for bit
 on every routing field, weights included, for both forms of moe_route's
-kernel (one token per lane; one token per warp for E > 128 or E not a multiple
-of 4k), and the routing is also checked once against the oracle's route and
+kernel (four lanes per token; one token per warp for E > 128, E not a multiple
+of 4 or E < 4k), and the routing is also checked once against the oracle's route and
 dispatch.  It sits in a file of its own that pytest collects last.
 """
 import ctypes
@@ -42,10 +42,11 @@ def _route_both(T, d, E, k, I, seed):
 
 
 @pytest.mark.parametrize("sizes", [
-    dict(T=16384, d=2048, E=128, k=8, I=768),  # one token per lane
-    dict(T=1000, d=256, E=16, k=4, I=128),     # one token per lane
+    dict(T=16384, d=2048, E=128, k=8, I=768),  # four lanes per token
+    dict(T=1000, d=256, E=16, k=4, I=128),     # four lanes per token
+    dict(T=999, d=256, E=128, k=6, I=128),     # four lanes per token, k = 6
     dict(T=1000, d=256, E=256, k=8, I=128),    # one token per warp (E > 128)
-    dict(T=999, d=256, E=128, k=6, I=128),     # one token per warp (E not a multiple of 4k)
+    dict(T=999, d=256, E=130, k=6, I=128),     # one token per warp (E not a multiple of 4)
 ])
 def test_noalloc_routing_matches_workspace_routing_on_two_calls(sizes):
     for call, seed in enumerate((3, 4)):  # two calls in a row reuse the same library scratch
