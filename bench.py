@@ -114,6 +114,7 @@ def routing_sweep(M, IN, dev, stream, peak_gbs, E, k, Ts=(16384, 65536, 262144, 
         for _ in range(3):
             M.route(sh, logits, saved, ws, stream)
         times = []
+        torch.cuda.nvtx.range_push(f"route_sweep_T{T}")  # for profilers: ncu --nvtx --nvtx-include route_sweep_T<T>/
         for _ in range(reps):
             flush.zero_()
             e0.record(stream)
@@ -121,6 +122,7 @@ def routing_sweep(M, IN, dev, stream, peak_gbs, E, k, Ts=(16384, 65536, 262144, 
             e1.record(stream)
             e1.synchronize()
             times.append(e0.elapsed_time(e1))
+        torch.cuda.nvtx.range_pop()
         if M.get_status(ws, stream) != 0:
             raise SystemExit(f"device status {M.get_status(ws, stream)} in the routing sweep (T={T})")
         us = statistics.median(times) * 1e3
