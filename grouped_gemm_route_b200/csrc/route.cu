@@ -946,7 +946,6 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
     int *dlt = call;  // sorted position minus chunk-local slot, per expert
     const bool vec_k = (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.idx) | reinterpret_cast<uintptr_t>(a.inv)) & 15u) == 0;
     const uint32_t below = (1u << lane) - 1u;
-    const int xper = (E + nw - 1) / nw, xw0 = warp * xper;  // this warp's experts in the scans
     // the experts of token t (written in phase 1, before the barrier)
     auto load_row = [&](int t, int (&e)[K]) {
         const int32_t *irow = a.idx + static_cast<size_t>(t) * K;
@@ -987,27 +986,27 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
         int en[K] = {};
         const int tn = t + static_cast<int>(blockDim.x);
         if (tn < t1) load_row(tn, en);
-        // each of this warp's experts: its pairs per warp, scanned over the warps
-        int wt = 0;
-        for (int x = xw0; x < xw0 + xper && x < E; ++x) {
-            const int cw = lane < nw ? __popc(msk[x * ws + lane]) : 0;
-            const int ci = warp_incl_scan(cw);
-            if (lane < nw) woff[x * ws + lane] = ci - cw;
-            const int cx = __shfl_sync(0xffffffffu, ci, 31);
-            if (lane == 0) ccnt[x] = cx;
-            wt += cx;
+        // expert x (thread x): its pairs per warp, counted and scanned over the warps;
+        // then the chunk-local starts, an exclusive scan over the experts
+        int xt = 0;
+        if (static_cast<int>(threadIdx.x) < E) {
+            const uint32_t *mx = msk + threadIdx.x * ws;
+            for (int w = 0; w < nw; ++w) xt += __popc(mx[w]);
         }
-        if (lane == 0) wsum[warp] = wt;
+        const int xi = warp_incl_scan(xt);  // warps 0 .. E/32 - 1 hold the experts
+        if (lane == 31 && warp < (E + 31) / 32) wsum[warp] = xi;
         __syncthreads();
-        // chunk-local starts: earlier warps' experts, then this warp's earlier experts
-        {
-            const int v = lane < nw ? wsum[lane] : 0;
-            const int vi = warp_incl_scan(v);
-            int base = __shfl_sync(0xffffffffu, vi - v, warp);
-            for (int x = xw0; x < xw0 + xper && x < E; ++x) {
-                if (lane < nw) woff[x * ws + lane] += base;
-                if (lane == 0) dlt[x] = run[x] - base;
-                base += ccnt[x];
+        if (static_cast<int>(threadIdx.x) < E) {
+            const int x = threadIdx.x;
+            int base = xi - xt;
+            for (int w = 0; w < warp; ++w) base += wsum[w];
+            ccnt[x] = xt;
+            dlt[x] = run[x] - base;
+            const uint32_t *mx = msk + x * ws;
+            int *wo = woff + x * ws;
+            for (int w = 0; w < nw; ++w) {
+                wo[w] = base;
+                base += __popc(mx[w]);
             }
         }
         __syncthreads();
