@@ -547,10 +547,11 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
 // starts (block 0 publishes counts, offsets and group starts), the tile table
 // and padding rows of experts b, b+G, ...
 // Phase 3: the block's tokens in chunks of one token per thread.  A pair's
-// rank within its expert in the chunk comes from per-warp lane masks and a
-// scan over the warps; the chunk's pairs are counting-sorted by expert in
-// shared memory and written to perm one expert's run at a time (an expert's
-// pairs of one chunk are consecutive in perm), so the stores are coalesced.
+// rank within its expert in the chunk comes from per-warp lane masks, counted
+// and scanned over the warps by one thread per expert; the chunk's pairs are
+// counting-sorted by expert in shared memory (pair and sorted position side
+// by side) and written to perm one expert's run at a time (an expert's pairs
+// of one chunk are consecutive in perm), so the stores are coalesced.
 // ---------------------------------------------------------------------------
 constexpr int kQuadThreads = 768;  // at most; see quad_cfg
 constexpr int kQuadTok = 8;    // tokens per warp batch
@@ -563,7 +564,7 @@ constexpr size_t kQuadSmemLimit = 227u * 1024u;
 // rows' area for buf .. call.
 struct QuadSmem {
     size_t cand, sval, sidx, msk, woff, gst, wsum, total;
-    size_t buf, ebuf, run, ccnt, pre, tot, call;
+    size_t buf, gbuf, run, ccnt, pre, tot, call;
 };
 
 __host__ __device__ inline QuadSmem quad_smem_layout(int E, int warps) {
@@ -573,8 +574,8 @@ __host__ __device__ inline QuadSmem quad_smem_layout(int E, int warps) {
     size_t p3 = 0;
     L.buf = p3;                                  // [threads * kQuadMaxK] pair of each chunk-sorted slot
     p3 += threads * kQuadMaxK * 4;
-    L.ebuf = p3;                                 // [threads * kQuadMaxK] its expert (16 bit)
-    p3 += threads * kQuadMaxK * 2;
+    L.gbuf = p3;                                 // [threads * kQuadMaxK] its sorted position
+    p3 += threads * kQuadMaxK * 4;
     L.run = p3;                                  // [E] next sorted position of each expert
     p3 += static_cast<size_t>(E) * 4;
     L.ccnt = p3;                                 // [E] the chunk's pairs per expert
@@ -942,7 +943,7 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
     uint32_t *msk = reinterpret_cast<uint32_t *>(sm_b + L.msk);
     int *woff = reinterpret_cast<int *>(sm_b + L.woff);
     int *buf = reinterpret_cast<int *>(sm_b + L.buf);
-    uint16_t *ebuf = reinterpret_cast<uint16_t *>(sm_b + L.ebuf);
+    int *gbuf = reinterpret_cast<int *>(sm_b + L.gbuf);
     int *dlt = call;  // sorted position minus chunk-local slot, per expert
     const bool vec_k = (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.idx) | reinterpret_cast<uintptr_t>(a.inv)) & 15u) == 0;
     const uint32_t below = (1u << lane) - 1u;
@@ -1016,9 +1017,9 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
             for (int j = 0; j < K; ++j) {
                 const int x = e[j];
                 const int lp = woff[x * ws + warp] + __popc(msk[x * ws + warp] & below);
-                buf[lp] = t * K + j;
-                ebuf[lp] = static_cast<uint16_t>(x);
                 pos[j] = lp + dlt[x];
+                buf[lp] = t * K + j;
+                gbuf[lp] = pos[j];
             }
             int32_t *vrow = a.inv + static_cast<size_t>(t) * K;
             if (vec_k) {
@@ -1032,10 +1033,10 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
         }
         __syncthreads();
         const int np = min(t1 - c0, static_cast<int>(blockDim.x)) * K;  // the chunk's pairs
+        const int prows = gst[E];
         for (int i = threadIdx.x; i < np; i += blockDim.x) {
-            const int x = ebuf[i];
-            const int p = i + dlt[x];
-            if (p >= 0 && p < gst[x + 1])
+            const int p = gbuf[i];  // consecutive i of one expert: consecutive p
+            if (p >= 0 && p < prows)
                 a.perm[p] = buf[i];
             else
                 bad = true;
