@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="skip sampling nvidia-smi during the timed region")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-recompute", action="store_true", help="skip the recompute-mode timing")
     ap.add_argument("--no-routing-sweep", action="store_true",
                     help="skip the routing-only timing over token counts")
@@ -609,7 +609,8 @@ def main():
         bo = sum(t.numel() * t.element_size() for t in (hout[0], hdx[0], hds[0]))
         e2e = {"value": job_tflops(flops_step, world, e_ms / args.e2e_steps), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": args.e2e_steps,
-               "overlap": "copies of step i+1 / i-1 overlap compute of step i (two layer buffers)",
+               "overlap": "copies of step i+1 / i-1 overlap compute of step i (two layer buffers); the first "
+                          "step's inputs and the last step's results cross the bus with nothing to overlap",
                "note": "the step's result read back is out, dx and dscore; dW_gate_up and dW_down stay on the "
                        "device, as in a training loop whose optimizer runs on the GPU"}
         del layers
