@@ -318,6 +318,41 @@ def timed_loop(step, n_steps, stream, dev, barrier):
     return t0.elapsed_time(t1) / n_steps
 
 
+def graph_loop(step_on, n_steps, dev, barrier):
+    """The step captured once in a CUDA graph on a side stream (after an eager
+    warm-up there) and replayed n_steps times: ms per step from CUDA events on
+    that stream, or the reason the capture failed."""
+    import torch
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    try:
+        with torch.cuda.stream(s):
+            step_on(s)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            step_on(s)
+        with torch.cuda.stream(s):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+    except Exception as exc:  # noqa: BLE001 -- reported, not hidden
+        torch.cuda.synchronize(dev)
+        return None, f"{type(exc).__name__}: {exc}"[:200]
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        t0.record(s)
+        for _ in range(n_steps):
+            graph.replay()
+        t1.record(s)
+    torch.cuda.synchronize(dev)
+    barrier()
+    del graph
+    return t0.elapsed_time(t1) / n_steps, None
+
+
 def profiled_loop(M, step, n_steps, stream, dev, barrier):
     """The same steps with the library's per-kernel events on: returns
     {kernel: (total ms, launches)} and the loop's ms per step."""
@@ -390,6 +425,8 @@ def time_other_config(M, IN, name, n_steps, n_warmup, dev, stream, barrier, peak
     ms = timed_loop(step, n_steps, stream, dev, barrier)
     clk = clocks.stop() if clk_gpu is not None else None
     per_kernel, _ = profiled_loop(M, step, n_steps, stream, dev, barrier)
+    g_ms, g_err = graph_loop(lambda s: (layer.forward(x, lg, wgu, wd, s), layer.backward(gout, x, wgu, wd, True, s)),
+                             n_steps, dev, barrier)
     status = layer.status(stream)
     if status != 0:
         raise SystemExit(f"device status {status} in workload {name}")
@@ -403,7 +440,8 @@ def time_other_config(M, IN, name, n_steps, n_warmup, dev, stream, barrier, peak
            "gemm_only_frac": (flops / (gemm_ms * 1e-3) / 1e12) / peak if gemm_ms else None,
            "gemm_ms_per_step": gemm_ms, "peak": peak, "peak_source": note, "clocks": clk,
            "config": workload_config(name, cfg), "dtype": "mxfp8 (e4m3, ue8m0/32)" if mx else "bf16",
-           "kernels": {n: v["ms_per_step"] for n, v in kernel_breakdown(per_kernel, n_steps).items()}}
+           "kernels": {n: v["ms_per_step"] for n, v in kernel_breakdown(per_kernel, n_steps).items()},
+           "graph": ({"ms_per_step": g_ms, "value": flops / (g_ms * 1e-3) / 1e12} if g_ms else {"unavailable": g_err})}
     if "zipf_s" in cfg:
         counts = layer.saved["counts"].cpu()
         out["routing_skew"] = {"max_count": int(counts.max()), "empty_experts": int((counts == 0).sum())}
@@ -482,6 +520,20 @@ def main():
     per_kernel, prof_ms = profiled_loop(M, step, args.steps, stream, dev, barrier)
     if layer.status(stream) != 0:
         raise SystemExit("device status error in the profiled loop")
+
+    # ---- the same step captured once in a CUDA graph and replayed ----
+    g_ms, g_err = graph_loop(lambda s: (layer.forward(x, lg, wgu, wd, s), layer.backward(gout, x, wgu, wd, True, s)),
+                             args.steps, dev, barrier)
+    if layer.status(stream) != 0:
+        raise SystemExit("device status error in the graph replays")
+    g_fail = max_over_ranks(0.0 if g_ms is not None else 1.0, pg, dev)  # every rank takes both collectives
+    g_ms = max_over_ranks(g_ms if g_ms is not None else 0.0, pg, dev)
+    if g_fail == 0.0:
+        graph = {"ms_per_step": g_ms, "value": job_tflops(flops_step, world, g_ms), "unit": UNIT,
+                 "note": "forward + backward captured once in a CUDA graph (routing's cooperative launch, "
+                         "the persistent GEMMs, the second stream of the dx sum) and replayed; same work"}
+    else:
+        graph = {"unavailable": g_err or "the capture failed on another rank"}
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
@@ -646,7 +698,7 @@ def main():
         "frac_of_peak": {"step": value / world / peak, "gemm_only": (flops_step / (gemm_ms * 1e-3) / 1e12) / peak
                               if gemm_ms else None, "peak": peak, "peak_source": roofline["peak_source"]},
         "roofline": roofline, "routing": routing, "kernels": breakdown, "gpu_launches": launches,
-        "clocks": clk, "e2e": e2e, "recompute": recompute, "cpu_baseline": cpu,
+        "clocks": clk, "e2e": e2e, "graph": graph, "recompute": recompute, "cpu_baseline": cpu,
         "timing": "value and ms_per_step from a loop without per-kernel events; kernels and roofline from a "
                   f"second loop of the same steps with them ({prof_ms:.4f} ms per step there)",
         "configs": others,
