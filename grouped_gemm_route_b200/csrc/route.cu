@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
             }
         }
         // weights: exp(l_j - l_max) over the chosen k, normalised by their sum
-        // taken in slot order (the same sum, bit for bit, as the lane form's)
+        // taken in slot order (the same sum, bit for bit, as the quad form's)
 #pragma unroll
         for (int u = 0; u < kTokPar; ++u) {
             const int tt = t + u;
