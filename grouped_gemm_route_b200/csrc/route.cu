@@ -539,8 +539,10 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(const RouteF
 //     first on ties).  A token with more than kQuadCap candidates (many exact
 //     ties) takes its k largest one per round instead: the four lanes compare
 //     their best remaining keys and the winner leaves.
-//   * Weights as in route_fused_kernel, the sum taken in slot order.  The
-//     block's expert histogram goes to blk_hist[b].
+//   * Weights as in route_fused_kernel, the sum taken in slot order: each
+//     lane computes its own slots' numerators and reads the others' back from
+//     the token's slot array.  The block's expert histogram goes to
+//     blk_hist[b].
 // Grid barrier.
 // Phase 2, in every block: each expert's total over all blocks and its sum
 // over the blocks before b (all G histograms read from L2), the padded group
@@ -781,6 +783,9 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
             }
         }
         __syncwarp();
+        // ranks; a warp whose tokens all have at most 12 candidates skips the
+        // fourth owned candidate's compares
+        const bool few = __all_sync(kFull, !ranked || ncand <= 12);
         if (ranked) {
             uint64_t own[4];
             int rk[4];
@@ -789,10 +794,18 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
                 own[u] = q + 4 * u < ncand ? cand[q + 4 * u] : ~0ull;
                 rk[u] = 0;
             }
-            for (int j = 0; j < ncand; ++j) {
-                const uint64_t kj = cand[j];
+            if (few) {
+                for (int j = 0; j < ncand; ++j) {
+                    const uint64_t kj = cand[j];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) rk[u] += kj > own[u] ? 1 : 0;
+                    for (int u = 0; u < 3; ++u) rk[u] += kj > own[u] ? 1 : 0;
+                }
+            } else {
+                for (int j = 0; j < ncand; ++j) {
+                    const uint64_t kj = cand[j];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) rk[u] += kj > own[u] ? 1 : 0;
+                }
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -830,19 +843,33 @@ __global__ void __launch_bounds__(kQuadThreads, 1) route_quad_kernel(const Route
             }
         }
         __syncwarp();
+        // weights: each lane the numerators of its own slots, published in the
+        // token's slot array so that every lane adds all k in slot order
+        int ej[SPL];
+        float pj[SPL];
         if (live) {
             const float mx = topk_value(sval[0]);
-            float sum = 0.f;
-#pragma unroll
-            for (int j = 0; j < K; ++j) sum += expf(topk_value(sval[j]) - mx);  // slot order
-            int ej[SPL];
-            float wj[SPL];
 #pragma unroll
             for (int u = 0; u < SPL; ++u) {
                 const int j = q * SPL + u;
                 ej[u] = j < K ? sidx[j] : 0;
-                wj[u] = j < K ? expf(topk_value(sval[j]) - mx) / sum : 0.f;
+                pj[u] = j < K ? expf(topk_value(sval[j]) - mx) : 0.f;
             }
+        }
+        __syncwarp();
+        if (live) {
+#pragma unroll
+            for (int u = 0; u < SPL; ++u)
+                if (q * SPL + u < K) reinterpret_cast<float *>(sval)[q * SPL + u] = pj[u];
+        }
+        __syncwarp();
+        if (live) {
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < K; ++j) sum += reinterpret_cast<const float *>(sval)[j];  // slot order
+            float wj[SPL];
+#pragma unroll
+            for (int u = 0; u < SPL; ++u) wj[u] = pj[u] / sum;
             int32_t *irow = a.idx + static_cast<size_t>(t) * K + q * SPL;
             float *wrow = a.w + static_cast<size_t>(t) * K + q * SPL;
             if constexpr (SPL == 2 && K % 2 == 0) {
