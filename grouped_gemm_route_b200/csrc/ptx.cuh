@@ -1,5 +1,5 @@
 // Inline-PTX helpers for sm_100a: mbarriers with bounded waits, TMA tensor
-// loads (tile and tile::gather4, never multicast), tcgen05 tensor-core MMA,
+// loads (tiles, never multicast), tcgen05 tensor-core MMA,
 // tensor-memory allocation and loads, and the shared-memory / instruction
 // descriptors the MMA consumes.  Every helper is a thin wrapper around one PTX
 // instruction as described in the PTX ISA.
@@ -128,17 +128,6 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Four rows (r0..r3) of a 2-d tensor, columns [x, x + box width), written to
-// shared memory as four consecutive rows.  The tensor map's box is one row high.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int r0,
-                                            int r1, int r2, int r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
         : "memory");
 }
 
