@@ -56,6 +56,7 @@ def test_tiny_workload():
     dict(T=130, d=256, E=8, k=8, I=128),     # k = E
     dict(T=1, d=256, E=8, k=2, I=128),       # a single token
     dict(T=200, d=256, E=48, k=40, I=128),   # k > 32: the sort reads inv in two chunks, the combine five
+    dict(T=96, d=128, E=64, k=64, I=128),    # the largest k, = E: every expert takes every token
     dict(T=500, d=128, E=8, k=2, I=128),     # d = 128: rows of 16 pieces, half of each sorting warp idle
 ])
 def test_multi_tile_ragged(sizes):

@@ -30,6 +30,7 @@ pytestmark = pytest.mark.gpu
     (1000, 8, 2, True),      # quad form, E = 4k
     (3000, 160, 8, False),   # warp form: E > 128
     (300, 512, 16, True),    # warp form: largest E, k > 8
+    (200, 96, 64, True),     # warp form: the largest k (two slots per lane)
     (1000, 130, 4, True),    # warp form: E not a multiple of 4
     (500, 8, 4, True),       # warp form: E < 4k
 ])
