@@ -24,6 +24,9 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "moe_internal.h"
 #include "ptx.cuh"
 
@@ -1339,29 +1342,50 @@ cudaError_t launch_route_bwd(int T, int E, int k, const float *w, const int32_t 
     return cudaGetLastError();
 }
 
+// Resident blocks per SM of a routing kernel at (threads, dynamic shared
+// memory), with the kernel's shared-memory opt-in set; looked up once per
+// device and configuration (0 on failure, which is not kept).
+int routing_blocks_per_sm(const void *fn, int threads, size_t smem) {
+    struct Entry {
+        int dev;
+        const void *fn;
+        int threads;
+        size_t smem;
+        int per_sm;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        for (const Entry &c : cache)
+            if (c.dev == dev && c.fn == fn && c.threads == threads && c.smem == smem) return c.per_sm;
+    }
+    int per_sm = 0;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess || per_sm < 1)
+        return 0;
+    std::lock_guard<std::mutex> g(mu);
+    cache.push_back(Entry{dev, fn, threads, smem, per_sm});
+    return per_sm;
+}
+
 int route_fused_grid(const float *logits, int T, int E, int k, int sms, int n_chunks) {
     int per_sm = 0;
-    cudaError_t e;
     if (route_quad_ok(E, k, logits)) {
-        const void *fn = route_quad_fn(E, k);
         const QuadCfg c = quad_cfg(E, T, sms);
-        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
-        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, c.warps * 32, c.smem);
+        per_sm = routing_blocks_per_sm(route_quad_fn(E, k), c.warps * 32, c.smem);
     } else {
         const int nv = (E + 31) / 32;
-        const size_t smem = route_fused_smem(E, k);
-        if (nv <= 1)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<1>, kFusedThreads, smem);
-        else if (nv <= 2)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<2>, kFusedThreads, smem);
-        else if (nv <= 4)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<4>, kFusedThreads, smem);
-        else if (nv <= 8)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<8>, kFusedThreads, smem);
-        else
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel<16>, kFusedThreads, smem);
+        const void *fn = nv <= 1   ? reinterpret_cast<const void *>(route_fused_kernel<1>)
+                         : nv <= 2 ? reinterpret_cast<const void *>(route_fused_kernel<2>)
+                         : nv <= 4 ? reinterpret_cast<const void *>(route_fused_kernel<4>)
+                         : nv <= 8 ? reinterpret_cast<const void *>(route_fused_kernel<8>)
+                                   : reinterpret_cast<const void *>(route_fused_kernel<16>);
+        per_sm = routing_blocks_per_sm(fn, kFusedThreads, route_fused_smem(E, k));
     }
-    if (e != cudaSuccess || per_sm < 1) return 0;
+    if (per_sm < 1) return 0;
     const int g = per_sm * sms;
     return g < n_chunks ? g : n_chunks;
 }
