@@ -211,12 +211,13 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint
     return r == CUDA_SUCCESS;
 }
 
-// 2-d bf16 tensor [rows, cols], box = 128 rows x 32 columns (64-byte rows), 64-byte swizzle: the
-// chunks of h the down dgrad's loader warp moves into its ring.
-bool make_map_h(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+// 2-d bf16 tensor [rows, cols], box = box_rows rows x 32 columns (64-byte rows), 64-byte swizzle:
+// the chunks of h the down dgrad's loader warp moves into its ring (128 rows), and the 32 x 32
+// pieces of dW the weight gradients' epilogue warps store.
+bool make_map_h(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint32_t box_rows = 128) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    cuuint32_t box[2] = {32, 128};
+    cuuint32_t box[2] = {32, box_rows};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -650,10 +651,14 @@ int bwd_gemms(const Plan &pl, const DeviceInfo &dev, int grid, GemmArgs a, const
     a.dw = static_cast<__nv_bfloat16 *>(dw_down);
     {
         Launch L(kKindGemmDownWgrad, st);
-        if ((rc = L.done(gemm_pair_ok(kDownWgrad, pl.bn_i, false, a.m_tiles, grid)
-                             ? launch_gemm_pair(kDownWgrad, a, tm_gs_mn, tm_aw_mn, grid, st)
-                             : launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st))))
-            return rc;
+        if (gemm_pair_ok(kDownWgrad, pl.bn_i, false, a.m_tiles, grid)) {
+            CUtensorMap tm_dw;  // the epilogue's TMA stores
+            if (!make_map_h(&tm_dw, dw_down, Ed, pl.I, 32)) return MOE_ERR_LAUNCH;
+            rc = L.done(launch_gemm_pair(kDownWgrad, a, tm_gs_mn, tm_aw_mn, grid, st, &tm_dw));
+        } else {
+            rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st));
+        }
+        if (rc) return rc;
     }
     // b4: gate/up dgrad, rows staged for the ordered scatter-sum into dx
     a.n_tiles = pl.d / pl.bn_d;
@@ -671,9 +676,12 @@ int bwd_gemms(const Plan &pl, const DeviceInfo &dev, int grid, GemmArgs a, const
     a.n_tiles = pl.d / pl.bn_d;
     a.dw = static_cast<__nv_bfloat16 *>(dw_gate_up);
     Launch L(kKindGemmGateUpWgrad, st);
-    return L.done(gemm_pair_ok(kGateUpWgrad, pl.bn_d, false, a.m_tiles, grid)
-                      ? launch_gemm_pair(kGateUpWgrad, a, tm_dh_mn, tm_xs_mn, grid, st)
-                      : launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st));
+    if (gemm_pair_ok(kGateUpWgrad, pl.bn_d, false, a.m_tiles, grid)) {
+        CUtensorMap tm_dw;
+        if (!make_map_h(&tm_dw, dw_gate_up, EI2, pl.d, 32)) return MOE_ERR_LAUNCH;
+        return L.done(launch_gemm_pair(kGateUpWgrad, a, tm_dh_mn, tm_xs_mn, grid, st, &tm_dw));
+    }
+    return L.done(launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st));
 }
 
 }  // namespace
@@ -804,27 +812,26 @@ int moe_bwd(const moe_shape_t *shape, const void *grad_out, const void *x, const
                                        saved->inv, dpart, pl.dpart_stride, dscore, dlogits, st));
     }
     // The scatter-sum into dx (bandwidth bound) needs only the gate/up dgrad's
-    // staged rows: it runs on a second stream beside the gate/up wgrad (tensor
-    // bound; its persistent CTAs leave threads and registers free on every SM),
-    // joined back before the call's last kernel.
+    // staged rows, and b6 (dscore as the ordered sum of the partials, then
+    // dlogits) only the down dgrad's partials: both run on a second stream
+    // beside the gate/up wgrad (tensor bound; its persistent CTAs leave threads
+    // and registers free on every SM), joined back before the call returns.
     SideStream *side = side_stream();
     bool forked = false;
-    auto fork_combine = [&]() -> int {
+    auto fork_tail = [&]() -> int {
+        cudaStream_t s2 = st;
         if (side != nullptr && side->link(side->fork, st, side->s)) {
             forked = true;
-            return run_combine(pl, dev, w8, dx, side->s);
+            s2 = side->s;
         }
-        return run_combine(pl, dev, w8, dx, st);
+        int r = run_combine(pl, dev, w8, dx, s2);
+        if (r) return r;
+        Launch L(kKindRouteBwd, s2);
+        return L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_w, saved->topk_idx, saved->inv,
+                                       dpart, pl.dpart_stride, dscore, dlogits, s2));
     };
-    rc = bwd_gemms(pl, dev, grid, a, gs, xs, w_gate_up, w_down, saved, dw_gate_up, dw_down, nullptr, st, fork_combine);
+    rc = bwd_gemms(pl, dev, grid, a, gs, xs, w_gate_up, w_down, saved, dw_gate_up, dw_down, nullptr, st, fork_tail);
     if (forked && !side->link(side->join, side->s, st)) return MOE_ERR_LAUNCH;
-    if (rc) return rc;
-    // b6: dscore (ordered sum of partials) and dlogits
-    {
-        Launch L(kKindRouteBwd, st);
-        rc = L.done(launch_route_bwd(static_cast<int>(pl.T), pl.E, pl.k, saved->topk_w, saved->topk_idx, saved->inv,
-                                     dpart, pl.dpart_stride, dscore, dlogits, st));
-    }
     return rc;
 }
 

@@ -555,6 +555,61 @@ __device__ __forceinline__ void store_chunk_bf16(uint8_t *xbuf, const uint32_t (
     warp_store_rows(xbuf, pv, row);
 }
 
+// One 32-column chunk of this warp's 32 accumulator rows as bf16, stored by
+// TMA through `map` at (x, y): the rows go to `buf` in the map's 64-byte
+// swizzle (the transposes' layout), and lane 0 issues the store once every
+// lane's writes are visible to the async proxy.  `buf` is one of the warp's
+// two buffers, used alternately: before it is overwritten, lane 0's store from
+// it two chunks earlier must have read it (at most one younger group pending).
+__device__ __forceinline__ void store_chunk_tma(uint8_t *buf, const uint32_t (&v)[32], const CUtensorMap *map, int x,
+                                                int y) {
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) bulk_wait_read<1>();
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(buf + xpose_off(lane, q)) =
+            make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                       pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                       pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                       pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(map, buf, x, y);
+        bulk_commit();
+    }
+}
+
+// store_accumulator_bf16 with TMA stores: this warp's 32 rows of the tile go to
+// rows y .. y + 31 and columns x0 .. x0 + BN - 1 of the tensor behind `map`,
+// chunk c from buffer c & 1 of xbuf2 (two kXposeBytes buffers).
+template <int BN, bool PAIR>
+__device__ __forceinline__ void store_accumulator_tma(uint32_t taddr, uint8_t *xbuf2, const CUtensorMap *map, int x0,
+                                                      int y, uint64_t *tempty_acc) {
+    static_assert((BN / 32) % 2 == 0, "an even number of chunks keeps the buffers alternating across tiles");
+    uint32_t ra[32], rb[32];
+    tmem_load32(taddr, ra);
+    tmem_load_wait();
+    tmem_regs_ready(ra);
+#pragma unroll
+    for (int c = 0; c < BN / 32; c += 2) {
+        tmem_load32(taddr + (c + 1) * 32, rb);
+        store_chunk_tma(xbuf2, ra, map, x0 + c * 32, y);
+        tmem_load_wait();
+        tmem_regs_ready(rb);
+        if (c + 2 < BN / 32)
+            tmem_load32(taddr + (c + 2) * 32, ra);
+        else
+            release_acc<PAIR>(tempty_acc);
+        store_chunk_tma(xbuf2 + kXposeBytes, rb, map, x0 + (c + 1) * 32, y);
+        if (c + 2 < BN / 32) {
+            tmem_load_wait();
+            tmem_regs_ready(ra);
+        }
+    }
+}
+
 // Streams this warp's 32 accumulator rows (BN fp32 columns) to bf16 rows at
 // row (nullptr: skipped), 32 columns at a time, with the tensor-memory load of
 // chunk c + 1 in flight while chunk c is converted and stored.  Releases the
@@ -843,20 +898,31 @@ __device__ __forceinline__ bool epi_down_dgrad_ring(const GemmArgs &a, const Til
     return true;
 }
 
-// weight gradients: store the tile (zeros for an expert without tokens)
+// weight gradients: store the tile (zeros for an expert without tokens).
+// With dw_map (CTA pairs) the tile goes out by TMA stores of the dW rows
+// [E * Mtot, Ntot] from the warp's two buffers at xbuf; otherwise by the
+// transposes, row by row.
 template <int MODE, int BN, bool PAIR = false>
 __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
-                                          uint64_t *tempty_acc, uint8_t *xbuf) {
+                                          uint64_t *tempty_acc, uint8_t *xbuf, const CUtensorMap *dw_map = nullptr) {
     const int Mtot = MODE == kDownWgrad ? a.d : 2 * a.I;
     const int Ntot = MODE == kDownWgrad ? a.I : a.d;
     constexpr int BH = BN;
     __nv_bfloat16 *row = a.dw + (static_cast<size_t>(t.e) * Mtot + t.mt * kTileM + r) * static_cast<size_t>(Ntot) +
                          t.nt * BN;
     if (t.nkb > 0) {
-        store_accumulator_bf16<BH, PAIR>(taddr, xbuf, row, tempty_acc);
+        if (dw_map != nullptr)
+            store_accumulator_tma<BH, PAIR>(taddr, xbuf, dw_map, t.nt * BN, t.e * Mtot + t.mt * kTileM + (r & ~31),
+                                            tempty_acc);
+        else
+            store_accumulator_bf16<BH, PAIR>(taddr, xbuf, row, tempty_acc);
         return;
     }
     release_acc<PAIR>(tempty_acc);  // an expert without tokens: exact zeros, the accumulator is not read
+    if (dw_map != nullptr) {  // the first buffer is reused below: its earlier stores must have read it
+        if ((threadIdx.x & 31) == 0) bulk_wait_read<0>();
+        __syncwarp();
+    }
     uint32_t zero[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) zero[i] = 0u;
@@ -1039,8 +1105,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// GEMMs on CTA pairs (bf16, BN = 256): the gate/up forward (on x gathered into
-// the sorted layout first), the gate/up dgrad and the weight gradients.  A cluster of two CTAs computes one 256 x 256 tile with
+// GEMMs on CTA pairs (bf16, BN = 256): all six modes (the gate/up forward on x
+// copied into the sorted layout first).  A cluster of two CTAs computes one 256 x 256 tile with
 // tcgen05.mma.cta_group::2: each CTA loads its own 128 M rows of A and one
 // half (128 columns) of B, so a CTA moves half the B bytes per MMA it takes
 // part in; 32 KB stages instead of 48 KB.  The leader (rank 0) arms the stage
@@ -1058,6 +1124,11 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
 // them and the peer's epilogue only releases the accumulator.  Pair rows are
 // numbered expert by expert from a per-CTA table of their starts.
 //
+// The third tensor map, tmC, is per mode: A in 64-row boxes (the forward GEMMs'
+// half tiles), h in 128-row x 32-column boxes (the down dgrad's ring loads), or
+// dW in 32 x 32 boxes (the weight gradients' epilogue stores).  The gate/up
+// dgrad does not use it.
+//
 // No load is multicast.  Every wait is bounded, and both CTAs always reach the
 // final cluster barrier (no early exit), after which the pair frees its tensor
 // memory.
@@ -1068,18 +1139,24 @@ struct PairCfg {
     static constexpr int kBHalfBytes = (BN / 2) * kTileK * 2;  // this CTA's half of a B stage
     static constexpr int kStageBytes = kABytes + kBHalfBytes;
     static constexpr int kOrderBytes = 8 * kMaxExperts;  // wgrads: counts + order; M-tiled: pair-row starts
-    static constexpr int kXposeTotal = TR::kEpiWarps * kXposeBytes;
+    // transpose buffers per epilogue warp: two for the weight gradients, whose
+    // epilogue stores by TMA from one while it fills the other
+    static constexpr int kXposePerWarp = TR::kMTiled ? 1 : 2;
+    static constexpr int kXposeTotal = TR::kEpiWarps * kXposePerWarp * kXposeBytes;
     // down dgrad: a ring of two h chunks (gate and up, 128 rows x 32 columns each)
     static constexpr int kRingSlotBytes = 2 * kTileM * 32 * 2;
     static constexpr int kRingBytes = MODE == kDownDgrad ? 2 * kRingSlotBytes : 0;
     static constexpr int kFixed = 512 + kOrderBytes + kXposeTotal + kRingBytes + 1024;
     static constexpr int kFit = (227 * 1024 - kFixed) / kStageBytes;
     static constexpr int kStages = kFit < 6 ? kFit : 6;
-    static constexpr int kRingOffset = kStages * kStageBytes;  // 1024-byte aligned (stages are 32 KB)
-    static constexpr int kBarOffset = kRingOffset + kRingBytes;
+    // stages, ring and transpose buffers are 1024-byte aligned (the 64-byte
+    // swizzle the ring's loads and the wgrads' stores use repeats every 512 bytes)
+    static constexpr int kRingOffset = kStages * kStageBytes;
+    static constexpr int kXposeOffset = kRingOffset + kRingBytes;
+    static constexpr int kBarOffset = kXposeOffset + kXposeTotal;
     static constexpr int kOrderOffset = kBarOffset + 512;
-    static constexpr int kXposeOffset = kOrderOffset + kOrderBytes;
-    static constexpr int kSmemBytes = kXposeOffset + kXposeTotal + 1024;
+    static constexpr int kSmemBytes = kOrderOffset + kOrderBytes + 1024;
+    static_assert(kStageBytes % 1024 == 0 && kRingBytes % 1024 == 0 && kXposeTotal % 1024 == 0, "alignment");
     static_assert(kStages >= 4 && kSmemBytes <= 227 * 1024, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = 2 * BN;
 };
@@ -1143,7 +1220,7 @@ __device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, co
 template <int MODE, int BN>
 __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const __grid_constant__ CUtensorMap tmA64, const GemmArgs args) {
+                             const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
     static_assert(MODE == kGateUpFwd || MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad ||
                       MODE == kDownDgrad || MODE == kDownFwd,
                   "the modes where pairs measured faster than one CTA");
@@ -1243,7 +1320,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                // a half tile's A is 64 rows (tmA64) in each CTA
+                // a half tile's A is 64 rows (tmC) in each CTA
                 if (leader && lane == 0)
                     mbar_arrive_expect_tx(&full[s], t.half ? 2u * (P::kStageBytes - kABytes / 2) : 2u * P::kStageBytes);
                 __syncwarp();
@@ -1259,14 +1336,14 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                     // other 64 (64-row boxes, K-major), so that accumulator columns hold, per
                     // 64-column group, gate then up of the same expert columns -- in a half tile
                     // each TMEM lane half then holds whole (gate, up) pairs
-                    if (lane == 0) tma_load_2d_pair(As, t.half ? &tmA64 : &tmA, fb, k0, t.row0);
+                    if (lane == 0) tma_load_2d_pair(As, t.half ? &tmC : &tmA, fb, k0, t.row0);
                     const int grow = t.e * 2 * a.I + t.nt * (BN / 2) + 64 * static_cast<int>(rank);
                     if (lane == 1) tma_load_2d_pair(Bs, &tmB, fb, k0, grow);
                     if (lane == 2) tma_load_2d_pair(Bs + 64 * 128, &tmB, fb, k0, grow + a.I);
                 } else if constexpr (MODE == kDownFwd) {
                     // A: 128 sorted rows of aw from row0 (a half tile: 64 rows); B: this CTA's 128 of the
                     // tile's 256 rows of W_down[e] (output columns), K-major
-                    if (lane == 0) tma_load_2d_pair(As, t.half ? &tmA64 : &tmA, fb, k0, t.row0);
+                    if (lane == 0) tma_load_2d_pair(As, t.half ? &tmC : &tmA, fb, k0, t.row0);
                     if (lane == 1) tma_load_2d_pair(Bs, &tmB, fb, k0, t.e * a.d + t.nt * BN + static_cast<int>(rank) * (BN / 2));
                 } else if constexpr (MODE == kDownDgrad) {
                     // A: 128 sorted rows of grad_out, K-major; B: this CTA's half of W_down[e]
@@ -1344,7 +1421,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
         // ---- epilogue: this CTA's 128 rows of the tile ----
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
-        uint8_t *xbuf = smem + P::kXposeOffset + (warp - kEpiWarp0) * kXposeBytes;
+        uint8_t *xbuf = smem + P::kXposeOffset + (warp - kEpiWarp0) * P::kXposePerWarp * kXposeBytes;
         int hit = 0;  // down dgrad: h ring chunks consumed so far
         int local = 0;
         for (int tile = nth_tile<MODE>(0, pair, npairs); tile < total;
@@ -1377,8 +1454,13 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 else
                     epi_stage<BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
             } else {
-                epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf);
+                epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf, &tmC);
             }
+        }
+        if constexpr (!TR::kMTiled) {
+            // the tile stores are complete before the CTA ends
+            if (lane == 0) bulk_wait_all();
+            __syncwarp();
         }
     }
 
@@ -1400,8 +1482,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                     mbar_arrive_expect_tx(&hfull[slot], P::kRingSlotBytes);
                     uint8_t *dst = ring + slot * P::kRingSlotBytes;
                     const int col = t.nt * BN + c * 32;
-                    tma_load_2d(dst, &tmA64, &hfull[slot], col, t.row0);                        // gate
-                    tma_load_2d(dst + P::kRingSlotBytes / 2, &tmA64, &hfull[slot], a.I + col, t.row0);  // up
+                    tma_load_2d(dst, &tmC, &hfull[slot], col, t.row0);                        // gate
+                    tma_load_2d(dst + P::kRingSlotBytes / 2, &tmC, &hfull[slot], a.I + col, t.row0);  // up
                 }
             }
             if (!ok) {
@@ -1460,7 +1542,7 @@ cudaError_t launch_mode(int bn, bool mx, const GemmArgs &args, const CUtensorMap
 // at once (capped by the grid the caller offers).
 template <int MODE>
 cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const CUtensorMap &tmA64, int grid, cudaStream_t s) {
+                        const CUtensorMap &tmC, int grid, cudaStream_t s) {
     using P = PairCfg<MODE, 256>;
     auto *fn = grouped_gemm_pair_kernel<MODE, 256>;
     static std::atomic<int> max_pairs_plus1[kMaxDevices];  // per instantiation and device: resident
@@ -1492,7 +1574,7 @@ cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUte
     const int pairs = (grid / 2) < max_pairs ? grid / 2 : max_pairs;
     if (pairs < 1) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3(2 * pairs);
-    return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, tmA64, args);
+    return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, tmC, args);
 }
 
 }  // namespace
@@ -1517,18 +1599,16 @@ bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid) {
 }
 
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                             int grid, cudaStream_t s, const CUtensorMap *tmA64) {
-    const CUtensorMap &a64 = tmA64 != nullptr ? *tmA64 : tmA;
+                             int grid, cudaStream_t s, const CUtensorMap *tmC) {
+    if (tmC == nullptr && mode != kGateUpDgrad) return cudaErrorInvalidValue;  // every other mode uses the third map
+    const CUtensorMap &c = tmC != nullptr ? *tmC : tmA;
     switch (mode) {
-        case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, a64, grid, s);
-        case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, a64, grid, s);
-        case kGateUpFwd: return tmA64 != nullptr ? launch_pair<kGateUpFwd>(args, tmA, tmB, a64, grid, s)
-                                                 : cudaErrorInvalidValue;  // half tiles need the 64-row map
-        case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, a64, grid, s);
-        case kDownDgrad: return tmA64 != nullptr ? launch_pair<kDownDgrad>(args, tmA, tmB, a64, grid, s)
-                                                 : cudaErrorInvalidValue;  // needs the map of h
-        case kDownFwd: return tmA64 != nullptr ? launch_pair<kDownFwd>(args, tmA, tmB, a64, grid, s)
-                                               : cudaErrorInvalidValue;  // half tiles need the 64-row map
+        case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, c, grid, s);
+        case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, c, grid, s);
+        case kGateUpFwd: return launch_pair<kGateUpFwd>(args, tmA, tmB, c, grid, s);
+        case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, c, grid, s);
+        case kDownDgrad: return launch_pair<kDownDgrad>(args, tmA, tmB, c, grid, s);
+        case kDownFwd: return launch_pair<kDownFwd>(args, tmA, tmB, c, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -130,14 +130,16 @@ cudaError_t launch_expire_wait(int *status, cudaStream_t s);
 
 cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, const CUtensorMap &tmA,
                         const CUtensorMap &tmB, int grid, cudaStream_t s);
-// GEMMs on CTA pairs (tcgen05 cta_group::2, bf16, BN = 256): the gate/up
-// forward, the gate/up dgrad and the weight gradients; used where gemm_pair_ok
-// holds, with the same arguments and results as launch_gemm.
+// GEMMs on CTA pairs (tcgen05 cta_group::2, bf16, BN = 256), all six modes;
+// used where gemm_pair_ok holds, with the same arguments and results as
+// launch_gemm.
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid);
-// tmA64: the gate/up forward's A operand in 64-row boxes (an expert's unpaired
-// last tile loads 64 rows per CTA); unused by the other modes.
+// tmC, the third tensor map: the forward GEMMs' A operand in 64-row boxes (an
+// expert's unpaired last tile loads 64 rows per CTA), h for the down dgrad
+// (make_map_h), dW for the weight gradients (32 x 32 boxes, 64-byte swizzle:
+// their epilogues store by TMA); null only for the gate/up dgrad.
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                             int grid, cudaStream_t s, const CUtensorMap *tmA64 = nullptr);
+                             int grid, cudaStream_t s, const CUtensorMap *tmC = nullptr);
 
 cudaError_t launch_mx_quant_rows(const __nv_bfloat16 *src, int64_t R, int K, uint8_t *dst, uint8_t *sf, int sf_mode,
                                  int I, const int32_t *rows_used, int sms, cudaStream_t s);

@@ -1,5 +1,5 @@
 // Inline-PTX helpers for sm_100a: mbarriers with bounded waits, TMA tensor
-// loads (tiles, never multicast), tcgen05 tensor-core MMA,
+// loads (tiles, never multicast) and tile stores, tcgen05 tensor-core MMA,
 // tensor-memory allocation and loads, and the shared-memory / instruction
 // descriptors the MMA consumes.  Every helper is a thin wrapper around one PTX
 // instruction as described in the PTX ISA.
@@ -113,7 +113,8 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
 }
 
 // ---------------------------------------------------------------------------
-// TMA (bulk tensor copies global -> shared, completion on an mbarrier)
+// TMA (bulk tensor copies global -> shared, completion on an mbarrier; and
+// shared -> global tile stores)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
     asm volatile(
@@ -122,6 +123,24 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+
+// Shared -> global tile store through a tensor map (x: innermost coordinate,
+// its byte offset a multiple of 16), tracked in the issuing thread's bulk
+// async-groups: commit with bulk_commit, then wait with bulk_wait_read (the
+// shared source may be reused) or bulk_wait_all (the writes are done).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// At most N of this thread's committed groups still reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Contiguous bytes global -> shared (16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
