@@ -480,16 +480,17 @@ int sort_x(const Plan &pl, const DeviceInfo &dev, const void *x, const moe_saved
 int gateup_pair_sorted(const Plan &pl, const moe_shape_t *shape, const DeviceInfo &dev, const void *xs,
                        const void *w_gate_up, moe_saved_t *saved, uint8_t *w8, cudaStream_t st) {
     // the pair kernel loads W_gate_up in 64-row boxes (gate and up halves), and x in 128-row boxes
-    // (64-row boxes for an expert's unpaired last tile)
-    CUtensorMap tm_wgu, tm_xs, tm_xs64;
+    // (64-row boxes for an expert's unpaired last tile); its epilogue stores h and aw by TMA
+    CUtensorMap tm_wgu, tm_xs, tm_xs64, tm_h, tm_aw;
     if (!make_map(&tm_wgu, w_gate_up, static_cast<int64_t>(pl.E) * 2 * pl.I, pl.d, 64) ||
-        !make_map(&tm_xs, xs, pl.p_cap, pl.d, 128) || !make_map(&tm_xs64, xs, pl.p_cap, pl.d, 64))
+        !make_map(&tm_xs, xs, pl.p_cap, pl.d, 128) || !make_map(&tm_xs64, xs, pl.p_cap, pl.d, 64) ||
+        !make_map_h(&tm_h, saved->h, pl.p_cap, 2 * pl.I, 32) || !make_map_h(&tm_aw, saved->aw, pl.p_cap, pl.I, 32))
         return MOE_ERR_LAUNCH;
     GemmArgs a = base_args(pl, saved, w8);
     a.n_tiles = pl.I / 128;
     a.num_k_blocks = pl.d / kTileK;
     Launch L(kKindGemmGateUpFwd, st);
-    return L.done(launch_gemm_pair(kGateUpFwd, a, tm_xs, tm_wgu, grid_for(shape, dev), st, &tm_xs64));
+    return L.done(launch_gemm_pair(kGateUpFwd, a, tm_xs, tm_wgu, grid_for(shape, dev), st, &tm_xs64, &tm_h, &tm_aw));
 }
 
 int gateup_fwd(const Plan &pl, const DeviceInfo &dev, const moe_shape_t *shape, const void *x, const void *w_gate_up,

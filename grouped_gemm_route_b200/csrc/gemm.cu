@@ -581,6 +581,16 @@ __device__ __forceinline__ void store_chunk_tma(uint8_t *buf, const uint32_t (&v
     }
 }
 
+// This lane's 64 bytes of packed bf16 (row = lane) into buf in the 64-byte
+// swizzle of the TMA stores (the caller fences and issues the store).
+__device__ __forceinline__ void put_row_swz64(uint8_t *buf, const uint32_t (&pv)[16]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(buf + xpose_off(lane, q)) =
+            make_uint4(pv[4 * q], pv[4 * q + 1], pv[4 * q + 2], pv[4 * q + 3]);
+}
+
 // store_accumulator_bf16 with TMA stores: this warp's 32 rows of the tile go to
 // rows y .. y + 31 and columns x0 .. x0 + BN - 1 of the tensor behind `map`,
 // chunk c from buffer c & 1 of xbuf2 (two kXposeBytes buffers).
@@ -644,13 +654,11 @@ __device__ __forceinline__ void store_accumulator_bf16(uint32_t taddr, uint8_t *
 // (a.limit = L; +inf leaves gate and up unchanged, bit for bit).
 // MXFP8: also aw's E4M3 codes and scale atoms along I (the down GEMM's K).
 // One 32-column chunk c of gate (gr) and up (ur) accumulator values.
-template <int BN, bool MX>
-__device__ __forceinline__ void gateup_chunk(const GemmArgs &a, const Tile &t, int r, int pos, bool valid, float wv,
-                                             int c, const uint32_t (&gr)[32], const uint32_t (&ur)[32],
-                                             __nv_bfloat16 *hrow, __nv_bfloat16 *arow, uint8_t *xbuf) {
-    constexpr int kHalf = BN / 2;
-    uint32_t pg[16], pu[16], pa[16];
-    float av[32];
+// The SwiGLU of one 32-column chunk: gate and up as bf16 pairs (pg, pu) and
+// aw = w * silu(gate) * up, in fp32 (av) and as bf16 pairs (pa).
+__device__ __forceinline__ void gateup_math(const GemmArgs &a, bool valid, float wv, const uint32_t (&gr)[32],
+                                            const uint32_t (&ur)[32], uint32_t (&pg)[16], uint32_t (&pu)[16],
+                                            uint32_t (&pa)[16], float (&av)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const float g = fminf(__uint_as_float(gr[i]), a.limit);
@@ -663,6 +671,16 @@ __device__ __forceinline__ void gateup_chunk(const GemmArgs &a, const Tile &t, i
         pu[i] = valid ? pack_bf16x2(__uint_as_float(ur[2 * i]), __uint_as_float(ur[2 * i + 1])) : 0u;
         pa[i] = pack_bf16x2(av[2 * i], av[2 * i + 1]);
     }
+}
+
+template <int BN, bool MX>
+__device__ __forceinline__ void gateup_chunk(const GemmArgs &a, const Tile &t, int r, int pos, bool valid, float wv,
+                                             int c, const uint32_t (&gr)[32], const uint32_t (&ur)[32],
+                                             __nv_bfloat16 *hrow, __nv_bfloat16 *arow, uint8_t *xbuf) {
+    constexpr int kHalf = BN / 2;
+    uint32_t pg[16], pu[16], pa[16];
+    float av[32];
+    gateup_math(a, valid, wv, gr, ur, pg, pu, pa, av);
     warp_store_rows(xbuf, pg, hrow + c * 32);
     warp_store_rows(xbuf, pu, hrow + a.I + c * 32);
     warp_store_rows(xbuf, pa, arow + c * 32);
@@ -930,6 +948,33 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
     for (int c = 0; c < BH / 32; ++c) warp_store_rows(xbuf, zero, row + c * 32);
 }
 
+// One chunk of the gate/up forward on CTA pairs, stored by TMA: this warp's 32
+// rows (from y) of gate, up and aw go to the three buffers of xbuf3 and out
+// through hmap (columns x and I + x of h) and amap (columns x of aw).  The
+// buffers are reused chunk after chunk, once the previous chunk's stores have
+// read them.
+__device__ __forceinline__ void gateup_chunk_tma(const GemmArgs &a, bool valid, float wv, const uint32_t (&gr)[32],
+                                                 const uint32_t (&ur)[32], uint8_t *xbuf3, const CUtensorMap *hmap,
+                                                 const CUtensorMap *amap, int x, int y) {
+    uint32_t pg[16], pu[16], pa[16];
+    float av[32];
+    gateup_math(a, valid, wv, gr, ur, pg, pu, pa, av);
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+    put_row_swz64(xbuf3, pg);
+    put_row_swz64(xbuf3 + kXposeBytes, pu);
+    put_row_swz64(xbuf3 + 2 * kXposeBytes, pa);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(hmap, xbuf3, x, y);
+        tma_store_2d(hmap, xbuf3 + kXposeBytes, a.I + x, y);
+        tma_store_2d(amap, xbuf3 + 2 * kXposeBytes, x, y);
+        bulk_commit();
+    }
+}
+
 // Gate/up forward on CTA pairs (BN = 256): a tile covers gate/up columns
 // nt*128 .. +128, laid out in the accumulator as [gate 0..63 | up 0..63 |
 // gate 64..127 | up 64..127] (see the producer).  Output chunk c (32 gate
@@ -939,16 +984,17 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int 
 // this CTA's 64 rows in lanes 0..63 with columns [0, 128) of the tile and in
 // lanes 64..127 with columns [128, 256), both at TMEM columns [0, 128): the
 // thread owns row (quad & 1) * 32 + lane of its 64 and chunks 2h, 2h + 1 with
-// h = quad >> 1.  Same SwiGLU arithmetic as the one-CTA kernel.
+// h = quad >> 1.  Same SwiGLU arithmetic as the one-CTA kernel; h and aw go
+// out by TMA stores (gateup_chunk_tma).
 __device__ __forceinline__ void epi_gateup_fwd_pair(const GemmArgs &a, const Tile &t, int quad, int lane,
-                                                    uint32_t taddr, uint64_t *tempty_acc, uint8_t *xbuf) {
+                                                    uint32_t taddr, uint64_t *tempty_acc, uint8_t *xbuf3,
+                                                    const CUtensorMap *hmap, const CUtensorMap *amap) {
     const int r = t.half ? (quad & 1) * 32 + lane : quad * 32 + lane;
     const int pos = t.row0 + r;
+    const int y = t.row0 + (r & ~31);  // this warp's first row
     const int p = __ldg(a.perm + pos);
     const bool valid = p >= 0 && p < a.T * a.k;
     const float wv = valid ? __ldg(a.topk_w + p) : 0.f;
-    __nv_bfloat16 *hrow = a.h + static_cast<size_t>(pos) * 2 * a.I + t.nt * 128;
-    __nv_bfloat16 *arow = a.aw + static_cast<size_t>(pos) * a.I + t.nt * 128;
     const int c_first = t.half ? 2 * (quad >> 1) : 0;
     const int n_chunks = t.half ? 2 : 4;
     auto gate_col = [&](int c) -> uint32_t {
@@ -965,7 +1011,7 @@ __device__ __forceinline__ void epi_gateup_fwd_pair(const GemmArgs &a, const Til
         const int c = c_first + i;
         tmem_load32(taddr + gate_col(c + 1), gb);
         tmem_load32(taddr + gate_col(c + 1) + 64, ub);
-        gateup_chunk<256, false>(a, t, r, pos, valid, wv, c, ga, ua, hrow, arow, xbuf);
+        gateup_chunk_tma(a, valid, wv, ga, ua, xbuf3, hmap, amap, t.nt * 128 + c * 32, y);
         tmem_load_wait();
         tmem_regs_ready(gb);
         tmem_regs_ready(ub);
@@ -975,7 +1021,7 @@ __device__ __forceinline__ void epi_gateup_fwd_pair(const GemmArgs &a, const Til
         } else {
             release_acc<true>(tempty_acc);  // TMEM no longer needed
         }
-        gateup_chunk<256, false>(a, t, r, pos, valid, wv, c + 1, gb, ub, hrow, arow, xbuf);
+        gateup_chunk_tma(a, valid, wv, gb, ub, xbuf3, hmap, amap, t.nt * 128 + (c + 1) * 32, y);
         if (i + 2 < n_chunks) {
             tmem_load_wait();
             tmem_regs_ready(ga);
@@ -1127,7 +1173,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
 // The third tensor map, tmC, is per mode: A in 64-row boxes (the forward GEMMs'
 // half tiles), h in 128-row x 32-column boxes (the down dgrad's ring loads), or
 // dW in 32 x 32 boxes (the weight gradients' epilogue stores).  The gate/up
-// dgrad does not use it.
+// dgrad does not use it.  tmD and tmE, h and aw in 32 x 32 boxes, are the
+// gate/up forward's epilogue stores.
 //
 // No load is multicast.  Every wait is bounded, and both CTAs always reach the
 // final cluster barrier (no early exit), after which the pair frees its tensor
@@ -1140,8 +1187,9 @@ struct PairCfg {
     static constexpr int kStageBytes = kABytes + kBHalfBytes;
     static constexpr int kOrderBytes = 8 * kMaxExperts;  // wgrads: counts + order; M-tiled: pair-row starts
     // transpose buffers per epilogue warp: two for the weight gradients, whose
-    // epilogue stores by TMA from one while it fills the other
-    static constexpr int kXposePerWarp = TR::kMTiled ? 1 : 2;
+    // epilogue stores by TMA from one while it fills the other; three (gate, up,
+    // aw) for the gate/up forward's TMA stores
+    static constexpr int kXposePerWarp = MODE == kGateUpFwd ? 3 : (TR::kMTiled ? 1 : 2);
     static constexpr int kXposeTotal = TR::kEpiWarps * kXposePerWarp * kXposeBytes;
     // down dgrad: a ring of two h chunks (gate and up, 128 rows x 32 columns each)
     static constexpr int kRingSlotBytes = 2 * kTileM * 32 * 2;
@@ -1220,7 +1268,8 @@ __device__ __forceinline__ Tile decode_pair_tile(int tile, const GemmArgs &a, co
 template <int MODE, int BN>
 __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+                             const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
+                             const __grid_constant__ CUtensorMap tmE, const GemmArgs args) {
     static_assert(MODE == kGateUpFwd || MODE == kDownWgrad || MODE == kGateUpWgrad || MODE == kGateUpDgrad ||
                       MODE == kDownDgrad || MODE == kDownFwd,
                   "the modes where pairs measured faster than one CTA");
@@ -1437,7 +1486,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
             const uint32_t taddr =
                 tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
             if constexpr (MODE == kGateUpFwd) {
-                epi_gateup_fwd_pair(a, t, quad, lane, taddr, &tempty[acc], xbuf);
+                epi_gateup_fwd_pair(a, t, quad, lane, taddr, &tempty[acc], xbuf, &tmD, &tmE);
             } else if constexpr (MODE == kDownDgrad) {
                 if (t.skip) {
                     release_acc<true>(&tempty[acc]);
@@ -1457,8 +1506,8 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
                 epi_wgrad<MODE, BN, true>(a, t, r, taddr, &tempty[acc], xbuf, &tmC);
             }
         }
-        if constexpr (!TR::kMTiled) {
-            // the tile stores are complete before the CTA ends
+        if constexpr (!TR::kMTiled || MODE == kGateUpFwd) {
+            // the TMA tile stores are complete before the CTA ends
             if (lane == 0) bulk_wait_all();
             __syncwarp();
         }
@@ -1542,7 +1591,8 @@ cudaError_t launch_mode(int bn, bool mx, const GemmArgs &args, const CUtensorMap
 // at once (capped by the grid the caller offers).
 template <int MODE>
 cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const CUtensorMap &tmC, int grid, cudaStream_t s) {
+                        const CUtensorMap &tmC, const CUtensorMap &tmD, const CUtensorMap &tmE, int grid,
+                        cudaStream_t s) {
     using P = PairCfg<MODE, 256>;
     auto *fn = grouped_gemm_pair_kernel<MODE, 256>;
     static std::atomic<int> max_pairs_plus1[kMaxDevices];  // per instantiation and device: resident
@@ -1574,7 +1624,7 @@ cudaError_t launch_pair(const GemmArgs &args, const CUtensorMap &tmA, const CUte
     const int pairs = (grid / 2) < max_pairs ? grid / 2 : max_pairs;
     if (pairs < 1) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3(2 * pairs);
-    return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, tmC, args);
+    return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, tmC, tmD, tmE, args);
 }
 
 }  // namespace
@@ -1599,16 +1649,20 @@ bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid) {
 }
 
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                             int grid, cudaStream_t s, const CUtensorMap *tmC) {
+                             int grid, cudaStream_t s, const CUtensorMap *tmC, const CUtensorMap *tmD,
+                             const CUtensorMap *tmE) {
     if (tmC == nullptr && mode != kGateUpDgrad) return cudaErrorInvalidValue;  // every other mode uses the third map
+    if ((tmD == nullptr || tmE == nullptr) && mode == kGateUpFwd) return cudaErrorInvalidValue;  // h and aw stores
     const CUtensorMap &c = tmC != nullptr ? *tmC : tmA;
+    const CUtensorMap &d = tmD != nullptr ? *tmD : tmA;
+    const CUtensorMap &e = tmE != nullptr ? *tmE : tmA;
     switch (mode) {
-        case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, c, grid, s);
-        case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, c, grid, s);
-        case kGateUpFwd: return launch_pair<kGateUpFwd>(args, tmA, tmB, c, grid, s);
-        case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, c, grid, s);
-        case kDownDgrad: return launch_pair<kDownDgrad>(args, tmA, tmB, c, grid, s);
-        case kDownFwd: return launch_pair<kDownFwd>(args, tmA, tmB, c, grid, s);
+        case kDownWgrad: return launch_pair<kDownWgrad>(args, tmA, tmB, c, d, e, grid, s);
+        case kGateUpWgrad: return launch_pair<kGateUpWgrad>(args, tmA, tmB, c, d, e, grid, s);
+        case kGateUpFwd: return launch_pair<kGateUpFwd>(args, tmA, tmB, c, d, e, grid, s);
+        case kGateUpDgrad: return launch_pair<kGateUpDgrad>(args, tmA, tmB, c, d, e, grid, s);
+        case kDownDgrad: return launch_pair<kDownDgrad>(args, tmA, tmB, c, d, e, grid, s);
+        case kDownFwd: return launch_pair<kDownFwd>(args, tmA, tmB, c, d, e, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }

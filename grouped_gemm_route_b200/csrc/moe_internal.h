@@ -137,9 +137,11 @@ bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid);
 // tmC, the third tensor map: the forward GEMMs' A operand in 64-row boxes (an
 // expert's unpaired last tile loads 64 rows per CTA), h for the down dgrad
 // (make_map_h), dW for the weight gradients (32 x 32 boxes, 64-byte swizzle:
-// their epilogues store by TMA); null only for the gate/up dgrad.
+// their epilogues store by TMA); null only for the gate/up dgrad.  tmD, tmE:
+// the gate/up forward's h and aw in 32 x 32 boxes (its epilogue's TMA stores).
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                             int grid, cudaStream_t s, const CUtensorMap *tmC = nullptr);
+                             int grid, cudaStream_t s, const CUtensorMap *tmC = nullptr,
+                             const CUtensorMap *tmD = nullptr, const CUtensorMap *tmE = nullptr);
 
 cudaError_t launch_mx_quant_rows(const __nv_bfloat16 *src, int64_t R, int K, uint8_t *dst, uint8_t *sf, int sf_mode,
                                  int I, const int32_t *rows_used, int sms, cudaStream_t s);
