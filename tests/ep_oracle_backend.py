@@ -82,48 +82,58 @@ class OracleEP:
         return torch.from_numpy(dx), torch.from_numpy(dscore), torch.from_numpy(dlogits)
 
     # ---- expert side ----
-    def expert_buffers(self, rows):
-        self.rows = rows
-        return torch.zeros(rows + 128 * self.E_loc, self.d, dtype=torch.float64), torch.zeros(rows,
-                                                                                              dtype=torch.float64)
+    def weight_grads(self, w_gate_up, w_down):
+        return (torch.zeros(np.shape(w_gate_up), dtype=torch.float64),
+                torch.zeros(np.shape(w_down), dtype=torch.float64))
 
-    def _layout(self, recv):
-        recv = np.asarray(recv, dtype=np.int64).reshape(self.G, self.E_loc)
-        n = recv.sum(axis=0)
-        gs = padded_starts(n)
-        off = np.zeros(self.E_loc + 1, dtype=np.int64)
-        off[1:] = np.cumsum(n)
-        return n, gs, off
+    def expert_side(self, recv_dev, rows, e0, e1):
+        return _OracleExpertSide(self, recv_dev, rows, e1 - e0)
 
-    def expert_forward(self, recv_dev, rows, xr, wr, w_gate_up, w_down):
-        n, gs, off = self._layout(recv_dev.numpy())
-        xr, wr = xr.numpy(), wr.numpy()
+
+class _OracleExpertSide:
+    """One chunk of local experts: E_c experts, `rows` received rows in the
+    padded layout restated from recv[s][e] (sources in rank order inside each
+    expert's group)."""
+
+    def __init__(self, b, recv_dev, rows, E_c):
+        self.b, self.rows, self.E_c = b, rows, E_c
+        recv = np.asarray(recv_dev, dtype=np.int64).reshape(b.G, E_c)
+        self.n = recv.sum(axis=0)
+        self.gs = padded_starts(self.n)
+        self.off = np.zeros(E_c + 1, dtype=np.int64)
+        self.off[1:] = np.cumsum(self.n)
+        self.xr = torch.zeros(rows + 128 * E_c, b.d, dtype=torch.float64)
+        self.wr = torch.zeros(rows, dtype=torch.float64)
+
+    def forward(self, w_gate_up, w_down):
+        xr, wr = self.xr.numpy(), self.wr.numpy()
         wgu, wd = np.asarray(w_gate_up, dtype=np.float64), np.asarray(w_down, dtype=np.float64)
-        y = np.zeros((rows, self.d))
+        y = np.zeros((self.rows, self.b.d))
         self.loc = []
-        for e in range(self.E_loc):
-            xe = xr[gs[e]:gs[e] + n[e]]
-            we = wr[off[e]:off[e + 1]]
-            if n[e]:
-                h, _, ye = O.expert_forward(xe, wgu[e], wd[e], self.limit)
-                y[off[e]:off[e + 1]] = we[:, None] * ye
-            self.loc.append((xe.copy(), we.copy(), gs[e], off[e], n[e]))
+        for e in range(self.E_c):
+            xe = xr[self.gs[e]:self.gs[e] + self.n[e]]
+            we = wr[self.off[e]:self.off[e + 1]]
+            if self.n[e]:
+                h, _, ye = O.expert_forward(xe, wgu[e], wd[e], self.b.limit)
+                y[self.off[e]:self.off[e + 1]] = we[:, None] * ye
+            self.loc.append((xe.copy(), we.copy(), self.gs[e], self.off[e], self.n[e]))
         return torch.from_numpy(y)
 
-    def expert_grad_buffer(self):
-        return torch.zeros(self.rows + 128 * self.E_loc, self.d, dtype=torch.float64)
+    def grad_buffer(self):
+        return torch.zeros_like(self.xr)
 
-    def expert_backward(self, gr, w_gate_up, w_down):
+    def backward(self, gr, w_gate_up, w_down, dwgu_out, dwd_out):
         gr = gr.numpy()
         wgu, wd = np.asarray(w_gate_up, dtype=np.float64), np.asarray(w_down, dtype=np.float64)
-        dx_rows = np.zeros((self.rows, self.d))
+        dx_rows = np.zeros((self.rows, self.b.d))
         ds_rows = np.zeros(self.rows)
         dwgu, dwd = np.zeros_like(wgu), np.zeros_like(wd)
         for e, (xe, we, g0, o0, ne) in enumerate(self.loc):
             if not ne:
                 continue
-            dxr, ds, dwgu[e], dwd[e], _ = O._pair_backward(xe, gr[g0:g0 + ne], we, wgu[e], wd[e], self.limit)
+            dxr, ds, dwgu[e], dwd[e], _ = O._pair_backward(xe, gr[g0:g0 + ne], we, wgu[e], wd[e], self.b.limit)
             dx_rows[o0:o0 + ne] = dxr
             ds_rows[o0:o0 + ne] = ds
-        return (torch.from_numpy(dx_rows), torch.from_numpy(ds_rows), torch.from_numpy(dwgu),
-                torch.from_numpy(dwd))
+        dwgu_out.copy_(torch.from_numpy(dwgu))
+        dwd_out.copy_(torch.from_numpy(dwd))
+        return torch.from_numpy(dx_rows), torch.from_numpy(ds_rows)

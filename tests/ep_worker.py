@@ -2,7 +2,8 @@
 the gloo backend on CPU, each holding T tokens and E/G experts.  The layer's
 device steps are done by the fp64 oracle (ep_oracle_backend); the plan, the
 counts all-to-all and the point-to-point exchanges are the product's
-(grouped_gemm_route_b200.ep).  Every rank compares its outputs and its
+(grouped_gemm_route_b200.ep), with the local experts' exchanges and device
+steps in one chunk and in several overlapping ones.  Every rank compares its outputs and its
 experts' weight gradients with the oracle's layer over all ranks' tokens;
 rank 0 prints the largest errors as one JSON line."""
 import datetime
@@ -51,11 +52,11 @@ def main():
     T, d, E, k, I = 37, 24, 8, 3, 16
     E_loc = E // G
     results = []
-    for case in range(3):
+    for case, chunks in [(0, 1), (0, 3), (1, 1), (1, 2), (2, 3), (2, 8)]:
         x, logits, wgu, wd, gout = case_inputs(case, G, T, d, E, k, I)
         mine = slice(rank * T, (rank + 1) * T)
         experts = slice(rank * E_loc, (rank + 1) * E_loc)
-        layer = EPMoELayer(OracleEP(T, d, E, k, I, G))
+        layer = EPMoELayer(OracleEP(T, d, E, k, I, G), chunks=chunks)
         out = layer.forward(x[mine], logits[mine], wgu[experts], wd[experts]).numpy()
         g = layer.backward(gout[mine], wgu[experts], wd[experts])
         ref = O.forward(x, logits, wgu, wd, k)
@@ -64,7 +65,7 @@ def main():
                     dscore=rel(g["dscore"].numpy(), rg["dscore"][mine]),
                     dlogits=rel(g["dlogits"].numpy(), rg["dlogits"][mine]),
                     dwgu=rel(g["dwgu"].numpy(), rg["dwgu"][experts]), dwd=rel(g["dwd"].numpy(), rg["dwd"][experts]))
-        results.append(dict(case=case, rank=rank, rows_received=layer.plan.rows, errs=errs))
+        results.append(dict(case=case, chunks=len(layer.bounds), rank=rank, rows_received=layer.plan.rows, errs=errs))
     got = [None] * G
     dist.all_gather_object(got, results)
     dist.barrier()

@@ -62,7 +62,8 @@ def test_two_ranks_match_the_oracle_layer():
     res = lines[0]
     assert res["world"] == 2
     flat = [c for per_rank in res["results"] for c in per_rank]
-    assert len(flat) == 6
+    assert len(flat) == 12
+    assert {c["chunks"] for c in flat} == {1, 2, 3, 4}  # E/G = 4 local experts: 8 chunks become 4
     # case 1 routes every token to rank 0's experts: rank 1 receives no rows
     assert any(c["case"] == 1 and c["rank"] == 1 and c["rows_received"] == 0 for c in flat)
     for c in flat:
