@@ -232,7 +232,8 @@ class EPMoELayer:
             ro, co, n, pad = M.ep_expert_layout(G, e1 - e0, rc)
             plans.append(Plan(G, e1 - e0, src["counts"], src["group_start"], src["offsets"], rc, ro, co, n, pad,
                               E_all=E_loc, e0=e0))
-            sides.append(b.expert_side(recv_2d[:, e0:e1].contiguous().view(-1), n, e0, e1))
+            # a fresh copy: the library wants 16-byte aligned device arrays
+            sides.append(b.expert_side(recv_2d[:, e0:e1].clone().view(-1), n, e0, e1))
         self.plans, self.sides = plans, sides
         tag = 0
         inbound = []
