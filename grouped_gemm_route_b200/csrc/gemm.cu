@@ -1198,7 +1198,8 @@ struct PairCfg {
     static constexpr int kFit = (227 * 1024 - kFixed) / kStageBytes;
     static constexpr int kStages = kFit < 6 ? kFit : 6;
     // stages, ring and transpose buffers are 1024-byte aligned (the 64-byte
-    // swizzle the ring's loads and the wgrads' stores use repeats every 512 bytes)
+    // swizzle of the ring's loads and of the epilogues' TMA stores repeats every
+    // 512 bytes)
     static constexpr int kRingOffset = kStages * kStageBytes;
     static constexpr int kXposeOffset = kRingOffset + kRingBytes;
     static constexpr int kBarOffset = kXposeOffset + kXposeTotal;
