@@ -28,7 +28,7 @@ def case_inputs(case, G, T, d, E, k, I):
     rng = np.random.default_rng(100 + case)
     x = rng.standard_normal((G * T, d))
     logits = rng.standard_normal((G * T, E)).astype(np.float32)
-    if case == 1:  # every token routes to rank 0's experts only: rank 1 receives nothing
+    if case == 1:  # every token picks rank 0's experts first (with two ranks, rank 1 receives nothing)
         logits[:, : E // G] += 100.0
     if case == 2:  # one expert of each rank never chosen; a few experts dominate
         logits[:, 1] = -100.0

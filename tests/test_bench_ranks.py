@@ -19,8 +19,8 @@ def free_port():
         return s.getsockname()[1]
 
 
-def torchrun(args, timeout=240):
-    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+def torchrun(args, timeout=240, nproc=2):
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(nproc),
            "--master-addr", "127.0.0.1", "--master-port", str(free_port())] + args
     env = dict(os.environ, OMP_NUM_THREADS="2")
     return subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=timeout, env=env)

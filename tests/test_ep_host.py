@@ -1,8 +1,8 @@
 """Expert parallelism on CPU: the library's host-side layout of the received
 rows against a restatement, and the whole exchange choreography of
-grouped_gemm_route_b200.ep on two gloo ranks (torchrun, loopback), with the
+grouped_gemm_route_b200.ep on two and four gloo ranks (torchrun, loopback), with the
 device steps done by the fp64 oracle.  Each rank's out, dx, dscore and dlogits
-and its experts' weight gradients must equal the oracle's layer over both
+and its experts' weight gradients must equal the oracle's layer over all
 ranks' tokens (the concatenated batch; the oracle's dispatch order -- experts
 ascending, tokens ascending -- is the order EP builds: sources in rank order,
 tokens ascending inside each)."""
@@ -54,18 +54,22 @@ def test_expert_layout_rejects_negative_counts():
         M.ep_expert_layout(2, 2, [[1, -1], [0, 0]])
 
 
-def test_two_ranks_match_the_oracle_layer():
-    r = torchrun([os.path.join("tests", "ep_worker.py")], timeout=300)
+@pytest.mark.parametrize("G", [2, 4])
+def test_ranks_match_the_oracle_layer(G):
+    r = torchrun([os.path.join("tests", "ep_worker.py")], timeout=300, nproc=G)
     assert r.returncode == 0, r.stderr[-3000:]
     lines = json_lines(r.stdout)
     assert len(lines) == 1
     res = lines[0]
-    assert res["world"] == 2
+    assert res["world"] == G
     flat = [c for per_rank in res["results"] for c in per_rank]
-    assert len(flat) == 12
-    assert {c["chunks"] for c in flat} == {1, 2, 3, 4}  # E/G = 4 local experts: 8 chunks become 4
-    # case 1 routes every token to rank 0's experts: rank 1 receives no rows
-    assert any(c["case"] == 1 and c["rank"] == 1 and c["rows_received"] == 0 for c in flat)
+    assert len(flat) == 6 * G
+    E_loc = 8 // G
+    assert {c["chunks"] for c in flat} == {min(n, E_loc) for n in (1, 2, 3, 8)}
+    # case 1 routes every token to rank 0's experts first: with two ranks (top-3 of rank 0's
+    # four experts) rank 1 receives no rows
+    if G == 2:
+        assert all(c["rows_received"] == 0 for c in flat if c["case"] == 1 and c["rank"] == 1)
     for c in flat:
         bad = {n: v for n, v in c["errs"].items() if not v <= 1e-12}
         assert not bad, (c["case"], c["rank"], bad)
