@@ -213,7 +213,7 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint
 
 // 2-d bf16 tensor [rows, cols], box = box_rows rows x 32 columns (64-byte rows), 64-byte swizzle:
 // the chunks of h the down dgrad's loader warp moves into its ring (128 rows), and the 32 x 32
-// pieces of dW the weight gradients' epilogue warps store.
+// pieces of h and aw the gate/up forward's epilogue warps store.
 bool make_map_h(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, uint32_t box_rows = 128) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
@@ -653,8 +653,8 @@ int bwd_gemms(const Plan &pl, const DeviceInfo &dev, int grid, GemmArgs a, const
     {
         Launch L(kKindGemmDownWgrad, st);
         if (gemm_pair_ok(kDownWgrad, pl.bn_i, false, a.m_tiles, grid)) {
-            CUtensorMap tm_dw;  // the epilogue's TMA stores
-            if (!make_map_h(&tm_dw, dw_down, Ed, pl.I, 32)) return MOE_ERR_LAUNCH;
+            CUtensorMap tm_dw;  // the epilogue's TMA stores (32 x 64 boxes)
+            if (!make_map(&tm_dw, dw_down, Ed, pl.I, 32)) return MOE_ERR_LAUNCH;
             rc = L.done(launch_gemm_pair(kDownWgrad, a, tm_gs_mn, tm_aw_mn, grid, st, &tm_dw));
         } else {
             rc = L.done(launch_gemm(kDownWgrad, pl.bn_i, false, a, tm_gs_mn, tm_aw_mn, grid, st));
@@ -679,7 +679,7 @@ int bwd_gemms(const Plan &pl, const DeviceInfo &dev, int grid, GemmArgs a, const
     Launch L(kKindGemmGateUpWgrad, st);
     if (gemm_pair_ok(kGateUpWgrad, pl.bn_d, false, a.m_tiles, grid)) {
         CUtensorMap tm_dw;
-        if (!make_map_h(&tm_dw, dw_gate_up, EI2, pl.d, 32)) return MOE_ERR_LAUNCH;
+        if (!make_map(&tm_dw, dw_gate_up, EI2, pl.d, 32)) return MOE_ERR_LAUNCH;
         return L.done(launch_gemm_pair(kGateUpWgrad, a, tm_dh_mn, tm_xs_mn, grid, st, &tm_dw));
     }
     return L.done(launch_gemm(kGateUpWgrad, pl.bn_d, false, a, tm_dh_mn, tm_xs_mn, grid, st));

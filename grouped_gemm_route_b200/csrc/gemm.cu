@@ -555,32 +555,6 @@ __device__ __forceinline__ void store_chunk_bf16(uint8_t *xbuf, const uint32_t (
     warp_store_rows(xbuf, pv, row);
 }
 
-// One 32-column chunk of this warp's 32 accumulator rows as bf16, stored by
-// TMA through `map` at (x, y): the rows go to `buf` in the map's 64-byte
-// swizzle (the transposes' layout), and lane 0 issues the store once every
-// lane's writes are visible to the async proxy.  `buf` is one of the warp's
-// two buffers, used alternately: before it is overwritten, lane 0's store from
-// it two chunks earlier must have read it (at most one younger group pending).
-__device__ __forceinline__ void store_chunk_tma(uint8_t *buf, const uint32_t (&v)[32], const CUtensorMap *map, int x,
-                                                int y) {
-    const int lane = threadIdx.x & 31;
-    if (lane == 0) bulk_wait_read<1>();
-    __syncwarp();
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4 *>(buf + xpose_off(lane, q)) =
-            make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                       pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                       pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                       pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-        tma_store_2d(map, buf, x, y);
-        bulk_commit();
-    }
-}
-
 // This lane's 64 bytes of packed bf16 (row = lane) into buf in the 64-byte
 // swizzle of the TMA stores (the caller fences and issues the store).
 __device__ __forceinline__ void put_row_swz64(uint8_t *buf, const uint32_t (&pv)[16]) {
@@ -592,30 +566,52 @@ __device__ __forceinline__ void put_row_swz64(uint8_t *buf, const uint32_t (&pv)
 }
 
 // store_accumulator_bf16 with TMA stores: this warp's 32 rows of the tile go to
-// rows y .. y + 31 and columns x0 .. x0 + BN - 1 of the tensor behind `map`,
-// chunk c from buffer c & 1 of xbuf2 (two kXposeBytes buffers).
+// rows y .. y + 31 and columns x0 .. x0 + BN - 1 of the tensor behind `map`
+// (boxes of 32 rows x 64 columns, 128-byte swizzle), 64 columns at a time from
+// one 4 KB buffer at xbuf: the two 32-column chunks of a box are loaded from
+// tensor memory together, packed, and written to the buffer once the previous
+// box's store has read it; one proxy fence and one store per box.
 template <int BN, bool PAIR>
-__device__ __forceinline__ void store_accumulator_tma(uint32_t taddr, uint8_t *xbuf2, const CUtensorMap *map, int x0,
+__device__ __forceinline__ void store_accumulator_tma(uint32_t taddr, uint8_t *xbuf, const CUtensorMap *map, int x0,
                                                       int y, uint64_t *tempty_acc) {
-    static_assert((BN / 32) % 2 == 0, "an even number of chunks keeps the buffers alternating across tiles");
+    static_assert((BN / 32) % 2 == 0, "whole 64-column boxes");
+    const int lane = threadIdx.x & 31;
     uint32_t ra[32], rb[32];
     tmem_load32(taddr, ra);
+    tmem_load32(taddr + 32, rb);
     tmem_load_wait();
     tmem_regs_ready(ra);
+    tmem_regs_ready(rb);
 #pragma unroll
     for (int c = 0; c < BN / 32; c += 2) {
-        tmem_load32(taddr + (c + 1) * 32, rb);
-        store_chunk_tma(xbuf2, ra, map, x0 + c * 32, y);
-        tmem_load_wait();
-        tmem_regs_ready(rb);
-        if (c + 2 < BN / 32)
+        uint32_t pv[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            pv[i] = pack_bf16x2(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
+            pv[16 + i] = pack_bf16x2(__uint_as_float(rb[2 * i]), __uint_as_float(rb[2 * i + 1]));
+        }
+        if (c + 2 < BN / 32) {
             tmem_load32(taddr + (c + 2) * 32, ra);
-        else
+            tmem_load32(taddr + (c + 3) * 32, rb);
+        } else {
             release_acc<PAIR>(tempty_acc);
-        store_chunk_tma(xbuf2 + kXposeBytes, rb, map, x0 + (c + 1) * 32, y);
+        }
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)  // 128-byte swizzle: 16-byte piece q of row `lane` at piece q ^ (lane & 7)
+            *reinterpret_cast<uint4 *>(xbuf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                make_uint4(pv[4 * q], pv[4 * q + 1], pv[4 * q + 2], pv[4 * q + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(map, xbuf, x0 + c * 32, y);
+            bulk_commit();
+        }
         if (c + 2 < BN / 32) {
             tmem_load_wait();
             tmem_regs_ready(ra);
+            tmem_regs_ready(rb);
         }
     }
 }
@@ -918,8 +914,8 @@ __device__ __forceinline__ bool epi_down_dgrad_ring(const GemmArgs &a, const Til
 
 // weight gradients: store the tile (zeros for an expert without tokens).
 // With dw_map (CTA pairs) the tile goes out by TMA stores of the dW rows
-// [E * Mtot, Ntot] from the warp's two buffers at xbuf; otherwise by the
-// transposes, row by row.
+// [E * Mtot, Ntot] (32 x 64 boxes) from the warp's 4 KB buffer at xbuf;
+// otherwise by the transposes, row by row.
 template <int MODE, int BN, bool PAIR = false>
 __device__ __forceinline__ void epi_wgrad(const GemmArgs &a, const Tile &t, int r, uint32_t taddr,
                                           uint64_t *tempty_acc, uint8_t *xbuf, const CUtensorMap *dw_map = nullptr) {
@@ -1172,7 +1168,7 @@ __global__ void __launch_bounds__(ModeTraits<MODE>::kThreads, 1)
 //
 // The third tensor map, tmC, is per mode: A in 64-row boxes (the forward GEMMs'
 // half tiles), h in 128-row x 32-column boxes (the down dgrad's ring loads), or
-// dW in 32 x 32 boxes (the weight gradients' epilogue stores).  The gate/up
+// dW in 32-row x 64-column boxes (the weight gradients' epilogue stores).  The gate/up
 // dgrad does not use it.  tmD and tmE, h and aw in 32 x 32 boxes, are the
 // gate/up forward's epilogue stores.
 //
@@ -1186,9 +1182,9 @@ struct PairCfg {
     static constexpr int kBHalfBytes = (BN / 2) * kTileK * 2;  // this CTA's half of a B stage
     static constexpr int kStageBytes = kABytes + kBHalfBytes;
     static constexpr int kOrderBytes = 8 * kMaxExperts;  // wgrads: counts + order; M-tiled: pair-row starts
-    // transpose buffers per epilogue warp: two for the weight gradients, whose
-    // epilogue stores by TMA from one while it fills the other; three (gate, up,
-    // aw) for the gate/up forward's TMA stores
+    // transpose buffers per epilogue warp: two (one 4 KB box of 32 rows x 64
+    // columns) for the weight gradients' TMA stores; three (gate, up, aw) for the
+    // gate/up forward's
     static constexpr int kXposePerWarp = MODE == kGateUpFwd ? 3 : (TR::kMTiled ? 1 : 2);
     static constexpr int kXposeTotal = TR::kEpiWarps * kXposePerWarp * kXposeBytes;
     // down dgrad: a ring of two h chunks (gate and up, 128 rows x 32 columns each)
@@ -1197,9 +1193,9 @@ struct PairCfg {
     static constexpr int kFixed = 512 + kOrderBytes + kXposeTotal + kRingBytes + 1024;
     static constexpr int kFit = (227 * 1024 - kFixed) / kStageBytes;
     static constexpr int kStages = kFit < 6 ? kFit : 6;
-    // stages, ring and transpose buffers are 1024-byte aligned (the 64-byte
-    // swizzle of the ring's loads and of the epilogues' TMA stores repeats every
-    // 512 bytes)
+    // stages, ring and transpose buffers are 1024-byte aligned (the 64- and
+    // 128-byte swizzles of the ring's loads and of the epilogues' TMA stores
+    // repeat every 512 and 1024 bytes)
     static constexpr int kRingOffset = kStages * kStageBytes;
     static constexpr int kXposeOffset = kRingOffset + kRingBytes;
     static constexpr int kBarOffset = kXposeOffset + kXposeTotal;

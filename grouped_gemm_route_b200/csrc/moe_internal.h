@@ -136,8 +136,8 @@ cudaError_t launch_gemm(GemmMode mode, int bn, bool mx, const GemmArgs &args, co
 bool gemm_pair_ok(GemmMode mode, int bn, bool mx, int m_tiles, int grid);
 // tmC, the third tensor map: the forward GEMMs' A operand in 64-row boxes (an
 // expert's unpaired last tile loads 64 rows per CTA), h for the down dgrad
-// (make_map_h), dW for the weight gradients (32 x 32 boxes, 64-byte swizzle:
-// their epilogues store by TMA); null only for the gate/up dgrad.  tmD, tmE:
+// (make_map_h), dW for the weight gradients (32-row x 64-column boxes, 128-byte
+// swizzle: their epilogues store by TMA); null only for the gate/up dgrad.  tmD, tmE:
 // the gate/up forward's h and aw in 32 x 32 boxes (its epilogue's TMA stores).
 cudaError_t launch_gemm_pair(GemmMode mode, const GemmArgs &args, const CUtensorMap &tmA, const CUtensorMap &tmB,
                              int grid, cudaStream_t s, const CUtensorMap *tmC = nullptr,
