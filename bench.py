@@ -146,6 +146,10 @@ def workload_config(name, cfg, extra=None):
 # clocks during the timed region
 # ----------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi samples of one GPU every 25 ms, each stamped with the host
+    time it arrived; stop() keeps those inside the [mark_start, mark_end]
+    window (the timed region), or, when the region is shorter than the
+    sampling interval and none fell inside it, the sample nearest to it."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -153,36 +157,70 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
+        self.reader = None
+        self.t0 = self.t1 = None
 
-    def start(self):
+    def start(self, wait_s=5.0):
+        """Start sampling; returns once the first sample has arrived (or after wait_s)."""
+        import threading
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "25",
                  "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
+            return
+
+        def read():
+            for line in self.proc.stdout:
+                self.lines.append((time.time(), line))
+
+        self.reader = threading.Thread(target=read, daemon=True)
+        self.reader.start()
+        t_end = time.time() + wait_s
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
             return None
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=10)
+            self.proc.wait(timeout=10)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = []
-        for line in out.splitlines():
+            self.proc.wait()
+        if self.reader is not None:
+            self.reader.join(timeout=5)
+        stamped = []
+        for t, line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
-                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+                stamped.append((t, dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                        hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8])))
             except ValueError:
                 continue
-        if not rows:
+        if not stamped:
             return None
+        window = "timed region"
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for t, r in stamped if self.t0 <= t <= self.t1]
+            if not inside:
+                mid = 0.5 * (self.t0 + self.t1)
+                inside = [min(stamped, key=lambda tr: abs(tr[0] - mid))[1]]
+                window = "nearest sample to the timed region (shorter than the sampling interval)"
+            rows = inside
+        else:
+            rows = [r for _, r in stamped]
         loaded = [r for r in rows if r["power"] > 200.0] or rows
         reasons = set()
         for r in loaded:
@@ -191,7 +229,8 @@ class ClockSampler:
                 if r[key].lower() in ("active", "1"):
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
-                "samples": len(loaded), "power_w_max": max(r["power"] for r in rows), "reasons": sorted(reasons)}
+                "samples": len(loaded), "power_w_max": max(r["power"] for r in rows), "reasons": sorted(reasons),
+                "window": window}
 
 
 # ----------------------------------------------------------------------------
@@ -301,12 +340,15 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------
 # timing helpers (our arm)
 # ----------------------------------------------------------------------------
-def timed_loop(step, n_steps, stream, dev, barrier):
+def timed_loop(step, n_steps, stream, dev, barrier, clocks=None):
     """Device time of n_steps calls of step(), CUDA events on the launching
-    stream, a barrier and a synchronize on both sides; ms per step."""
+    stream, a barrier and a synchronize on both sides; ms per step.  clocks
+    (a ClockSampler) gets the host times between the two synchronizes."""
     import torch
     barrier()
     torch.cuda.synchronize(dev)
+    if clocks is not None:
+        clocks.mark_start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -314,6 +356,8 @@ def timed_loop(step, n_steps, stream, dev, barrier):
         step()
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    if clocks is not None:
+        clocks.mark_end()
     barrier()
     return t0.elapsed_time(t1) / n_steps
 
@@ -421,8 +465,7 @@ def time_other_config(M, IN, name, n_steps, n_warmup, dev, stream, barrier, peak
     clocks = ClockSampler(clk_gpu)
     if clk_gpu is not None:
         clocks.start()
-        time.sleep(0.3)
-    ms = timed_loop(step, n_steps, stream, dev, barrier)
+    ms = timed_loop(step, n_steps, stream, dev, barrier, clocks if clk_gpu is not None else None)
     clk = clocks.stop() if clk_gpu is not None else None
     per_kernel, _ = profiled_loop(M, step, n_steps, stream, dev, barrier)
     g_ms, g_err = graph_loop(lambda s: (layer.forward(x, lg, wgu, wd, s), layer.backward(gout, x, wgu, wd, True, s)),
@@ -506,8 +549,7 @@ def main():
     clocks = ClockSampler(local)
     if not args.no_clocks:
         clocks.start()
-        time.sleep(0.3)
-    ms_per_step = timed_loop(step, args.steps, stream, dev, barrier)
+    ms_per_step = timed_loop(step, args.steps, stream, dev, barrier, None if args.no_clocks else clocks)
     clk = clocks.stop()
     if layer.status(stream) != 0:
         raise SystemExit("device status error in the timed region")
