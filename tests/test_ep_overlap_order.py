@@ -45,6 +45,10 @@ def run(chunks, log=None, monkeypatch=None):
         real_side = b.expert_side
 
         def side(recv_dev, rows, e0, e1):
+            # the library takes 16-byte aligned device arrays: each chunk's counts are a fresh tensor,
+            # not a view into the whole step's counts at an offset
+            assert recv_dev.storage_offset() == 0 and recv_dev.is_contiguous()
+            assert recv_dev.numel() == e1 - e0  # one rank: [G * (e1 - e0)]
             sd = real_side(recv_dev, rows, e0, e1)
             fwd, bwd = sd.forward, sd.backward
             sd.forward = lambda *a: (log.append(("forward", e0)), fwd(*a))[1]
